@@ -1,0 +1,437 @@
+#!/usr/bin/env python
+"""Benchmark of the context-parallel attention hot path on B200.
+
+One step = one pass of the whole hot path over the image-DiT workload
+(B=1, H=24, S=4608, D=128, seeded synthetic bf16, RMS-normalised Q/K):
+  * ring attention, ring_degree 4 (fused: one kernel walks the K/V chunks in
+    ring order and merges them with the LSE rule on chip),
+  * Ulysses attention, degree 4: permute Q, K, V to the head-sharded layout,
+    head-sharded local attention, unpermute the output.
+Metric: attention TFLOP/s = (4*B*H*S^2*D per attention pass) * passes / time.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 (torchrun): independent replicas, one per GPU (the workload does not
+shard across GPUs here: every shard is emulated in one GPU's memory); the step
+time is the max over ranks and `value` counts the work of all ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+REPO = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, REPO)
+
+METRIC = "attention TFLOP/s (4·B·H·S²·D) & % BF16 peak; permute/merge GB/s & % HBM"
+WORKLOAD = "dit"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    path = os.path.join(REPO, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    """Hash of the attention kernel sources; a stored ncu traffic figure is only
+    reported while it matches the current kernel."""
+    h = hashlib.sha256()
+    csrc = os.path.join(REPO, "context_attention_long_b200", "csrc")
+    for name in ("attn_kernel.cuh", "cpattn_ptx.cuh", "cpattn_internal.h"):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def stored_traffic(kernel_key):
+    path = os.path.join(REPO, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(kernel_key)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("bytes_per_launch")
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML (read-only) in a
+    background thread; keeps the samples whose timestamps fall in a window."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting",
+               0x10: "sync_boost", 0x1: "gpu_idle"}
+
+    def __init__(self, torch_dev):
+        self.samples = []
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            p = torch.cuda.get_device_properties(torch_dev)
+            bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # noqa: BLE001
+            self.err = repr(e)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                sm = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                reasons = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.perf_counter(), sm, reasons))
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(0.005)
+
+    def start(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self, t0, t1):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "error": getattr(self, "err", "")}
+        win = [s for s in self.samples if t0 <= s[0] <= t1]
+        if not win:   # region shorter than the sampling period: nearest samples
+            win = sorted(self.samples, key=lambda s: min(abs(s[0] - t0), abs(s[0] - t1)))[:3]
+        mask = 0
+        for s in win:
+            mask |= s[2]
+        reasons = sorted(name for bit, name in self.REASONS.items() if mask & bit and name != "gpu_idle")
+        return {"sm_mhz": float(statistics.median(s[1] for s in win)) if win else None,
+                "sm_max_mhz": float(self.max_mhz), "reasons": reasons, "samples": len(win)}
+
+
+# ----------------------------------------------------------------- reference arm (the oracle)
+def oracle_sample_step(cfg, q, k, v, rows_per_shard, seed):
+    """The oracle's hot path on a bounded sample of query rows: for each ring
+    shard, sampled rows attend every K/V chunk in ring order (partials + LSE
+    merge), and the same rows through the Ulysses layout (head-sharded local
+    attention = monolithic attention per head group).  Returns attention FLOPs
+    processed (4 * rows * S * D per head and pass)."""
+    import oracle
+    from context_attention_long_b200 import inputs as inp
+    B, S, H, D = q.shape
+    P = cfg["ring_degree"]
+    lens = [S // P] * P
+    off = oracle.offsets(lens)
+    rng = np.random.Generator(np.random.PCG64(seed))
+    flops = 0
+    for r in range(P):
+        rows = off[r] + rng.integers(0, lens[r], size=rows_per_shard)
+        for b in range(B):
+            for h in range(H):
+                qh = inp.bf16_bits_to_f64(q[b, rows, h, :])
+                kh = inp.bf16_bits_to_f64(k[b, :, h, :])
+                vh = inp.bf16_bits_to_f64(v[b, :, h, :])
+                outs, lses = [], []
+                for c in oracle.ring_order(r, P):
+                    o, l = oracle.attention_rows(qh, kh[off[c]:off[c + 1]], vh[off[c]:off[c + 1]])
+                    outs.append(o[None, :, None, :])
+                    lses.append(l[None, None, :])
+                oracle.lse_merge(outs, lses)
+                oracle.attention_rows(qh, kh, vh)   # Ulysses: local attention of the head group
+                flops += 2 * 4 * len(rows) * S * D
+    return flops
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from context_attention_long_b200 import inputs
+    import torch
+    cfg, q, k, v = inputs.config_inputs(WORKLOAD)
+    threads = torch.get_num_threads()
+    rows = 8
+    for _ in range(args.warmup):
+        oracle_sample_step(cfg, q, k, v, rows, 0)
+    t0 = time.perf_counter()
+    flops = 0
+    for i in range(args.steps):
+        flops += oracle_sample_step(cfg, q, k, v, rows, i + 1)
+    dt = time.perf_counter() - t0
+    value = flops / dt / 1e12
+    B, S, H, D = q.shape
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1), RMS-normalised Q/K, bf16-rounded)",
+        "config": config_block(cfg),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{rows} query rows per ring shard per step, all {H} heads, ring path + Ulysses "
+                                   f"local attention, against the full S={S} K/V (fp64 numpy oracle)"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+def config_block(cfg):
+    return {"workload": f"image-DiT B{cfg['B']} H{cfg['H']} S{cfg['S']} D{cfg['D']}: ring {cfg['ring_degree']} "
+                        f"(fused) + Ulysses {cfg['ulysses_degree']} (permute, local attention, unpermute)",
+            "B": cfg["B"], "H": cfg["H"], "S": cfg["S"], "D": cfg["D"], "ring_degree": cfg["ring_degree"],
+            "ulysses_degree": cfg["ulysses_degree"], "parallelism": "replicas",
+            "l2": "flushed before every timed step (256 MiB write outside the timed events)"}
+
+
+def cpu_baseline(cfg, q, k, v, budget_s=12.0):
+    """The oracle, as it stands, on a bounded sample of the same workload."""
+    import torch
+    t0 = time.perf_counter()
+    flops, i, rows = 0, 0, 16
+    while time.perf_counter() - t0 < budget_s:
+        flops += oracle_sample_step(cfg, q, k, v, rows, 1000 + i)
+        i += 1
+    dt = time.perf_counter() - t0
+    B, S, H, D = q.shape
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": torch.get_num_threads(), "kind": "oracle",
+            "sample": f"{i} x ({rows} query rows per ring shard, all {H} heads, ring path with LSE merge + Ulysses "
+                      f"local attention, against the full S={S} K/V); fp64 numpy oracle, {dt:.1f} s"}
+
+
+# ----------------------------------------------------------------- our arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-breakdown", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from context_attention_long_b200 import api, build, inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+
+    cfg, qb, kb, vb = inputs.config_inputs(WORKLOAD)
+    B, S, H, D = qb.shape
+    P, U = cfg["ring_degree"], cfg["ulysses_degree"]
+
+    def host_bf16(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+
+    hq, hk, hv = host_bf16(qb), host_bf16(kb), host_bf16(vb)
+    q, k, v = (t.to(dev) for t in (hq, hk, hv))
+    out_r = torch.empty_like(q)
+    lse_r = torch.empty((B, H, S), dtype=torch.float32, device=dev)
+    yq, yk, yv, yo = (torch.empty(B * S * H * D, dtype=torch.bfloat16, device=dev) for _ in range(4))
+    out_u = torch.empty(B * S * H * D, dtype=torch.bfloat16, device=dev)
+    lse_u = torch.empty((B, H, S), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    qf, kf, vf = q.reshape(-1), k.reshape(-1), v.reshape(-1)
+
+    attn_flops = 4.0 * B * H * S * S * D      # one attention pass
+    step_flops = 2 * attn_flops               # ring + Ulysses
+    launches_per_step = 6                     # ring, 3 permutes, head-sharded attention, unpermute
+    n_ev = 7
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+
+    def step(e=None):
+        if e: e[0].record(stream)
+        api.cpattn_ring_attention(q, k, v, P, out=out_r, lse=lse_r, stream=stream)
+        if e: e[1].record(stream)
+        api.cpattn_ulysses_permute(qf, B, S, H, D, U, y=yq, stream=stream)
+        if e: e[2].record(stream)
+        api.cpattn_ulysses_permute(kf, B, S, H, D, U, y=yk, stream=stream)
+        if e: e[3].record(stream)
+        api.cpattn_ulysses_permute(vf, B, S, H, D, U, y=yv, stream=stream)
+        if e: e[4].record(stream)
+        api.cpattn_head_sharded_attention(yq, yk, yv, B, S, H, D, U, yo=yo, lse=lse_u, stream=stream)
+        if e: e[5].record(stream)
+        api.cpattn_ulysses_unpermute(yo, B, S, H, D, U, x=out_u, stream=stream)
+        if e: e[6].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    st, code = api.cpattn_device_status()
+    if st != 0:
+        raise RuntimeError(f"device wait expired during warm-up: {code:#x}")
+
+    clocks = ClockSampler(dev)
+    clocks.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.perf_counter()
+    for i in range(args.steps):
+        flush.zero_()                 # evict L2 (outside the timed events)
+        step(ev[i])
+    torch.cuda.synchronize()
+    t_wall1 = time.perf_counter()
+    if world > 1:
+        dist.barrier()
+    clocks.stop()
+
+    per = np.array([[ev[i][j].elapsed_time(ev[i][j + 1]) for j in range(n_ev - 1)] for i in range(args.steps)])
+    step_ms = per.sum(axis=1)
+    ms_total = float(step_ms.sum())
+    if world > 1:
+        t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_per_step = ms_total / args.steps
+    value = world * step_flops * args.steps / (ms_total * 1e-3) / 1e12
+
+    peaks, peaks_kind = load_peaks()
+    ring_ms = float(per[:, 0].mean())
+    ring_tflops = attn_flops / (ring_ms * 1e-3) / 1e12
+    uattn_ms = float(per[:, 4].mean())
+    perm_ms = float(per[:, 1:4].mean())
+    unperm_ms = float(per[:, 5].mean())
+    tensor_bytes = B * S * H * D * 2
+    peak_tf = float(peaks["bf16_tflops"])
+    roofline = {"bound": "tensor", "kernel": "attn_fwd_kernel<128,bf16> (ring fused, P=4)",
+                "achieved": ring_tflops, "peak": peak_tf, "unit": "TFLOP/s", "frac": ring_tflops / peak_tf,
+                "peak_kind": f"bf16_tflops burst, {peaks_kind}",
+                "traffic": stored_traffic("attn_fwd_ring_dit"),
+                "algorithmic_flops_per_launch": attn_flops}
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if True:
+        hout_r = torch.empty_like(out_r, device="cpu").pin_memory()
+        hout_u = torch.empty_like(out_u, device="cpu").pin_memory()
+        e2e_steps = max(3, min(args.steps, 50))
+        for _ in range(2):
+            q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True); v.copy_(hv, non_blocking=True)
+            step()
+            hout_r.copy_(out_r, non_blocking=True); hout_u.copy_(out_u, non_blocking=True)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True); v.copy_(hv, non_blocking=True)
+            step()
+            hout_r.copy_(out_r, non_blocking=True); hout_u.copy_(out_u, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / e2e_steps
+        e2e = {"value": world * step_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": 3 * tensor_bytes, "d2h_bytes_per_step": 2 * tensor_bytes,
+               "note": "pinned host Q/K/V copied in and both attention outputs copied out every step"}
+
+    kernels = {
+        "ring_fused_attention": {"ms": ring_ms, "TFLOP/s": ring_tflops, "frac_bf16_peak": ring_tflops / peak_tf},
+        "head_sharded_attention": {"ms": uattn_ms, "TFLOP/s": attn_flops / (uattn_ms * 1e-3) / 1e12,
+                                   "frac_bf16_peak": attn_flops / (uattn_ms * 1e-3) / 1e12 / peak_tf},
+        "ulysses_permute_dit": {"ms": perm_ms, "GB/s": 2 * tensor_bytes / (perm_ms * 1e-3) / 1e9},
+        "ulysses_unpermute_dit": {"ms": unperm_ms, "GB/s": 2 * tensor_bytes / (unperm_ms * 1e-3) / 1e9},
+    }
+    if not args.no_breakdown:
+        kernels.update(breakdown(api, torch, dev, flush, peaks, inputs))
+
+    st, code = api.cpattn_device_status()
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1), RMS-normalised Q/K, bf16)",
+        "config": config_block(cfg), "roofline": roofline, "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks.summary(t_wall0, t_wall1), "e2e": e2e, "kernels": kernels,
+        "device_status": code,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, qb, kb, vb)
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def breakdown(api, torch, dev, flush, peaks, inputs):
+    """HBM-bound kernels on tensors larger than L2 (video-DiT sizes), each rep
+    after an L2 flush: Ulysses permute / unpermute (degree 2, bf16) and the
+    8-way LSE merge of float32 partials."""
+    vcfg = inputs.CONFIGS["video"]
+    B, S, H, D = vcfg["B"], vcfg["S"], vcfg["H"], vcfg["D"]
+    hbm = float(peaks["hbm_gbs"])
+    n = B * S * H * D
+    x = torch.randn(n, device=dev).to(torch.bfloat16)
+    y = torch.empty_like(x)
+    stream = torch.cuda.current_stream()
+    res = {}
+
+    def timeit(fn, reps=10):
+        fn()
+        times = []
+        for _ in range(reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            b.synchronize()
+            times.append(a.elapsed_time(b))
+        return float(np.median(times))
+
+    ms = timeit(lambda: api.cpattn_ulysses_permute(x, B, S, H, D, 2, y=y, stream=stream))
+    gbs = 2 * n * 2 / (ms * 1e-3) / 1e9
+    res["ulysses_permute_video"] = {"ms": ms, "GB/s": gbs, "frac_hbm": gbs / hbm, "bytes": 4 * n}
+    ms = timeit(lambda: api.cpattn_ulysses_unpermute(y, B, S, H, D, 2, x=x, stream=stream))
+    gbs = 2 * n * 2 / (ms * 1e-3) / 1e9
+    res["ulysses_unpermute_video"] = {"ms": ms, "GB/s": gbs, "frac_hbm": gbs / hbm, "bytes": 4 * n}
+    del x, y
+    P = 8
+    po = torch.randn((P, B, S, H, D), device=dev, dtype=torch.float32)
+    pl = torch.randn((P, B, H, S), device=dev, dtype=torch.float32)
+    ob = torch.empty((B, S, H, D), device=dev, dtype=torch.bfloat16)
+    lo = torch.empty((B, H, S), device=dev, dtype=torch.float32)
+    ms = timeit(lambda: api.cpattn_lse_merge(po, pl, out_bf16=ob, lse_out=lo, want_f32=False, stream=stream))
+    mbytes = B * H * S * (P * (4 * D + 4) + 2 * D + 4)
+    gbs = mbytes / (ms * 1e-3) / 1e9
+    res["lse_merge_video_p8"] = {"ms": ms, "GB/s": gbs, "frac_hbm": gbs / hbm, "bytes": mbytes}
+    del po, pl, ob, lo
+    torch.cuda.empty_cache()
+    return res
+
+
+if __name__ == "__main__":
+    main()

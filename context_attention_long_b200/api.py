@@ -1,0 +1,216 @@
+"""Thin PyTorch binding of the C ABI (include/cpattn.h), same function names.
+
+Argument marshalling only: shapes and pointers are read from torch tensors,
+outputs are allocated with torch when not given, and every step of the hot path
+runs in libcpattn.so's CUDA kernels on the current (or given) CUDA stream.
+There is no CPU path: calling without a CUDA device or without the built
+library raises.
+
+Layouts: Q/K/V/out are bf16 (B, S, H, D) contiguous; LSE is float32 (B, H, S),
+natural log.  See include/cpattn.h for the exact semantics of each call.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _native
+
+__all__ = [
+    "CpattnError", "cpattn_ring_attention", "cpattn_ring_step", "cpattn_lse_merge",
+    "cpattn_kv_gather_attention", "cpattn_ulysses_permute", "cpattn_ulysses_unpermute",
+    "cpattn_head_sharded_attention", "cpattn_ulysses_attention", "cpattn_unified_attention",
+    "cpattn_ulysses_workspace_bytes", "cpattn_unified_workspace_bytes",
+    "cpattn_front_loaded_splits", "cpattn_device_status", "cpattn_debug_wait_timeout",
+    "status_string",
+]
+
+
+class CpattnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+def status_string(status: int) -> str:
+    return _native.load().cpattn_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise CpattnError(status, where)
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _bshd(q: torch.Tensor, name="q"):
+    if q.dim() != 4:
+        raise ValueError(f"{name} must be (B, S, H, D)")
+    if not q.is_cuda or q.dtype != torch.bfloat16 or not q.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+    B, S, H, D = q.shape
+    return B, S, H, D
+
+
+def cpattn_ring_attention(q, k, v, ring_degree, chunk_lens=None, out=None, lse=None, want_lse=True, stream=None):
+    """Fused ring attention; returns (out bf16 (B,S,H,D), lse float32 (B,H,S) or None)."""
+    B, S, H, D = _bshd(q)
+    out = torch.empty_like(q) if out is None else out
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    _check(_native.load().cpattn_ring_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, S, D,
+                                                int(ring_degree), _native.int_array(chunk_lens), _stream(stream)),
+           "cpattn_ring_attention")
+    return out, lse
+
+
+def cpattn_ring_step(q, k, v, ring_degree, step, chunk_lens=None, part_out=None, part_lse=None, stream=None):
+    """One ring step for every rank; returns float32 (partial out (B,S,H,D), partial lse (B,H,S))."""
+    B, S, H, D = _bshd(q)
+    if part_out is None:
+        part_out = torch.empty((B, S, H, D), dtype=torch.float32, device=q.device)
+    if part_lse is None:
+        part_lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    _check(_native.load().cpattn_ring_step(_ptr(q), _ptr(k), _ptr(v), _ptr(part_out), _ptr(part_lse), B, H, S, D,
+                                           int(ring_degree), _native.int_array(chunk_lens), int(step),
+                                           _stream(stream)), "cpattn_ring_step")
+    return part_out, part_lse
+
+
+def cpattn_lse_merge(part_out, part_lse, out_f32=None, out_bf16=None, lse_out=None, want_f32=False,
+                     want_bf16=True, stream=None):
+    """Merge P float32 partials: part_out (P,B,S,H,D), part_lse (P,B,H,S).
+    Returns (out_f32 or None, out_bf16 or None, lse_out)."""
+    P, B, S, H, D = part_out.shape
+    dev = part_out.device
+    if out_f32 is None and want_f32:
+        out_f32 = torch.empty((B, S, H, D), dtype=torch.float32, device=dev)
+    if out_bf16 is None and want_bf16:
+        out_bf16 = torch.empty((B, S, H, D), dtype=torch.bfloat16, device=dev)
+    if lse_out is None:
+        lse_out = torch.empty((B, H, S), dtype=torch.float32, device=dev)
+    _check(_native.load().cpattn_lse_merge(_ptr(part_out), _ptr(part_lse), P, B, H, S, D, _ptr(out_f32),
+                                           _ptr(out_bf16), _ptr(lse_out), _stream(stream)), "cpattn_lse_merge")
+    return out_f32, out_bf16, lse_out
+
+
+def cpattn_kv_gather_attention(q, k, v, degree, q_lens=None, out=None, lse=None, want_lse=True, stream=None):
+    """kv_gather attention; returns (out, lse)."""
+    B, S, H, D = _bshd(q)
+    out = torch.empty_like(q) if out is None else out
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    _check(_native.load().cpattn_kv_gather_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, S, D,
+                                                     int(degree), _native.int_array(q_lens), _stream(stream)),
+           "cpattn_kv_gather_attention")
+    return out, lse
+
+
+def _flat_numel(B, S, H, D):
+    return B * S * H * D
+
+
+def cpattn_ulysses_permute(x, B, S, H, D, degree, seq_splits=None, head_splits=None, y=None, stream=None):
+    """Sequence-sharded rank buffers (flat, any 1/2/4/8-byte dtype) -> head-sharded rank buffers."""
+    if y is None:
+        y = torch.empty_like(x)
+    _check(_native.load().cpattn_ulysses_permute(_ptr(x), _ptr(y), B, S, H, D, x.element_size(), int(degree),
+                                                 _native.int_array(seq_splits), _native.int_array(head_splits),
+                                                 _stream(stream)), "cpattn_ulysses_permute")
+    return y
+
+
+def cpattn_ulysses_unpermute(y, B, S, H, D, degree, seq_splits=None, head_splits=None, x=None, stream=None):
+    """Head-sharded rank buffers -> sequence-sharded rank buffers (inverse permute)."""
+    if x is None:
+        x = torch.empty_like(y)
+    _check(_native.load().cpattn_ulysses_unpermute(_ptr(y), _ptr(x), B, S, H, D, y.element_size(), int(degree),
+                                                   _native.int_array(seq_splits), _native.int_array(head_splits),
+                                                   _stream(stream)), "cpattn_ulysses_unpermute")
+    return x
+
+
+def cpattn_head_sharded_attention(yq, yk, yv, B, S, H, D, degree, head_splits=None, yo=None, lse=None,
+                                  want_lse=True, stream=None):
+    """Local attention on head-sharded rank buffers; returns (yo, lse (B,H,S))."""
+    yo = torch.empty_like(yq) if yo is None else yo
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, S), dtype=torch.float32, device=yq.device)
+    _check(_native.load().cpattn_head_sharded_attention(_ptr(yq), _ptr(yk), _ptr(yv), _ptr(yo), _ptr(lse), B, H, S,
+                                                        D, int(degree), _native.int_array(head_splits),
+                                                        _stream(stream)), "cpattn_head_sharded_attention")
+    return yo, lse
+
+
+def cpattn_ulysses_workspace_bytes(B, H, S, D) -> int:
+    return int(_native.load().cpattn_ulysses_workspace_bytes(B, H, S, D))
+
+
+def cpattn_unified_workspace_bytes(B, H, S, D) -> int:
+    return int(_native.load().cpattn_unified_workspace_bytes(B, H, S, D))
+
+
+def _workspace(nbytes, device, workspace):
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    return workspace
+
+
+def cpattn_ulysses_attention(q, k, v, B, S, H, D, degree, seq_splits=None, head_splits=None, out=None, lse=None,
+                             want_lse=True, workspace=None, stream=None):
+    """Ulysses attention on sequence-sharded rank buffers (flat bf16); returns (out, lse)."""
+    out = torch.empty_like(q) if out is None else out
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    nbytes = cpattn_ulysses_workspace_bytes(B, H, S, D)
+    workspace = _workspace(nbytes, q.device, workspace)
+    _check(_native.load().cpattn_ulysses_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, S, D,
+                                                   int(degree), _native.int_array(seq_splits),
+                                                   _native.int_array(head_splits), _ptr(workspace),
+                                                   workspace.numel() * workspace.element_size(), _stream(stream)),
+           "cpattn_ulysses_attention")
+    return out, lse
+
+
+def cpattn_unified_attention(q, k, v, ring_degree, ulysses_degree, ring_lens=None, head_splits=None, out=None,
+                             lse=None, want_lse=True, workspace=None, stream=None):
+    """Unified ring x Ulysses attention on full (B,S,H,D) tensors; returns (out, lse)."""
+    B, S, H, D = _bshd(q)
+    out = torch.empty_like(q) if out is None else out
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    nbytes = cpattn_unified_workspace_bytes(B, H, S, D)
+    workspace = _workspace(nbytes, q.device, workspace)
+    _check(_native.load().cpattn_unified_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, S, D,
+                                                   int(ring_degree), int(ulysses_degree),
+                                                   _native.int_array(ring_lens), _native.int_array(head_splits),
+                                                   _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                                   _stream(stream)), "cpattn_unified_attention")
+    return out, lse
+
+
+def cpattn_front_loaded_splits(total, parts):
+    arr = (ctypes.c_int * max(1, int(parts)))()
+    _check(_native.load().cpattn_front_loaded_splits(int(total), int(parts), arr), "cpattn_front_loaded_splits")
+    return [int(arr[i]) for i in range(int(parts))]
+
+
+def cpattn_device_status(stream=None):
+    """Synchronise the stream and read-and-clear the device status word.
+    Returns (status, code)."""
+    code = ctypes.c_uint(0)
+    st = _native.load().cpattn_device_status(_stream(stream), ctypes.byref(code))
+    return int(st), int(code.value)
+
+
+def cpattn_debug_wait_timeout(timeout_us, stream=None):
+    _check(_native.load().cpattn_debug_wait_timeout(int(timeout_us), _stream(stream)), "cpattn_debug_wait_timeout")

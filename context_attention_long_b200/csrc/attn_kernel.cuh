@@ -1,0 +1,390 @@
+// attn_kernel.cuh -- blockwise non-causal softmax attention for sm_100a.
+//
+// What it computes (diffusers "Context parallelism", "Ring Attention": each
+// GPU computes attention against the K/V block it holds, then passes it on;
+// diffusers "parallel", convert_to_fp32: output and LSE kept in float32;
+// SGLang "Sequence Parallelism", "Numerics across node boundaries": the
+// partial results are combined by an online-softmax merge):
+//   for a 128-row Q tile and the K/V row ranges of its segment, visited in the
+//   order given (ring order for ring attention), one 128-key tile at a time:
+//     S = Q K^T                      (tcgen05.mma, bf16 x bf16 -> f32 in TMEM)
+//     m <- max(m, rowmax(S) * c)     (c = D**-0.5 * log2 e; the stored m is only
+//                                     raised when it grows by more than 8, so
+//                                     O and l are rescaled rarely -- exact either way)
+//     P = 2^(S*c - m)                (registers, bf16 into TMEM over S)
+//     O = O * 2^(m_old - m) + P V    (tcgen05.mma, P from TMEM, V from smem)
+//     l = l * 2^(m_old - m) + rowsum(P)
+//   out = O / l, LSE = (m + log2 l) * ln 2.
+// The running (m, l, O) state *is* the LSE merge applied one chunk (and one
+// tile) at a time, so ring attention is one launch with no partials in HBM.
+//
+// CTA organisation (one CTA per SM: 192 KB smem, 512 TMEM columns):
+//   warp 0      TMA producer: Q once, then K and V tiles into 2-stage rings
+//   warp 1      TMEM allocator + single-thread MMA issuer
+//   warps 2-3   idle
+//   warps 4-7   softmax + correction + epilogue for Q tile 0 (one row per thread)
+//   warps 8-11  the same for Q tile 1
+// TMEM columns: S0 [0,128)  S1 [128,256)  O0 [256, 256+D)  O1 [256+D, 256+2D);
+// P_i (bf16 pairs) overwrites S_i columns [0, 64).
+// MMA order per K/V tile j: PV0(j), QK0(j+1), PV1(j), QK1(j+1), so that the
+// tensor core works on one Q tile while the other one's softmax runs.  A commit
+// after QK_i(j) also covers PV_i(j-1), so when softmax i sees S_i(j), O_i
+// already holds every tile before j and may be rescaled in place.
+#pragma once
+
+#include "cpattn_internal.h"
+#include "cpattn_ptx.cuh"
+
+namespace cpattn {
+
+template <int D>
+struct AttnSmem {
+  static constexpr int kHalves = D / 64;             // 64-element (128-byte) column blocks
+  static constexpr int kBoxBytes = 128 * 128;        // [128 rows][64 bf16], 128B-swizzled
+  static constexpr int kTileBytes = kHalves * kBoxBytes;
+  static constexpr int kStages = 2;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kOffQ + kQTilesPerCTA * kTileBytes;
+  static constexpr int kOffV = kOffK + kStages * kTileBytes;
+  static constexpr int kOffBar = kOffV + kStages * kTileBytes;
+  // q, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2], o_final[2], tail
+  static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 2 + 1;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kBytes = kOffMisc + 16;
+  static constexpr int kAllocBytes = kBytes + 1024;  // slack to align the base to 1024
+};
+
+constexpr int kAttnThreads = 384;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale only if the max grows by > 2^8
+
+template <int D, bool OUT_F32>
+__global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnParams p) {
+  using L = AttnSmem<D>;
+  constexpr int NST = L::kStages;
+  constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, kKVTile, false);
+  constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, true);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
+  uint64_t *bar_q = bars;
+  uint64_t *bar_kf = bars + 1;
+  uint64_t *bar_ke = bar_kf + NST;
+  uint64_t *bar_vf = bar_ke + NST;
+  uint64_t *bar_ve = bar_vf + NST;
+  uint64_t *bar_s = bar_ve + NST;
+  uint64_t *bar_p = bar_s + 2;
+  uint64_t *bar_o = bar_p + 2;
+  uint64_t *bar_tail = bar_o + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint64_t tmo = p.timeout_ns;
+
+  // ---- which unit: group -> head -> segment -> pair of Q tiles
+  const int unit = blockIdx.x;
+  int gi = 0;
+  while (gi + 1 < p.num_groups && p.group[gi + 1].unit_base <= unit) ++gi;
+  const AttnGroup &G = p.group[gi];
+  const int local = unit - G.unit_base;
+  const int h = local / G.tiles_per_head;
+  const int t = local - h * G.tiles_per_head;
+  int si = G.seg_first;
+  while (si + 1 < G.seg_first + G.seg_count && p.seg[si + 1].tile_base <= t) ++si;
+  const AttnSeg &SG = p.seg[si];
+  const AttnProblem &PB = p.prob[G.prob];
+  const int pair = t - SG.tile_base;
+  const int q_row0 = SG.row0 + pair * (kQTilesPerCTA * kQTile);
+  const int rows_left = SG.nrows - pair * (kQTilesPerCTA * kQTile);
+  const bool has_q1 = rows_left > kQTile;
+  int n_tiles = 0;
+  for (int i = 0; i < SG.kv_count; ++i) n_tiles += (p.kv[SG.kv_first + i].nrows + kKVTile - 1) / kKVTile;
+
+  // ---- setup
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&bar_kf[s], 1);
+      mbar_init(&bar_ke[s], 1);
+      mbar_init(&bar_vf[s], 1);
+      mbar_init(&bar_ve[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar_s[i], 1);
+      mbar_init(&bar_p[i], 4);  // one arrival per softmax warp
+      mbar_init(&bar_o[i], 1);
+    }
+    mbar_init(bar_tail, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&PB.tm_q);
+    tma_prefetch_desc(&PB.tm_k);
+    tma_prefetch_desc(&PB.tm_v);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // =========================================================== producer
+    if (lane == 0 && n_tiles > 0) {
+      uint8_t *sQ = smem + L::kOffQ;
+      mbar_arrive_expect_tx(bar_q, (has_q1 ? 2 : 1) * L::kTileBytes);
+      for (int hf = 0; hf < L::kHalves; ++hf)
+        tma_load_3d(sQ + hf * L::kBoxBytes, &PB.tm_q, hf * 64, h, q_row0, bar_q);
+      if (has_q1)
+        for (int hf = 0; hf < L::kHalves; ++hf)
+          tma_load_3d(sQ + L::kTileBytes + hf * L::kBoxBytes, &PB.tm_q, hf * 64, h, q_row0 + kQTile, bar_q);
+      int it = 0;
+      bool ok = true;
+      for (int i = 0; ok && i < SG.kv_count; ++i) {
+        const AttnKV kv = p.kv[SG.kv_first + i];
+        for (int r = 0; r < kv.nrows; r += kKVTile, ++it) {
+          const int st = it % NST;
+          const uint32_t ph = (it / NST) & 1;
+          if (!mbar_wait(&bar_ke[st], ph ^ 1, abort_flag, tmo, SITE_PRODUCER)) { ok = false; break; }
+          mbar_arrive_expect_tx(&bar_kf[st], L::kTileBytes);
+          uint8_t *sK = smem + L::kOffK + st * L::kTileBytes;
+          for (int hf = 0; hf < L::kHalves; ++hf)
+            tma_load_3d(sK + hf * L::kBoxBytes, &PB.tm_k, hf * 64, h, kv.row0 + r, &bar_kf[st]);
+          if (!mbar_wait(&bar_ve[st], ph ^ 1, abort_flag, tmo, SITE_PRODUCER)) { ok = false; break; }
+          mbar_arrive_expect_tx(&bar_vf[st], L::kTileBytes);
+          uint8_t *sV = smem + L::kOffV + st * L::kTileBytes;
+          for (int hf = 0; hf < L::kHalves; ++hf)
+            tma_load_3d(sV + hf * L::kBoxBytes, &PB.tm_v, hf * 64, h, kv.row0 + r, &bar_vf[st]);
+        }
+      }
+      // Tail: every stage's last use must be released by the MMA before the
+      // CTA exits (the releases are asynchronous arrivals on our barriers).
+      for (int st = 0; st < NST && st < n_tiles; ++st) {
+        const int last = st + ((n_tiles - 1 - st) / NST) * NST;
+        const uint32_t ph = (last / NST) & 1;
+        mbar_wait(&bar_ke[st], ph, nullptr, tmo, SITE_TAIL);
+        mbar_wait(&bar_ve[st], ph, nullptr, tmo, SITE_TAIL);
+      }
+    }
+  } else if (warp == 1) {
+    // =========================================================== MMA issuer
+    if (lane == 0 && n_tiles > 0) {
+      const uint32_t sQ = smem_u32(smem + L::kOffQ);
+      const uint32_t sK = smem_u32(smem + L::kOffK);
+      const uint32_t sV = smem_u32(smem + L::kOffV);
+      // S_qt = Q_qt K^T: K-major A and B, 128B swizzle, K advances 16 elements
+      // (32 bytes) inside a 128-byte row, then jumps to the next column block.
+      auto issue_qk = [&](int qt, int st) {
+        const uint32_t d = tmem + qt * 128;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
+          const uint64_t a = smem_desc_sw128(sQ + qt * L::kTileBytes + off, 16, 1024);
+          const uint64_t b = smem_desc_sw128(sK + st * L::kTileBytes + off, 16, 1024);
+          mma_ss(d, a, b, IDESC_QK, kk > 0 ? 1u : 0u);
+        }
+      };
+      // O_qt (+)= P_qt V: P (bf16 pairs) from TMEM over S_qt, V MN-major
+      // (keys are rows of 128 bytes): 16 keys = 2 groups of 8 rows = 2048
+      // bytes per MMA, column blocks of 64 head-dim elements 16 KB apart.
+      auto issue_pv = [&](int qt, int st, bool acc) {
+        const uint32_t d = tmem + 256 + qt * D;
+        const uint32_t a = tmem + qt * 128;
+#pragma unroll
+        for (int kk = 0; kk < kKVTile / 16; ++kk) {
+          const uint64_t b = smem_desc_sw128(sV + st * L::kTileBytes + kk * 2048, L::kBoxBytes, 1024);
+          mma_ts(d, a + kk * 8, b, IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(bar_q, 0, abort_flag, tmo, SITE_MMA);
+      if (ok) ok = mbar_wait(&bar_kf[0], 0, abort_flag, tmo, SITE_MMA);
+      if (ok) {
+        tc_fence_after();
+        issue_qk(0, 0);
+        mma_commit(&bar_s[0]);
+        if (has_q1) {
+          issue_qk(1, 0);
+          mma_commit(&bar_s[1]);
+        }
+        mma_commit(&bar_ke[0]);
+      }
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        const int st = j % NST;
+        const uint32_t ph = (j / NST) & 1;
+        const int st1 = (j + 1) % NST;
+        const uint32_t ph1 = ((j + 1) / NST) & 1;
+        const bool more = j + 1 < n_tiles;
+        if (!mbar_wait(&bar_vf[st], ph, abort_flag, tmo, SITE_MMA)) break;
+        if (!mbar_wait(&bar_p[0], j & 1, abort_flag, tmo, SITE_MMA)) break;
+        tc_fence_after();
+        issue_pv(0, st, j > 0);
+        if (!more) mma_commit(&bar_o[0]);
+        if (more) {
+          if (!mbar_wait(&bar_kf[st1], ph1, abort_flag, tmo, SITE_MMA)) break;
+          tc_fence_after();
+          issue_qk(0, st1);
+          mma_commit(&bar_s[0]);
+        }
+        if (has_q1) {
+          if (!mbar_wait(&bar_p[1], j & 1, abort_flag, tmo, SITE_MMA)) break;
+          tc_fence_after();
+          issue_pv(1, st, j > 0);
+          if (!more) mma_commit(&bar_o[1]);
+        }
+        mma_commit(&bar_ve[st]);
+        if (more) {
+          if (has_q1) {
+            issue_qk(1, st1);
+            mma_commit(&bar_s[1]);
+          }
+          mma_commit(&bar_ke[st1]);
+        }
+      }
+      // Drain: everything issued has completed before TMEM is released.
+      mma_commit(bar_tail);
+      mbar_wait(bar_tail, 0, nullptr, tmo, SITE_TAIL);
+    }
+  } else if (warp >= 4) {
+    // =========================================================== softmax
+    const int qt = (warp - 4) >> 2;
+    const int row = ((warp & 3) << 5) + lane;  // TMEM lane == row of the Q tile
+    const bool active = (qt == 0) || has_q1;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) << 5) << 16;
+    const uint32_t tS = tmem + lane_base + qt * 128;
+    const uint32_t tO = tmem + lane_base + 256 + qt * D;
+    const float c = p.scale_log2;
+    float m = -INFINITY;  // running max, scaled (log2) domain
+    float l = 0.f;        // running sum of 2^(x - m)
+    bool ok = true;
+    if (active && n_tiles > 0) {
+      int j = 0;
+      for (int i = 0; ok && i < SG.kv_count; ++i) {
+        const int kv_n = p.kv[SG.kv_first + i].nrows;
+        for (int r = 0; r < kv_n; r += kKVTile, ++j) {
+          const bool w = mbar_wait(&bar_s[qt], j & 1, abort_flag, tmo, SITE_SOFTMAX);
+          if (__any_sync(0xffffffffu, !w)) { ok = false; break; }
+          __syncwarp();
+          tc_fence_after();
+          uint32_t s[128];
+          tmem_ld128_wait(tS, s);
+          const int kvalid = min(kKVTile, kv_n - r);
+          if (kvalid < kKVTile) {
+#pragma unroll
+            for (int k = 0; k < 128; ++k)
+              if (k >= kvalid) s[k] = __float_as_uint(-INFINITY);
+          }
+          float mx[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mx[k] = __uint_as_float(s[k]);
+#pragma unroll
+          for (int k = 8; k < 128; ++k) mx[k & 7] = fmaxf(mx[k & 7], __uint_as_float(s[k]));
+          const float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * c;
+          if (j == 0) {
+            m = tmax;
+          } else {
+            const bool need = tmax > m + kRescaleThreshold;
+            if (__any_sync(0xffffffffu, need)) {
+              const float alpha = need ? ex2_approx(m - tmax) : 1.0f;
+              if (need) {
+                l *= alpha;
+                m = tmax;
+              }
+#pragma unroll
+              for (int c0 = 0; c0 < D; c0 += 32) {
+                uint32_t o[32];
+                tmem_ld32_wait(tO + c0, o);
+#pragma unroll
+                for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+                tmem_st32(tO + c0, o);
+              }
+            }
+          }
+          const float neg_m = -m;
+          float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int c0 = 0; c0 < 128; c0 += 32) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              const float p0 = ex2_approx(fmaf(__uint_as_float(s[c0 + 2 * k]), c, neg_m));
+              const float p1 = ex2_approx(fmaf(__uint_as_float(s[c0 + 2 * k + 1]), c, neg_m));
+              ls[k & 3] += p0 + p1;
+              pk[k] = pack_bf16x2(p0, p1);
+            }
+            tmem_st16(tS + c0 / 2, pk);
+          }
+          l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar_p[qt]);
+        }
+      }
+      if (ok) {
+        const bool w = mbar_wait(&bar_o[qt], 0, abort_flag, tmo, SITE_EPILOGUE);
+        if (__any_sync(0xffffffffu, !w)) ok = false;
+        __syncwarp();
+        tc_fence_after();
+      }
+    }
+    // =========================================================== epilogue
+    if (active && ok) {
+      const int valid_rows = qt == 0 ? min(kQTile, rows_left) : rows_left - kQTile;
+      const bool row_valid = row < valid_rows;
+      const int grow = q_row0 + qt * kQTile + row;
+      const float inv_l = n_tiles > 0 ? 1.0f / l : 0.0f;
+      const size_t row_elems = (static_cast<size_t>(grow) * PB.H + h) * D;
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t o[32];
+        if (n_tiles > 0) {
+          tmem_ld32_wait(tO + c0, o);
+        } else {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] = 0u;
+        }
+        if (row_valid) {
+          if constexpr (OUT_F32) {
+            float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(PB.out) + row_elems + c0);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              dst[k] = make_float4(__uint_as_float(o[4 * k]) * inv_l, __uint_as_float(o[4 * k + 1]) * inv_l,
+                                   __uint_as_float(o[4 * k + 2]) * inv_l, __uint_as_float(o[4 * k + 3]) * inv_l);
+          } else {
+            uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(PB.out) + row_elems + c0);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              dst[k] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * k]) * inv_l, __uint_as_float(o[8 * k + 1]) * inv_l),
+                                  pack_bf16x2(__uint_as_float(o[8 * k + 2]) * inv_l, __uint_as_float(o[8 * k + 3]) * inv_l),
+                                  pack_bf16x2(__uint_as_float(o[8 * k + 4]) * inv_l, __uint_as_float(o[8 * k + 5]) * inv_l),
+                                  pack_bf16x2(__uint_as_float(o[8 * k + 6]) * inv_l, __uint_as_float(o[8 * k + 7]) * inv_l));
+          }
+        }
+      }
+      if (row_valid && PB.lse != nullptr) {
+        const float lse = n_tiles > 0 ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+        const int s = SG.s0 + pair * (kQTilesPerCTA * kQTile) + qt * kQTile + row;
+        PB.lse[static_cast<long long>(G.b) * PB.lse_b + static_cast<long long>(h + PB.lse_h0) * PB.lse_h + s] = lse;
+      }
+    }
+  }
+
+  // ---- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace cpattn

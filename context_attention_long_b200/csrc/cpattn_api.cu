@@ -1,0 +1,765 @@
+// cpattn_api.cu -- the C ABI of libcpattn.so (declared in include/cpattn.h):
+// argument validation, launch planning (row ranges for every shard / chunk),
+// TMA descriptor encoding and kernel launches.  Single translation unit.
+#include "cpattn.h"
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <memory>
+#include <mutex>
+#include <vector>
+
+#include "cpattn_internal.h"
+#include "cpattn_ptx.cuh"
+#include "attn_kernel.cuh"
+#include "merge_kernel.cuh"
+#include "permute_kernel.cuh"
+
+namespace cpattn {
+
+// ------------------------------------------------------------------ helpers
+
+constexpr int kMaxRingDegree = 1024;
+constexpr int kMaxDevices = 64;
+
+static unsigned long long wait_timeout_ns() {
+  static unsigned long long v = [] {
+    const char *e = std::getenv("CPATTN_WAIT_TIMEOUT_MS");
+    long long ms = e ? std::atoll(e) : 2000;
+    if (ms < 1) ms = 1;
+    return static_cast<unsigned long long>(ms) * 1000000ull;
+  }();
+  return v;
+}
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+static bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+static int check_attn_shape(int B, int H, int S, int D) {
+  if (B < 1 || H < 1 || S < 1) return CPATTN_ERR_SHAPE;
+  if (D != 64 && D != 128) return CPATTN_ERR_SHAPE;
+  if (static_cast<long long>(B) * S > INT_MAX) return CPATTN_ERR_SHAPE;
+  if (static_cast<long long>(B) * S * H * D > (1ll << 46)) return CPATTN_ERR_SHAPE;
+  return CPATTN_OK;
+}
+
+// Equal split (NULL: total % degree == 0 required, [CP] variants table) or
+// explicit non-negative lengths summing to total ('anything' modes).
+static int resolve_splits(int total, int degree, const int *splits, std::vector<int> &out) {
+  if (degree < 1) return CPATTN_ERR_DEGREE;
+  if (splits == nullptr) {
+    if (degree > total) return CPATTN_ERR_DEGREE;
+    if (total % degree != 0) return CPATTN_ERR_INDIVISIBLE;
+    out.assign(degree, total / degree);
+    return CPATTN_OK;
+  }
+  long long sum = 0;
+  out.resize(degree);
+  for (int i = 0; i < degree; ++i) {
+    if (splits[i] < 0) return CPATTN_ERR_SPLITS;
+    out[i] = splits[i];
+    sum += splits[i];
+  }
+  return sum == total ? CPATTN_OK : CPATTN_ERR_SPLITS;
+}
+
+static std::vector<int> prefix(const std::vector<int> &lens) {
+  std::vector<int> off(lens.size() + 1, 0);
+  for (size_t i = 0; i < lens.size(); ++i) off[i + 1] = off[i] + lens[i];
+  return off;
+}
+
+// Is the current device an sm_100 part?
+static int check_device(int *dev_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return CPATTN_ERR_CUDA;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return CPATTN_ERR_UNSUPPORTED;
+  static int cc_major[kMaxDevices] = {0};
+  if (cc_major[dev] == 0) {
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return CPATTN_ERR_CUDA;
+    }
+    cc_major[dev] = major;
+  }
+  if (cc_major[dev] != 10) return CPATTN_ERR_UNSUPPORTED;
+  if (dev_out) *dev_out = dev;
+  return CPATTN_OK;
+}
+
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess) {
+      cudaGetLastError();
+      ptr = nullptr;
+    }
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }();
+  return fn;
+}
+
+// 3-D view [rows, H, D] of a bf16 tensor, box {64, 1, 128}, 128-byte swizzle.
+static bool encode_rows_map(CUtensorMap *tm, const void *ptr, int D, int H, long long rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2};
+  cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(kQTile)};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ launchers
+
+template <int D, bool F32>
+static cudaError_t launch_attn_t(const AttnParams &p, cudaStream_t stream) {
+  static std::mutex mu;
+  static bool configured[kMaxDevices] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!configured[dev]) {
+      cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, F32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           AttnSmem<D>::kAllocBytes);
+      if (e != cudaSuccess) return e;
+      configured[dev] = true;
+    }
+  }
+  attn_fwd_kernel<D, F32><<<p.total_units, kAttnThreads, AttnSmem<D>::kAllocBytes, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attention(const AttnParams &p, int D, bool out_f32, cudaStream_t stream) {
+  if (p.total_units <= 0) return cudaSuccess;
+  if (D == 128) return out_f32 ? launch_attn_t<128, true>(p, stream) : launch_attn_t<128, false>(p, stream);
+  return out_f32 ? launch_attn_t<64, true>(p, stream) : launch_attn_t<64, false>(p, stream);
+}
+
+static int grid_for(long long work_items, int items_per_block) {
+  long long blocks = (work_items + items_per_block - 1) / items_per_block;
+  blocks = std::max<long long>(1, std::min<long long>(blocks, 148ll * 16));
+  return static_cast<int>(blocks);
+}
+
+template <int D>
+static cudaError_t launch_merge_d(const MergeParams &p, cudaStream_t stream) {
+  const long long nrows = static_cast<long long>(p.B) * p.H * p.S;
+  const int rows_per_block = (kMergeThreads / 32) * (32 / (D / 4));
+  const int grid = grid_for(nrows, rows_per_block);
+  if (p.P <= 2) lse_merge_kernel<D, 2><<<grid, kMergeThreads, 0, stream>>>(p);
+  else if (p.P <= 4) lse_merge_kernel<D, 4><<<grid, kMergeThreads, 0, stream>>>(p);
+  else if (p.P <= 8) lse_merge_kernel<D, 8><<<grid, kMergeThreads, 0, stream>>>(p);
+  else if (p.P <= 16) lse_merge_kernel<D, 16><<<grid, kMergeThreads, 0, stream>>>(p);
+  else lse_merge_kernel_anyp<D><<<grid, kMergeThreads, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_lse_merge(const MergeParams &p, cudaStream_t stream) {
+  return p.D == 128 ? launch_merge_d<128>(p, stream) : launch_merge_d<64>(p, stream);
+}
+
+cudaError_t launch_permute(const PermuteParams &p, cudaStream_t stream) {
+  const long long ntok = static_cast<long long>(p.B) * p.S;
+  const int grid = grid_for(ntok, kPermuteThreads / 32);
+  permute_kernel<<<grid, kPermuteThreads, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+__global__ void debug_wait_kernel(unsigned long long timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    // Nothing ever arrives: the wait must give up after timeout_ns.
+    mbar_wait(&bar, 0, &abort_flag, timeout_ns, SITE_DEBUG);
+  }
+}
+
+cudaError_t launch_debug_wait(unsigned long long timeout_ns, cudaStream_t stream) {
+  debug_wait_kernel<<<1, 32, 0, stream>>>(timeout_ns);
+  return cudaGetLastError();
+}
+
+cudaError_t read_and_clear_device_status(unsigned int *code, cudaStream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return e;
+  unsigned int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v));
+  if (e != cudaSuccess) return e;
+  if (v != 0) {
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero));
+    if (e != cudaSuccess) return e;
+  }
+  *code = v;
+  return cudaSuccess;
+}
+
+// ------------------------------------------------------------ attention plans
+
+struct ProblemSpec {
+  const void *q, *k, *v;
+  void *out;
+  float *lse;
+  long long lse_b, lse_h;
+  int lse_h0;
+  int H;
+  long long rows;
+};
+struct SegSpec {
+  int row0, nrows, s0;
+  std::vector<AttnKV> kv;
+};
+struct GroupSpec {
+  int prob, b;
+  std::vector<SegSpec> segs;
+};
+
+// Packs the groups into as few launches as the parameter tables allow and
+// launches them in order on `stream`.
+static int run_attention(const std::vector<ProblemSpec> &probs, const std::vector<GroupSpec> &groups, int D,
+                         bool out_f32, cudaStream_t stream) {
+  std::vector<AttnProblem> encoded(probs.size());
+  for (size_t i = 0; i < probs.size(); ++i) {
+    const ProblemSpec &ps = probs[i];
+    AttnProblem &ap = encoded[i];
+    std::memset(&ap, 0, sizeof(ap));
+    if (!encode_rows_map(&ap.tm_q, ps.q, D, ps.H, ps.rows) || !encode_rows_map(&ap.tm_k, ps.k, D, ps.H, ps.rows) ||
+        !encode_rows_map(&ap.tm_v, ps.v, D, ps.H, ps.rows))
+      return CPATTN_ERR_CUDA;
+    ap.out = ps.out;
+    ap.lse = ps.lse;
+    ap.lse_b = ps.lse_b;
+    ap.lse_h = ps.lse_h;
+    ap.lse_h0 = ps.lse_h0;
+    ap.H = ps.H;
+  }
+  const float scale_log2 = static_cast<float>((1.0 / std::sqrt(static_cast<double>(D))) * 1.4426950408889634);
+
+  std::unique_ptr<AttnParams> P(new AttnParams);
+  std::vector<int> prob_slot(probs.size(), -1);
+  int n_prob = 0, n_seg = 0, n_kv = 0;
+  int open_group = -1;  // index into P->group of the group being filled
+
+  auto reset = [&] {
+    std::memset(P.get(), 0, sizeof(AttnParams));
+    std::fill(prob_slot.begin(), prob_slot.end(), -1);
+    n_prob = n_seg = n_kv = 0;
+    open_group = -1;
+    P->scale_log2 = scale_log2;
+    P->timeout_ns = wait_timeout_ns();
+  };
+  auto close_group = [&] {
+    if (open_group >= 0) {
+      AttnGroup &g = P->group[open_group];
+      P->total_units += P->prob[g.prob].H * g.tiles_per_head;
+      open_group = -1;
+    }
+  };
+  auto flush = [&]() -> int {
+    close_group();
+    if (P->total_units > 0) {
+      if (launch_attention(*P, D, out_f32, stream) != cudaSuccess) return CPATTN_ERR_CUDA;
+    }
+    reset();
+    return CPATTN_OK;
+  };
+  reset();
+
+  for (const GroupSpec &gs : groups) {
+    bool group_started_here = false;
+    for (const SegSpec &ss : gs.segs) {
+      if (ss.nrows <= 0) continue;
+      const int need_kv = static_cast<int>(ss.kv.size());
+      if (need_kv > kMaxKV) return CPATTN_ERR_DEGREE;
+      const bool need_prob = prob_slot[gs.prob] < 0;
+      const bool need_group = !group_started_here || open_group < 0;
+      if ((need_prob && n_prob >= kMaxProblems) || (need_group && P->num_groups >= kMaxGroups) ||
+          n_seg >= kMaxSegs || n_kv + need_kv > kMaxKV) {
+        int st = flush();
+        if (st != CPATTN_OK) return st;
+        group_started_here = false;
+      }
+      if (prob_slot[gs.prob] < 0) {
+        prob_slot[gs.prob] = n_prob;
+        P->prob[n_prob++] = encoded[gs.prob];
+      }
+      if (!group_started_here || open_group < 0) {
+        close_group();
+        open_group = P->num_groups++;
+        AttnGroup &g = P->group[open_group];
+        g.prob = prob_slot[gs.prob];
+        g.b = gs.b;
+        g.seg_first = n_seg;
+        g.seg_count = 0;
+        g.tiles_per_head = 0;
+        g.unit_base = P->total_units;
+        group_started_here = true;
+      }
+      AttnGroup &g = P->group[open_group];
+      AttnSeg &sg = P->seg[n_seg++];
+      sg.row0 = ss.row0;
+      sg.nrows = ss.nrows;
+      sg.s0 = ss.s0;
+      sg.kv_first = n_kv;
+      sg.kv_count = need_kv;
+      sg.tile_base = g.tiles_per_head;
+      for (const AttnKV &kv : ss.kv) P->kv[n_kv++] = kv;
+      g.seg_count += 1;
+      g.tiles_per_head += (ss.nrows + kQTilesPerCTA * kQTile - 1) / (kQTilesPerCTA * kQTile);
+    }
+    close_group();
+  }
+  return flush();
+}
+
+static ProblemSpec full_problem(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H,
+                                int S) {
+  ProblemSpec ps;
+  ps.q = q;
+  ps.k = k;
+  ps.v = v;
+  ps.out = out;
+  ps.lse = lse;
+  ps.lse_b = static_cast<long long>(H) * S;
+  ps.lse_h = S;
+  ps.lse_h0 = 0;
+  ps.H = H;
+  ps.rows = static_cast<long long>(B) * S;
+  return ps;
+}
+
+// Ring plan over a [rows, H, D] tensor whose batch-b chunk c occupies rows
+// row_of(b, c) .. + lens[c]; `step` < 0: all chunks in ring order (fused);
+// otherwise only chunk (r - step) mod P.
+template <class RowOf>
+static void ring_groups(std::vector<GroupSpec> &groups, int prob, int B, const std::vector<int> &lens,
+                        const std::vector<int> &off, int step, RowOf row_of) {
+  const int P = static_cast<int>(lens.size());
+  for (int b = 0; b < B; ++b) {
+    GroupSpec g;
+    g.prob = prob;
+    g.b = b;
+    for (int r = 0; r < P; ++r) {
+      SegSpec s;
+      s.row0 = row_of(b, r);
+      s.nrows = lens[r];
+      s.s0 = off[r];
+      for (int t = 0; t < P; ++t) {
+        if (step >= 0 && t != step) continue;
+        const int c = ((r - t) % P + P) % P;  // chunk held by rank r after t hand-offs
+        if (lens[c] > 0) s.kv.push_back(AttnKV{row_of(b, c), lens[c]});
+      }
+      g.segs.push_back(std::move(s));
+    }
+    groups.push_back(std::move(g));
+  }
+}
+
+static int permute_common(const void *src, void *dst, int B, int S, int H, int D, int elem_bytes, int degree,
+                          const int *seq_splits, const int *head_splits, int direction, PermuteParams &pp) {
+  if (src == nullptr || dst == nullptr) return CPATTN_ERR_NULL;
+  if (B < 1 || S < 1 || H < 1 || D < 1) return CPATTN_ERR_SHAPE;
+  if (elem_bytes != 1 && elem_bytes != 2 && elem_bytes != 4 && elem_bytes != 8) return CPATTN_ERR_SHAPE;
+  if ((static_cast<long long>(D) * elem_bytes) % 16 != 0 || static_cast<long long>(D) * elem_bytes > (1 << 20))
+    return CPATTN_ERR_SHAPE;
+  if (H > kMaxHeads || static_cast<long long>(B) * S > INT_MAX) return CPATTN_ERR_SHAPE;
+  if (degree < 1 || degree > kMaxRanks) return CPATTN_ERR_DEGREE;
+  std::vector<int> seq, heads;
+  int st = resolve_splits(S, degree, seq_splits, seq);
+  if (st != CPATTN_OK) return st;
+  st = resolve_splits(H, degree, head_splits, heads);
+  if (st != CPATTN_OK) return st;
+  if (!aligned16(src) || !aligned16(dst)) return CPATTN_ERR_ALIGNMENT;
+  std::memset(&pp, 0, sizeof(pp));
+  pp.src = static_cast<const unsigned char *>(src);
+  pp.dst = static_cast<unsigned char *>(dst);
+  pp.B = B;
+  pp.S = S;
+  pp.H = H;
+  pp.row_bytes = D * elem_bytes;
+  pp.direction = direction;
+  pp.seq_mode = 1;
+  pp.n_seq = degree;
+  std::vector<int> so = prefix(seq), ho = prefix(heads);
+  for (int i = 0; i <= degree; ++i) {
+    pp.seq_off[i] = so[i];
+    pp.head_off[i] = ho[i];
+  }
+  pp.n_groups = 1;
+  pp.group_off[0] = 0;
+  pp.group_off[1] = S;
+  pp.n_head = degree;
+  return CPATTN_OK;
+}
+
+}  // namespace cpattn
+
+using namespace cpattn;
+
+// =================================================================== C ABI
+
+extern "C" {
+
+const char *cpattn_status_string(int status) {
+  switch (status) {
+    case CPATTN_OK: return "CPATTN_OK";
+    case CPATTN_ERR_NULL: return "CPATTN_ERR_NULL: a required pointer is NULL";
+    case CPATTN_ERR_SHAPE: return "CPATTN_ERR_SHAPE: unsupported shape";
+    case CPATTN_ERR_INDIVISIBLE: return "CPATTN_ERR_INDIVISIBLE: length not divisible by the degree (pass explicit splits)";
+    case CPATTN_ERR_SPLITS: return "CPATTN_ERR_SPLITS: negative lengths or lengths not summing to the total";
+    case CPATTN_ERR_DEGREE: return "CPATTN_ERR_DEGREE: degree or step out of range";
+    case CPATTN_ERR_CUDA: return "CPATTN_ERR_CUDA: CUDA runtime/driver error";
+    case CPATTN_ERR_DEVICE_TIMEOUT: return "CPATTN_ERR_DEVICE_TIMEOUT: a device-side bounded wait expired";
+    case CPATTN_ERR_WORKSPACE: return "CPATTN_ERR_WORKSPACE: workspace missing or too small";
+    case CPATTN_ERR_ALIGNMENT: return "CPATTN_ERR_ALIGNMENT: tensor pointer not 16-byte aligned";
+    case CPATTN_ERR_UNSUPPORTED: return "CPATTN_ERR_UNSUPPORTED: current device is not sm_100";
+    default: return "CPATTN: unknown status";
+  }
+}
+
+int cpattn_version(void) { return 1 * 10000 + 0 * 100 + 0; }
+
+int cpattn_front_loaded_splits(int total, int parts, int *out) {
+  if (out == nullptr) return CPATTN_ERR_NULL;
+  if (parts < 1) return CPATTN_ERR_DEGREE;
+  if (total < 0) return CPATTN_ERR_SHAPE;
+  const int base = total / parts, rem = total % parts;
+  for (int i = 0; i < parts; ++i) out[i] = base + (i < rem ? 1 : 0);
+  return CPATTN_OK;
+}
+
+static int ring_common(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H, int S, int D,
+                       int ring_degree, const int *chunk_lens, int step, bool out_f32, cudaStream_t stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return CPATTN_ERR_NULL;
+  if (out_f32 && lse == nullptr) return CPATTN_ERR_NULL;
+  int st = check_attn_shape(B, H, S, D);
+  if (st != CPATTN_OK) return st;
+  if (ring_degree < 1 || ring_degree > kMaxRingDegree) return CPATTN_ERR_DEGREE;
+  if (step >= ring_degree) return CPATTN_ERR_DEGREE;
+  std::vector<int> lens;
+  st = resolve_splits(S, ring_degree, chunk_lens, lens);
+  if (st != CPATTN_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || (lse && !aligned4(lse)))
+    return CPATTN_ERR_ALIGNMENT;
+  st = check_device(nullptr);
+  if (st != CPATTN_OK) return st;
+  const std::vector<int> off = prefix(lens);
+  std::vector<ProblemSpec> probs{full_problem(q, k, v, out, lse, B, H, S)};
+  std::vector<GroupSpec> groups;
+  ring_groups(groups, 0, B, lens, off, step,
+              [&](int b, int c) { return b * S + off[c]; });
+  return run_attention(probs, groups, D, out_f32, stream);
+}
+
+int cpattn_ring_attention(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H, int S,
+                          int D, int ring_degree, const int *chunk_lens, cpattn_stream_t stream) {
+  return ring_common(q, k, v, out, lse, B, H, S, D, ring_degree, chunk_lens, -1, false, stream);
+}
+
+int cpattn_ring_step(const void *q, const void *k, const void *v, float *part_out, float *part_lse, int B, int H,
+                     int S, int D, int ring_degree, const int *chunk_lens, int step, cpattn_stream_t stream) {
+  if (step < 0) return CPATTN_ERR_DEGREE;
+  return ring_common(q, k, v, part_out, part_lse, B, H, S, D, ring_degree, chunk_lens, step, true, stream);
+}
+
+int cpattn_lse_merge(const float *part_out, const float *part_lse, int P, int B, int H, int S, int D, float *out_f32,
+                     void *out_bf16, float *lse_out, cpattn_stream_t stream) {
+  if (part_out == nullptr || part_lse == nullptr) return CPATTN_ERR_NULL;
+  if (out_f32 == nullptr && out_bf16 == nullptr) return CPATTN_ERR_NULL;
+  if (P < 1) return CPATTN_ERR_SHAPE;
+  int st = check_attn_shape(B, H, S, D);
+  if (st != CPATTN_OK) return st;
+  if (!aligned16(part_out) || !aligned4(part_lse) || (out_f32 && !aligned16(out_f32)) ||
+      (out_bf16 && !aligned16(out_bf16)) || (lse_out && !aligned4(lse_out)))
+    return CPATTN_ERR_ALIGNMENT;
+  st = check_device(nullptr);
+  if (st != CPATTN_OK) return st;
+  MergeParams mp;
+  mp.part_out = part_out;
+  mp.part_lse = part_lse;
+  mp.out_f32 = out_f32;
+  mp.out_bf16 = static_cast<__nv_bfloat16 *>(out_bf16);
+  mp.lse_out = lse_out;
+  mp.P = P;
+  mp.B = B;
+  mp.H = H;
+  mp.S = S;
+  mp.D = D;
+  return launch_lse_merge(mp, stream) == cudaSuccess ? CPATTN_OK : CPATTN_ERR_CUDA;
+}
+
+int cpattn_kv_gather_attention(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H,
+                               int S, int D, int degree, const int *q_lens, cpattn_stream_t stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return CPATTN_ERR_NULL;
+  int st = check_attn_shape(B, H, S, D);
+  if (st != CPATTN_OK) return st;
+  if (degree < 1 || degree > kMaxRingDegree) return CPATTN_ERR_DEGREE;
+  std::vector<int> lens;
+  st = resolve_splits(S, degree, q_lens, lens);
+  if (st != CPATTN_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || (lse && !aligned4(lse)))
+    return CPATTN_ERR_ALIGNMENT;
+  st = check_device(nullptr);
+  if (st != CPATTN_OK) return st;
+  const std::vector<int> off = prefix(lens);
+  std::vector<ProblemSpec> probs{full_problem(q, k, v, out, lse, B, H, S)};
+  std::vector<GroupSpec> groups;
+  for (int b = 0; b < B; ++b) {
+    GroupSpec g;
+    g.prob = 0;
+    g.b = b;
+    for (int r = 0; r < degree; ++r) {
+      SegSpec s;
+      s.row0 = b * S + off[r];
+      s.nrows = lens[r];
+      s.s0 = off[r];
+      s.kv.push_back(AttnKV{b * S, S});   // the gathered, full K/V of batch b
+      g.segs.push_back(std::move(s));
+    }
+    groups.push_back(std::move(g));
+  }
+  return run_attention(probs, groups, D, false, stream);
+}
+
+int cpattn_ulysses_permute(const void *x, void *y, int B, int S, int H, int D, int elem_bytes, int degree,
+                           const int *seq_splits, const int *head_splits, cpattn_stream_t stream) {
+  PermuteParams pp;
+  int st = permute_common(x, y, B, S, H, D, elem_bytes, degree, seq_splits, head_splits, 0, pp);
+  if (st != CPATTN_OK) return st;
+  st = check_device(nullptr);
+  if (st != CPATTN_OK) return st;
+  return launch_permute(pp, stream) == cudaSuccess ? CPATTN_OK : CPATTN_ERR_CUDA;
+}
+
+int cpattn_ulysses_unpermute(const void *y, void *x, int B, int S, int H, int D, int elem_bytes, int degree,
+                             const int *seq_splits, const int *head_splits, cpattn_stream_t stream) {
+  PermuteParams pp;
+  int st = permute_common(y, x, B, S, H, D, elem_bytes, degree, seq_splits, head_splits, 1, pp);
+  if (st != CPATTN_OK) return st;
+  st = check_device(nullptr);
+  if (st != CPATTN_OK) return st;
+  return launch_permute(pp, stream) == cudaSuccess ? CPATTN_OK : CPATTN_ERR_CUDA;
+}
+
+// Head-sharded problems: head rank u's buffers start at element B*S*hoff_u*D.
+static void head_sharded_problems(std::vector<ProblemSpec> &probs, std::vector<int> &prob_rank, const void *yq,
+                                  const void *yk, const void *yv, void *yo, float *lse, int B, int H, int S, int D,
+                                  const std::vector<int> &heads) {
+  const std::vector<int> ho = prefix(heads);
+  for (size_t u = 0; u < heads.size(); ++u) {
+    if (heads[u] == 0) continue;
+    const size_t off_bytes = static_cast<size_t>(B) * S * ho[u] * D * 2;
+    ProblemSpec ps;
+    ps.q = static_cast<const char *>(yq) + off_bytes;
+    ps.k = static_cast<const char *>(yk) + off_bytes;
+    ps.v = static_cast<const char *>(yv) + off_bytes;
+    ps.out = static_cast<char *>(yo) + off_bytes;
+    ps.lse = lse;
+    ps.lse_b = static_cast<long long>(H) * S;
+    ps.lse_h = S;
+    ps.lse_h0 = ho[u];
+    ps.H = heads[u];
+    ps.rows = static_cast<long long>(B) * S;
+    probs.push_back(ps);
+    prob_rank.push_back(static_cast<int>(u));
+  }
+}
+
+static int head_sharded_attention_impl(const void *yq, const void *yk, const void *yv, void *yo, float *lse, int B,
+                                       int H, int S, int D, const std::vector<int> &heads, cudaStream_t stream) {
+  std::vector<ProblemSpec> probs;
+  std::vector<int> prob_rank;
+  head_sharded_problems(probs, prob_rank, yq, yk, yv, yo, lse, B, H, S, D, heads);
+  std::vector<GroupSpec> groups;
+  for (size_t pi = 0; pi < probs.size(); ++pi) {
+    for (int b = 0; b < B; ++b) {
+      GroupSpec g;
+      g.prob = static_cast<int>(pi);
+      g.b = b;
+      SegSpec s;
+      s.row0 = b * S;
+      s.nrows = S;
+      s.s0 = 0;
+      s.kv.push_back(AttnKV{b * S, S});
+      g.segs.push_back(std::move(s));
+      groups.push_back(std::move(g));
+    }
+  }
+  return run_attention(probs, groups, D, false, stream);
+}
+
+int cpattn_head_sharded_attention(const void *yq, const void *yk, const void *yv, void *yo, float *lse, int B, int H,
+                                  int S, int D, int degree, const int *head_splits, cpattn_stream_t stream) {
+  if (yq == nullptr || yk == nullptr || yv == nullptr || yo == nullptr) return CPATTN_ERR_NULL;
+  int st = check_attn_shape(B, H, S, D);
+  if (st != CPATTN_OK) return st;
+  if (degree < 1 || degree > kMaxRanks) return CPATTN_ERR_DEGREE;
+  std::vector<int> heads;
+  st = resolve_splits(H, degree, head_splits, heads);
+  if (st != CPATTN_OK) return st;
+  if (!aligned16(yq) || !aligned16(yk) || !aligned16(yv) || !aligned16(yo) || (lse && !aligned4(lse)))
+    return CPATTN_ERR_ALIGNMENT;
+  st = check_device(nullptr);
+  if (st != CPATTN_OK) return st;
+  return head_sharded_attention_impl(yq, yk, yv, yo, lse, B, H, S, D, heads, stream);
+}
+
+size_t cpattn_ulysses_workspace_bytes(int B, int H, int S, int D) {
+  if (B < 1 || H < 1 || S < 1 || D < 1) return 0;
+  return static_cast<size_t>(4) * B * S * H * D * 2;
+}
+
+size_t cpattn_unified_workspace_bytes(int B, int H, int S, int D) { return cpattn_ulysses_workspace_bytes(B, H, S, D); }
+
+int cpattn_ulysses_attention(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H, int S,
+                             int D, int degree, const int *seq_splits, const int *head_splits, void *workspace,
+                             size_t workspace_bytes, cpattn_stream_t stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return CPATTN_ERR_NULL;
+  int st = check_attn_shape(B, H, S, D);
+  if (st != CPATTN_OK) return st;
+  if (degree < 1 || degree > kMaxRanks) return CPATTN_ERR_DEGREE;
+  std::vector<int> seq_chk, heads_chk;
+  st = resolve_splits(S, degree, seq_splits, seq_chk);
+  if (st != CPATTN_OK) return st;
+  st = resolve_splits(H, degree, head_splits, heads_chk);
+  if (st != CPATTN_OK) return st;
+  if (workspace == nullptr || workspace_bytes < cpattn_ulysses_workspace_bytes(B, H, S, D)) return CPATTN_ERR_WORKSPACE;
+  PermuteParams pq;
+  st = permute_common(q, workspace, B, S, H, D, 2, degree, seq_splits, head_splits, 0, pq);
+  if (st != CPATTN_OK) return st;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(out) || (lse && !aligned4(lse))) return CPATTN_ERR_ALIGNMENT;
+  st = check_device(nullptr);
+  if (st != CPATTN_OK) return st;
+  const size_t tensor_bytes = static_cast<size_t>(B) * S * H * D * 2;
+  char *ws = static_cast<char *>(workspace);
+  void *yq = ws, *yk = ws + tensor_bytes, *yv = ws + 2 * tensor_bytes, *yo = ws + 3 * tensor_bytes;
+  std::vector<int> heads;
+  resolve_splits(H, degree, head_splits, heads);
+  // first all-to-all: Q, K, V to the head-sharded layout
+  const void *srcs[3] = {q, k, v};
+  void *dsts[3] = {yq, yk, yv};
+  for (int i = 0; i < 3; ++i) {
+    PermuteParams pp = pq;
+    pp.src = static_cast<const unsigned char *>(srcs[i]);
+    pp.dst = static_cast<unsigned char *>(dsts[i]);
+    if (launch_permute(pp, stream) != cudaSuccess) return CPATTN_ERR_CUDA;
+  }
+  // local attention of every head rank over all S tokens of its heads
+  st = head_sharded_attention_impl(yq, yk, yv, yo, lse, B, H, S, D, heads, stream);
+  if (st != CPATTN_OK) return st;
+  // second all-to-all: the output back to the sequence-sharded layout
+  PermuteParams po = pq;
+  po.src = static_cast<const unsigned char *>(yo);
+  po.dst = static_cast<unsigned char *>(out);
+  po.direction = 1;
+  return launch_permute(po, stream) == cudaSuccess ? CPATTN_OK : CPATTN_ERR_CUDA;
+}
+
+int cpattn_unified_attention(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H, int S,
+                             int D, int ring_degree, int ulysses_degree, const int *ring_lens,
+                             const int *head_splits, void *workspace, size_t workspace_bytes,
+                             cpattn_stream_t stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return CPATTN_ERR_NULL;
+  int st = check_attn_shape(B, H, S, D);
+  if (st != CPATTN_OK) return st;
+  if (ring_degree < 1 || ring_degree > kMaxRanks || ulysses_degree < 1 || ulysses_degree > kMaxRanks)
+    return CPATTN_ERR_DEGREE;
+  std::vector<int> lens, heads;
+  st = resolve_splits(S, ring_degree, ring_lens, lens);
+  if (st != CPATTN_OK) return st;
+  st = resolve_splits(H, ulysses_degree, head_splits, heads);
+  if (st != CPATTN_OK) return st;
+  if (H > kMaxHeads) return CPATTN_ERR_SHAPE;
+  if (workspace == nullptr || workspace_bytes < cpattn_unified_workspace_bytes(B, H, S, D)) return CPATTN_ERR_WORKSPACE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(workspace) ||
+      (lse && !aligned4(lse)))
+    return CPATTN_ERR_ALIGNMENT;
+  st = check_device(nullptr);
+  if (st != CPATTN_OK) return st;
+  const std::vector<int> off = prefix(lens), ho = prefix(heads);
+  const size_t tensor_bytes = static_cast<size_t>(B) * S * H * D * 2;
+  char *ws = static_cast<char *>(workspace);
+  void *yq = ws, *yk = ws + tensor_bytes, *yv = ws + 2 * tensor_bytes, *yo = ws + 3 * tensor_bytes;
+
+  // Permutation within every ring group (ring chunk i): full BSHD rows of the
+  // chunk -> head group u buffer laid out [i][B, len_i, H_u, D].
+  PermuteParams pp;
+  std::memset(&pp, 0, sizeof(pp));
+  pp.B = B;
+  pp.S = S;
+  pp.H = H;
+  pp.row_bytes = D * 2;
+  pp.seq_mode = 0;
+  pp.n_seq = 1;
+  pp.n_groups = ring_degree;
+  for (int i = 0; i <= ring_degree; ++i) pp.group_off[i] = off[i];
+  pp.n_head = ulysses_degree;
+  for (int u = 0; u <= ulysses_degree; ++u) pp.head_off[u] = ho[u];
+  const void *srcs[3] = {q, k, v};
+  void *dsts[3] = {yq, yk, yv};
+  for (int i = 0; i < 3; ++i) {
+    PermuteParams p1 = pp;
+    p1.src = static_cast<const unsigned char *>(srcs[i]);
+    p1.dst = static_cast<unsigned char *>(dsts[i]);
+    p1.direction = 0;
+    if (launch_permute(p1, stream) != cudaSuccess) return CPATTN_ERR_CUDA;
+  }
+  // Ring attention per head group over the chunks (rows B*off_i + b*len_i).
+  std::vector<ProblemSpec> probs;
+  std::vector<int> prob_rank;
+  head_sharded_problems(probs, prob_rank, yq, yk, yv, yo, lse, B, H, S, D, heads);
+  std::vector<GroupSpec> groups;
+  for (size_t pi = 0; pi < probs.size(); ++pi)
+    ring_groups(groups, static_cast<int>(pi), B, lens, off, -1,
+                [&](int b, int c) { return B * off[c] + b * lens[c]; });
+  st = run_attention(probs, groups, D, false, stream);
+  if (st != CPATTN_OK) return st;
+  PermuteParams p2 = pp;
+  p2.src = static_cast<const unsigned char *>(yo);
+  p2.dst = static_cast<unsigned char *>(out);
+  p2.direction = 1;
+  return launch_permute(p2, stream) == cudaSuccess ? CPATTN_OK : CPATTN_ERR_CUDA;
+}
+
+int cpattn_device_status(cpattn_stream_t stream, unsigned int *code) {
+  if (code == nullptr) return CPATTN_ERR_NULL;
+  int st = check_device(nullptr);
+  if (st != CPATTN_OK) return st;
+  unsigned int v = 0;
+  if (read_and_clear_device_status(&v, stream) != cudaSuccess) return CPATTN_ERR_CUDA;
+  *code = v;
+  return v == 0 ? CPATTN_OK : CPATTN_ERR_DEVICE_TIMEOUT;
+}
+
+int cpattn_debug_wait_timeout(unsigned int timeout_us, cpattn_stream_t stream) {
+  if (timeout_us < 1 || timeout_us > 1000000) return CPATTN_ERR_SHAPE;
+  int st = check_device(nullptr);
+  if (st != CPATTN_OK) return st;
+  return launch_debug_wait(static_cast<unsigned long long>(timeout_us) * 1000ull, stream) == cudaSuccess
+             ? CPATTN_OK
+             : CPATTN_ERR_CUDA;
+}
+
+}  // extern "C"

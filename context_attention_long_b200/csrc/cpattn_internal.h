@@ -1,0 +1,127 @@
+// cpattn_internal.h -- launch plans shared by the host planner (cpattn_api.cu)
+// and the kernels.  Not part of the public ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace cpattn {
+
+// ---------------------------------------------------------------- attention
+//
+// The attention kernel sees every Q/K/V tensor as a 3-D array [rows, H, D]
+// (D contiguous).  A full BSHD tensor has rows = B*S with row = b*S + s; the
+// rank-buffer layouts used by the Ulysses/unified flows are also [rows, H, D]
+// with other row formulas.  Work is described with row ranges:
+//   problem : one (Q, K, V, out, lse) tensor set with its head count H,
+//   group   : (problem, batch index b) -- the set of Q segments sharing
+//             K/V row numbering; units are ordered head-major inside it,
+//   segment : a range of Q rows (one sequence shard) with its list of K/V
+//             row ranges, visited in order (ring order for ring attention),
+//   kv      : a K/V row range (one chunk).
+// One CTA processes one unit = (group, head, segment, pair of 128-row Q tiles).
+
+constexpr int kMaxProblems = 8;
+constexpr int kMaxGroups = 64;
+constexpr int kMaxSegs = 128;
+constexpr int kMaxKV = 512;
+constexpr int kQTile = 128;     // rows per Q tile (one TMEM lane per row)
+constexpr int kKVTile = 128;    // keys per K/V tile
+constexpr int kQTilesPerCTA = 2;
+
+struct alignas(64) AttnProblem {
+  CUtensorMap tm_q, tm_k, tm_v;   // 3-D maps over [rows, H, D] bf16, box {64, 1, 128}, 128B swizzle
+  void *out;                      // [rows, H, D] bf16 or float32 (same rows as Q)
+  float *lse;                     // may be null; index b*lse_b + (h + lse_h0)*lse_h + s
+  long long lse_b;
+  long long lse_h;
+  int lse_h0;
+  int H;
+};
+
+struct AttnGroup {
+  int prob;
+  int b;
+  int seg_first;
+  int seg_count;
+  int tiles_per_head;   // sum over the group's segments of their CTA tile pairs
+  int unit_base;        // first unit (blockIdx) of this group
+};
+
+struct AttnSeg {
+  int row0;       // first Q row
+  int nrows;      // Q rows in the segment
+  int s0;         // sequence position of row0 (for the LSE index)
+  int kv_first;   // index into kv[]
+  int kv_count;   // number of K/V ranges (0: empty -> out 0, lse -inf)
+  int tile_base;  // first tile pair of this segment within the group's head
+};
+
+struct AttnKV {
+  int row0;
+  int nrows;
+};
+
+struct AttnParams {
+  AttnProblem prob[kMaxProblems];
+  AttnGroup group[kMaxGroups];
+  AttnSeg seg[kMaxSegs];
+  AttnKV kv[kMaxKV];
+  int num_groups;
+  int total_units;
+  float scale_log2;              // D**-0.5 * log2(e)
+  unsigned long long timeout_ns; // bound for every pipeline wait
+};
+
+// Launches the attention kernel for a plan.  D in {64, 128}; out_f32 selects
+// float32 partial outputs (ring step) instead of bf16.
+cudaError_t launch_attention(const AttnParams &p, int D, bool out_f32, cudaStream_t stream);
+
+// ---------------------------------------------------------------- LSE merge
+struct MergeParams {
+  const float *part_out;  // P x [B, S, H, D]
+  const float *part_lse;  // P x [B, H, S]
+  float *out_f32;         // may be null
+  __nv_bfloat16 *out_bf16; // may be null
+  float *lse_out;         // may be null
+  int P, B, H, S, D;
+};
+cudaError_t launch_lse_merge(const MergeParams &p, cudaStream_t stream);
+
+// ----------------------------------------------------------------- permute
+//
+// Moves token rows between a sequence-side layout and a head-side layout.
+// Every token (b, s) owns one source row of H*D elements on the sequence side;
+// on the head side it owns, for every head rank u, a row of H_u*D elements.
+//   sequence side row:  seq_mode 0 (full BSHD):     b*S + s
+//                       seq_mode 1 (rank buffers):   B*off_r + b*len_r + (s - off_r)
+//   head side row in buffer u (groups = outer sequence ranges, one group for
+//   plain Ulysses):     B*goff_i + b*glen_i + (s - goff_i)
+//   head buffer u starts at element B*S*hoff_u*D.
+constexpr int kMaxRanks = 64;
+constexpr int kMaxHeads = 1024;
+
+struct PermuteParams {
+  const unsigned char *src;
+  unsigned char *dst;
+  int B, S, H;
+  int row_bytes;        // D * elem_bytes (multiple of 16)
+  int direction;        // 0: sequence side -> head side, 1: head side -> sequence side
+  int seq_mode;         // 0 full BSHD, 1 rank buffers
+  int n_seq;            // sequence ranks (seq_mode 1)
+  int seq_off[kMaxRanks + 1];
+  int n_groups;         // head-side groups
+  int group_off[kMaxRanks + 1];
+  int n_head;           // head ranks
+  int head_off[kMaxRanks + 1];
+};
+cudaError_t launch_permute(const PermuteParams &p, cudaStream_t stream);
+
+// ------------------------------------------------------------------- misc
+cudaError_t launch_debug_wait(unsigned long long timeout_ns, cudaStream_t stream);
+cudaError_t read_and_clear_device_status(unsigned int *code, cudaStream_t stream);
+
+}  // namespace cpattn

@@ -1,0 +1,273 @@
+/*
+ * cpattn.h -- C ABI of libcpattn.so, the B200 (sm_100a) hot path of
+ * context-parallel attention emulated on one GPU.
+ *
+ * Sources (web pages, cited by title and section):
+ *   [CP]  diffusers v0.43.0 docs, "Context parallelism": variants table;
+ *         "Ring Attention"; "Ulysses Attention"; "Unified Attention";
+ *         "Ulysses Anything Attention"; "Ring Anything Attention".
+ *   [SP]  SGLang Diffusion docs, "Sequence Parallelism": "Choosing The
+ *         Attention Exchange"; "Numerics across node boundaries".
+ *   [USP] "Ulysses Sequence Parallelism: training with million-token
+ *         contexts": sections 3 (core idea), 4 (steps), 5 (communication).
+ *   [API] diffusers docs, "parallel": ContextParallelConfig parameters
+ *         ring_degree, ulysses_degree, convert_to_fp32, rotate_method,
+ *         ulysses_anything, ring_anything.
+ *   [PR]  sglang PR #30086 analysis: (B, S, H, D) q/k/v view, scale
+ *         head_dim**-0.5.
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ * Tensors.  Q, K, V and attention outputs are bf16, (batch B, seq S, heads H,
+ *   head_dim D) contiguous ("BSHD", [PR]).  D must be 64 or 128.  Softmax
+ *   scale is D**-0.5 ([PR]).  Attention is non-causal with no mask ([SP]
+ *   kv_gather constraint; [CP] Ring Anything requires attn_mask None).
+ *   LSE outputs are float32, natural log, layout (B, H, S).
+ * Shards.  A "sequence shard" r of a full BSHD tensor is rows off_r ..
+ *   off_r + len_r - 1 of every batch element, with off_r the prefix sum of the
+ *   lengths.  NULL length arrays mean the standard equal split, which requires
+ *   divisibility by the degree ([CP] variants table); explicit lengths are the
+ *   'anything' modes ([CP] Ring Anything / Ulysses Anything), may be uneven and
+ *   may contain zeros.
+ * Memory.  All tensor pointers are DEVICE pointers owned by the caller; the
+ *   library allocates nothing.  Length/split arrays are HOST arrays read only
+ *   during the call.  Q, K, V and outputs must be 16-byte aligned.  Outputs
+ *   must not alias inputs unless stated.
+ * Streams.  `stream` is a cudaStream_t (NULL = legacy default stream).  Every
+ *   call only enqueues work; none synchronises the host.  Arguments are fully
+ *   validated before anything is enqueued; on a non-zero return nothing was
+ *   enqueued except for CPATTN_ERR_CUDA, which reports a launch failure.
+ * Errors.  Return value is a cpattn_status.  No C++ exception crosses the ABI.
+ *   Device-side bounded waits (see cpattn_device_status) report a pipeline that
+ *   stopped making progress instead of hanging the GPU.
+ */
+#ifndef CPATTN_H
+#define CPATTN_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *cpattn_stream_t; /* == cudaStream_t */
+
+typedef enum {
+  CPATTN_OK = 0,
+  CPATTN_ERR_NULL = 1,           /* a required pointer is NULL                        */
+  CPATTN_ERR_SHAPE = 2,          /* B, H, S < 1, D not 64/128, elem size unsupported  */
+  CPATTN_ERR_INDIVISIBLE = 3,    /* lengths NULL and S or H not divisible by degree   */
+  CPATTN_ERR_SPLITS = 4,         /* negative lengths or lengths not summing to S / H  */
+  CPATTN_ERR_DEGREE = 5,         /* degree < 1, degree > S (or > H), step out of range */
+  CPATTN_ERR_CUDA = 6,           /* CUDA runtime/driver error (no device, launch)     */
+  CPATTN_ERR_DEVICE_TIMEOUT = 7, /* a device-side bounded wait expired                */
+  CPATTN_ERR_WORKSPACE = 8,      /* workspace NULL or smaller than required           */
+  CPATTN_ERR_ALIGNMENT = 9,      /* a tensor pointer is not 16-byte aligned           */
+  CPATTN_ERR_UNSUPPORTED = 10    /* current device is not sm_100 (B200)               */
+} cpattn_status;
+
+/* Human-readable name of a status code; never NULL. */
+const char *cpattn_status_string(int status);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+int cpattn_version(void);
+
+/* ------------------------------------------------------------------ ring */
+
+/*
+ * Ring attention, fused ([CP] "Ring Attention", "Ring Anything Attention";
+ * [API] ring_degree, convert_to_fp32, rotate_method).
+ *
+ * The sequence is cut into `ring_degree` shards; rank r holds shard r of Q, K
+ * and V.  For every rank the kernel walks the K/V chunks in ring order
+ * c = r, r-1, ..., r-P+1 (mod P) -- the block a GPU holds after t hand-offs --
+ * computing the attention of Q shard r against one chunk at a time and merging
+ * it into a running float32 (out, LSE) state with the online-softmax / LSE
+ * rule, so that after the full ring every query has seen every key.  The merge
+ * is held on chip (TMEM/registers) instead of in HBM; cpattn_ring_step +
+ * cpattn_lse_merge is the same computation with the partials in memory.
+ *
+ *   q, k, v    [B, S, H, D] bf16 device, read only.
+ *   out        [B, S, H, D] bf16 device, written (all rows).
+ *   lse        [B, H, S] float32 device, natural log; may be NULL.
+ *   chunk_lens host int[ring_degree] (Ring Anything) or NULL (equal split,
+ *              S % ring_degree must be 0 else CPATTN_ERR_INDIVISIBLE).
+ * Errors: NULL, SHAPE, DEGREE (ring_degree < 1 or > S), INDIVISIBLE, SPLITS,
+ * ALIGNMENT, UNSUPPORTED, CUDA.
+ */
+int cpattn_ring_attention(const void *q, const void *k, const void *v, void *out, float *lse,
+                          int B, int H, int S, int D, int ring_degree, const int *chunk_lens,
+                          cpattn_stream_t stream);
+
+/*
+ * One ring step for every rank ([CP] "Ring Attention"; [API] convert_to_fp32):
+ * rank r attends its Q shard to chunk c = (r - step) mod P and writes the
+ * partial result normalised over that chunk, in float32, plus its LSE.
+ * A rank whose chunk is empty writes out = 0 and LSE = -inf for its rows.
+ *
+ *   part_out   [B, S, H, D] float32 device (rows of shard r hold rank r's partial).
+ *   part_lse   [B, H, S] float32 device.
+ *   step       0 <= step < ring_degree (else CPATTN_ERR_DEGREE).
+ * Other arguments as cpattn_ring_attention.
+ */
+int cpattn_ring_step(const void *q, const void *k, const void *v, float *part_out,
+                     float *part_lse, int B, int H, int S, int D, int ring_degree,
+                     const int *chunk_lens, int step, cpattn_stream_t stream);
+
+/*
+ * LSE merge of P float32 partials ([SP] "Numerics across node boundaries":
+ * online-softmax merge of the ring's partial results; [API] convert_to_fp32):
+ *   M = max_p LSE_p,  LSE = M + ln sum_p exp(LSE_p - M),
+ *   out = sum_p exp(LSE_p - LSE) * out_p.
+ * Partials with LSE = -inf carry no keys and get weight 0; rows where every
+ * partial is empty produce out = 0, LSE = -inf.
+ *
+ *   part_out   P consecutive [B, S, H, D] float32 tensors (device).
+ *   part_lse   P consecutive [B, H, S] float32 tensors (device).
+ *   out_f32    [B, S, H, D] float32 or NULL.  May alias part_out (partial 0):
+ *              each element is read before it is written, by the same thread.
+ *   out_bf16   [B, S, H, D] bf16 or NULL.  At least one of out_f32/out_bf16.
+ *   lse_out    [B, H, S] float32 or NULL.  May alias part_lse (partial 0).
+ * Errors: NULL, SHAPE (P < 1), ALIGNMENT, CUDA.
+ */
+int cpattn_lse_merge(const float *part_out, const float *part_lse, int P, int B, int H, int S,
+                     int D, float *out_f32, void *out_bf16, float *lse_out,
+                     cpattn_stream_t stream);
+
+/* ------------------------------------------------------------- kv_gather */
+
+/*
+ * kv_gather exchange ([SP] "Choosing The Attention Exchange"): Q and the
+ * output stay sequence-sharded, K and V are gathered in full (on one GPU they
+ * already are), and every rank computes the attention of its own Q rows
+ * against all S keys; non-causal, ring degree 1.
+ *
+ *   q_lens     host int[degree] or NULL (equal split).
+ * Other arguments as cpattn_ring_attention.
+ */
+int cpattn_kv_gather_attention(const void *q, const void *k, const void *v, void *out,
+                               float *lse, int B, int H, int S, int D, int degree,
+                               const int *q_lens, cpattn_stream_t stream);
+
+/* --------------------------------------------------------------- Ulysses */
+
+/*
+ * Ulysses permute, sequence-sharded -> head-sharded: the first all-to-all
+ * ([CP] "Ulysses Attention": every GPU ends up with every token for a subset
+ * of the heads; [USP] section 4), with uneven splits ([CP] "Ulysses Anything
+ * Attention"):
+ *     y_{r'}[b, s, h - hoff_{r'}, :] = x_{r(s)}[b, s - off_{r(s)}, h, :]
+ *
+ *   x  sequence side: the `degree` rank buffers concatenated in rank order,
+ *      rank r = [B, seq_r, H, D] (for B = 1 this is the full [1, S, H, D]).
+ *   y  head side: the rank buffers concatenated in rank order,
+ *      rank r' = [B, S, head_r', D].
+ *   elem_bytes  element size (2 for bf16 Q/K/V, 4 for float32); D*elem_bytes
+ *      must be a multiple of 16.  Data is moved bit-exactly.
+ *   seq_splits / head_splits  host int[degree] or NULL (equal split; S and H
+ *      must then be divisible by degree, else CPATTN_ERR_INDIVISIBLE).
+ * x and y must not overlap.  Errors: NULL, SHAPE, DEGREE (degree < 1),
+ * INDIVISIBLE, SPLITS, ALIGNMENT, CUDA.
+ */
+int cpattn_ulysses_permute(const void *x, void *y, int B, int S, int H, int D, int elem_bytes,
+                           int degree, const int *seq_splits, const int *head_splits,
+                           cpattn_stream_t stream);
+
+/*
+ * Ulysses unpermute, head-sharded -> sequence-sharded: the second all-to-all,
+ * which regroups the attention output by token ([CP] "Ulysses Attention");
+ * the exact inverse of cpattn_ulysses_permute (same arguments, y is read and
+ * x is written).
+ */
+int cpattn_ulysses_unpermute(const void *y, void *x, int B, int S, int H, int D, int elem_bytes,
+                             int degree, const int *seq_splits, const int *head_splits,
+                             cpattn_stream_t stream);
+
+/*
+ * Head-sharded local attention ([USP] section 4: after the first all-to-all
+ * every GPU runs ordinary attention over all tokens of its heads): for every
+ * head rank r', attention of its [B, S, head_r', D] Q/K/V buffers.
+ *
+ *   yq, yk, yv, yo  head-sharded layouts as in cpattn_ulysses_permute (bf16).
+ *   lse        [B, H, S] float32 indexed by global head, or NULL.
+ */
+int cpattn_head_sharded_attention(const void *yq, const void *yk, const void *yv, void *yo,
+                                  float *lse, int B, int H, int S, int D, int degree,
+                                  const int *head_splits, cpattn_stream_t stream);
+
+/* Bytes of workspace cpattn_ulysses_attention needs: 4 * B*S*H*D * 2. */
+size_t cpattn_ulysses_workspace_bytes(int B, int H, int S, int D);
+
+/*
+ * Ulysses attention ([CP] "Ulysses Attention"; [USP] section 4): permute Q, K,
+ * V to the head-sharded layout, local attention per head rank, unpermute the
+ * output.  q, k, v, out are sequence-side rank buffers as `x` in
+ * cpattn_ulysses_permute; lse is [B, H, S] (global head and token) or NULL.
+ * workspace: device, >= cpattn_ulysses_workspace_bytes, 16-byte aligned,
+ * caller-owned scratch (contents undefined after the call).
+ */
+int cpattn_ulysses_attention(const void *q, const void *k, const void *v, void *out, float *lse,
+                             int B, int H, int S, int D, int degree, const int *seq_splits,
+                             const int *head_splits, void *workspace, size_t workspace_bytes,
+                             cpattn_stream_t stream);
+
+/* --------------------------------------------------------------- unified */
+
+/* Bytes of workspace cpattn_unified_attention needs: 4 * B*S*H*D * 2. */
+size_t cpattn_unified_workspace_bytes(int B, int H, int S, int D);
+
+/*
+ * Unified ring x Ulysses attention ([CP] "Unified Attention": an all-to-all
+ * redistributes heads and tokens, ring attention runs on the result, and the
+ * inverse all-to-all restores the layout; the GPUs form a
+ * ring_degree x ulysses_degree grid).
+ *
+ * Ring chunks are the outer split of the sequence (ring_lens, or equal);
+ * inside ring chunk i the ulysses_degree ranks of that Ulysses group hold
+ * sub-shards of it; heads are split by head_splits (or equally).  Steps: per
+ * ring group, Ulysses permute of its chunk to head groups; per head group,
+ * ring attention over the chunks with the LSE merge; per ring group, the
+ * inverse permute of the output.
+ *
+ *   q, k, v, out  full [B, S, H, D] bf16.  lse [B, H, S] or NULL.
+ *   ring_lens     host int[ring_degree] or NULL (equal split).
+ *   head_splits   host int[ulysses_degree] or NULL (equal split).
+ *   workspace     >= cpattn_unified_workspace_bytes.
+ */
+int cpattn_unified_attention(const void *q, const void *k, const void *v, void *out, float *lse,
+                             int B, int H, int S, int D, int ring_degree, int ulysses_degree,
+                             const int *ring_lens, const int *head_splits, void *workspace,
+                             size_t workspace_bytes, cpattn_stream_t stream);
+
+/* ------------------------------------------------------------- utilities */
+
+/*
+ * The uneven split used by the 'anything' workloads ([CP] "Ulysses Anything
+ * Attention" removes the divisibility requirement; the page does not fix the
+ * rule, this library uses front-loaded ceil): the first total % parts entries
+ * get ceil(total / parts), the rest floor(total / parts).  out: host
+ * int[parts].  Errors: NULL, DEGREE (parts < 1), SHAPE (total < 0).
+ */
+int cpattn_front_loaded_splits(int total, int parts, int *out);
+
+/*
+ * Synchronises `stream`, then reads and clears the device status word that the
+ * kernels' bounded waits set when a pipeline wait expires.  *code receives the
+ * raw word (0 = healthy; otherwise a bit per wait site).  Returns CPATTN_OK,
+ * CPATTN_ERR_DEVICE_TIMEOUT if the word was non-zero, or CPATTN_ERR_CUDA.
+ */
+int cpattn_device_status(cpattn_stream_t stream, unsigned int *code);
+
+/*
+ * Test hook for the bounded-wait mechanism: launches one block that waits on
+ * an mbarrier nothing ever arrives at, with a limit of `timeout_us`
+ * microseconds (1 .. 1000000), then sets the timeout bit and returns.  The
+ * caller then sees CPATTN_ERR_DEVICE_TIMEOUT from cpattn_device_status.
+ */
+int cpattn_debug_wait_timeout(unsigned int timeout_us, cpattn_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CPATTN_H */

@@ -1,0 +1,152 @@
+"""The C ABI without a GPU: the library loads, exports every symbol the header
+declares, and rejects invalid arguments with the documented status codes
+before touching CUDA.  Pointers passed here are fake (never dereferenced):
+every call below must fail validation."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from context_attention_long_b200 import _native, build, inputs
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "cpattn.h")
+
+OK, NULL, SHAPE, INDIV, SPLITS, DEGREE, CUDA, TIMEOUT, WS, ALIGN, UNSUP = range(11)
+FAKE = ctypes.c_void_p(1 << 20)      # non-null, 16-byte aligned, never dereferenced
+FAKE_MIS = ctypes.c_void_p((1 << 20) + 8)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _native.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(cpattn_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_north_star_calls():
+    names = declared_functions()
+    for required in ("cpattn_ring_attention", "cpattn_lse_merge", "cpattn_ulysses_permute",
+                     "cpattn_ulysses_unpermute", "cpattn_kv_gather_attention"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 15
+    for name in names:
+        assert hasattr(lib, name), name
+        assert name in _native.SIGNATURES, f"{name} has no ctypes signature"
+
+
+def test_status_strings(lib):
+    for code in range(11):
+        s = lib.cpattn_status_string(code).decode()
+        assert s.startswith("CPATTN")
+    assert b"unknown" in lib.cpattn_status_string(99)
+    assert lib.cpattn_version() >= 10000
+
+
+def test_front_loaded_splits_agree_with_input_recipe(lib):
+    for total, parts in [(30, 4), (10007, 4), (4095, 2), (7, 7), (5, 8), (0, 3), (4608, 4)]:
+        arr = (ctypes.c_int * parts)()
+        assert lib.cpattn_front_loaded_splits(total, parts, arr) == OK
+        assert list(arr) == inputs.front_loaded_splits(total, parts)
+    assert lib.cpattn_front_loaded_splits(5, 0, (ctypes.c_int * 1)()) == DEGREE
+    assert lib.cpattn_front_loaded_splits(5, 2, None) == NULL
+
+
+def _ring(lib, q=FAKE, out=FAKE, B=1, H=2, S=256, D=64, P=4, lens=None, lse=FAKE):
+    return lib.cpattn_ring_attention(q, FAKE, FAKE, out, lse, B, H, S, D, P, _native.int_array(lens), None)
+
+
+def test_ring_validation(lib):
+    assert _ring(lib, q=None) == NULL
+    assert _ring(lib, out=None) == NULL
+    assert _ring(lib, D=96) == SHAPE
+    assert _ring(lib, B=0) == SHAPE
+    assert _ring(lib, S=0) == SHAPE
+    assert _ring(lib, P=0) == DEGREE
+    assert _ring(lib, S=10, P=3) == INDIV                    # standard ring: S % ring_degree != 0
+    assert _ring(lib, S=3, P=4) == DEGREE                    # more ranks than tokens, equal split
+    assert _ring(lib, S=10, P=3, lens=[3, 3, 3]) == SPLITS   # Ring Anything lengths must sum to S
+    assert _ring(lib, S=10, P=3, lens=[11, -1, 0]) == SPLITS
+    assert _ring(lib, q=FAKE_MIS) == ALIGN
+
+
+def test_ring_step_validation(lib):
+    f = lambda step, lse=FAKE: lib.cpattn_ring_step(FAKE, FAKE, FAKE, FAKE, lse, 1, 2, 256, 64, 4, None, step, None)
+    assert f(-1) == DEGREE
+    assert f(4) == DEGREE
+    assert f(0, lse=None) == NULL
+
+
+def test_merge_validation(lib):
+    f = lambda **kw: lib.cpattn_lse_merge(kw.get("po", FAKE), kw.get("pl", FAKE), kw.get("P", 4), 1, 2, 8,
+                                          kw.get("D", 64), kw.get("of", FAKE), kw.get("ob", None), FAKE, None)
+    assert f(po=None) == NULL
+    assert f(of=None, ob=None) == NULL
+    assert f(P=0) == SHAPE
+    assert f(D=32) == SHAPE
+    assert f(po=FAKE_MIS) == ALIGN
+
+
+def test_kv_gather_validation(lib):
+    f = lambda S=16, P=4, lens=None: lib.cpattn_kv_gather_attention(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, S, 64, P,
+                                                                    _native.int_array(lens), None)
+    assert f(S=18) == INDIV
+    assert f(lens=[4, 4, 4, 5]) == SPLITS
+    assert f(P=0) == DEGREE
+
+
+def test_permute_validation(lib):
+    def f(x=FAKE, y=FAKE, B=1, S=8, H=4, D=64, eb=2, P=2, seq=None, heads=None):
+        return lib.cpattn_ulysses_permute(x, y, B, S, H, D, eb, P, _native.int_array(seq), _native.int_array(heads), None)
+    assert f(x=None) == NULL
+    assert f(eb=3) == SHAPE
+    assert f(D=3, eb=2) == SHAPE        # rows must be a multiple of 16 bytes
+    assert f(P=0) == DEGREE
+    assert f(H=5) == INDIV              # standard Ulysses: heads % degree != 0
+    assert f(S=9) == INDIV              # standard Ulysses: seq % degree != 0
+    assert f(H=5, heads=[3, 3]) == SPLITS
+    assert f(S=9, seq=[5, 5]) == SPLITS
+    assert f(y=FAKE_MIS) == ALIGN
+    g = lambda H=5: lib.cpattn_ulysses_unpermute(FAKE, FAKE, 1, 8, H, 64, 2, 2, None, None, None)
+    assert g() == INDIV
+
+
+def test_flow_validation(lib):
+    need = lib.cpattn_ulysses_workspace_bytes(1, 4, 8, 64)
+    assert need == 4 * 1 * 8 * 4 * 64 * 2
+    assert lib.cpattn_unified_workspace_bytes(1, 4, 8, 64) == need
+    u = lambda ws=FAKE, nbytes=need, H=4: lib.cpattn_ulysses_attention(FAKE, FAKE, FAKE, FAKE, FAKE, 1, H, 8, 64, 2,
+                                                                       None, None, ws, nbytes, None)
+    assert u(ws=None) == WS
+    assert u(nbytes=need - 1) == WS
+    assert u(H=5) == INDIV
+    v = lambda ws=FAKE, R=2, U=2: lib.cpattn_unified_attention(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 4, 8, 64, R, U, None,
+                                                               None, ws, need, None)
+    assert v(ws=None) == WS
+    assert v(R=3) == INDIV
+    assert v(U=3) == INDIV
+    assert v(R=0) == DEGREE
+    h = lambda H=4: lib.cpattn_head_sharded_attention(FAKE, FAKE, FAKE, FAKE, FAKE, 1, H, 8, 64, 2, None, None)
+    assert h(H=5) == INDIV
+
+
+def test_debug_hook_validation(lib):
+    assert lib.cpattn_debug_wait_timeout(0, None) == SHAPE
+    assert lib.cpattn_device_status(None, None) == NULL
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_valid_call_without_gpu_reports_cuda_error(lib):
+    # Arguments pass validation; with no device the call must return
+    # CPATTN_ERR_CUDA before launching anything.
+    assert _ring(lib) == CUDA
