@@ -225,11 +225,16 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-breakdown", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel", default=None, choices=["ring", "head_sharded", "permute", "merge", "ring_step"],
+                    help="profiling mode: run only this kernel (warmup + steps launches) on the workload")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+        return
+    if args.kernel is not None:
+        run_single_kernel(args)
         return
 
     import torch
@@ -431,6 +436,41 @@ def breakdown(api, torch, dev, flush, peaks, inputs):
     del po, pl, ob, lo
     torch.cuda.empty_cache()
     return res
+
+
+def run_single_kernel(args):
+    """Profiling mode: `warmup + steps` launches of one kernel of the step on
+    the image-DiT workload (merge: 4 float32 partials of it), nothing else."""
+    import torch
+    from context_attention_long_b200 import api, build, inputs
+    build.build()
+    cfg, qb, kb, vb = inputs.config_inputs(WORKLOAD)
+    B, S, H, D = qb.shape
+    P, U = cfg["ring_degree"], cfg["ulysses_degree"]
+    dev = torch.device("cuda", 0)
+    q, k, v = (torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev) for x in (qb, kb, vb))
+    if args.kernel == "ring":
+        fn = lambda: api.cpattn_ring_attention(q, k, v, P)
+    elif args.kernel == "ring_step":
+        fn = lambda: api.cpattn_ring_step(q, k, v, P, 1)
+    elif args.kernel == "head_sharded":
+        yq, yk, yv = (api.cpattn_ulysses_permute(t.reshape(-1), B, S, H, D, U) for t in (q, k, v))
+        fn = lambda: api.cpattn_head_sharded_attention(yq, yk, yv, B, S, H, D, U)
+    elif args.kernel == "permute":
+        fn = lambda: api.cpattn_ulysses_permute(q.reshape(-1), B, S, H, D, U)
+    else:
+        po = torch.randn((P, B, S, H, D), device=dev)
+        pl = torch.randn((P, B, H, S), device=dev)
+        fn = lambda: api.cpattn_lse_merge(po, pl)
+    t0 = time.perf_counter()
+    for _ in range(args.warmup + args.steps):
+        fn()
+    torch.cuda.synchronize()
+    st, code = api.cpattn_device_status()
+    print(json.dumps({"kernel": args.kernel, "launches": args.warmup + args.steps, "status": st, "code": code,
+                      "wall_s": time.perf_counter() - t0}))
+    if st != 0:
+        sys.exit(1)
 
 
 if __name__ == "__main__":

@@ -56,7 +56,51 @@ struct AttnSmem {
 
 constexpr int kAttnThreads = 384;
 constexpr uint32_t kTmemCols = 512;
+// Register split: launched at 168 per thread (384 x 168 = 64512); the
+// producer/MMA warpgroup drops to 104 and the two softmax warpgroups rise to
+// 200: 128 x 104 + 256 x 200 = 64512, exactly the launch allocation.  (The
+// softmax row -- 128 fp32 scores -- lives in registers.)
+constexpr int kRegsLaunch = 168;
+constexpr int kRegsControl = 104;
+constexpr int kRegsSoftmax = 200;
+static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= kAttnThreads * kRegsLaunch, "register split exceeds launch");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale only if the max grows by > 2^8
+// Of every 8 score pairs, this many take 2^x on the FMA pipe (exp2_poly_x2)
+// and the rest on the SFU.  Measured on B200 with this pipeline the SFU is not
+// the limiter (the FMA-pipe share only lengthened the softmax), so it is 0.
+constexpr int kPolyEighths = 0;
+
+// The work unit of this CTA: group -> head -> segment -> pair of Q tiles.
+// Recomputed inside every role (after its register budget is set) so that no
+// decoded value stays live across the role split.
+struct Unit {
+  int gi, si, h, pair, q_row0, rows_left, n_tiles;
+  bool has_q1;
+};
+
+__device__ __forceinline__ Unit decode_unit(const AttnParams &p) {
+  Unit u;
+  const int unit = blockIdx.x;
+  int gi = 0;
+  while (gi + 1 < p.num_groups && p.group[gi + 1].unit_base <= unit) ++gi;
+  const AttnGroup &G = p.group[gi];
+  const int local = unit - G.unit_base;
+  u.h = local / G.tiles_per_head;
+  const int t = local - u.h * G.tiles_per_head;
+  int si = G.seg_first;
+  while (si + 1 < G.seg_first + G.seg_count && p.seg[si + 1].tile_base <= t) ++si;
+  const AttnSeg &SG = p.seg[si];
+  u.gi = gi;
+  u.si = si;
+  u.pair = t - SG.tile_base;
+  u.q_row0 = SG.row0 + u.pair * (kQTilesPerCTA * kQTile);
+  u.rows_left = SG.nrows - u.pair * (kQTilesPerCTA * kQTile);
+  u.has_q1 = u.rows_left > kQTile;
+  int n = 0;
+  for (int i = 0; i < SG.kv_count; ++i) n += (p.kv[SG.kv_first + i].nrows + kKVTile - 1) / kKVTile;
+  u.n_tiles = n;
+  return u;
+}
 
 template <int D, bool OUT_F32>
 __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnParams p) {
@@ -66,85 +110,73 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
   constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, true);
 
   extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
-  uint64_t *bar_q = bars;
-  uint64_t *bar_kf = bars + 1;
-  uint64_t *bar_ke = bar_kf + NST;
-  uint64_t *bar_vf = bar_ke + NST;
-  uint64_t *bar_ve = bar_vf + NST;
-  uint64_t *bar_s = bar_ve + NST;
-  uint64_t *bar_p = bar_s + 2;
-  uint64_t *bar_o = bar_p + 2;
-  uint64_t *bar_tail = bar_o + 2;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
+  // 32-bit shared-window addresses of everything (1024-aligned base).
+  const uint32_t sb = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  constexpr uint32_t BAR_Q = L::kOffBar;
+  constexpr uint32_t BAR_KF = BAR_Q + 8;               // [NST]
+  constexpr uint32_t BAR_KE = BAR_KF + 8 * NST;        // [NST]
+  constexpr uint32_t BAR_VF = BAR_KE + 8 * NST;        // [NST]
+  constexpr uint32_t BAR_VE = BAR_VF + 8 * NST;        // [NST]
+  constexpr uint32_t BAR_S = BAR_VE + 8 * NST;         // [2]
+  constexpr uint32_t BAR_P = BAR_S + 16;               // [2]
+  constexpr uint32_t BAR_O = BAR_P + 16;               // [2]
+  constexpr uint32_t BAR_TAIL = BAR_O + 16;
+  constexpr uint32_t TMEM_SLOT = L::kOffMisc;
+  constexpr uint32_t ABORT = L::kOffMisc + 4;
+  static_assert(BAR_TAIL + 8 <= L::kOffMisc, "barrier area");
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint64_t tmo = p.timeout_ns;
 
-  // ---- which unit: group -> head -> segment -> pair of Q tiles
-  const int unit = blockIdx.x;
-  int gi = 0;
-  while (gi + 1 < p.num_groups && p.group[gi + 1].unit_base <= unit) ++gi;
-  const AttnGroup &G = p.group[gi];
-  const int local = unit - G.unit_base;
-  const int h = local / G.tiles_per_head;
-  const int t = local - h * G.tiles_per_head;
-  int si = G.seg_first;
-  while (si + 1 < G.seg_first + G.seg_count && p.seg[si + 1].tile_base <= t) ++si;
-  const AttnSeg &SG = p.seg[si];
-  const AttnProblem &PB = p.prob[G.prob];
-  const int pair = t - SG.tile_base;
-  const int q_row0 = SG.row0 + pair * (kQTilesPerCTA * kQTile);
-  const int rows_left = SG.nrows - pair * (kQTilesPerCTA * kQTile);
-  const bool has_q1 = rows_left > kQTile;
-  int n_tiles = 0;
-  for (int i = 0; i < SG.kv_count; ++i) n_tiles += (p.kv[SG.kv_first + i].nrows + kKVTile - 1) / kKVTile;
-
   // ---- setup
   if (threadIdx.x == 0) {
-    mbar_init(bar_q, 1);
+    mbar_init(sb + BAR_Q, 1);
     for (int s = 0; s < NST; ++s) {
-      mbar_init(&bar_kf[s], 1);
-      mbar_init(&bar_ke[s], 1);
-      mbar_init(&bar_vf[s], 1);
-      mbar_init(&bar_ve[s], 1);
+      mbar_init(sb + BAR_KF + 8 * s, 1);
+      mbar_init(sb + BAR_KE + 8 * s, 1);
+      mbar_init(sb + BAR_VF + 8 * s, 1);
+      mbar_init(sb + BAR_VE + 8 * s, 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bar_s[i], 1);
-      mbar_init(&bar_p[i], 4);  // one arrival per softmax warp
-      mbar_init(&bar_o[i], 1);
+      mbar_init(sb + BAR_S + 8 * i, 1);
+      mbar_init(sb + BAR_P + 8 * i, 4);  // one arrival per softmax warp
+      mbar_init(sb + BAR_O + 8 * i, 1);
     }
-    mbar_init(bar_tail, 1);
-    *abort_flag = 0;
+    mbar_init(sb + BAR_TAIL, 1);
+    st_shared_volatile(sb + ABORT, 0u);
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&PB.tm_q);
-    tma_prefetch_desc(&PB.tm_k);
-    tma_prefetch_desc(&PB.tm_v);
-  }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_alloc(sb + TMEM_SLOT, kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem = ld_shared_volatile(sb + TMEM_SLOT);
+  const uint32_t abort_flag = sb + ABORT;
 
-  if (warp == 0) {
+  if (warp < 4) {
+   setmaxnreg_dec<kRegsControl>();
+   const Unit U = decode_unit(p);
+   const AttnSeg &SG = p.seg[U.si];
+   const AttnProblem &PB = p.prob[p.group[U.gi].prob];
+   const int h = U.h, q_row0 = U.q_row0, n_tiles = U.n_tiles;
+   const bool has_q1 = U.has_q1;
+   if (warp == 0) {
     // =========================================================== producer
     if (lane == 0 && n_tiles > 0) {
-      uint8_t *sQ = smem + L::kOffQ;
-      mbar_arrive_expect_tx(bar_q, (has_q1 ? 2 : 1) * L::kTileBytes);
+      tma_prefetch_desc(&PB.tm_q);
+      tma_prefetch_desc(&PB.tm_k);
+      tma_prefetch_desc(&PB.tm_v);
+      const uint32_t sQ = sb + L::kOffQ;
+      mbar_arrive_expect_tx(sb + BAR_Q, (has_q1 ? 2 : 1) * L::kTileBytes);
       for (int hf = 0; hf < L::kHalves; ++hf)
-        tma_load_3d(sQ + hf * L::kBoxBytes, &PB.tm_q, hf * 64, h, q_row0, bar_q);
+        tma_load_3d(sQ + hf * L::kBoxBytes, &PB.tm_q, hf * 64, h, q_row0, sb + BAR_Q);
       if (has_q1)
         for (int hf = 0; hf < L::kHalves; ++hf)
-          tma_load_3d(sQ + L::kTileBytes + hf * L::kBoxBytes, &PB.tm_q, hf * 64, h, q_row0 + kQTile, bar_q);
+          tma_load_3d(sQ + L::kTileBytes + hf * L::kBoxBytes, &PB.tm_q, hf * 64, h, q_row0 + kQTile, sb + BAR_Q);
       int it = 0;
       bool ok = true;
       for (int i = 0; ok && i < SG.kv_count; ++i) {
@@ -152,16 +184,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
         for (int r = 0; r < kv.nrows; r += kKVTile, ++it) {
           const int st = it % NST;
           const uint32_t ph = (it / NST) & 1;
-          if (!mbar_wait(&bar_ke[st], ph ^ 1, abort_flag, tmo, SITE_PRODUCER)) { ok = false; break; }
-          mbar_arrive_expect_tx(&bar_kf[st], L::kTileBytes);
-          uint8_t *sK = smem + L::kOffK + st * L::kTileBytes;
+          if (!mbar_wait(sb + BAR_KE + 8 * st, ph ^ 1, abort_flag, tmo, SITE_PRODUCER)) { ok = false; break; }
+          mbar_arrive_expect_tx(sb + BAR_KF + 8 * st, L::kTileBytes);
+          const uint32_t sK = sb + L::kOffK + st * L::kTileBytes;
           for (int hf = 0; hf < L::kHalves; ++hf)
-            tma_load_3d(sK + hf * L::kBoxBytes, &PB.tm_k, hf * 64, h, kv.row0 + r, &bar_kf[st]);
-          if (!mbar_wait(&bar_ve[st], ph ^ 1, abort_flag, tmo, SITE_PRODUCER)) { ok = false; break; }
-          mbar_arrive_expect_tx(&bar_vf[st], L::kTileBytes);
-          uint8_t *sV = smem + L::kOffV + st * L::kTileBytes;
+            tma_load_3d(sK + hf * L::kBoxBytes, &PB.tm_k, hf * 64, h, kv.row0 + r, sb + BAR_KF + 8 * st);
+          if (!mbar_wait(sb + BAR_VE + 8 * st, ph ^ 1, abort_flag, tmo, SITE_PRODUCER)) { ok = false; break; }
+          mbar_arrive_expect_tx(sb + BAR_VF + 8 * st, L::kTileBytes);
+          const uint32_t sV = sb + L::kOffV + st * L::kTileBytes;
           for (int hf = 0; hf < L::kHalves; ++hf)
-            tma_load_3d(sV + hf * L::kBoxBytes, &PB.tm_v, hf * 64, h, kv.row0 + r, &bar_vf[st]);
+            tma_load_3d(sV + hf * L::kBoxBytes, &PB.tm_v, hf * 64, h, kv.row0 + r, sb + BAR_VF + 8 * st);
         }
       }
       // Tail: every stage's last use must be released by the MMA before the
@@ -169,26 +201,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       for (int st = 0; st < NST && st < n_tiles; ++st) {
         const int last = st + ((n_tiles - 1 - st) / NST) * NST;
         const uint32_t ph = (last / NST) & 1;
-        mbar_wait(&bar_ke[st], ph, nullptr, tmo, SITE_TAIL);
-        mbar_wait(&bar_ve[st], ph, nullptr, tmo, SITE_TAIL);
+        mbar_wait(sb + BAR_KE + 8 * st, ph, 0u, tmo, SITE_TAIL);
+        mbar_wait(sb + BAR_VE + 8 * st, ph, 0u, tmo, SITE_TAIL);
       }
     }
   } else if (warp == 1) {
     // =========================================================== MMA issuer
     if (lane == 0 && n_tiles > 0) {
-      const uint32_t sQ = smem_u32(smem + L::kOffQ);
-      const uint32_t sK = smem_u32(smem + L::kOffK);
-      const uint32_t sV = smem_u32(smem + L::kOffV);
+      const uint32_t sQ = sb + L::kOffQ;
+      const uint32_t sK = sb + L::kOffK;
+      const uint32_t sV = sb + L::kOffV;
       // S_qt = Q_qt K^T: K-major A and B, 128B swizzle, K advances 16 elements
       // (32 bytes) inside a 128-byte row, then jumps to the next column block.
+      // Descriptors are built once; advancing the start address only
+      // touches the low 14 bits (addresses stay below 256 KB, no carry).
+      const uint64_t dQ = smem_desc_sw128(sQ, 16, 1024);
+      const uint64_t dK = smem_desc_sw128(sK, 16, 1024);
+      const uint64_t dV = smem_desc_sw128(sV, L::kBoxBytes, 1024);
       auto issue_qk = [&](int qt, int st) {
         const uint32_t d = tmem + qt * 128;
+        const uint64_t a0 = opaque_u64(dQ + ((qt * L::kTileBytes) >> 4));
+        const uint64_t b0 = opaque_u64(dK + ((st * L::kTileBytes) >> 4));
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::kBoxBytes + (kk & 3) * 32;
-          const uint64_t a = smem_desc_sw128(sQ + qt * L::kTileBytes + off, 16, 1024);
-          const uint64_t b = smem_desc_sw128(sK + st * L::kTileBytes + off, 16, 1024);
-          mma_ss(d, a, b, IDESC_QK, kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk >> 2) * L::kBoxBytes + (kk & 3) * 32) >> 4;
+          mma_ss(d, a0 + off, b0 + off, IDESC_QK, kk > 0 ? 1u : 0u);
         }
       };
       // O_qt (+)= P_qt V: P (bf16 pairs) from TMEM over S_qt, V MN-major
@@ -197,23 +234,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       auto issue_pv = [&](int qt, int st, bool acc) {
         const uint32_t d = tmem + 256 + qt * D;
         const uint32_t a = tmem + qt * 128;
+        const uint64_t b0 = opaque_u64(dV + ((st * L::kTileBytes) >> 4));
 #pragma unroll
-        for (int kk = 0; kk < kKVTile / 16; ++kk) {
-          const uint64_t b = smem_desc_sw128(sV + st * L::kTileBytes + kk * 2048, L::kBoxBytes, 1024);
-          mma_ts(d, a + kk * 8, b, IDESC_PV, (acc || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < kKVTile / 16; ++kk)
+          mma_ts(d, a + kk * 8, b0 + ((kk * 2048) >> 4), IDESC_PV, (acc || kk > 0) ? 1u : 0u);
       };
-      bool ok = mbar_wait(bar_q, 0, abort_flag, tmo, SITE_MMA);
-      if (ok) ok = mbar_wait(&bar_kf[0], 0, abort_flag, tmo, SITE_MMA);
+      bool ok = mbar_wait(sb + BAR_Q, 0, abort_flag, tmo, SITE_MMA);
+      if (ok) ok = mbar_wait(sb + BAR_KF, 0, abort_flag, tmo, SITE_MMA);
       if (ok) {
         tc_fence_after();
         issue_qk(0, 0);
-        mma_commit(&bar_s[0]);
+        mma_commit(sb + BAR_S);
         if (has_q1) {
           issue_qk(1, 0);
-          mma_commit(&bar_s[1]);
+          mma_commit(sb + BAR_S + 8);
         }
-        mma_commit(&bar_ke[0]);
+        mma_commit(sb + BAR_KE);
       }
       for (int j = 0; ok && j < n_tiles; ++j) {
         const int st = j % NST;
@@ -221,37 +257,45 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
         const int st1 = (j + 1) % NST;
         const uint32_t ph1 = ((j + 1) / NST) & 1;
         const bool more = j + 1 < n_tiles;
-        if (!mbar_wait(&bar_vf[st], ph, abort_flag, tmo, SITE_MMA)) break;
-        if (!mbar_wait(&bar_p[0], j & 1, abort_flag, tmo, SITE_MMA)) break;
+        if (!mbar_wait(sb + BAR_VF + 8 * st, ph, abort_flag, tmo, SITE_MMA)) break;
+        if (!mbar_wait(sb + BAR_P, j & 1, abort_flag, tmo, SITE_MMA)) break;
         tc_fence_after();
         issue_pv(0, st, j > 0);
-        if (!more) mma_commit(&bar_o[0]);
+        if (!more) mma_commit(sb + BAR_O);
         if (more) {
-          if (!mbar_wait(&bar_kf[st1], ph1, abort_flag, tmo, SITE_MMA)) break;
+          if (!mbar_wait(sb + BAR_KF + 8 * st1, ph1, abort_flag, tmo, SITE_MMA)) break;
           tc_fence_after();
           issue_qk(0, st1);
-          mma_commit(&bar_s[0]);
+          mma_commit(sb + BAR_S);
         }
         if (has_q1) {
-          if (!mbar_wait(&bar_p[1], j & 1, abort_flag, tmo, SITE_MMA)) break;
+          if (!mbar_wait(sb + BAR_P + 8, j & 1, abort_flag, tmo, SITE_MMA)) break;
           tc_fence_after();
           issue_pv(1, st, j > 0);
-          if (!more) mma_commit(&bar_o[1]);
+          if (!more) mma_commit(sb + BAR_O + 8);
         }
-        mma_commit(&bar_ve[st]);
+        mma_commit(sb + BAR_VE + 8 * st);
         if (more) {
           if (has_q1) {
             issue_qk(1, st1);
-            mma_commit(&bar_s[1]);
+            mma_commit(sb + BAR_S + 8);
           }
-          mma_commit(&bar_ke[st1]);
+          mma_commit(sb + BAR_KE + 8 * st1);
         }
       }
       // Drain: everything issued has completed before TMEM is released.
-      mma_commit(bar_tail);
-      mbar_wait(bar_tail, 0, nullptr, tmo, SITE_TAIL);
+      mma_commit(sb + BAR_TAIL);
+      mbar_wait(sb + BAR_TAIL, 0, 0u, tmo, SITE_TAIL);
     }
-  } else if (warp >= 4) {
+   }
+  } else {
+    setmaxnreg_inc<kRegsSoftmax>();
+    const Unit U = decode_unit(p);
+    const AttnSeg &SG = p.seg[U.si];
+    const AttnGroup &G = p.group[U.gi];
+    const AttnProblem &PB = p.prob[G.prob];
+    const int h = U.h, q_row0 = U.q_row0, n_tiles = U.n_tiles, rows_left = U.rows_left, pair = U.pair;
+    const bool has_q1 = U.has_q1;
     // =========================================================== softmax
     const int qt = (warp - 4) >> 2;
     const int row = ((warp & 3) << 5) + lane;  // TMEM lane == row of the Q tile
@@ -268,7 +312,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       for (int i = 0; ok && i < SG.kv_count; ++i) {
         const int kv_n = p.kv[SG.kv_first + i].nrows;
         for (int r = 0; r < kv_n; r += kKVTile, ++j) {
-          const bool w = mbar_wait(&bar_s[qt], j & 1, abort_flag, tmo, SITE_SOFTMAX);
+          const bool w = mbar_wait(sb + BAR_S + 8 * qt, j & 1, abort_flag, tmo, SITE_SOFTMAX);
           if (__any_sync(0xffffffffu, !w)) { ok = false; break; }
           __syncwarp();
           tc_fence_after();
@@ -287,49 +331,73 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
           for (int k = 8; k < 128; ++k) mx[k & 7] = fmaxf(mx[k & 7], __uint_as_float(s[k]));
           const float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                    fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * c;
+          // Raise the stored max only when it grows by more than the
+          // threshold; rows that keep a stale max see P <= 2^threshold.
+          float alpha = 1.0f;
+          bool rescale = false;
           if (j == 0) {
             m = tmax;
           } else {
             const bool need = tmax > m + kRescaleThreshold;
-            if (__any_sync(0xffffffffu, need)) {
-              const float alpha = need ? ex2_approx(m - tmax) : 1.0f;
-              if (need) {
-                l *= alpha;
-                m = tmax;
-              }
-#pragma unroll
-              for (int c0 = 0; c0 < D; c0 += 32) {
-                uint32_t o[32];
-                tmem_ld32_wait(tO + c0, o);
-#pragma unroll
-                for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-                tmem_st32(tO + c0, o);
-              }
+            rescale = __any_sync(0xffffffffu, need);
+            if (need) {
+              alpha = ex2_approx(m - tmax);
+              l *= alpha;
+              m = tmax;
             }
           }
-          const float neg_m = -m;
-          float ls[4] = {0.f, 0.f, 0.f, 0.f};
+          // P = 2^(S*c - m): pairs of scores through packed f32x2 FMAs, a
+          // fixed share of the exponentials on the FMA pipe, the rest on the SFU.
+          const uint64_t cc = f2_pack(c, c);
+          const uint64_t mm = f2_pack(-m, -m);
+          uint64_t lsum0 = 0, lsum1 = 0;   // packed partial row sums (0.0f bits)
 #pragma unroll
           for (int c0 = 0; c0 < 128; c0 += 32) {
             uint32_t pk[16];
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
-              const float p0 = ex2_approx(fmaf(__uint_as_float(s[c0 + 2 * k]), c, neg_m));
-              const float p1 = ex2_approx(fmaf(__uint_as_float(s[c0 + 2 * k + 1]), c, neg_m));
-              ls[k & 3] += p0 + p1;
+              const uint64_t x = f2_fma(f2_pack(__uint_as_float(s[c0 + 2 * k]), __uint_as_float(s[c0 + 2 * k + 1])), cc, mm);
+              uint64_t pp;
+              if ((k & 7) < kPolyEighths) {
+                pp = exp2_poly_x2(x);
+              } else {
+                float x0, x1;
+                f2_unpack(x, x0, x1);
+                pp = f2_pack(ex2_approx(x0), ex2_approx(x1));
+              }
+              if (k & 1) lsum1 = f2_add(lsum1, pp); else lsum0 = f2_add(lsum0, pp);
+              float p0, p1;
+              f2_unpack(pp, p0, p1);
               pk[k] = pack_bf16x2(p0, p1);
             }
             tmem_st16(tS + c0 / 2, pk);
           }
-          l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+          {
+            float a0, a1, b0, b1;
+            f2_unpack(lsum0, a0, a1);
+            f2_unpack(lsum1, b0, b1);
+            l += (a0 + a1) + (b0 + b1);
+          }
+          // O holds every earlier tile (the commit that published S covered
+          // the previous PV); rescale it in place before this tile's PV.
+          if (rescale) {
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 32) {
+              uint32_t o[32];
+              tmem_ld32_wait(tO + c0, o);
+#pragma unroll
+              for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+              tmem_st32(tO + c0, o);
+            }
+          }
           tmem_st_wait();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&bar_p[qt]);
+          if (lane == 0) mbar_arrive(sb + BAR_P + 8 * qt);
         }
       }
       if (ok) {
-        const bool w = mbar_wait(&bar_o[qt], 0, abort_flag, tmo, SITE_EPILOGUE);
+        const bool w = mbar_wait(sb + BAR_O + 8 * qt, 0, abort_flag, tmo, SITE_EPILOGUE);
         if (__any_sync(0xffffffffu, !w)) ok = false;
         __syncwarp();
         tc_fence_after();
@@ -380,10 +448,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
   // ---- teardown
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if ((threadIdx.x >> 5) == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(ld_shared_volatile(((smem_u32(smem_raw) + 1023u) & ~1023u) + TMEM_SLOT), kTmemCols);
   }
 }
 

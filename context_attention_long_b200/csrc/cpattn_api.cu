@@ -188,11 +188,11 @@ __global__ void debug_wait_kernel(unsigned long long timeout_ns) {
   __shared__ uint64_t bar;
   __shared__ int abort_flag;
   if (threadIdx.x == 0) {
-    abort_flag = 0;
-    mbar_init(&bar, 1);
+    st_shared_volatile(smem_u32(&abort_flag), 0u);
+    mbar_init(smem_u32(&bar), 1);
     fence_mbar_init();
     // Nothing ever arrives: the wait must give up after timeout_ns.
-    mbar_wait(&bar, 0, &abort_flag, timeout_ns, SITE_DEBUG);
+    mbar_wait(smem_u32(&bar), 0, smem_u32(&abort_flag), timeout_ns, SITE_DEBUG);
   }
 }
 
@@ -236,10 +236,42 @@ struct GroupSpec {
   std::vector<SegSpec> segs;
 };
 
+// Longest-first ordering of the CTAs: a segment whose row count leaves a
+// lone 128-row Q tile (rows mod 256 in 1..128) is split into its full tile
+// pairs and that lone tile; the lone-tile units (about half the work of a pair)
+// are placed after every full pair, so they fill the gaps of the last wave
+// instead of adding a wave.
+static std::vector<GroupSpec> longest_first(const std::vector<GroupSpec> &groups) {
+  constexpr int kPairRows = kQTilesPerCTA * kQTile;
+  std::vector<GroupSpec> head, tail;
+  for (const GroupSpec &g : groups) {
+    GroupSpec main_g{g.prob, g.b, {}}, tail_g{g.prob, g.b, {}};
+    for (const SegSpec &s : g.segs) {
+      const int rem = s.nrows % kPairRows;
+      if (rem == 0 || rem > kQTile || s.nrows < kPairRows) {
+        main_g.segs.push_back(s);
+        continue;
+      }
+      SegSpec m = s, t = s;
+      m.nrows = s.nrows - rem;
+      t.row0 = s.row0 + m.nrows;
+      t.s0 = s.s0 + m.nrows;
+      t.nrows = rem;
+      main_g.segs.push_back(std::move(m));
+      tail_g.segs.push_back(std::move(t));
+    }
+    if (!main_g.segs.empty()) head.push_back(std::move(main_g));
+    if (!tail_g.segs.empty()) tail.push_back(std::move(tail_g));
+  }
+  for (GroupSpec &g : tail) head.push_back(std::move(g));
+  return head;
+}
+
 // Packs the groups into as few launches as the parameter tables allow and
 // launches them in order on `stream`.
-static int run_attention(const std::vector<ProblemSpec> &probs, const std::vector<GroupSpec> &groups, int D,
+static int run_attention(const std::vector<ProblemSpec> &probs, const std::vector<GroupSpec> &groups_in, int D,
                          bool out_f32, cudaStream_t stream) {
+  const std::vector<GroupSpec> groups = longest_first(groups_in);
   std::vector<AttnProblem> encoded(probs.size());
   for (size_t i = 0; i < probs.size(); ++i) {
     const ProblemSpec &ps = probs[i];

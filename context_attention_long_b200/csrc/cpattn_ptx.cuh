@@ -36,47 +36,56 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 }
 
 // ------------------------------------------------------------------ mbarrier
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+// All shared-memory operands are 32-bit shared-window addresses.
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
 __device__ __forceinline__ void fence_mbar_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(bar), "r"(parity)
       : "memory");
   return ok != 0;
 }
+__device__ __forceinline__ uint32_t ld_shared_volatile(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_shared_volatile(uint32_t addr, uint32_t v) {
+  asm volatile("st.volatile.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
 
 // Waits until the phase of `bar` with parity `parity` has completed.  Gives up
-// when `*abort` becomes non-zero (another role gave up) or after `timeout_ns`,
-// in which case it records `site` in the device status word, raises `*abort`
-// for the whole CTA and returns false.  Every pipeline wait goes through here,
-// so a pipeline bug ends the kernel with an error instead of hanging the GPU.
-// `abort` may be null: the wait then ignores other roles (used to drain work
-// already in flight before the CTA releases its resources).
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                          uint64_t timeout_ns, unsigned int site) {
+// when the CTA's abort word (shared address `abort`) becomes non-zero -- another
+// role gave up -- or after `timeout_ns`, in which case it records `site` in the
+// device status word, raises the abort word for the whole CTA and returns
+// false.  Every pipeline wait goes through here, so a pipeline bug ends the
+// kernel with an error instead of hanging the GPU.  `abort` == 0: the wait
+// ignores other roles (used to drain work already in flight before the CTA
+// releases its resources).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t abort, uint64_t timeout_ns,
+                                          unsigned int site) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (abort != nullptr && *abort) return false;
+    if (abort != 0 && ld_shared_volatile(abort) != 0) return false;
     if (globaltimer_ns() - t0 > timeout_ns) {
-      if (abort != nullptr) *abort = 1;
+      if (abort != 0) st_shared_volatile(abort, 1u);
       atomicOr(&g_device_status, site);
       return false;
     }
@@ -90,6 +99,69 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// ------------------------------------------------------- packed f32x2 math
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^x for a pair, on the FMA pipe instead of the SFU (x <= 2^7).  Written
+// from the textbook range reduction 2^x = 2^j * 2^f, j = round(x),
+// f = x - j in [-0.5, 0.5]:
+//   * x is clamped at -125 so that 2^j stays a normal number (2^-125 ~ 0);
+//   * adding 1.5 * 2^23 rounds x to the integer j (round to nearest) and
+//     leaves j in the low mantissa bits of t; subtracting it back gives j;
+//   * 2^f is a degree-3 polynomial whose coefficients were fitted here by a
+//     Remez exchange for minimal relative error on [-0.5, 0.5] (max relative
+//     error 7.5e-5, below the 2^-9 rounding of P to bf16);
+//   * 2^j is applied by adding j to the exponent field: the low bits of t
+//     shifted left by 23 (the high bits of t shift out of the word).
+__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x) {
+  const float kRound = 12582912.0f;     // 1.5 * 2^23
+  const float kC3 = 0.05517166853f;
+  const float kC2 = 0.24261112511f;
+  const float kC1 = 0.69326096773f;
+  const float kC0 = 0.99992805719f;
+  float x0, x1;
+  f2_unpack(x, x0, x1);
+  x = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+  const uint64_t rr = f2_pack(kRound, kRound);
+  const uint64_t t = f2_add(x, rr);
+  const uint64_t f = f2_sub(x, f2_sub(t, rr));
+  uint64_t q = f2_fma(f, f2_pack(kC3, kC3), f2_pack(kC2, kC2));
+  q = f2_fma(q, f, f2_pack(kC1, kC1));
+  q = f2_fma(q, f, f2_pack(kC0, kC0));
+  const uint32_t lo = static_cast<uint32_t>(q) + (static_cast<uint32_t>(t) << 23);
+  const uint32_t hi = static_cast<uint32_t>(q >> 32) + (static_cast<uint32_t>(t >> 32) << 23);
+  return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+
+// Keeps a value in a register without letting the compiler hoist or
+// rematerialise expressions built from it across loop iterations.
+__device__ __forceinline__ uint64_t opaque_u64(uint64_t v) {
+  asm volatile("mov.b64 %0, %0;" : "+l"(v));
+  return v;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);   // .x (low 16 bits) = lo
   return *reinterpret_cast<uint32_t *>(&v);
@@ -98,12 +170,12 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // ---------------------------------------------------------------------- TMA
 // 3-D tiled bulk tensor load global -> shared, completing on an mbarrier with
 // transaction bytes.  No multicast.
-__device__ __forceinline__ void tma_load_3d(void *smem_dst, const CUtensorMap *tm, int c0, int c1,
-                                            int c2, uint64_t *bar) {
+__device__ __forceinline__ void tma_load_3d(uint32_t smem_dst, const CUtensorMap *tm, int c0, int c1, int c2,
+                                            uint32_t bar) {
   asm volatile(
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
       : "memory");
 }
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *tm) {
@@ -111,10 +183,8 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *tm) {
 }
 
 // ------------------------------------------------------------------ tcgen05
-__device__ __forceinline__ void tmem_alloc(uint32_t *smem_result, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                   smem_u32(smem_result)),
-               "r"(ncols)
+__device__ __forceinline__ void tmem_alloc(uint32_t smem_result, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_result), "r"(ncols)
                : "memory");
 }
 __device__ __forceinline__ void tmem_relinquish() {
@@ -153,12 +223,20 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
 }
 // Arrive once on `bar` when every tcgen05 operation issued so far by this
 // thread has completed.
-__device__ __forceinline__ void mma_commit(uint64_t *bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-          smem_u32(bar))
-      : "memory");
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
 }
+// Per-warpgroup register budget (all four warps of the warpgroup execute it).
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
