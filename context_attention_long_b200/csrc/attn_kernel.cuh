@@ -47,8 +47,8 @@ struct AttnSmem {
   static constexpr int kOffK = kOffQ + kQTilesPerCTA * kTileBytes;
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
   static constexpr int kOffBar = kOffV + kStages * kTileBytes;
-  // q, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2], o_final[2], tail
-  static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 2 + 1;
+  // q, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2], o_final[2], tail, p_half[2]
+  static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 2 + 1 + 2;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffMisc + 16;
   static constexpr int kAllocBytes = kBytes + 1024;  // slack to align the base to 1024
@@ -121,9 +121,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
   constexpr uint32_t BAR_P = BAR_S + 16;               // [2]
   constexpr uint32_t BAR_O = BAR_P + 16;               // [2]
   constexpr uint32_t BAR_TAIL = BAR_O + 16;
+  constexpr uint32_t BAR_PH = BAR_TAIL + 8;            // [2] first half of P written
   constexpr uint32_t TMEM_SLOT = L::kOffMisc;
   constexpr uint32_t ABORT = L::kOffMisc + 4;
-  static_assert(BAR_TAIL + 8 <= L::kOffMisc, "barrier area");
+  static_assert(BAR_PH + 16 <= L::kOffMisc, "barrier area");
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -144,6 +145,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       mbar_init(sb + BAR_O + 8 * i, 1);
     }
     mbar_init(sb + BAR_TAIL, 1);
+    mbar_init(sb + BAR_PH, 4);        // one arrival per softmax warp
+    mbar_init(sb + BAR_PH + 8, 4);
     st_shared_volatile(sb + ABORT, 0u);
     fence_mbar_init();
   }
@@ -231,13 +234,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       // O_qt (+)= P_qt V: P (bf16 pairs) from TMEM over S_qt, V MN-major
       // (keys are rows of 128 bytes): 16 keys = 2 groups of 8 rows = 2048
       // bytes per MMA, column blocks of 64 head-dim elements 16 KB apart.
-      auto issue_pv = [&](int qt, int st, bool acc) {
+      // Half h of the keys (kk = 4h .. 4h+3).
+      auto issue_pv = [&](int qt, int st, bool acc, int half) {
         const uint32_t d = tmem + 256 + qt * D;
         const uint32_t a = tmem + qt * 128;
         const uint64_t b0 = opaque_u64(dV + ((st * L::kTileBytes) >> 4));
 #pragma unroll
-        for (int kk = 0; kk < kKVTile / 16; ++kk)
+        for (int k4 = 0; k4 < kKVTile / 32; ++k4) {
+          const int kk = half * (kKVTile / 32) + k4;
           mma_ts(d, a + kk * 8, b0 + ((kk * 2048) >> 4), IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+        }
       };
       bool ok = mbar_wait(sb + BAR_Q, 0, abort_flag, tmo, SITE_MMA);
       if (ok) ok = mbar_wait(sb + BAR_KF, 0, abort_flag, tmo, SITE_MMA);
@@ -258,9 +264,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
         const uint32_t ph1 = ((j + 1) / NST) & 1;
         const bool more = j + 1 < n_tiles;
         if (!mbar_wait(sb + BAR_VF + 8 * st, ph, abort_flag, tmo, SITE_MMA)) break;
+        if (!mbar_wait(sb + BAR_PH, j & 1, abort_flag, tmo, SITE_MMA)) break;
+        tc_fence_after();
+        issue_pv(0, st, j > 0, 0);
         if (!mbar_wait(sb + BAR_P, j & 1, abort_flag, tmo, SITE_MMA)) break;
         tc_fence_after();
-        issue_pv(0, st, j > 0);
+        issue_pv(0, st, j > 0, 1);
         if (!more) mma_commit(sb + BAR_O);
         if (more) {
           if (!mbar_wait(sb + BAR_KF + 8 * st1, ph1, abort_flag, tmo, SITE_MMA)) break;
@@ -269,9 +278,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
           mma_commit(sb + BAR_S);
         }
         if (has_q1) {
+          if (!mbar_wait(sb + BAR_PH + 8, j & 1, abort_flag, tmo, SITE_MMA)) break;
+          tc_fence_after();
+          issue_pv(1, st, j > 0, 0);
           if (!mbar_wait(sb + BAR_P + 8, j & 1, abort_flag, tmo, SITE_MMA)) break;
           tc_fence_after();
-          issue_pv(1, st, j > 0);
+          issue_pv(1, st, j > 0, 1);
           if (!more) mma_commit(sb + BAR_O + 8);
         }
         mma_commit(sb + BAR_VE + 8 * st);
@@ -324,30 +336,45 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
             for (int k = 0; k < 128; ++k)
               if (k >= kvalid) s[k] = __float_as_uint(-INFINITY);
           }
+          // Row max: 8 independent chains of 3-input max.
           float mx[8];
 #pragma unroll
           for (int k = 0; k < 8; ++k) mx[k] = __uint_as_float(s[k]);
 #pragma unroll
-          for (int k = 8; k < 128; ++k) mx[k & 7] = fmaxf(mx[k & 7], __uint_as_float(s[k]));
-          const float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * c;
+          for (int k = 8; k < 128; k += 16)
+#pragma unroll
+            for (int q = 0; q < 8; ++q) mx[q] = fmax3(mx[q], __uint_as_float(s[k + q]), __uint_as_float(s[k + 8 + q]));
+          const float tmax = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * c;
           // Raise the stored max only when it grows by more than the
           // threshold; rows that keep a stale max see P <= 2^threshold.
-          float alpha = 1.0f;
-          bool rescale = false;
           if (j == 0) {
             m = tmax;
           } else {
             const bool need = tmax > m + kRescaleThreshold;
-            rescale = __any_sync(0xffffffffu, need);
-            if (need) {
-              alpha = ex2_approx(m - tmax);
-              l *= alpha;
-              m = tmax;
+            if (__any_sync(0xffffffffu, need)) {
+              const float alpha = need ? ex2_approx(m - tmax) : 1.0f;
+              if (need) {
+                l *= alpha;
+                m = tmax;
+              }
+              // O holds every earlier tile (the commit that published S
+              // covered the previous PV): rescale it in place before this
+              // tile's first PV.
+#pragma unroll 1
+              for (int c0 = 0; c0 < D; c0 += 16) {
+                uint32_t o[16];
+                tmem_ld16_wait(tO + c0, o);
+#pragma unroll
+                for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+                tmem_st16(tO + c0, o);
+              }
             }
           }
-          // P = 2^(S*c - m): pairs of scores through packed f32x2 FMAs, a
-          // fixed share of the exponentials on the FMA pipe, the rest on the SFU.
+          // P = 2^(S*c - m), pairs of scores through packed f32x2 FMAs, a
+          // fixed share of the exponentials on the FMA pipe, the rest on the
+          // SFU.  P is published in two halves (keys 0-63, 64-127) so that
+          // the MMA warp starts PV on the first half while the second half
+          // is computed.
           const uint64_t cc = f2_pack(c, c);
           const uint64_t mm = f2_pack(-m, -m);
           uint64_t lsum0 = 0, lsum1 = 0;   // packed partial row sums (0.0f bits)
@@ -371,24 +398,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
               pk[k] = pack_bf16x2(p0, p1);
             }
             tmem_st16(tS + c0 / 2, pk);
+            if (c0 == 32) {
+              tmem_st_wait();
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(sb + BAR_PH + 8 * qt);
+            }
           }
           {
             float a0, a1, b0, b1;
             f2_unpack(lsum0, a0, a1);
             f2_unpack(lsum1, b0, b1);
             l += (a0 + a1) + (b0 + b1);
-          }
-          // O holds every earlier tile (the commit that published S covered
-          // the previous PV); rescale it in place before this tile's PV.
-          if (rescale) {
-#pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) {
-              uint32_t o[32];
-              tmem_ld32_wait(tO + c0, o);
-#pragma unroll
-              for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-              tmem_st32(tO + c0, o);
-            }
           }
           tmem_st_wait();
           tc_fence_before();
