@@ -22,6 +22,7 @@ __all__ = [
     "cpattn_kv_gather_attention", "cpattn_ulysses_permute", "cpattn_ulysses_unpermute",
     "cpattn_head_sharded_attention", "cpattn_ulysses_attention", "cpattn_unified_attention",
     "cpattn_ulysses_workspace_bytes", "cpattn_unified_workspace_bytes",
+    "cpattn_ulysses_attention_noalloc", "NOALLOC_SCRATCH_BYTES",
     "cpattn_front_loaded_splits", "cpattn_device_status", "cpattn_debug_wait_timeout",
     "status_string",
 ]
@@ -195,6 +196,28 @@ def cpattn_unified_attention(q, k, v, ring_degree, ulysses_degree, ring_lens=Non
                                                    _native.int_array(ring_lens), _native.int_array(head_splits),
                                                    _ptr(workspace), workspace.numel() * workspace.element_size(),
                                                    _stream(stream)), "cpattn_unified_attention")
+    return out, lse
+
+
+# Size of the library-held scratch of cpattn_ulysses_attention_noalloc
+# (CPATTN_NOALLOC_SCRATCH_BYTES in cpattn.h).
+NOALLOC_SCRATCH_BYTES = 64 << 20
+
+
+def cpattn_ulysses_attention_noalloc(q, k, v, B, S, H, D, degree, seq_splits=None, head_splits=None, out=None,
+                                     lse=None, want_lse=True, stream=None):
+    """Ulysses attention for callers that cannot allocate device memory when
+    they call: the scratch lives in a fixed 64 MiB array inside the library
+    (see cpattn.h).  `out` and `lse` should be passed in by such callers; when
+    omitted they are allocated here with torch for convenience.  Concurrent
+    calls on different streams race on the shared scratch."""
+    out = torch.empty_like(q) if out is None else out
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    _check(_native.load().cpattn_ulysses_attention_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, S,
+                                                           D, int(degree), _native.int_array(seq_splits),
+                                                           _native.int_array(head_splits), _stream(stream)),
+           "cpattn_ulysses_attention_noalloc")
     return out, lse
 
 

@@ -795,3 +795,62 @@ int cpattn_debug_wait_timeout(unsigned int timeout_us, cpattn_stream_t stream) {
 }
 
 }  // extern "C"
+
+// ======================================================= no-allocation variant
+//
+// Ulysses attention whose scratch is a file-scope device array instead of a
+// caller-provided workspace (see cpattn_ulysses_attention_noalloc in
+// cpattn.h).  In host code `g_noalloc_scratch` only names the symbol; its
+// device address comes from cudaGetSymbolAddress, looked up once per device
+// with that device current.
+
+namespace cpattn {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[CPATTN_NOALLOC_SCRATCH_BYTES];
+
+static int noalloc_scratch_address(void **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return CPATTN_ERR_CUDA;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return CPATTN_ERR_UNSUPPORTED;
+  static std::mutex mu;
+  static void *addr[kMaxDevices] = {nullptr};
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return CPATTN_ERR_CUDA;
+    }
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return CPATTN_OK;
+}
+
+}  // namespace cpattn
+
+extern "C" int cpattn_ulysses_attention_noalloc(const void *q, const void *k, const void *v, void *out, float *lse,
+                                                int B, int H, int S, int D, int degree, const int *seq_splits,
+                                                const int *head_splits, cpattn_stream_t stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return CPATTN_ERR_NULL;
+  int st = check_attn_shape(B, H, S, D);
+  if (st != CPATTN_OK) return st;
+  if (degree < 1 || degree > kMaxRanks) return CPATTN_ERR_DEGREE;
+  std::vector<int> seq_chk, heads_chk;
+  st = resolve_splits(S, degree, seq_splits, seq_chk);
+  if (st != CPATTN_OK) return st;
+  st = resolve_splits(H, degree, head_splits, heads_chk);
+  if (st != CPATTN_OK) return st;
+  if (cpattn_ulysses_workspace_bytes(B, H, S, D) > static_cast<size_t>(CPATTN_NOALLOC_SCRATCH_BYTES))
+    return CPATTN_ERR_WORKSPACE;
+  st = check_device(nullptr);
+  if (st != CPATTN_OK) return st;
+  void *scratch = nullptr;
+  st = noalloc_scratch_address(&scratch);
+  if (st != CPATTN_OK) return st;
+  return cpattn_ulysses_attention(q, k, v, out, lse, B, H, S, D, degree, seq_splits, head_splits, scratch,
+                                  static_cast<size_t>(CPATTN_NOALLOC_SCRATCH_BYTES), stream);
+}

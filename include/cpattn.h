@@ -239,6 +239,42 @@ int cpattn_unified_attention(const void *q, const void *k, const void *v, void *
                              const int *ring_lens, const int *head_splits, void *workspace,
                              size_t workspace_bytes, cpattn_stream_t stream);
 
+/* ------------------------------------------------- no-allocation variant */
+
+/*
+ * Ulysses attention with scratch held inside the library.  The source pages
+ * have no counterpart to this entry point.
+ *
+ * Who it is for: callers that cannot allocate device memory when they call --
+ * for example a plug-in running inside another framework that owns every
+ * device allocation (its caching allocator is not reachable from the plug-in),
+ * or a service that reserves all GPU memory at start-up and forbids
+ * cudaMalloc/cudaFree on the request path.  Such callers can still provide
+ * inputs and outputs, but not the workspace cpattn_ulysses_attention needs.
+ *
+ * Same computation, arguments, layouts and results as cpattn_ulysses_attention
+ * minus the two workspace arguments.  The four head-sharded scratch buffers
+ * live in one fixed device array compiled into the library,
+ * CPATTN_NOALLOC_SCRATCH_BYTES (64 MiB), present on every GPU that loads the
+ * library and held until the process exits.  A problem that needs more than
+ * that (8 * B*S*H*D bytes) is rejected with CPATTN_ERR_WORKSPACE before any
+ * work is enqueued.
+ *
+ * The first call on a device, with that device current, looks up the array's
+ * device address (cudaGetSymbolAddress); make that first call on each device
+ * before any stream capture.  Every call uses the same array, which keeps the
+ * previous call's contents (nothing in it needs to start at zero): calls that
+ * overlap on the GPU -- on different streams, or from different host threads
+ * without ordering -- race on the array and corrupt each other's results, so
+ * serialise them.  This entry point calls no cudaMalloc, cudaFree or other
+ * allocating routine.
+ */
+#define CPATTN_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+int cpattn_ulysses_attention_noalloc(const void *q, const void *k, const void *v, void *out, float *lse,
+                                     int B, int H, int S, int D, int degree, const int *seq_splits,
+                                     const int *head_splits, cpattn_stream_t stream);
+
 /* ------------------------------------------------------------- utilities */
 
 /*
