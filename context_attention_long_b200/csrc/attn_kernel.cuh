@@ -18,18 +18,30 @@
 // The running (m, l, O) state *is* the LSE merge applied one chunk (and one
 // tile) at a time, so ring attention is one launch with no partials in HBM.
 //
-// CTA organisation (one CTA per SM: 192 KB smem, 512 TMEM columns):
-//   warp 0      TMA producer: Q once, then K and V tiles into 2-stage rings
+// CTA organisation (one CTA per SM: 192 KB smem, 512 TMEM columns), two
+// "slots" each with a 128-row Q tile, its S (scores / P) and O in TMEM:
+//   warp 0      TMA producer: Q, then K and V tiles into 2-stage rings
 //   warp 1      TMEM allocator + single-thread MMA issuer
 //   warps 2-3   idle
-//   warps 4-7   softmax + correction + epilogue for Q tile 0 (one row per thread)
-//   warps 8-11  the same for Q tile 1
+//   warps 4-7   softmax + correction + epilogue for slot 0 (one row per thread)
+//   warps 8-11  the same for slot 1
+// A unit is either
+//   * a pair: two consecutive Q tiles of a segment, one per slot, both walking
+//     the segment's whole K/V tile list (each K/V tile serves both slots), or
+//   * a split (a lone Q tile left over at the end of a segment): the same Q
+//     tile in both slots, slot 0 walking the first half of the K/V tile list
+//     and slot 1 the second half, each with its own K/V stage; the two partial
+//     (m, l, O) states are merged with the LSE rule at the end.  This keeps
+//     two softmax streams in flight for a lone tile instead of serialising
+//     one tile's softmax and MMAs.
 // TMEM columns: S0 [0,128)  S1 [128,256)  O0 [256, 256+D)  O1 [256+D, 256+2D);
 // P_i (bf16 pairs) overwrites S_i columns [0, 64).
-// MMA order per K/V tile j: PV0(j), QK0(j+1), PV1(j), QK1(j+1), so that the
-// tensor core works on one Q tile while the other one's softmax runs.  A commit
-// after QK_i(j) also covers PV_i(j-1), so when softmax i sees S_i(j), O_i
-// already holds every tile before j and may be rescaled in place.
+// MMA order per step j: PV0(j), QK0(j+1), PV1(j), QK1(j+1), so that the
+// tensor core works on one slot while the other slot's softmax runs.  A
+// commit after QK_i(j) also covers PV_i(j-1), so when softmax i sees S_i(j),
+// O_i already holds every earlier tile and may be rescaled in place.  P is
+// published in two halves so that PV starts on keys 0-63 while keys 64-127
+// are still being exponentiated.
 #pragma once
 
 #include "cpattn_internal.h"
@@ -47,10 +59,11 @@ struct AttnSmem {
   static constexpr int kOffK = kOffQ + kQTilesPerCTA * kTileBytes;
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
   static constexpr int kOffBar = kOffV + kStages * kTileBytes;
-  // q, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2], o_final[2], tail, p_half[2]
-  static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 2 + 1 + 2;
+  // q, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2], o_final[2], tail, p_half[2], ml
+  static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 2 + 1 + 2 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kBytes = kOffMisc + 16;
+  static constexpr int kOffML = kOffMisc + 16;        // split units: slot 1's m[128], l[128]
+  static constexpr int kBytes = kOffML + 2 * 128 * 4;
   static constexpr int kAllocBytes = kBytes + 1024;  // slack to align the base to 1024
 };
 
@@ -70,12 +83,14 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale only if the ma
 // the limiter (the FMA-pipe share only lengthened the softmax), so it is 0.
 constexpr int kPolyEighths = 0;
 
-// The work unit of this CTA: group -> head -> segment -> pair of Q tiles.
-// Recomputed inside every role (after its register budget is set) so that no
-// decoded value stays live across the role split.
+// The work unit of this CTA: group -> head -> segment -> pair of Q tiles (or a
+// split lone tile).  Recomputed inside every role (after its register budget
+// is set) so that no decoded value stays live across the role split.
 struct Unit {
   int gi, si, h, pair, q_row0, rows_left, n_tiles;
-  bool has_q1;
+  int n0, n1;      // K/V tiles walked by slot 0 / slot 1
+  bool has_q1;     // pair with a second Q tile
+  bool split;      // lone tile whose K/V list is split between the slots
 };
 
 __device__ __forceinline__ Unit decode_unit(const AttnParams &p) {
@@ -99,7 +114,32 @@ __device__ __forceinline__ Unit decode_unit(const AttnParams &p) {
   int n = 0;
   for (int i = 0; i < SG.kv_count; ++i) n += (p.kv[SG.kv_first + i].nrows + kKVTile - 1) / kKVTile;
   u.n_tiles = n;
+  u.split = SG.split != 0 && !u.has_q1 && n >= 2;
+  if (u.split) {
+    u.n0 = (n + 1) / 2;
+    u.n1 = n - u.n0;
+  } else {
+    u.n0 = n;
+    u.n1 = u.has_q1 ? n : 0;
+  }
   return u;
+}
+
+// Row and number of valid keys of K/V tile `g` of a segment (tiles are
+// numbered across the segment's K/V ranges in order).
+__device__ __forceinline__ void kv_tile(const AttnParams &p, const AttnSeg &SG, int g, int &row, int &valid) {
+  for (int i = 0; i < SG.kv_count; ++i) {
+    const AttnKV kv = p.kv[SG.kv_first + i];
+    const int nt = (kv.nrows + kKVTile - 1) / kKVTile;
+    if (g < nt) {
+      row = kv.row0 + g * kKVTile;
+      valid = min(kKVTile, kv.nrows - g * kKVTile);
+      return;
+    }
+    g -= nt;
+  }
+  row = 0;
+  valid = 0;
 }
 
 template <int D, bool OUT_F32>
@@ -122,9 +162,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
   constexpr uint32_t BAR_O = BAR_P + 16;               // [2]
   constexpr uint32_t BAR_TAIL = BAR_O + 16;
   constexpr uint32_t BAR_PH = BAR_TAIL + 8;            // [2] first half of P written
+  constexpr uint32_t BAR_ML = BAR_PH + 16;             // split: slot 1's (m, l) published
   constexpr uint32_t TMEM_SLOT = L::kOffMisc;
   constexpr uint32_t ABORT = L::kOffMisc + 4;
-  static_assert(BAR_PH + 16 <= L::kOffMisc, "barrier area");
+  static_assert(BAR_ML + 8 <= L::kOffMisc, "barrier area");
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -147,6 +188,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
     mbar_init(sb + BAR_TAIL, 1);
     mbar_init(sb + BAR_PH, 4);        // one arrival per softmax warp
     mbar_init(sb + BAR_PH + 8, 4);
+    mbar_init(sb + BAR_ML, 4);        // one arrival per warp of softmax warpgroup 1
     st_shared_volatile(sb + ABORT, 0u);
     fence_mbar_init();
   }
@@ -165,8 +207,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
    const Unit U = decode_unit(p);
    const AttnSeg &SG = p.seg[U.si];
    const AttnProblem &PB = p.prob[p.group[U.gi].prob];
-   const int h = U.h, q_row0 = U.q_row0, n_tiles = U.n_tiles;
-   const bool has_q1 = U.has_q1;
+   const int h = U.h, q_row0 = U.q_row0, n_tiles = U.n_tiles, n0 = U.n0, n1 = U.n1;
+   const bool has_q1 = U.has_q1, split = U.split;
    if (warp == 0) {
     // =========================================================== producer
     if (lane == 0 && n_tiles > 0) {
@@ -180,50 +222,70 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       if (has_q1)
         for (int hf = 0; hf < L::kHalves; ++hf)
           tma_load_3d(sQ + L::kTileBytes + hf * L::kBoxBytes, &PB.tm_q, hf * 64, h, q_row0 + kQTile, sb + BAR_Q);
-      int it = 0;
       bool ok = true;
-      for (int i = 0; ok && i < SG.kv_count; ++i) {
-        const AttnKV kv = p.kv[SG.kv_first + i];
-        for (int r = 0; r < kv.nrows; r += kKVTile, ++it) {
-          const int st = it % NST;
-          const uint32_t ph = (it / NST) & 1;
-          if (!mbar_wait(sb + BAR_KE + 8 * st, ph ^ 1, abort_flag, tmo, SITE_PRODUCER)) { ok = false; break; }
-          mbar_arrive_expect_tx(sb + BAR_KF + 8 * st, L::kTileBytes);
-          const uint32_t sK = sb + L::kOffK + st * L::kTileBytes;
-          for (int hf = 0; hf < L::kHalves; ++hf)
-            tma_load_3d(sK + hf * L::kBoxBytes, &PB.tm_k, hf * 64, h, kv.row0 + r, sb + BAR_KF + 8 * st);
-          if (!mbar_wait(sb + BAR_VE + 8 * st, ph ^ 1, abort_flag, tmo, SITE_PRODUCER)) { ok = false; break; }
-          mbar_arrive_expect_tx(sb + BAR_VF + 8 * st, L::kTileBytes);
-          const uint32_t sV = sb + L::kOffV + st * L::kTileBytes;
-          for (int hf = 0; hf < L::kHalves; ++hf)
-            tma_load_3d(sV + hf * L::kBoxBytes, &PB.tm_v, hf * 64, h, kv.row0 + r, sb + BAR_VF + 8 * st);
+      auto load_kv = [&](int st, uint32_t ph, int row) -> bool {
+        if (!mbar_wait(sb + BAR_KE + 8 * st, ph ^ 1, abort_flag, tmo, SITE_PRODUCER)) return false;
+        mbar_arrive_expect_tx(sb + BAR_KF + 8 * st, L::kTileBytes);
+        const uint32_t sK = sb + L::kOffK + st * L::kTileBytes;
+        for (int hf = 0; hf < L::kHalves; ++hf)
+          tma_load_3d(sK + hf * L::kBoxBytes, &PB.tm_k, hf * 64, h, row, sb + BAR_KF + 8 * st);
+        if (!mbar_wait(sb + BAR_VE + 8 * st, ph ^ 1, abort_flag, tmo, SITE_PRODUCER)) return false;
+        mbar_arrive_expect_tx(sb + BAR_VF + 8 * st, L::kTileBytes);
+        const uint32_t sV = sb + L::kOffV + st * L::kTileBytes;
+        for (int hf = 0; hf < L::kHalves; ++hf)
+          tma_load_3d(sV + hf * L::kBoxBytes, &PB.tm_v, hf * 64, h, row, sb + BAR_VF + 8 * st);
+        return true;
+      };
+      if (!split) {
+        // Tiles in order through the NST-stage ring.
+        int it = 0;
+        for (int i = 0; ok && i < SG.kv_count; ++i) {
+          const AttnKV kv = p.kv[SG.kv_first + i];
+          for (int r = 0; r < kv.nrows; r += kKVTile, ++it)
+            if (!load_kv(it % NST, (it / NST) & 1, kv.row0 + r)) { ok = false; break; }
+        }
+      } else {
+        // Slot 0's tile j and slot 1's tile j alternate; slot s uses stage s.
+        for (int j = 0; ok && j < n0; ++j) {
+          int row, valid;
+          kv_tile(p, SG, j, row, valid);
+          if (!load_kv(0, j & 1, row)) { ok = false; break; }
+          if (j < n1) {
+            kv_tile(p, SG, n0 + j, row, valid);
+            if (!load_kv(1, j & 1, row)) { ok = false; break; }
+          }
         }
       }
       // Tail: every stage's last use must be released by the MMA before the
       // CTA exits (the releases are asynchronous arrivals on our barriers).
-      for (int st = 0; st < NST && st < n_tiles; ++st) {
-        const int last = st + ((n_tiles - 1 - st) / NST) * NST;
-        const uint32_t ph = (last / NST) & 1;
+      for (int st = 0; st < NST; ++st) {
+        int uses;   // loads that went to stage st
+        if (split) uses = st == 0 ? n0 : n1;
+        else uses = n_tiles > st ? (n_tiles - 1 - st) / NST + 1 : 0;
+        if (uses == 0) continue;
+        const uint32_t ph = split ? ((uses - 1) & 1) : (((uses - 1) * NST + st) / NST) & 1;
         mbar_wait(sb + BAR_KE + 8 * st, ph, 0u, tmo, SITE_TAIL);
         mbar_wait(sb + BAR_VE + 8 * st, ph, 0u, tmo, SITE_TAIL);
       }
     }
-  } else if (warp == 1) {
+   } else if (warp == 1) {
     // =========================================================== MMA issuer
     if (lane == 0 && n_tiles > 0) {
       const uint32_t sQ = sb + L::kOffQ;
       const uint32_t sK = sb + L::kOffK;
       const uint32_t sV = sb + L::kOffV;
-      // S_qt = Q_qt K^T: K-major A and B, 128B swizzle, K advances 16 elements
+      // S_s = Q K^T: K-major A and B, 128B swizzle, K advances 16 elements
       // (32 bytes) inside a 128-byte row, then jumps to the next column block.
       // Descriptors are built once; advancing the start address only
       // touches the low 14 bits (addresses stay below 256 KB, no carry).
       const uint64_t dQ = smem_desc_sw128(sQ, 16, 1024);
       const uint64_t dK = smem_desc_sw128(sK, 16, 1024);
       const uint64_t dV = smem_desc_sw128(sV, L::kBoxBytes, 1024);
-      auto issue_qk = [&](int qt, int st) {
-        const uint32_t d = tmem + qt * 128;
-        const uint64_t a0 = opaque_u64(dQ + ((qt * L::kTileBytes) >> 4));
+      // slot s: S/P in TMEM columns s*128, O at 256 + s*D; its Q tile is
+      // smem tile s for a pair, tile 0 (the same rows) for a split.
+      auto issue_qk = [&](int s, int st) {
+        const uint32_t d = tmem + s * 128;
+        const uint64_t a0 = opaque_u64(dQ + (((split ? 0 : s) * L::kTileBytes) >> 4));
         const uint64_t b0 = opaque_u64(dK + ((st * L::kTileBytes) >> 4));
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -231,13 +293,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
           mma_ss(d, a0 + off, b0 + off, IDESC_QK, kk > 0 ? 1u : 0u);
         }
       };
-      // O_qt (+)= P_qt V: P (bf16 pairs) from TMEM over S_qt, V MN-major
+      // O_s (+)= P_s V: P (bf16 pairs) from TMEM over S_s, V MN-major
       // (keys are rows of 128 bytes): 16 keys = 2 groups of 8 rows = 2048
       // bytes per MMA, column blocks of 64 head-dim elements 16 KB apart.
       // Half h of the keys (kk = 4h .. 4h+3).
-      auto issue_pv = [&](int qt, int st, bool acc, int half) {
-        const uint32_t d = tmem + 256 + qt * D;
-        const uint32_t a = tmem + qt * 128;
+      auto issue_pv = [&](int s, int st, bool acc, int half) {
+        const uint32_t d = tmem + 256 + s * D;
+        const uint32_t a = tmem + s * 128;
         const uint64_t b0 = opaque_u64(dV + ((st * L::kTileBytes) >> 4));
 #pragma unroll
         for (int k4 = 0; k4 < kKVTile / 32; ++k4) {
@@ -246,53 +308,88 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
         }
       };
       bool ok = mbar_wait(sb + BAR_Q, 0, abort_flag, tmo, SITE_MMA);
-      if (ok) ok = mbar_wait(sb + BAR_KF, 0, abort_flag, tmo, SITE_MMA);
-      if (ok) {
-        tc_fence_after();
-        issue_qk(0, 0);
-        mma_commit(sb + BAR_S);
-        if (has_q1) {
-          issue_qk(1, 0);
-          mma_commit(sb + BAR_S + 8);
-        }
-        mma_commit(sb + BAR_KE);
-      }
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        const int st = j % NST;
-        const uint32_t ph = (j / NST) & 1;
-        const int st1 = (j + 1) % NST;
-        const uint32_t ph1 = ((j + 1) / NST) & 1;
-        const bool more = j + 1 < n_tiles;
-        if (!mbar_wait(sb + BAR_VF + 8 * st, ph, abort_flag, tmo, SITE_MMA)) break;
-        if (!mbar_wait(sb + BAR_PH, j & 1, abort_flag, tmo, SITE_MMA)) break;
-        tc_fence_after();
-        issue_pv(0, st, j > 0, 0);
-        if (!mbar_wait(sb + BAR_P, j & 1, abort_flag, tmo, SITE_MMA)) break;
-        tc_fence_after();
-        issue_pv(0, st, j > 0, 1);
-        if (!more) mma_commit(sb + BAR_O);
-        if (more) {
-          if (!mbar_wait(sb + BAR_KF + 8 * st1, ph1, abort_flag, tmo, SITE_MMA)) break;
+      if (!split) {
+        // Pair (or a lone tile with one K/V tile): both slots read every K/V
+        // stage; a stage is released after slot 1 (or slot 0 alone) read it.
+        if (ok) ok = mbar_wait(sb + BAR_KF, 0, abort_flag, tmo, SITE_MMA);
+        if (ok) {
           tc_fence_after();
-          issue_qk(0, st1);
+          issue_qk(0, 0);
           mma_commit(sb + BAR_S);
-        }
-        if (has_q1) {
-          if (!mbar_wait(sb + BAR_PH + 8, j & 1, abort_flag, tmo, SITE_MMA)) break;
-          tc_fence_after();
-          issue_pv(1, st, j > 0, 0);
-          if (!mbar_wait(sb + BAR_P + 8, j & 1, abort_flag, tmo, SITE_MMA)) break;
-          tc_fence_after();
-          issue_pv(1, st, j > 0, 1);
-          if (!more) mma_commit(sb + BAR_O + 8);
-        }
-        mma_commit(sb + BAR_VE + 8 * st);
-        if (more) {
           if (has_q1) {
-            issue_qk(1, st1);
+            issue_qk(1, 0);
             mma_commit(sb + BAR_S + 8);
           }
-          mma_commit(sb + BAR_KE + 8 * st1);
+          mma_commit(sb + BAR_KE);
+        }
+        for (int j = 0; ok && j < n_tiles; ++j) {
+          const int st = j % NST;
+          const uint32_t ph = (j / NST) & 1;
+          const int st1 = (j + 1) % NST;
+          const uint32_t ph1 = ((j + 1) / NST) & 1;
+          const bool more = j + 1 < n_tiles;
+          if (!mbar_wait(sb + BAR_VF + 8 * st, ph, abort_flag, tmo, SITE_MMA)) break;
+          if (!mbar_wait(sb + BAR_PH, j & 1, abort_flag, tmo, SITE_MMA)) break;
+          tc_fence_after();
+          issue_pv(0, st, j > 0, 0);
+          if (!mbar_wait(sb + BAR_P, j & 1, abort_flag, tmo, SITE_MMA)) break;
+          tc_fence_after();
+          issue_pv(0, st, j > 0, 1);
+          if (!more) mma_commit(sb + BAR_O);
+          if (more) {
+            if (!mbar_wait(sb + BAR_KF + 8 * st1, ph1, abort_flag, tmo, SITE_MMA)) break;
+            tc_fence_after();
+            issue_qk(0, st1);
+            mma_commit(sb + BAR_S);
+          }
+          if (has_q1) {
+            if (!mbar_wait(sb + BAR_PH + 8, j & 1, abort_flag, tmo, SITE_MMA)) break;
+            tc_fence_after();
+            issue_pv(1, st, j > 0, 0);
+            if (!mbar_wait(sb + BAR_P + 8, j & 1, abort_flag, tmo, SITE_MMA)) break;
+            tc_fence_after();
+            issue_pv(1, st, j > 0, 1);
+            if (!more) mma_commit(sb + BAR_O + 8);
+          }
+          mma_commit(sb + BAR_VE + 8 * st);
+          if (more) {
+            if (has_q1) {
+              issue_qk(1, st1);
+              mma_commit(sb + BAR_S + 8);
+            }
+            mma_commit(sb + BAR_KE + 8 * st1);
+          }
+        }
+      } else {
+        // Split: slot s owns stage s; its j-th tile is that stage's j-th use.
+        for (int s = 0; ok && s < 2; ++s) {
+          if (!mbar_wait(sb + BAR_KF + 8 * s, 0, abort_flag, tmo, SITE_MMA)) { ok = false; break; }
+          tc_fence_after();
+          issue_qk(s, s);
+          mma_commit(sb + BAR_S + 8 * s);
+          mma_commit(sb + BAR_KE + 8 * s);
+        }
+        for (int j = 0; ok && j < n0; ++j) {
+          for (int s = 0; s < 2; ++s) {
+            const int ns = s == 0 ? n0 : n1;
+            if (j >= ns) continue;
+            if (!mbar_wait(sb + BAR_VF + 8 * s, j & 1, abort_flag, tmo, SITE_MMA)) { ok = false; break; }
+            if (!mbar_wait(sb + BAR_PH + 8 * s, j & 1, abort_flag, tmo, SITE_MMA)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(s, s, j > 0, 0);
+            if (!mbar_wait(sb + BAR_P + 8 * s, j & 1, abort_flag, tmo, SITE_MMA)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(s, s, j > 0, 1);
+            if (j == ns - 1) mma_commit(sb + BAR_O + 8 * s);
+            mma_commit(sb + BAR_VE + 8 * s);
+            if (j + 1 < ns) {
+              if (!mbar_wait(sb + BAR_KF + 8 * s, (j + 1) & 1, abort_flag, tmo, SITE_MMA)) { ok = false; break; }
+              tc_fence_after();
+              issue_qk(s, s);
+              mma_commit(sb + BAR_S + 8 * s);
+              mma_commit(sb + BAR_KE + 8 * s);
+            }
+          }
         }
       }
       // Drain: everything issued has completed before TMEM is released.
@@ -307,30 +404,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
     const AttnGroup &G = p.group[U.gi];
     const AttnProblem &PB = p.prob[G.prob];
     const int h = U.h, q_row0 = U.q_row0, n_tiles = U.n_tiles, rows_left = U.rows_left, pair = U.pair;
-    const bool has_q1 = U.has_q1;
+    const bool has_q1 = U.has_q1, split = U.split;
     // =========================================================== softmax
-    const int qt = (warp - 4) >> 2;
+    const int qt = (warp - 4) >> 2;            // slot
     const int row = ((warp & 3) << 5) + lane;  // TMEM lane == row of the Q tile
-    const bool active = (qt == 0) || has_q1;
+    const bool active = (qt == 0) || has_q1 || split;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) << 5) << 16;
     const uint32_t tS = tmem + lane_base + qt * 128;
     const uint32_t tO = tmem + lane_base + 256 + qt * D;
     const float c = p.scale_log2;
+    // K/V tiles [g_lo, g_hi) of the segment belong to this slot.
+    const int g_lo = (split && qt == 1) ? U.n0 : 0;
+    const int g_hi = split ? (qt == 0 ? U.n0 : U.n0 + U.n1) : n_tiles;
     float m = -INFINITY;  // running max, scaled (log2) domain
     float l = 0.f;        // running sum of 2^(x - m)
     bool ok = true;
     if (active && n_tiles > 0) {
-      int j = 0;
-      for (int i = 0; ok && i < SG.kv_count; ++i) {
+      int g = 0;   // segment tile index; this slot handles g_lo <= g < g_hi
+      for (int i = 0; ok && i < SG.kv_count && g < g_hi; ++i) {
         const int kv_n = p.kv[SG.kv_first + i].nrows;
-        for (int r = 0; r < kv_n; r += kKVTile, ++j) {
+        for (int r = 0; r < kv_n && g < g_hi; r += kKVTile, ++g) {
+          if (g < g_lo) continue;
+          const int j = g - g_lo;
+          const int kvalid = min(kKVTile, kv_n - r);
           const bool w = mbar_wait(sb + BAR_S + 8 * qt, j & 1, abort_flag, tmo, SITE_SOFTMAX);
           if (__any_sync(0xffffffffu, !w)) { ok = false; break; }
           __syncwarp();
           tc_fence_after();
           uint32_t s[128];
           tmem_ld128_wait(tS, s);
-          const int kvalid = min(kKVTile, kv_n - r);
           if (kvalid < kKVTile) {
 #pragma unroll
             for (int k = 0; k < 128; ++k)
@@ -425,7 +527,62 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       }
     }
     // =========================================================== epilogue
-    if (active && ok) {
+    if (split) {
+      // Merge the two slots' partial states (same rows, disjoint keys) with
+      // the LSE rule: slot 1 publishes (m, l) through shared memory, slot 0
+      // combines O0 and O1 from TMEM and writes the rows.
+      const uint32_t ml = sb + L::kOffML;
+      if (qt == 1) {
+        st_shared_f32(ml + 4 * row, m);            // published even after an abort,
+        st_shared_f32(ml + 512 + 4 * row, l);      // so that slot 0 never waits in vain
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sb + BAR_ML);
+      } else {
+        bool w = ok && mbar_wait(sb + BAR_ML, 0, abort_flag, tmo, SITE_EPILOGUE);
+        w = w && mbar_wait(sb + BAR_O + 8, 0, abort_flag, tmo, SITE_EPILOGUE);
+        if (__any_sync(0xffffffffu, !w)) ok = false;
+        __syncwarp();
+        tc_fence_after();
+        if (ok) {
+          const float m1 = ld_shared_f32(ml + 4 * row);
+          const float l1 = ld_shared_f32(ml + 512 + 4 * row);
+          const float mm = fmaxf(m, m1);
+          const float a0 = ex2_approx(m - mm), a1 = ex2_approx(m1 - mm);
+          const float lt = l * a0 + l1 * a1;
+          const float w0 = a0 / lt, w1 = a1 / lt;
+          const bool row_valid = row < rows_left;
+          const int grow = q_row0 + row;
+          const size_t row_elems = (static_cast<size_t>(grow) * PB.H + h) * D;
+#pragma unroll
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t o0[32], o1[32];
+            tmem_ld32_wait(tO + c0, o0);
+            tmem_ld32_wait(tO + D + c0, o1);
+            float v[32];
+#pragma unroll
+            for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(o0[k]) * w0 + __uint_as_float(o1[k]) * w1;
+            if (row_valid) {
+              if constexpr (OUT_F32) {
+                float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(PB.out) + row_elems + c0);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) dst[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+              } else {
+                uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(PB.out) + row_elems + c0);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                  dst[k] = make_uint4(pack_bf16x2(v[8 * k], v[8 * k + 1]), pack_bf16x2(v[8 * k + 2], v[8 * k + 3]),
+                                      pack_bf16x2(v[8 * k + 4], v[8 * k + 5]), pack_bf16x2(v[8 * k + 6], v[8 * k + 7]));
+              }
+            }
+          }
+          if (row_valid && PB.lse != nullptr) {
+            const int sq = SG.s0 + pair * (kQTilesPerCTA * kQTile) + row;
+            PB.lse[static_cast<long long>(G.b) * PB.lse_b + static_cast<long long>(h + PB.lse_h0) * PB.lse_h + sq] =
+                (mm + log2f(lt)) * 0.69314718055994531f;
+          }
+        }
+      }
+    } else if (active && ok) {
       const int valid_rows = qt == 0 ? min(kQTile, rows_left) : rows_left - kQTile;
       const bool row_valid = row < valid_rows;
       const int grow = q_row0 + qt * kQTile + row;

@@ -230,6 +230,7 @@ struct ProblemSpec {
 struct SegSpec {
   int row0, nrows, s0;
   std::vector<AttnKV> kv;
+  int split = 0;   // a lone Q tile: split its K/V tiles between the two slots
 };
 struct GroupSpec {
   int prob, b;
@@ -238,9 +239,10 @@ struct GroupSpec {
 
 // Longest-first ordering of the CTAs: a segment whose row count leaves a
 // lone 128-row Q tile (rows mod 256 in 1..128) is split into its full tile
-// pairs and that lone tile; the lone-tile units (about half the work of a pair)
-// are placed after every full pair, so they fill the gaps of the last wave
-// instead of adding a wave.
+// pairs and that lone tile.  The lone tile becomes a "split" unit (both slots
+// hold its rows and divide its K/V tiles, merged with the LSE rule at the
+// end), about half the work of a pair; those units are placed after every
+// full pair, so they fill the gaps of the last wave instead of adding one.
 static std::vector<GroupSpec> longest_first(const std::vector<GroupSpec> &groups) {
   constexpr int kPairRows = kQTilesPerCTA * kQTile;
   std::vector<GroupSpec> head, tail;
@@ -248,7 +250,13 @@ static std::vector<GroupSpec> longest_first(const std::vector<GroupSpec> &groups
     GroupSpec main_g{g.prob, g.b, {}}, tail_g{g.prob, g.b, {}};
     for (const SegSpec &s : g.segs) {
       const int rem = s.nrows % kPairRows;
-      if (rem == 0 || rem > kQTile || s.nrows < kPairRows) {
+      if (s.nrows <= kQTile) {          // the whole segment is one lone tile
+        SegSpec t = s;
+        t.split = 1;
+        tail_g.segs.push_back(std::move(t));
+        continue;
+      }
+      if (rem == 0 || rem > kQTile) {
         main_g.segs.push_back(s);
         continue;
       }
@@ -257,6 +265,7 @@ static std::vector<GroupSpec> longest_first(const std::vector<GroupSpec> &groups
       t.row0 = s.row0 + m.nrows;
       t.s0 = s.s0 + m.nrows;
       t.nrows = rem;
+      t.split = 1;
       main_g.segs.push_back(std::move(m));
       tail_g.segs.push_back(std::move(t));
     }
@@ -357,6 +366,7 @@ static int run_attention(const std::vector<ProblemSpec> &probs, const std::vecto
       sg.kv_first = n_kv;
       sg.kv_count = need_kv;
       sg.tile_base = g.tiles_per_head;
+      sg.split = ss.split;
       for (const AttnKV &kv : ss.kv) P->kv[n_kv++] = kv;
       g.seg_count += 1;
       g.tiles_per_head += (ss.nrows + kQTilesPerCTA * kQTile - 1) / (kQTilesPerCTA * kQTile);

@@ -58,6 +58,7 @@ struct AttnSeg {
   int kv_first;   // index into kv[]
   int kv_count;   // number of K/V ranges (0: empty -> out 0, lse -inf)
   int tile_base;  // first tile pair of this segment within the group's head
+  int split;      // 1: a lone Q tile whose K/V tiles are split between the two slots
 };
 
 struct AttnKV {

@@ -69,6 +69,15 @@ __device__ __forceinline__ void st_shared_volatile(uint32_t addr, uint32_t v) {
   asm volatile("st.volatile.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
+__device__ __forceinline__ void st_shared_f32(uint32_t addr, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+__device__ __forceinline__ float ld_shared_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+
 // Waits until the phase of `bar` with parity `parity` has completed.  Gives up
 // when the CTA's abort word (shared address `abort`) becomes non-zero -- another
 // role gave up -- or after `timeout_ns`, in which case it records `site` in the
