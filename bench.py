@@ -225,6 +225,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-breakdown", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time every workload's paths (one JSON line per path) instead of the step")
     ap.add_argument("--kernel", default=None, choices=["ring", "head_sharded", "permute", "merge", "ring_step"],
                     help="profiling mode: run only this kernel (warmup + steps launches) on the workload")
     args = ap.parse_args()
@@ -235,6 +237,9 @@ def main():
         return
     if args.kernel is not None:
         run_single_kernel(args)
+        return
+    if args.sweep:
+        run_sweep(args)
         return
 
     import torch
@@ -436,6 +441,83 @@ def breakdown(api, torch, dev, flush, peaks, inputs):
     del po, pl, ob, lo
     torch.cuda.empty_cache()
     return res
+
+
+def run_sweep(args):
+    """Every workload's paths, each timed on its own (median of `steps` reps,
+    L2 flushed before each rep): attention TFLOP/s per path."""
+    import torch
+    from context_attention_long_b200 import api, build, inputs
+    build.build()
+    dev = torch.device("cuda", 0)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    peaks, kind = load_peaks()
+    reps = max(3, args.steps)
+
+    def timeit(fn):
+        for _ in range(args.warmup):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            b.synchronize()
+            ts.append(a.elapsed_time(b))
+        return float(np.median(ts))
+
+    for name in ("tiny", "dit", "hires", "anything", "video"):
+        cfg, qb, kb, vb = inputs.config_inputs(name)
+        B, S, H, D = qb.shape
+        q, k, v = (torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev) for x in (qb, kb, vb))
+        del qb, kb, vb
+        flops = 4.0 * B * H * S * S * D
+        paths = []
+        P = cfg["ring_degree"]
+        lens = None
+        if name == "anything":
+            lens = inputs.ring_anything_lens(S, P, cfg["seed"])
+        paths.append((f"ring fused P={P}" + (" (Ring Anything)" if lens else ""),
+                      lambda: api.cpattn_ring_attention(q, k, v, P, lens, want_lse=True)))
+        if name in ("tiny", "dit"):
+            po = torch.empty((P, B, S, H, D), dtype=torch.float32, device=dev)
+            pl = torch.empty((P, B, H, S), dtype=torch.float32, device=dev)
+            ob = torch.empty_like(q)
+            lo = torch.empty((B, H, S), dtype=torch.float32, device=dev)
+
+            def unfused():
+                for t in range(P):
+                    api.cpattn_ring_step(q, k, v, P, t, lens, part_out=po[t], part_lse=pl[t])
+                api.cpattn_lse_merge(po, pl, out_bf16=ob, lse_out=lo)
+            paths.append((f"ring unfused P={P} (steps + LSE merge)", unfused))
+        kvd = cfg.get("kv_gather_degree", P)
+        if S % kvd == 0:
+            paths.append((f"kv_gather {kvd}", lambda: api.cpattn_kv_gather_attention(q, k, v, kvd)))
+        U = cfg["ulysses_degree"]
+        if name == "video":
+            ws = torch.empty(api.cpattn_unified_workspace_bytes(B, H, S, D), dtype=torch.uint8, device=dev)
+            paths.append((f"unified ring {P} x Ulysses {U}",
+                          lambda: api.cpattn_unified_attention(q, k, v, P, U, workspace=ws)))
+        else:
+            seq = inputs.front_loaded_splits(S, U) if name == "anything" else None
+            heads = inputs.front_loaded_splits(H, U) if name == "anything" else None
+            ws = torch.empty(api.cpattn_ulysses_workspace_bytes(B, H, S, D), dtype=torch.uint8, device=dev)
+            qf, kf, vf = q.reshape(-1), k.reshape(-1), v.reshape(-1)
+            paths.append((f"Ulysses {U}" + (" (Anything)" if seq else "") + " flow: 3 permutes + attention + unpermute",
+                          lambda: api.cpattn_ulysses_attention(qf, kf, vf, B, S, H, D, U, seq, heads, workspace=ws)))
+        for label, fn in paths:
+            ms = timeit(fn)
+            tf = flops / (ms * 1e-3) / 1e12
+            print(json.dumps({"workload": name, "shape": f"B{B} H{H} S{S} D{D}", "path": label, "ms": round(ms, 4),
+                              "TFLOP/s": round(tf, 1), "frac_bf16_peak": round(tf / float(peaks["bf16_tflops"]), 4),
+                              "peak_kind": kind}), flush=True)
+        st, code = api.cpattn_device_status()
+        if st != 0:
+            raise RuntimeError(f"device wait expired: {code:#x}")
+        del q, k, v
+        torch.cuda.empty_cache()
 
 
 def run_single_kernel(args):
