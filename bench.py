@@ -128,6 +128,20 @@ class ClockSampler:
                 "sm_max_mhz": float(self.max_mhz), "reasons": reasons, "samples": len(win)}
 
 
+def aggregate_over_ranks(ms_local, steps, units_per_step, world, dist=None, device="cpu"):
+    """Whole-job figures from every rank's device-timed milliseconds for
+    `steps` steps: the job time is the max over ranks (all ranks do the same
+    work, emulated independently), and the throughput counts every rank's
+    units.  Returns (ms per step, units per second)."""
+    import torch
+    ms = float(ms_local)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return ms / steps, world * units_per_step * steps / (ms * 1e-3)
+
+
 # ----------------------------------------------------------------- reference arm (the oracle)
 def oracle_sample_step(cfg, q, k, v, rows_per_shard, seed):
     """The oracle's hot path on a bounded sample of query rows: for each ring
@@ -323,13 +337,9 @@ def main():
 
     per = np.array([[ev[i][j].elapsed_time(ev[i][j + 1]) for j in range(n_ev - 1)] for i in range(args.steps)])
     step_ms = per.sum(axis=1)
-    ms_total = float(step_ms.sum())
-    if world > 1:
-        t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
-    ms_per_step = ms_total / args.steps
-    value = world * step_flops * args.steps / (ms_total * 1e-3) / 1e12
+    ms_per_step, flops_per_s = aggregate_over_ranks(float(step_ms.sum()), args.steps, step_flops, world,
+                                                    dist if world > 1 else None, dev)
+    value = flops_per_s / 1e12
 
     peaks, peaks_kind = load_peaks()
     ring_ms = float(per[:, 0].mean())
@@ -379,6 +389,14 @@ def main():
     if not args.no_breakdown:
         kernels.update(breakdown(api, torch, dev, flush, peaks, inputs))
 
+    # Accounting: what P GPUs would exchange per rank for this workload (on one
+    # GPU the exchanges are emulated in memory).
+    exch = {}
+    for mode, deg in (("ring", P), ("ulysses", U), ("kv_gather", P)):
+        snd, rcv = api.cpattn_exchange_bytes(mode, B, H, S, D, deg)
+        exch[f"{mode}_{deg}"] = {"send": snd[0], "recv": rcv[0]}
+    exch["kv_gather_over_ulysses"] = exch[f"kv_gather_{P}"]["recv"] / max(1, exch[f"ulysses_{U}"]["recv"])
+
     st, code = api.cpattn_device_status()
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -386,7 +404,7 @@ def main():
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1), RMS-normalised Q/K, bf16)",
         "config": config_block(cfg), "roofline": roofline, "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks.summary(t_wall0, t_wall1), "e2e": e2e, "kernels": kernels,
-        "device_status": code,
+        "device_status": code, "exchange_bytes_per_rank": exch,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, qb, kb, vb)

@@ -23,7 +23,7 @@ __all__ = [
     "cpattn_head_sharded_attention", "cpattn_ulysses_attention", "cpattn_unified_attention",
     "cpattn_ulysses_workspace_bytes", "cpattn_unified_workspace_bytes",
     "cpattn_ulysses_attention_noalloc", "NOALLOC_SCRATCH_BYTES",
-    "cpattn_front_loaded_splits", "cpattn_device_status", "cpattn_debug_wait_timeout",
+    "cpattn_front_loaded_splits", "cpattn_exchange_bytes", "cpattn_device_status", "cpattn_debug_wait_timeout",
     "status_string",
 ]
 
@@ -225,6 +225,20 @@ def cpattn_front_loaded_splits(total, parts):
     arr = (ctypes.c_int * max(1, int(parts)))()
     _check(_native.load().cpattn_front_loaded_splits(int(total), int(parts), arr), "cpattn_front_loaded_splits")
     return [int(arr[i]) for i in range(int(parts))]
+
+
+EXCHANGE_MODES = {"ring": 0, "ulysses": 1, "kv_gather": 2}
+
+
+def cpattn_exchange_bytes(mode, B, H, S, D, degree, seq_splits=None, head_splits=None, elem_bytes=2):
+    """Per-rank (send, recv) bytes of one attention call under an exchange
+    ('ring', 'ulysses' or 'kv_gather'); host arithmetic only."""
+    send = (ctypes.c_ulonglong * int(degree))()
+    recv = (ctypes.c_ulonglong * int(degree))()
+    _check(_native.load().cpattn_exchange_bytes(EXCHANGE_MODES[mode], B, H, S, D, elem_bytes, int(degree),
+                                                _native.int_array(seq_splits), _native.int_array(head_splits),
+                                                send, recv), "cpattn_exchange_bytes")
+    return [int(x) for x in send], [int(x) for x in recv]
 
 
 def cpattn_device_status(stream=None):

@@ -307,11 +307,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
           mma_ts(d, a + kk * 8, b0 + ((kk * 2048) >> 4), IDESC_PV, (acc || kk > 0) ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(sb + BAR_Q, 0, abort_flag, tmo, SITE_MMA);
+      bool ok = mbar_wait_spin(sb + BAR_Q, 0, abort_flag, tmo, SITE_MMA);
       if (!split) {
         // Pair (or a lone tile with one K/V tile): both slots read every K/V
         // stage; a stage is released after slot 1 (or slot 0 alone) read it.
-        if (ok) ok = mbar_wait(sb + BAR_KF, 0, abort_flag, tmo, SITE_MMA);
+        if (ok) ok = mbar_wait_spin(sb + BAR_KF, 0, abort_flag, tmo, SITE_MMA);
         if (ok) {
           tc_fence_after();
           issue_qk(0, 0);
@@ -328,25 +328,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
           const int st1 = (j + 1) % NST;
           const uint32_t ph1 = ((j + 1) / NST) & 1;
           const bool more = j + 1 < n_tiles;
-          if (!mbar_wait(sb + BAR_VF + 8 * st, ph, abort_flag, tmo, SITE_MMA)) break;
-          if (!mbar_wait(sb + BAR_PH, j & 1, abort_flag, tmo, SITE_MMA)) break;
+          if (!mbar_wait_spin(sb + BAR_VF + 8 * st, ph, abort_flag, tmo, SITE_MMA)) break;
+          if (!mbar_wait_spin(sb + BAR_PH, j & 1, abort_flag, tmo, SITE_MMA)) break;
           tc_fence_after();
           issue_pv(0, st, j > 0, 0);
-          if (!mbar_wait(sb + BAR_P, j & 1, abort_flag, tmo, SITE_MMA)) break;
+          if (!mbar_wait_spin(sb + BAR_P, j & 1, abort_flag, tmo, SITE_MMA)) break;
           tc_fence_after();
           issue_pv(0, st, j > 0, 1);
           if (!more) mma_commit(sb + BAR_O);
           if (more) {
-            if (!mbar_wait(sb + BAR_KF + 8 * st1, ph1, abort_flag, tmo, SITE_MMA)) break;
+            if (!mbar_wait_spin(sb + BAR_KF + 8 * st1, ph1, abort_flag, tmo, SITE_MMA)) break;
             tc_fence_after();
             issue_qk(0, st1);
             mma_commit(sb + BAR_S);
           }
           if (has_q1) {
-            if (!mbar_wait(sb + BAR_PH + 8, j & 1, abort_flag, tmo, SITE_MMA)) break;
+            if (!mbar_wait_spin(sb + BAR_PH + 8, j & 1, abort_flag, tmo, SITE_MMA)) break;
             tc_fence_after();
             issue_pv(1, st, j > 0, 0);
-            if (!mbar_wait(sb + BAR_P + 8, j & 1, abort_flag, tmo, SITE_MMA)) break;
+            if (!mbar_wait_spin(sb + BAR_P + 8, j & 1, abort_flag, tmo, SITE_MMA)) break;
             tc_fence_after();
             issue_pv(1, st, j > 0, 1);
             if (!more) mma_commit(sb + BAR_O + 8);
@@ -363,7 +363,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       } else {
         // Split: slot s owns stage s; its j-th tile is that stage's j-th use.
         for (int s = 0; ok && s < 2; ++s) {
-          if (!mbar_wait(sb + BAR_KF + 8 * s, 0, abort_flag, tmo, SITE_MMA)) { ok = false; break; }
+          if (!mbar_wait_spin(sb + BAR_KF + 8 * s, 0, abort_flag, tmo, SITE_MMA)) { ok = false; break; }
           tc_fence_after();
           issue_qk(s, s);
           mma_commit(sb + BAR_S + 8 * s);
@@ -373,17 +373,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
           for (int s = 0; s < 2; ++s) {
             const int ns = s == 0 ? n0 : n1;
             if (j >= ns) continue;
-            if (!mbar_wait(sb + BAR_VF + 8 * s, j & 1, abort_flag, tmo, SITE_MMA)) { ok = false; break; }
-            if (!mbar_wait(sb + BAR_PH + 8 * s, j & 1, abort_flag, tmo, SITE_MMA)) { ok = false; break; }
+            if (!mbar_wait_spin(sb + BAR_VF + 8 * s, j & 1, abort_flag, tmo, SITE_MMA)) { ok = false; break; }
+            if (!mbar_wait_spin(sb + BAR_PH + 8 * s, j & 1, abort_flag, tmo, SITE_MMA)) { ok = false; break; }
             tc_fence_after();
             issue_pv(s, s, j > 0, 0);
-            if (!mbar_wait(sb + BAR_P + 8 * s, j & 1, abort_flag, tmo, SITE_MMA)) { ok = false; break; }
+            if (!mbar_wait_spin(sb + BAR_P + 8 * s, j & 1, abort_flag, tmo, SITE_MMA)) { ok = false; break; }
             tc_fence_after();
             issue_pv(s, s, j > 0, 1);
             if (j == ns - 1) mma_commit(sb + BAR_O + 8 * s);
             mma_commit(sb + BAR_VE + 8 * s);
             if (j + 1 < ns) {
-              if (!mbar_wait(sb + BAR_KF + 8 * s, (j + 1) & 1, abort_flag, tmo, SITE_MMA)) { ok = false; break; }
+              if (!mbar_wait_spin(sb + BAR_KF + 8 * s, (j + 1) & 1, abort_flag, tmo, SITE_MMA)) { ok = false; break; }
               tc_fence_after();
               issue_qk(s, s);
               mma_commit(sb + BAR_S + 8 * s);

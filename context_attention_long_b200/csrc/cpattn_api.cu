@@ -785,6 +785,34 @@ int cpattn_unified_attention(const void *q, const void *k, const void *v, void *
   return launch_permute(p2, stream) == cudaSuccess ? CPATTN_OK : CPATTN_ERR_CUDA;
 }
 
+int cpattn_exchange_bytes(int mode, int B, int H, int S, int D, int elem_bytes, int degree, const int *seq_splits,
+                          const int *head_splits, unsigned long long *send, unsigned long long *recv) {
+  if (send == nullptr || recv == nullptr) return CPATTN_ERR_NULL;
+  if (B < 1 || H < 1 || S < 1 || D < 1 || elem_bytes < 1 || mode < 0 || mode > 2) return CPATTN_ERR_SHAPE;
+  std::vector<int> seq, heads;
+  int st = resolve_splits(S, degree, seq_splits, seq);
+  if (st != CPATTN_OK) return st;
+  if (mode == 1) {
+    st = resolve_splits(H, degree, head_splits, heads);
+    if (st != CPATTN_OK) return st;
+  }
+  const unsigned long long row = static_cast<unsigned long long>(D) * elem_bytes;   // one (token, head)
+  for (int r = 0; r < degree; ++r) {
+    const unsigned long long sr = static_cast<unsigned long long>(seq[r]);
+    const unsigned long long so = static_cast<unsigned long long>(S) - sr;
+    if (mode == 1) {
+      const unsigned long long hr = static_cast<unsigned long long>(heads[r]);
+      const unsigned long long ho = static_cast<unsigned long long>(H) - hr;
+      send[r] = (3ull * B * sr * ho + 1ull * B * so * hr) * row;
+      recv[r] = (3ull * B * so * hr + 1ull * B * sr * ho) * row;
+    } else {
+      recv[r] = 2ull * B * so * static_cast<unsigned long long>(H) * row;
+      send[r] = 2ull * static_cast<unsigned long long>(degree - 1) * B * sr * static_cast<unsigned long long>(H) * row;
+    }
+  }
+  return CPATTN_OK;
+}
+
 int cpattn_device_status(cpattn_stream_t stream, unsigned int *code) {
   if (code == nullptr) return CPATTN_ERR_NULL;
   int st = check_device(nullptr);

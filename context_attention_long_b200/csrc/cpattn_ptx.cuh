@@ -78,6 +78,38 @@ __device__ __forceinline__ float ld_shared_f32(uint32_t addr) {
   return v;
 }
 
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Same contract as mbar_wait below, but polls without suspending the thread
+// (test_wait): used by the single MMA-issuing thread, whose wake-up latency is
+// on the critical path; abort word and time limit are checked every 64 polls.
+__device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity, uint32_t abort, uint64_t timeout_ns,
+                                               unsigned int site) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if ((i & 63) == 0) {
+      if (abort != 0 && ld_shared_volatile(abort) != 0) return false;
+      if (globaltimer_ns() - t0 > timeout_ns) {
+        if (abort != 0) st_shared_volatile(abort, 1u);
+        atomicOr(&g_device_status, site);
+        return false;
+      }
+    }
+  }
+}
+
 // Waits until the phase of `bar` with parity `parity` has completed.  Gives up
 // when the CTA's abort word (shared address `abort`) becomes non-zero -- another
 // role gave up -- or after `timeout_ns`, in which case it records `site` in the

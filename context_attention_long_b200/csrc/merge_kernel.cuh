@@ -19,6 +19,41 @@ namespace cpattn {
 
 constexpr int kMergeThreads = 256;
 
+// Rows are visited in (b, h, s) order, grid-stride; each thread carries its
+// row's (b, h, s) and advances it by the constant stride, so no row needs a
+// division (the stride is split into whole sequences and a remainder once).
+struct RowCursor {
+  int s, h, b;
+  int ds, dh, db;   // stride in rows = ((db * H) + dh) * S + ds
+  int S, H;
+  __device__ __forceinline__ void init(long long r, long long stride, int S_, int H_) {
+    S = S_;
+    H = H_;
+    s = static_cast<int>(r % S);
+    const long long bh = r / S;
+    h = static_cast<int>(bh % H);
+    b = static_cast<int>(bh / H);
+    ds = static_cast<int>(stride % S);
+    const long long sbh = stride / S;
+    dh = static_cast<int>(sbh % H);
+    db = static_cast<int>(sbh / H);
+  }
+  __device__ __forceinline__ void advance() {
+    s += ds;
+    int carry = 0;
+    if (s >= S) {
+      s -= S;
+      carry = 1;
+    }
+    h += dh + carry;
+    b += db;
+    if (h >= H) {
+      h -= H;
+      b += 1;
+    }
+  }
+};
+
 template <int D, int MAXP>
 __global__ void __launch_bounds__(kMergeThreads) lse_merge_kernel(const MergeParams p) {
   constexpr int LPR = D / 4;            // lanes per row
@@ -26,21 +61,16 @@ __global__ void __launch_bounds__(kMergeThreads) lse_merge_kernel(const MergePar
   const long long nrows = static_cast<long long>(p.B) * p.H * p.S;
   const long long tensor = nrows * D;   // elements of one partial output
   const int lane = threadIdx.x & 31;
-  const int sub = lane / LPR;
   const int col = (lane % LPR) * 4;
   const long long warp_id = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const long long nwarps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  const long long stride = nwarps * RPW;
   const int P = p.P;
-
-  for (long long base = warp_id * RPW; base < nrows; base += nwarps * RPW) {
-    const long long r = base + sub;              // row index in (b, h, s) order
-    if (r >= nrows) continue;
-    const long long s = r % p.S;
-    const long long bh = r / p.S;
-    const long long hh = bh % p.H;
-    const long long b = bh / p.H;
-    const long long o_off = ((b * p.S + s) * p.H + hh) * D + col;   // BSHD element offset
-
+  long long r = warp_id * RPW + lane / LPR;   // row index in (b, h, s) order
+  RowCursor cur;
+  cur.init(r, stride, p.S, p.H);
+  for (; r < nrows; r += stride, cur.advance()) {
+    const long long o_off = ((static_cast<long long>(cur.b) * p.S + cur.s) * p.H + cur.h) * D + col;
     float lse_p[MAXP];
     float4 o_p[MAXP];
 #pragma unroll
@@ -97,18 +127,15 @@ __global__ void __launch_bounds__(kMergeThreads) lse_merge_kernel_anyp(const Mer
   const long long nrows = static_cast<long long>(p.B) * p.H * p.S;
   const long long tensor = nrows * D;
   const int lane = threadIdx.x & 31;
-  const int sub = lane / LPR;
   const int col = (lane % LPR) * 4;
   const long long warp_id = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const long long nwarps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
-  for (long long base = warp_id * RPW; base < nrows; base += nwarps * RPW) {
-    const long long r = base + sub;
-    if (r >= nrows) continue;
-    const long long s = r % p.S;
-    const long long bh = r / p.S;
-    const long long hh = bh % p.H;
-    const long long b = bh / p.H;
-    const long long o_off = ((b * p.S + s) * p.H + hh) * D + col;
+  const long long stride = nwarps * RPW;
+  long long r = warp_id * RPW + lane / LPR;
+  RowCursor cur;
+  cur.init(r, stride, p.S, p.H);
+  for (; r < nrows; r += stride, cur.advance()) {
+    const long long o_off = ((static_cast<long long>(cur.b) * p.S + cur.s) * p.H + cur.h) * D + col;
     float M = -INFINITY;
     for (int i = 0; i < p.P; ++i) M = fmaxf(M, p.part_lse[i * nrows + r]);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);

@@ -287,6 +287,31 @@ int cpattn_ulysses_attention_noalloc(const void *q, const void *k, const void *v
 int cpattn_front_loaded_splits(int total, int parts, int *out);
 
 /*
+ * Per-rank exchange volume of one attention call, the accounting behind the
+ * choice of exchange ([USP] section 5: Ulysses moves O(n*d/P) per GPU with
+ * two all-to-alls, ring O(n*d) over P-1 point-to-point hops; [SP] "Choosing
+ * The Attention Exchange": kv_gather moves about P/2 times the Ulysses payload
+ * per rank, excluding the rank's local shard).  Host-only arithmetic on the
+ * shard sizes; nothing runs on the GPU (on one GPU the exchanges are emulated
+ * in memory, so these bytes are what P GPUs would send and receive).
+ *
+ *   mode         0 ring (K and V chunks rotate through every rank),
+ *                1 Ulysses (Q, K, V to head-sharded, O back),
+ *                2 kv_gather (K and V all-gathered; Q, O stay local).
+ *   seq_splits   host int[degree] or NULL (equal split of S).
+ *   head_splits  host int[degree] or NULL (equal split of H; Ulysses only).
+ *   send, recv   host unsigned long long[degree]: bytes rank r sends/receives.
+ * For rank r with S_r tokens and H_r heads, N_r = B*S_r*H*D*elem_bytes:
+ *   ring, kv_gather: recv = 2 * B*(S-S_r)*H*D*e,  send = 2 * (P-1) * N_r
+ *   Ulysses:        send = 3 * B*S_r*(H-H_r)*D*e + B*(S-S_r)*H_r*D*e,
+ *                   recv = 3 * B*(S-S_r)*H_r*D*e + B*S_r*(H-H_r)*D*e.
+ * Errors: NULL, SHAPE, DEGREE, INDIVISIBLE, SPLITS.
+ */
+int cpattn_exchange_bytes(int mode, int B, int H, int S, int D, int elem_bytes, int degree,
+                          const int *seq_splits, const int *head_splits, unsigned long long *send,
+                          unsigned long long *recv);
+
+/*
  * Synchronises `stream`, then reads and clears the device status word that the
  * kernels' bounded waits set when a pipeline wait expires.  *code receives the
  * raw word (0 = healthy; otherwise a bit per wait site).  Returns CPATTN_OK,
