@@ -441,9 +441,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
           // Row max: 8 independent chains of 3-input max.
           float mx[8];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) mx[k] = __uint_as_float(s[k]);
+          for (int k = 0; k < 8; ++k) mx[k] = fmaxf(__uint_as_float(s[k]), __uint_as_float(s[k + 8]));
 #pragma unroll
-          for (int k = 8; k < 128; k += 16)
+          for (int k = 16; k < 128; k += 16)
 #pragma unroll
             for (int q = 0; q < 8; ++q) mx[q] = fmax3(mx[q], __uint_as_float(s[k + q]), __uint_as_float(s[k + 8 + q]));
           const float tmax = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * c;

@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -85,16 +86,16 @@ static int check_device(int *dev_out) {
     return CPATTN_ERR_CUDA;
   }
   if (dev < 0 || dev >= kMaxDevices) return CPATTN_ERR_UNSUPPORTED;
-  static int cc_major[kMaxDevices] = {0};
-  if (cc_major[dev] == 0) {
-    int major = 0;
+  static std::atomic<int> cc_major[kMaxDevices];   // 0 = not queried yet
+  int major = cc_major[dev].load(std::memory_order_relaxed);
+  if (major == 0) {
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
       cudaGetLastError();
       return CPATTN_ERR_CUDA;
     }
-    cc_major[dev] = major;
+    cc_major[dev].store(major, std::memory_order_relaxed);
   }
-  if (cc_major[dev] != 10) return CPATTN_ERR_UNSUPPORTED;
+  if (major != 10) return CPATTN_ERR_UNSUPPORTED;
   if (dev_out) *dev_out = dev;
   return CPATTN_OK;
 }
