@@ -3,7 +3,8 @@
 TEST INFRASTRUCTURE, NOT PART OF THE PRODUCT.  A plain, slow, obviously
 correct CPU restatement, in float64, of what the hot path computes:
 
-* monolithic non-causal softmax attention (the plain definition),
+* monolithic non-causal softmax attention (the plain definition), and the
+  causal variant masked by sequence positions,
 * per-chunk partial attention with its log-sum-exp, and the LSE merge of
   partials (ring attention; Ring Anything chunk lengths),
 * the kv_gather exchange (each Q shard against the full K/V),
@@ -23,7 +24,7 @@ Sources (web pages, cited by title and section):
   [SP]   SGLang Diffusion docs, "Sequence Parallelism" -- "Choosing The
          Attention Exchange", "Numerics across node boundaries".
   [USP]  "Ulysses Sequence Parallelism: training with million-token contexts"
-         (article summary) -- sections 2, 3, 4, 5.
+         (article summary) -- sections 2, 3, 4, 5, 7.
   [API]  diffusers docs, "parallel" -- ContextParallelConfig parameters.
   [PR]   sglang PR #30086 analysis -- Gemma 3 attention (B, S, H, D) view and
          head_dim**-0.5 scale.
@@ -36,6 +37,8 @@ from .attention import (
     softmax_scale,
     attention,
     attention_rows,
+    causal_attention,
+    causal_attention_rows,
     lse_merge,
     equal_splits,
     offsets,
@@ -52,7 +55,8 @@ from .permute import (
 )
 
 __all__ = [
-    "softmax_scale", "attention", "attention_rows", "lse_merge", "equal_splits",
+    "softmax_scale", "attention", "attention_rows", "causal_attention",
+    "causal_attention_rows", "lse_merge", "equal_splits",
     "offsets", "ring_order", "ring_attention", "ring_step_partials",
     "kv_gather_attention", "ulysses_permute", "ulysses_unpermute",
     "ulysses_attention", "unified_attention",

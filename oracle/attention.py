@@ -37,21 +37,65 @@ def attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray):
     return out, lse
 
 
-def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray):
-    """Monolithic non-causal softmax attention softmax(Q K^T / sqrt(D)) V.
+def causal_attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, q_pos, k_pos):
+    """Attention of query rows against keys under a causal mask given by
+    sequence positions, for a single (batch, head).
+
+    [USP] section 7: for causal masking over long sequences, Ulysses and ring
+    attention use position ids instead of a materialised 4-D attention mask.
+    Written out: key j is visible to query i iff k_pos[j] <= q_pos[i]; over
+    the visible keys the result is attention_rows' formula.  A query that sees
+    no key gets out = 0, lse = -inf (the neutral element of the LSE merge).
+    """
+    q_pos = np.asarray(q_pos, dtype=np.int64)
+    k_pos = np.asarray(k_pos, dtype=np.int64)
+    n, D = q.shape
+    m = k.shape[0]
+    dv = v.shape[1] if v.ndim == 2 else D
+    out = np.zeros((n, dv))
+    lse = np.full((n,), -np.inf)
+    if m == 0 or n == 0:
+        return out, lse
+    visible = k_pos[None, :] <= q_pos[:, None]                     # (n, m)
+    s = np.where(visible, (q @ k.T) * softmax_scale(D), -np.inf)
+    seen = visible.any(axis=1)
+    row_max = np.where(seen, s.max(axis=1), 0.0)[:, None]
+    e = np.where(visible, np.exp(s - row_max), 0.0)
+    ell = e.sum(axis=1, keepdims=True)
+    out[seen] = (e[seen] @ v) / ell[seen]
+    lse[seen] = (row_max + np.log(np.where(ell > 0, ell, 1.0)))[seen, 0]
+    return out, lse
+
+
+def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, q_pos=None, k_pos=None):
+    """Monolithic softmax attention softmax(Q K^T / sqrt(D)) V, non-causal
+    unless sequence positions are given.
 
     q: (B, Sq, H, D); k, v: (B, Sk, H, D).  Returns out (B, Sq, H, D) and
     lse (B, H, Sq), natural log.  Heads are independent ([USP] section 3).
+    With q_pos (Sq,) and k_pos (Sk,) the causal mask of causal_attention_rows
+    applies.
     """
     B, Sq, H, D = q.shape
     out = np.zeros((B, Sq, H, v.shape[3]))
     lse = np.full((B, H, Sq), -np.inf)
     for b in range(B):
         for h in range(H):
-            o, l = attention_rows(q[b, :, h, :], k[b, :, h, :], v[b, :, h, :])
+            if q_pos is None:
+                o, l = attention_rows(q[b, :, h, :], k[b, :, h, :], v[b, :, h, :])
+            else:
+                o, l = causal_attention_rows(q[b, :, h, :], k[b, :, h, :], v[b, :, h, :], q_pos, k_pos)
             out[b, :, h, :] = o
             lse[b, h, :] = l
     return out, lse
+
+
+def causal_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray):
+    """Monolithic causal attention over one sequence: token i (position i)
+    sees keys 0..i.  q, k, v: (B, S, H, D)."""
+    S = q.shape[1]
+    pos = np.arange(S)
+    return attention(q, k, v, pos, pos)
 
 
 def lse_merge(outs, lses):
@@ -117,11 +161,18 @@ def _chunk_lens(S: int, degree: int, chunk_lens):
     return lens
 
 
-def ring_step_partials(q, k, v, degree: int, step: int, chunk_lens=None):
+def _positions(off, r):
+    """Sequence positions of chunk r's tokens."""
+    return np.arange(off[r], off[r + 1])
+
+
+def ring_step_partials(q, k, v, degree: int, step: int, chunk_lens=None, causal=False):
     """One ring step for every rank: rank r attends its Q shard to the K/V chunk
     it holds at `step`, c = (r - step) mod P.  Returns the partial output
     (B, S, H, D) and LSE (B, H, S) over all Q rows (shard r's rows hold rank
-    r's partial)."""
+    r's partial).  causal: the position mask of causal_attention_rows, with
+    every token's position its index in the full sequence (a chunk after the
+    rank's own shard gives out = 0, lse = -inf)."""
     B, S, H, D = q.shape
     lens = _chunk_lens(S, degree, chunk_lens)
     off = offsets(lens)
@@ -131,13 +182,16 @@ def ring_step_partials(q, k, v, degree: int, step: int, chunk_lens=None):
         c = ring_order(r, degree)[step]
         qs = slice(off[r], off[r + 1])
         ks = slice(off[c], off[c + 1])
-        o, l = attention(q[:, qs], k[:, ks], v[:, ks])
+        if causal:
+            o, l = attention(q[:, qs], k[:, ks], v[:, ks], _positions(off, r), _positions(off, c))
+        else:
+            o, l = attention(q[:, qs], k[:, ks], v[:, ks])
         out[:, qs] = o
         lse[:, :, qs] = l
     return out, lse
 
 
-def ring_attention(q, k, v, degree: int, chunk_lens=None):
+def ring_attention(q, k, v, degree: int, chunk_lens=None, causal=False):
     """Ring attention emulated on one host ([CP] "Ring Attention", "Ring Anything
     Attention"; [API] ring_degree, convert_to_fp32, rotate_method).
 
@@ -147,7 +201,9 @@ def ring_attention(q, k, v, degree: int, chunk_lens=None):
     enter the result).  Rank r holds shard r of Q, K and V.  For t = 0..P-1 it
     computes the partial attention of its Q shard against chunk (r - t) mod P,
     keeping partial output and LSE, and merges all P partials with the LSE rule.
-    Returns out (B, S, H, D) and lse (B, H, S).
+    Returns out (B, S, H, D) and lse (B, H, S).  causal: every partial takes
+    the position mask of causal_attention_rows ([USP] section 7), positions
+    being indices in the full sequence.
     """
     B, S, H, D = q.shape
     lens = _chunk_lens(S, degree, chunk_lens)
@@ -159,7 +215,10 @@ def ring_attention(q, k, v, degree: int, chunk_lens=None):
         outs, lses = [], []
         for c in ring_order(r, degree):
             ks = slice(off[c], off[c + 1])
-            o, l = attention(q[:, qs], k[:, ks], v[:, ks])
+            if causal:
+                o, l = attention(q[:, qs], k[:, ks], v[:, ks], _positions(off, r), _positions(off, c))
+            else:
+                o, l = attention(q[:, qs], k[:, ks], v[:, ks])
             outs.append(o)
             lses.append(l)
         o, l = lse_merge(outs, lses)

@@ -94,14 +94,16 @@ def ulysses_unpermute(y_flat, B, S, H, D, degree, seq_splits=None, head_splits=N
 
 
 def ulysses_attention(q_flat, k_flat, v_flat, B, S, H, D, degree,
-                      seq_splits=None, head_splits=None):
+                      seq_splits=None, head_splits=None, causal=False):
     """Ulysses attention ([USP] section 4; [CP] "Ulysses Attention"): all-to-all
     to the head-sharded layout, local attention of every rank over all S tokens
     of its heads, inverse all-to-all of the output.
 
     q/k/v_flat: float64, sequence-sharded rank buffers.  Returns
     (out_flat in the sequence-sharded layout, lse (B, H, S) indexed by the
-    global head and token)."""
+    global head and token).  causal: the local attention takes the position
+    mask of causal_attention_rows; after the first all-to-all every rank holds
+    all S tokens, so a token's position is its index s ([USP] section 7)."""
     heads = _splits(H, degree, head_splits, "head")
     hoff = offsets(heads)
     yq = ulysses_permute(q_flat, B, S, H, D, degree, seq_splits, heads)
@@ -113,8 +115,9 @@ def ulysses_attention(q_flat, k_flat, v_flat, B, S, H, D, degree,
     kv = head_rank_views(yk, B, S, D, heads)
     vv = head_rank_views(yv, B, S, D, heads)
     ov = head_rank_views(yo, B, S, D, heads)
+    pos = np.arange(S) if causal else None
     for rp in range(degree):
-        o, l = attention(qv[rp], kv[rp], vv[rp])
+        o, l = attention(qv[rp], kv[rp], vv[rp], pos, pos)
         ov[rp][...] = o
         lse[:, hoff[rp]:hoff[rp + 1], :] = l
     out = ulysses_unpermute(yo, B, S, H, D, degree, seq_splits, heads)
@@ -122,7 +125,7 @@ def ulysses_attention(q_flat, k_flat, v_flat, B, S, H, D, degree,
 
 
 def unified_attention(q, k, v, ring_degree, ulysses_degree, ring_lens=None,
-                      head_splits=None, sub_splits=None):
+                      head_splits=None, sub_splits=None, causal=False):
     """Unified (ring x Ulysses) attention ([CP] "Unified Attention"): an
     all-to-all that redistributes heads and tokens, ring attention on the
     result, and the inverse all-to-all.  The GPUs form a ring_degree x
@@ -138,7 +141,9 @@ def unified_attention(q, k, v, ring_degree, ulysses_degree, ring_lens=None,
       2. for every head group u: ring attention over the chunks (ring order,
          LSE merge), Q shard i against K/V chunks (i - t) mod R;
       3. within every ring group: the inverse permute of the output.
-    Returns out (B, S, H, D) and lse (B, H, S)."""
+    Returns out (B, S, H, D) and lse (B, H, S).  causal: step 2 takes the
+    position mask of causal_attention_rows, chunk i's tokens sitting at
+    positions off_i .. off_i + len_i - 1 ([USP] section 7)."""
     B, S, H, D = q.shape
     R, U = ring_degree, ulysses_degree
     rl = equal_splits(S, R) if ring_lens is None else [int(x) for x in ring_lens]
@@ -168,7 +173,11 @@ def unified_attention(q, k, v, ring_degree, ulysses_degree, ring_lens=None,
         for i in range(R):
             outs, lses = [], []
             for c in ring_order(i, R):
-                o, l = attention(Yq[i][u], Yk[c][u], Yv[c][u])
+                if causal:
+                    o, l = attention(Yq[i][u], Yk[c][u], Yv[c][u],
+                                     np.arange(roff[i], roff[i + 1]), np.arange(roff[c], roff[c + 1]))
+                else:
+                    o, l = attention(Yq[i][u], Yk[c][u], Yv[c][u])
                 outs.append(o)
                 lses.append(l)
             o, l = lse_merge(outs, lses)

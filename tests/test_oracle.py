@@ -292,6 +292,114 @@ def test_unified_equals_monolithic(B, R, U, ring_lens, heads):
     assert np.max(np.abs(o - ref_o)) < 1e-12 and np.max(np.abs(l - ref_l)) < 1e-12
 
 
+# ----------------------------------------------------------------- causal
+
+def test_causal_attention_matches_scalar_brute_force():
+    """Scalar loops over the visible keys j <= i only, math.exp, no max."""
+    B, S, H, D = 2, 6, 2, 4
+    q, k, v = _rand((B, S, H, D), 50), _rand((B, S, H, D), 51), _rand((B, S, H, D), 52)
+    out, lse = oracle.causal_attention(q, k, v)
+    for b in range(B):
+        for h in range(H):
+            for i in range(S):
+                w = [math.exp(sum(q[b, i, h, d] * k[b, j, h, d] for d in range(D)) / math.sqrt(D)) for j in range(i + 1)]
+                z = sum(w)
+                assert abs(lse[b, h, i] - math.log(z)) < 1e-12
+                for d in range(D):
+                    assert abs(out[b, i, h, d] - sum(w[j] * v[b, j, h, d] for j in range(i + 1)) / z) < 1e-12
+
+
+def test_causal_matches_torch_sdpa_float64():
+    """Independent library routine: torch SDPA with is_causal=True (float64, CPU)."""
+    cfg, q, k, v = _tiny_f64()
+    out, lse = oracle.causal_attention(q, k, v)
+    tq, tk, tv = (torch.from_numpy(x).permute(0, 2, 1, 3) for x in (q, k, v))
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=True).permute(0, 2, 1, 3).numpy()
+    assert np.max(np.abs(out - ref)) < 1e-12
+    S = q.shape[1]
+    scores = torch.matmul(tq, tk.transpose(-1, -2)) / math.sqrt(cfg["D"])
+    scores = scores.masked_fill(torch.ones(S, S, dtype=torch.bool).triu(1), float("-inf"))
+    assert np.max(np.abs(lse - torch.logsumexp(scores, dim=-1).numpy())) < 1e-12
+
+
+def test_causal_zero_keys_closed_form():
+    """K = 0: query i sees i + 1 equal scores, so lse_i = ln(i + 1) and out_i is
+    the running mean of v_0..v_i (an off-by-one in the mask changes both)."""
+    B, S, H, D = 2, 23, 3, 8
+    q, v = _rand((B, S, H, D), 53), _rand((B, S, H, D), 54)
+    out, lse = oracle.causal_attention(q, np.zeros((B, S, H, D)), v)
+    n = np.arange(1, S + 1)
+    assert np.max(np.abs(lse - np.log(n)[None, None, :])) < 1e-13
+    running_mean = np.cumsum(v, axis=1) / n[None, :, None, None]
+    assert np.max(np.abs(out - running_mean)) < 1e-13
+
+
+def test_causal_first_token_returns_its_value():
+    B, S, H, D = 1, 9, 2, 4
+    q, k, v = _rand((B, S, H, D), 55, 3.0), _rand((B, S, H, D), 56, 3.0), _rand((B, S, H, D), 57)
+    out, lse = oracle.causal_attention(q, k, v)
+    assert np.max(np.abs(out[:, 0] - v[:, 0])) < 1e-15
+    s00 = np.einsum("bhd,bhd->bh", q[:, 0], k[:, 0]) / math.sqrt(D)
+    assert np.max(np.abs(lse[:, :, 0] - s00)) < 1e-13
+
+
+def test_causal_query_without_visible_key_is_neutral():
+    q, k, v = _rand((1, 2, 1, 4), 58), _rand((1, 3, 1, 4), 59), _rand((1, 3, 1, 4), 60)
+    out, lse = oracle.attention(q, k, v, np.array([4, 7]), np.array([6, 7, 9]))
+    assert np.all(out[0, 0] == 0) and np.isneginf(lse[0, 0, 0])
+    o1, l1 = oracle.attention(q[:, 1:], k[:, :2], v[:, :2])        # query 7 sees keys 6 and 7
+    assert np.max(np.abs(out[:, 1:] - o1)) < 1e-14 and np.max(np.abs(lse[:, :, 1:] - l1)) < 1e-14
+
+
+@pytest.mark.parametrize("degree,lens", [(1, None), (4, None), (3, [5, 0, 9]), (5, [1, 7, 0, 3, 6]), (2, [13, 1])])
+def test_causal_ring_equals_monolithic(degree, lens):
+    S = 16 if lens is None else sum(lens)
+    B, H, D = 2, 3, 4
+    q, k, v = (_rand((B, S, H, D), s) for s in (61, 62, 63))
+    ref_o, ref_l = oracle.causal_attention(q, k, v)
+    o, l = oracle.ring_attention(q, k, v, degree, lens, causal=True)
+    assert np.max(np.abs(o - ref_o)) < 1e-12 and np.max(np.abs(l - ref_l)) < 1e-12
+
+
+def test_causal_ring_steps_after_the_shard_are_empty_and_merge_to_ring():
+    B, S, H, D, P = 1, 12, 2, 4, 3
+    q, k, v = (_rand((B, S, H, D), s) for s in (64, 65, 66))
+    parts = [oracle.ring_step_partials(q, k, v, P, t, causal=True) for t in range(P)]
+    off = oracle.offsets([4, 4, 4])
+    for t, (o, l) in enumerate(parts):
+        for r in range(P):
+            c = (r - t) % P
+            rows = slice(off[r], off[r + 1])
+            if c > r:
+                assert np.all(o[:, rows] == 0) and np.all(np.isneginf(l[:, :, rows]))
+            else:
+                assert np.all(np.isfinite(l[:, :, rows]))
+    o, l = oracle.lse_merge([p[0] for p in parts], [p[1] for p in parts])
+    ref_o, ref_l = oracle.causal_attention(q, k, v)
+    assert np.max(np.abs(o - ref_o)) < 1e-12 and np.max(np.abs(l - ref_l)) < 1e-12
+
+
+@pytest.mark.parametrize("B,seq,heads", [(1, [6, 6], [2, 2]), (2, [5, 0, 7], [3, 1, 0])])
+def test_causal_ulysses_equals_monolithic(B, seq, heads):
+    S, H, D = sum(seq), sum(heads), 4
+    q, k, v = (_rand((B, S, H, D), s) for s in (67, 68, 69))
+    ref_o, ref_l = oracle.causal_attention(q, k, v)
+    qf, kf, vf = (_seq_rank_buffers_from_full(x, seq) for x in (q, k, v))
+    o, l = oracle.ulysses_attention(qf, kf, vf, B, S, H, D, len(seq), seq, heads, causal=True)
+    assert np.max(np.abs(o - _seq_rank_buffers_from_full(ref_o, seq))) < 1e-12
+    assert np.max(np.abs(l - ref_l)) < 1e-12
+
+
+@pytest.mark.parametrize("B,R,U,ring_lens,heads", [(1, 2, 2, None, None), (2, 3, 2, [5, 0, 9], [3, 1])])
+def test_causal_unified_equals_monolithic(B, R, U, ring_lens, heads):
+    S = 16 if ring_lens is None else sum(ring_lens)
+    H = 4 if heads is None else sum(heads)
+    q, k, v = (_rand((B, S, H, 4), s) for s in (70, 71, 72))
+    ref_o, ref_l = oracle.causal_attention(q, k, v)
+    o, l = oracle.unified_attention(q, k, v, R, U, ring_lens, heads, causal=True)
+    assert np.max(np.abs(o - ref_o)) < 1e-12 and np.max(np.abs(l - ref_l)) < 1e-12
+
+
 # ----------------------------------------------------------------- planted mistakes
 
 def _pins_pass(fn):
@@ -340,6 +448,14 @@ def test_planted_mistakes_are_caught(monkeypatch):
         monkeypatch.setattr(oa, name, good)
         if hasattr(oracle, name):
             monkeypatch.setattr(oracle, name, good)
+    good_causal = oa.causal_attention_rows
+
+    def causal_strict(q, k, v, q_pos, k_pos):
+        return good_causal(q, k, v, np.asarray(q_pos) - 1, k_pos)   # key j visible iff j < i
+
+    monkeypatch.setattr(oa, "causal_attention_rows", causal_strict)
+    assert not _pins_pass(test_causal_zero_keys_closed_form), "planted strict causal mask not caught"
+    monkeypatch.setattr(oa, "causal_attention_rows", good_causal)
     monkeypatch.setattr(op, "ulysses_permute", permute_off_by_one)
     monkeypatch.setattr(oracle, "ulysses_permute", permute_off_by_one)
     assert not _pins_pass(test_permute_hand_worked_cases)
