@@ -241,7 +241,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true",
                     help="time every workload's paths (one JSON line per path) instead of the step")
-    ap.add_argument("--kernel", default=None, choices=["ring", "head_sharded", "permute", "merge", "ring_step"],
+    ap.add_argument("--kernel", default=None, choices=["ring", "causal_ring", "head_sharded", "permute", "merge", "ring_step"],
                     help="profiling mode: run only this kernel (warmup + steps launches) on the workload")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -388,6 +388,7 @@ def main():
     }
     if not args.no_breakdown:
         kernels.update(breakdown(api, torch, dev, flush, peaks, inputs))
+        kernels.update(causal_paths(api, torch, flush, peaks, q, k, v, P, U))
 
     # Accounting: what P GPUs would exchange per rank for this workload (on one
     # GPU the exchanges are emulated in memory).
@@ -412,6 +413,51 @@ def main():
         print(json.dumps(line))
     if world > 1:
         dist.destroy_process_group()
+
+
+def causal_flops(B, H, S, D):
+    """4*D FLOPs per visible (query, key) pair; query i sees keys 0..i."""
+    return 4.0 * B * H * D * S * (S + 1) / 2
+
+
+def causal_paths(api, torch, flush, peaks, q, k, v, P, U):
+    """The causal variants on the bench workload, outside the timed step: the
+    fused causal ring and the causal Ulysses flow, each rep after an L2 flush."""
+    B, S, H, D = q.shape
+    stream = torch.cuda.current_stream()
+    flops = causal_flops(B, H, S, D)
+    peak_tf = float(peaks["bf16_tflops"])
+    out = torch.empty_like(q)
+    lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    ws = torch.empty(api.cpattn_ulysses_workspace_bytes(B, H, S, D), dtype=torch.uint8, device=q.device)
+    qf, kf, vf, of = q.reshape(-1), k.reshape(-1), v.reshape(-1), out.reshape(-1)
+
+    def timeit(fn, reps=10):
+        fn()
+        times = []
+        for _ in range(reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            b.synchronize()
+            times.append(a.elapsed_time(b))
+        return float(np.median(times))
+
+    res = {}
+    for name, fn in (
+        (f"causal_ring_fused_p{P}", lambda: api.cpattn_causal_ring_attention(q, k, v, P, out=out, lse=lse,
+                                                                              stream=stream)),
+        (f"causal_ulysses_{U}_flow", lambda: api.cpattn_causal_ulysses_attention(qf, kf, vf, B, S, H, D, U, out=of,
+                                                                                 lse=lse, workspace=ws,
+                                                                                 stream=stream)),
+    ):
+        ms = timeit(fn)
+        tf = flops / (ms * 1e-3) / 1e12
+        res[name] = {"ms": ms, "TFLOP/s": tf, "frac_bf16_peak": tf / peak_tf,
+                     "flops": "4*D per visible (query, key) pair: 2*B*H*D*S*(S+1)"}
+    return res
 
 
 def breakdown(api, torch, dev, flush, peaks, inputs):
@@ -492,6 +538,7 @@ def run_sweep(args):
         q, k, v = (torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev) for x in (qb, kb, vb))
         del qb, kb, vb
         flops = 4.0 * B * H * S * S * D
+        cflops = causal_flops(B, H, S, D)
         paths = []
         P = cfg["ring_degree"]
         lens = None
@@ -499,6 +546,8 @@ def run_sweep(args):
             lens = inputs.ring_anything_lens(S, P, cfg["seed"])
         paths.append((f"ring fused P={P}" + (" (Ring Anything)" if lens else ""),
                       lambda: api.cpattn_ring_attention(q, k, v, P, lens, want_lse=True)))
+        paths.append((f"causal ring fused P={P}" + (" (Ring Anything)" if lens else ""),
+                      lambda: api.cpattn_causal_ring_attention(q, k, v, P, lens, want_lse=True), cflops))
         if name in ("tiny", "dit"):
             po = torch.empty((P, B, S, H, D), dtype=torch.float32, device=dev)
             pl = torch.empty((P, B, H, S), dtype=torch.float32, device=dev)
@@ -518,6 +567,8 @@ def run_sweep(args):
             ws = torch.empty(api.cpattn_unified_workspace_bytes(B, H, S, D), dtype=torch.uint8, device=dev)
             paths.append((f"unified ring {P} x Ulysses {U}",
                           lambda: api.cpattn_unified_attention(q, k, v, P, U, workspace=ws)))
+            paths.append((f"causal unified ring {P} x Ulysses {U}",
+                          lambda: api.cpattn_causal_unified_attention(q, k, v, P, U, workspace=ws), cflops))
         else:
             seq = inputs.front_loaded_splits(S, U) if name == "anything" else None
             heads = inputs.front_loaded_splits(H, U) if name == "anything" else None
@@ -525,9 +576,13 @@ def run_sweep(args):
             qf, kf, vf = q.reshape(-1), k.reshape(-1), v.reshape(-1)
             paths.append((f"Ulysses {U}" + (" (Anything)" if seq else "") + " flow: 3 permutes + attention + unpermute",
                           lambda: api.cpattn_ulysses_attention(qf, kf, vf, B, S, H, D, U, seq, heads, workspace=ws)))
-        for label, fn in paths:
+            paths.append((f"causal Ulysses {U}" + (" (Anything)" if seq else "") + " flow",
+                          lambda: api.cpattn_causal_ulysses_attention(qf, kf, vf, B, S, H, D, U, seq, heads,
+                                                                      workspace=ws), cflops))
+        for entry in paths:
+            label, fn = entry[0], entry[1]
             ms = timeit(fn)
-            tf = flops / (ms * 1e-3) / 1e12
+            tf = (entry[2] if len(entry) > 2 else flops) / (ms * 1e-3) / 1e12
             print(json.dumps({"workload": name, "shape": f"B{B} H{H} S{S} D{D}", "path": label, "ms": round(ms, 4),
                               "TFLOP/s": round(tf, 1), "frac_bf16_peak": round(tf / float(peaks["bf16_tflops"]), 4),
                               "peak_kind": kind}), flush=True)
@@ -551,6 +606,8 @@ def run_single_kernel(args):
     q, k, v = (torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev) for x in (qb, kb, vb))
     if args.kernel == "ring":
         fn = lambda: api.cpattn_ring_attention(q, k, v, P)
+    elif args.kernel == "causal_ring":
+        fn = lambda: api.cpattn_causal_ring_attention(q, k, v, P)
     elif args.kernel == "ring_step":
         fn = lambda: api.cpattn_ring_step(q, k, v, P, 1)
     elif args.kernel == "head_sharded":

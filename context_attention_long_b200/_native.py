@@ -39,6 +39,18 @@ SIGNATURES = {
     "cpattn_unified_attention": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                          c_int, c_int, c_int, c_int, c_int, c_int, P_INT, P_INT,
                                          c_void_p, c_size_t, c_void_p]),
+    "cpattn_causal_ring_attention": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                             c_int, c_int, c_int, c_int, c_int, P_INT, c_void_p]),
+    "cpattn_causal_ring_step": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                        c_int, c_int, c_int, c_int, c_int, P_INT, c_int, c_void_p]),
+    "cpattn_causal_head_sharded_attention": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                                     c_int, c_int, c_int, c_int, c_int, P_INT, c_void_p]),
+    "cpattn_causal_ulysses_attention": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                                c_int, c_int, c_int, c_int, c_int, P_INT, P_INT,
+                                                c_void_p, c_size_t, c_void_p]),
+    "cpattn_causal_unified_attention": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                                c_int, c_int, c_int, c_int, c_int, c_int, P_INT, P_INT,
+                                                c_void_p, c_size_t, c_void_p]),
     "cpattn_ulysses_attention_noalloc": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                                  c_int, c_int, c_int, c_int, c_int, P_INT, P_INT, c_void_p]),
     "cpattn_front_loaded_splits": (c_int, [c_int, c_int, P_INT]),

@@ -62,29 +62,48 @@ def _bshd(q: torch.Tensor, name="q"):
     return B, S, H, D
 
 
-def cpattn_ring_attention(q, k, v, ring_degree, chunk_lens=None, out=None, lse=None, want_lse=True, stream=None):
-    """Fused ring attention; returns (out bf16 (B,S,H,D), lse float32 (B,H,S) or None)."""
+def _ring(entry, q, k, v, ring_degree, chunk_lens, out, lse, want_lse, stream):
     B, S, H, D = _bshd(q)
     out = torch.empty_like(q) if out is None else out
     if lse is None and want_lse:
         lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
-    _check(_native.load().cpattn_ring_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, S, D,
-                                                int(ring_degree), _native.int_array(chunk_lens), _stream(stream)),
-           "cpattn_ring_attention")
+    _check(getattr(_native.load(), entry)(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, S, D,
+                                          int(ring_degree), _native.int_array(chunk_lens), _stream(stream)), entry)
     return out, lse
 
 
-def cpattn_ring_step(q, k, v, ring_degree, step, chunk_lens=None, part_out=None, part_lse=None, stream=None):
-    """One ring step for every rank; returns float32 (partial out (B,S,H,D), partial lse (B,H,S))."""
+def cpattn_ring_attention(q, k, v, ring_degree, chunk_lens=None, out=None, lse=None, want_lse=True, stream=None):
+    """Fused ring attention; returns (out bf16 (B,S,H,D), lse float32 (B,H,S) or None)."""
+    return _ring("cpattn_ring_attention", q, k, v, ring_degree, chunk_lens, out, lse, want_lse, stream)
+
+
+def cpattn_causal_ring_attention(q, k, v, ring_degree, chunk_lens=None, out=None, lse=None, want_lse=True,
+                                 stream=None):
+    """Fused causal ring attention (key j visible to query i iff j <= i); returns (out, lse)."""
+    return _ring("cpattn_causal_ring_attention", q, k, v, ring_degree, chunk_lens, out, lse, want_lse, stream)
+
+
+def _ring_step(entry, q, k, v, ring_degree, step, chunk_lens, part_out, part_lse, stream):
     B, S, H, D = _bshd(q)
     if part_out is None:
         part_out = torch.empty((B, S, H, D), dtype=torch.float32, device=q.device)
     if part_lse is None:
         part_lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
-    _check(_native.load().cpattn_ring_step(_ptr(q), _ptr(k), _ptr(v), _ptr(part_out), _ptr(part_lse), B, H, S, D,
-                                           int(ring_degree), _native.int_array(chunk_lens), int(step),
-                                           _stream(stream)), "cpattn_ring_step")
+    _check(getattr(_native.load(), entry)(_ptr(q), _ptr(k), _ptr(v), _ptr(part_out), _ptr(part_lse), B, H, S, D,
+                                          int(ring_degree), _native.int_array(chunk_lens), int(step),
+                                          _stream(stream)), entry)
     return part_out, part_lse
+
+
+def cpattn_ring_step(q, k, v, ring_degree, step, chunk_lens=None, part_out=None, part_lse=None, stream=None):
+    """One ring step for every rank; returns float32 (partial out (B,S,H,D), partial lse (B,H,S))."""
+    return _ring_step("cpattn_ring_step", q, k, v, ring_degree, step, chunk_lens, part_out, part_lse, stream)
+
+
+def cpattn_causal_ring_step(q, k, v, ring_degree, step, chunk_lens=None, part_out=None, part_lse=None,
+                            stream=None):
+    """One causal ring step for every rank (a chunk after the rank's shard gives out 0, lse -inf)."""
+    return _ring_step("cpattn_causal_ring_step", q, k, v, ring_degree, step, chunk_lens, part_out, part_lse, stream)
 
 
 def cpattn_lse_merge(part_out, part_lse, out_f32=None, out_bf16=None, lse_out=None, want_f32=False,
@@ -140,16 +159,27 @@ def cpattn_ulysses_unpermute(y, B, S, H, D, degree, seq_splits=None, head_splits
     return x
 
 
-def cpattn_head_sharded_attention(yq, yk, yv, B, S, H, D, degree, head_splits=None, yo=None, lse=None,
-                                  want_lse=True, stream=None):
-    """Local attention on head-sharded rank buffers; returns (yo, lse (B,H,S))."""
+def _head_sharded(entry, yq, yk, yv, B, S, H, D, degree, head_splits, yo, lse, want_lse, stream):
     yo = torch.empty_like(yq) if yo is None else yo
     if lse is None and want_lse:
         lse = torch.empty((B, H, S), dtype=torch.float32, device=yq.device)
-    _check(_native.load().cpattn_head_sharded_attention(_ptr(yq), _ptr(yk), _ptr(yv), _ptr(yo), _ptr(lse), B, H, S,
-                                                        D, int(degree), _native.int_array(head_splits),
-                                                        _stream(stream)), "cpattn_head_sharded_attention")
+    _check(getattr(_native.load(), entry)(_ptr(yq), _ptr(yk), _ptr(yv), _ptr(yo), _ptr(lse), B, H, S, D,
+                                          int(degree), _native.int_array(head_splits), _stream(stream)), entry)
     return yo, lse
+
+
+def cpattn_head_sharded_attention(yq, yk, yv, B, S, H, D, degree, head_splits=None, yo=None, lse=None,
+                                  want_lse=True, stream=None):
+    """Local attention on head-sharded rank buffers; returns (yo, lse (B,H,S))."""
+    return _head_sharded("cpattn_head_sharded_attention", yq, yk, yv, B, S, H, D, degree, head_splits, yo, lse,
+                         want_lse, stream)
+
+
+def cpattn_causal_head_sharded_attention(yq, yk, yv, B, S, H, D, degree, head_splits=None, yo=None, lse=None,
+                                         want_lse=True, stream=None):
+    """Causal local attention on head-sharded rank buffers; returns (yo, lse (B,H,S))."""
+    return _head_sharded("cpattn_causal_head_sharded_attention", yq, yk, yv, B, S, H, D, degree, head_splits, yo,
+                         lse, want_lse, stream)
 
 
 def cpattn_ulysses_workspace_bytes(B, H, S, D) -> int:
@@ -166,37 +196,60 @@ def _workspace(nbytes, device, workspace):
     return workspace
 
 
-def cpattn_ulysses_attention(q, k, v, B, S, H, D, degree, seq_splits=None, head_splits=None, out=None, lse=None,
-                             want_lse=True, workspace=None, stream=None):
-    """Ulysses attention on sequence-sharded rank buffers (flat bf16); returns (out, lse)."""
+def _ulysses(entry, q, k, v, B, S, H, D, degree, seq_splits, head_splits, out, lse, want_lse, workspace, stream):
     out = torch.empty_like(q) if out is None else out
     if lse is None and want_lse:
         lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
     nbytes = cpattn_ulysses_workspace_bytes(B, H, S, D)
     workspace = _workspace(nbytes, q.device, workspace)
-    _check(_native.load().cpattn_ulysses_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, S, D,
-                                                   int(degree), _native.int_array(seq_splits),
-                                                   _native.int_array(head_splits), _ptr(workspace),
-                                                   workspace.numel() * workspace.element_size(), _stream(stream)),
-           "cpattn_ulysses_attention")
+    _check(getattr(_native.load(), entry)(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, S, D,
+                                          int(degree), _native.int_array(seq_splits),
+                                          _native.int_array(head_splits), _ptr(workspace),
+                                          workspace.numel() * workspace.element_size(), _stream(stream)), entry)
     return out, lse
 
 
-def cpattn_unified_attention(q, k, v, ring_degree, ulysses_degree, ring_lens=None, head_splits=None, out=None,
-                             lse=None, want_lse=True, workspace=None, stream=None):
-    """Unified ring x Ulysses attention on full (B,S,H,D) tensors; returns (out, lse)."""
+def cpattn_ulysses_attention(q, k, v, B, S, H, D, degree, seq_splits=None, head_splits=None, out=None, lse=None,
+                             want_lse=True, workspace=None, stream=None):
+    """Ulysses attention on sequence-sharded rank buffers (flat bf16); returns (out, lse)."""
+    return _ulysses("cpattn_ulysses_attention", q, k, v, B, S, H, D, degree, seq_splits, head_splits, out, lse,
+                    want_lse, workspace, stream)
+
+
+def cpattn_causal_ulysses_attention(q, k, v, B, S, H, D, degree, seq_splits=None, head_splits=None, out=None,
+                                    lse=None, want_lse=True, workspace=None, stream=None):
+    """Causal Ulysses attention on sequence-sharded rank buffers (flat bf16); returns (out, lse)."""
+    return _ulysses("cpattn_causal_ulysses_attention", q, k, v, B, S, H, D, degree, seq_splits, head_splits, out,
+                    lse, want_lse, workspace, stream)
+
+
+def _unified(entry, q, k, v, ring_degree, ulysses_degree, ring_lens, head_splits, out, lse, want_lse, workspace,
+             stream):
     B, S, H, D = _bshd(q)
     out = torch.empty_like(q) if out is None else out
     if lse is None and want_lse:
         lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
     nbytes = cpattn_unified_workspace_bytes(B, H, S, D)
     workspace = _workspace(nbytes, q.device, workspace)
-    _check(_native.load().cpattn_unified_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, S, D,
-                                                   int(ring_degree), int(ulysses_degree),
-                                                   _native.int_array(ring_lens), _native.int_array(head_splits),
-                                                   _ptr(workspace), workspace.numel() * workspace.element_size(),
-                                                   _stream(stream)), "cpattn_unified_attention")
+    _check(getattr(_native.load(), entry)(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, S, D,
+                                          int(ring_degree), int(ulysses_degree), _native.int_array(ring_lens),
+                                          _native.int_array(head_splits), _ptr(workspace),
+                                          workspace.numel() * workspace.element_size(), _stream(stream)), entry)
     return out, lse
+
+
+def cpattn_unified_attention(q, k, v, ring_degree, ulysses_degree, ring_lens=None, head_splits=None, out=None,
+                             lse=None, want_lse=True, workspace=None, stream=None):
+    """Unified ring x Ulysses attention on full (B,S,H,D) tensors; returns (out, lse)."""
+    return _unified("cpattn_unified_attention", q, k, v, ring_degree, ulysses_degree, ring_lens, head_splits, out,
+                    lse, want_lse, workspace, stream)
+
+
+def cpattn_causal_unified_attention(q, k, v, ring_degree, ulysses_degree, ring_lens=None, head_splits=None,
+                                    out=None, lse=None, want_lse=True, workspace=None, stream=None):
+    """Causal unified ring x Ulysses attention on full (B,S,H,D) tensors; returns (out, lse)."""
+    return _unified("cpattn_causal_unified_attention", q, k, v, ring_degree, ulysses_degree, ring_lens,
+                    head_splits, out, lse, want_lse, workspace, stream)
 
 
 # Size of the library-held scratch of cpattn_ulysses_attention_noalloc

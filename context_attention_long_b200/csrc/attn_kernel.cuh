@@ -88,10 +88,18 @@ constexpr int kPolyEighths = 0;
 // is set) so that no decoded value stays live across the role split.
 struct Unit {
   int gi, si, h, pair, q_row0, rows_left, n_tiles;
+  int q_last;      // sequence position of the unit's last query row
   int n0, n1;      // K/V tiles walked by slot 0 / slot 1
   bool has_q1;     // pair with a second Q tile
   bool split;      // lone tile whose K/V list is split between the slots
 };
+
+// Rows of K/V range `kv` that a unit walks: all of them, or under the causal
+// mask those at positions <= q_last (later rows are invisible to every query
+// of the unit).
+__device__ __forceinline__ int kv_rows_seen(const AttnParams &p, const AttnKV &kv, int q_last) {
+  return p.causal ? max(0, min(kv.nrows, q_last - kv.s0 + 1)) : kv.nrows;
+}
 
 __device__ __forceinline__ Unit decode_unit(const AttnParams &p) {
   Unit u;
@@ -100,19 +108,38 @@ __device__ __forceinline__ Unit decode_unit(const AttnParams &p) {
   while (gi + 1 < p.num_groups && p.group[gi + 1].unit_base <= unit) ++gi;
   const AttnGroup &G = p.group[gi];
   const int local = unit - G.unit_base;
-  u.h = local / G.tiles_per_head;
-  const int t = local - u.h * G.tiles_per_head;
+  int t;
+  if (!p.causal) {
+    // Head-major: the CTAs running at once share one head's K/V through L2.
+    u.h = local / G.tiles_per_head;
+    t = local - u.h * G.tiles_per_head;
+  } else {
+    // Causal units differ in length: within a block of heads whose K/V fit
+    // in L2 together, order them pair-major (the pair order below runs
+    // heaviest first), so the launch order is close to longest first.
+    const int H = p.prob[G.prob].H;
+    const int block = local / (G.head_block * G.tiles_per_head);
+    const int h0 = block * G.head_block;
+    const int nb = min(G.head_block, H - h0);
+    const int within = local - h0 * G.tiles_per_head;
+    t = within / nb;
+    u.h = h0 + (within - t * nb);
+  }
   int si = G.seg_first;
   while (si + 1 < G.seg_first + G.seg_count && p.seg[si + 1].tile_base <= t) ++si;
   const AttnSeg &SG = p.seg[si];
   u.gi = gi;
   u.si = si;
   u.pair = t - SG.tile_base;
+  // Under the causal mask a later pair walks more K/V tiles: launch a
+  // segment's pairs last-first so the heaviest units start in the first wave.
+  if (p.causal) u.pair = (SG.nrows + kQTilesPerCTA * kQTile - 1) / (kQTilesPerCTA * kQTile) - 1 - u.pair;
   u.q_row0 = SG.row0 + u.pair * (kQTilesPerCTA * kQTile);
   u.rows_left = SG.nrows - u.pair * (kQTilesPerCTA * kQTile);
   u.has_q1 = u.rows_left > kQTile;
+  u.q_last = SG.s0 + u.pair * (kQTilesPerCTA * kQTile) + min(u.rows_left, kQTilesPerCTA * kQTile) - 1;
   int n = 0;
-  for (int i = 0; i < SG.kv_count; ++i) n += (p.kv[SG.kv_first + i].nrows + kKVTile - 1) / kKVTile;
+  for (int i = 0; i < SG.kv_count; ++i) n += (kv_rows_seen(p, p.kv[SG.kv_first + i], u.q_last) + kKVTile - 1) / kKVTile;
   u.n_tiles = n;
   u.split = SG.split != 0 && !u.has_q1 && n >= 2;
   if (u.split) {
@@ -125,15 +152,18 @@ __device__ __forceinline__ Unit decode_unit(const AttnParams &p) {
   return u;
 }
 
-// Row and number of valid keys of K/V tile `g` of a segment (tiles are
-// numbered across the segment's K/V ranges in order).
-__device__ __forceinline__ void kv_tile(const AttnParams &p, const AttnSeg &SG, int g, int &row, int &valid) {
+// Row and number of valid keys of K/V tile `g` of a unit (tiles are numbered
+// across the segment's K/V ranges in order, each range cut to the rows the
+// unit walks).
+__device__ __forceinline__ void kv_tile(const AttnParams &p, const AttnSeg &SG, int q_last, int g, int &row,
+                                        int &valid) {
   for (int i = 0; i < SG.kv_count; ++i) {
     const AttnKV kv = p.kv[SG.kv_first + i];
-    const int nt = (kv.nrows + kKVTile - 1) / kKVTile;
+    const int seen = kv_rows_seen(p, kv, q_last);
+    const int nt = (seen + kKVTile - 1) / kKVTile;
     if (g < nt) {
       row = kv.row0 + g * kKVTile;
-      valid = min(kKVTile, kv.nrows - g * kKVTile);
+      valid = min(kKVTile, seen - g * kKVTile);
       return;
     }
     g -= nt;
@@ -241,17 +271,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
         int it = 0;
         for (int i = 0; ok && i < SG.kv_count; ++i) {
           const AttnKV kv = p.kv[SG.kv_first + i];
-          for (int r = 0; r < kv.nrows; r += kKVTile, ++it)
+          const int seen = kv_rows_seen(p, kv, U.q_last);
+          for (int r = 0; r < seen; r += kKVTile, ++it)
             if (!load_kv(it % NST, (it / NST) & 1, kv.row0 + r)) { ok = false; break; }
         }
       } else {
         // Slot 0's tile j and slot 1's tile j alternate; slot s uses stage s.
         for (int j = 0; ok && j < n0; ++j) {
           int row, valid;
-          kv_tile(p, SG, j, row, valid);
+          kv_tile(p, SG, U.q_last, j, row, valid);
           if (!load_kv(0, j & 1, row)) { ok = false; break; }
           if (j < n1) {
-            kv_tile(p, SG, n0 + j, row, valid);
+            kv_tile(p, SG, U.q_last, n0 + j, row, valid);
             if (!load_kv(1, j & 1, row)) { ok = false; break; }
           }
         }
@@ -404,6 +435,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
     const AttnGroup &G = p.group[U.gi];
     const AttnProblem &PB = p.prob[G.prob];
     const int h = U.h, q_row0 = U.q_row0, n_tiles = U.n_tiles, rows_left = U.rows_left, pair = U.pair;
+    const int q_last = U.q_last;
     const bool has_q1 = U.has_q1, split = U.split;
     // =========================================================== softmax
     const int qt = (warp - 4) >> 2;            // slot
@@ -413,6 +445,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
     const uint32_t tS = tmem + lane_base + qt * 128;
     const uint32_t tO = tmem + lane_base + 256 + qt * D;
     const float c = p.scale_log2;
+    // Sequence position of this thread's query row (both slots of a split
+    // unit hold the same rows).
+    const int q_pos = SG.s0 + pair * (kQTilesPerCTA * kQTile) + (split ? 0 : qt * kQTile) + row;
+    const bool causal = p.causal != 0;
     // K/V tiles [g_lo, g_hi) of the segment belong to this slot.
     const int g_lo = (split && qt == 1) ? U.n0 : 0;
     const int g_hi = split ? (qt == 0 ? U.n0 : U.n0 + U.n1) : n_tiles;
@@ -422,18 +458,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
     if (active && n_tiles > 0) {
       int g = 0;   // segment tile index; this slot handles g_lo <= g < g_hi
       for (int i = 0; ok && i < SG.kv_count && g < g_hi; ++i) {
-        const int kv_n = p.kv[SG.kv_first + i].nrows;
+        const AttnKV kv = p.kv[SG.kv_first + i];
+        const int kv_n = kv_rows_seen(p, kv, q_last);
         for (int r = 0; r < kv_n && g < g_hi; r += kKVTile, ++g) {
           if (g < g_lo) continue;
           const int j = g - g_lo;
-          const int kvalid = min(kKVTile, kv_n - r);
+          // Keys of this tile visible to this row: the tile's valid keys, cut
+          // under the causal mask at the row's own position (may be <= 0).
+          int kvalid = min(kKVTile, kv_n - r);
+          if (causal) kvalid = min(kvalid, q_pos - (kv.s0 + r) + 1);
           const bool w = mbar_wait(sb + BAR_S + 8 * qt, j & 1, abort_flag, tmo, SITE_SOFTMAX);
           if (__any_sync(0xffffffffu, !w)) { ok = false; break; }
           __syncwarp();
           tc_fence_after();
           uint32_t s[128];
           tmem_ld128_wait(tS, s);
-          if (kvalid < kKVTile) {
+          if (__any_sync(0xffffffffu, kvalid < kKVTile)) {
 #pragma unroll
             for (int k = 0; k < 128; ++k)
               if (k >= kvalid) s[k] = __float_as_uint(-INFINITY);
@@ -478,7 +518,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
           // the MMA warp starts PV on the first half while the second half
           // is computed.
           const uint64_t cc = f2_pack(c, c);
-          const uint64_t mm = f2_pack(-m, -m);
+          // A row that has seen no key yet (only under the causal mask) keeps
+          // m = -inf: exponentiate against 0 so its masked scores give P = 0.
+          const float mb = m == -INFINITY ? 0.0f : m;
+          const uint64_t mm = f2_pack(-mb, -mb);
           uint64_t lsum0 = 0, lsum1 = 0;   // packed partial row sums (0.0f bits)
 #pragma unroll
           for (int c0 = 0; c0 < 128; c0 += 32) {
@@ -586,7 +629,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       const int valid_rows = qt == 0 ? min(kQTile, rows_left) : rows_left - kQTile;
       const bool row_valid = row < valid_rows;
       const int grow = q_row0 + qt * kQTile + row;
-      const float inv_l = n_tiles > 0 ? 1.0f / l : 0.0f;
+      const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
       const size_t row_elems = (static_cast<size_t>(grow) * PB.H + h) * D;
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {

@@ -277,10 +277,26 @@ static std::vector<GroupSpec> longest_first(const std::vector<GroupSpec> &groups
   return head;
 }
 
+// Causal plans interleave the units of this many heads pair by pair: as many
+// heads as have K and V (bf16, the distinct K/V rows of the group) within a
+// 64 MiB share of the 126 MB L2, at least one.
+static int causal_head_block(const GroupSpec &gs, int D, int H) {
+  std::vector<std::pair<int, int>> ranges;
+  for (const SegSpec &ss : gs.segs)
+    for (const AttnKV &kv : ss.kv) ranges.emplace_back(kv.row0, kv.nrows);
+  std::sort(ranges.begin(), ranges.end());
+  ranges.erase(std::unique(ranges.begin(), ranges.end()), ranges.end());
+  long long rows = 0;
+  for (const auto &r : ranges) rows += r.second;
+  const long long per_head = std::max(1LL, rows * D * 2 * 2);
+  const long long fit = (64LL << 20) / per_head;
+  return static_cast<int>(std::max(1LL, std::min<long long>(H, fit)));
+}
+
 // Packs the groups into as few launches as the parameter tables allow and
 // launches them in order on `stream`.
 static int run_attention(const std::vector<ProblemSpec> &probs, const std::vector<GroupSpec> &groups_in, int D,
-                         bool out_f32, cudaStream_t stream) {
+                         bool out_f32, bool causal, cudaStream_t stream) {
   const std::vector<GroupSpec> groups = longest_first(groups_in);
   std::vector<AttnProblem> encoded(probs.size());
   for (size_t i = 0; i < probs.size(); ++i) {
@@ -310,6 +326,7 @@ static int run_attention(const std::vector<ProblemSpec> &probs, const std::vecto
     n_prob = n_seg = n_kv = 0;
     open_group = -1;
     P->scale_log2 = scale_log2;
+    P->causal = causal ? 1 : 0;
     P->timeout_ns = wait_timeout_ns();
   };
   auto close_group = [&] {
@@ -357,6 +374,7 @@ static int run_attention(const std::vector<ProblemSpec> &probs, const std::vecto
         g.seg_count = 0;
         g.tiles_per_head = 0;
         g.unit_base = P->total_units;
+        g.head_block = causal_head_block(gs, D, probs[gs.prob].H);
         group_started_here = true;
       }
       AttnGroup &g = P->group[open_group];
@@ -394,17 +412,20 @@ static ProblemSpec full_problem(const void *q, const void *k, const void *v, voi
 }
 
 // Ring plan over a [rows, H, D] tensor whose batch-b chunk c occupies rows
-// row_of(b, c) .. + lens[c]; `step` < 0: all chunks in ring order (fused);
-// otherwise only chunk (r - step) mod P.
+// row_of(b, c) .. + lens[c] at sequence positions off[c] ..; `step` < 0: all
+// chunks in ring order (fused); otherwise only chunk (r - step) mod P.  Under
+// the causal mask a chunk after shard r is invisible to all of its queries
+// and is left out (its ring-step partial is the empty one: out 0, lse -inf).
 template <class RowOf>
 static void ring_groups(std::vector<GroupSpec> &groups, int prob, int B, const std::vector<int> &lens,
-                        const std::vector<int> &off, int step, RowOf row_of) {
+                        const std::vector<int> &off, int step, bool causal, RowOf row_of) {
   const int P = static_cast<int>(lens.size());
   for (int b = 0; b < B; ++b) {
     GroupSpec g;
     g.prob = prob;
     g.b = b;
-    for (int r = 0; r < P; ++r) {
+    for (int i = 0; i < P; ++i) {
+      const int r = causal ? P - 1 - i : i;   // causal: the shard that sees most chunks first
       SegSpec s;
       s.row0 = row_of(b, r);
       s.nrows = lens[r];
@@ -412,7 +433,8 @@ static void ring_groups(std::vector<GroupSpec> &groups, int prob, int B, const s
       for (int t = 0; t < P; ++t) {
         if (step >= 0 && t != step) continue;
         const int c = ((r - t) % P + P) % P;  // chunk held by rank r after t hand-offs
-        if (lens[c] > 0) s.kv.push_back(AttnKV{row_of(b, c), lens[c]});
+        if (causal && c > r) continue;
+        if (lens[c] > 0) s.kv.push_back(AttnKV{row_of(b, c), lens[c], off[c]});
       }
       g.segs.push_back(std::move(s));
     }
@@ -482,7 +504,7 @@ const char *cpattn_status_string(int status) {
   }
 }
 
-int cpattn_version(void) { return 1 * 10000 + 0 * 100 + 0; }
+int cpattn_version(void) { return 1 * 10000 + 1 * 100 + 0; }
 
 int cpattn_front_loaded_splits(int total, int parts, int *out) {
   if (out == nullptr) return CPATTN_ERR_NULL;
@@ -494,7 +516,8 @@ int cpattn_front_loaded_splits(int total, int parts, int *out) {
 }
 
 static int ring_common(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H, int S, int D,
-                       int ring_degree, const int *chunk_lens, int step, bool out_f32, cudaStream_t stream) {
+                       int ring_degree, const int *chunk_lens, int step, bool out_f32, bool causal,
+                       cudaStream_t stream) {
   if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return CPATTN_ERR_NULL;
   if (out_f32 && lse == nullptr) return CPATTN_ERR_NULL;
   int st = check_attn_shape(B, H, S, D);
@@ -511,20 +534,32 @@ static int ring_common(const void *q, const void *k, const void *v, void *out, f
   const std::vector<int> off = prefix(lens);
   std::vector<ProblemSpec> probs{full_problem(q, k, v, out, lse, B, H, S)};
   std::vector<GroupSpec> groups;
-  ring_groups(groups, 0, B, lens, off, step,
+  ring_groups(groups, 0, B, lens, off, step, causal,
               [&](int b, int c) { return b * S + off[c]; });
-  return run_attention(probs, groups, D, out_f32, stream);
+  return run_attention(probs, groups, D, out_f32, causal, stream);
 }
 
 int cpattn_ring_attention(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H, int S,
                           int D, int ring_degree, const int *chunk_lens, cpattn_stream_t stream) {
-  return ring_common(q, k, v, out, lse, B, H, S, D, ring_degree, chunk_lens, -1, false, stream);
+  return ring_common(q, k, v, out, lse, B, H, S, D, ring_degree, chunk_lens, -1, false, false, stream);
+}
+
+int cpattn_causal_ring_attention(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H,
+                                 int S, int D, int ring_degree, const int *chunk_lens, cpattn_stream_t stream) {
+  return ring_common(q, k, v, out, lse, B, H, S, D, ring_degree, chunk_lens, -1, false, true, stream);
 }
 
 int cpattn_ring_step(const void *q, const void *k, const void *v, float *part_out, float *part_lse, int B, int H,
                      int S, int D, int ring_degree, const int *chunk_lens, int step, cpattn_stream_t stream) {
   if (step < 0) return CPATTN_ERR_DEGREE;
-  return ring_common(q, k, v, part_out, part_lse, B, H, S, D, ring_degree, chunk_lens, step, true, stream);
+  return ring_common(q, k, v, part_out, part_lse, B, H, S, D, ring_degree, chunk_lens, step, true, false, stream);
+}
+
+int cpattn_causal_ring_step(const void *q, const void *k, const void *v, float *part_out, float *part_lse, int B,
+                            int H, int S, int D, int ring_degree, const int *chunk_lens, int step,
+                            cpattn_stream_t stream) {
+  if (step < 0) return CPATTN_ERR_DEGREE;
+  return ring_common(q, k, v, part_out, part_lse, B, H, S, D, ring_degree, chunk_lens, step, true, true, stream);
 }
 
 int cpattn_lse_merge(const float *part_out, const float *part_lse, int P, int B, int H, int S, int D, float *out_f32,
@@ -578,12 +613,12 @@ int cpattn_kv_gather_attention(const void *q, const void *k, const void *v, void
       s.row0 = b * S + off[r];
       s.nrows = lens[r];
       s.s0 = off[r];
-      s.kv.push_back(AttnKV{b * S, S});   // the gathered, full K/V of batch b
+      s.kv.push_back(AttnKV{b * S, S, 0});   // the gathered, full K/V of batch b
       g.segs.push_back(std::move(s));
     }
     groups.push_back(std::move(g));
   }
-  return run_attention(probs, groups, D, false, stream);
+  return run_attention(probs, groups, D, false, false, stream);
 }
 
 int cpattn_ulysses_permute(const void *x, void *y, int B, int S, int H, int D, int elem_bytes, int degree,
@@ -631,7 +666,8 @@ static void head_sharded_problems(std::vector<ProblemSpec> &probs, std::vector<i
 }
 
 static int head_sharded_attention_impl(const void *yq, const void *yk, const void *yv, void *yo, float *lse, int B,
-                                       int H, int S, int D, const std::vector<int> &heads, cudaStream_t stream) {
+                                       int H, int S, int D, const std::vector<int> &heads, bool causal,
+                                       cudaStream_t stream) {
   std::vector<ProblemSpec> probs;
   std::vector<int> prob_rank;
   head_sharded_problems(probs, prob_rank, yq, yk, yv, yo, lse, B, H, S, D, heads);
@@ -645,16 +681,16 @@ static int head_sharded_attention_impl(const void *yq, const void *yk, const voi
       s.row0 = b * S;
       s.nrows = S;
       s.s0 = 0;
-      s.kv.push_back(AttnKV{b * S, S});
+      s.kv.push_back(AttnKV{b * S, S, 0});
       g.segs.push_back(std::move(s));
       groups.push_back(std::move(g));
     }
   }
-  return run_attention(probs, groups, D, false, stream);
+  return run_attention(probs, groups, D, false, causal, stream);
 }
 
-int cpattn_head_sharded_attention(const void *yq, const void *yk, const void *yv, void *yo, float *lse, int B, int H,
-                                  int S, int D, int degree, const int *head_splits, cpattn_stream_t stream) {
+static int head_sharded_common(const void *yq, const void *yk, const void *yv, void *yo, float *lse, int B, int H,
+                               int S, int D, int degree, const int *head_splits, bool causal, cudaStream_t stream) {
   if (yq == nullptr || yk == nullptr || yv == nullptr || yo == nullptr) return CPATTN_ERR_NULL;
   int st = check_attn_shape(B, H, S, D);
   if (st != CPATTN_OK) return st;
@@ -666,7 +702,18 @@ int cpattn_head_sharded_attention(const void *yq, const void *yk, const void *yv
     return CPATTN_ERR_ALIGNMENT;
   st = check_device(nullptr);
   if (st != CPATTN_OK) return st;
-  return head_sharded_attention_impl(yq, yk, yv, yo, lse, B, H, S, D, heads, stream);
+  return head_sharded_attention_impl(yq, yk, yv, yo, lse, B, H, S, D, heads, causal, stream);
+}
+
+int cpattn_head_sharded_attention(const void *yq, const void *yk, const void *yv, void *yo, float *lse, int B, int H,
+                                  int S, int D, int degree, const int *head_splits, cpattn_stream_t stream) {
+  return head_sharded_common(yq, yk, yv, yo, lse, B, H, S, D, degree, head_splits, false, stream);
+}
+
+int cpattn_causal_head_sharded_attention(const void *yq, const void *yk, const void *yv, void *yo, float *lse, int B,
+                                         int H, int S, int D, int degree, const int *head_splits,
+                                         cpattn_stream_t stream) {
+  return head_sharded_common(yq, yk, yv, yo, lse, B, H, S, D, degree, head_splits, true, stream);
 }
 
 size_t cpattn_ulysses_workspace_bytes(int B, int H, int S, int D) {
@@ -676,9 +723,9 @@ size_t cpattn_ulysses_workspace_bytes(int B, int H, int S, int D) {
 
 size_t cpattn_unified_workspace_bytes(int B, int H, int S, int D) { return cpattn_ulysses_workspace_bytes(B, H, S, D); }
 
-int cpattn_ulysses_attention(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H, int S,
-                             int D, int degree, const int *seq_splits, const int *head_splits, void *workspace,
-                             size_t workspace_bytes, cpattn_stream_t stream) {
+static int ulysses_common(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H, int S,
+                          int D, int degree, const int *seq_splits, const int *head_splits, void *workspace,
+                          size_t workspace_bytes, bool causal, cudaStream_t stream) {
   if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return CPATTN_ERR_NULL;
   int st = check_attn_shape(B, H, S, D);
   if (st != CPATTN_OK) return st;
@@ -710,7 +757,7 @@ int cpattn_ulysses_attention(const void *q, const void *k, const void *v, void *
     if (launch_permute(pp, stream) != cudaSuccess) return CPATTN_ERR_CUDA;
   }
   // local attention of every head rank over all S tokens of its heads
-  st = head_sharded_attention_impl(yq, yk, yv, yo, lse, B, H, S, D, heads, stream);
+  st = head_sharded_attention_impl(yq, yk, yv, yo, lse, B, H, S, D, heads, causal, stream);
   if (st != CPATTN_OK) return st;
   // second all-to-all: the output back to the sequence-sharded layout
   PermuteParams po = pq;
@@ -720,10 +767,23 @@ int cpattn_ulysses_attention(const void *q, const void *k, const void *v, void *
   return launch_permute(po, stream) == cudaSuccess ? CPATTN_OK : CPATTN_ERR_CUDA;
 }
 
-int cpattn_unified_attention(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H, int S,
-                             int D, int ring_degree, int ulysses_degree, const int *ring_lens,
-                             const int *head_splits, void *workspace, size_t workspace_bytes,
-                             cpattn_stream_t stream) {
+int cpattn_ulysses_attention(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H, int S,
+                             int D, int degree, const int *seq_splits, const int *head_splits, void *workspace,
+                             size_t workspace_bytes, cpattn_stream_t stream) {
+  return ulysses_common(q, k, v, out, lse, B, H, S, D, degree, seq_splits, head_splits, workspace, workspace_bytes,
+                        false, stream);
+}
+
+int cpattn_causal_ulysses_attention(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H,
+                                    int S, int D, int degree, const int *seq_splits, const int *head_splits,
+                                    void *workspace, size_t workspace_bytes, cpattn_stream_t stream) {
+  return ulysses_common(q, k, v, out, lse, B, H, S, D, degree, seq_splits, head_splits, workspace, workspace_bytes,
+                        true, stream);
+}
+
+static int unified_common(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H, int S,
+                          int D, int ring_degree, int ulysses_degree, const int *ring_lens, const int *head_splits,
+                          void *workspace, size_t workspace_bytes, bool causal, cudaStream_t stream) {
   if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return CPATTN_ERR_NULL;
   int st = check_attn_shape(B, H, S, D);
   if (st != CPATTN_OK) return st;
@@ -775,15 +835,31 @@ int cpattn_unified_attention(const void *q, const void *k, const void *v, void *
   head_sharded_problems(probs, prob_rank, yq, yk, yv, yo, lse, B, H, S, D, heads);
   std::vector<GroupSpec> groups;
   for (size_t pi = 0; pi < probs.size(); ++pi)
-    ring_groups(groups, static_cast<int>(pi), B, lens, off, -1,
+    ring_groups(groups, static_cast<int>(pi), B, lens, off, -1, causal,
                 [&](int b, int c) { return B * off[c] + b * lens[c]; });
-  st = run_attention(probs, groups, D, false, stream);
+  st = run_attention(probs, groups, D, false, causal, stream);
   if (st != CPATTN_OK) return st;
   PermuteParams p2 = pp;
   p2.src = static_cast<const unsigned char *>(yo);
   p2.dst = static_cast<unsigned char *>(out);
   p2.direction = 1;
   return launch_permute(p2, stream) == cudaSuccess ? CPATTN_OK : CPATTN_ERR_CUDA;
+}
+
+int cpattn_unified_attention(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H, int S,
+                             int D, int ring_degree, int ulysses_degree, const int *ring_lens,
+                             const int *head_splits, void *workspace, size_t workspace_bytes,
+                             cpattn_stream_t stream) {
+  return unified_common(q, k, v, out, lse, B, H, S, D, ring_degree, ulysses_degree, ring_lens, head_splits, workspace,
+                        workspace_bytes, false, stream);
+}
+
+int cpattn_causal_unified_attention(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H,
+                                    int S, int D, int ring_degree, int ulysses_degree, const int *ring_lens,
+                                    const int *head_splits, void *workspace, size_t workspace_bytes,
+                                    cpattn_stream_t stream) {
+  return unified_common(q, k, v, out, lse, B, H, S, D, ring_degree, ulysses_degree, ring_lens, head_splits, workspace,
+                        workspace_bytes, true, stream);
 }
 
 int cpattn_exchange_bytes(int mode, int B, int H, int S, int D, int elem_bytes, int degree, const int *seq_splits,

@@ -22,6 +22,9 @@ namespace cpattn {
 //   segment : a range of Q rows (one sequence shard) with its list of K/V
 //             row ranges, visited in order (ring order for ring attention),
 //   kv      : a K/V row range (one chunk).
+// Segments and K/V ranges carry the sequence position of their first row; a
+// causal plan masks by positions (no mask tensor), and a unit never walks a
+// K/V tile that lies wholly after its last query.
 // One CTA processes one unit = (group, head, segment, pair of 128-row Q tiles).
 
 constexpr int kMaxProblems = 8;
@@ -49,6 +52,7 @@ struct AttnGroup {
   int seg_count;
   int tiles_per_head;   // sum over the group's segments of their CTA tile pairs
   int unit_base;        // first unit (blockIdx) of this group
+  int head_block;       // causal plans: heads whose units interleave pair by pair
 };
 
 struct AttnSeg {
@@ -64,6 +68,7 @@ struct AttnSeg {
 struct AttnKV {
   int row0;
   int nrows;
+  int s0;         // sequence position of row0 (for the causal mask)
 };
 
 struct AttnParams {
@@ -73,6 +78,7 @@ struct AttnParams {
   AttnKV kv[kMaxKV];
   int num_groups;
   int total_units;
+  int causal;                    // 1: key visible to a query iff its position <= the query's
   float scale_log2;              // D**-0.5 * log2(e)
   unsigned long long timeout_ns; // bound for every pipeline wait
 };

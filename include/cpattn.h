@@ -9,7 +9,8 @@
  *   [SP]  SGLang Diffusion docs, "Sequence Parallelism": "Choosing The
  *         Attention Exchange"; "Numerics across node boundaries".
  *   [USP] "Ulysses Sequence Parallelism: training with million-token
- *         contexts": sections 3 (core idea), 4 (steps), 5 (communication).
+ *         contexts": sections 3 (core idea), 4 (steps), 5 (communication),
+ *         7 (causal masking by position ids).
  *   [API] diffusers docs, "parallel": ContextParallelConfig parameters
  *         ring_degree, ulysses_degree, convert_to_fp32, rotate_method,
  *         ulysses_anything, ring_anything.
@@ -21,7 +22,8 @@
  * Tensors.  Q, K, V and attention outputs are bf16, (batch B, seq S, heads H,
  *   head_dim D) contiguous ("BSHD", [PR]).  D must be 64 or 128.  Softmax
  *   scale is D**-0.5 ([PR]).  Attention is non-causal with no mask ([SP]
- *   kv_gather constraint; [CP] Ring Anything requires attn_mask None).
+ *   kv_gather constraint; [CP] Ring Anything requires attn_mask None), except
+ *   in the cpattn_causal_* entry points (section "causal" below).
  *   LSE outputs are float32, natural log, layout (B, H, S).
  * Shards.  A "sequence shard" r of a full BSHD tensor is rows off_r ..
  *   off_r + len_r - 1 of every batch element, with off_r the prefix sum of the
@@ -238,6 +240,51 @@ int cpattn_unified_attention(const void *q, const void *k, const void *v, void *
                              int B, int H, int S, int D, int ring_degree, int ulysses_degree,
                              const int *ring_lens, const int *head_splits, void *workspace,
                              size_t workspace_bytes, cpattn_stream_t stream);
+
+/* ---------------------------------------------------------------- causal */
+
+/*
+ * Causal variants ([USP] section 7: for causal masking over long sequences,
+ * Ulysses and ring attention use position ids instead of an attention-mask
+ * tensor).  Every token's position is its index s in the full sequence; key
+ * j is visible to query i iff j <= i.  No mask tensor exists: the kernel
+ * derives the mask from the positions of the row ranges it walks, skips every
+ * K/V tile that lies wholly after a Q tile's last query, and masks inside the
+ * tiles that straddle the diagonal.  The kv_gather exchange has no causal
+ * variant ([SP] "Choosing The Attention Exchange": kv_gather is non-causal).
+ *
+ * Each function takes exactly the arguments, layouts, ownership and error
+ * behaviour of its non-causal namesake:
+ *   cpattn_causal_ring_attention        as cpattn_ring_attention.  In ring
+ *       order rank r walks c = r, r-1, ..., 0; chunks after shard r are
+ *       invisible to all of its queries and are not visited.
+ *   cpattn_causal_ring_step             as cpattn_ring_step.  A step whose
+ *       chunk lies after shard r writes out = 0 and LSE = -inf for its rows
+ *       (the neutral partial), so cpattn_lse_merge of all steps equals
+ *       cpattn_causal_ring_attention.
+ *   cpattn_causal_head_sharded_attention as cpattn_head_sharded_attention
+ *       (positions 0 .. S-1 in every head-side buffer).
+ *   cpattn_causal_ulysses_attention     as cpattn_ulysses_attention.
+ *   cpattn_causal_unified_attention     as cpattn_unified_attention (ring
+ *       chunk i holds positions off_i .. off_i + len_i - 1).
+ */
+int cpattn_causal_ring_attention(const void *q, const void *k, const void *v, void *out, float *lse,
+                                 int B, int H, int S, int D, int ring_degree,
+                                 const int *chunk_lens, cpattn_stream_t stream);
+int cpattn_causal_ring_step(const void *q, const void *k, const void *v, float *part_out,
+                            float *part_lse, int B, int H, int S, int D, int ring_degree,
+                            const int *chunk_lens, int step, cpattn_stream_t stream);
+int cpattn_causal_head_sharded_attention(const void *yq, const void *yk, const void *yv, void *yo,
+                                         float *lse, int B, int H, int S, int D, int degree,
+                                         const int *head_splits, cpattn_stream_t stream);
+int cpattn_causal_ulysses_attention(const void *q, const void *k, const void *v, void *out,
+                                    float *lse, int B, int H, int S, int D, int degree,
+                                    const int *seq_splits, const int *head_splits, void *workspace,
+                                    size_t workspace_bytes, cpattn_stream_t stream);
+int cpattn_causal_unified_attention(const void *q, const void *k, const void *v, void *out,
+                                    float *lse, int B, int H, int S, int D, int ring_degree,
+                                    int ulysses_degree, const int *ring_lens, const int *head_splits,
+                                    void *workspace, size_t workspace_bytes, cpattn_stream_t stream);
 
 /* ------------------------------------------------- no-allocation variant */
 

@@ -150,3 +150,26 @@ def test_valid_call_without_gpu_reports_cuda_error(lib):
     # Arguments pass validation; with no device the call must return
     # CPATTN_ERR_CUDA before launching anything.
     assert _ring(lib) == CUDA
+
+
+def test_causal_entry_points_validate_like_their_namesakes(lib):
+    r = lambda q=FAKE, S=256, P=4, lens=None: lib.cpattn_causal_ring_attention(q, FAKE, FAKE, FAKE, FAKE, 1, 2, S, 64,
+                                                                              P, _native.int_array(lens), None)
+    assert r(q=None) == NULL
+    assert r(S=10, P=3) == INDIV
+    assert r(S=10, P=3, lens=[3, 3, 3]) == SPLITS
+    assert r(q=FAKE_MIS) == ALIGN
+    st = lambda step, lse=FAKE: lib.cpattn_causal_ring_step(FAKE, FAKE, FAKE, FAKE, lse, 1, 2, 256, 64, 4, None,
+                                                             step, None)
+    assert st(-1) == DEGREE and st(4) == DEGREE and st(0, lse=None) == NULL
+    h = lambda H=4: lib.cpattn_causal_head_sharded_attention(FAKE, FAKE, FAKE, FAKE, FAKE, 1, H, 8, 64, 2, None, None)
+    assert h(H=5) == INDIV
+    need = lib.cpattn_ulysses_workspace_bytes(1, 4, 8, 64)
+    u = lambda ws=FAKE, H=4: lib.cpattn_causal_ulysses_attention(FAKE, FAKE, FAKE, FAKE, FAKE, 1, H, 8, 64, 2, None,
+                                                                 None, ws, need, None)
+    assert u(ws=None) == WS and u(H=5) == INDIV
+    v = lambda ws=FAKE, R=2: lib.cpattn_causal_unified_attention(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 4, 8, 64, R, 2,
+                                                                 None, None, ws, need, None)
+    assert v(ws=None) == WS and v(R=3) == INDIV
+    if not torch.cuda.is_available():
+        assert r() == CUDA       # valid arguments, no device: fails before any launch
