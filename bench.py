@@ -35,6 +35,9 @@ METRIC = "attention TFLOP/s (4·B·H·S²·D) & % BF16 peak; permute/merge GB/s 
 WORKLOAD = "dit"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
+# Measured NVLink peer copy of this machine's B200s, GB/s per direction (input of
+# the exchange-selection model only; no collective runs here).
+NVLINK_PEER_GBS = 770.0
 
 
 def load_peaks():
@@ -397,6 +400,19 @@ def main():
         snd, rcv = api.cpattn_exchange_bytes(mode, B, H, S, D, deg)
         exch[f"{mode}_{deg}"] = {"send": snd[0], "recv": rcv[0]}
     exch["kv_gather_over_ulysses"] = exch[f"kv_gather_{P}"]["recv"] / max(1, exch[f"ulysses_{U}"]["recv"])
+    # The exchange-selection model fed with this run's measured attention
+    # throughput, the measured HBM bandwidth and the measured NVLink peer-copy
+    # bandwidth of this machine's B200s (770 GB/s per direction).
+    exch_plan = {"inputs": {"link_gbs": NVLINK_PEER_GBS, "attn_tflops": round(ring_tflops, 1),
+                            "hbm_gbs": float(peaks["hbm_gbs"])}}
+    for deg in (2, 4, 8):
+        for causal in (False, True):
+            pl = api.cpattn_plan_exchange(B, H, S, D, deg, NVLINK_PEER_GBS, ring_tflops, float(peaks["hbm_gbs"]),
+                                          causal=causal)
+            exch_plan[f"P{deg}" + ("_causal" if causal else "")] = {
+                "best": pl["best"],
+                "us": {m: (None if pl[m]["seconds"] is None else round(pl[m]["seconds"] * 1e6, 1))
+                       for m in ("ring", "ulysses", "kv_gather")}}
 
     st, code = api.cpattn_device_status()
     line = {
@@ -405,7 +421,7 @@ def main():
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1), RMS-normalised Q/K, bf16)",
         "config": config_block(cfg), "roofline": roofline, "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks.summary(t_wall0, t_wall1), "e2e": e2e, "kernels": kernels,
-        "device_status": code, "exchange_bytes_per_rank": exch,
+        "device_status": code, "exchange_bytes_per_rank": exch, "exchange_plan": exch_plan,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, qb, kb, vb)

@@ -56,6 +56,8 @@ SIGNATURES = {
     "cpattn_front_loaded_splits": (c_int, [c_int, c_int, P_INT]),
     "cpattn_exchange_bytes": (c_int, [c_int, c_int, c_int, c_int, c_int, c_int, c_int, P_INT, P_INT,
                                       ctypes.POINTER(ctypes.c_ulonglong), ctypes.POINTER(ctypes.c_ulonglong)]),
+    "cpattn_plan_exchange": (c_int, [c_int, c_int, c_int, c_int, c_int, c_int, P_INT, P_INT,
+                                     ctypes.c_void_p, ctypes.c_void_p]),
     "cpattn_device_status": (c_int, [c_void_p, P_UINT]),
     "cpattn_debug_wait_timeout": (c_int, [c_uint, c_void_p]),
 }

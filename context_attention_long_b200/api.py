@@ -294,6 +294,35 @@ def cpattn_exchange_bytes(mode, B, H, S, D, degree, seq_splits=None, head_splits
     return [int(x) for x in send], [int(x) for x in recv]
 
 
+class _ExchangeEnv(ctypes.Structure):
+    _fields_ = [("link_gbs", ctypes.c_double), ("attn_tflops", ctypes.c_double), ("hbm_gbs", ctypes.c_double),
+                ("causal", ctypes.c_int)]
+
+
+class _ExchangePlan(ctypes.Structure):
+    _fields_ = [("seconds", ctypes.c_double * 3), ("recv_bytes", ctypes.c_ulonglong * 3),
+                ("resident_bytes", ctypes.c_ulonglong * 3), ("flops", ctypes.c_double * 3), ("best", ctypes.c_int)]
+
+
+def cpattn_plan_exchange(B, H, S, D, degree, link_gbs, attn_tflops, hbm_gbs, causal=False, seq_splits=None,
+                         head_splits=None, elem_bytes=2):
+    """Exchange-selection model for one attention call over `degree` ranks.
+    Returns {"best": mode name, mode name: {"seconds" (None if infeasible),
+    "recv_bytes", "resident_bytes", "flops"}}; host arithmetic only."""
+    env = _ExchangeEnv(float(link_gbs), float(attn_tflops), float(hbm_gbs), 1 if causal else 0)
+    plan = _ExchangePlan()
+    _check(_native.load().cpattn_plan_exchange(B, H, S, D, elem_bytes, int(degree), _native.int_array(seq_splits),
+                                               _native.int_array(head_splits), ctypes.byref(env),
+                                               ctypes.byref(plan)), "cpattn_plan_exchange")
+    names = {v: k for k, v in EXCHANGE_MODES.items()}
+    out = {"best": names[plan.best]}
+    for m, name in names.items():
+        out[name] = {"seconds": None if plan.seconds[m] < 0 else float(plan.seconds[m]),
+                     "recv_bytes": int(plan.recv_bytes[m]), "resident_bytes": int(plan.resident_bytes[m]),
+                     "flops": float(plan.flops[m])}
+    return out
+
+
 def cpattn_device_status(stream=None):
     """Synchronise the stream and read-and-clear the device status word.
     Returns (status, code)."""

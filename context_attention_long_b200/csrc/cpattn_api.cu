@@ -890,6 +890,96 @@ int cpattn_exchange_bytes(int mode, int B, int H, int S, int D, int elem_bytes, 
   return CPATTN_OK;
 }
 
+// (query, key) pairs of queries at positions q0 .. q0+nq-1 and keys at
+// k0 .. k0+nk-1 that attention sees: all of them, or under the causal mask
+// those with key position <= query position.
+static double visible_pairs(long long q0, long long nq, long long k0, long long nk, bool causal) {
+  if (nq <= 0 || nk <= 0) return 0.0;
+  if (!causal) return static_cast<double>(nq) * static_cast<double>(nk);
+  // query i sees clamp(i - k0 + 1, 0, nk) keys; sum it in closed form over
+  // the three stretches (none, a growing run, all nk)
+  double total = 0.0;
+  const long long q1 = q0 + nq;                       // exclusive
+  const long long a = std::max(q0, k0);               // first query that sees a key
+  const long long b = std::min(q1, k0 + nk - 1);      // first query that sees all nk
+  if (a < b) {
+    const double first = static_cast<double>(a - k0 + 1), last = static_cast<double>(b - 1 - k0 + 1);
+    total += (first + last) * static_cast<double>(b - a) / 2.0;
+  }
+  const long long full_from = std::max(q0, k0 + nk - 1);
+  if (q1 > full_from) total += static_cast<double>(q1 - full_from) * static_cast<double>(nk);
+  return total;
+}
+
+int cpattn_plan_exchange(int B, int H, int S, int D, int elem_bytes, int degree, const int *seq_splits,
+                         const int *head_splits, const cpattn_exchange_env *env, cpattn_exchange_plan *plan) {
+  if (env == nullptr || plan == nullptr) return CPATTN_ERR_NULL;
+  if (B < 1 || H < 1 || S < 1 || D < 1 || elem_bytes < 1) return CPATTN_ERR_SHAPE;
+  if (!(env->link_gbs > 0.0) || !(env->attn_tflops > 0.0) || !(env->hbm_gbs > 0.0)) return CPATTN_ERR_SHAPE;
+  if (degree < 1 || degree > kMaxRanks) return CPATTN_ERR_DEGREE;
+  std::vector<int> seq, heads;
+  int st = resolve_splits(S, degree, seq_splits, seq);
+  if (st != CPATTN_OK) return st;
+  const bool ulysses_ok = resolve_splits(H, degree, head_splits, heads) == CPATTN_OK;
+  if (!ulysses_ok && head_splits != nullptr) return resolve_splits(H, degree, head_splits, heads);
+  const bool causal = env->causal != 0;
+  const std::vector<int> off = prefix(seq);
+  std::vector<unsigned long long> snd(degree), rcv_ring(degree), rcv_uly(degree);
+  st = cpattn_exchange_bytes(0, B, H, S, D, elem_bytes, degree, seq_splits, nullptr, snd.data(), rcv_ring.data());
+  if (st != CPATTN_OK) return st;
+  if (ulysses_ok) {
+    st = cpattn_exchange_bytes(1, B, H, S, D, elem_bytes, degree, seq_splits, head_splits, snd.data(),
+                               rcv_uly.data());
+    if (st != CPATTN_OK) return st;
+  }
+  const double link = env->link_gbs * 1e9, flops_s = env->attn_tflops * 1e12, hbm = env->hbm_gbs * 1e9;
+  const double row = static_cast<double>(D) * elem_bytes;          // bytes of one (token, head)
+  const double pair_flops = 4.0 * D * B;                           // per (query, key, head)
+  std::memset(plan, 0, sizeof(*plan));
+  for (int m = 0; m < 3; ++m) plan->seconds[m] = 0.0;
+  int max_chunk = 0;
+  for (int c = 0; c < degree; ++c) max_chunk = std::max(max_chunk, seq[c]);
+  for (int r = 0; r < degree; ++r) {
+    // ring (and kv_gather, which attends to the same chunks)
+    double t_ring = 0.0, f_all = 0.0;
+    for (int t = 0; t < degree; ++t) {
+      const int c = ((r - t) % degree + degree) % degree;
+      const double f = pair_flops * H * visible_pairs(off[r], seq[r], off[c], seq[c], causal);
+      const double a = f / flops_s;
+      f_all += f;
+      if (t == 0) t_ring += a;
+      else t_ring += std::max(a, 2.0 * B * static_cast<double>(seq[c]) * H * row / link);
+    }
+    plan->seconds[0] = std::max(plan->seconds[0], t_ring);
+    plan->flops[0] = std::max(plan->flops[0], f_all);
+    plan->recv_bytes[0] = std::max(plan->recv_bytes[0], rcv_ring[r]);
+    plan->resident_bytes[0] = std::max(plan->resident_bytes[0],
+        static_cast<unsigned long long>((2.0 * seq[r] + 4.0 * max_chunk) * B * H * row));
+    if (!causal) {
+      plan->seconds[2] = std::max(plan->seconds[2], static_cast<double>(rcv_ring[r]) / link + f_all / flops_s);
+      plan->flops[2] = std::max(plan->flops[2], f_all);
+      plan->recv_bytes[2] = std::max(plan->recv_bytes[2], rcv_ring[r]);
+      plan->resident_bytes[2] = std::max(plan->resident_bytes[2],
+          static_cast<unsigned long long>((2.0 * seq[r] + 2.0 * S) * B * H * row));
+    }
+    if (ulysses_ok) {
+      const double f = pair_flops * heads[r] * visible_pairs(0, S, 0, S, causal);
+      const double t_u = static_cast<double>(rcv_uly[r]) / link + 8.0 * B * seq[r] * H * row / hbm + f / flops_s;
+      plan->seconds[1] = std::max(plan->seconds[1], t_u);
+      plan->flops[1] = std::max(plan->flops[1], f);
+      plan->recv_bytes[1] = std::max(plan->recv_bytes[1], rcv_uly[r]);
+      plan->resident_bytes[1] = std::max(plan->resident_bytes[1],
+          static_cast<unsigned long long>(4.0 * B * S * heads[r] * row));
+    }
+  }
+  if (!ulysses_ok) plan->seconds[1] = -1.0;
+  if (causal) plan->seconds[2] = -1.0;
+  plan->best = 0;
+  for (int m = 1; m < 3; ++m)
+    if (plan->seconds[m] >= 0.0 && plan->seconds[m] < plan->seconds[plan->best]) plan->best = m;
+  return CPATTN_OK;
+}
+
 int cpattn_device_status(cpattn_stream_t stream, unsigned int *code) {
   if (code == nullptr) return CPATTN_ERR_NULL;
   int st = check_device(nullptr);

@@ -359,6 +359,63 @@ int cpattn_exchange_bytes(int mode, int B, int H, int S, int D, int elem_bytes, 
                           unsigned long long *recv);
 
 /*
+ * Exchange-selection model: which exchange serves one attention call over P
+ * ranks fastest, from the shapes and the measured speeds of the machine.
+ * [SP] "Choosing The Attention Exchange": neither exchange is universally
+ * faster; kv_gather moves about P/2 times the Ulysses payload but skips the
+ * inverse all-to-all and keeps the local attention layout, Ulysses holds less
+ * attention activation memory, and kv_gather is non-causal only.  [USP]
+ * section 5: ring moves O(n*d) per GPU over P-1 sequential hops, Ulysses
+ * O(n*d/P) in all-to-alls.  [SP] "Cross-Node Sequence Parallelism": the ring's
+ * point-to-point K/V rotation is pipelined against attention compute.
+ * Host-only arithmetic; nothing runs on the GPU.
+ *
+ * For every rank r the model charges (times in seconds, e = elem_bytes):
+ *   ring      T = A(r, r) + sum over the P-1 later chunks c in ring order of
+ *                 max(A(r, c), 2*B*S_c*H*D*e / link)
+ *   ulysses   T = recv_r / link + 8*B*S_r*H*D*e / hbm + A_heads(r)
+ *             (one local read+write pass over the Q, K, V and O shards)
+ *   kv_gather T = recv_r / link + sum over c of A(r, c)        (no overlap)
+ * where A(r, c) = 4*D*B*H*(query, key) pairs of shard r and chunk c that the
+ * mask lets through / attn_flops, A_heads(r) the same for H_r heads over all
+ * S tokens, recv_r the bytes of cpattn_exchange_bytes.  A mode's time is that
+ * of its slowest rank.  Resident bytes: what a rank holds during attention
+ *   ring      (2*S_r + 4*max_c S_c) * B*H*D*e  (Q, O, two K/V chunks in flight)
+ *   ulysses   4 * B*S*H_r*D*e                  (Q, K, V, O of its heads)
+ *   kv_gather (2*S_r + 2*S) * B*H*D*e          (Q, O, the full K and V)
+ *
+ *   env->link_gbs     interconnect bandwidth one rank receives at, GB/s (> 0)
+ *   env->attn_tflops  attention throughput of one GPU, TFLOP/s (> 0)
+ *   env->hbm_gbs      HBM bandwidth of one GPU, GB/s (> 0)
+ *   env->causal       1: causal (kv_gather infeasible), 0: non-causal
+ *   plan              written: per mode (0 ring, 1 Ulysses, 2 kv_gather) the
+ *                     time (-1 if infeasible), max recv bytes, max resident
+ *                     bytes and max attention FLOPs over ranks; best = the
+ *                     feasible mode with the least time.
+ * Ulysses is infeasible when head_splits is NULL and H % degree != 0.
+ * Errors: NULL, SHAPE (a size or an env value out of range), DEGREE,
+ * INDIVISIBLE (sequence), SPLITS.
+ */
+typedef struct {
+  double link_gbs;
+  double attn_tflops;
+  double hbm_gbs;
+  int causal;
+} cpattn_exchange_env;
+
+typedef struct {
+  double seconds[3];
+  unsigned long long recv_bytes[3];
+  unsigned long long resident_bytes[3];
+  double flops[3];
+  int best;
+} cpattn_exchange_plan;
+
+int cpattn_plan_exchange(int B, int H, int S, int D, int elem_bytes, int degree,
+                         const int *seq_splits, const int *head_splits,
+                         const cpattn_exchange_env *env, cpattn_exchange_plan *plan);
+
+/*
  * Synchronises `stream`, then reads and clears the device status word that the
  * kernels' bounded waits set when a pipeline wait expires.  *code receives the
  * raw word (0 = healthy; otherwise a bit per wait site).  Returns CPATTN_OK,
