@@ -244,7 +244,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true",
                     help="time every workload's paths (one JSON line per path) instead of the step")
-    ap.add_argument("--kernel", default=None, choices=["ring", "causal_ring", "head_sharded", "permute", "merge", "ring_step"],
+    ap.add_argument("--kernel", default=None, choices=["ring", "causal_ring", "head_sharded", "permute", "permute_qkv", "merge", "ring_step"],
                     help="profiling mode: run only this kernel (warmup + steps launches) on the workload")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -296,24 +296,20 @@ def main():
 
     attn_flops = 4.0 * B * H * S * S * D      # one attention pass
     step_flops = 2 * attn_flops               # ring + Ulysses
-    launches_per_step = 6                     # ring, 3 permutes, head-sharded attention, unpermute
-    n_ev = 7
+    launches_per_step = 4                     # ring, Q/K/V permute, head-sharded attention, unpermute
+    n_ev = 5
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
 
     def step(e=None):
         if e: e[0].record(stream)
         api.cpattn_ring_attention(q, k, v, P, out=out_r, lse=lse_r, stream=stream)
         if e: e[1].record(stream)
-        api.cpattn_ulysses_permute(qf, B, S, H, D, U, y=yq, stream=stream)
+        api.cpattn_ulysses_permute_qkv(qf, kf, vf, B, S, H, D, U, yq=yq, yk=yk, yv=yv, stream=stream)
         if e: e[2].record(stream)
-        api.cpattn_ulysses_permute(kf, B, S, H, D, U, y=yk, stream=stream)
-        if e: e[3].record(stream)
-        api.cpattn_ulysses_permute(vf, B, S, H, D, U, y=yv, stream=stream)
-        if e: e[4].record(stream)
         api.cpattn_head_sharded_attention(yq, yk, yv, B, S, H, D, U, yo=yo, lse=lse_u, stream=stream)
-        if e: e[5].record(stream)
+        if e: e[3].record(stream)
         api.cpattn_ulysses_unpermute(yo, B, S, H, D, U, x=out_u, stream=stream)
-        if e: e[6].record(stream)
+        if e: e[4].record(stream)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -347,9 +343,9 @@ def main():
     peaks, peaks_kind = load_peaks()
     ring_ms = float(per[:, 0].mean())
     ring_tflops = attn_flops / (ring_ms * 1e-3) / 1e12
-    uattn_ms = float(per[:, 4].mean())
-    perm_ms = float(per[:, 1:4].mean())
-    unperm_ms = float(per[:, 5].mean())
+    uattn_ms = float(per[:, 2].mean())
+    perm_ms = float(per[:, 1].mean())        # Q, K and V in one launch
+    unperm_ms = float(per[:, 3].mean())
     tensor_bytes = B * S * H * D * 2
     peak_tf = float(peaks["bf16_tflops"])
     roofline = {"bound": "tensor", "kernel": "attn_fwd_kernel<128,bf16> (ring fused, P=4)",
@@ -386,7 +382,7 @@ def main():
         "ring_fused_attention": {"ms": ring_ms, "TFLOP/s": ring_tflops, "frac_bf16_peak": ring_tflops / peak_tf},
         "head_sharded_attention": {"ms": uattn_ms, "TFLOP/s": attn_flops / (uattn_ms * 1e-3) / 1e12,
                                    "frac_bf16_peak": attn_flops / (uattn_ms * 1e-3) / 1e12 / peak_tf},
-        "ulysses_permute_dit": {"ms": perm_ms, "GB/s": 2 * tensor_bytes / (perm_ms * 1e-3) / 1e9},
+        "ulysses_permute_qkv_dit": {"ms": perm_ms, "GB/s": 6 * tensor_bytes / (perm_ms * 1e-3) / 1e9},
         "ulysses_unpermute_dit": {"ms": unperm_ms, "GB/s": 2 * tensor_bytes / (unperm_ms * 1e-3) / 1e9},
     }
     if not args.no_breakdown:
@@ -629,6 +625,10 @@ def run_single_kernel(args):
     elif args.kernel == "head_sharded":
         yq, yk, yv = (api.cpattn_ulysses_permute(t.reshape(-1), B, S, H, D, U) for t in (q, k, v))
         fn = lambda: api.cpattn_head_sharded_attention(yq, yk, yv, B, S, H, D, U)
+    elif args.kernel == "permute_qkv":
+        qf, kf, vf = q.reshape(-1), k.reshape(-1), v.reshape(-1)
+        yq, yk, yv = torch.empty_like(qf), torch.empty_like(kf), torch.empty_like(vf)
+        fn = lambda: api.cpattn_ulysses_permute_qkv(qf, kf, vf, B, S, H, D, U, yq=yq, yk=yk, yv=yv)
     elif args.kernel == "permute":
         fn = lambda: api.cpattn_ulysses_permute(q.reshape(-1), B, S, H, D, U)
     else:

@@ -27,6 +27,8 @@ SIGNATURES = {
                                            c_int, c_int, c_int, c_int, c_int, P_INT, c_void_p]),
     "cpattn_ulysses_permute": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
                                        P_INT, P_INT, c_void_p]),
+    "cpattn_ulysses_permute_qkv": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                           c_int, c_int, c_int, c_int, c_int, c_int, P_INT, P_INT, c_void_p]),
     "cpattn_ulysses_unpermute": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
                                          P_INT, P_INT, c_void_p]),
     "cpattn_head_sharded_attention": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,

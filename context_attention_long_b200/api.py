@@ -149,6 +149,19 @@ def cpattn_ulysses_permute(x, B, S, H, D, degree, seq_splits=None, head_splits=N
     return y
 
 
+def cpattn_ulysses_permute_qkv(q, k, v, B, S, H, D, degree, seq_splits=None, head_splits=None, yq=None, yk=None,
+                               yv=None, stream=None):
+    """The Q, K and V permutes of the first all-to-all in one launch; returns (yq, yk, yv)."""
+    yq = torch.empty_like(q) if yq is None else yq
+    yk = torch.empty_like(k) if yk is None else yk
+    yv = torch.empty_like(v) if yv is None else yv
+    _check(_native.load().cpattn_ulysses_permute_qkv(_ptr(q), _ptr(k), _ptr(v), _ptr(yq), _ptr(yk), _ptr(yv), B, S,
+                                                     H, D, q.element_size(), int(degree),
+                                                     _native.int_array(seq_splits), _native.int_array(head_splits),
+                                                     _stream(stream)), "cpattn_ulysses_permute_qkv")
+    return yq, yk, yv
+
+
 def cpattn_ulysses_unpermute(y, B, S, H, D, degree, seq_splits=None, head_splits=None, x=None, stream=None):
     """Head-sharded rank buffers -> sequence-sharded rank buffers (inverse permute)."""
     if x is None:

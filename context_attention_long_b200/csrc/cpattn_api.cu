@@ -442,6 +442,17 @@ static void ring_groups(std::vector<GroupSpec> &groups, int prob, int B, const s
   }
 }
 
+// Q, K and V (same shape and splits) as the three tensors of one permute launch.
+static void set_qkv(PermuteParams &pp, const void *q, const void *k, const void *v, void *yq, void *yk, void *yv) {
+  const void *srcs[3] = {q, k, v};
+  void *dsts[3] = {yq, yk, yv};
+  for (int i = 0; i < 3; ++i) {
+    pp.src[i] = static_cast<const unsigned char *>(srcs[i]);
+    pp.dst[i] = static_cast<unsigned char *>(dsts[i]);
+  }
+  pp.n_tensors = 3;
+}
+
 static int permute_common(const void *src, void *dst, int B, int S, int H, int D, int elem_bytes, int degree,
                           const int *seq_splits, const int *head_splits, int direction, PermuteParams &pp) {
   if (src == nullptr || dst == nullptr) return CPATTN_ERR_NULL;
@@ -458,8 +469,9 @@ static int permute_common(const void *src, void *dst, int B, int S, int H, int D
   if (st != CPATTN_OK) return st;
   if (!aligned16(src) || !aligned16(dst)) return CPATTN_ERR_ALIGNMENT;
   std::memset(&pp, 0, sizeof(pp));
-  pp.src = static_cast<const unsigned char *>(src);
-  pp.dst = static_cast<unsigned char *>(dst);
+  pp.src[0] = static_cast<const unsigned char *>(src);
+  pp.dst[0] = static_cast<unsigned char *>(dst);
+  pp.n_tensors = 1;
   pp.B = B;
   pp.S = S;
   pp.H = H;
@@ -631,6 +643,20 @@ int cpattn_ulysses_permute(const void *x, void *y, int B, int S, int H, int D, i
   return launch_permute(pp, stream) == cudaSuccess ? CPATTN_OK : CPATTN_ERR_CUDA;
 }
 
+int cpattn_ulysses_permute_qkv(const void *q, const void *k, const void *v, void *yq, void *yk, void *yv, int B,
+                               int S, int H, int D, int elem_bytes, int degree, const int *seq_splits,
+                               const int *head_splits, cpattn_stream_t stream) {
+  PermuteParams pp;
+  int st = permute_common(q, yq, B, S, H, D, elem_bytes, degree, seq_splits, head_splits, 0, pp);
+  if (st != CPATTN_OK) return st;
+  if (k == nullptr || v == nullptr || yk == nullptr || yv == nullptr) return CPATTN_ERR_NULL;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(yk) || !aligned16(yv)) return CPATTN_ERR_ALIGNMENT;
+  st = check_device(nullptr);
+  if (st != CPATTN_OK) return st;
+  set_qkv(pp, q, k, v, yq, yk, yv);
+  return launch_permute(pp, stream) == cudaSuccess ? CPATTN_OK : CPATTN_ERR_CUDA;
+}
+
 int cpattn_ulysses_unpermute(const void *y, void *x, int B, int S, int H, int D, int elem_bytes, int degree,
                              const int *seq_splits, const int *head_splits, cpattn_stream_t stream) {
   PermuteParams pp;
@@ -747,13 +773,10 @@ static int ulysses_common(const void *q, const void *k, const void *v, void *out
   void *yq = ws, *yk = ws + tensor_bytes, *yv = ws + 2 * tensor_bytes, *yo = ws + 3 * tensor_bytes;
   std::vector<int> heads;
   resolve_splits(H, degree, head_splits, heads);
-  // first all-to-all: Q, K, V to the head-sharded layout
-  const void *srcs[3] = {q, k, v};
-  void *dsts[3] = {yq, yk, yv};
-  for (int i = 0; i < 3; ++i) {
+  // first all-to-all: Q, K, V to the head-sharded layout, one launch
+  {
     PermuteParams pp = pq;
-    pp.src = static_cast<const unsigned char *>(srcs[i]);
-    pp.dst = static_cast<unsigned char *>(dsts[i]);
+    set_qkv(pp, q, k, v, yq, yk, yv);
     if (launch_permute(pp, stream) != cudaSuccess) return CPATTN_ERR_CUDA;
   }
   // local attention of every head rank over all S tokens of its heads
@@ -761,8 +784,9 @@ static int ulysses_common(const void *q, const void *k, const void *v, void *out
   if (st != CPATTN_OK) return st;
   // second all-to-all: the output back to the sequence-sharded layout
   PermuteParams po = pq;
-  po.src = static_cast<const unsigned char *>(yo);
-  po.dst = static_cast<unsigned char *>(out);
+  po.src[0] = static_cast<const unsigned char *>(yo);
+  po.dst[0] = static_cast<unsigned char *>(out);
+  po.n_tensors = 1;
   po.direction = 1;
   return launch_permute(po, stream) == cudaSuccess ? CPATTN_OK : CPATTN_ERR_CUDA;
 }
@@ -820,12 +844,9 @@ static int unified_common(const void *q, const void *k, const void *v, void *out
   for (int i = 0; i <= ring_degree; ++i) pp.group_off[i] = off[i];
   pp.n_head = ulysses_degree;
   for (int u = 0; u <= ulysses_degree; ++u) pp.head_off[u] = ho[u];
-  const void *srcs[3] = {q, k, v};
-  void *dsts[3] = {yq, yk, yv};
-  for (int i = 0; i < 3; ++i) {
+  {
     PermuteParams p1 = pp;
-    p1.src = static_cast<const unsigned char *>(srcs[i]);
-    p1.dst = static_cast<unsigned char *>(dsts[i]);
+    set_qkv(p1, q, k, v, yq, yk, yv);
     p1.direction = 0;
     if (launch_permute(p1, stream) != cudaSuccess) return CPATTN_ERR_CUDA;
   }
@@ -840,8 +861,9 @@ static int unified_common(const void *q, const void *k, const void *v, void *out
   st = run_attention(probs, groups, D, false, causal, stream);
   if (st != CPATTN_OK) return st;
   PermuteParams p2 = pp;
-  p2.src = static_cast<const unsigned char *>(yo);
-  p2.dst = static_cast<unsigned char *>(out);
+  p2.src[0] = static_cast<const unsigned char *>(yo);
+  p2.dst[0] = static_cast<unsigned char *>(out);
+  p2.n_tensors = 1;
   p2.direction = 1;
   return launch_permute(p2, stream) == cudaSuccess ? CPATTN_OK : CPATTN_ERR_CUDA;
 }

@@ -111,9 +111,12 @@ cudaError_t launch_lse_merge(const MergeParams &p, cudaStream_t stream);
 constexpr int kMaxRanks = 64;
 constexpr int kMaxHeads = 1024;
 
+constexpr int kMaxPermuteTensors = 3;   // Q, K and V move in one launch
+
 struct PermuteParams {
-  const unsigned char *src;
-  unsigned char *dst;
+  const unsigned char *src[kMaxPermuteTensors];
+  unsigned char *dst[kMaxPermuteTensors];
+  int n_tensors;        // tensors with the same shape and splits, 1..kMaxPermuteTensors
   int B, S, H;
   int row_bytes;        // D * elem_bytes (multiple of 16)
   int direction;        // 0: sequence side -> head side, 1: head side -> sequence side

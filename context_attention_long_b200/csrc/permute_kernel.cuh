@@ -12,6 +12,8 @@
 // elements: every moved unit is a contiguous run of >= 128 bytes and no
 // shared-memory transpose is needed to keep both sides coalesced.
 //
+// Up to three tensors of the same shape (Q, K and V of the first all-to-all)
+// move in one launch: every warp takes its tokens of each tensor in turn.
 // One warp moves one token per iteration: lanes take consecutive 16-byte
 // vectors of the token's H*D run (coalesced on the sequence side, and on the
 // head side within each head rank's contiguous block), four vectors in flight
@@ -47,6 +49,7 @@ __global__ void __launch_bounds__(kPermuteThreads) permute_kernel(const __grid_c
   const int nvec = p.H * vpr;                       // vectors per token
   const long long seq_row_bytes = static_cast<long long>(p.H) * p.row_bytes;
 
+  for (int t = 0; t < p.n_tensors; ++t)
   for (long long tok = warp_id; tok < ntok; tok += nwarps) {
     const int b = static_cast<int>(tok / p.S);
     const int s = static_cast<int>(tok - static_cast<long long>(b) * p.S);
@@ -61,8 +64,8 @@ __global__ void __launch_bounds__(kPermuteThreads) permute_kernel(const __grid_c
     const int gi = find_range(p.group_off, p.n_groups, s);
     const int goff = p.group_off[gi], glen = p.group_off[gi + 1] - goff;
     const long long head_row = static_cast<long long>(p.B) * goff + static_cast<long long>(b) * glen + (s - goff);
-    const unsigned char *seq_base = (p.direction == 0 ? p.src : p.dst) + seq_row * seq_row_bytes;
-    unsigned char *const head_buf = p.direction == 0 ? p.dst : const_cast<unsigned char *>(p.src);
+    const unsigned char *seq_base = (p.direction == 0 ? p.src[t] : p.dst[t]) + seq_row * seq_row_bytes;
+    unsigned char *const head_buf = p.direction == 0 ? p.dst[t] : const_cast<unsigned char *>(p.src[t]);
 
     for (int v0 = lane; v0 < nvec; v0 += 32 * 4) {
       uint4 val[4];

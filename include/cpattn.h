@@ -176,6 +176,17 @@ int cpattn_ulysses_permute(const void *x, void *y, int B, int S, int H, int D, i
                            cpattn_stream_t stream);
 
 /*
+ * The first all-to-all of the Ulysses flow for Q, K and V at once: the
+ * cpattn_ulysses_permute of each of the three tensors (same shape, element
+ * size and splits), in one launch.  q, k, v are read, yq, yk, yv written; the
+ * six buffers must not alias.  Arguments and errors as cpattn_ulysses_permute.
+ */
+int cpattn_ulysses_permute_qkv(const void *q, const void *k, const void *v, void *yq, void *yk,
+                               void *yv, int B, int S, int H, int D, int elem_bytes, int degree,
+                               const int *seq_splits, const int *head_splits,
+                               cpattn_stream_t stream);
+
+/*
  * Ulysses unpermute, head-sharded -> sequence-sharded: the second all-to-all,
  * which regroups the attention output by token ([CP] "Ulysses Attention");
  * the exact inverse of cpattn_ulysses_permute (same arguments, y is read and

@@ -119,6 +119,11 @@ def test_permute_validation(lib):
     assert f(y=FAKE_MIS) == ALIGN
     g = lambda H=5: lib.cpattn_ulysses_unpermute(FAKE, FAKE, 1, 8, H, 64, 2, 2, None, None, None)
     assert g() == INDIV
+    t = lambda k=FAKE, yv=FAKE, H=4: lib.cpattn_ulysses_permute_qkv(FAKE, k, FAKE, FAKE, FAKE, yv, 1, 8, H, 64, 2, 2,
+                                                                    None, None, None)
+    assert t(k=None) == NULL
+    assert t(yv=FAKE_MIS) == ALIGN
+    assert t(H=5) == INDIV
 
 
 def test_flow_validation(lib):

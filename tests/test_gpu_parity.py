@@ -165,6 +165,24 @@ def test_permute_bit_exact_and_round_trip(B, S, H, D, P, seq, heads, dtype):
     assert torch.equal(back.view(torch.uint8), x.view(torch.uint8))
 
 
+@pytest.mark.parametrize("B,S,H,D,P,seq,heads", [
+    (1, 4608, 24, 128, 4, None, None),                    # image-DiT Ulysses 4
+    (2, 300, 7, 64, 3, [100, 0, 200], [3, 2, 2]),        # uneven, an empty sequence shard
+])
+def test_permute_qkv_equals_three_permutes(B, S, H, D, P, seq, heads):
+    """The one-launch Q/K/V permute is bit-identical to the oracle's permute of
+    each tensor."""
+    n = B * S * H * D
+    rng = np.random.Generator(np.random.PCG64(n + 5))
+    raws = [rng.integers(0, 1 << 16, size=n, dtype=np.uint16) for _ in range(3)]
+    xs = [torch.from_numpy(r.view(np.int16)).cuda().view(torch.bfloat16) for r in raws]
+    ys = api.cpattn_ulysses_permute_qkv(*xs, B, S, H, D, P, seq, heads)
+    torch.cuda.synchronize()
+    for raw, y in zip(raws, ys):
+        ref = oracle.ulysses_permute(raw, B, S, H, D, P, seq, heads)
+        assert np.array_equal(bits_of(y).reshape(-1), ref)
+
+
 # ------------------------------------------------------------------ Ulysses / unified
 
 @pytest.mark.parametrize("B,S,H,D,P,seq,heads", [
