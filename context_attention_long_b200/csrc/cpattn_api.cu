@@ -28,7 +28,11 @@ namespace cpattn {
 
 // ------------------------------------------------------------------ helpers
 
-constexpr int kMaxRingDegree = 1024;
+// A fused-ring unit walks one K/V range per chunk, and one launch holds at
+// most kMaxKV ranges, so the ring degree is capped there; kv_gather walks a
+// single range per shard and may use more shards.
+constexpr int kMaxRingDegree = kMaxKV;
+constexpr int kMaxGatherDegree = 1024;
 constexpr int kMaxDevices = 64;
 
 static unsigned long long wait_timeout_ns() {
@@ -605,7 +609,7 @@ int cpattn_kv_gather_attention(const void *q, const void *k, const void *v, void
   if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return CPATTN_ERR_NULL;
   int st = check_attn_shape(B, H, S, D);
   if (st != CPATTN_OK) return st;
-  if (degree < 1 || degree > kMaxRingDegree) return CPATTN_ERR_DEGREE;
+  if (degree < 1 || degree > kMaxGatherDegree) return CPATTN_ERR_DEGREE;
   std::vector<int> lens;
   st = resolve_splits(S, degree, q_lens, lens);
   if (st != CPATTN_OK) return st;

@@ -94,7 +94,7 @@ int cpattn_version(void);
  *   lse        [B, H, S] float32 device, natural log; may be NULL.
  *   chunk_lens host int[ring_degree] (Ring Anything) or NULL (equal split,
  *              S % ring_degree must be 0 else CPATTN_ERR_INDIVISIBLE).
- * Errors: NULL, SHAPE, DEGREE (ring_degree < 1 or > S), INDIVISIBLE, SPLITS,
+ * Errors: NULL, SHAPE, DEGREE (ring_degree < 1, > S, or > 512), INDIVISIBLE, SPLITS,
  * ALIGNMENT, UNSUPPORTED, CUDA.
  */
 int cpattn_ring_attention(const void *q, const void *k, const void *v, void *out, float *lse,
@@ -145,7 +145,7 @@ int cpattn_lse_merge(const float *part_out, const float *part_lse, int P, int B,
  * against all S keys; non-causal, ring degree 1.
  *
  *   q_lens     host int[degree] or NULL (equal split).
- * Other arguments as cpattn_ring_attention.
+ * Other arguments as cpattn_ring_attention; degree may be up to 1024.
  */
 int cpattn_kv_gather_attention(const void *q, const void *k, const void *v, void *out,
                                float *lse, int B, int H, int S, int D, int degree,
