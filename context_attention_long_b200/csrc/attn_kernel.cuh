@@ -148,6 +148,24 @@ __device__ __forceinline__ Unit decode_unit(const AttnParams &p) {
   } else {
     u.n0 = n;
     u.n1 = u.has_q1 ? n : 0;
+    if (p.causal && u.has_q1) {
+      // The first Q tile of a causal pair sees keys up to its own last row
+      // only.  When the tiles it cannot see form a suffix of the walk (the
+      // plan lists the chunk that the mask cuts last), slot 0 stops after the
+      // prefix it sees; otherwise it walks every tile, fully masked ones too.
+      const int q_last0 = SG.s0 + u.pair * (kQTilesPerCTA * kQTile) + kQTile - 1;
+      int n0 = 0;
+      bool cut = false, prefix = true;
+      for (int i = 0; i < SG.kv_count; ++i) {
+        const AttnKV kv = p.kv[SG.kv_first + i];
+        const int t_all = (kv_rows_seen(p, kv, u.q_last) + kKVTile - 1) / kKVTile;
+        const int t_own = (kv_rows_seen(p, kv, q_last0) + kKVTile - 1) / kKVTile;
+        if (cut && t_all > 0) prefix = false;
+        n0 += t_own;
+        if (t_own < t_all) cut = true;
+      }
+      if (prefix && n0 >= 1) u.n0 = n0;
+    }
   }
   return u;
 }
@@ -360,18 +378,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
           const uint32_t ph1 = ((j + 1) / NST) & 1;
           const bool more = j + 1 < n_tiles;
           if (!mbar_wait_spin(sb + BAR_VF + 8 * st, ph, abort_flag, tmo, SITE_MMA)) break;
-          if (!mbar_wait_spin(sb + BAR_PH, j & 1, abort_flag, tmo, SITE_MMA)) break;
-          tc_fence_after();
-          issue_pv(0, st, j > 0, 0);
-          if (!mbar_wait_spin(sb + BAR_P, j & 1, abort_flag, tmo, SITE_MMA)) break;
-          tc_fence_after();
-          issue_pv(0, st, j > 0, 1);
-          if (!more) mma_commit(sb + BAR_O);
+          if (j < n0) {   // slot 0 may stop before slot 1 (causal pairs)
+            if (!mbar_wait_spin(sb + BAR_PH, j & 1, abort_flag, tmo, SITE_MMA)) break;
+            tc_fence_after();
+            issue_pv(0, st, j > 0, 0);
+            if (!mbar_wait_spin(sb + BAR_P, j & 1, abort_flag, tmo, SITE_MMA)) break;
+            tc_fence_after();
+            issue_pv(0, st, j > 0, 1);
+            if (j == n0 - 1) mma_commit(sb + BAR_O);
+          }
           if (more) {
             if (!mbar_wait_spin(sb + BAR_KF + 8 * st1, ph1, abort_flag, tmo, SITE_MMA)) break;
             tc_fence_after();
-            issue_qk(0, st1);
-            mma_commit(sb + BAR_S);
+            if (j + 1 < n0) {
+              issue_qk(0, st1);
+              mma_commit(sb + BAR_S);
+            }
           }
           if (has_q1) {
             if (!mbar_wait_spin(sb + BAR_PH + 8, j & 1, abort_flag, tmo, SITE_MMA)) break;
@@ -451,7 +473,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
     const bool causal = p.causal != 0;
     // K/V tiles [g_lo, g_hi) of the segment belong to this slot.
     const int g_lo = (split && qt == 1) ? U.n0 : 0;
-    const int g_hi = split ? (qt == 0 ? U.n0 : U.n0 + U.n1) : n_tiles;
+    const int g_hi = split ? (qt == 0 ? U.n0 : U.n0 + U.n1) : (qt == 0 ? U.n0 : n_tiles);
     float m = -INFINITY;  // running max, scaled (log2) domain
     float l = 0.f;        // running sum of 2^(x - m)
     bool ok = true;

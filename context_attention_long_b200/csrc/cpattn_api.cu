@@ -434,7 +434,11 @@ static void ring_groups(std::vector<GroupSpec> &groups, int prob, int B, const s
       s.row0 = row_of(b, r);
       s.nrows = lens[r];
       s.s0 = off[r];
-      for (int t = 0; t < P; ++t) {
+      for (int i_t = 0; i_t < P; ++i_t) {
+        // Causal fused plans visit the shard's own chunk (the one the mask
+        // cuts) after the earlier chunks, so that the keys the first Q tile
+        // of a pair cannot see come last in the walk.
+        const int t = (causal && step < 0) ? (i_t + 1) % P : i_t;
         if (step >= 0 && t != step) continue;
         const int c = ((r - t) % P + P) % P;  // chunk held by rank r after t hand-offs
         if (causal && c > r) continue;

@@ -266,9 +266,11 @@ int cpattn_unified_attention(const void *q, const void *k, const void *v, void *
  *
  * Each function takes exactly the arguments, layouts, ownership and error
  * behaviour of its non-causal namesake:
- *   cpattn_causal_ring_attention        as cpattn_ring_attention.  In ring
- *       order rank r walks c = r, r-1, ..., 0; chunks after shard r are
- *       invisible to all of its queries and are not visited.
+ *   cpattn_causal_ring_attention        as cpattn_ring_attention.  Rank r
+ *       walks the chunks before its shard in ring order (r-1, ..., 0) and its
+ *       own chunk, the one the mask cuts, last; chunks after shard r are
+ *       invisible to all of its queries and are not visited.  The merge is
+ *       order-independent in exact arithmetic.
  *   cpattn_causal_ring_step             as cpattn_ring_step.  A step whose
  *       chunk lies after shard r writes out = 0 and LSE = -inf for its rows
  *       (the neutral partial), so cpattn_lse_merge of all steps equals
