@@ -97,3 +97,26 @@ def test_permute_and_flows_write_only_their_outputs():
     torch.cuda.synchronize()
     for raw in (ws_raw, o_raw, wu_raw, ou_raw):
         assert guards_intact(raw)
+
+
+@pytest.mark.parametrize("B,H,S,D,P,lens", [
+    (1, 3, 333, 128, 3, [100, 0, 233]),
+    (1, 2, 1152 * 2, 128, 2, None),
+])
+def test_causal_paths_write_only_their_outputs(B, H, S, D, P, lens):
+    q, k, v = (to_dev(x) for x in inputs.make_qkv(B, S, H, D, 17 + S, True))
+    out_raw, out = guarded((B, S, H, D), torch.bfloat16)
+    lse_raw, lse = guarded((B, H, S), torch.float32)
+    api.cpattn_causal_ring_attention(q, k, v, P, lens, out=out, lse=lse)
+    po_raw, po = guarded((B, S, H, D), torch.float32)
+    pl_raw, pl = guarded((B, H, S), torch.float32)
+    api.cpattn_causal_ring_step(q, k, v, P, P - 1, lens, part_out=po, part_lse=pl)
+    seq = lens or [S // P] * P
+    qf, kf, vf = (t.reshape(-1) for t in (q, k, v))
+    ws_raw, ws = guarded((api.cpattn_ulysses_workspace_bytes(B, H, S, D),), torch.uint8)
+    ou_raw, ou = guarded((B * S * H * D,), torch.bfloat16)
+    api.cpattn_causal_ulysses_attention(qf, kf, vf, B, S, H, D, P, seq, [H - 1] + [1] * (P - 2) + [0] if P > 2 else None,
+                                        out=ou, workspace=ws)
+    torch.cuda.synchronize()
+    for raw in (out_raw, lse_raw, po_raw, pl_raw, ws_raw, ou_raw):
+        assert guards_intact(raw)
