@@ -8,6 +8,7 @@ correct CPU restatement, in float64, of what the hot path computes:
 * per-chunk partial attention with its log-sum-exp, and the LSE merge of
   partials (ring attention; Ring Anything chunk lengths),
 * the kv_gather exchange (each Q shard against the full K/V),
+* the gradient of attention with respect to Q, K and V (causal or not),
 * the Ulysses sequence-sharded <-> head-sharded permutation and its inverse
   (including the uneven Ulysses Anything splits), and the Ulysses and unified
   (ring x Ulysses) attention flows composed from the pieces above.
@@ -24,7 +25,7 @@ Sources (web pages, cited by title and section):
   [SP]   SGLang Diffusion docs, "Sequence Parallelism" -- "Choosing The
          Attention Exchange", "Numerics across node boundaries".
   [USP]  "Ulysses Sequence Parallelism: training with million-token contexts"
-         (article summary) -- sections 2, 3, 4, 5, 7.
+         (article summary) -- sections 1, 2, 3, 4, 5, 7.
   [API]  diffusers docs, "parallel" -- ContextParallelConfig parameters.
   [PR]   sglang PR #30086 analysis -- Gemma 3 attention (B, S, H, D) view and
          head_dim**-0.5 scale.
@@ -47,6 +48,7 @@ from .attention import (
     ring_step_partials,
     kv_gather_attention,
 )
+from .backward import attention_backward, attention_backward_rows
 from .permute import (
     ulysses_permute,
     ulysses_unpermute,
@@ -59,5 +61,5 @@ __all__ = [
     "causal_attention_rows", "lse_merge", "equal_splits",
     "offsets", "ring_order", "ring_attention", "ring_step_partials",
     "kv_gather_attention", "ulysses_permute", "ulysses_unpermute",
-    "ulysses_attention", "unified_attention",
+    "ulysses_attention", "unified_attention", "attention_backward", "attention_backward_rows",
 ]
