@@ -265,6 +265,26 @@ def cpattn_causal_unified_attention(q, k, v, ring_degree, ulysses_degree, ring_l
                     head_splits, out, lse, want_lse, workspace, stream)
 
 
+def cpattn_attention_backward_workspace_bytes(B, H, S) -> int:
+    return int(_native.load().cpattn_attention_backward_workspace_bytes(B, H, S))
+
+
+def cpattn_attention_backward(q, k, v, out, lse, dout, causal=False, dq=None, dk=None, dv=None, workspace=None,
+                              stream=None):
+    """Gradient of attention over full (B,S,H,D) bf16 tensors given the
+    forward's output and LSE; returns (dq, dk, dv) in bf16."""
+    B, S, H, D = _bshd(q)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    workspace = _workspace(cpattn_attention_backward_workspace_bytes(B, H, S), q.device, workspace)
+    _check(_native.load().cpattn_attention_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout),
+                                                    _ptr(dq), _ptr(dk), _ptr(dv), B, H, S, D, 1 if causal else 0,
+                                                    _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                                    _stream(stream)), "cpattn_attention_backward")
+    return dq, dk, dv
+
+
 # Size of the library-held scratch of cpattn_ulysses_attention_noalloc
 # (CPATTN_NOALLOC_SCRATCH_BYTES in cpattn.h).
 NOALLOC_SCRATCH_BYTES = 64 << 20

@@ -1,0 +1,651 @@
+// attn_bwd_kernel.cuh -- gradient of softmax attention for sm_100a.
+//
+// The derivative of the forward definition (attn_kernel.cuh), per (batch,
+// head), with S = Q K^T * scale, P = softmax(S) recomputed from the forward's
+// log-sum-exp, and the upstream gradient dO of the output O:
+//   Delta = rowsum(dO * O)                       (attn_bwd_delta_kernel)
+//   dP    = dO V^T,   dS = P * (dP - Delta)
+//   dQ    = dS K * scale                         (attn_bwd_dq_kernel)
+//   dV    = P^T dO,   dK = dS^T Q * scale        (attn_bwd_dkv_kernel)
+// The pages train with Ulysses over long contexts (the Ulysses Sequence
+// Parallelism article, sections 1 and 7, causal masking by position ids); the
+// causal mask here is the forward's: key j is visible to query i iff j <= i.
+//
+// Two kernels, so that no gradient needs atomics: the dQ kernel owns a Q tile
+// and walks the K/V tiles; the dK/dV kernel owns a K/V tile and walks the Q
+// tiles (S and dP are computed in both).  CTA organisation of each (192
+// threads, one CTA per SM):
+//   warp 0      TMA producer: the owned tiles once, the walked tiles through
+//               a 2-stage ring
+//   warp 1      TMEM allocator + single-thread MMA issuer (tcgen05.mma)
+//   warps 2-5   one row of the owned tile per thread (TMEM lane): P and dS in
+//               registers, bf16 results back into TMEM, the epilogue
+// TMEM columns: S [0,128) (later P), dP [128,256) (later dS), then the
+// accumulators (dQ; or dV and dK).  The next tile's S is issued as soon as
+// the row threads have read the current S (dQ kernel) or the current P has
+// been consumed (dK/dV kernel), so the tensor core works while the row
+// threads exponentiate.  Every wait is bounded as in the forward.
+#pragma once
+
+#include "cpattn_internal.h"
+#include "cpattn_ptx.cuh"
+
+namespace cpattn {
+
+template <int D>
+struct BwdSmem {
+  static constexpr int kHalves = D / 64;
+  static constexpr int kBoxBytes = 128 * 128;          // [128 rows][64 bf16], 128B-swizzled
+  static constexpr int kTileBytes = kHalves * kBoxBytes;
+  static constexpr int kStages = 2;
+  static constexpr int kOffA = 0;                       // owned tile 0: Q (dq) or K (dkv)
+  static constexpr int kOffB = kOffA + kTileBytes;      // owned tile 1: dO (dq) or V (dkv)
+  static constexpr int kOffC = kOffB + kTileBytes;      // walked tile 0 per stage: K (dq) or Q (dkv)
+  static constexpr int kOffE = kOffC + kStages * kTileBytes;   // walked tile 1 per stage: V or dO
+  static constexpr int kOffVec = kOffE + kStages * kTileBytes; // dkv: [stage][lse2 128 | delta 128] floats
+  static constexpr int kOffBar = kOffVec + kStages * 2 * 128 * 4;
+  static constexpr int kNumBars = 16;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kBytes = kOffMisc + 16;
+  static constexpr int kAllocBytes = kBytes + 1024;
+};
+
+constexpr int kBwdThreads = 192;
+constexpr uint32_t kBwdTmemCols = 512;
+
+// Delta[b, h, s] = sum_d dO[b, s, h, d] * O[b, s, h, d], one warp per
+// (token, head) row: lanes read 8-byte pieces of both rows (coalesced).
+__global__ void __launch_bounds__(256) attn_bwd_delta_kernel(const __nv_bfloat16 *__restrict__ out,
+                                                             const __nv_bfloat16 *__restrict__ dout,
+                                                             float *__restrict__ delta, int B, int S, int H,
+                                                             int D) {
+  const int lane = threadIdx.x & 31;
+  const long long warp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const long long nwarps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  const long long nrows = static_cast<long long>(B) * S * H;
+  for (long long r = warp; r < nrows; r += nwarps) {
+    const __nv_bfloat16 *o = out + r * D;
+    const __nv_bfloat16 *g = dout + r * D;
+    float acc = 0.f;
+    for (int d = lane * 4; d < D; d += 128) {
+      const uint2 ov = __ldcs(reinterpret_cast<const uint2 *>(o + d));
+      const uint2 gv = __ldcs(reinterpret_cast<const uint2 *>(g + d));
+      const float2 o0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ov.x));
+      const float2 o1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ov.y));
+      const float2 g0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&gv.x));
+      const float2 g1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&gv.y));
+      acc = fmaf(o0.x, g0.x, fmaf(o0.y, g0.y, fmaf(o1.x, g1.x, fmaf(o1.y, g1.y, acc))));
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) {
+      const long long tok = r / H;
+      const int h = static_cast<int>(r - tok * H);
+      const int b = static_cast<int>(tok / S);
+      const int s = static_cast<int>(tok - static_cast<long long>(b) * S);
+      delta[(static_cast<long long>(b) * H + h) * S + s] = acc;
+    }
+  }
+}
+
+// Units of both kernels: (b, h, 128-row tile) with the tile index fastest.
+struct BwdUnit {
+  int b, h, t;
+};
+__device__ __forceinline__ BwdUnit bwd_unit(const BwdParams &p, bool last_first) {
+  const int nt = (p.S + 127) / 128;
+  BwdUnit u;
+  const int t_in = blockIdx.x % nt;
+  const int bh = blockIdx.x / nt;
+  u.h = bh % p.H;
+  u.b = bh / p.H;
+  u.t = last_first ? nt - 1 - t_in : t_in;
+  return u;
+}
+
+// ===================================================================== dQ
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
+  using L = BwdSmem<D>;
+  constexpr uint32_t IDESC_SS = idesc_bf16_f32(128, 128, false);   // S = Q K^T, dP = dO V^T
+  constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, D, true);      // dQ += dS K, K MN-major
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t sb = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  constexpr uint32_t BAR_QD = L::kOffBar;          // Q and dO loaded
+  constexpr uint32_t BAR_KF = BAR_QD + 8;          // [2]
+  constexpr uint32_t BAR_KE = BAR_KF + 16;         // [2]
+  constexpr uint32_t BAR_VF = BAR_KE + 16;         // [2]
+  constexpr uint32_t BAR_VE = BAR_VF + 16;         // [2]
+  constexpr uint32_t BAR_S = BAR_VE + 16;          // S(j) in TMEM
+  constexpr uint32_t BAR_SC = BAR_S + 8;           // S(j) read by the row threads
+  constexpr uint32_t BAR_DP = BAR_SC + 8;          // dP(j) in TMEM
+  constexpr uint32_t BAR_DS = BAR_DP + 8;          // dS(j) in TMEM
+  constexpr uint32_t BAR_DQ = BAR_DS + 8;          // dQ complete
+  constexpr uint32_t BAR_TAIL = BAR_DQ + 8;
+  constexpr uint32_t TMEM_SLOT = L::kOffMisc;
+  constexpr uint32_t ABORT = L::kOffMisc + 4;
+  static_assert(BAR_TAIL + 8 <= L::kOffMisc, "barrier area");
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint64_t tmo = p.timeout_ns;
+  const BwdUnit U = bwd_unit(p, p.causal != 0);   // causal: heavier (later) Q tiles first
+  const int q0 = U.t * 128;
+  const int q_rows = min(128, p.S - q0);
+  const int kv_len = p.causal ? min(p.S, q0 + q_rows) : p.S;   // keys at positions < kv_len
+  const int n = (kv_len + 127) / 128;
+  const int row_base = U.b * p.S;
+
+  if (threadIdx.x == 0) {
+    mbar_init(sb + BAR_QD, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(sb + BAR_KF + 8 * s, 1);
+      mbar_init(sb + BAR_KE + 8 * s, 1);
+      mbar_init(sb + BAR_VF + 8 * s, 1);
+      mbar_init(sb + BAR_VE + 8 * s, 1);
+    }
+    mbar_init(sb + BAR_S, 1);
+    mbar_init(sb + BAR_SC, 4);
+    mbar_init(sb + BAR_DP, 1);
+    mbar_init(sb + BAR_DS, 4);
+    mbar_init(sb + BAR_DQ, 1);
+    mbar_init(sb + BAR_TAIL, 1);
+    st_shared_volatile(sb + ABORT, 0u);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(sb + TMEM_SLOT, kBwdTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ld_shared_volatile(sb + TMEM_SLOT);
+  const uint32_t abort_flag = sb + ABORT;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&p.tm_q);
+      tma_prefetch_desc(&p.tm_k);
+      tma_prefetch_desc(&p.tm_v);
+      tma_prefetch_desc(&p.tm_do);
+      mbar_arrive_expect_tx(sb + BAR_QD, 2 * L::kTileBytes);
+      for (int hf = 0; hf < L::kHalves; ++hf) {
+        tma_load_3d(sb + L::kOffA + hf * L::kBoxBytes, &p.tm_q, hf * 64, U.h, row_base + q0, sb + BAR_QD);
+        tma_load_3d(sb + L::kOffB + hf * L::kBoxBytes, &p.tm_do, hf * 64, U.h, row_base + q0, sb + BAR_QD);
+      }
+      for (int j = 0; j < n; ++j) {
+        const int st = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        if (!mbar_wait(sb + BAR_KE + 8 * st, ph ^ 1, abort_flag, tmo, SITE_PRODUCER)) break;
+        mbar_arrive_expect_tx(sb + BAR_KF + 8 * st, L::kTileBytes);
+        for (int hf = 0; hf < L::kHalves; ++hf)
+          tma_load_3d(sb + L::kOffC + st * L::kTileBytes + hf * L::kBoxBytes, &p.tm_k, hf * 64, U.h,
+                      row_base + j * 128, sb + BAR_KF + 8 * st);
+        if (!mbar_wait(sb + BAR_VE + 8 * st, ph ^ 1, abort_flag, tmo, SITE_PRODUCER)) break;
+        mbar_arrive_expect_tx(sb + BAR_VF + 8 * st, L::kTileBytes);
+        for (int hf = 0; hf < L::kHalves; ++hf)
+          tma_load_3d(sb + L::kOffE + st * L::kTileBytes + hf * L::kBoxBytes, &p.tm_v, hf * 64, U.h,
+                      row_base + j * 128, sb + BAR_VF + 8 * st);
+      }
+      // every stage's last release must arrive before the CTA exits
+      for (int st = 0; st < 2; ++st) {
+        const int uses = n > st ? (n - 1 - st) / 2 + 1 : 0;
+        if (uses == 0) continue;
+        const uint32_t ph = (uses - 1) & 1;
+        mbar_wait(sb + BAR_KE + 8 * st, ph, 0u, tmo, SITE_TAIL);
+        mbar_wait(sb + BAR_VE + 8 * st, ph, 0u, tmo, SITE_TAIL);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint64_t dQo = smem_desc_sw128(sb + L::kOffA, 16, 1024);
+      const uint64_t dDO = smem_desc_sw128(sb + L::kOffB, 16, 1024);
+      const uint64_t dK = smem_desc_sw128(sb + L::kOffC, 16, 1024);                  // K-major (S)
+      const uint64_t dKmn = smem_desc_sw128(sb + L::kOffC, L::kBoxBytes, 1024);       // MN-major (dQ)
+      const uint64_t dV = smem_desc_sw128(sb + L::kOffE, 16, 1024);
+      auto issue_ss = [&](uint32_t d, uint64_t a0, uint64_t b0) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk >> 2) * L::kBoxBytes + (kk & 3) * 32) >> 4;
+          mma_ss(d, a0 + off, b0 + off, IDESC_SS, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_s = [&](int st) { issue_ss(tmem, opaque_u64(dQo), opaque_u64(dK + ((st * L::kTileBytes) >> 4))); };
+      auto issue_dp = [&](int st) {
+        issue_ss(tmem + 128, opaque_u64(dDO), opaque_u64(dV + ((st * L::kTileBytes) >> 4)));
+      };
+      // dQ (+)= dS K: dS (bf16 pairs) from TMEM over dP, K MN-major (keys
+      // are rows of 128 bytes): 16 keys = 2048 bytes per MMA.
+      auto issue_dq = [&](int st, bool acc) {
+        const uint64_t b0 = opaque_u64(dKmn + ((st * L::kTileBytes) >> 4));
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + 256, tmem + 128 + kk * 8, b0 + ((kk * 2048) >> 4), IDESC_DQ, (acc || kk > 0) ? 1u : 0u);
+      };
+      bool ok = n > 0 && mbar_wait_spin(sb + BAR_QD, 0, abort_flag, tmo, SITE_MMA);
+      if (ok) ok = mbar_wait_spin(sb + BAR_KF, 0, abort_flag, tmo, SITE_MMA);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+        mma_commit(sb + BAR_S);
+      }
+      if (ok) ok = mbar_wait_spin(sb + BAR_VF, 0, abort_flag, tmo, SITE_MMA);
+      if (ok) {
+        tc_fence_after();
+        issue_dp(0);
+        mma_commit(sb + BAR_DP);
+      }
+      for (int j = 0; ok && j < n; ++j) {
+        const int st = j & 1, st1 = (j + 1) & 1;
+        const uint32_t ph1 = ((j + 1) >> 1) & 1;
+        const bool more = j + 1 < n;
+        if (!mbar_wait_spin(sb + BAR_SC, j & 1, abort_flag, tmo, SITE_MMA)) break;
+        if (more) {   // S(j) has been read: the next S may overwrite it
+          if (!mbar_wait_spin(sb + BAR_KF + 8 * st1, ph1, abort_flag, tmo, SITE_MMA)) break;
+          tc_fence_after();
+          issue_s(st1);
+          mma_commit(sb + BAR_S);
+        }
+        if (!mbar_wait_spin(sb + BAR_DS, j & 1, abort_flag, tmo, SITE_MMA)) break;
+        tc_fence_after();
+        issue_dq(st, j > 0);
+        mma_commit(sb + BAR_KE + 8 * st);
+        mma_commit(sb + BAR_VE + 8 * st);
+        if (more) {   // dS(j) is consumed in order before dP(j+1) overwrites it
+          if (!mbar_wait_spin(sb + BAR_VF + 8 * st1, ph1, abort_flag, tmo, SITE_MMA)) break;
+          tc_fence_after();
+          issue_dp(st1);
+          mma_commit(sb + BAR_DP);
+        }
+      }
+      if (n > 0) mma_commit(sb + BAR_DQ);
+      mma_commit(sb + BAR_TAIL);
+      mbar_wait(sb + BAR_TAIL, 0, 0u, tmo, SITE_TAIL);
+    }
+  } else {
+    // ------------------------------------------------------------ row threads
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const int q_pos = q0 + row;
+    const bool row_valid = row < q_rows;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t tS = tmem + lane_base;
+    const uint32_t tDP = tmem + lane_base + 128;
+    const uint32_t tDQ = tmem + lane_base + 256;
+    const float c = p.scale_log2;
+    const long long vi = (static_cast<long long>(U.b) * p.H + U.h) * p.S + q_pos;
+    const float lse2 = row_valid ? p.lse[vi] * 1.4426950408889634f : 0.f;
+    const float delta = row_valid ? p.delta[vi] : 0.f;
+    bool ok = true;
+    for (int j = 0; ok && j < n; ++j) {
+      // keys of tile j this row sees: all valid keys, cut at the row's own
+      // position under the causal mask; none for rows past the sequence
+      int kvalid = min(128, kv_len - j * 128);
+      if (p.causal) kvalid = min(kvalid, q_pos - j * 128 + 1);
+      if (!row_valid) kvalid = 0;
+      bool w = mbar_wait(sb + BAR_S, j & 1, abort_flag, tmo, SITE_SOFTMAX);
+      if (__any_sync(0xffffffffu, !w)) { ok = false; break; }
+      __syncwarp();
+      tc_fence_after();
+      uint32_t s[128];
+      tmem_ld128_wait(tS, s);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sb + BAR_SC);
+      // P = 2^(S*c - lse2), kept in fp32 over the scores
+#pragma unroll
+      for (int k = 0; k < 128; ++k)
+        s[k] = __float_as_uint(k < kvalid ? ex2_approx(__uint_as_float(s[k]) * c - lse2) : 0.f);
+      w = mbar_wait(sb + BAR_DP, j & 1, abort_flag, tmo, SITE_SOFTMAX);
+      if (__any_sync(0xffffffffu, !w)) { ok = false; break; }
+      __syncwarp();
+      tc_fence_after();
+      // dS = P * (dP - delta), bf16 pairs over the dP columns already read
+#pragma unroll
+      for (int c0 = 0; c0 < 128; c0 += 32) {
+        uint32_t dp[32];
+        tmem_ld32_wait(tDP + c0, dp);
+        uint32_t pk[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const float d0 = __uint_as_float(s[c0 + 2 * k]) * (__uint_as_float(dp[2 * k]) - delta);
+          const float d1 = __uint_as_float(s[c0 + 2 * k + 1]) * (__uint_as_float(dp[2 * k + 1]) - delta);
+          pk[k] = pack_bf16x2(d0, d1);
+        }
+        tmem_st16(tDP + c0 / 2, pk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sb + BAR_DS);
+    }
+    if (ok && n > 0) {
+      const bool w = mbar_wait(sb + BAR_DQ, 0, abort_flag, tmo, SITE_EPILOGUE);
+      if (__any_sync(0xffffffffu, !w)) ok = false;
+      __syncwarp();
+      tc_fence_after();
+    }
+    if (ok) {
+      const float scale = p.scale;
+      __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.dq) +
+                           ((static_cast<long long>(U.b) * p.S + q_pos) * p.H + U.h) * D;
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t o[32];
+        if (n > 0) {
+          tmem_ld32_wait(tDQ + c0, o);
+        } else {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] = 0u;
+        }
+        if (row_valid) {
+          uint4 *d4 = reinterpret_cast<uint4 *>(dst + c0);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            d4[k] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * k]) * scale, __uint_as_float(o[8 * k + 1]) * scale),
+                               pack_bf16x2(__uint_as_float(o[8 * k + 2]) * scale, __uint_as_float(o[8 * k + 3]) * scale),
+                               pack_bf16x2(__uint_as_float(o[8 * k + 4]) * scale, __uint_as_float(o[8 * k + 5]) * scale),
+                               pack_bf16x2(__uint_as_float(o[8 * k + 6]) * scale, __uint_as_float(o[8 * k + 7]) * scale));
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kBwdTmemCols);
+  }
+}
+
+// =================================================================== dK, dV
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __grid_constant__ BwdParams p) {
+  using L = BwdSmem<D>;
+  constexpr uint32_t IDESC_SS = idesc_bf16_f32(128, 128, false);   // S^T = K Q^T, dP^T = V dO^T
+  constexpr uint32_t IDESC_ACC = idesc_bf16_f32(128, D, true);     // dV += P^T dO, dK += dS^T Q
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t sb = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  constexpr uint32_t BAR_KV = L::kOffBar;          // K and V loaded
+  constexpr uint32_t BAR_QF = BAR_KV + 8;          // [2]
+  constexpr uint32_t BAR_QE = BAR_QF + 16;         // [2]
+  constexpr uint32_t BAR_OF = BAR_QE + 16;         // [2] dO tile full
+  constexpr uint32_t BAR_OE = BAR_OF + 16;         // [2]
+  constexpr uint32_t BAR_S = BAR_OE + 16;          // S^T(i) in TMEM
+  constexpr uint32_t BAR_P = BAR_S + 8;            // P^T(i) written
+  constexpr uint32_t BAR_DP = BAR_P + 8;           // dP^T(i) in TMEM
+  constexpr uint32_t BAR_DS = BAR_DP + 8;          // dS^T(i) written
+  constexpr uint32_t BAR_ACC = BAR_DS + 8;         // dV and dK complete
+  constexpr uint32_t BAR_TAIL = BAR_ACC + 8;
+  constexpr uint32_t BAR_VEC = BAR_TAIL + 8;       // this Q tile's LSE / Delta in smem (4 warps)
+  constexpr uint32_t TMEM_SLOT = L::kOffMisc;
+  constexpr uint32_t ABORT = L::kOffMisc + 4;
+  static_assert(BAR_VEC + 8 <= L::kOffMisc, "barrier area");
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint64_t tmo = p.timeout_ns;
+  const BwdUnit U = bwd_unit(p, false);        // causal: earlier K/V tiles see more queries and run first
+  const int nt = (p.S + 127) / 128;
+  const int k0 = U.t * 128;
+  const int k_rows = min(128, p.S - k0);
+  const int qt0 = p.causal ? U.t : 0;         // Q tiles with a query at or after k0
+  const int n = nt - qt0;
+  const int row_base = U.b * p.S;
+
+  if (threadIdx.x == 0) {
+    mbar_init(sb + BAR_KV, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(sb + BAR_QF + 8 * s, 1);
+      mbar_init(sb + BAR_QE + 8 * s, 1);
+      mbar_init(sb + BAR_OF + 8 * s, 1);
+      mbar_init(sb + BAR_OE + 8 * s, 1);
+    }
+    mbar_init(sb + BAR_S, 1);
+    mbar_init(sb + BAR_P, 4);
+    mbar_init(sb + BAR_DP, 1);
+    mbar_init(sb + BAR_DS, 4);
+    mbar_init(sb + BAR_ACC, 1);
+    mbar_init(sb + BAR_TAIL, 1);
+    mbar_init(sb + BAR_VEC, 4);
+    st_shared_volatile(sb + ABORT, 0u);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(sb + TMEM_SLOT, kBwdTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ld_shared_volatile(sb + TMEM_SLOT);
+  const uint32_t abort_flag = sb + ABORT;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&p.tm_q);
+      tma_prefetch_desc(&p.tm_k);
+      tma_prefetch_desc(&p.tm_v);
+      tma_prefetch_desc(&p.tm_do);
+      mbar_arrive_expect_tx(sb + BAR_KV, 2 * L::kTileBytes);
+      for (int hf = 0; hf < L::kHalves; ++hf) {
+        tma_load_3d(sb + L::kOffA + hf * L::kBoxBytes, &p.tm_k, hf * 64, U.h, row_base + k0, sb + BAR_KV);
+        tma_load_3d(sb + L::kOffB + hf * L::kBoxBytes, &p.tm_v, hf * 64, U.h, row_base + k0, sb + BAR_KV);
+      }
+      for (int i = 0; i < n; ++i) {
+        const int st = i & 1;
+        const uint32_t ph = (i >> 1) & 1;
+        const int qrow = row_base + (qt0 + i) * 128;
+        if (!mbar_wait(sb + BAR_QE + 8 * st, ph ^ 1, abort_flag, tmo, SITE_PRODUCER)) break;
+        mbar_arrive_expect_tx(sb + BAR_QF + 8 * st, L::kTileBytes);
+        for (int hf = 0; hf < L::kHalves; ++hf)
+          tma_load_3d(sb + L::kOffC + st * L::kTileBytes + hf * L::kBoxBytes, &p.tm_q, hf * 64, U.h, qrow,
+                      sb + BAR_QF + 8 * st);
+        if (!mbar_wait(sb + BAR_OE + 8 * st, ph ^ 1, abort_flag, tmo, SITE_PRODUCER)) break;
+        mbar_arrive_expect_tx(sb + BAR_OF + 8 * st, L::kTileBytes);
+        for (int hf = 0; hf < L::kHalves; ++hf)
+          tma_load_3d(sb + L::kOffE + st * L::kTileBytes + hf * L::kBoxBytes, &p.tm_do, hf * 64, U.h, qrow,
+                      sb + BAR_OF + 8 * st);
+      }
+      for (int st = 0; st < 2; ++st) {
+        const int uses = n > st ? (n - 1 - st) / 2 + 1 : 0;
+        if (uses == 0) continue;
+        const uint32_t ph = (uses - 1) & 1;
+        mbar_wait(sb + BAR_QE + 8 * st, ph, 0u, tmo, SITE_TAIL);
+        mbar_wait(sb + BAR_OE + 8 * st, ph, 0u, tmo, SITE_TAIL);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint64_t dK = smem_desc_sw128(sb + L::kOffA, 16, 1024);
+      const uint64_t dV = smem_desc_sw128(sb + L::kOffB, 16, 1024);
+      const uint64_t dQk = smem_desc_sw128(sb + L::kOffC, 16, 1024);                 // K-major (S^T)
+      const uint64_t dQmn = smem_desc_sw128(sb + L::kOffC, L::kBoxBytes, 1024);      // MN-major (dK)
+      const uint64_t dOk = smem_desc_sw128(sb + L::kOffE, 16, 1024);                 // K-major (dP^T)
+      const uint64_t dOmn = smem_desc_sw128(sb + L::kOffE, L::kBoxBytes, 1024);      // MN-major (dV)
+      auto issue_ss = [&](uint32_t d, uint64_t a0, uint64_t b0) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk >> 2) * L::kBoxBytes + (kk & 3) * 32) >> 4;
+          mma_ss(d, a0 + off, b0 + off, IDESC_SS, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_acc = [&](uint32_t d, uint32_t a_tmem, uint64_t b0, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(d, a_tmem + kk * 8, b0 + ((kk * 2048) >> 4), IDESC_ACC, (acc || kk > 0) ? 1u : 0u);
+      };
+      auto stage_off = [&](int st) { return static_cast<uint64_t>((st * L::kTileBytes) >> 4); };
+      bool ok = n > 0 && mbar_wait_spin(sb + BAR_KV, 0, abort_flag, tmo, SITE_MMA);
+      if (ok) ok = mbar_wait_spin(sb + BAR_QF, 0, abort_flag, tmo, SITE_MMA);
+      if (ok) {
+        tc_fence_after();
+        issue_ss(tmem, opaque_u64(dK), opaque_u64(dQk + stage_off(0)));
+        mma_commit(sb + BAR_S);
+      }
+      if (ok) ok = mbar_wait_spin(sb + BAR_OF, 0, abort_flag, tmo, SITE_MMA);
+      if (ok) {
+        tc_fence_after();
+        issue_ss(tmem + 128, opaque_u64(dV), opaque_u64(dOk + stage_off(0)));
+        mma_commit(sb + BAR_DP);
+      }
+      for (int i = 0; ok && i < n; ++i) {
+        const int st = i & 1, st1 = (i + 1) & 1;
+        const uint32_t ph1 = ((i + 1) >> 1) & 1;
+        const bool more = i + 1 < n;
+        // dV (+)= P^T dO: P^T (bf16 pairs) from TMEM over S^T, dO MN-major
+        if (!mbar_wait_spin(sb + BAR_P, i & 1, abort_flag, tmo, SITE_MMA)) break;
+        tc_fence_after();
+        issue_acc(tmem + 256, tmem, opaque_u64(dOmn + stage_off(st)), i > 0);
+        if (more) {   // P^T(i) is consumed in order before S^T(i+1) overwrites it
+          if (!mbar_wait_spin(sb + BAR_QF + 8 * st1, ph1, abort_flag, tmo, SITE_MMA)) break;
+          tc_fence_after();
+          issue_ss(tmem, opaque_u64(dK), opaque_u64(dQk + stage_off(st1)));
+          mma_commit(sb + BAR_S);
+        }
+        // dK (+)= dS^T Q: dS^T (bf16 pairs) from TMEM over dP^T, Q MN-major
+        if (!mbar_wait_spin(sb + BAR_DS, i & 1, abort_flag, tmo, SITE_MMA)) break;
+        tc_fence_after();
+        issue_acc(tmem + 256 + D, tmem + 128, opaque_u64(dQmn + stage_off(st)), i > 0);
+        mma_commit(sb + BAR_QE + 8 * st);
+        mma_commit(sb + BAR_OE + 8 * st);
+        if (more) {
+          if (!mbar_wait_spin(sb + BAR_OF + 8 * st1, ph1, abort_flag, tmo, SITE_MMA)) break;
+          tc_fence_after();
+          issue_ss(tmem + 128, opaque_u64(dV), opaque_u64(dOk + stage_off(st1)));
+          mma_commit(sb + BAR_DP);
+        }
+      }
+      if (n > 0) mma_commit(sb + BAR_ACC);
+      mma_commit(sb + BAR_TAIL);
+      mbar_wait(sb + BAR_TAIL, 0, 0u, tmo, SITE_TAIL);
+    }
+  } else {
+    // ------------------------------------------------------------ row threads (one key each)
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const int tid = threadIdx.x - 64;            // 0..127 across the four row warps
+    const int k_pos = k0 + row;
+    const bool row_valid = row < k_rows;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t tS = tmem + lane_base;
+    const uint32_t tDP = tmem + lane_base + 128;
+    const uint32_t tDV = tmem + lane_base + 256;
+    const uint32_t tDK = tmem + lane_base + 256 + D;
+    const float c = p.scale_log2;
+    const long long vbase = (static_cast<long long>(U.b) * p.H + U.h) * p.S;
+    bool ok = true;
+    for (int i = 0; ok && i < n; ++i) {
+      const int q0 = (qt0 + i) * 128;
+      // this Q tile's log2-domain LSE and Delta, one value per row thread;
+      // queries past the sequence get LSE = +inf, i.e. P = 0
+      const uint32_t vec = sb + L::kOffVec + (i & 1) * 1024;
+      {
+        const int q = q0 + tid;
+        st_shared_f32(vec + 4 * tid, q < p.S ? p.lse[vbase + q] * 1.4426950408889634f : INFINITY);
+        st_shared_f32(vec + 512 + 4 * tid, q < p.S ? p.delta[vbase + q] : 0.f);
+      }
+      // Every row warp has finished reading the previous use of this buffer
+      // (tile i-2) before it writes tile i's values, and the bounded barrier
+      // below publishes them; no unbounded named barrier.
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sb + BAR_VEC);
+      bool w = mbar_wait(sb + BAR_VEC, i & 1, abort_flag, tmo, SITE_SOFTMAX);
+      if (__any_sync(0xffffffffu, !w)) { ok = false; break; }
+      w = mbar_wait(sb + BAR_S, i & 1, abort_flag, tmo, SITE_SOFTMAX);
+      if (__any_sync(0xffffffffu, !w)) { ok = false; break; }
+      __syncwarp();
+      tc_fence_after();
+      uint32_t s[128];
+      tmem_ld128_wait(tS, s);
+      // P^T[k][q] = 2^(S^T*c - lse2[q]) for the queries that see key k
+      const int qlim = p.causal ? k_pos - q0 : 0;   // queries q < qlim do not see this key
+#pragma unroll
+      for (int q = 0; q < 128; ++q) {
+        const float pv = ex2_approx(__uint_as_float(s[q]) * c - ld_shared_f32(vec + 4 * q));
+        s[q] = __float_as_uint(q >= qlim ? pv : 0.f);
+      }
+#pragma unroll
+      for (int c0 = 0; c0 < 128; c0 += 32) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) pk[k] = pack_bf16x2(__uint_as_float(s[c0 + 2 * k]), __uint_as_float(s[c0 + 2 * k + 1]));
+        tmem_st16(tS + c0 / 2, pk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sb + BAR_P);
+      w = mbar_wait(sb + BAR_DP, i & 1, abort_flag, tmo, SITE_SOFTMAX);
+      if (__any_sync(0xffffffffu, !w)) { ok = false; break; }
+      __syncwarp();
+      tc_fence_after();
+      // dS^T = P^T * (dP^T - delta[q]), bf16 pairs over the dP^T columns read
+#pragma unroll
+      for (int c0 = 0; c0 < 128; c0 += 32) {
+        uint32_t dp[32];
+        tmem_ld32_wait(tDP + c0, dp);
+        uint32_t pk[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const int q = c0 + 2 * k;
+          const float d0 = __uint_as_float(s[q]) * (__uint_as_float(dp[2 * k]) - ld_shared_f32(vec + 512 + 4 * q));
+          const float d1 =
+              __uint_as_float(s[q + 1]) * (__uint_as_float(dp[2 * k + 1]) - ld_shared_f32(vec + 512 + 4 * (q + 1)));
+          pk[k] = pack_bf16x2(d0, d1);
+        }
+        tmem_st16(tDP + c0 / 2, pk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sb + BAR_DS);
+    }
+    if (ok && n > 0) {
+      const bool w = mbar_wait(sb + BAR_ACC, 0, abort_flag, tmo, SITE_EPILOGUE);
+      if (__any_sync(0xffffffffu, !w)) ok = false;
+      __syncwarp();
+      tc_fence_after();
+    }
+    if (ok) {
+      const long long roff = ((static_cast<long long>(U.b) * p.S + k_pos) * p.H + U.h) * D;
+      for (int which = 0; which < 2; ++which) {   // 0: dV, 1: dK (times the softmax scale)
+        const float mul = which == 0 ? 1.0f : p.scale;
+        __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(which == 0 ? p.dv : p.dk) + roff;
+        const uint32_t tsrc = which == 0 ? tDV : tDK;
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t o[32];
+          if (n > 0) {
+            tmem_ld32_wait(tsrc + c0, o);
+          } else {
+#pragma unroll
+            for (int k = 0; k < 32; ++k) o[k] = 0u;
+          }
+          if (row_valid) {
+            uint4 *d4 = reinterpret_cast<uint4 *>(dst + c0);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              d4[k] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * k]) * mul, __uint_as_float(o[8 * k + 1]) * mul),
+                                 pack_bf16x2(__uint_as_float(o[8 * k + 2]) * mul, __uint_as_float(o[8 * k + 3]) * mul),
+                                 pack_bf16x2(__uint_as_float(o[8 * k + 4]) * mul, __uint_as_float(o[8 * k + 5]) * mul),
+                                 pack_bf16x2(__uint_as_float(o[8 * k + 6]) * mul, __uint_as_float(o[8 * k + 7]) * mul));
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kBwdTmemCols);
+  }
+}
+
+}  // namespace cpattn

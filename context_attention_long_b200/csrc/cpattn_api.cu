@@ -21,6 +21,7 @@
 #include "cpattn_internal.h"
 #include "cpattn_ptx.cuh"
 #include "attn_kernel.cuh"
+#include "attn_bwd_kernel.cuh"
 #include "merge_kernel.cuh"
 #include "permute_kernel.cuh"
 
@@ -180,6 +181,42 @@ static cudaError_t launch_merge_d(const MergeParams &p, cudaStream_t stream) {
 
 cudaError_t launch_lse_merge(const MergeParams &p, cudaStream_t stream) {
   return p.D == 128 ? launch_merge_d<128>(p, stream) : launch_merge_d<64>(p, stream);
+}
+
+template <int D>
+static cudaError_t launch_bwd_d(const BwdParams &p, cudaStream_t stream) {
+  static std::mutex mu;
+  static bool configured[kMaxDevices] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!configured[dev]) {
+      cudaError_t e = cudaFuncSetAttribute(attn_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           BwdSmem<D>::kAllocBytes);
+      if (e != cudaSuccess) return e;
+      e = cudaFuncSetAttribute(attn_bwd_dkv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               BwdSmem<D>::kAllocBytes);
+      if (e != cudaSuccess) return e;
+      configured[dev] = true;
+    }
+  }
+  const long long units = static_cast<long long>(p.B) * p.H * ((p.S + 127) / 128);
+  attn_bwd_dq_kernel<D><<<static_cast<unsigned>(units), kBwdThreads, BwdSmem<D>::kAllocBytes, stream>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  attn_bwd_dkv_kernel<D><<<static_cast<unsigned>(units), kBwdThreads, BwdSmem<D>::kAllocBytes, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attention_backward(const BwdParams &p, int D, const void *out, const void *dout, float *delta,
+                                      cudaStream_t stream) {
+  const long long rows = static_cast<long long>(p.B) * p.S * p.H;
+  attn_bwd_delta_kernel<<<grid_for(rows, 256 / 32), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16 *>(out), static_cast<const __nv_bfloat16 *>(dout), delta, p.B, p.S, p.H, D);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return D == 128 ? launch_bwd_d<128>(p, stream) : launch_bwd_d<64>(p, stream);
 }
 
 cudaError_t launch_permute(const PermuteParams &p, cudaStream_t stream) {
@@ -890,6 +927,50 @@ int cpattn_causal_unified_attention(const void *q, const void *k, const void *v,
                                     cpattn_stream_t stream) {
   return unified_common(q, k, v, out, lse, B, H, S, D, ring_degree, ulysses_degree, ring_lens, head_splits, workspace,
                         workspace_bytes, true, stream);
+}
+
+size_t cpattn_attention_backward_workspace_bytes(int B, int H, int S) {
+  if (B < 1 || H < 1 || S < 1) return 0;
+  return static_cast<size_t>(B) * H * S * sizeof(float);
+}
+
+int cpattn_attention_backward(const void *q, const void *k, const void *v, const void *out, const float *lse,
+                              const void *dout, void *dq, void *dk, void *dv, int B, int H, int S, int D,
+                              int causal, void *workspace, size_t workspace_bytes, cpattn_stream_t stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || lse == nullptr || dout == nullptr ||
+      dq == nullptr || dk == nullptr || dv == nullptr)
+    return CPATTN_ERR_NULL;
+  int st = check_attn_shape(B, H, S, D);
+  if (st != CPATTN_OK) return st;
+  if (workspace == nullptr || workspace_bytes < cpattn_attention_backward_workspace_bytes(B, H, S))
+    return CPATTN_ERR_WORKSPACE;
+  const void *ptrs[8] = {q, k, v, out, dout, dq, dk, dv};
+  for (const void *ptr : ptrs)
+    if (!aligned16(ptr)) return CPATTN_ERR_ALIGNMENT;
+  if (!aligned4(lse) || !aligned4(workspace)) return CPATTN_ERR_ALIGNMENT;
+  st = check_device(nullptr);
+  if (st != CPATTN_OK) return st;
+  std::unique_ptr<BwdParams> P(new BwdParams);
+  std::memset(P.get(), 0, sizeof(BwdParams));
+  const long long rows = static_cast<long long>(B) * S;
+  if (!encode_rows_map(&P->tm_q, q, D, H, rows) || !encode_rows_map(&P->tm_k, k, D, H, rows) ||
+      !encode_rows_map(&P->tm_v, v, D, H, rows) || !encode_rows_map(&P->tm_do, dout, D, H, rows))
+    return CPATTN_ERR_CUDA;
+  P->lse = lse;
+  P->delta = static_cast<float *>(workspace);
+  P->dq = dq;
+  P->dk = dk;
+  P->dv = dv;
+  P->B = B;
+  P->H = H;
+  P->S = S;
+  P->causal = causal ? 1 : 0;
+  P->scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+  P->scale_log2 = static_cast<float>((1.0 / std::sqrt(static_cast<double>(D))) * 1.4426950408889634);
+  P->timeout_ns = wait_timeout_ns();
+  return launch_attention_backward(*P, D, out, dout, static_cast<float *>(workspace), stream) == cudaSuccess
+             ? CPATTN_OK
+             : CPATTN_ERR_CUDA;
 }
 
 int cpattn_exchange_bytes(int mode, int B, int H, int S, int D, int elem_bytes, int degree, const int *seq_splits,

@@ -87,6 +87,22 @@ struct AttnParams {
 // float32 partial outputs (ring step) instead of bf16.
 cudaError_t launch_attention(const AttnParams &p, int D, bool out_f32, cudaStream_t stream);
 
+// ---------------------------------------------------------------- backward
+// Gradient of attention over full [B, S, H, D] tensors (rows = B*S).
+struct alignas(64) BwdParams {
+  CUtensorMap tm_q, tm_k, tm_v, tm_do;   // 3-D maps over [rows, H, D] bf16, box {64, 1, 128}, 128B swizzle
+  const float *lse;                      // [B, H, S] natural log, from the forward
+  const float *delta;                    // [B, H, S] rowsum(dO * O)
+  void *dq, *dk, *dv;                    // [B, S, H, D] bf16
+  int B, H, S;
+  int causal;
+  float scale_log2;                      // D**-0.5 * log2(e)
+  float scale;                           // D**-0.5
+  unsigned long long timeout_ns;
+};
+cudaError_t launch_attention_backward(const BwdParams &p, int D, const void *out, const void *dout, float *delta,
+                                      cudaStream_t stream);
+
 // ---------------------------------------------------------------- LSE merge
 struct MergeParams {
   const float *part_out;  // P x [B, S, H, D]

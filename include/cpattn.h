@@ -299,6 +299,39 @@ int cpattn_causal_unified_attention(const void *q, const void *k, const void *v,
                                     int ulysses_degree, const int *ring_lens, const int *head_splits,
                                     void *workspace, size_t workspace_bytes, cpattn_stream_t stream);
 
+/* -------------------------------------------------------------- backward */
+
+/*
+ * Gradient of attention with respect to Q, K and V, for training over long
+ * contexts ([USP] sections 1 and 7).  It is the derivative of the forward
+ * definition; the pages print no backward formulas.  Per (batch, head), with
+ * S = Q K^T * D**-0.5, P = softmax(S) recomputed from the forward's LSE, and
+ * dO the upstream gradient of the output O:
+ *   dV = P^T dO,  dS = P * (dO V^T - rowsum(dO * O)),
+ *   dQ = dS K * D**-0.5,  dK = dS^T Q * D**-0.5.
+ * The ring, Ulysses and unified paths compute this same attention, so this is
+ * their gradient too; causal = 1 applies the cpattn_causal_* mask (key j
+ * visible to query i iff j <= i).
+ *
+ *   q, k, v, out, dout  [B, S, H, D] bf16 device, read only (out: the forward
+ *                       output; dout: the gradient of the loss with respect
+ *                       to it).
+ *   lse                 [B, H, S] float32 device, natural log (the forward's).
+ *   dq, dk, dv          [B, S, H, D] bf16 device, written.
+ *   workspace           device, at least
+ *                       cpattn_attention_backward_workspace_bytes(B, H, S)
+ *                       bytes, 4-byte aligned (holds rowsum(dO * O)).
+ * Three launches on `stream`: the row sums, a dQ kernel (one CTA per Q tile,
+ * walking the K/V tiles) and a dK/dV kernel (one CTA per K/V tile, walking the
+ * Q tiles); no atomics.  Errors: NULL, SHAPE, WORKSPACE, ALIGNMENT,
+ * UNSUPPORTED, CUDA.
+ */
+size_t cpattn_attention_backward_workspace_bytes(int B, int H, int S);
+int cpattn_attention_backward(const void *q, const void *k, const void *v, const void *out,
+                              const float *lse, const void *dout, void *dq, void *dk, void *dv,
+                              int B, int H, int S, int D, int causal, void *workspace,
+                              size_t workspace_bytes, cpattn_stream_t stream);
+
 /* ------------------------------------------------- no-allocation variant */
 
 /*

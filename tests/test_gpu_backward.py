@@ -1,0 +1,99 @@
+"""Parity of the attention backward (through the C ABI) with the fp64
+backward oracle: dQ, dK and dV for seeded inputs and a seeded upstream
+gradient, causal and not, over tile-spanning and ragged shapes, D = 64 and
+128, S = 1, and the image-DiT workload on sampled rows.  The forward output
+and LSE come from the library's own forward.
+
+Tolerance: every gradient is compared relative to its largest reference
+entry g = max|ref|: max-abs error <= 2e-2 * g and mean-abs error <= 2e-3 * g.
+P and dS are rounded to bf16 (relative 2^-9) before their MMAs and the
+gradients are stored in bf16, as the forward's output is, so the bar is the
+forward's bar scaled to the gradient's size."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from context_attention_long_b200 import api, build, inputs
+
+from gpu_util import f64_of, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    build.build()
+
+
+def _no_timeouts():
+    st, code = api.cpattn_device_status()
+    assert st == 0 and code == 0, f"device wait expired: code {code:#x}"
+
+
+def assert_grad_close(got, ref, what):
+    got, ref = np.asarray(got, dtype=np.float64), np.asarray(ref, dtype=np.float64)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite"
+    g = max(np.max(np.abs(ref)), 1e-30)
+    err = np.abs(got - ref)
+    assert err.max() <= 2e-2 * g, f"{what}: max-abs {err.max():.3e} vs {g:.3e}"
+    assert err.mean() <= 2e-3 * g, f"{what}: mean-abs {err.mean():.3e} vs {g:.3e}"
+
+
+def _run(B, S, H, D, causal, seed):
+    qb, kb, vb = inputs.make_qkv(B, S, H, D, seed, D == 128)
+    rng = np.random.Generator(np.random.PCG64(seed + 1))
+    dob = inputs.f32_to_bf16_bits(rng.standard_normal((B, S, H, D)).astype(np.float32))
+    q, k, v, do = (to_dev(x) for x in (qb, kb, vb, dob))
+    fwd = api.cpattn_causal_ring_attention if causal else api.cpattn_ring_attention
+    out, lse = fwd(q, k, v, 1)
+    dq, dk, dv = api.cpattn_attention_backward(q, k, v, out, lse, do, causal=causal)
+    torch.cuda.synchronize()
+    _no_timeouts()
+    return (qb, kb, vb, dob), (dq, dk, dv)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("B,S,H,D", [(1, 256, 2, 64), (2, 300, 3, 128), (1, 129, 2, 128), (1, 1, 1, 64),
+                                     (1, 640, 2, 128)])
+def test_backward_matches_oracle(B, S, H, D, causal):
+    bits, grads = _run(B, S, H, D, causal, 31 + S)
+    q, k, v, do = (inputs.bf16_bits_to_f64(x) for x in bits)
+    refs = oracle.attention_backward(q, k, v, do, causal=causal)
+    for name, got, ref in zip(("dq", "dk", "dv"), grads, refs):
+        assert_grad_close(f64_of(got), ref, f"{name} B{B} S{S} H{H} D{D} causal={causal}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_dit_workload_sampled_heads(causal):
+    """Image-DiT shapes (B1 H24 S4608 D128) in full on the GPU; the oracle
+    checks three heads in full (its cost grows with S^2 per head)."""
+    cfg, qb, kb, vb = inputs.config_inputs("dit")
+    B, S, H, D = qb.shape
+    rng = np.random.Generator(np.random.PCG64(77))
+    dob = inputs.f32_to_bf16_bits(rng.standard_normal((B, S, H, D)).astype(np.float32))
+    q, k, v, do = (to_dev(x) for x in (qb, kb, vb, dob))
+    fwd = api.cpattn_causal_ring_attention if causal else api.cpattn_ring_attention
+    out, lse = fwd(q, k, v, cfg["ring_degree"])
+    dq, dk, dv = api.cpattn_attention_backward(q, k, v, out, lse, do, causal=causal)
+    torch.cuda.synchronize()
+    _no_timeouts()
+    pos = np.arange(S) if causal else None
+    for h in (0, 11, 23):
+        ref = oracle.attention_backward_rows(*(inputs.bf16_bits_to_f64(x[0, :, h]) for x in (qb, kb, vb, dob)),
+                                             pos, pos)
+        for name, got, r in zip(("dq", "dk", "dv"), (dq, dk, dv), ref):
+            assert_grad_close(f64_of(got)[0, :, h], r, f"dit {name} head {h} causal={causal}")
+
+
+def test_backward_is_deterministic_and_validates():
+    bits, g1 = _run(1, 384, 2, 128, True, 5)
+    _, g2 = _run(1, 384, 2, 128, True, 5)
+    for a, b in zip(g1, g2):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    lib = api._native.load()
+    F = g1[0].data_ptr()
+    assert lib.cpattn_attention_backward(F, F, F, F, None, F, F, F, F, 1, 2, 384, 128, 0, F, 1 << 20, None) == 1
+    assert lib.cpattn_attention_backward(F, F, F, F, F, F, F, F, F, 1, 2, 384, 128, 0, F, 16, None) == 8
