@@ -244,7 +244,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true",
                     help="time every workload's paths (one JSON line per path) instead of the step")
-    ap.add_argument("--kernel", default=None, choices=["ring", "causal_ring", "head_sharded", "permute", "permute_qkv", "merge", "ring_step"],
+    ap.add_argument("--kernel", default=None, choices=["ring", "causal_ring", "head_sharded", "permute", "permute_qkv", "merge", "ring_step", "backward"],
                     help="profiling mode: run only this kernel (warmup + steps launches) on the workload")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -431,6 +431,7 @@ def main():
     if not args.no_breakdown:
         kernels.update(breakdown(api, torch, dev, flush, peaks, inputs))
         kernels.update(causal_paths(api, torch, flush, peaks, q, k, v, P, U))
+        kernels.update(backward_paths(api, torch, flush, peaks, q, k, v, P))
 
     # Accounting: what P GPUs would exchange per rank for this workload (on one
     # GPU the exchanges are emulated in memory).
@@ -512,6 +513,49 @@ def causal_paths(api, torch, flush, peaks, q, k, v, P, U):
         tf = flops / (ms * 1e-3) / 1e12
         res[name] = {"ms": ms, "TFLOP/s": tf, "frac_bf16_peak": tf / peak_tf,
                      "flops": "4*D per visible (query, key) pair: 2*B*H*D*S*(S+1)"}
+    return res
+
+
+def backward_flops(B, H, S, D, causal):
+    """2.5x the forward's count (five S-sized matmuls against two), the usual
+    accounting for an attention backward; causal: visible pairs only."""
+    return 2.5 * (causal_flops(B, H, S, D) if causal else 4.0 * B * H * S * S * D)
+
+
+def backward_paths(api, torch, flush, peaks, q, k, v, P):
+    """The attention backward on the bench workload (dQ, dK, dV from the
+    forward's output and LSE and a seeded upstream gradient), non-causal and
+    causal, each rep after an L2 flush."""
+    B, S, H, D = q.shape
+    stream = torch.cuda.current_stream()
+    gen = torch.Generator(device=q.device).manual_seed(7)
+    do = torch.randn(q.shape, generator=gen, device=q.device).to(torch.bfloat16)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    ws = torch.empty(api.cpattn_attention_backward_workspace_bytes(B, H, S), dtype=torch.uint8, device=q.device)
+    peak_tf = float(peaks["bf16_tflops"])
+    res = {}
+    for causal in (False, True):
+        fwd = api.cpattn_causal_ring_attention if causal else api.cpattn_ring_attention
+        out, lse = fwd(q, k, v, P, stream=stream)
+
+        def run():
+            api.cpattn_attention_backward(q, k, v, out, lse, do, causal, dq, dk, dv, ws, stream=stream)
+
+        run()
+        times = []
+        for _ in range(10):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            run()
+            b.record(stream)
+            b.synchronize()
+            times.append(a.elapsed_time(b))
+        ms = float(np.median(times))
+        tf = backward_flops(B, H, S, D, causal) / (ms * 1e-3) / 1e12
+        res["attention_backward" + ("_causal" if causal else "")] = {
+            "ms": ms, "TFLOP/s": tf, "frac_bf16_peak": tf / peak_tf,
+            "flops": "2.5x the forward's (10*B*H*S^2*D; causal: visible pairs)", "launches": 3}
     return res
 
 
@@ -634,6 +678,19 @@ def run_sweep(args):
             paths.append((f"causal Ulysses {U}" + (" (Anything)" if seq else "") + " flow",
                           lambda: api.cpattn_causal_ulysses_attention(qf, kf, vf, B, S, H, D, U, seq, heads,
                                                                       workspace=ws), cflops))
+        if name in ("dit", "hires", "video"):
+            gen = torch.Generator(device=dev).manual_seed(7)
+            do = torch.randn(q.shape, generator=gen, device=dev).to(torch.bfloat16)
+            bq, bk, bv = (torch.empty_like(q) for _ in range(3))
+            bws = torch.empty(api.cpattn_attention_backward_workspace_bytes(B, H, S), dtype=torch.uint8, device=dev)
+            o_f, l_f = api.cpattn_ring_attention(q, k, v, P, lens)
+            o_c, l_c = api.cpattn_causal_ring_attention(q, k, v, P, lens)
+            paths.append(("attention backward (dQ, dK, dV)",
+                          lambda: api.cpattn_attention_backward(q, k, v, o_f, l_f, do, False, bq, bk, bv, bws),
+                          backward_flops(B, H, S, D, False)))
+            paths.append(("causal attention backward",
+                          lambda: api.cpattn_attention_backward(q, k, v, o_c, l_c, do, True, bq, bk, bv, bws),
+                          backward_flops(B, H, S, D, True)))
         for entry in paths:
             label, fn = entry[0], entry[1]
             ms = timeit(fn)
@@ -668,6 +725,10 @@ def run_single_kernel(args):
     elif args.kernel == "head_sharded":
         yq, yk, yv = (api.cpattn_ulysses_permute(t.reshape(-1), B, S, H, D, U) for t in (q, k, v))
         fn = lambda: api.cpattn_head_sharded_attention(yq, yk, yv, B, S, H, D, U)
+    elif args.kernel == "backward":
+        out, lse = api.cpattn_ring_attention(q, k, v, P)
+        do = torch.randn(q.shape, device=dev).to(torch.bfloat16)
+        fn = lambda: api.cpattn_attention_backward(q, k, v, out, lse, do)
     elif args.kernel == "permute_qkv":
         qf, kf, vf = q.reshape(-1), k.reshape(-1), v.reshape(-1)
         yq, yk, yv = torch.empty_like(qf), torch.empty_like(kf), torch.empty_like(vf)

@@ -563,12 +563,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __gr
       tc_fence_after();
       uint32_t s[128];
       tmem_ld128_wait(tS, s);
-      // P^T[k][q] = 2^(S^T*c - lse2[q]) for the queries that see key k
+      // P^T[k][q] = 2^(S^T*c - lse2[q]) for the queries that see key k.  The
+      // per-query values are read as float4 through a plain shared-memory
+      // pointer (the barrier waits above are compiler fences), so the loads
+      // schedule freely around the exponentials.
+      const float4 *lse4 = reinterpret_cast<const float4 *>(smem_raw + (vec - smem_u32(smem_raw)));
+      const float4 *del4 = lse4 + 32;
       const int qlim = p.causal ? k_pos - q0 : 0;   // queries q < qlim do not see this key
 #pragma unroll
-      for (int q = 0; q < 128; ++q) {
-        const float pv = ex2_approx(__uint_as_float(s[q]) * c - ld_shared_f32(vec + 4 * q));
-        s[q] = __float_as_uint(q >= qlim ? pv : 0.f);
+      for (int q4 = 0; q4 < 32; ++q4) {
+        const float4 l = lse4[q4];
+        const float lv[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int q = 4 * q4 + e;
+          const float pv = ex2_approx(__uint_as_float(s[q]) * c - lv[e]);
+          s[q] = __float_as_uint(q >= qlim ? pv : 0.f);
+        }
       }
 #pragma unroll
       for (int c0 = 0; c0 < 128; c0 += 32) {
@@ -592,12 +603,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __gr
         tmem_ld32_wait(tDP + c0, dp);
         uint32_t pk[16];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const int q = c0 + 2 * k;
-          const float d0 = __uint_as_float(s[q]) * (__uint_as_float(dp[2 * k]) - ld_shared_f32(vec + 512 + 4 * q));
-          const float d1 =
-              __uint_as_float(s[q + 1]) * (__uint_as_float(dp[2 * k + 1]) - ld_shared_f32(vec + 512 + 4 * (q + 1)));
-          pk[k] = pack_bf16x2(d0, d1);
+        for (int k4 = 0; k4 < 8; ++k4) {
+          const float4 dl = del4[(c0 >> 2) + k4];
+          const int q = c0 + 4 * k4;
+          pk[2 * k4] = pack_bf16x2(__uint_as_float(s[q]) * (__uint_as_float(dp[4 * k4]) - dl.x),
+                                   __uint_as_float(s[q + 1]) * (__uint_as_float(dp[4 * k4 + 1]) - dl.y));
+          pk[2 * k4 + 1] = pack_bf16x2(__uint_as_float(s[q + 2]) * (__uint_as_float(dp[4 * k4 + 2]) - dl.z),
+                                       __uint_as_float(s[q + 3]) * (__uint_as_float(dp[4 * k4 + 3]) - dl.w));
         }
         tmem_st16(tDP + c0 / 2, pk);
       }
