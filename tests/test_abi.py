@@ -178,3 +178,22 @@ def test_causal_entry_points_validate_like_their_namesakes(lib):
     assert v(ws=None) == WS and v(R=3) == INDIV
     if not torch.cuda.is_available():
         assert r() == CUDA       # valid arguments, no device: fails before any launch
+
+
+def test_backward_validation(lib):
+    need = lib.cpattn_attention_backward_workspace_bytes(1, 2, 256)
+    assert need == 1 * 2 * 256 * 4
+    assert lib.cpattn_attention_backward_workspace_bytes(0, 2, 256) == 0
+
+    def f(q=FAKE, lse=FAKE, dq=FAKE, D=64, S=256, ws=FAKE, nbytes=need):
+        return lib.cpattn_attention_backward(q, FAKE, FAKE, FAKE, lse, FAKE, dq, FAKE, FAKE, 1, 2, S, D, 1, ws,
+                                             nbytes, None)
+    assert f(q=None) == NULL
+    assert f(lse=None) == NULL
+    assert f(D=96) == SHAPE
+    assert f(S=0) == SHAPE
+    assert f(ws=None) == WS
+    assert f(nbytes=need - 4) == WS
+    assert f(dq=FAKE_MIS) == ALIGN
+    if not torch.cuda.is_available():
+        assert f() == CUDA
