@@ -454,6 +454,16 @@ def main():
                 "us": {m: (None if pl[m]["seconds"] is None else round(pl[m]["seconds"] * 1e6, 1))
                        for m in ("ring", "ulysses", "kv_gather")}}
 
+    # Mean absolute difference of the sharded paths' outputs from unsharded
+    # attention (the fused kernel with one shard), in the MAE style of the
+    # pages' sharded-vs-unsharded check; the paths differ only in rounding order.
+    mono, _ = api.cpattn_ring_attention(q, k, v, 1, stream=stream)
+    torch.cuda.synchronize()
+    mono_f = mono.float()
+    mae = {"ring": float((out_r.float() - mono_f).abs().mean()),
+           "ulysses": float((out_u.view(B, S, H, D).float() - mono_f).abs().mean())}
+    del mono, mono_f
+
     st, code = api.cpattn_device_status()
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -462,6 +472,7 @@ def main():
         "config": config_block(cfg), "roofline": roofline, "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks.summary(t_wall0, t_wall1), "e2e": e2e, "kernels": kernels,
         "device_status": code, "exchange_bytes_per_rank": exch, "exchange_plan": exch_plan,
+        "mae_vs_unsharded": mae,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, qb, kb, vb)
@@ -643,6 +654,8 @@ def run_sweep(args):
         lens = None
         if name == "anything":
             lens = inputs.ring_anything_lens(S, P, cfg["seed"])
+        paths.append(("unsharded (the fused kernel with one shard: the single-GPU baseline)",
+                      lambda: api.cpattn_ring_attention(q, k, v, 1, want_lse=True)))
         paths.append((f"ring fused P={P}" + (" (Ring Anything)" if lens else ""),
                       lambda: api.cpattn_ring_attention(q, k, v, P, lens, want_lse=True)))
         paths.append((f"causal ring fused P={P}" + (" (Ring Anything)" if lens else ""),
