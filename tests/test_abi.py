@@ -30,7 +30,7 @@ def declared_functions():
     return sorted(set(re.findall(r"\b(cpattn_[a-z_0-9]+)\s*\(", text)))
 
 
-def test_header_declares_the_north_star_calls():
+def test_header_declares_the_hot_path_calls():
     names = declared_functions()
     for required in ("cpattn_ring_attention", "cpattn_lse_merge", "cpattn_ulysses_permute",
                      "cpattn_ulysses_unpermute", "cpattn_kv_gather_attention"):
