@@ -567,6 +567,31 @@ def backward_paths(api, torch, flush, peaks, q, k, v, P):
         res["attention_backward" + ("_causal" if causal else "")] = {
             "ms": ms, "TFLOP/s": tf, "frac_bf16_peak": tf / peak_tf,
             "flops": "2.5x the forward's (10*B*H*S^2*D; causal: visible pairs)", "launches": 3}
+    # the backward of the Ulysses flow (rank buffers; B = 1 here, so they are the full tensors)
+    U = 4
+    out, lse = api.cpattn_ulysses_attention(q.reshape(-1), k.reshape(-1), v.reshape(-1), B, S, H, D, U, stream=stream)
+    wsu = torch.empty(api.cpattn_ulysses_attention_backward_workspace_bytes(B, H, S, D), dtype=torch.uint8,
+                      device=q.device)
+
+    def run_u():
+        api.cpattn_ulysses_attention_backward(q.reshape(-1), k.reshape(-1), v.reshape(-1), out, lse, do.reshape(-1),
+                                              B, S, H, D, U, dq=dq.reshape(-1), dk=dk.reshape(-1), dv=dv.reshape(-1),
+                                              workspace=wsu, stream=stream)
+
+    run_u()
+    times = []
+    for _ in range(10):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        run_u()
+        b.record(stream)
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    ms = float(np.median(times))
+    tf = backward_flops(B, H, S, D, False) / (ms * 1e-3) / 1e12
+    res[f"ulysses_{U}_backward_flow"] = {"ms": ms, "TFLOP/s": tf, "frac_bf16_peak": tf / peak_tf,
+                                         "launches": 7, "note": "5 permuted in, backward of 4 head ranks, 3 permuted out"}
     return res
 
 

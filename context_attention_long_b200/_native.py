@@ -57,6 +57,10 @@ SIGNATURES = {
     "cpattn_attention_backward": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                           c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int,
                                           c_void_p, c_size_t, c_void_p]),
+    "cpattn_ulysses_attention_backward_workspace_bytes": (c_size_t, [c_int, c_int, c_int, c_int]),
+    "cpattn_ulysses_attention_backward": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                                  c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int,
+                                                  P_INT, P_INT, c_int, c_void_p, c_size_t, c_void_p]),
     "cpattn_ulysses_attention_noalloc": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                                  c_int, c_int, c_int, c_int, c_int, P_INT, P_INT, c_void_p]),
     "cpattn_front_loaded_splits": (c_int, [c_int, c_int, P_INT]),

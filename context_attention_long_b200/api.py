@@ -285,6 +285,27 @@ def cpattn_attention_backward(q, k, v, out, lse, dout, causal=False, dq=None, dk
     return dq, dk, dv
 
 
+def cpattn_ulysses_attention_backward_workspace_bytes(B, H, S, D) -> int:
+    return int(_native.load().cpattn_ulysses_attention_backward_workspace_bytes(B, H, S, D))
+
+
+def cpattn_ulysses_attention_backward(q, k, v, out, lse, dout, B, S, H, D, degree, seq_splits=None,
+                                      head_splits=None, causal=False, dq=None, dk=None, dv=None, workspace=None,
+                                      stream=None):
+    """Backward of the Ulysses flow on sequence-sharded rank buffers (flat
+    bf16); returns (dq, dk, dv) in the same layout."""
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    workspace = _workspace(cpattn_ulysses_attention_backward_workspace_bytes(B, H, S, D), q.device, workspace)
+    _check(_native.load().cpattn_ulysses_attention_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), B, H, S, D,
+        int(degree), _native.int_array(seq_splits), _native.int_array(head_splits), 1 if causal else 0,
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)),
+        "cpattn_ulysses_attention_backward")
+    return dq, dk, dv
+
+
 # Size of the library-held scratch of cpattn_ulysses_attention_noalloc
 # (CPATTN_NOALLOC_SCRATCH_BYTES in cpattn.h).
 NOALLOC_SCRATCH_BYTES = 64 << 20

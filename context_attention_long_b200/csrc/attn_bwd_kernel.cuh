@@ -88,17 +88,23 @@ __global__ void __launch_bounds__(256) attn_bwd_delta_kernel(const __nv_bfloat16
   }
 }
 
-// Units of both kernels: (b, h, 128-row tile) with the tile index fastest.
+// Units of both kernels: (problem, b, h, 128-row tile) with the tile index
+// fastest; problems occupy consecutive unit ranges.
 struct BwdUnit {
-  int b, h, t;
+  int pi, b, h, t;
 };
 __device__ __forceinline__ BwdUnit bwd_unit(const BwdParams &p, bool last_first) {
   const int nt = (p.S + 127) / 128;
   BwdUnit u;
-  const int t_in = blockIdx.x % nt;
-  const int bh = blockIdx.x / nt;
-  u.h = bh % p.H;
-  u.b = bh / p.H;
+  int pi = 0;
+  while (pi + 1 < p.n_prob && p.prob[pi + 1].unit_base <= static_cast<int>(blockIdx.x)) ++pi;
+  const int local = static_cast<int>(blockIdx.x) - p.prob[pi].unit_base;
+  const int H = p.prob[pi].H;
+  const int t_in = local % nt;
+  const int bh = local / nt;
+  u.pi = pi;
+  u.h = bh % H;
+  u.b = bh / H;
   u.t = last_first ? nt - 1 - t_in : t_in;
   return u;
 }
@@ -130,6 +136,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __gri
   const int lane = threadIdx.x & 31;
   const uint64_t tmo = p.timeout_ns;
   const BwdUnit U = bwd_unit(p, p.causal != 0);   // causal: heavier (later) Q tiles first
+  const BwdProblem &PB = p.prob[U.pi];
   const int q0 = U.t * 128;
   const int q_rows = min(128, p.S - q0);
   const int kv_len = p.causal ? min(p.S, q0 + q_rows) : p.S;   // keys at positions < kv_len
@@ -166,14 +173,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __gri
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      tma_prefetch_desc(&p.tm_q);
-      tma_prefetch_desc(&p.tm_k);
-      tma_prefetch_desc(&p.tm_v);
-      tma_prefetch_desc(&p.tm_do);
+      tma_prefetch_desc(&PB.tm_q);
+      tma_prefetch_desc(&PB.tm_k);
+      tma_prefetch_desc(&PB.tm_v);
+      tma_prefetch_desc(&PB.tm_do);
       mbar_arrive_expect_tx(sb + BAR_QD, 2 * L::kTileBytes);
       for (int hf = 0; hf < L::kHalves; ++hf) {
-        tma_load_3d(sb + L::kOffA + hf * L::kBoxBytes, &p.tm_q, hf * 64, U.h, row_base + q0, sb + BAR_QD);
-        tma_load_3d(sb + L::kOffB + hf * L::kBoxBytes, &p.tm_do, hf * 64, U.h, row_base + q0, sb + BAR_QD);
+        tma_load_3d(sb + L::kOffA + hf * L::kBoxBytes, &PB.tm_q, hf * 64, U.h, row_base + q0, sb + BAR_QD);
+        tma_load_3d(sb + L::kOffB + hf * L::kBoxBytes, &PB.tm_do, hf * 64, U.h, row_base + q0, sb + BAR_QD);
       }
       for (int j = 0; j < n; ++j) {
         const int st = j & 1;
@@ -181,12 +188,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __gri
         if (!mbar_wait(sb + BAR_KE + 8 * st, ph ^ 1, abort_flag, tmo, SITE_PRODUCER)) break;
         mbar_arrive_expect_tx(sb + BAR_KF + 8 * st, L::kTileBytes);
         for (int hf = 0; hf < L::kHalves; ++hf)
-          tma_load_3d(sb + L::kOffC + st * L::kTileBytes + hf * L::kBoxBytes, &p.tm_k, hf * 64, U.h,
+          tma_load_3d(sb + L::kOffC + st * L::kTileBytes + hf * L::kBoxBytes, &PB.tm_k, hf * 64, U.h,
                       row_base + j * 128, sb + BAR_KF + 8 * st);
         if (!mbar_wait(sb + BAR_VE + 8 * st, ph ^ 1, abort_flag, tmo, SITE_PRODUCER)) break;
         mbar_arrive_expect_tx(sb + BAR_VF + 8 * st, L::kTileBytes);
         for (int hf = 0; hf < L::kHalves; ++hf)
-          tma_load_3d(sb + L::kOffE + st * L::kTileBytes + hf * L::kBoxBytes, &p.tm_v, hf * 64, U.h,
+          tma_load_3d(sb + L::kOffE + st * L::kTileBytes + hf * L::kBoxBytes, &PB.tm_v, hf * 64, U.h,
                       row_base + j * 128, sb + BAR_VF + 8 * st);
       }
       // every stage's last release must arrive before the CTA exits
@@ -276,9 +283,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __gri
     const uint32_t tDP = tmem + lane_base + 128;
     const uint32_t tDQ = tmem + lane_base + 256;
     const float c = p.scale_log2;
-    const long long vi = (static_cast<long long>(U.b) * p.H + U.h) * p.S + q_pos;
-    const float lse2 = row_valid ? p.lse[vi] * 1.4426950408889634f : 0.f;
-    const float delta = row_valid ? p.delta[vi] : 0.f;
+    const long long li = static_cast<long long>(U.b) * PB.lse_b + static_cast<long long>(U.h + PB.lse_h0) * PB.lse_h + q_pos;
+    const long long di = (static_cast<long long>(U.b) * PB.H + U.h) * p.S + q_pos;
+    const float lse2 = row_valid ? PB.lse[li] * 1.4426950408889634f : 0.f;
+    const float delta = row_valid ? PB.delta[di] : 0.f;
     bool ok = true;
     for (int j = 0; ok && j < n; ++j) {
       // keys of tile j this row sees: all valid keys, cut at the row's own
@@ -330,8 +338,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __gri
     }
     if (ok) {
       const float scale = p.scale;
-      __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.dq) +
-                           ((static_cast<long long>(U.b) * p.S + q_pos) * p.H + U.h) * D;
+      __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(PB.dq) +
+                           ((static_cast<long long>(U.b) * p.S + q_pos) * PB.H + U.h) * D;
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t o[32];
@@ -389,6 +397,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __gr
   const int lane = threadIdx.x & 31;
   const uint64_t tmo = p.timeout_ns;
   const BwdUnit U = bwd_unit(p, false);        // causal: earlier K/V tiles see more queries and run first
+  const BwdProblem &PB = p.prob[U.pi];
   const int nt = (p.S + 127) / 128;
   const int k0 = U.t * 128;
   const int k_rows = min(128, p.S - k0);
@@ -427,14 +436,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __gr
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      tma_prefetch_desc(&p.tm_q);
-      tma_prefetch_desc(&p.tm_k);
-      tma_prefetch_desc(&p.tm_v);
-      tma_prefetch_desc(&p.tm_do);
+      tma_prefetch_desc(&PB.tm_q);
+      tma_prefetch_desc(&PB.tm_k);
+      tma_prefetch_desc(&PB.tm_v);
+      tma_prefetch_desc(&PB.tm_do);
       mbar_arrive_expect_tx(sb + BAR_KV, 2 * L::kTileBytes);
       for (int hf = 0; hf < L::kHalves; ++hf) {
-        tma_load_3d(sb + L::kOffA + hf * L::kBoxBytes, &p.tm_k, hf * 64, U.h, row_base + k0, sb + BAR_KV);
-        tma_load_3d(sb + L::kOffB + hf * L::kBoxBytes, &p.tm_v, hf * 64, U.h, row_base + k0, sb + BAR_KV);
+        tma_load_3d(sb + L::kOffA + hf * L::kBoxBytes, &PB.tm_k, hf * 64, U.h, row_base + k0, sb + BAR_KV);
+        tma_load_3d(sb + L::kOffB + hf * L::kBoxBytes, &PB.tm_v, hf * 64, U.h, row_base + k0, sb + BAR_KV);
       }
       for (int i = 0; i < n; ++i) {
         const int st = i & 1;
@@ -443,12 +452,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __gr
         if (!mbar_wait(sb + BAR_QE + 8 * st, ph ^ 1, abort_flag, tmo, SITE_PRODUCER)) break;
         mbar_arrive_expect_tx(sb + BAR_QF + 8 * st, L::kTileBytes);
         for (int hf = 0; hf < L::kHalves; ++hf)
-          tma_load_3d(sb + L::kOffC + st * L::kTileBytes + hf * L::kBoxBytes, &p.tm_q, hf * 64, U.h, qrow,
+          tma_load_3d(sb + L::kOffC + st * L::kTileBytes + hf * L::kBoxBytes, &PB.tm_q, hf * 64, U.h, qrow,
                       sb + BAR_QF + 8 * st);
         if (!mbar_wait(sb + BAR_OE + 8 * st, ph ^ 1, abort_flag, tmo, SITE_PRODUCER)) break;
         mbar_arrive_expect_tx(sb + BAR_OF + 8 * st, L::kTileBytes);
         for (int hf = 0; hf < L::kHalves; ++hf)
-          tma_load_3d(sb + L::kOffE + st * L::kTileBytes + hf * L::kBoxBytes, &p.tm_do, hf * 64, U.h, qrow,
+          tma_load_3d(sb + L::kOffE + st * L::kTileBytes + hf * L::kBoxBytes, &PB.tm_do, hf * 64, U.h, qrow,
                       sb + BAR_OF + 8 * st);
       }
       for (int st = 0; st < 2; ++st) {
@@ -538,7 +547,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __gr
     const uint32_t tDV = tmem + lane_base + 256;
     const uint32_t tDK = tmem + lane_base + 256 + D;
     const float c = p.scale_log2;
-    const long long vbase = (static_cast<long long>(U.b) * p.H + U.h) * p.S;
+    const long long lbase = static_cast<long long>(U.b) * PB.lse_b + static_cast<long long>(U.h + PB.lse_h0) * PB.lse_h;
+    const long long dbase = (static_cast<long long>(U.b) * PB.H + U.h) * p.S;
     bool ok = true;
     for (int i = 0; ok && i < n; ++i) {
       const int q0 = (qt0 + i) * 128;
@@ -547,8 +557,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __gr
       const uint32_t vec = sb + L::kOffVec + (i & 1) * 1024;
       {
         const int q = q0 + tid;
-        st_shared_f32(vec + 4 * tid, q < p.S ? p.lse[vbase + q] * 1.4426950408889634f : INFINITY);
-        st_shared_f32(vec + 512 + 4 * tid, q < p.S ? p.delta[vbase + q] : 0.f);
+        st_shared_f32(vec + 4 * tid, q < p.S ? PB.lse[lbase + q] * 1.4426950408889634f : INFINITY);
+        st_shared_f32(vec + 512 + 4 * tid, q < p.S ? PB.delta[dbase + q] : 0.f);
       }
       // Every row warp has finished reading the previous use of this buffer
       // (tile i-2) before it writes tile i's values, and the bounded barrier
@@ -625,10 +635,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __gr
       tc_fence_after();
     }
     if (ok) {
-      const long long roff = ((static_cast<long long>(U.b) * p.S + k_pos) * p.H + U.h) * D;
+      const long long roff = ((static_cast<long long>(U.b) * p.S + k_pos) * PB.H + U.h) * D;
       for (int which = 0; which < 2; ++which) {   // 0: dV, 1: dK (times the softmax scale)
         const float mul = which == 0 ? 1.0f : p.scale;
-        __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(which == 0 ? p.dv : p.dk) + roff;
+        __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(which == 0 ? PB.dv : PB.dk) + roff;
         const uint32_t tsrc = which == 0 ? tDV : tDK;
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {

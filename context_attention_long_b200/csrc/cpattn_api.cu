@@ -184,7 +184,7 @@ cudaError_t launch_lse_merge(const MergeParams &p, cudaStream_t stream) {
 }
 
 template <int D>
-static cudaError_t launch_bwd_d(const BwdParams &p, cudaStream_t stream) {
+static cudaError_t launch_bwd_d(const BwdParams &p, int units, cudaStream_t stream) {
   static std::mutex mu;
   static bool configured[kMaxDevices] = {false};
   int dev = 0;
@@ -201,7 +201,6 @@ static cudaError_t launch_bwd_d(const BwdParams &p, cudaStream_t stream) {
       configured[dev] = true;
     }
   }
-  const long long units = static_cast<long long>(p.B) * p.H * ((p.S + 127) / 128);
   attn_bwd_dq_kernel<D><<<static_cast<unsigned>(units), kBwdThreads, BwdSmem<D>::kAllocBytes, stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -209,14 +208,21 @@ static cudaError_t launch_bwd_d(const BwdParams &p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_attention_backward(const BwdParams &p, int D, const void *out, const void *dout, float *delta,
+cudaError_t launch_attention_backward(const BwdParams &p, int D, const void *const *outs, const void *const *douts,
                                       cudaStream_t stream) {
-  const long long rows = static_cast<long long>(p.B) * p.S * p.H;
-  attn_bwd_delta_kernel<<<grid_for(rows, 256 / 32), 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16 *>(out), static_cast<const __nv_bfloat16 *>(dout), delta, p.B, p.S, p.H, D);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  return D == 128 ? launch_bwd_d<128>(p, stream) : launch_bwd_d<64>(p, stream);
+  const int nt = (p.S + 127) / 128;
+  int units = 0;
+  for (int i = 0; i < p.n_prob; ++i) {
+    const long long rows = static_cast<long long>(p.B) * p.S * p.prob[i].H;
+    attn_bwd_delta_kernel<<<grid_for(rows, 256 / 32), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16 *>(outs[i]), static_cast<const __nv_bfloat16 *>(douts[i]), p.prob[i].delta,
+        p.B, p.S, p.prob[i].H, D);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    units += p.B * p.prob[i].H * nt;
+  }
+  if (units == 0) return cudaSuccess;
+  return D == 128 ? launch_bwd_d<128>(p, units, stream) : launch_bwd_d<64>(p, units, stream);
 }
 
 cudaError_t launch_permute(const PermuteParams &p, cudaStream_t stream) {
@@ -934,6 +940,37 @@ size_t cpattn_attention_backward_workspace_bytes(int B, int H, int S) {
   return static_cast<size_t>(B) * H * S * sizeof(float);
 }
 
+// One backward problem over [B, S, H, D] tensors; LSE index b*lse_b + (h + lse_h0)*lse_h + s.
+static bool backward_problem(BwdProblem &pb, const void *q, const void *k, const void *v, const void *dout,
+                             const float *lse, long long lse_b, long long lse_h, int lse_h0, float *delta, void *dq,
+                             void *dk, void *dv, int B, int S, int H, int D, int unit_base) {
+  std::memset(&pb, 0, sizeof(pb));
+  const long long rows = static_cast<long long>(B) * S;
+  if (!encode_rows_map(&pb.tm_q, q, D, H, rows) || !encode_rows_map(&pb.tm_k, k, D, H, rows) ||
+      !encode_rows_map(&pb.tm_v, v, D, H, rows) || !encode_rows_map(&pb.tm_do, dout, D, H, rows))
+    return false;
+  pb.lse = lse;
+  pb.lse_b = lse_b;
+  pb.lse_h = lse_h;
+  pb.lse_h0 = lse_h0;
+  pb.H = H;
+  pb.delta = delta;
+  pb.dq = dq;
+  pb.dk = dk;
+  pb.dv = dv;
+  pb.unit_base = unit_base;
+  return true;
+}
+
+static void backward_common_params(BwdParams &P, int B, int S, int D, bool causal) {
+  P.B = B;
+  P.S = S;
+  P.causal = causal ? 1 : 0;
+  P.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+  P.scale_log2 = static_cast<float>((1.0 / std::sqrt(static_cast<double>(D))) * 1.4426950408889634);
+  P.timeout_ns = wait_timeout_ns();
+}
+
 int cpattn_attention_backward(const void *q, const void *k, const void *v, const void *out, const float *lse,
                               const void *dout, void *dq, void *dk, void *dv, int B, int H, int S, int D,
                               int causal, void *workspace, size_t workspace_bytes, cpattn_stream_t stream) {
@@ -952,25 +989,105 @@ int cpattn_attention_backward(const void *q, const void *k, const void *v, const
   if (st != CPATTN_OK) return st;
   std::unique_ptr<BwdParams> P(new BwdParams);
   std::memset(P.get(), 0, sizeof(BwdParams));
-  const long long rows = static_cast<long long>(B) * S;
-  if (!encode_rows_map(&P->tm_q, q, D, H, rows) || !encode_rows_map(&P->tm_k, k, D, H, rows) ||
-      !encode_rows_map(&P->tm_v, v, D, H, rows) || !encode_rows_map(&P->tm_do, dout, D, H, rows))
+  if (!backward_problem(P->prob[0], q, k, v, dout, lse, static_cast<long long>(H) * S, S, 0,
+                        static_cast<float *>(workspace), dq, dk, dv, B, S, H, D, 0))
     return CPATTN_ERR_CUDA;
-  P->lse = lse;
-  P->delta = static_cast<float *>(workspace);
-  P->dq = dq;
-  P->dk = dk;
-  P->dv = dv;
-  P->B = B;
-  P->H = H;
-  P->S = S;
-  P->causal = causal ? 1 : 0;
-  P->scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
-  P->scale_log2 = static_cast<float>((1.0 / std::sqrt(static_cast<double>(D))) * 1.4426950408889634);
-  P->timeout_ns = wait_timeout_ns();
-  return launch_attention_backward(*P, D, out, dout, static_cast<float *>(workspace), stream) == cudaSuccess
-             ? CPATTN_OK
-             : CPATTN_ERR_CUDA;
+  P->n_prob = 1;
+  backward_common_params(*P, B, S, D, causal != 0);
+  const void *outs[1] = {out}, *douts[1] = {dout};
+  return launch_attention_backward(*P, D, outs, douts, stream) == cudaSuccess ? CPATTN_OK : CPATTN_ERR_CUDA;
+}
+
+size_t cpattn_ulysses_attention_backward_workspace_bytes(int B, int H, int S, int D) {
+  if (B < 1 || H < 1 || S < 1 || D < 1) return 0;
+  return static_cast<size_t>(8) * B * S * H * D * 2 + static_cast<size_t>(B) * H * S * sizeof(float);
+}
+
+int cpattn_ulysses_attention_backward(const void *q, const void *k, const void *v, const void *out,
+                                      const float *lse, const void *dout, void *dq, void *dk, void *dv, int B,
+                                      int H, int S, int D, int degree, const int *seq_splits,
+                                      const int *head_splits, int causal, void *workspace, size_t workspace_bytes,
+                                      cpattn_stream_t stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || lse == nullptr || dout == nullptr ||
+      dq == nullptr || dk == nullptr || dv == nullptr)
+    return CPATTN_ERR_NULL;
+  int st = check_attn_shape(B, H, S, D);
+  if (st != CPATTN_OK) return st;
+  if (degree < 1 || degree > kMaxRanks) return CPATTN_ERR_DEGREE;
+  std::vector<int> seq_chk, heads;
+  st = resolve_splits(S, degree, seq_splits, seq_chk);
+  if (st != CPATTN_OK) return st;
+  st = resolve_splits(H, degree, head_splits, heads);
+  if (st != CPATTN_OK) return st;
+  if (workspace == nullptr || workspace_bytes < cpattn_ulysses_attention_backward_workspace_bytes(B, H, S, D))
+    return CPATTN_ERR_WORKSPACE;
+  PermuteParams pq;
+  st = permute_common(q, workspace, B, S, H, D, 2, degree, seq_splits, head_splits, 0, pq);
+  if (st != CPATTN_OK) return st;
+  const void *ptrs[8] = {k, v, out, dout, dq, dk, dv, workspace};
+  for (const void *ptr : ptrs)
+    if (!aligned16(ptr)) return CPATTN_ERR_ALIGNMENT;
+  if (!aligned4(lse)) return CPATTN_ERR_ALIGNMENT;
+  st = check_device(nullptr);
+  if (st != CPATTN_OK) return st;
+  // workspace: head-side yq, yk, yv, yo, ydo, ydq, ydk, ydv, then Delta per head rank
+  const size_t tb = static_cast<size_t>(B) * S * H * D * 2;
+  char *ws = static_cast<char *>(workspace);
+  void *y[8];
+  for (int i = 0; i < 8; ++i) y[i] = ws + i * tb;
+  float *delta = reinterpret_cast<float *>(ws + 8 * tb);
+  // first all-to-all: Q, K, V, then O and dO, to the head-sharded layout
+  {
+    PermuteParams pp = pq;
+    set_qkv(pp, q, k, v, y[0], y[1], y[2]);
+    if (launch_permute(pp, stream) != cudaSuccess) return CPATTN_ERR_CUDA;
+    pp.src[0] = static_cast<const unsigned char *>(out);
+    pp.dst[0] = static_cast<unsigned char *>(y[3]);
+    pp.src[1] = static_cast<const unsigned char *>(dout);
+    pp.dst[1] = static_cast<unsigned char *>(y[4]);
+    pp.n_tensors = 2;
+    if (launch_permute(pp, stream) != cudaSuccess) return CPATTN_ERR_CUDA;
+  }
+  // the backward of every head rank's local attention, one launch per kernel
+  std::unique_ptr<BwdParams> P(new BwdParams);
+  std::memset(P.get(), 0, sizeof(BwdParams));
+  const std::vector<int> ho = prefix(heads);
+  const int nt = (S + 127) / 128;
+  std::vector<const void *> outs, douts;
+  int n_prob = 0, units = 0;
+  for (int u = 0; u < degree; ++u) {
+    if (heads[u] == 0) continue;
+    if (n_prob == kMaxProblems) {   // a full parameter table: launch it and start the next
+      P->n_prob = n_prob;
+      backward_common_params(*P, B, S, D, causal != 0);
+      if (launch_attention_backward(*P, D, outs.data(), douts.data(), stream) != cudaSuccess) return CPATTN_ERR_CUDA;
+      std::memset(P.get(), 0, sizeof(BwdParams));
+      outs.clear();
+      douts.clear();
+      n_prob = 0;
+      units = 0;
+    }
+    const size_t off = static_cast<size_t>(B) * S * ho[u] * D * 2;
+    auto at = [&](int i) { return static_cast<void *>(static_cast<char *>(y[i]) + off); };
+    if (!backward_problem(P->prob[n_prob], at(0), at(1), at(2), at(4), lse, static_cast<long long>(H) * S, S, ho[u],
+                          delta + static_cast<size_t>(B) * ho[u] * S, at(5), at(6), at(7), B, S, heads[u], D,
+                          units))
+      return CPATTN_ERR_CUDA;
+    outs.push_back(at(3));
+    douts.push_back(at(4));
+    units += B * heads[u] * nt;
+    ++n_prob;
+  }
+  if (n_prob > 0) {
+    P->n_prob = n_prob;
+    backward_common_params(*P, B, S, D, causal != 0);
+    if (launch_attention_backward(*P, D, outs.data(), douts.data(), stream) != cudaSuccess) return CPATTN_ERR_CUDA;
+  }
+  // second all-to-all: dQ, dK, dV back to the sequence-sharded layout
+  PermuteParams pb = pq;
+  set_qkv(pb, y[5], y[6], y[7], dq, dk, dv);
+  pb.direction = 1;
+  return launch_permute(pb, stream) == cudaSuccess ? CPATTN_OK : CPATTN_ERR_CUDA;
 }
 
 int cpattn_exchange_bytes(int mode, int B, int H, int S, int D, int elem_bytes, int degree, const int *seq_splits,

@@ -88,19 +88,31 @@ struct AttnParams {
 cudaError_t launch_attention(const AttnParams &p, int D, bool out_f32, cudaStream_t stream);
 
 // ---------------------------------------------------------------- backward
-// Gradient of attention over full [B, S, H, D] tensors (rows = B*S).
-struct alignas(64) BwdParams {
+// Gradient of attention.  A problem is one (Q, K, V, dO) tensor set laid out
+// [B, S, H, D] (rows = B*S) with its own head count: the full tensors, or one
+// head rank's head-side buffer of the Ulysses flow.
+struct alignas(64) BwdProblem {
   CUtensorMap tm_q, tm_k, tm_v, tm_do;   // 3-D maps over [rows, H, D] bf16, box {64, 1, 128}, 128B swizzle
-  const float *lse;                      // [B, H, S] natural log, from the forward
-  const float *delta;                    // [B, H, S] rowsum(dO * O)
+  const float *lse;                      // natural log, from the forward: index b*lse_b + (h + lse_h0)*lse_h + s
+  long long lse_b;
+  long long lse_h;
+  int lse_h0;
+  int H;
+  float *delta;                          // [B, H, S] rowsum(dO * O) of this problem
   void *dq, *dk, *dv;                    // [B, S, H, D] bf16
-  int B, H, S;
+  int unit_base;                         // first unit (blockIdx) of this problem
+};
+struct BwdParams {
+  BwdProblem prob[kMaxProblems];
+  int n_prob;
+  int B, S;
   int causal;
   float scale_log2;                      // D**-0.5 * log2(e)
   float scale;                           // D**-0.5
   unsigned long long timeout_ns;
 };
-cudaError_t launch_attention_backward(const BwdParams &p, int D, const void *out, const void *dout, float *delta,
+// outs/douts: per problem the forward output and its gradient (for the row sums).
+cudaError_t launch_attention_backward(const BwdParams &p, int D, const void *const *outs, const void *const *douts,
                                       cudaStream_t stream);
 
 // ---------------------------------------------------------------- LSE merge

@@ -332,6 +332,32 @@ int cpattn_attention_backward(const void *q, const void *k, const void *v, const
                               int B, int H, int S, int D, int causal, void *workspace,
                               size_t workspace_bytes, cpattn_stream_t stream);
 
+/*
+ * Backward of the Ulysses flow ([USP] section 4 run in reverse for training,
+ * sections 1 and 7): the first all-to-all takes Q, K, V, the forward output O
+ * and its gradient dO to the head-sharded layout (two launches), the attention
+ * backward runs on every head rank's buffers (one dQ and one dK/dV launch for
+ * up to 8 head ranks), and the second all-to-all brings dQ, dK and dV back to
+ * the sequence-sharded layout.
+ *
+ *   q, k, v, out, dout  sequence-sharded rank buffers, as the inputs and the
+ *                       output of cpattn_ulysses_attention; read only.
+ *   lse                 [B, H, S] float32 device, from the forward.
+ *   dq, dk, dv          sequence-sharded rank buffers, written.
+ *   workspace           device, 16-byte aligned, at least
+ *                       cpattn_ulysses_attention_backward_workspace_bytes()
+ *                       = 16 * B*S*H*D + 4 * B*H*S bytes.
+ * Other arguments, splits and errors as cpattn_ulysses_attention; causal = 1
+ * for the causal mask.
+ */
+size_t cpattn_ulysses_attention_backward_workspace_bytes(int B, int H, int S, int D);
+int cpattn_ulysses_attention_backward(const void *q, const void *k, const void *v,
+                                      const void *out, const float *lse, const void *dout,
+                                      void *dq, void *dk, void *dv, int B, int H, int S, int D,
+                                      int degree, const int *seq_splits, const int *head_splits,
+                                      int causal, void *workspace, size_t workspace_bytes,
+                                      cpattn_stream_t stream);
+
 /* ------------------------------------------------- no-allocation variant */
 
 /*

@@ -197,3 +197,18 @@ def test_backward_validation(lib):
     assert f(dq=FAKE_MIS) == ALIGN
     if not torch.cuda.is_available():
         assert f() == CUDA
+
+
+def test_ulysses_backward_validation(lib):
+    need = lib.cpattn_ulysses_attention_backward_workspace_bytes(1, 4, 8, 64)
+    assert need == 16 * 1 * 8 * 4 * 64 + 4 * 1 * 4 * 8
+
+    def f(ws=FAKE, nbytes=need, H=4, heads=None, lse=FAKE):
+        return lib.cpattn_ulysses_attention_backward(FAKE, FAKE, FAKE, FAKE, lse, FAKE, FAKE, FAKE, FAKE, 1, H, 8,
+                                                     64, 2, None, _native.int_array(heads), 0, ws, nbytes, None)
+    assert f(lse=None) == NULL
+    assert f(ws=None) == WS
+    assert f(nbytes=need - 1) == WS
+    assert f(H=5) == INDIV
+    assert f(heads=[3, 3]) == SPLITS
+    assert f(ws=FAKE_MIS) == ALIGN

@@ -16,7 +16,7 @@ import torch
 import oracle
 from context_attention_long_b200 import api, build, inputs
 
-from gpu_util import f64_of, to_dev
+from gpu_util import f64_of, full_to_rank_buffers, rank_buffers_to_full, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -97,3 +97,28 @@ def test_backward_is_deterministic_and_validates():
     F = g1[0].data_ptr()
     assert lib.cpattn_attention_backward(F, F, F, F, None, F, F, F, F, 1, 2, 384, 128, 0, F, 1 << 20, None) == 1
     assert lib.cpattn_attention_backward(F, F, F, F, F, F, F, F, F, 1, 2, 384, 128, 0, F, 16, None) == 8
+
+
+@pytest.mark.parametrize("B,S,H,D,P,seq,heads,causal", [
+    (1, 256, 4, 64, 2, None, None, False),
+    (2, 300, 7, 128, 3, [100, 50, 150], [3, 2, 2], True),
+    (1, 1000, 6, 128, 4, [250, 250, 250, 250], [2, 2, 1, 1], False),
+    (1, 320, 10, 64, 10, None, None, True),     # 10 head ranks: more problems than one launch holds
+])
+def test_ulysses_backward_matches_oracle(B, S, H, D, P, seq, heads, causal):
+    """The backward of the Ulysses flow on sequence-sharded rank buffers, with
+    the forward's output and LSE from the Ulysses forward."""
+    seq_l = seq or [S // P] * P
+    qb, kb, vb = inputs.make_qkv(B, S, H, D, 90 + S, D == 128)
+    rng = np.random.Generator(np.random.PCG64(91 + S))
+    dob = inputs.f32_to_bf16_bits(rng.standard_normal((B, S, H, D)).astype(np.float32))
+    q, k, v, do = (to_dev(full_to_rank_buffers(x, seq_l)) for x in (qb, kb, vb, dob))
+    fwd = api.cpattn_causal_ulysses_attention if causal else api.cpattn_ulysses_attention
+    out, lse = fwd(q, k, v, B, S, H, D, P, seq, heads)
+    dq, dk, dv = api.cpattn_ulysses_attention_backward(q, k, v, out, lse, do, B, S, H, D, P, seq, heads, causal)
+    torch.cuda.synchronize()
+    _no_timeouts()
+    refs = oracle.attention_backward(*(inputs.bf16_bits_to_f64(x) for x in (qb, kb, vb, dob)), causal=causal)
+    for name, got, ref in zip(("dq", "dk", "dv"), (dq, dk, dv), refs):
+        full = rank_buffers_to_full(f64_of(got), B, S, H, D, seq_l)
+        assert_grad_close(full, ref, f"ulysses {name} B{B} S{S} H{H} P{P} causal={causal}")
