@@ -13,8 +13,10 @@
 //
 // Two kernels, so that no gradient needs atomics: the dQ kernel owns a Q tile
 // and walks the K/V tiles; the dK/dV kernel owns a K/V tile and walks the Q
-// tiles (S and dP are computed in both).  CTA organisation of each (192
-// threads, one CTA per SM):
+// tiles (S and dP are computed in both).  A launch covers up to 8 problems
+// (the full tensors, or the head ranks' buffers of the Ulysses flow), each
+// with its own tensor maps, LSE strides and Delta slice.  CTA organisation of
+// each kernel (192 threads, one CTA per SM):
 //   warp 0      TMA producer: the owned tiles once, the walked tiles through
 //               a 2-stage ring
 //   warp 1      TMEM allocator + single-thread MMA issuer (tcgen05.mma)
