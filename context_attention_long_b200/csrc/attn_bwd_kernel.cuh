@@ -552,16 +552,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __gr
     const long long lbase = static_cast<long long>(U.b) * PB.lse_b + static_cast<long long>(U.h + PB.lse_h0) * PB.lse_h;
     const long long dbase = (static_cast<long long>(U.b) * PB.H + U.h) * p.S;
     bool ok = true;
+    // Each Q tile's log2-domain LSE and Delta, one value per row thread
+    // (queries past the sequence get LSE = +inf, i.e. P = 0), are loaded one
+    // tile ahead so that their global-memory latency hides behind a tile.
+    auto load_vec = [&](int i, float &l2, float &dl) {
+      const int q = (qt0 + i) * 128 + tid;
+      l2 = q < p.S ? PB.lse[lbase + q] * 1.4426950408889634f : INFINITY;
+      dl = q < p.S ? PB.delta[dbase + q] : 0.f;
+    };
+    float nl2 = 0.f, ndl = 0.f;
+    if (n > 0) load_vec(0, nl2, ndl);
     for (int i = 0; ok && i < n; ++i) {
       const int q0 = (qt0 + i) * 128;
-      // this Q tile's log2-domain LSE and Delta, one value per row thread;
-      // queries past the sequence get LSE = +inf, i.e. P = 0
       const uint32_t vec = sb + L::kOffVec + (i & 1) * 1024;
-      {
-        const int q = q0 + tid;
-        st_shared_f32(vec + 4 * tid, q < p.S ? PB.lse[lbase + q] * 1.4426950408889634f : INFINITY);
-        st_shared_f32(vec + 512 + 4 * tid, q < p.S ? PB.delta[dbase + q] : 0.f);
-      }
+      st_shared_f32(vec + 4 * tid, nl2);
+      st_shared_f32(vec + 512 + 4 * tid, ndl);
+      if (i + 1 < n) load_vec(i + 1, nl2, ndl);
       // Every row warp has finished reading the previous use of this buffer
       // (tile i-2) before it writes tile i's values, and the bounded barrier
       // below publishes them; no unbounded named barrier.
