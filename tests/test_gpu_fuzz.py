@@ -1,0 +1,89 @@
+"""Seeded random configurations for every attention path against the oracle:
+batch, heads, sequence length, head dimension, degrees and uneven splits
+(zeros and one-token chunks included) are drawn from a fixed seed, so a
+failure is reproducible from its case number.  Small sizes keep the oracle
+fast; many cases exercise the planner's segment/tile/split logic."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from context_attention_long_b200 import api, build, inputs
+
+from gpu_util import assert_close, f64_of, full_to_rank_buffers, rank_buffers_to_full, to_dev
+
+pytestmark = pytest.mark.gpu
+
+N_CASES = 64
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    build.build()
+
+
+def _case(i):
+    rng = np.random.Generator(np.random.PCG64(9000 + i))
+    B = int(rng.integers(1, 3))
+    H = int(rng.integers(1, 6))
+    S = int(rng.integers(1, 700))
+    D = int(rng.choice([64, 128]))
+    P = int(rng.integers(1, min(8, S) + 1))
+    lens = inputs.random_splits(S, P, 9100 + i) if rng.random() < 0.7 else None
+    if lens is None and S % P:
+        lens = inputs.random_splits(S, P, 9200 + i)
+    causal = bool(rng.random() < 0.5)
+    return B, H, S, D, P, lens, causal
+
+
+@pytest.mark.parametrize("i", range(N_CASES))
+def test_fuzz_ring_paths(i):
+    B, H, S, D, P, lens, causal = _case(i)
+    qb, kb, vb = inputs.make_qkv(B, S, H, D, 9300 + i, D == 128)
+    q, k, v = (inputs.bf16_bits_to_f64(x) for x in (qb, kb, vb))
+    dq, dk, dv = (to_dev(x) for x in (qb, kb, vb))
+    what = f"case {i}: B{B} H{H} S{S} D{D} P{P} lens={lens} causal={causal}"
+    ref_o, ref_l = oracle.ring_attention(q, k, v, P, lens, causal=causal)
+    fused = api.cpattn_causal_ring_attention if causal else api.cpattn_ring_attention
+    o, l = fused(dq, dk, dv, P, lens)
+    step = api.cpattn_causal_ring_step if causal else api.cpattn_ring_step
+    parts = [step(dq, dk, dv, P, t, lens) for t in range(P)]
+    _, mo, ml = api.cpattn_lse_merge(torch.stack([x[0] for x in parts]), torch.stack([x[1] for x in parts]))
+    torch.cuda.synchronize()
+    st, code = api.cpattn_device_status()
+    assert st == 0, f"{what}: device wait expired {code:#x}"
+    assert_close(f64_of(o), f64_of(l), ref_o, ref_l, what + " fused")
+    assert_close(f64_of(mo), f64_of(ml), ref_o, ref_l, what + " steps+merge")
+    if not causal:
+        go, gl = api.cpattn_kv_gather_attention(dq, dk, dv, P, lens)
+        torch.cuda.synchronize()
+        assert_close(f64_of(go), f64_of(gl), ref_o, ref_l, what + " kv_gather")
+
+
+@pytest.mark.parametrize("i", range(N_CASES))
+def test_fuzz_ulysses_and_unified(i):
+    B, H, S, D, P, lens, causal = _case(i)
+    rng = np.random.Generator(np.random.PCG64(9400 + i))
+    U = int(rng.integers(1, min(H, 4) + 1))
+    seq = inputs.random_splits(S, U, 9500 + i)
+    heads = inputs.random_splits(H, U, 9600 + i)
+    qb, kb, vb = inputs.make_qkv(B, S, H, D, 9700 + i, D == 128)
+    q, k, v = (inputs.bf16_bits_to_f64(x) for x in (qb, kb, vb))
+    what = f"case {i}: B{B} H{H} S{S} D{D} U{U} seq={seq} heads={heads} causal={causal}"
+    ref_o, ref_l = (oracle.causal_attention(q, k, v) if causal else oracle.attention(q, k, v))
+    flat = [to_dev(full_to_rank_buffers(x, seq)) for x in (qb, kb, vb)]
+    fn = api.cpattn_causal_ulysses_attention if causal else api.cpattn_ulysses_attention
+    uo, ul = fn(*flat, B, S, H, D, U, seq, heads)
+    # unified: the ring lengths of this case (or an equal split) over U head groups
+    R = P if P <= 64 else 1
+    ring_lens = lens or [S // R] * R
+    dq, dk, dv = (to_dev(x) for x in (qb, kb, vb))
+    fu = api.cpattn_causal_unified_attention if causal else api.cpattn_unified_attention
+    fo, fl = fu(dq, dk, dv, R, U, ring_lens, heads)
+    torch.cuda.synchronize()
+    st, code = api.cpattn_device_status()
+    assert st == 0, f"{what}: device wait expired {code:#x}"
+    assert_close(rank_buffers_to_full(f64_of(uo), B, S, H, D, seq), f64_of(ul), ref_o, ref_l, what + " ulysses")
+    assert_close(f64_of(fo), f64_of(fl), ref_o, ref_l, what + f" unified R{R} ring_lens={ring_lens}")
