@@ -32,13 +32,19 @@
  *   'anything' modes ([CP] Ring Anything / Ulysses Anything), may be uneven and
  *   may contain zeros.
  * Memory.  All tensor pointers are DEVICE pointers owned by the caller; the
- *   library allocates nothing.  Length/split arrays are HOST arrays read only
+ *   library allocates no device memory on any call (workspaces come from the
+ *   caller; cpattn_ulysses_attention_noalloc uses a static scratch).  Length/split arrays are HOST arrays read only
  *   during the call.  Q, K, V and outputs must be 16-byte aligned.  Outputs
  *   must not alias inputs unless stated.
  * Streams.  `stream` is a cudaStream_t (NULL = legacy default stream).  Every
  *   call only enqueues work; none synchronises the host.  Arguments are fully
  *   validated before anything is enqueued; on a non-zero return nothing was
  *   enqueued except for CPATTN_ERR_CUDA, which reports a launch failure.
+ *   The compute calls can be captured in a CUDA graph (after one eager call
+ *   per kernel shape, which sets the kernels' shared-memory attribute):
+ *   nothing on their launch path synchronises or allocates, and each launch
+ *   carries its plan by value.  cpattn_device_status synchronises and is not
+ *   capturable.
  * Errors.  Return value is a cpattn_status.  No C++ exception crosses the ABI.
  *   Device-side bounded waits (see cpattn_device_status) report a pipeline that
  *   stopped making progress instead of hanging the GPU.
