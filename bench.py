@@ -146,6 +146,24 @@ def aggregate_over_ranks(ms_local, steps, units_per_step, world, dist=None, devi
 
 
 # ----------------------------------------------------------------- reference arm (the oracle)
+def median_event_ms(fn, flush, stream, reps=10, warmup=1):
+    """Median CUDA-event time of fn() on `stream`, each rep after an L2 flush
+    (a write of a buffer larger than L2) outside the timed events."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    times = []
+    for _ in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    return float(np.median(times))
+
+
 def oracle_sample_step(cfg, q, k, v, rows_per_shard, seed):
     """The oracle's hot path on a bounded sample of query rows: for each ring
     shard, sampled rows attend every K/V chunk in ring order (partials + LSE
@@ -499,19 +517,6 @@ def causal_paths(api, torch, flush, peaks, q, k, v, P, U):
     ws = torch.empty(api.cpattn_ulysses_workspace_bytes(B, H, S, D), dtype=torch.uint8, device=q.device)
     qf, kf, vf, of = q.reshape(-1), k.reshape(-1), v.reshape(-1), out.reshape(-1)
 
-    def timeit(fn, reps=10):
-        fn()
-        times = []
-        for _ in range(reps):
-            flush.zero_()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            fn()
-            b.record(stream)
-            b.synchronize()
-            times.append(a.elapsed_time(b))
-        return float(np.median(times))
-
     res = {}
     for name, fn in (
         (f"causal_ring_fused_p{P}", lambda: api.cpattn_causal_ring_attention(q, k, v, P, out=out, lse=lse,
@@ -520,7 +525,7 @@ def causal_paths(api, torch, flush, peaks, q, k, v, P, U):
                                                                                  lse=lse, workspace=ws,
                                                                                  stream=stream)),
     ):
-        ms = timeit(fn)
+        ms = median_event_ms(fn, flush, stream)
         tf = flops / (ms * 1e-3) / 1e12
         res[name] = {"ms": ms, "TFLOP/s": tf, "frac_bf16_peak": tf / peak_tf,
                      "flops": "4*D per visible (query, key) pair: 2*B*H*D*S*(S+1)"}
@@ -552,17 +557,7 @@ def backward_paths(api, torch, flush, peaks, q, k, v, P):
         def run():
             api.cpattn_attention_backward(q, k, v, out, lse, do, causal, dq, dk, dv, ws, stream=stream)
 
-        run()
-        times = []
-        for _ in range(10):
-            flush.zero_()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            run()
-            b.record(stream)
-            b.synchronize()
-            times.append(a.elapsed_time(b))
-        ms = float(np.median(times))
+        ms = median_event_ms(run, flush, stream)
         tf = backward_flops(B, H, S, D, causal) / (ms * 1e-3) / 1e12
         res["attention_backward" + ("_causal" if causal else "")] = {
             "ms": ms, "TFLOP/s": tf, "frac_bf16_peak": tf / peak_tf,
@@ -578,17 +573,7 @@ def backward_paths(api, torch, flush, peaks, q, k, v, P):
                                               B, S, H, D, U, dq=dq.reshape(-1), dk=dk.reshape(-1), dv=dv.reshape(-1),
                                               workspace=wsu, stream=stream)
 
-    run_u()
-    times = []
-    for _ in range(10):
-        flush.zero_()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        run_u()
-        b.record(stream)
-        b.synchronize()
-        times.append(a.elapsed_time(b))
-    ms = float(np.median(times))
+    ms = median_event_ms(run_u, flush, stream)
     tf = backward_flops(B, H, S, D, False) / (ms * 1e-3) / 1e12
     res[f"ulysses_{U}_backward_flow"] = {"ms": ms, "TFLOP/s": tf, "frac_bf16_peak": tf / peak_tf,
                                          "launches": 7, "note": "5 permuted in, backward of 4 head ranks, 3 permuted out"}
@@ -608,18 +593,8 @@ def breakdown(api, torch, dev, flush, peaks, inputs):
     stream = torch.cuda.current_stream()
     res = {}
 
-    def timeit(fn, reps=10):
-        fn()
-        times = []
-        for _ in range(reps):
-            flush.zero_()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            fn()
-            b.record(stream)
-            b.synchronize()
-            times.append(a.elapsed_time(b))
-        return float(np.median(times))
+    def timeit(fn):
+        return median_event_ms(fn, flush, stream)
 
     ms = timeit(lambda: api.cpattn_ulysses_permute(x, B, S, H, D, 2, y=y, stream=stream))
     gbs = 2 * n * 2 / (ms * 1e-3) / 1e9
@@ -653,19 +628,10 @@ def run_sweep(args):
     peaks, kind = load_peaks()
     reps = max(3, args.steps)
 
+    stream = torch.cuda.current_stream()
+
     def timeit(fn):
-        for _ in range(args.warmup):
-            fn()
-        ts = []
-        for _ in range(reps):
-            flush.zero_()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record()
-            fn()
-            b.record()
-            b.synchronize()
-            ts.append(a.elapsed_time(b))
-        return float(np.median(ts))
+        return median_event_ms(fn, flush, stream, reps=reps, warmup=args.warmup)
 
     for name in ("tiny", "dit", "hires", "anything", "video"):
         cfg, qb, kb, vb = inputs.config_inputs(name)
