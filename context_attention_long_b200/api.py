@@ -50,7 +50,19 @@ def _stream(stream):
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    """Device address of a tensor the library may read or write.  The kernels
+    launch on the current CUDA device and index the memory densely, so a host
+    tensor, a tensor on another device or a non-contiguous view is refused
+    here, before the library sees the pointer."""
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError("tensor arguments must be CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("tensor arguments must be contiguous")
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"tensor on {t.device}, but the current device is cuda:{torch.cuda.current_device()}")
+    return ctypes.c_void_p(t.data_ptr())
 
 
 def _bshd(q: torch.Tensor, name="q"):

@@ -212,3 +212,15 @@ def test_ulysses_backward_validation(lib):
     assert f(H=5) == INDIV
     assert f(heads=[3, 3]) == SPLITS
     assert f(ws=FAKE_MIS) == ALIGN
+
+
+def test_binding_refuses_host_and_strided_tensors():
+    """Host tensors never reach the library as pointers (they would be device
+    addresses to the kernels); the check runs before any library call."""
+    from context_attention_long_b200 import api
+    x = torch.zeros(2 * 8 * 4 * 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        api.cpattn_ulysses_permute(x, 2, 8, 4, 64, 2, y=torch.empty_like(x))
+    with pytest.raises(ValueError):
+        api._ptr(torch.zeros(4, 4).t())      # a CPU, non-contiguous view
+    assert api._ptr(None) is None
