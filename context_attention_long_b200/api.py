@@ -65,6 +65,19 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _need(t, numel, dtype, name):
+    """A tensor argument must hold at least `numel` elements of `dtype`: the
+    library indexes the memory behind the pointer by the sizes it is given."""
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor):
+        raise ValueError(f"{name} must be a tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.numel() < numel:
+        raise ValueError(f"{name} holds {t.numel()} elements, {numel} needed")
+
+
 def _bshd(q: torch.Tensor, name="q"):
     if q.dim() != 4:
         raise ValueError(f"{name} must be (B, S, H, D)")
@@ -79,6 +92,9 @@ def _ring(entry, q, k, v, ring_degree, chunk_lens, out, lse, want_lse, stream):
     out = torch.empty_like(q) if out is None else out
     if lse is None and want_lse:
         lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    for t, name in ((k, "k"), (v, "v"), (out, "out")):
+        _need(t, q.numel(), torch.bfloat16, name)
+    _need(lse, B * H * S, torch.float32, "lse")
     _check(getattr(_native.load(), entry)(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, S, D,
                                           int(ring_degree), _native.int_array(chunk_lens), _stream(stream)), entry)
     return out, lse
@@ -101,6 +117,10 @@ def _ring_step(entry, q, k, v, ring_degree, step, chunk_lens, part_out, part_lse
         part_out = torch.empty((B, S, H, D), dtype=torch.float32, device=q.device)
     if part_lse is None:
         part_lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    _need(k, q.numel(), torch.bfloat16, "k")
+    _need(v, q.numel(), torch.bfloat16, "v")
+    _need(part_out, q.numel(), torch.float32, "part_out")
+    _need(part_lse, B * H * S, torch.float32, "part_lse")
     _check(getattr(_native.load(), entry)(_ptr(q), _ptr(k), _ptr(v), _ptr(part_out), _ptr(part_lse), B, H, S, D,
                                           int(ring_degree), _native.int_array(chunk_lens), int(step),
                                           _stream(stream)), entry)
@@ -130,6 +150,12 @@ def cpattn_lse_merge(part_out, part_lse, out_f32=None, out_bf16=None, lse_out=No
         out_bf16 = torch.empty((B, S, H, D), dtype=torch.bfloat16, device=dev)
     if lse_out is None:
         lse_out = torch.empty((B, H, S), dtype=torch.float32, device=dev)
+    n = B * S * H * D
+    _need(part_out, P * n, torch.float32, "part_out")
+    _need(part_lse, P * B * H * S, torch.float32, "part_lse")
+    _need(out_f32, n, torch.float32, "out_f32")
+    _need(out_bf16, n, torch.bfloat16, "out_bf16")
+    _need(lse_out, B * H * S, torch.float32, "lse_out")
     _check(_native.load().cpattn_lse_merge(_ptr(part_out), _ptr(part_lse), P, B, H, S, D, _ptr(out_f32),
                                            _ptr(out_bf16), _ptr(lse_out), _stream(stream)), "cpattn_lse_merge")
     return out_f32, out_bf16, lse_out
@@ -141,6 +167,9 @@ def cpattn_kv_gather_attention(q, k, v, degree, q_lens=None, out=None, lse=None,
     out = torch.empty_like(q) if out is None else out
     if lse is None and want_lse:
         lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    for t, name in ((k, "k"), (v, "v"), (out, "out")):
+        _need(t, q.numel(), torch.bfloat16, name)
+    _need(lse, B * H * S, torch.float32, "lse")
     _check(_native.load().cpattn_kv_gather_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, S, D,
                                                      int(degree), _native.int_array(q_lens), _stream(stream)),
            "cpattn_kv_gather_attention")
@@ -155,6 +184,8 @@ def cpattn_ulysses_permute(x, B, S, H, D, degree, seq_splits=None, head_splits=N
     """Sequence-sharded rank buffers (flat, any 1/2/4/8-byte dtype) -> head-sharded rank buffers."""
     if y is None:
         y = torch.empty_like(x)
+    _need(x, _flat_numel(B, S, H, D), None, "x")
+    _need(y, _flat_numel(B, S, H, D), x.dtype, "y")
     _check(_native.load().cpattn_ulysses_permute(_ptr(x), _ptr(y), B, S, H, D, x.element_size(), int(degree),
                                                  _native.int_array(seq_splits), _native.int_array(head_splits),
                                                  _stream(stream)), "cpattn_ulysses_permute")
@@ -167,6 +198,8 @@ def cpattn_ulysses_permute_qkv(q, k, v, B, S, H, D, degree, seq_splits=None, hea
     yq = torch.empty_like(q) if yq is None else yq
     yk = torch.empty_like(k) if yk is None else yk
     yv = torch.empty_like(v) if yv is None else yv
+    for t, name in ((q, "q"), (k, "k"), (v, "v"), (yq, "yq"), (yk, "yk"), (yv, "yv")):
+        _need(t, _flat_numel(B, S, H, D), q.dtype, name)
     _check(_native.load().cpattn_ulysses_permute_qkv(_ptr(q), _ptr(k), _ptr(v), _ptr(yq), _ptr(yk), _ptr(yv), B, S,
                                                      H, D, q.element_size(), int(degree),
                                                      _native.int_array(seq_splits), _native.int_array(head_splits),
@@ -178,6 +211,8 @@ def cpattn_ulysses_unpermute(y, B, S, H, D, degree, seq_splits=None, head_splits
     """Head-sharded rank buffers -> sequence-sharded rank buffers (inverse permute)."""
     if x is None:
         x = torch.empty_like(y)
+    _need(y, _flat_numel(B, S, H, D), None, "y")
+    _need(x, _flat_numel(B, S, H, D), y.dtype, "x")
     _check(_native.load().cpattn_ulysses_unpermute(_ptr(y), _ptr(x), B, S, H, D, y.element_size(), int(degree),
                                                    _native.int_array(seq_splits), _native.int_array(head_splits),
                                                    _stream(stream)), "cpattn_ulysses_unpermute")
@@ -188,6 +223,9 @@ def _head_sharded(entry, yq, yk, yv, B, S, H, D, degree, head_splits, yo, lse, w
     yo = torch.empty_like(yq) if yo is None else yo
     if lse is None and want_lse:
         lse = torch.empty((B, H, S), dtype=torch.float32, device=yq.device)
+    for t, name in ((yq, "yq"), (yk, "yk"), (yv, "yv"), (yo, "yo")):
+        _need(t, _flat_numel(B, S, H, D), torch.bfloat16, name)
+    _need(lse, B * H * S, torch.float32, "lse")
     _check(getattr(_native.load(), entry)(_ptr(yq), _ptr(yk), _ptr(yv), _ptr(yo), _ptr(lse), B, H, S, D,
                                           int(degree), _native.int_array(head_splits), _stream(stream)), entry)
     return yo, lse
@@ -227,6 +265,9 @@ def _ulysses(entry, q, k, v, B, S, H, D, degree, seq_splits, head_splits, out, l
         lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
     nbytes = cpattn_ulysses_workspace_bytes(B, H, S, D)
     workspace = _workspace(nbytes, q.device, workspace)
+    for t, name in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
+        _need(t, _flat_numel(B, S, H, D), torch.bfloat16, name)
+    _need(lse, B * H * S, torch.float32, "lse")
     _check(getattr(_native.load(), entry)(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, S, D,
                                           int(degree), _native.int_array(seq_splits),
                                           _native.int_array(head_splits), _ptr(workspace),
@@ -256,6 +297,9 @@ def _unified(entry, q, k, v, ring_degree, ulysses_degree, ring_lens, head_splits
         lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
     nbytes = cpattn_unified_workspace_bytes(B, H, S, D)
     workspace = _workspace(nbytes, q.device, workspace)
+    for t, name in ((k, "k"), (v, "v"), (out, "out")):
+        _need(t, q.numel(), torch.bfloat16, name)
+    _need(lse, B * H * S, torch.float32, "lse")
     _check(getattr(_native.load(), entry)(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, S, D,
                                           int(ring_degree), int(ulysses_degree), _native.int_array(ring_lens),
                                           _native.int_array(head_splits), _ptr(workspace),
@@ -290,6 +334,11 @@ def cpattn_attention_backward(q, k, v, out, lse, dout, causal=False, dq=None, dk
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
     workspace = _workspace(cpattn_attention_backward_workspace_bytes(B, H, S), q.device, workspace)
+    for t, name in ((k, "k"), (v, "v"), (out, "out"), (dout, "dout"), (dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _need(t, q.numel(), torch.bfloat16, name)
+    _need(lse, B * H * S, torch.float32, "lse")
+    if lse is None:
+        raise ValueError("lse is required")
     _check(_native.load().cpattn_attention_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout),
                                                     _ptr(dq), _ptr(dk), _ptr(dv), B, H, S, D, 1 if causal else 0,
                                                     _ptr(workspace), workspace.numel() * workspace.element_size(),
@@ -310,6 +359,11 @@ def cpattn_ulysses_attention_backward(q, k, v, out, lse, dout, B, S, H, D, degre
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
     workspace = _workspace(cpattn_ulysses_attention_backward_workspace_bytes(B, H, S, D), q.device, workspace)
+    for t, name in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout"), (dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _need(t, _flat_numel(B, S, H, D), torch.bfloat16, name)
+    _need(lse, B * H * S, torch.float32, "lse")
+    if lse is None:
+        raise ValueError("lse is required")
     _check(_native.load().cpattn_ulysses_attention_backward(
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), B, H, S, D,
         int(degree), _native.int_array(seq_splits), _native.int_array(head_splits), 1 if causal else 0,
@@ -333,6 +387,9 @@ def cpattn_ulysses_attention_noalloc(q, k, v, B, S, H, D, degree, seq_splits=Non
     out = torch.empty_like(q) if out is None else out
     if lse is None and want_lse:
         lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    for t, name in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
+        _need(t, _flat_numel(B, S, H, D), torch.bfloat16, name)
+    _need(lse, B * H * S, torch.float32, "lse")
     _check(_native.load().cpattn_ulysses_attention_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, S,
                                                            D, int(degree), _native.int_array(seq_splits),
                                                            _native.int_array(head_splits), _stream(stream)),

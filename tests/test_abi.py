@@ -224,3 +224,18 @@ def test_binding_refuses_host_and_strided_tensors():
     with pytest.raises(ValueError):
         api._ptr(torch.zeros(4, 4).t())      # a CPU, non-contiguous view
     assert api._ptr(None) is None
+
+
+def test_binding_refuses_short_or_mistyped_buffers():
+    """A buffer smaller than the sizes passed, or of the wrong dtype, is refused
+    before the library would index past it."""
+    from context_attention_long_b200 import api
+    with pytest.raises(ValueError):
+        api._need(torch.zeros(10, dtype=torch.bfloat16), 11, torch.bfloat16, "x")
+    with pytest.raises(ValueError):
+        api._need(torch.zeros(10, dtype=torch.float32), 10, torch.bfloat16, "x")
+    api._need(torch.zeros(12, dtype=torch.bfloat16), 11, torch.bfloat16, "x")
+    api._need(None, 11, torch.bfloat16, "x")
+    x = torch.zeros(2 * 8 * 4 * 64 - 1, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        api.cpattn_ulysses_permute(x, 2, 8, 4, 64, 2)
