@@ -617,6 +617,26 @@ def breakdown(api, torch, dev, flush, peaks, inputs):
     return res
 
 
+def library_context_paths(torch, q, k, v, cflops):
+    """Unsharded attention by torch's SDPA library backends on the same bf16
+    (B, S, H, D) tensors (strided (B, H, S, D) views, no copy).  Context rows
+    only: the pages run such a library kernel once per chunk; nothing of this
+    library's path uses them."""
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    qt, kt, vt = (x.transpose(1, 2) for x in (q, k, v))
+
+    def sdpa(backend, causal):
+        def run():
+            with sdpa_kernel([backend]):
+                torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=causal)
+        return run
+    out = []
+    for backend, tag in ((SDPBackend.CUDNN_ATTENTION, "cuDNN"), (SDPBackend.FLASH_ATTENTION, "FlashAttention-2")):
+        out.append((f"library context: torch SDPA {tag}, unsharded", sdpa(backend, False)))
+        out.append((f"library context: torch SDPA {tag}, unsharded, causal", sdpa(backend, True), cflops))
+    return out
+
+
 def run_sweep(args):
     """Every workload's paths, each timed on its own (median of `steps` reps,
     L2 flushed before each rep): attention TFLOP/s per path."""
@@ -695,9 +715,16 @@ def run_sweep(args):
             paths.append(("causal attention backward",
                           lambda: api.cpattn_attention_backward(q, k, v, o_c, l_c, do, True, bq, bk, bv, bws),
                           backward_flops(B, H, S, D, True)))
+        if name in ("dit", "hires", "video"):
+            paths += library_context_paths(torch, q, k, v, cflops)
         for entry in paths:
             label, fn = entry[0], entry[1]
-            ms = timeit(fn)
+            try:
+                ms = timeit(fn)
+            except RuntimeError as e:    # a library backend that refuses this shape
+                print(json.dumps({"workload": name, "path": label, "unavailable": str(e).splitlines()[0][:200]}),
+                      flush=True)
+                continue
             tf = (entry[2] if len(entry) > 2 else flops) / (ms * 1e-3) / 1e12
             print(json.dumps({"workload": name, "shape": f"B{B} H{H} S{S} D{D}", "path": label, "ms": round(ms, 4),
                               "TFLOP/s": round(tf, 1), "frac_bf16_peak": round(tf / float(peaks["bf16_tflops"]), 4),
