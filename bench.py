@@ -630,10 +630,30 @@ def library_context_paths(torch, q, k, v, cflops):
             with sdpa_kernel([backend]):
                 torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=causal)
         return run
+    def sdpa_backward(backend, causal):
+        # The graph is built once; each call runs only the library's backward.
+        leaves = [x.detach().requires_grad_(True) for x in (q, k, v)]
+        gen = torch.Generator(device=q.device).manual_seed(7)
+        do = torch.randn(q.shape, generator=gen, device=q.device).to(q.dtype).transpose(1, 2)
+        with sdpa_kernel([backend]):
+            o = torch.nn.functional.scaled_dot_product_attention(*(x.transpose(1, 2) for x in leaves),
+                                                                 is_causal=causal)
+
+        def run():
+            torch.autograd.grad(o, leaves, do, retain_graph=True)
+        return run
+    B, S, H, D = q.shape
     out = []
     for backend, tag in ((SDPBackend.CUDNN_ATTENTION, "cuDNN"), (SDPBackend.FLASH_ATTENTION, "FlashAttention-2")):
         out.append((f"library context: torch SDPA {tag}, unsharded", sdpa(backend, False)))
         out.append((f"library context: torch SDPA {tag}, unsharded, causal", sdpa(backend, True), cflops))
+    for causal in (False, True):
+        try:
+            fn = sdpa_backward(SDPBackend.CUDNN_ATTENTION, causal)
+        except RuntimeError as e:
+            fn = e
+        label = "library context: torch SDPA cuDNN backward" + (", causal" if causal else "")
+        out.append((label, fn, backward_flops(B, H, S, D, causal)))
     return out
 
 
@@ -720,6 +740,8 @@ def run_sweep(args):
         for entry in paths:
             label, fn = entry[0], entry[1]
             try:
+                if isinstance(fn, Exception):
+                    raise fn
                 ms = timeit(fn)
             except RuntimeError as e:    # a library backend that refuses this shape
                 print(json.dumps({"workload": name, "path": label, "unavailable": str(e).splitlines()[0][:200]}),
