@@ -80,6 +80,22 @@ def make_qkv(B: int, S: int, H: int, D: int, seed: int, rms_qk: bool):
     return out[0], out[1], out[2]
 
 
+def make_projection_inputs(B: int, S: int, H: int, D: int, Dm: int, seed: int):
+    """Activations and weights of the Ulysses projections, as bf16 bits.
+
+    From PCG64(seed), in this order: x ~ N(0, 1) of (B*S, Dm) (the
+    sequence-side rank buffers concatenated, any split: the rows are just
+    tokens), w_qkv ~ N(0, 1/Dm) of (3*H*D, Dm) and w_o ~ N(0, 1/(H*D)) of
+    (Dm, H*D), so that every projection output has unit scale.  The
+    nn.Linear weight layout (out_features, in_features).
+    """
+    rng = np.random.Generator(np.random.PCG64(seed))
+    x = f32_to_bf16_bits(rng.standard_normal(size=(B * S, Dm), dtype=np.float32))
+    w_qkv = f32_to_bf16_bits(rng.standard_normal(size=(3 * H * D, Dm), dtype=np.float32) / np.float32(np.sqrt(Dm)))
+    w_o = f32_to_bf16_bits(rng.standard_normal(size=(Dm, H * D), dtype=np.float32) / np.float32(np.sqrt(H * D)))
+    return x, w_qkv, w_o
+
+
 def config_inputs(name: str):
     """(cfg, q, k, v) for a named workload."""
     cfg = dict(CONFIGS[name])

@@ -11,7 +11,8 @@ correct CPU restatement, in float64, of what the hot path computes:
 * the gradient of attention with respect to Q, K and V (causal or not),
 * the Ulysses sequence-sharded <-> head-sharded permutation and its inverse
   (including the uneven Ulysses Anything splits), and the Ulysses and unified
-  (ring x Ulysses) attention flows composed from the pieces above.
+  (ring x Ulysses) attention flows composed from the pieces above,
+* the Ulysses Q/K/V and output projections composed with their all-to-all.
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
 reference leg of ``bench.py`` may import this package.  It shares no code with
@@ -49,6 +50,12 @@ from .attention import (
     kv_gather_attention,
 )
 from .backward import attention_backward, attention_backward_rows
+from .projection import (
+    project_rows,
+    ulysses_qkv_projection,
+    ulysses_output_projection,
+    token_order_rows,
+)
 from .permute import (
     ulysses_permute,
     ulysses_unpermute,
@@ -62,4 +69,5 @@ __all__ = [
     "offsets", "ring_order", "ring_attention", "ring_step_partials",
     "kv_gather_attention", "ulysses_permute", "ulysses_unpermute",
     "ulysses_attention", "unified_attention", "attention_backward", "attention_backward_rows",
+    "project_rows", "ulysses_qkv_projection", "ulysses_output_projection", "token_order_rows",
 ]
