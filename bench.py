@@ -262,7 +262,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true",
                     help="time every workload's paths (one JSON line per path) instead of the step")
-    ap.add_argument("--kernel", default=None, choices=["ring", "causal_ring", "head_sharded", "permute", "permute_qkv", "merge", "ring_step", "backward"],
+    ap.add_argument("--kernel", default=None, choices=["ring", "causal_ring", "head_sharded", "permute", "permute_qkv", "merge", "ring_step", "backward",
+                             "qkv_projection", "output_projection"],
                     help="profiling mode: run only this kernel (warmup + steps launches) on the workload")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -450,6 +451,7 @@ def main():
         kernels.update(breakdown(api, torch, dev, flush, peaks, inputs))
         kernels.update(causal_paths(api, torch, flush, peaks, q, k, v, P, U))
         kernels.update(backward_paths(api, torch, flush, peaks, q, k, v, P))
+        kernels.update(projection_paths(api, torch, flush, peaks, inputs, B, S, H, D, U))
 
     # Accounting: what P GPUs would exchange per rank for this workload (on one
     # GPU the exchanges are emulated in memory).
@@ -577,6 +579,57 @@ def backward_paths(api, torch, flush, peaks, q, k, v, P):
     tf = backward_flops(B, H, S, D, False) / (ms * 1e-3) / 1e12
     res[f"ulysses_{U}_backward_flow"] = {"ms": ms, "TFLOP/s": tf, "frac_bf16_peak": tf / peak_tf,
                                          "launches": 7, "note": "5 permuted in, backward of 4 head ranks, 3 permuted out"}
+    return res
+
+
+def projection_paths(api, torch, flush, peaks, inputs, B, S, H, D, U):
+    """The Ulysses projections with the all-to-all fused in, on the bench
+    workload's sizes (model width H*D), each rep after an L2 flush: the Q/K/V
+    projection storing the head-sharded layout, and the output projection
+    reading it in place.  For context, the unfused form with a library GEMM
+    (torch.matmul, cuBLAS) and this library's permute kernels is timed beside
+    them; it is not part of this library's path."""
+    Dm = H * D                      # model width = heads x head dim (3072 on image-DiT)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+    xb, wb, wob = inputs.make_projection_inputs(B, S, H, D, Dm, 4321)
+    x, w, wo = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev) for a in (xb, wb, wob))
+    n = B * S * H * D
+    yq, yk, yv, yo = (torch.empty(n, dtype=torch.bfloat16, device=dev) for _ in range(4))
+    out = torch.empty(B * S * Dm, dtype=torch.bfloat16, device=dev)
+    peak_tf = float(peaks["bf16_tflops"])
+    f_qkv = 2.0 * B * S * Dm * 3 * H * D
+    f_out = 2.0 * B * S * H * D * Dm
+    res = {}
+
+    def rec(name, fn, flops, note):
+        ms = median_event_ms(fn, flush, stream)
+        tf = flops / (ms * 1e-3) / 1e12
+        res[name] = {"ms": ms, "TFLOP/s": tf, "frac_bf16_peak": tf / peak_tf, "note": note}
+
+    rec(f"ulysses_{U}_qkv_projection_fused",
+        lambda: api.cpattn_ulysses_qkv_projection(x, w, B, S, H, D, Dm, U, yq=yq, yk=yk, yv=yv, stream=stream),
+        f_qkv, f"X W_qkv^T (Dm {Dm}) stored head-sharded, one launch; FLOPs 2*B*S*Dm*3*H*D")
+    rec(f"ulysses_{U}_output_projection_fused",
+        lambda: api.cpattn_ulysses_output_projection(yq, wo, B, S, H, D, Dm, U, out=out, stream=stream),
+        f_out, "O W_o^T read from the head-sharded layout, one launch; FLOPs 2*B*S*H*D*Dm")
+    x2 = x.view(B * S, Dm)
+    w3 = w.view(3, H * D, Dm)
+    q3, k3, v3 = (torch.empty(n, dtype=torch.bfloat16, device=dev) for _ in range(3))
+
+    def unfused_qkv():
+        for t, y in enumerate((q3, k3, v3)):
+            torch.matmul(x2, w3[t].t(), out=y.view(B * S, H * D))
+        api.cpattn_ulysses_permute_qkv(q3, k3, v3, B, S, H, D, U, yq=yq, yk=yk, yv=yv, stream=stream)
+
+    def unfused_out():
+        api.cpattn_ulysses_unpermute(yq, B, S, H, D, U, x=yo, stream=stream)
+        torch.matmul(yo.view(B * S, H * D), wo.view(Dm, H * D).t(), out=out.view(B * S, Dm))
+
+    rec("context_unfused_qkv_projection_cublas_plus_permute", unfused_qkv, f_qkv,
+        "three library GEMMs (Q, K, V) and the Q/K/V permute kernel (context only)")
+    rec("context_unfused_output_projection_unpermute_plus_cublas", unfused_out, f_out,
+        "unpermute kernel and library GEMM (context only)")
     return res
 
 
@@ -788,6 +841,15 @@ def run_single_kernel(args):
         fn = lambda: api.cpattn_ulysses_permute_qkv(qf, kf, vf, B, S, H, D, U, yq=yq, yk=yk, yv=yv)
     elif args.kernel == "permute":
         fn = lambda: api.cpattn_ulysses_permute(q.reshape(-1), B, S, H, D, U)
+    elif args.kernel in ("qkv_projection", "output_projection"):
+        Dm = H * D
+        xb, wb, wob = inputs.make_projection_inputs(B, S, H, D, Dm, 4321)
+        x, w, wo = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev) for a in (xb, wb, wob))
+        yq, yk, yv = api.cpattn_ulysses_qkv_projection(x, w, B, S, H, D, Dm, U)
+        if args.kernel == "qkv_projection":
+            fn = lambda: api.cpattn_ulysses_qkv_projection(x, w, B, S, H, D, Dm, U, yq=yq, yk=yk, yv=yv)
+        else:
+            fn = lambda: api.cpattn_ulysses_output_projection(yq, wo, B, S, H, D, Dm, U)
     else:
         po = torch.randn((P, B, S, H, D), device=dev)
         pl = torch.randn((P, B, H, S), device=dev)

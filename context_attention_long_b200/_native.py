@@ -31,6 +31,10 @@ SIGNATURES = {
                                            c_int, c_int, c_int, c_int, c_int, c_int, P_INT, P_INT, c_void_p]),
     "cpattn_ulysses_unpermute": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
                                          P_INT, P_INT, c_void_p]),
+    "cpattn_ulysses_qkv_projection": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                              c_int, c_int, c_int, c_int, c_int, c_int, P_INT, P_INT, c_void_p]),
+    "cpattn_ulysses_output_projection": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int,
+                                                 c_int, P_INT, P_INT, c_void_p]),
     "cpattn_head_sharded_attention": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                               c_int, c_int, c_int, c_int, c_int, P_INT, c_void_p]),
     "cpattn_ulysses_workspace_bytes": (c_size_t, [c_int, c_int, c_int, c_int]),

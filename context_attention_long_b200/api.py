@@ -18,12 +18,17 @@ import torch
 from . import _native
 
 __all__ = [
-    "CpattnError", "cpattn_ring_attention", "cpattn_ring_step", "cpattn_lse_merge",
-    "cpattn_kv_gather_attention", "cpattn_ulysses_permute", "cpattn_ulysses_unpermute",
-    "cpattn_head_sharded_attention", "cpattn_ulysses_attention", "cpattn_unified_attention",
-    "cpattn_ulysses_workspace_bytes", "cpattn_unified_workspace_bytes",
-    "cpattn_ulysses_attention_noalloc", "NOALLOC_SCRATCH_BYTES",
-    "cpattn_front_loaded_splits", "cpattn_exchange_bytes", "cpattn_device_status", "cpattn_debug_wait_timeout",
+    "CpattnError", "cpattn_ring_attention", "cpattn_causal_ring_attention", "cpattn_ring_step",
+    "cpattn_causal_ring_step", "cpattn_lse_merge", "cpattn_kv_gather_attention", "cpattn_ulysses_permute",
+    "cpattn_ulysses_permute_qkv", "cpattn_ulysses_unpermute", "cpattn_ulysses_qkv_projection",
+    "cpattn_ulysses_output_projection", "cpattn_head_sharded_attention",
+    "cpattn_causal_head_sharded_attention", "cpattn_ulysses_workspace_bytes",
+    "cpattn_unified_workspace_bytes", "cpattn_ulysses_attention", "cpattn_causal_ulysses_attention",
+    "cpattn_unified_attention", "cpattn_causal_unified_attention",
+    "cpattn_attention_backward_workspace_bytes", "cpattn_attention_backward",
+    "cpattn_ulysses_attention_backward_workspace_bytes", "cpattn_ulysses_attention_backward",
+    "cpattn_ulysses_attention_noalloc", "cpattn_front_loaded_splits", "cpattn_exchange_bytes",
+    "cpattn_plan_exchange", "cpattn_device_status", "cpattn_debug_wait_timeout", "NOALLOC_SCRATCH_BYTES",
     "status_string",
 ]
 
@@ -217,6 +222,40 @@ def cpattn_ulysses_unpermute(y, B, S, H, D, degree, seq_splits=None, head_splits
                                                    _native.int_array(seq_splits), _native.int_array(head_splits),
                                                    _stream(stream)), "cpattn_ulysses_unpermute")
     return x
+
+
+def cpattn_ulysses_qkv_projection(x, w_qkv, B, S, H, D, Dm, degree, seq_splits=None, head_splits=None, yq=None,
+                                  yk=None, yv=None, stream=None):
+    """Q, K, V projections of the sequence-side activations x (rank buffers
+    (B, S_r, Dm) concatenated, bf16) by w_qkv (3*H*D, Dm), stored straight into
+    the head-sharded layout; returns flat (yq, yk, yv) of B*S*H*D bf16 each."""
+    n = _flat_numel(B, S, H, D)
+    yq, yk, yv = (torch.empty(n, dtype=torch.bfloat16, device=x.device) if t is None else t for t in (yq, yk, yv))
+    _need(x, B * S * Dm, torch.bfloat16, "x")
+    _need(w_qkv, 3 * H * D * Dm, torch.bfloat16, "w_qkv")
+    for t, name in ((yq, "yq"), (yk, "yk"), (yv, "yv")):
+        _need(t, n, torch.bfloat16, name)
+    _check(_native.load().cpattn_ulysses_qkv_projection(_ptr(x), _ptr(w_qkv), _ptr(yq), _ptr(yk), _ptr(yv), B, S, H,
+                                                        D, Dm, int(degree), _native.int_array(seq_splits),
+                                                        _native.int_array(head_splits), _stream(stream)),
+           "cpattn_ulysses_qkv_projection")
+    return yq, yk, yv
+
+
+def cpattn_ulysses_output_projection(yo, w_o, B, S, H, D, Dm, degree, seq_splits=None, head_splits=None, out=None,
+                                     stream=None):
+    """Output projection by w_o (Dm, H*D) of the head-sharded attention output yo,
+    read in place; returns the sequence-side result (rank buffers (B, S_r, Dm)
+    concatenated), flat bf16 of B*S*Dm."""
+    out = torch.empty(B * S * Dm, dtype=torch.bfloat16, device=yo.device) if out is None else out
+    _need(yo, _flat_numel(B, S, H, D), torch.bfloat16, "yo")
+    _need(w_o, Dm * H * D, torch.bfloat16, "w_o")
+    _need(out, B * S * Dm, torch.bfloat16, "out")
+    _check(_native.load().cpattn_ulysses_output_projection(_ptr(yo), _ptr(w_o), _ptr(out), B, S, H, D, Dm,
+                                                           int(degree), _native.int_array(seq_splits),
+                                                           _native.int_array(head_splits), _stream(stream)),
+           "cpattn_ulysses_output_projection")
+    return out
 
 
 def _head_sharded(entry, yq, yk, yv, B, S, H, D, degree, head_splits, yo, lse, want_lse, stream):

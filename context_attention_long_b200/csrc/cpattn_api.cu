@@ -24,6 +24,7 @@
 #include "attn_bwd_kernel.cuh"
 #include "merge_kernel.cuh"
 #include "permute_kernel.cuh"
+#include "proj_kernel.cuh"
 
 namespace cpattn {
 
@@ -133,6 +134,21 @@ static bool encode_rows_map(CUtensorMap *tm, const void *ptr, int D, int H, long
   return r == CUDA_SUCCESS;
 }
 
+// 2-D view [rows, cols] of a bf16 row-major matrix, box {64, box_rows},
+// 128-byte swizzle; rows past the end read as zero.
+static bool encode_matrix_map(CUtensorMap *tm, const void *ptr, long long rows, long long cols, int box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------------ launchers
 
 template <int D, bool F32>
@@ -223,6 +239,31 @@ cudaError_t launch_attention_backward(const BwdParams &p, int D, const void *con
   }
   if (units == 0) return cudaSuccess;
   return D == 128 ? launch_bwd_d<128>(p, units, stream) : launch_bwd_d<64>(p, units, stream);
+}
+
+// Persistent projection GEMM: one CTA per SM (or per tile, if fewer).
+static cudaError_t launch_projection(const ProjParams &p, cudaStream_t stream) {
+  static std::mutex mu;
+  static int sms[kMaxDevices] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (sms[dev] == 0) {
+      cudaError_t e = cudaFuncSetAttribute(proj_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           ProjSmem::kAllocBytes);
+      if (e != cudaSuccess) return e;
+      int n = 0;
+      e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+      if (e != cudaSuccess) return e;
+      sms[dev] = std::max(1, n);
+    }
+  }
+  const long long tiles = static_cast<long long>((p.M + kProjBM - 1) / kProjBM) * ((p.N + kProjBN - 1) / kProjBN);
+  if (tiles <= 0) return cudaSuccess;
+  const int grid = static_cast<int>(std::min<long long>(tiles, sms[dev]));
+  proj_gemm_kernel<<<grid, kProjThreads, ProjSmem::kAllocBytes, stream>>>(p);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_permute(const PermuteParams &p, cudaStream_t stream) {
@@ -542,6 +583,60 @@ static int permute_common(const void *src, void *dst, int B, int S, int H, int D
   return CPATTN_OK;
 }
 
+// Shared set-up of the two fused projections: shapes, splits, alignment and
+// (with `fill` non-null, once the device is known to be usable) the rank
+// tables and tensor maps.  QKV: M = B*S sequence-side token rows, N = 3*H*D, K = Dm;
+// OUT: M = B*S tokens (head-side order), N = Dm, K = H*D.
+static int projection_common(const void *a, const void *w, int B, int S, int H, int D, int Dm, int degree,
+                             const int *seq_splits, const int *head_splits, bool out_mode, ProjParams *fill,
+                             ProjParams &pp) {
+  if (a == nullptr || w == nullptr) return CPATTN_ERR_NULL;
+  if (B < 1 || S < 1 || H < 1 || (D != 64 && D != 128)) return CPATTN_ERR_SHAPE;
+  if (Dm < kProjBK || Dm % kProjBK != 0 || Dm > (1 << 20)) return CPATTN_ERR_SHAPE;
+  if (H > kMaxHeads || static_cast<long long>(B) * S > INT_MAX / 2) return CPATTN_ERR_SHAPE;
+  if (3ll * H * D > INT_MAX / 2) return CPATTN_ERR_SHAPE;
+  if (degree < 1 || degree > kMaxRanks) return CPATTN_ERR_DEGREE;
+  std::vector<int> seq, heads;
+  int st = resolve_splits(S, degree, seq_splits, seq);
+  if (st != CPATTN_OK) return st;
+  st = resolve_splits(H, degree, head_splits, heads);
+  if (st != CPATTN_OK) return st;
+  if (!aligned16(a) || !aligned16(w)) return CPATTN_ERR_ALIGNMENT;
+  if (fill == nullptr) return CPATTN_OK;   // arguments checked; nothing encoded yet
+  std::memset(&pp, 0, sizeof(pp));
+  pp.out_mode = out_mode ? 1 : 0;
+  pp.B = B;
+  pp.S = S;
+  pp.H = H;
+  pp.D = D;
+  pp.M = B * S;
+  pp.N = out_mode ? Dm : 3 * H * D;
+  pp.K = out_mode ? H * D : Dm;
+  pp.n_seq = degree;
+  pp.n_head = degree;
+  std::vector<int> so = prefix(seq), ho = prefix(heads);
+  for (int i = 0; i <= degree; ++i) {
+    pp.seq_off[i] = so[i];
+    pp.head_off[i] = ho[i];
+  }
+  for (int u = 0; u < degree; ++u)
+    for (int h = ho[u]; h < ho[u + 1]; ++h) pp.head_rank[h] = static_cast<unsigned short>(u);
+  if (!encode_matrix_map(&pp.tm_w, w, pp.N, pp.K, kProjBN)) return CPATTN_ERR_CUDA;
+  if (out_mode) {
+    const char *base = static_cast<const char *>(a);
+    for (int u = 0; u < degree; ++u) {
+      const int Hu = ho[u + 1] - ho[u];
+      if (Hu == 0) continue;
+      const size_t off = static_cast<size_t>(B) * S * ho[u] * D * 2;
+      if (!encode_rows_map(&pp.tm_a[u], base + off, D, Hu, static_cast<long long>(B) * S)) return CPATTN_ERR_CUDA;
+    }
+  } else if (!encode_matrix_map(&pp.tm_a[0], a, pp.M, pp.K, kProjBM)) {
+    return CPATTN_ERR_CUDA;
+  }
+  pp.timeout_ns = wait_timeout_ns();
+  return CPATTN_OK;
+}
+
 }  // namespace cpattn
 
 using namespace cpattn;
@@ -791,6 +886,40 @@ int cpattn_causal_head_sharded_attention(const void *yq, const void *yk, const v
                                          int H, int S, int D, int degree, const int *head_splits,
                                          cpattn_stream_t stream) {
   return head_sharded_common(yq, yk, yv, yo, lse, B, H, S, D, degree, head_splits, true, stream);
+}
+
+int cpattn_ulysses_qkv_projection(const void *x, const void *w_qkv, void *yq, void *yk, void *yv, int B, int S,
+                                  int H, int D, int Dm, int degree, const int *seq_splits, const int *head_splits,
+                                  cpattn_stream_t stream) {
+  if (yq == nullptr || yk == nullptr || yv == nullptr) return CPATTN_ERR_NULL;
+  ProjParams pp;
+  int st = projection_common(x, w_qkv, B, S, H, D, Dm, degree, seq_splits, head_splits, false, nullptr, pp);
+  if (st != CPATTN_OK) return st;
+  if (!aligned16(yq) || !aligned16(yk) || !aligned16(yv)) return CPATTN_ERR_ALIGNMENT;
+  st = check_device(nullptr);
+  if (st != CPATTN_OK) return st;
+  st = projection_common(x, w_qkv, B, S, H, D, Dm, degree, seq_splits, head_splits, false, &pp, pp);
+  if (st != CPATTN_OK) return st;
+  pp.y[0] = yq;
+  pp.y[1] = yk;
+  pp.y[2] = yv;
+  return launch_projection(pp, stream) == cudaSuccess ? CPATTN_OK : CPATTN_ERR_CUDA;
+}
+
+int cpattn_ulysses_output_projection(const void *yo, const void *w_o, void *out, int B, int S, int H, int D, int Dm,
+                                     int degree, const int *seq_splits, const int *head_splits,
+                                     cpattn_stream_t stream) {
+  if (out == nullptr) return CPATTN_ERR_NULL;
+  ProjParams pp;
+  int st = projection_common(yo, w_o, B, S, H, D, Dm, degree, seq_splits, head_splits, true, nullptr, pp);
+  if (st != CPATTN_OK) return st;
+  if (!aligned16(out)) return CPATTN_ERR_ALIGNMENT;
+  st = check_device(nullptr);
+  if (st != CPATTN_OK) return st;
+  st = projection_common(yo, w_o, B, S, H, D, Dm, degree, seq_splits, head_splits, true, &pp, pp);
+  if (st != CPATTN_OK) return st;
+  pp.y[0] = out;
+  return launch_projection(pp, stream) == cudaSuccess ? CPATTN_OK : CPATTN_ERR_CUDA;
 }
 
 size_t cpattn_ulysses_workspace_bytes(int B, int H, int S, int D) {

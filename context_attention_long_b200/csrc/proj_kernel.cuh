@@ -1,0 +1,306 @@
+// proj_kernel.cuh -- the Ulysses projections with the all-to-all fused in.
+//
+// The Ulysses flow (the Ulysses Sequence Parallelism article, section 4):
+// each rank projects its own sequence chunk to Q, K and V, the first
+// all-to-all regroups them by head, local attention runs, the second
+// all-to-all regroups the output by token, and each rank applies the output
+// projection to its own chunk.  Emulated on one GPU the all-to-alls are the
+// permutations of permute_kernel.cuh; here they are folded into the two
+// projection GEMMs instead:
+//   QKV mode:  C = X W_qkv^T over the sequence-side token rows, and the
+//              epilogue stores each (token, head) run of D outputs straight
+//              into its head rank's buffer (the first all-to-all);
+//   OUT mode:  C = O W_o^T over the tokens, whose A operand is loaded by TMA
+//              from the head ranks' buffers (one tensor map per head rank,
+//              chosen per 64-wide K block), and the epilogue stores each
+//              token row into its sequence rank's buffer (the second
+//              all-to-all).
+// Layouts as in permute_kernel.cuh: the sequence side is the rank buffers
+// (B, S_r, .) concatenated in rank order, the head side the rank buffers
+// (B, S, H_u, D).  W is (N, K) row-major (the nn.Linear layout); the columns
+// of W_qkv are [Q heads | K heads | V heads], head h at [h*D, (h+1)*D).
+//
+// Kernel: persistent, one CTA per SM, 128 x 256 output tiles, K in blocks of
+// 64 (one 128-byte swizzle row), 4-stage TMA ring, tcgen05.mma (M = 128,
+// N = 256, bf16 in, f32 accumulate) into one of two 256-column TMEM
+// accumulators, so that the epilogue of tile i overlaps the main loop of
+// tile i + 1:
+//   warp 0      TMA producer (A tile 16 KB + W tile 32 KB per stage)
+//   warp 1      TMEM allocator + single-thread MMA issuer
+//   warps 2-5   epilogue: one accumulator row per thread (TMEM lane
+//               (warp % 4) * 32 + lane), bf16 rounding, permuted stores
+// Every wait is bounded as in attn_kernel.cuh.
+#pragma once
+
+#include "cpattn_internal.h"
+#include "cpattn_ptx.cuh"
+
+namespace cpattn {
+
+constexpr int kProjThreads = 192;
+constexpr int kProjBM = 128;
+constexpr int kProjBN = 256;
+constexpr int kProjBK = 64;
+constexpr int kProjStages = 4;
+constexpr int kProjMaxMaps = kMaxRanks;
+constexpr uint32_t kProjTmemCols = 512;
+
+struct ProjSmem {
+  static constexpr int kABytes = kProjBM * kProjBK * 2;   // 16 KB
+  static constexpr int kWBytes = kProjBN * kProjBK * 2;   // 32 KB
+  static constexpr int kOffA = 0;
+  static constexpr int kOffW = kOffA + kProjStages * kABytes;
+  static constexpr int kOffBar = kOffW + kProjStages * kWBytes;
+  // full[S], empty[S], acc_full[2], acc_empty[2], tail
+  static constexpr int kNumBars = 2 * kProjStages + 5;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kBytes = kOffMisc + 16;
+  static constexpr int kAllocBytes = kBytes + 1024;
+};
+
+struct alignas(64) ProjParams {
+  CUtensorMap tm_a[kProjMaxMaps];   // QKV: [0] = X as 2-D [M, K]; OUT: head rank u as 3-D [B*S, H_u, D]
+  CUtensorMap tm_w;                 // 2-D [N, K]
+  int out_mode;                     // 0: QKV (permuting stores), 1: OUT (gathering loads)
+  int M, N, K;                      // token rows, output columns, reduction length
+  int B, S, H, D;
+  int n_seq, n_head;
+  int seq_off[kMaxRanks + 1];       // token offsets of the sequence ranks
+  int head_off[kMaxRanks + 1];      // head offsets of the head ranks
+  unsigned short head_rank[kMaxHeads];
+  void *y[3];                       // QKV: head-side Q, K, V; OUT: y[0] = sequence-side output
+  unsigned long long timeout_ns;
+};
+
+// 2-D tiled bulk tensor load global -> shared (no multicast).
+__device__ __forceinline__ void proj_tma_load_2d(uint32_t smem_dst, const CUtensorMap *tm, int c0, int c1,
+                                                 uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+
+// Tile order: groups of kProjGroupM row tiles, column tiles walked inside a
+// group.  The CTAs running at once then share a few row tiles of A (kept in
+// L2 while every column tile of the group passes) and a few column tiles of
+// W, instead of streaming all of A from HBM once per column tile.
+constexpr int kProjGroupM = 16;
+__device__ __forceinline__ void proj_tile(int tile, int mt, int nt, int &mi, int &ni) {
+  const int group = tile / (kProjGroupM * nt);
+  const int first = group * kProjGroupM;
+  const int gm = min(kProjGroupM, mt - first);
+  const int within = tile - group * kProjGroupM * nt;
+  mi = first + within % gm;
+  ni = within / gm;
+}
+
+__device__ __forceinline__ int proj_find(const int *off, int n, int x) {
+  // largest i in [0, n) with off[i] <= x (empty ranges are skipped)
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (off[mid] <= x) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__global__ void __launch_bounds__(kProjThreads, 1) proj_gemm_kernel(const __grid_constant__ ProjParams p) {
+  using L = ProjSmem;
+  constexpr uint32_t IDESC = idesc_bf16_f32(kProjBM, kProjBN, false);
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t sb = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  constexpr uint32_t BAR_FULL = L::kOffBar;                       // [S]
+  constexpr uint32_t BAR_EMPTY = BAR_FULL + 8 * kProjStages;      // [S]
+  constexpr uint32_t BAR_AF = BAR_EMPTY + 8 * kProjStages;        // [2] accumulator written
+  constexpr uint32_t BAR_AE = BAR_AF + 16;                        // [2] accumulator read out
+  constexpr uint32_t BAR_TAIL = BAR_AE + 16;
+  constexpr uint32_t TMEM_SLOT = L::kOffMisc;
+  constexpr uint32_t ABORT = L::kOffMisc + 4;
+  static_assert(BAR_TAIL + 8 <= L::kOffMisc, "barrier area");
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint64_t tmo = p.timeout_ns;
+  const int mt = (p.M + kProjBM - 1) / kProjBM;
+  const int nt = (p.N + kProjBN - 1) / kProjBN;
+  const int n_tiles = mt * nt;
+  const int nkb = p.K / kProjBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kProjStages; ++s) {
+      mbar_init(sb + BAR_FULL + 8 * s, 1);
+      mbar_init(sb + BAR_EMPTY + 8 * s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(sb + BAR_AF + 8 * a, 1);
+      mbar_init(sb + BAR_AE + 8 * a, 4);   // one arrival per epilogue warp
+    }
+    mbar_init(sb + BAR_TAIL, 1);
+    st_shared_volatile(sb + ABORT, 0u);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(sb + TMEM_SLOT, kProjTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ld_shared_volatile(sb + TMEM_SLOT);
+  const uint32_t abort_flag = sb + ABORT;
+
+  if (warp == 0) {
+    // ================================================================ producer
+    if (lane == 0) {
+      if (p.out_mode) {
+        for (int u = 0; u < p.n_head; ++u)
+          if (p.head_off[u + 1] > p.head_off[u]) tma_prefetch_desc(&p.tm_a[u]);
+      } else {
+        tma_prefetch_desc(&p.tm_a[0]);
+      }
+      tma_prefetch_desc(&p.tm_w);
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x) {
+        int mi, ni;
+        proj_tile(tile, mt, nt, mi, ni);
+        const int m0 = mi * kProjBM;
+        const int n0 = ni * kProjBN;
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int st = it % kProjStages;
+          const uint32_t ph = (it / kProjStages) & 1;
+          if (!mbar_wait(sb + BAR_EMPTY + 8 * st, ph ^ 1, abort_flag, tmo, SITE_PRODUCER)) { ok = false; break; }
+          const uint32_t full = sb + BAR_FULL + 8 * st;
+          mbar_arrive_expect_tx(full, L::kABytes + L::kWBytes);
+          const uint32_t sA = sb + L::kOffA + st * L::kABytes;
+          if (p.out_mode) {
+            const int k0 = kb * kProjBK;
+            const int h = k0 / p.D;
+            const int u = p.head_rank[h];
+            tma_load_3d(sA, &p.tm_a[u], k0 - h * p.D, h - p.head_off[u], m0, full);
+          } else {
+            proj_tma_load_2d(sA, &p.tm_a[0], kb * kProjBK, m0, full);
+          }
+          proj_tma_load_2d(sb + L::kOffW + st * L::kWBytes, &p.tm_w, kb * kProjBK, n0, full);
+        }
+      }
+      // No load may still be landing in shared memory when the CTA exits:
+      // wait for the last loads of every stage (abort ignored, time-bounded).
+      for (int j = 0; j < kProjStages && j < it; ++j) {
+        const int i = it - 1 - j;
+        mbar_wait(sb + BAR_FULL + 8 * (i % kProjStages), (i / kProjStages) & 1, 0u, tmo, SITE_TAIL);
+      }
+    }
+  } else if (warp == 1) {
+    // ============================================================== MMA issuer
+    if (lane == 0) {
+      int it = 0, local = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x, ++local) {
+        const int a = local & 1;
+        if (!mbar_wait_spin(sb + BAR_AE + 8 * a, ((local >> 1) & 1) ^ 1, abort_flag, tmo, SITE_MMA)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + a * kProjBN;
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int st = it % kProjStages;
+          const uint32_t ph = (it / kProjStages) & 1;
+          if (!mbar_wait_spin(sb + BAR_FULL + 8 * st, ph, abort_flag, tmo, SITE_MMA)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t da = smem_desc_sw128(sb + L::kOffA + st * L::kABytes, 16, 1024);
+          const uint64_t dw = smem_desc_sw128(sb + L::kOffW + st * L::kWBytes, 16, 1024);
+#pragma unroll
+          for (int kk = 0; kk < kProjBK / 16; ++kk)
+            mma_ss(d, da + ((kk * 32) >> 4), dw + ((kk * 32) >> 4), IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(sb + BAR_EMPTY + 8 * st);
+        }
+        if (ok) mma_commit(sb + BAR_AF + 8 * a);
+      }
+      // Drain: every issued MMA has completed before TMEM is released.
+      mma_commit(sb + BAR_TAIL);
+      mbar_wait(sb + BAR_TAIL, 0, 0u, tmo, SITE_TAIL);
+    }
+  } else {
+    // ================================================================ epilogue
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;   // accumulator row = TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const int HD = p.H * p.D;
+    int local = 0;
+    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++local) {
+      const int a = local & 1;
+      const bool w = mbar_wait(sb + BAR_AF + 8 * a, (local >> 1) & 1, abort_flag, tmo, SITE_EPILOGUE);
+      if (__any_sync(0xffffffffu, !w)) break;
+      __syncwarp();
+      tc_fence_after();
+      int mi, ni;
+      proj_tile(tile, mt, nt, mi, ni);
+      const int m = mi * kProjBM + r;
+      const int n0 = ni * kProjBN;
+      const bool row_ok = m < p.M;
+      // Row-dependent part of the destination.
+      long long row_elems = 0;   // OUT: element offset of the row; QKV: token index (b*S + s)
+      if (row_ok) {
+        if (p.out_mode) {
+          const int b = m / p.S, s = m - (m / p.S) * p.S;
+          const int rs = proj_find(p.seq_off, p.n_seq, s);
+          const int len = p.seq_off[rs + 1] - p.seq_off[rs];
+          row_elems = (static_cast<long long>(p.B) * p.seq_off[rs] + static_cast<long long>(b) * len +
+                       (s - p.seq_off[rs])) * p.N;
+        } else {
+          // sequence-side order: rank rs, batch b, local position
+          int lo = 0, hi = p.n_seq - 1;
+          while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (p.B * p.seq_off[mid] <= m) lo = mid; else hi = mid - 1;
+          }
+          const int len = p.seq_off[lo + 1] - p.seq_off[lo];
+          const int within = m - p.B * p.seq_off[lo];
+          const int b = within / len;
+          row_elems = static_cast<long long>(b) * p.S + p.seq_off[lo] + (within - b * len);
+        }
+      }
+#pragma unroll 1
+      for (int c = 0; c < kProjBN; c += 32) {
+        uint32_t v[32];
+        __syncwarp();
+        tmem_ld32_wait(tmem + lane_base + a * kProjBN + c, v);   // the whole warp, converged
+        const int n = n0 + c;
+        if (!row_ok || n >= p.N) continue;                         // store skipped; lanes rejoin above
+        __nv_bfloat16 *dst;
+        if (p.out_mode) {
+          dst = static_cast<__nv_bfloat16 *>(p.y[0]) + row_elems + n;
+        } else {
+          const int t = n / HD;
+          const int h = (n - t * HD) / p.D;
+          const int u = p.head_rank[h];
+          const int Hu = p.head_off[u + 1] - p.head_off[u];
+          const long long base = static_cast<long long>(p.B) * p.S * p.head_off[u] * p.D;
+          dst = static_cast<__nv_bfloat16 *>(p.y[t]) + base +
+                (row_elems * Hu + (h - p.head_off[u])) * p.D + (n - t * HD - h * p.D);
+        }
+        uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          d4[k] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * k]), __uint_as_float(v[8 * k + 1])),
+                             pack_bf16x2(__uint_as_float(v[8 * k + 2]), __uint_as_float(v[8 * k + 3])),
+                             pack_bf16x2(__uint_as_float(v[8 * k + 4]), __uint_as_float(v[8 * k + 5])),
+                             pack_bf16x2(__uint_as_float(v[8 * k + 6]), __uint_as_float(v[8 * k + 7])));
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sb + BAR_AE + 8 * a);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kProjTmemCols);
+  }
+}
+
+}  // namespace cpattn

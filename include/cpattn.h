@@ -203,6 +203,51 @@ int cpattn_ulysses_unpermute(const void *y, void *x, int B, int S, int H, int D,
                              cpattn_stream_t stream);
 
 /*
+ * The Ulysses projections with the all-to-alls fused in ([USP] section 4: each
+ * rank projects its sequence chunk to Q, K and V, the first all-to-all
+ * regroups them by head, and after local attention and the second all-to-all
+ * each rank applies the output projection to its chunk).
+ *
+ * cpattn_ulysses_qkv_projection: for every sequence rank r,
+ *     QKV_r = X_r W_qkv^T   (bf16 in, fp32 accumulate, rounded to bf16),
+ * split into Q | K | V, each (B, S_r, H, D), and stored directly in the
+ * head-sharded layout: the result equals cpattn_ulysses_permute_qkv applied
+ * to the three unfused projections, with no intermediate tensor.
+ *   x          sequence side: rank buffers (B, S_r, Dm) concatenated in rank
+ *              order, bf16 (for B = 1 the plain (S, Dm) activations).
+ *   w_qkv      (3*H*D, Dm) bf16 row-major (the nn.Linear weight layout):
+ *              rows [t*H*D + h*D, t*H*D + (h+1)*D) are head h of Q (t = 0),
+ *              K (t = 1) or V (t = 2).
+ *   yq, yk, yv head side: rank buffers (B, S, H_u, D) concatenated, bf16.
+ *   Dm         model width, a positive multiple of 64.  D is 64 or 128.
+ *   degree, seq_splits, head_splits as cpattn_ulysses_permute.
+ * No bias is added.
+ *
+ * cpattn_ulysses_output_projection: the second all-to-all fused into the
+ * output projection.  For every sequence rank r,
+ *     out_r = O_r W_o^T,  O_r = the rank's tokens of every head, (B, S_r, H*D),
+ * where O_r is read straight from the head-sharded attention output yo (the
+ * result equals cpattn_ulysses_unpermute followed by the projection).
+ *   yo         head side, as yq above (bf16).
+ *   w_o        (Dm, H*D) bf16 row-major.
+ *   out        sequence side: rank buffers (B, S_r, Dm) concatenated, bf16.
+ *
+ * All pointers are device memory owned by the caller, 16-byte aligned; inputs
+ * and outputs must not alias.  Errors: CPATTN_ERR_NULL, CPATTN_ERR_SHAPE (B, S,
+ * H < 1, D not 64/128, Dm not a positive multiple of 64, H > 1024),
+ * CPATTN_ERR_DEGREE (degree outside 1..64), CPATTN_ERR_INDIVISIBLE,
+ * CPATTN_ERR_SPLITS, CPATTN_ERR_ALIGNMENT, CPATTN_ERR_UNSUPPORTED,
+ * CPATTN_ERR_CUDA; nothing is launched on an error.
+ */
+int cpattn_ulysses_qkv_projection(const void *x, const void *w_qkv, void *yq, void *yk, void *yv,
+                                  int B, int S, int H, int D, int Dm, int degree,
+                                  const int *seq_splits, const int *head_splits,
+                                  cpattn_stream_t stream);
+int cpattn_ulysses_output_projection(const void *yo, const void *w_o, void *out, int B, int S,
+                                     int H, int D, int Dm, int degree, const int *seq_splits,
+                                     const int *head_splits, cpattn_stream_t stream);
+
+/*
  * Head-sharded local attention ([USP] section 4: after the first all-to-all
  * every GPU runs ordinary attention over all tokens of its heads): for every
  * head rank r', attention of its [B, S, head_r', D] Q/K/V buffers.

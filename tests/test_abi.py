@@ -126,6 +126,37 @@ def test_permute_validation(lib):
     assert t(H=5) == INDIV
 
 
+def test_projection_validation(lib):
+    def q(x=FAKE, w=FAKE, yq=FAKE, yv=FAKE, B=1, S=8, H=4, D=64, Dm=128, P=2, seq=None, heads=None):
+        return lib.cpattn_ulysses_qkv_projection(x, w, yq, FAKE, yv, B, S, H, D, Dm, P, _native.int_array(seq),
+                                                 _native.int_array(heads), None)
+    assert q(x=None) == NULL
+    assert q(w=None) == NULL
+    assert q(yv=None) == NULL
+    assert q(D=32) == SHAPE
+    assert q(Dm=96) == SHAPE            # Dm must be a multiple of 64
+    assert q(Dm=0) == SHAPE
+    assert q(B=0) == SHAPE
+    assert q(H=2000) == SHAPE
+    assert q(P=0) == DEGREE
+    assert q(P=65) == DEGREE
+    assert q(H=5) == INDIV
+    assert q(S=9, seq=[5, 5]) == SPLITS
+    assert q(H=5, heads=[4, 2]) == SPLITS
+    assert q(x=FAKE_MIS) == ALIGN
+    assert q(yq=FAKE_MIS) == ALIGN
+
+    def o(yo=FAKE, w=FAKE, out=FAKE, H=4, D=64, Dm=128, P=2):
+        return lib.cpattn_ulysses_output_projection(yo, w, out, 1, 8, H, D, Dm, P, None, None, None)
+    assert o(out=None) == NULL
+    assert o(yo=None) == NULL
+    assert o(Dm=100) == SHAPE
+    assert o(D=96) == SHAPE
+    assert o(H=5) == INDIV
+    assert o(out=FAKE_MIS) == ALIGN
+    assert o(w=FAKE_MIS) == ALIGN
+
+
 def test_flow_validation(lib):
     need = lib.cpattn_ulysses_workspace_bytes(1, 4, 8, 64)
     assert need == 4 * 1 * 8 * 4 * 64 * 2
