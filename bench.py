@@ -790,6 +790,12 @@ def run_sweep(args):
                           backward_flops(B, H, S, D, True)))
         if name in ("dit", "hires", "video"):
             paths += library_context_paths(torch, q, k, v, cflops)
+        if name in ("dit", "video"):
+            U_p = cfg["ulysses_degree"]
+            for key, r in projection_paths(api, torch, flush, peaks, inputs, B, S, H, D, U_p).items():
+                print(json.dumps({"workload": name, "shape": f"B{B} H{H} S{S} D{D} Dm{H * D}", "path": key,
+                                  "ms": round(r["ms"], 4), "TFLOP/s": round(r["TFLOP/s"], 1),
+                                  "frac_bf16_peak": round(r["frac_bf16_peak"], 4), "peak_kind": kind}), flush=True)
         for entry in paths:
             label, fn = entry[0], entry[1]
             try:
