@@ -241,29 +241,47 @@ cudaError_t launch_attention_backward(const BwdParams &p, int D, const void *con
   return D == 128 ? launch_bwd_d<128>(p, units, stream) : launch_bwd_d<64>(p, units, stream);
 }
 
-// Persistent projection GEMM: one CTA per SM (or per tile, if fewer).
+// Persistent projection GEMM in clusters of two CTAs: as many clusters as
+// can be resident at once (or one per 256 x 256 tile, if fewer), so that
+// every cluster runs from the start and the tile stride covers all tiles.
 static cudaError_t launch_projection(const ProjParams &p, cudaStream_t stream) {
   static std::mutex mu;
-  static int sms[kMaxDevices] = {0};
+  static int clusters[kMaxDevices] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kProjThreads, 1, 1);
+  cfg.dynamicSmemBytes = ProjSmem::kAllocBytes;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   {
     std::lock_guard<std::mutex> lock(mu);
-    if (sms[dev] == 0) {
+    if (clusters[dev] == 0) {
       cudaError_t e = cudaFuncSetAttribute(proj_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            ProjSmem::kAllocBytes);
       if (e != cudaSuccess) return e;
-      int n = 0;
-      e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+      int sms = 0;
+      e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
       if (e != cudaSuccess) return e;
-      sms[dev] = std::max(1, n);
+      cfg.gridDim = dim3(2 * std::max(1, sms / 2), 1, 1);
+      int n = 0;
+      e = cudaOccupancyMaxActiveClusters(&n, proj_gemm_kernel, &cfg);
+      if (e != cudaSuccess) return e;
+      if (n < 1) return cudaErrorInvalidConfiguration;
+      clusters[dev] = n;
     }
   }
-  const long long tiles = static_cast<long long>((p.M + kProjBM - 1) / kProjBM) * ((p.N + kProjBN - 1) / kProjBN);
+  const long long tiles = static_cast<long long>((p.M + 2 * kProjBM - 1) / (2 * kProjBM)) *
+                          ((p.N + kProjBN - 1) / kProjBN);
   if (tiles <= 0) return cudaSuccess;
-  const int grid = static_cast<int>(std::min<long long>(tiles, sms[dev]));
-  proj_gemm_kernel<<<grid, kProjThreads, ProjSmem::kAllocBytes, stream>>>(p);
-  return cudaGetLastError();
+  cfg.gridDim = dim3(2 * static_cast<unsigned>(std::min<long long>(tiles, clusters[dev])), 1, 1);
+  return cudaLaunchKernelEx(&cfg, proj_gemm_kernel, p);
 }
 
 cudaError_t launch_permute(const PermuteParams &p, cudaStream_t stream) {
@@ -621,7 +639,7 @@ static int projection_common(const void *a, const void *w, int B, int S, int H, 
   }
   for (int u = 0; u < degree; ++u)
     for (int h = ho[u]; h < ho[u + 1]; ++h) pp.head_rank[h] = static_cast<unsigned short>(u);
-  if (!encode_matrix_map(&pp.tm_w, w, pp.N, pp.K, kProjBN)) return CPATTN_ERR_CUDA;
+  if (!encode_matrix_map(&pp.tm_w, w, pp.N, pp.K, kProjBN / 2)) return CPATTN_ERR_CUDA;
   if (out_mode) {
     const char *base = static_cast<const char *>(a);
     for (int u = 0; u < degree; ++u) {

@@ -20,16 +20,24 @@
 // (B, S, H_u, D).  W is (N, K) row-major (the nn.Linear layout); the columns
 // of W_qkv are [Q heads | K heads | V heads], head h at [h*D, (h+1)*D).
 //
-// Kernel: persistent, one CTA per SM, 128 x 256 output tiles, K in blocks of
-// 64 (one 128-byte swizzle row), 4-stage TMA ring, tcgen05.mma (M = 128,
-// N = 256, bf16 in, f32 accumulate) into one of two 256-column TMEM
-// accumulators, so that the epilogue of tile i overlaps the main loop of
-// tile i + 1:
-//   warp 0      TMA producer (A tile 16 KB + W tile 32 KB per stage)
-//   warp 1      TMEM allocator + single-thread MMA issuer
+// Kernel: persistent, clusters of two CTAs on an SM pair.  Each cluster
+// computes 256 x 256 output tiles with tcgen05.mma.cta_group::2 (M = 256,
+// N = 256, bf16 in, f32 accumulate): each CTA holds 128 rows of the A tile
+// and half of the W tile in shared memory, so every SM stages and reads only
+// half of W.  (With one SM per 128 x 256 tile the TMA writes plus the MMA's
+// operand reads need about 190 B/clk of shared-memory bandwidth against 128;
+// the pair needs about 125.)  K in blocks of 64 (one 128-byte swizzle row),
+// a 6-stage TMA ring per CTA, two 256-column TMEM accumulators per CTA so
+// that the epilogue of tile i overlaps the main loop of tile i + 1:
+//   warp 0      TMA producer (A 16 KB + half of W 16 KB per stage); both
+//               CTAs' loads complete on the leader CTA's stage barrier
+//   warp 1      TMEM allocator (both CTAs, one paired allocation) and, in
+//               the leader CTA, the single-thread MMA issuer; its commits
+//               reach the barriers of both CTAs
 //   warps 2-5   epilogue: one accumulator row per thread (TMEM lane
-//               (warp % 4) * 32 + lane), bf16 rounding, permuted stores
-// Every wait is bounded as in attn_kernel.cuh.
+//               (warp % 4) * 32 + lane), bf16 rounding, permuted stores;
+//               accumulator releases go to the leader's barrier
+// Every mbarrier wait is bounded as in attn_kernel.cuh.
 #pragma once
 
 #include "cpattn_internal.h"
@@ -38,16 +46,16 @@
 namespace cpattn {
 
 constexpr int kProjThreads = 192;
-constexpr int kProjBM = 128;
-constexpr int kProjBN = 256;
+constexpr int kProjBM = 128;          // rows per CTA (the cluster tile has 256)
+constexpr int kProjBN = 256;          // columns per tile (each CTA stages half of W's rows)
 constexpr int kProjBK = 64;
-constexpr int kProjStages = 4;
+constexpr int kProjStages = 6;
 constexpr int kProjMaxMaps = kMaxRanks;
 constexpr uint32_t kProjTmemCols = 512;
 
 struct ProjSmem {
-  static constexpr int kABytes = kProjBM * kProjBK * 2;   // 16 KB
-  static constexpr int kWBytes = kProjBN * kProjBK * 2;   // 32 KB
+  static constexpr int kABytes = kProjBM * kProjBK * 2;         // 16 KB
+  static constexpr int kWBytes = (kProjBN / 2) * kProjBK * 2;   // 16 KB: this CTA's half of W
   static constexpr int kOffA = 0;
   static constexpr int kOffW = kOffA + kProjStages * kABytes;
   static constexpr int kOffBar = kOffW + kProjStages * kWBytes;
@@ -60,7 +68,7 @@ struct ProjSmem {
 
 struct alignas(64) ProjParams {
   CUtensorMap tm_a[kProjMaxMaps];   // QKV: [0] = X as 2-D [M, K]; OUT: head rank u as 3-D [B*S, H_u, D]
-  CUtensorMap tm_w;                 // 2-D [N, K]
+  CUtensorMap tm_w;                 // 2-D [N, K], box of 128 rows (half a tile)
   int out_mode;                     // 0: QKV (permuting stores), 1: OUT (gathering loads)
   int M, N, K;                      // token rows, output columns, reduction length
   int B, S, H, D;
@@ -82,11 +90,80 @@ __device__ __forceinline__ void proj_tma_load_2d(uint32_t smem_dst, const CUtens
       : "memory");
 }
 
+// ------------------------------------------------ CTA-pair (cta_group::2) forms
+__device__ __forceinline__ uint32_t proj_cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Shared::cluster address of the same shared-memory offset in CTA `rank`.
+__device__ __forceinline__ uint32_t proj_mapa(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void proj_cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void proj_arrive_remote(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
+// Tile loads into this CTA's shared memory whose completion is counted on the
+// leader CTA's barrier (a shared::cluster address).  No multicast.
+__device__ __forceinline__ void proj_tma_load_2d_pair(uint32_t smem_dst, const CUtensorMap *tm, int c0, int c1,
+                                                      uint32_t cluster_bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(cluster_bar)
+      : "memory");
+}
+__device__ __forceinline__ void proj_tma_load_3d_pair(uint32_t smem_dst, const CUtensorMap *tm, int c0, int c1,
+                                                      int c2, uint32_t cluster_bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(c2), "r"(cluster_bar)
+      : "memory");
+}
+__device__ __forceinline__ void proj_tmem_alloc_pair(uint32_t smem_result, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_result), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void proj_tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void proj_tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// D[tmem of both CTAs] (+)= A (128 rows in each CTA) * W^T (half of W's rows in each CTA).
+__device__ __forceinline__ void proj_mma_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive once on the barrier at offset `bar` of both CTAs of the pair when
+// every tcgen05 operation issued so far by this thread has completed.
+__device__ __forceinline__ void proj_commit_pair_both(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"(static_cast<uint16_t>(3))
+      : "memory");
+}
+// The same, on this CTA's barrier only.
+__device__ __forceinline__ void proj_commit_pair_self(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
 // Tile order: groups of kProjGroupM row tiles, column tiles walked inside a
 // group.  The CTAs running at once then share a few row tiles of A (kept in
 // L2 while every column tile of the group passes) and a few column tiles of
 // W, instead of streaming all of A from HBM once per column tile.
-constexpr int kProjGroupM = 16;
+constexpr int kProjGroupM = 8;   // of 256-row cluster tiles
 __device__ __forceinline__ void proj_tile(int tile, int mt, int nt, int &mi, int &ni) {
   const int group = tile / (kProjGroupM * nt);
   const int first = group * kProjGroupM;
@@ -106,15 +183,17 @@ __device__ __forceinline__ int proj_find(const int *off, int n, int x) {
   return lo;
 }
 
+// Launched in clusters of 2 CTAs (cudaLaunchAttributeClusterDimension), grid
+// even; CTA rank 0 of each cluster leads.
 __global__ void __launch_bounds__(kProjThreads, 1) proj_gemm_kernel(const __grid_constant__ ProjParams p) {
   using L = ProjSmem;
-  constexpr uint32_t IDESC = idesc_bf16_f32(kProjBM, kProjBN, false);
+  constexpr uint32_t IDESC = idesc_bf16_f32(2 * kProjBM, kProjBN, false);   // M = 256 over the pair
   extern __shared__ uint8_t smem_raw[];
   const uint32_t sb = (smem_u32(smem_raw) + 1023u) & ~1023u;
-  constexpr uint32_t BAR_FULL = L::kOffBar;                       // [S]
-  constexpr uint32_t BAR_EMPTY = BAR_FULL + 8 * kProjStages;      // [S]
+  constexpr uint32_t BAR_FULL = L::kOffBar;                       // [S] leader: both CTAs' loads landed
+  constexpr uint32_t BAR_EMPTY = BAR_FULL + 8 * kProjStages;      // [S] this CTA's stage consumed
   constexpr uint32_t BAR_AF = BAR_EMPTY + 8 * kProjStages;        // [2] accumulator written
-  constexpr uint32_t BAR_AE = BAR_AF + 16;                        // [2] accumulator read out
+  constexpr uint32_t BAR_AE = BAR_AF + 16;                        // [2] leader: accumulator read out by both
   constexpr uint32_t BAR_TAIL = BAR_AE + 16;
   constexpr uint32_t TMEM_SLOT = L::kOffMisc;
   constexpr uint32_t ABORT = L::kOffMisc + 4;
@@ -122,8 +201,12 @@ __global__ void __launch_bounds__(kProjThreads, 1) proj_gemm_kernel(const __grid
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = proj_cluster_rank();       // 0: leader (issues the MMAs), 1: peer
+  const bool leader = rank == 0;
+  const int cluster = blockIdx.x >> 1;
+  const int n_clusters = gridDim.x >> 1;
   const uint64_t tmo = p.timeout_ns;
-  const int mt = (p.M + kProjBM - 1) / kProjBM;
+  const int mt = (p.M + 2 * kProjBM - 1) / (2 * kProjBM);
   const int nt = (p.N + kProjBN - 1) / kProjBN;
   const int n_tiles = mt * nt;
   const int nkb = p.K / kProjBK;
@@ -135,18 +218,20 @@ __global__ void __launch_bounds__(kProjThreads, 1) proj_gemm_kernel(const __grid
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(sb + BAR_AF + 8 * a, 1);
-      mbar_init(sb + BAR_AE + 8 * a, 4);   // one arrival per epilogue warp
+      mbar_init(sb + BAR_AE + 8 * a, 8);   // one arrival per epilogue warp of both CTAs
     }
     mbar_init(sb + BAR_TAIL, 1);
     st_shared_volatile(sb + ABORT, 0u);
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(sb + TMEM_SLOT, kProjTmemCols);
-    tmem_relinquish();
+    proj_tmem_alloc_pair(sb + TMEM_SLOT, kProjTmemCols);
+    proj_tmem_relinquish_pair();
   }
   tc_fence_before();
   __syncthreads();
+  // Both CTAs' barriers are initialised before either signals the other's.
+  proj_cluster_sync();
   tc_fence_after();
   const uint32_t tmem = ld_shared_volatile(sb + TMEM_SLOT);
   const uint32_t abort_flag = sb + ABORT;
@@ -163,42 +248,42 @@ __global__ void __launch_bounds__(kProjThreads, 1) proj_gemm_kernel(const __grid
       tma_prefetch_desc(&p.tm_w);
       int it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x) {
+      for (int tile = cluster; ok && tile < n_tiles; tile += n_clusters) {
         int mi, ni;
         proj_tile(tile, mt, nt, mi, ni);
-        const int m0 = mi * kProjBM;
-        const int n0 = ni * kProjBN;
+        const int m0 = mi * 2 * kProjBM + static_cast<int>(rank) * kProjBM;   // this CTA's 128 rows
+        const int w0 = ni * kProjBN + static_cast<int>(rank) * (kProjBN / 2);  // this CTA's half of W
         for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int st = it % kProjStages;
           const uint32_t ph = (it / kProjStages) & 1;
           if (!mbar_wait(sb + BAR_EMPTY + 8 * st, ph ^ 1, abort_flag, tmo, SITE_PRODUCER)) { ok = false; break; }
-          const uint32_t full = sb + BAR_FULL + 8 * st;
-          mbar_arrive_expect_tx(full, L::kABytes + L::kWBytes);
+          const uint32_t full = proj_mapa(sb + BAR_FULL + 8 * st, 0);   // the leader's stage barrier
+          if (leader) mbar_arrive_expect_tx(sb + BAR_FULL + 8 * st, 2 * (L::kABytes + L::kWBytes));
           const uint32_t sA = sb + L::kOffA + st * L::kABytes;
           if (p.out_mode) {
             const int k0 = kb * kProjBK;
             const int h = k0 / p.D;
             const int u = p.head_rank[h];
-            tma_load_3d(sA, &p.tm_a[u], k0 - h * p.D, h - p.head_off[u], m0, full);
+            proj_tma_load_3d_pair(sA, &p.tm_a[u], k0 - h * p.D, h - p.head_off[u], m0, full);
           } else {
-            proj_tma_load_2d(sA, &p.tm_a[0], kb * kProjBK, m0, full);
+            proj_tma_load_2d_pair(sA, &p.tm_a[0], kb * kProjBK, m0, full);
           }
-          proj_tma_load_2d(sb + L::kOffW + st * L::kWBytes, &p.tm_w, kb * kProjBK, n0, full);
+          proj_tma_load_2d_pair(sb + L::kOffW + st * L::kWBytes, &p.tm_w, kb * kProjBK, w0, full);
         }
       }
-      // No load may still be landing in shared memory when the CTA exits:
-      // wait for the last loads of every stage (abort ignored, time-bounded).
+      // Before the CTA exits, every stage's last use has been consumed by the
+      // MMA (so its loads landed) and its release arrived here (bounded).
       for (int j = 0; j < kProjStages && j < it; ++j) {
         const int i = it - 1 - j;
-        mbar_wait(sb + BAR_FULL + 8 * (i % kProjStages), (i / kProjStages) & 1, 0u, tmo, SITE_TAIL);
+        mbar_wait(sb + BAR_EMPTY + 8 * (i % kProjStages), (i / kProjStages) & 1, 0u, tmo, SITE_TAIL);
       }
     }
   } else if (warp == 1) {
     // ============================================================== MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       int it = 0, local = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x, ++local) {
+      for (int tile = cluster; ok && tile < n_tiles; tile += n_clusters, ++local) {
         const int a = local & 1;
         if (!mbar_wait_spin(sb + BAR_AE + 8 * a, ((local >> 1) & 1) ^ 1, abort_flag, tmo, SITE_MMA)) break;
         tc_fence_after();
@@ -212,13 +297,13 @@ __global__ void __launch_bounds__(kProjThreads, 1) proj_gemm_kernel(const __grid
           const uint64_t dw = smem_desc_sw128(sb + L::kOffW + st * L::kWBytes, 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < kProjBK / 16; ++kk)
-            mma_ss(d, da + ((kk * 32) >> 4), dw + ((kk * 32) >> 4), IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(sb + BAR_EMPTY + 8 * st);
+            proj_mma_pair(d, da + ((kk * 32) >> 4), dw + ((kk * 32) >> 4), IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+          proj_commit_pair_both(sb + BAR_EMPTY + 8 * st);
         }
-        if (ok) mma_commit(sb + BAR_AF + 8 * a);
+        if (ok) proj_commit_pair_both(sb + BAR_AF + 8 * a);
       }
       // Drain: every issued MMA has completed before TMEM is released.
-      mma_commit(sb + BAR_TAIL);
+      proj_commit_pair_self(sb + BAR_TAIL);
       mbar_wait(sb + BAR_TAIL, 0, 0u, tmo, SITE_TAIL);
     }
   } else {
@@ -227,8 +312,9 @@ __global__ void __launch_bounds__(kProjThreads, 1) proj_gemm_kernel(const __grid
     const int r = quarter * 32 + lane;   // accumulator row = TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const int HD = p.H * p.D;
+    const uint32_t ae_leader = proj_mapa(sb + BAR_AE, 0);
     int local = 0;
-    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++local) {
+    for (int tile = cluster; tile < n_tiles; tile += n_clusters, ++local) {
       const int a = local & 1;
       const bool w = mbar_wait(sb + BAR_AF + 8 * a, (local >> 1) & 1, abort_flag, tmo, SITE_EPILOGUE);
       if (__any_sync(0xffffffffu, !w)) break;
@@ -236,7 +322,7 @@ __global__ void __launch_bounds__(kProjThreads, 1) proj_gemm_kernel(const __grid
       tc_fence_after();
       int mi, ni;
       proj_tile(tile, mt, nt, mi, ni);
-      const int m = mi * kProjBM + r;
+      const int m = mi * 2 * kProjBM + static_cast<int>(rank) * kProjBM + r;
       const int n0 = ni * kProjBN;
       const bool row_ok = m < p.M;
       // Row-dependent part of the destination.
@@ -290,16 +376,19 @@ __global__ void __launch_bounds__(kProjThreads, 1) proj_gemm_kernel(const __grid
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(sb + BAR_AE + 8 * a);
+      if (lane == 0) proj_arrive_remote(ae_leader + 8 * a);
     }
   }
 
+  // Teardown: both CTAs finished every access to the pair's TMEM and to each
+  // other's shared memory before the paired TMEM is released.
   tc_fence_before();
   __syncthreads();
+  proj_cluster_sync();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, kProjTmemCols);
+    proj_tmem_dealloc_pair(tmem, kProjTmemCols);
   }
 }
 
