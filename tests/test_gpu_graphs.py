@@ -61,3 +61,41 @@ def test_captured_forward_and_backward_replay_equal_eager():
     st, code = api.cpattn_device_status()
     assert st == 0, f"device status {code:#x}"
     del graph
+
+
+def test_captured_projection_flow_replay_equals_eager():
+    """The fused projections launch in clusters of two CTAs (cudaLaunchKernelEx);
+    captured together with the head-sharded attention between them, a replay
+    on new activations gives the bytes eager calls give."""
+    B, S, H, D, U = 1, 512, 4, 128, 2
+    Dm = H * D
+    xb, wb, wob = inputs.make_projection_inputs(B, S, H, D, Dm, 71)
+    x, w, wo = to_dev(xb), to_dev(wb), to_dev(wob)
+    n = B * S * H * D
+    yq, yk, yv, yo = (torch.empty(n, dtype=torch.bfloat16, device="cuda") for _ in range(4))
+    out = torch.empty(B * S * Dm, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, H, S), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.Stream()
+
+    def step():
+        api.cpattn_ulysses_qkv_projection(x, w, B, S, H, D, Dm, U, yq=yq, yk=yk, yv=yv, stream=stream)
+        api.cpattn_head_sharded_attention(yq, yk, yv, B, S, H, D, U, yo=yo, lse=lse, stream=stream)
+        api.cpattn_ulysses_output_projection(yo, wo, B, S, H, D, Dm, U, out=out, stream=stream)
+
+    with torch.cuda.stream(stream):
+        step()                                   # warm-up outside capture (one-time attribute setup)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step()
+    x.copy_(to_dev(inputs.make_projection_inputs(B, S, H, D, Dm, 72)[0]))
+    graph.replay()
+    torch.cuda.synchronize()
+    got = [t.clone() for t in (yq, yo, out)]
+    with torch.cuda.stream(stream):
+        step()
+    torch.cuda.synchronize()
+    for g, want in zip(got, (yq, yo, out)):
+        assert torch.equal(g.view(torch.int16), want.view(torch.int16))
+    st, code = api.cpattn_device_status()
+    assert st == 0, f"device status {code:#x}"
