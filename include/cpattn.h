@@ -41,9 +41,10 @@
  *   validated before anything is enqueued; on a non-zero return nothing was
  *   enqueued except for CPATTN_ERR_CUDA, which reports a launch failure.
  *   The compute calls can be captured in a CUDA graph (after one eager call
- *   per kernel shape, which sets the kernels' shared-memory attribute):
- *   nothing on their launch path synchronises or allocates, and each launch
- *   carries its plan by value.  cpattn_device_status synchronises and is not
+ *   per kernel shape, which sets the kernels' shared-memory attribute and,
+ *   for the projections, sizes their two-CTA cluster grid): nothing on their
+ *   launch path synchronises or allocates, and each launch carries its plan
+ *   by value.  cpattn_device_status synchronises and is not
  *   capturable.
  * Errors.  Return value is a cpattn_status.  No C++ exception crosses the ABI.
  *   Device-side bounded waits (see cpattn_device_status) report a pipeline that
