@@ -680,7 +680,7 @@ const char *cpattn_status_string(int status) {
   }
 }
 
-int cpattn_version(void) { return 1 * 10000 + 1 * 100 + 0; }
+int cpattn_version(void) { return 1 * 10000 + 2 * 100 + 0; }
 
 int cpattn_front_loaded_splits(int total, int parts, int *out) {
   if (out == nullptr) return CPATTN_ERR_NULL;
