@@ -613,6 +613,12 @@ static int projection_common(const void *a, const void *w, int B, int S, int H, 
   if (Dm < kProjBK || Dm % kProjBK != 0 || Dm > (1 << 20)) return CPATTN_ERR_SHAPE;
   if (H > kMaxHeads || static_cast<long long>(B) * S > INT_MAX / 2) return CPATTN_ERR_SHAPE;
   if (3ll * H * D > INT_MAX / 2) return CPATTN_ERR_SHAPE;
+  {
+    // the kernel numbers its 256 x 256 tiles with int
+    const long long rows = static_cast<long long>(B) * S, cols = out_mode ? Dm : 3ll * H * D;
+    if (((rows + 2 * kProjBM - 1) / (2 * kProjBM)) * ((cols + kProjBN - 1) / kProjBN) > INT_MAX)
+      return CPATTN_ERR_SHAPE;
+  }
   if (degree < 1 || degree > kMaxRanks) return CPATTN_ERR_DEGREE;
   std::vector<int> seq, heads;
   int st = resolve_splits(S, degree, seq_splits, seq);

@@ -138,6 +138,7 @@ def test_projection_validation(lib):
     assert q(Dm=0) == SHAPE
     assert q(B=0) == SHAPE
     assert q(H=2000) == SHAPE
+    assert q(S=1 << 29, H=1024, D=128) == SHAPE   # within every other bound, but more 256 x 256 tiles than an int numbers
     assert q(P=0) == DEGREE
     assert q(P=65) == DEGREE
     assert q(H=5) == INDIV
