@@ -80,16 +80,6 @@ struct alignas(64) ProjParams {
   unsigned long long timeout_ns;
 };
 
-// 2-D tiled bulk tensor load global -> shared (no multicast).
-__device__ __forceinline__ void proj_tma_load_2d(uint32_t smem_dst, const CUtensorMap *tm, int c0, int c1,
-                                                 uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_dst),
-      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(bar)
-      : "memory");
-}
-
 // ------------------------------------------------ CTA-pair (cta_group::2) forms
 __device__ __forceinline__ uint32_t proj_cluster_rank() {
   uint32_t r;
