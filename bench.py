@@ -582,6 +582,13 @@ def backward_paths(api, torch, flush, peaks, q, k, v, P):
     return res
 
 
+def projection_flops(B, S, H, D, Dm):
+    """2*K FLOPs per output element (one multiply and one add per term):
+    the Q/K/V projection (B*S x 3*H*D outputs, K = Dm) and the output
+    projection (B*S x Dm outputs, K = H*D)."""
+    return 2.0 * B * S * Dm * 3 * H * D, 2.0 * B * S * H * D * Dm
+
+
 def projection_paths(api, torch, flush, peaks, inputs, B, S, H, D, U):
     """The Ulysses projections with the all-to-all fused in, on the bench
     workload's sizes (model width H*D), each rep after an L2 flush: the Q/K/V
@@ -598,8 +605,7 @@ def projection_paths(api, torch, flush, peaks, inputs, B, S, H, D, U):
     yq, yk, yv, yo = (torch.empty(n, dtype=torch.bfloat16, device=dev) for _ in range(4))
     out = torch.empty(B * S * Dm, dtype=torch.bfloat16, device=dev)
     peak_tf = float(peaks["bf16_tflops"])
-    f_qkv = 2.0 * B * S * Dm * 3 * H * D
-    f_out = 2.0 * B * S * H * D * Dm
+    f_qkv, f_out = projection_flops(B, S, H, D, Dm)
     res = {}
 
     def rec(name, fn, flops, note):

@@ -1,0 +1,32 @@
+"""The work counts behind bench.py's throughputs and roofline, checked on the
+CPU against brute-force counts: causal attention counts 4*D FLOPs for every
+visible (query, key) pair, the backward 2.5x the forward, and the projections
+2*K FLOPs per output element (a multiply and an add per term)."""
+import pytest
+
+import bench
+
+
+@pytest.mark.parametrize("B,H,S,D", [(1, 1, 1, 64), (2, 3, 7, 128), (1, 2, 130, 64)])
+def test_causal_flops_count_visible_pairs(B, H, S, D):
+    visible = sum(1 for i in range(S) for j in range(S) if j <= i)
+    assert bench.causal_flops(B, H, S, D) == 4.0 * D * B * H * visible
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_flops_are_five_matmuls_of_the_forward_two(causal):
+    B, H, S, D = 2, 3, 9, 64
+    fwd = bench.causal_flops(B, H, S, D) if causal else 4.0 * B * H * S * S * D
+    assert bench.backward_flops(B, H, S, D, causal) == pytest.approx(fwd * 5 / 2)
+
+
+def test_projection_flops_match_counted_multiply_adds():
+    B, S, H, D, Dm = 2, 3, 2, 4, 5
+    count_qkv = sum(1 for _row in range(B * S) for _col in range(3 * H * D) for _k in range(Dm))
+    count_out = sum(1 for _row in range(B * S) for _col in range(Dm) for _k in range(H * D))
+    assert bench.projection_flops(B, S, H, D, Dm) == (2.0 * count_qkv, 2.0 * count_out)
+
+
+def test_aggregate_over_ranks_single_rank():
+    ms_per_step, per_s = bench.aggregate_over_ranks(10.0, 5, 1e12, 1)
+    assert ms_per_step == 2.0 and per_s == pytest.approx(5e12 / 10e-3)
