@@ -78,10 +78,6 @@ constexpr int kRegsControl = 104;
 constexpr int kRegsSoftmax = 200;
 static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= kAttnThreads * kRegsLaunch, "register split exceeds launch");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale only if the max grows by > 2^8
-// Of every 8 score pairs, this many take 2^x on the FMA pipe (exp2_poly_x2)
-// and the rest on the SFU.  Measured on B200 with this pipeline the SFU is not
-// the limiter (the FMA-pipe share only lengthened the softmax), so it is 0.
-constexpr int kPolyEighths = 0;
 
 // The work unit of this CTA: group -> head -> segment -> pair of Q tiles (or a
 // split lone tile).  Recomputed inside every role (after its register budget
@@ -534,9 +530,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
               }
             }
           }
-          // P = 2^(S*c - m), pairs of scores through packed f32x2 FMAs, a
-          // fixed share of the exponentials on the FMA pipe, the rest on the
-          // SFU.  P is published in two halves (keys 0-63, 64-127) so that
+          // P = 2^(S*c - m), pairs of scores through packed f32x2 FMAs and
+          // the exponentials on the SFU.  P is published in two halves (keys 0-63, 64-127) so that
           // the MMA warp starts PV on the first half while the second half
           // is computed.
           const uint64_t cc = f2_pack(c, c);
@@ -551,14 +546,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
               const uint64_t x = f2_fma(f2_pack(__uint_as_float(s[c0 + 2 * k]), __uint_as_float(s[c0 + 2 * k + 1])), cc, mm);
-              uint64_t pp;
-              if ((k & 7) < kPolyEighths) {
-                pp = exp2_poly_x2(x);
-              } else {
-                float x0, x1;
-                f2_unpack(x, x0, x1);
-                pp = f2_pack(ex2_approx(x0), ex2_approx(x1));
-              }
+              float x0, x1;
+              f2_unpack(x, x0, x1);
+              const uint64_t pp = f2_pack(ex2_approx(x0), ex2_approx(x1));
               if (k & 1) lsum1 = f2_add(lsum1, pp); else lsum0 = f2_add(lsum0, pp);
               float p0, p1;
               f2_unpack(pp, p0, p1);

@@ -166,43 +166,6 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
-__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-
-// 2^x for a pair, on the FMA pipe instead of the SFU (x <= 2^7).  Written
-// from the textbook range reduction 2^x = 2^j * 2^f, j = round(x),
-// f = x - j in [-0.5, 0.5]:
-//   * x is clamped at -125 so that 2^j stays a normal number (2^-125 ~ 0);
-//   * adding 1.5 * 2^23 rounds x to the integer j (round to nearest) and
-//     leaves j in the low mantissa bits of t; subtracting it back gives j;
-//   * 2^f is a degree-3 polynomial whose coefficients were fitted here by a
-//     Remez exchange for minimal relative error on [-0.5, 0.5] (max relative
-//     error 7.5e-5, below the 2^-9 rounding of P to bf16);
-//   * 2^j is applied by adding j to the exponent field: the low bits of t
-//     shifted left by 23 (the high bits of t shift out of the word).
-__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x) {
-  const float kRound = 12582912.0f;     // 1.5 * 2^23
-  const float kC3 = 0.05517166853f;
-  const float kC2 = 0.24261112511f;
-  const float kC1 = 0.69326096773f;
-  const float kC0 = 0.99992805719f;
-  float x0, x1;
-  f2_unpack(x, x0, x1);
-  x = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
-  const uint64_t rr = f2_pack(kRound, kRound);
-  const uint64_t t = f2_add(x, rr);
-  const uint64_t f = f2_sub(x, f2_sub(t, rr));
-  uint64_t q = f2_fma(f, f2_pack(kC3, kC3), f2_pack(kC2, kC2));
-  q = f2_fma(q, f, f2_pack(kC1, kC1));
-  q = f2_fma(q, f, f2_pack(kC0, kC0));
-  const uint32_t lo = static_cast<uint32_t>(q) + (static_cast<uint32_t>(t) << 23);
-  const uint32_t hi = static_cast<uint32_t>(q >> 32) + (static_cast<uint32_t>(t >> 32) << 23);
-  return (static_cast<uint64_t>(hi) << 32) | lo;
-}
-
 // Keeps a value in a register without letting the compiler hoist or
 // rematerialise expressions built from it across loop iterations.
 __device__ __forceinline__ uint64_t opaque_u64(uint64_t v) {
