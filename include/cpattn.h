@@ -31,6 +31,10 @@
  *   divisibility by the degree ([CP] variants table); explicit lengths are the
  *   'anything' modes ([CP] Ring Anything / Ulysses Anything), may be uneven and
  *   may contain zeros.
+ * Contexts.  The library keeps per-device state for the life of the process
+ *   (kernel attributes set on first use, cluster sizes, the no-allocation
+ *   scratch address): use it under each device's primary context, the one the
+ *   CUDA runtime uses, and not across a cudaDeviceReset.
  * Memory.  All tensor pointers are DEVICE pointers owned by the caller; the
  *   library allocates no device memory on any call (workspaces come from the
  *   caller; cpattn_ulysses_attention_noalloc uses a static scratch).  Length/split arrays are HOST arrays read only
@@ -431,9 +435,20 @@ int cpattn_ulysses_attention_backward(const void *q, const void *k, const void *
  * that (8 * B*S*H*D bytes) is rejected with CPATTN_ERR_WORKSPACE before any
  * work is enqueued.
  *
+ * When the memory is committed: CUDA loads the library's device code, and with
+ * it this array, on a device the first time any entry point of the library
+ * launches work or looks up the array there (under the default lazy module
+ * loading) -- not when the shared library is loaded into the process.  A
+ * caller that reserves all free GPU memory at start-up must therefore make one
+ * call on each device first (for example this entry point on a small shape),
+ * or that later first call fails with CPATTN_ERR_CUDA.
+ *
  * The first call on a device, with that device current, looks up the array's
- * device address (cudaGetSymbolAddress); make that first call on each device
- * before any stream capture.  Every call uses the same array, which keeps the
+ * device address (cudaGetSymbolAddress) and keeps it for the life of the
+ * process; make that first call on each device before any stream capture.
+ * The kept address belongs to the device's primary context (the one the CUDA
+ * runtime uses): do not call this entry point across a cudaDeviceReset or
+ * with another context current.  Every call uses the same array, which keeps the
  * previous call's contents (nothing in it needs to start at zero): calls that
  * overlap on the GPU -- on different streams, or from different host threads
  * without ordering -- race on the array and corrupt each other's results, so

@@ -177,6 +177,28 @@ def test_flow_validation(lib):
     assert h(H=5) == INDIV
 
 
+def test_noalloc_validation(lib):
+    # Every case returns before the library touches CUDA (the scratch-size
+    # check comes before the device check), so these run without a GPU.
+    def f(q=FAKE, out=FAKE, B=1, S=8, H=4, D=64, P=2, seq=None, heads=None):
+        return lib.cpattn_ulysses_attention_noalloc(q, FAKE, FAKE, out, FAKE, B, H, S, D, P, _native.int_array(seq),
+                                                    _native.int_array(heads), None)
+    assert f(q=None) == NULL
+    assert f(out=None) == NULL
+    assert f(D=96) == SHAPE
+    assert f(P=0) == DEGREE
+    assert f(P=65) == DEGREE
+    assert f(H=5) == INDIV
+    assert f(S=9) == INDIV
+    assert f(S=9, seq=[5, 5]) == SPLITS
+    assert f(H=5, heads=[3, 3]) == SPLITS
+    assert f(seq=[9, -1]) == SPLITS
+    # 8 * B*S*H*D bytes of scratch against the 64 MiB array: 1 x 8192 x 8 x 128
+    # fills it exactly, one more token does not fit.
+    assert f(S=8193, H=8, D=128, P=1) == WS
+    assert f(B=2, S=4097, H=8, D=128, P=1) == WS
+
+
 def test_debug_hook_validation(lib):
     assert lib.cpattn_debug_wait_timeout(0, None) == SHAPE
     assert lib.cpattn_device_status(None, None) == NULL

@@ -341,6 +341,88 @@ def test_constant_v_and_zero_k_closed_forms():
     _no_timeouts()
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_one_hot_key_selects_its_value(D):
+    """One-hot selection closed form: K = 0 except key j* = b e_0 and every query
+    q_i = a e_0 (a, b exact in bf16), so each row has one logit s* = a b D**-0.5
+    and S - 1 logits 0: out_i = v_j* up to e^-s* (S - 1), far below bf16's
+    resolution, and LSE_i = ln(e^s* + S - 1).  Pinned for the ring (uneven
+    chunks, j* in the middle chunk), kv_gather and the Ulysses flow."""
+    B, S, H = 1, 333, 3
+    a, b = 32.0, (25.0 if D == 64 else 36.0)      # D = 64: s* = 32 * 25 / 8 = 100 exactly
+    s_star = a * b / np.sqrt(D)
+    j_star = 170
+    q = torch.zeros((B, S, H, D), dtype=torch.bfloat16, device="cuda")
+    q[..., 0] = a
+    k = torch.zeros_like(q)
+    k[:, j_star, :, 0] = b
+    _, _, (_, _, v) = _qkv(B, S, H, D, 77, rms=False)
+    want_o = v[:, j_star:j_star + 1].expand(B, S, H, D)
+    want_l = s_star + np.log1p((S - 1) * np.exp(-s_star))
+    lens = [100, 133, 100]
+    ws = torch.empty(api.cpattn_ulysses_workspace_bytes(B, H, S, D), dtype=torch.uint8, device="cuda")
+    results = {
+        "ring": api.cpattn_ring_attention(q, k, v, 3, lens),
+        "kv_gather": api.cpattn_kv_gather_attention(q, k, v, 3, lens),
+        "ulysses": api.cpattn_ulysses_attention(q.reshape(-1), k.reshape(-1), v.reshape(-1), B, S, H, D, 3,
+                                                lens, [1, 1, 1], workspace=ws),
+    }
+    torch.cuda.synchronize()
+    _no_timeouts()
+    for name, (o, l) in results.items():
+        o = o.view(B, S, H, D)
+        assert torch.equal(o.view(torch.int16), want_o.contiguous().view(torch.int16)), f"{name}: not v_j*"
+        assert np.max(np.abs(f64_of(l) - want_l)) <= 1e-3, f"{name}: LSE {f64_of(l).ravel()[:3]} vs {want_l}"
+
+
+def test_lse_merge_dit_size_p4_full():
+    """The merge of the ring-step partials of the image-DiT workload (P = 4),
+    every row, against the oracle's merge of the same float32 partials."""
+    cfg, qb, kb, vb = inputs.config_inputs("dit")
+    B, S, H, D = qb.shape
+    P = cfg["ring_degree"]
+    dq, dk, dv = (to_dev(x) for x in (qb, kb, vb))
+    po = torch.empty((P, B, S, H, D), dtype=torch.float32, device="cuda")
+    pl = torch.empty((P, B, H, S), dtype=torch.float32, device="cuda")
+    for t in range(P):
+        api.cpattn_ring_step(dq, dk, dv, P, t, part_out=po[t], part_lse=pl[t])
+    f32, b16, lse = api.cpattn_lse_merge(po, pl, want_f32=True)
+    torch.cuda.synchronize()
+    _no_timeouts()
+    ref_o, ref_l = oracle.lse_merge(list(f64_of(po)), list(f64_of(pl)))
+    assert np.max(np.abs(f64_of(f32) - ref_o)) < 1e-5
+    assert np.max(np.abs(f64_of(lse) - ref_l)) < 1e-5
+    assert np.max(np.abs(f64_of(b16) - ref_o)) <= 2.0 ** -8 * np.max(np.abs(ref_o)) + 1e-6
+
+
+def test_lse_merge_video_size_p8_sampled():
+    """The 8-way merge at the video workload's size (B1 S32760 H40 D128, the
+    partials the bench times: 5.4 GB of float32), on sampled rows: the merge
+    is independent per (b, h, s) row, so rows can be checked one by one."""
+    B, S, H, D, P = 1, 32760, 40, 128, 8
+    gen = torch.Generator(device="cuda").manual_seed(11)
+    po = torch.randn((P, B, S, H, D), generator=gen, device="cuda", dtype=torch.float32)
+    pl = torch.randn((P, B, H, S), generator=gen, device="cuda", dtype=torch.float32) * 4
+    pl[1, :, :, ::7] = float("-inf")                 # empty partials
+    pl[:, :, 3, 5] = float("-inf")                   # a row with no keys at all
+    b16 = torch.empty((B, S, H, D), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, H, S), dtype=torch.float32, device="cuda")
+    api.cpattn_lse_merge(po, pl, out_bf16=b16, lse_out=lse, want_f32=False)
+    torch.cuda.synchronize()
+    _no_timeouts()
+    pos = np.unique(np.concatenate([[0, 5, 7, S - 1], sample_positions(S, [0, S], 60, 12)]))
+    pt = torch.from_numpy(pos).cuda()
+    ref_o, ref_l = oracle.lse_merge(list(f64_of(po[:, :, pt])), list(f64_of(pl[:, :, :, pt])))
+    got_l = f64_of(lse[:, :, pt])
+    fin = np.isfinite(ref_l)
+    assert np.array_equal(fin, np.isfinite(got_l))
+    assert np.max(np.abs(got_l[fin] - ref_l[fin])) < 1e-5
+    assert np.max(np.abs(f64_of(b16[:, pt]) - ref_o)) <= 2.0 ** -8 * np.max(np.abs(ref_o)) + 1e-6
+    assert np.all(f64_of(b16[:, 5, 3]) == 0)
+    del po, pl
+    torch.cuda.empty_cache()
+
+
 def test_bounded_wait_reports_timeout_and_context_survives():
     api.cpattn_debug_wait_timeout(2000)
     st, code = api.cpattn_device_status()
