@@ -67,6 +67,13 @@ SIGNATURES = {
                                                   P_INT, P_INT, c_int, c_void_p, c_size_t, c_void_p]),
     "cpattn_ulysses_attention_noalloc": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                                  c_int, c_int, c_int, c_int, c_int, P_INT, P_INT, c_void_p]),
+    "cpattn_ring_chunk_attention": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                            c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
+                                            c_void_p]),
+    "cpattn_gathered_kv_attention": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                             c_int, c_int, c_int, c_int, P_INT, c_int, c_int, c_int, c_void_p]),
+    "cpattn_rank_buffer_attention": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                             c_int, c_int, c_int, c_int, c_int, P_INT, c_int, c_void_p]),
     "cpattn_front_loaded_splits": (c_int, [c_int, c_int, P_INT]),
     "cpattn_exchange_bytes": (c_int, [c_int, c_int, c_int, c_int, c_int, c_int, c_int, P_INT, P_INT,
                                       ctypes.POINTER(ctypes.c_ulonglong), ctypes.POINTER(ctypes.c_ulonglong)]),

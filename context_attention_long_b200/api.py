@@ -27,7 +27,8 @@ __all__ = [
     "cpattn_unified_attention", "cpattn_causal_unified_attention",
     "cpattn_attention_backward_workspace_bytes", "cpattn_attention_backward",
     "cpattn_ulysses_attention_backward_workspace_bytes", "cpattn_ulysses_attention_backward",
-    "cpattn_ulysses_attention_noalloc", "cpattn_front_loaded_splits", "cpattn_exchange_bytes",
+    "cpattn_ulysses_attention_noalloc", "cpattn_ring_chunk_attention", "cpattn_gathered_kv_attention",
+    "cpattn_rank_buffer_attention", "cpattn_front_loaded_splits", "cpattn_exchange_bytes",
     "cpattn_plan_exchange", "cpattn_device_status", "cpattn_debug_wait_timeout", "NOALLOC_SCRATCH_BYTES",
     "status_string",
 ]
@@ -433,6 +434,72 @@ def cpattn_ulysses_attention_noalloc(q, k, v, B, S, H, D, degree, seq_splits=Non
                                                            D, int(degree), _native.int_array(seq_splits),
                                                            _native.int_array(head_splits), _stream(stream)),
            "cpattn_ulysses_attention_noalloc")
+    return out, lse
+
+
+def cpattn_ring_chunk_attention(q, k, v, Skv, out, lse, prev_out=None, q_pos0=0, kv_pos0=0, causal=False,
+                                kv_batch_rows=None, stream=None):
+    """One ring step of one rank over separate buffers, merged into its running
+    result.  q (B, Sq, H, D) bf16; k, v (B, kv_batch_rows, H, D) bf16 whose
+    first Skv rows per batch element are the chunk; out float32 (an
+    intermediate state) or bf16 (the final output), (B, Sq, H, D); lse
+    (B, H, Sq) float32, holding prev_out's LSE on entry when prev_out (float32,
+    may be `out` itself) is given.  Returns (out, lse)."""
+    B, Sq, H, D = _bshd(q)
+    rows = k.shape[1] if kv_batch_rows is None else int(kv_batch_rows)
+    for t, name in ((k, "k"), (v, "v")):
+        _need(t, B * rows * H * D, torch.bfloat16, name)
+    if out.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("out must be float32 or bf16")
+    _need(out, B * Sq * H * D, out.dtype, "out")
+    _need(lse, B * H * Sq, torch.float32, "lse")
+    _need(prev_out, B * Sq * H * D, torch.float32, "prev_out")
+    _check(_native.load().cpattn_ring_chunk_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                                                      _ptr(prev_out), B, H, Sq, int(Skv), rows, D, int(q_pos0),
+                                                      int(kv_pos0), int(bool(causal)),
+                                                      int(out.dtype == torch.float32), _stream(stream)),
+           "cpattn_ring_chunk_attention")
+    return out, lse
+
+
+def cpattn_gathered_kv_attention(q, k, v, degree, rank, kv_lens=None, out=None, lse=None, want_lse=True,
+                                 causal=False, stream=None):
+    """Attention of one rank's query shard q (B, kv_lens[rank], H, D) against
+    `degree` gathered K/V chunks, k and v (degree, B, kv_batch_rows, H, D)
+    bf16, chunk c holding kv_lens[c] valid rows.  Returns (out, lse)."""
+    B, Sq, H, D = _bshd(q)
+    if k.dim() != 5 or k.shape[0] != degree or k.shape[1] != B:
+        raise ValueError("k and v must be (degree, B, kv_batch_rows, H, D)")
+    rows = k.shape[2]
+    for t, name in ((k, "k"), (v, "v")):
+        _need(t, degree * B * rows * H * D, torch.bfloat16, name)
+    out = torch.empty_like(q) if out is None else out
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
+    _need(out, B * Sq * H * D, torch.bfloat16, "out")
+    _need(lse, B * H * Sq, torch.float32, "lse")
+    _check(_native.load().cpattn_gathered_kv_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, D,
+                                                       int(degree), _native.int_array(kv_lens), rows, int(rank),
+                                                       int(bool(causal)), _stream(stream)),
+           "cpattn_gathered_kv_attention")
+    return out, lse
+
+
+def cpattn_rank_buffer_attention(q, k, v, B, S, H, D, degree, seq_splits=None, out=None, lse=None, want_lse=True,
+                                 causal=False, stream=None):
+    """Attention over a sequence held as rank buffers (B, S_u, H, D)
+    concatenated (flat bf16), the layout an all-to-all delivers; every query
+    attends all S keys.  Returns (out in the same layout, lse (B, H, S))."""
+    out = torch.empty_like(q) if out is None else out
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    for t, name in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
+        _need(t, _flat_numel(B, S, H, D), torch.bfloat16, name)
+    _need(lse, B * H * S, torch.float32, "lse")
+    _check(_native.load().cpattn_rank_buffer_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, S, D,
+                                                       int(degree), _native.int_array(seq_splits),
+                                                       int(bool(causal)), _stream(stream)),
+           "cpattn_rank_buffer_attention")
     return out, lse
 
 

@@ -604,10 +604,32 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
           const float mm = fmaxf(m, m1);
           const float a0 = ex2_approx(m - mm), a1 = ex2_approx(m1 - mm);
           const float lt = l * a0 + l1 * a1;
-          const float w0 = a0 / lt, w1 = a1 / lt;
           const bool row_valid = row < rows_left;
           const int grow = q_row0 + row;
           const size_t row_elems = (static_cast<size_t>(grow) * PB.H + h) * D;
+          const int sq = SG.s0 + pair * (kQTilesPerCTA * kQTile) + row;
+          const long long lse_idx = static_cast<long long>(G.b) * PB.lse_b +
+                                    static_cast<long long>(h + PB.lse_h0) * PB.lse_h + (sq - PB.lse_pos0);
+          // This unit's own state (slots 0 and 1 merged), in log2 units, and
+          // its merge with a previous partial state when the plan carries one.
+          float own = lt > 0.0f ? mm + log2f(lt) : -INFINITY;
+          float w0 = lt > 0.0f ? a0 / lt : 0.0f, w1 = lt > 0.0f ? a1 / lt : 0.0f, wp = 0.0f;
+          const float *prev_row = nullptr;
+          if (PB.prev != nullptr && row_valid) {
+            const float lp = PB.lse[lse_idx] * 1.4426950408889634f;
+            const float M = fmaxf(own, lp);
+            if (M == -INFINITY) {
+              w0 = w1 = 0.0f;
+            } else {
+              const float as = ex2_approx(own - M), ap = ex2_approx(lp - M);
+              const float tot = as + ap;
+              w0 *= as / tot;
+              w1 *= as / tot;
+              wp = ap / tot;
+              own = M + log2f(tot);
+              if (wp != 0.0f) prev_row = PB.prev + row_elems;
+            }
+          }
 #pragma unroll
           for (int c0 = 0; c0 < D; c0 += 32) {
             uint32_t o0[32], o1[32];
@@ -616,6 +638,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
             float v[32];
 #pragma unroll
             for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(o0[k]) * w0 + __uint_as_float(o1[k]) * w1;
+            if (prev_row != nullptr) {
+              const float4 *src = reinterpret_cast<const float4 *>(prev_row + c0);
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                const float4 pv = src[k];
+                v[4 * k] += pv.x * wp;
+                v[4 * k + 1] += pv.y * wp;
+                v[4 * k + 2] += pv.z * wp;
+                v[4 * k + 3] += pv.w * wp;
+              }
+            }
             if (row_valid) {
               if constexpr (OUT_F32) {
                 float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(PB.out) + row_elems + c0);
@@ -630,19 +663,37 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
               }
             }
           }
-          if (row_valid && PB.lse != nullptr) {
-            const int sq = SG.s0 + pair * (kQTilesPerCTA * kQTile) + row;
-            PB.lse[static_cast<long long>(G.b) * PB.lse_b + static_cast<long long>(h + PB.lse_h0) * PB.lse_h + sq] =
-                (mm + log2f(lt)) * 0.69314718055994531f;
-          }
+          if (row_valid && PB.lse != nullptr) PB.lse[lse_idx] = own * 0.69314718055994531f;
         }
       }
     } else if (active && ok) {
       const int valid_rows = qt == 0 ? min(kQTile, rows_left) : rows_left - kQTile;
       const bool row_valid = row < valid_rows;
       const int grow = q_row0 + qt * kQTile + row;
-      const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
       const size_t row_elems = (static_cast<size_t>(grow) * PB.H + h) * D;
+      const int sq = SG.s0 + pair * (kQTilesPerCTA * kQTile) + qt * kQTile + row;
+      const long long lse_idx = static_cast<long long>(G.b) * PB.lse_b +
+                                static_cast<long long>(h + PB.lse_h0) * PB.lse_h + (sq - PB.lse_pos0);
+      // out = O * w_self + prev * w_prev: w_self = 1/l alone; with a previous
+      // partial state (LSE read before it is overwritten) both are the LSE-rule
+      // weights of the two states.
+      float own = (n_tiles > 0 && l > 0.0f) ? m + log2f(l) : -INFINITY;   // log2 units
+      float w_self = l > 0.0f ? 1.0f / l : 0.0f, wp = 0.0f;
+      const float *prev_row = nullptr;
+      if (PB.prev != nullptr && row_valid) {
+        const float lp = PB.lse[lse_idx] * 1.4426950408889634f;
+        const float M = fmaxf(own, lp);
+        if (M == -INFINITY) {
+          w_self = 0.0f;
+        } else {
+          const float as = ex2_approx(own - M), ap = ex2_approx(lp - M);
+          const float tot = as + ap;
+          w_self *= as / tot;
+          wp = ap / tot;
+          own = M + log2f(tot);
+          if (wp != 0.0f) prev_row = PB.prev + row_elems;
+        }
+      }
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t o[32];
@@ -652,29 +703,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
 #pragma unroll
           for (int k = 0; k < 32; ++k) o[k] = 0u;
         }
+        float v[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(o[k]) * w_self;
+        if (prev_row != nullptr) {
+          const float4 *src = reinterpret_cast<const float4 *>(prev_row + c0);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const float4 pv = src[k];
+            v[4 * k] += pv.x * wp;
+            v[4 * k + 1] += pv.y * wp;
+            v[4 * k + 2] += pv.z * wp;
+            v[4 * k + 3] += pv.w * wp;
+          }
+        }
         if (row_valid) {
           if constexpr (OUT_F32) {
             float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(PB.out) + row_elems + c0);
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-              dst[k] = make_float4(__uint_as_float(o[4 * k]) * inv_l, __uint_as_float(o[4 * k + 1]) * inv_l,
-                                   __uint_as_float(o[4 * k + 2]) * inv_l, __uint_as_float(o[4 * k + 3]) * inv_l);
+            for (int k = 0; k < 8; ++k) dst[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
           } else {
             uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(PB.out) + row_elems + c0);
 #pragma unroll
             for (int k = 0; k < 4; ++k)
-              dst[k] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * k]) * inv_l, __uint_as_float(o[8 * k + 1]) * inv_l),
-                                  pack_bf16x2(__uint_as_float(o[8 * k + 2]) * inv_l, __uint_as_float(o[8 * k + 3]) * inv_l),
-                                  pack_bf16x2(__uint_as_float(o[8 * k + 4]) * inv_l, __uint_as_float(o[8 * k + 5]) * inv_l),
-                                  pack_bf16x2(__uint_as_float(o[8 * k + 6]) * inv_l, __uint_as_float(o[8 * k + 7]) * inv_l));
+              dst[k] = make_uint4(pack_bf16x2(v[8 * k], v[8 * k + 1]), pack_bf16x2(v[8 * k + 2], v[8 * k + 3]),
+                                  pack_bf16x2(v[8 * k + 4], v[8 * k + 5]), pack_bf16x2(v[8 * k + 6], v[8 * k + 7]));
           }
         }
       }
-      if (row_valid && PB.lse != nullptr) {
-        const float lse = n_tiles > 0 ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
-        const int s = SG.s0 + pair * (kQTilesPerCTA * kQTile) + qt * kQTile + row;
-        PB.lse[static_cast<long long>(G.b) * PB.lse_b + static_cast<long long>(h + PB.lse_h0) * PB.lse_h + s] = lse;
-      }
+      if (row_valid && PB.lse != nullptr) PB.lse[lse_idx] = own * 0.69314718055994531f;
     }
   }
 

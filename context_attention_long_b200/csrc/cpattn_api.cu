@@ -332,7 +332,10 @@ struct ProblemSpec {
   long long lse_b, lse_h;
   int lse_h0;
   int H;
-  long long rows;
+  long long rows;              // rows of Q and out (and of K and V unless rows_kv > 0)
+  long long rows_kv = 0;       // rows of K and V when they are a separate buffer
+  const float *prev = nullptr; // previous partial state merged into the output (see AttnProblem)
+  int lse_pos0 = 0;            // sequence position of LSE column 0
 };
 struct SegSpec {
   int row0, nrows, s0;
@@ -409,14 +412,17 @@ static int run_attention(const std::vector<ProblemSpec> &probs, const std::vecto
     const ProblemSpec &ps = probs[i];
     AttnProblem &ap = encoded[i];
     std::memset(&ap, 0, sizeof(ap));
-    if (!encode_rows_map(&ap.tm_q, ps.q, D, ps.H, ps.rows) || !encode_rows_map(&ap.tm_k, ps.k, D, ps.H, ps.rows) ||
-        !encode_rows_map(&ap.tm_v, ps.v, D, ps.H, ps.rows))
+    const long long rows_kv = ps.rows_kv > 0 ? ps.rows_kv : ps.rows;
+    if (!encode_rows_map(&ap.tm_q, ps.q, D, ps.H, ps.rows) || !encode_rows_map(&ap.tm_k, ps.k, D, ps.H, rows_kv) ||
+        !encode_rows_map(&ap.tm_v, ps.v, D, ps.H, rows_kv))
       return CPATTN_ERR_CUDA;
     ap.out = ps.out;
     ap.lse = ps.lse;
+    ap.prev = ps.prev;
     ap.lse_b = ps.lse_b;
     ap.lse_h = ps.lse_h;
     ap.lse_h0 = ps.lse_h0;
+    ap.lse_pos0 = ps.lse_pos0;
     ap.H = ps.H;
   }
   const float scale_log2 = static_cast<float>((1.0 / std::sqrt(static_cast<double>(D))) * 1.4426950408889634);
@@ -1086,6 +1092,119 @@ int cpattn_causal_unified_attention(const void *q, const void *k, const void *v,
                                     cpattn_stream_t stream) {
   return unified_common(q, k, v, out, lse, B, H, S, D, ring_degree, ulysses_degree, ring_lens, head_splits, workspace,
                         workspace_bytes, true, stream);
+}
+
+// ------------------------------------------- building blocks of the exchanges
+
+int cpattn_ring_chunk_attention(const void *q, const void *k, const void *v, void *out, float *lse,
+                                const float *prev_out, int B, int H, int Sq, int Skv, int kv_batch_rows, int D,
+                                int q_pos0, int kv_pos0, int causal, int out_f32, cpattn_stream_t stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || lse == nullptr) return CPATTN_ERR_NULL;
+  int st = check_attn_shape(B, H, Sq, D);
+  if (st != CPATTN_OK) return st;
+  if (Skv < 0 || kv_batch_rows < 1 || kv_batch_rows < Skv || q_pos0 < 0 || kv_pos0 < 0) return CPATTN_ERR_SHAPE;
+  if (static_cast<long long>(B) * kv_batch_rows > INT_MAX ||
+      static_cast<long long>(B) * kv_batch_rows * H * D > (1ll << 46) ||
+      static_cast<long long>(q_pos0) + Sq > INT_MAX || static_cast<long long>(kv_pos0) + Skv > INT_MAX)
+    return CPATTN_ERR_SHAPE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned4(lse) ||
+      (prev_out && !aligned16(prev_out)))
+    return CPATTN_ERR_ALIGNMENT;
+  st = check_device(nullptr);
+  if (st != CPATTN_OK) return st;
+  ProblemSpec ps = full_problem(q, k, v, out, lse, B, H, Sq);
+  ps.rows_kv = static_cast<long long>(B) * kv_batch_rows;
+  ps.prev = prev_out;
+  ps.lse_pos0 = q_pos0;
+  std::vector<GroupSpec> groups;
+  for (int b = 0; b < B; ++b) {
+    GroupSpec g;
+    g.prob = 0;
+    g.b = b;
+    SegSpec sg;
+    sg.row0 = b * Sq;
+    sg.nrows = Sq;
+    sg.s0 = q_pos0;
+    if (Skv > 0) sg.kv.push_back(AttnKV{b * kv_batch_rows, Skv, kv_pos0});
+    g.segs.push_back(std::move(sg));
+    groups.push_back(std::move(g));
+  }
+  return run_attention({ps}, groups, D, out_f32 != 0, causal != 0, stream);
+}
+
+int cpattn_gathered_kv_attention(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H,
+                                 int D, int degree, const int *kv_lens, int kv_batch_rows, int rank, int causal,
+                                 cpattn_stream_t stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return CPATTN_ERR_NULL;
+  if (degree < 1 || degree > kMaxRingDegree || rank < 0 || rank >= degree) return CPATTN_ERR_DEGREE;
+  if (B < 1 || H < 1 || kv_batch_rows < 1) return CPATTN_ERR_SHAPE;
+  std::vector<int> lens(degree, kv_batch_rows);
+  if (kv_lens != nullptr)
+    for (int c = 0; c < degree; ++c) {
+      if (kv_lens[c] < 0 || kv_lens[c] > kv_batch_rows) return CPATTN_ERR_SPLITS;
+      lens[c] = kv_lens[c];
+    }
+  const int Sq = lens[rank];
+  long long total = 0;
+  for (int c = 0; c < degree; ++c) total += lens[c];
+  if (total > INT_MAX || Sq < 1) return CPATTN_ERR_SHAPE;
+  int st = check_attn_shape(B, H, Sq, D);
+  if (st != CPATTN_OK) return st;
+  const long long rows_kv = static_cast<long long>(degree) * B * kv_batch_rows;
+  if (rows_kv > INT_MAX || rows_kv * H * D > (1ll << 46)) return CPATTN_ERR_SHAPE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || (lse && !aligned4(lse)))
+    return CPATTN_ERR_ALIGNMENT;
+  st = check_device(nullptr);
+  if (st != CPATTN_OK) return st;
+  const std::vector<int> off = prefix(lens);
+  ProblemSpec ps = full_problem(q, k, v, out, lse, B, H, Sq);
+  ps.rows_kv = rows_kv;
+  ps.lse_pos0 = off[rank];
+  std::vector<GroupSpec> groups;
+  for (int b = 0; b < B; ++b) {
+    GroupSpec g;
+    g.prob = 0;
+    g.b = b;
+    SegSpec sg;
+    sg.row0 = b * Sq;
+    sg.nrows = Sq;
+    sg.s0 = off[rank];
+    for (int i_t = 0; i_t < degree; ++i_t) {
+      // Ring order from this rank's own chunk; under the causal mask the
+      // chunks after the shard are invisible and the own chunk, the one the
+      // mask cuts, is visited last (as in the fused causal ring).
+      const int t = causal ? (i_t + 1) % degree : i_t;
+      const int c = ((rank - t) % degree + degree) % degree;
+      if (causal && c > rank) continue;
+      if (lens[c] > 0) sg.kv.push_back(AttnKV{(c * B + b) * kv_batch_rows, lens[c], off[c]});
+    }
+    g.segs.push_back(std::move(sg));
+    groups.push_back(std::move(g));
+  }
+  return run_attention({ps}, groups, D, false, causal != 0, stream);
+}
+
+int cpattn_rank_buffer_attention(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H,
+                                 int S, int D, int degree, const int *seq_splits, int causal,
+                                 cpattn_stream_t stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return CPATTN_ERR_NULL;
+  int st = check_attn_shape(B, H, S, D);
+  if (st != CPATTN_OK) return st;
+  if (degree < 1 || degree > kMaxRanks) return CPATTN_ERR_DEGREE;
+  std::vector<int> lens;
+  st = resolve_splits(S, degree, seq_splits, lens);
+  if (st != CPATTN_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || (lse && !aligned4(lse)))
+    return CPATTN_ERR_ALIGNMENT;
+  st = check_device(nullptr);
+  if (st != CPATTN_OK) return st;
+  const std::vector<int> off = prefix(lens);
+  std::vector<ProblemSpec> probs{full_problem(q, k, v, out, lse, B, H, S)};
+  std::vector<GroupSpec> groups;
+  // Every rank buffer attends every rank buffer of its batch element: the
+  // ring plan over the buffers, rows B*off_u + b*len_u.
+  ring_groups(groups, 0, B, lens, off, -1, causal != 0, [&](int b, int c) { return B * off[c] + b * lens[c]; });
+  return run_attention(probs, groups, D, false, causal != 0, stream);
 }
 
 size_t cpattn_attention_backward_workspace_bytes(int B, int H, int S) {

@@ -38,10 +38,14 @@ constexpr int kQTilesPerCTA = 2;
 struct alignas(64) AttnProblem {
   CUtensorMap tm_q, tm_k, tm_v;   // 3-D maps over [rows, H, D] bf16, box {64, 1, 128}, 128B swizzle
   void *out;                      // [rows, H, D] bf16 or float32 (same rows as Q)
-  float *lse;                     // may be null; index b*lse_b + (h + lse_h0)*lse_h + s
+  float *lse;                     // may be null; index b*lse_b + (h + lse_h0)*lse_h + (s - lse_pos0)
+  const float *prev;              // null, or a previous partial state to merge into: float32 [rows, H, D]
+                                  // (same rows as Q, normalised over its keys) with its LSE read from
+                                  // `lse` before it is overwritten; may alias `out` when out is float32
   long long lse_b;
   long long lse_h;
   int lse_h0;
+  int lse_pos0;                   // sequence position of LSE column 0
   int H;
 };
 

@@ -308,6 +308,101 @@ int cpattn_unified_attention(const void *q, const void *k, const void *v, void *
                              const int *ring_lens, const int *head_splits, void *workspace,
                              size_t workspace_bytes, cpattn_stream_t stream);
 
+/* ------------------------------------- building blocks of the exchanges */
+
+/*
+ * The calls below are what one rank runs when the shards live on different
+ * GPUs and the exchanges are real collectives (the Python module
+ * context_attention_long_b200.exchange moves the data with torch.distributed
+ * over NCCL and calls these for every step of local compute).
+ */
+
+/*
+ * One ring step of one rank, merged into the rank's running result
+ * ([CP] "Ring Attention": each GPU computes attention against the K/V block it
+ * holds, then passes the block on; [API] convert_to_fp32: the partial output
+ * and its LSE are kept in float32; [SP] "Numerics across node boundaries":
+ * partial results are combined with the online-softmax merge; [SP]
+ * "Cross-Node Sequence Parallelism": the point-to-point rotation overlaps the
+ * attention of the block already held).
+ *
+ * Attention of the rank's queries against the one K/V chunk it holds now:
+ *   q          [B, Sq, H, D] bf16, sequence positions q_pos0 .. q_pos0+Sq-1.
+ *   k, v       [B, kv_batch_rows, H, D] bf16; the first Skv rows of every
+ *              batch element are the chunk (positions kv_pos0 ..);
+ *              kv_batch_rows = Skv for a contiguous chunk, larger for a chunk
+ *              padded to the longest one (the all-gather of [CP] "Ring
+ *              Anything Attention").  Skv may be 0 (an empty chunk).
+ *   prev_out   NULL: no earlier state; out and lse receive this chunk's
+ *              partial result (normalised over its keys) and its LSE.
+ *              Otherwise float32 [B, Sq, H, D], the running result over the
+ *              chunks already visited, whose LSE is in `lse` on entry; out and
+ *              lse receive the LSE-rule merge of the two.  May alias out when
+ *              out_f32 = 1 (each element is read before it is written, by the
+ *              same thread).
+ *   out        [B, Sq, H, D], float32 (out_f32 = 1: an intermediate state) or
+ *              bf16 (out_f32 = 0: the final output).
+ *   lse        [B, H, Sq] float32, natural log; required (see prev_out).
+ *   causal     1: key j is visible to query i iff kv_pos0 + j <= q_pos0 + i
+ *              ([USP] section 7: masking by positions).  A query that sees no
+ *              key of the chunk keeps the earlier state unchanged (out = 0 and
+ *              LSE = -inf without one).
+ * Errors: NULL, SHAPE (B, H, Sq < 1, Skv < 0, kv_batch_rows < max(Skv, 1),
+ * negative positions, D not 64/128), ALIGNMENT, UNSUPPORTED, CUDA.
+ */
+int cpattn_ring_chunk_attention(const void *q, const void *k, const void *v, void *out, float *lse,
+                                const float *prev_out, int B, int H, int Sq, int Skv, int kv_batch_rows, int D,
+                                int q_pos0, int kv_pos0, int causal, int out_f32, cpattn_stream_t stream);
+
+/*
+ * Attention of one rank's query shard against K/V chunks gathered from every
+ * rank ([SP] "Choosing The Attention Exchange": kv_gather all-gathers K and V
+ * and each rank computes its own rows; [API] rotate_method "allgather": ring
+ * attention gathers the chunks, then walks them; [CP] "Ring Anything
+ * Attention": chunks are padded to the longest before the all-gather and
+ * sliced back before attention).  One launch; the chunks are visited in ring
+ * order from the rank's own chunk with the running (m, l, O) state on chip.
+ *
+ *   k, v       `degree` consecutive [B, kv_batch_rows, H, D] bf16 blocks
+ *              (what an all-gather of padded chunks delivers); chunk c holds
+ *              kv_lens[c] <= kv_batch_rows valid rows per batch element, at
+ *              sequence positions off_c = kv_lens[0] + ... + kv_lens[c-1].
+ *   kv_lens    host int[degree], zeros allowed; NULL: every chunk has
+ *              kv_batch_rows rows.
+ *   rank       0 <= rank < degree: the shard the queries belong to.
+ *   q, out     [B, kv_lens[rank], H, D] bf16, the rank's own tokens.
+ *   lse        [B, H, kv_lens[rank]] float32 or NULL.
+ *   causal     1: chunks after `rank` are skipped and the own chunk is masked
+ *              by position (the ring's use; kv_gather itself is non-causal).
+ * Errors: NULL, SHAPE (kv_lens[rank] = 0 included), DEGREE (degree outside
+ * 1..512, rank outside 0..degree-1), SPLITS (a length < 0 or >
+ * kv_batch_rows), ALIGNMENT, UNSUPPORTED, CUDA.
+ */
+int cpattn_gathered_kv_attention(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H,
+                                 int D, int degree, const int *kv_lens, int kv_batch_rows, int rank, int causal,
+                                 cpattn_stream_t stream);
+
+/*
+ * Attention over a sequence held as `degree` rank buffers [B, S_u, H, D]
+ * concatenated in rank order -- the layout in which the first all-to-all of
+ * Ulysses attention delivers a rank's heads ([CP] "Ulysses Attention";
+ * [USP] section 4: after the all-to-all every GPU holds every token of a
+ * subset of the heads and runs ordinary attention over them).  Every query
+ * attends all S keys of its batch element (causal = 1: the keys at
+ * positions <= its own, a token's position being its index in the full
+ * sequence); the output is written in the same layout, ready for the second
+ * all-to-all.
+ *
+ *   q, k, v, out  rank-buffer layout, bf16 (for B = 1 the plain [1, S, H, D]).
+ *   lse           [B, H, S] float32 (global positions) or NULL.
+ *   seq_splits    host int[degree] or NULL (equal split).
+ * Errors: NULL, SHAPE, DEGREE (degree outside 1..64), INDIVISIBLE, SPLITS,
+ * ALIGNMENT, UNSUPPORTED, CUDA.
+ */
+int cpattn_rank_buffer_attention(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H,
+                                 int S, int D, int degree, const int *seq_splits, int causal,
+                                 cpattn_stream_t stream);
+
 /* ---------------------------------------------------------------- causal */
 
 /*
