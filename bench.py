@@ -1,19 +1,24 @@
 #!/usr/bin/env python
 """Benchmark of the context-parallel attention hot path on B200.
 
-One step = one pass of the whole hot path over the image-DiT workload
-(B=1, H=24, S=4608, D=128, seeded synthetic bf16, RMS-normalised Q/K):
-  * ring attention, ring_degree 4 (fused: one kernel walks the K/V chunks in
+One step = one pass of the whole hot path over the video-DiT workload
+(B=1, H=40, S=32760, D=128, seeded synthetic bf16, RMS-normalised Q/K), the
+largest single-GPU workload:
+  * ring attention, ring_degree 8 (fused: one kernel walks the K/V chunks in
     ring order and merges them with the LSE rule on chip),
-  * Ulysses attention, degree 4: permute Q, K, V to the head-sharded layout,
-    head-sharded local attention, unpermute the output.
+  * unified ring 8 x Ulysses 2 attention: permute Q, K, V to the head groups,
+    ring attention per head group, unpermute the output.
 Metric: attention TFLOP/s = (4*B*H*S^2*D per attention pass) * passes / time.
+The HBM-bound kernels (the Q/K/V permute, the unpermute and the 8-way LSE
+merge) are timed beside the step on the same sizes and reported inside
+`roofline` with the attention kernel.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--extras]
 
-N > 1 (torchrun): independent replicas, one per GPU (the workload does not
-shard across GPUs here: every shard is emulated in one GPU's memory); the step
-time is the max over ranks and `value` counts the work of all ranks.
+N > 1 (torchrun, one process per GPU, NCCL): the sequence is sharded over the
+GPUs and the exchanges are real collectives (context_attention_long_b200.exchange):
+ring over all N GPUs and unified (N/2 ring) x (Ulysses 2); the same total work
+as one GPU's step (strong scaling), timed as the max over ranks.
 """
 from __future__ import annotations
 
@@ -32,12 +37,13 @@ REPO = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, REPO)
 
 METRIC = "attention TFLOP/s (4·B·H·S²·D) & % BF16 peak; permute/merge GB/s & % HBM"
-WORKLOAD = "dit"
+WORKLOAD = "video"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
-# Measured NVLink peer copy of this machine's B200s, GB/s per direction (input of
-# the exchange-selection model only; no collective runs here).
-NVLINK_PEER_GBS = 770.0
+# Link bandwidth fed to the exchange-selection model (--extras) unless
+# --link-gbs is given: NVLink 5's nominal 900 GB/s per direction per GPU, an
+# assumption taken from the vendor's specification, not a measurement.
+NOMINAL_LINK_GBS = 900.0
 
 
 def load_peaks():
@@ -131,30 +137,47 @@ class ClockSampler:
                 "sm_max_mhz": float(self.max_mhz), "reasons": reasons, "samples": len(win)}
 
 
-def aggregate_over_ranks(ms_local, steps, units_per_step, world, dist=None, device="cpu"):
-    """Whole-job figures from every rank's device-timed milliseconds for
-    `steps` steps: the job time is the max over ranks (all ranks do the same
-    work, emulated independently), and the throughput counts every rank's
-    units.  Returns (ms per step, units per second)."""
+def max_over_ranks(values, world, dist=None, device="cpu"):
+    """Every rank's device-timed figures -> their maximum over the ranks (the
+    job takes as long as its slowest rank)."""
     import torch
-    ms = float(ms_local)
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
     if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=device)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    return ms / steps, world * units_per_step * steps / (ms * 1e-3)
+    return [float(x) for x in t.tolist()]
+
+
+def multi_gpu_shards(S, world, ulysses_degree=2):
+    """The sequence split of the multi-GPU step: every rank's tokens (front-
+    loaded split of S over the ranks), and the unified grid's view of the same
+    shards: rank (i, j) = i * ulysses_degree + j holds sub-shard j of ring
+    chunk i.  Returns (lens, ring_lens, subs)."""
+    base, extra = divmod(S, world)
+    lens = [base + (1 if r < extra else 0) for r in range(world)]
+    R = world // ulysses_degree
+    subs = [[lens[ulysses_degree * i + j] for j in range(ulysses_degree)] for i in range(R)]
+    return lens, [sum(x) for x in subs], subs
 
 
 # ----------------------------------------------------------------- reference arm (the oracle)
+def flush_l2(flush):
+    """Evicts L2: writes a buffer larger than L2, then reads it back, so that
+    L2 holds clean lines of the flush buffer (a write alone would leave dirty
+    lines that the next kernel must write back to HBM before it can use L2)."""
+    import torch
+    flush.zero_()
+    torch.sum(flush, dtype=torch.int64)
+
+
 def median_event_ms(fn, flush, stream, reps=10, warmup=1):
     """Median CUDA-event time of fn() on `stream`, each rep after an L2 flush
-    (a write of a buffer larger than L2) outside the timed events."""
+    (flush_l2) outside the timed events."""
     import torch
     for _ in range(warmup):
         fn()
     times = []
     for _ in range(reps):
-        flush.zero_()
+        flush_l2(flush)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         fn()
@@ -165,11 +188,12 @@ def median_event_ms(fn, flush, stream, reps=10, warmup=1):
 
 
 def oracle_sample_step(cfg, q, k, v, rows_per_shard, seed):
-    """The oracle's hot path on a bounded sample of query rows: for each ring
+    """The oracle's step on a bounded sample of query rows: for every ring
     shard, sampled rows attend every K/V chunk in ring order (partials + LSE
-    merge), and the same rows through the Ulysses layout (head-sharded local
-    attention = monolithic attention per head group).  Returns attention FLOPs
-    processed (4 * rows * S * D per head and pass)."""
+    merge) -- the ring pass -- and the same rows attend all S keys of their
+    head -- the unified pass, whose head groups run that attention per head in
+    exact arithmetic.  Each head's K/V is widened to float64 once per step.
+    Returns the attention FLOPs processed (4 * rows * S * D per head and pass)."""
     import oracle
     from context_attention_long_b200 import inputs as inp
     B, S, H, D = q.shape
@@ -177,22 +201,22 @@ def oracle_sample_step(cfg, q, k, v, rows_per_shard, seed):
     lens = [S // P] * P
     off = oracle.offsets(lens)
     rng = np.random.Generator(np.random.PCG64(seed))
+    rows = [off[r] + rng.integers(0, lens[r], size=rows_per_shard) for r in range(P)]
     flops = 0
-    for r in range(P):
-        rows = off[r] + rng.integers(0, lens[r], size=rows_per_shard)
-        for b in range(B):
-            for h in range(H):
-                qh = inp.bf16_bits_to_f64(q[b, rows, h, :])
-                kh = inp.bf16_bits_to_f64(k[b, :, h, :])
-                vh = inp.bf16_bits_to_f64(v[b, :, h, :])
+    for b in range(B):
+        for h in range(H):
+            kh = inp.bf16_bits_to_f64(k[b, :, h, :])
+            vh = inp.bf16_bits_to_f64(v[b, :, h, :])
+            for r in range(P):
+                qh = inp.bf16_bits_to_f64(q[b, rows[r], h, :])
                 outs, lses = [], []
                 for c in oracle.ring_order(r, P):
                     o, l = oracle.attention_rows(qh, kh[off[c]:off[c + 1]], vh[off[c]:off[c + 1]])
                     outs.append(o[None, :, None, :])
                     lses.append(l[None, None, :])
                 oracle.lse_merge(outs, lses)
-                oracle.attention_rows(qh, kh, vh)   # Ulysses: local attention of the head group
-                flops += 2 * 4 * len(rows) * S * D
+                oracle.attention_rows(qh, kh, vh)   # unified: attention of the head over all S keys
+                flops += 2 * 4 * len(rows[r]) * S * D
     return flops
 
 
@@ -204,7 +228,7 @@ def run_reference(args):
     import torch
     cfg, q, k, v = inputs.config_inputs(WORKLOAD)
     threads = torch.get_num_threads()
-    rows = 8
+    rows = 1
     for _ in range(args.warmup):
         oracle_sample_step(cfg, q, k, v, rows, 0)
     t0 = time.perf_counter()
@@ -217,54 +241,80 @@ def run_reference(args):
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1), RMS-normalised Q/K, bf16-rounded)",
-        "config": config_block(cfg),
+        "config": config_block(cfg, args.gpus),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-                         "sample": f"{rows} query rows per ring shard per step, all {H} heads, ring path + Ulysses "
-                                   f"local attention, against the full S={S} K/V (fp64 numpy oracle)"},
+                         "sample": f"per step {rows} query row per ring shard x {H} heads, ring + unified passes "
+                                   f"vs all S={S} keys (fp64 numpy oracle)"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
 
 
-def config_block(cfg):
-    return {"workload": f"image-DiT B{cfg['B']} H{cfg['H']} S{cfg['S']} D{cfg['D']}: ring {cfg['ring_degree']} "
-                        f"(fused) + Ulysses {cfg['ulysses_degree']} (permute, local attention, unpermute)",
-            "B": cfg["B"], "H": cfg["H"], "S": cfg["S"], "D": cfg["D"], "ring_degree": cfg["ring_degree"],
-            "ulysses_degree": cfg["ulysses_degree"], "parallelism": "replicas",
-            "l2": "flushed before every timed step (256 MiB write outside the timed events)"}
+def config_block(cfg, world=1):
+    """The `config` of the bench line for `world` GPUs (both arms print it)."""
+    B, H, S, D = cfg["B"], cfg["H"], cfg["S"], cfg["D"]
+    if world == 1:
+        return {"workload": f"video-DiT B{B} H{H} S{S} D{D}: ring {cfg['ring_degree']} (fused) + unified ring "
+                            f"{cfg['ring_degree']} x Ulysses {cfg['ulysses_degree']}",
+                "B": B, "H": H, "S": S, "D": D, "ring_degree": cfg["ring_degree"],
+                "ulysses_degree": cfg["ulysses_degree"], "parallelism": "1 GPU, shards emulated in memory",
+                "l2": "inputs larger than L2 (335 MB each) and an L2 flush (256 MiB written, then read) before every timed step"}
+    return {"workload": f"video-DiT B{B} H{H} S{S} D{D}: ring {world} (NCCL P2P rotation) + unified ring "
+                        f"{world // 2} x Ulysses 2 (NCCL all-to-all), sequence sharded over {world} GPUs",
+            "B": B, "H": H, "S": S, "D": D, "ring_degree": world, "ulysses_degree": 2,
+            "parallelism": f"context parallel over {world} GPUs", "l2": "inputs larger than L2"}
 
 
 def cpu_baseline(cfg, q, k, v, budget_s=12.0):
     """The oracle, as it stands, on a bounded sample of the same workload."""
     import torch
     t0 = time.perf_counter()
-    flops, i, rows = 0, 0, 16
+    flops, i, rows = 0, 0, 2
     while time.perf_counter() - t0 < budget_s:
         flops += oracle_sample_step(cfg, q, k, v, rows, 1000 + i)
         i += 1
     dt = time.perf_counter() - t0
     B, S, H, D = q.shape
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": torch.get_num_threads(), "kind": "oracle",
-            "sample": f"{i} x ({rows} query rows per ring shard, all {H} heads, ring path with LSE merge + Ulysses "
-                      f"local attention, against the full S={S} K/V); fp64 numpy oracle, {dt:.1f} s"}
+            "sample": f"{i} x ({rows} rows per ring shard x {H} heads, ring + unified passes vs S={S} keys), "
+                      f"{dt:.1f} s"}
+
+
+def hbm_entry(name, nbytes, ms, peak_gbs, peaks_kind):
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"kernel": name, "bound": "hbm", "achieved": round(gbs, 1), "unit": "GB/s", "peak": peak_gbs,
+            "frac": round(gbs / peak_gbs, 4), "bytes": int(nbytes), "ms": round(ms, 4), "peak_kind": peaks_kind}
+
+
+def tensor_entry(name, flops, ms, peak_tf):
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"kernel": name, "bound": "tensor", "achieved": round(tf, 1), "unit": "TFLOP/s",
+            "frac": round(tf / peak_tf, 4), "flops": flops, "ms": round(ms, 4)}
 
 
 # ----------------------------------------------------------------- our arm
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--no-breakdown", action="store_true")
+    ap.add_argument("--extras", action="store_true",
+                    help="also time the causal, backward and projection paths on the image-DiT workload and the "
+                         "exchange-selection model; printed as a second JSON line")
+    ap.add_argument("--link-gbs", type=float, default=NOMINAL_LINK_GBS,
+                    help="interconnect bandwidth per direction fed to the exchange-selection model (--extras); "
+                         "default: NVLink 5 nominal, an assumption")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true",
                     help="time every workload's paths (one JSON line per path) instead of the step")
-    ap.add_argument("--kernel", default=None, choices=["ring", "causal_ring", "head_sharded", "permute", "permute_qkv", "merge", "ring_step", "backward",
-                             "qkv_projection", "output_projection"],
-                    help="profiling mode: run only this kernel (warmup + steps launches) on the workload")
+    ap.add_argument("--kernel", default=None, choices=["ring", "causal_ring", "head_sharded", "permute", "permute_qkv",
+                                                       "unpermute", "merge", "ring_step", "backward",
+                                                       "qkv_projection", "output_projection", "unified"],
+                    help="profiling mode: run only this kernel (warmup + steps launches) on --workload")
+    ap.add_argument("--workload", default="dit", help="workload of --kernel mode")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -294,6 +344,8 @@ def main():
         build.build()
     if world > 1:
         dist.barrier()
+        run_multi_gpu(args, world, rank, dev)
+        return
 
     cfg, qb, kb, vb = inputs.config_inputs(WORKLOAD)
     B, S, H, D = qb.shape
@@ -306,33 +358,28 @@ def main():
     q, k, v = (t.to(dev) for t in (hq, hk, hv))
     out_r = torch.empty_like(q)
     lse_r = torch.empty((B, H, S), dtype=torch.float32, device=dev)
-    yq, yk, yv, yo = (torch.empty(B * S * H * D, dtype=torch.bfloat16, device=dev) for _ in range(4))
-    out_u = torch.empty(B * S * H * D, dtype=torch.bfloat16, device=dev)
+    out_u = torch.empty_like(q)
     lse_u = torch.empty((B, H, S), dtype=torch.float32, device=dev)
+    ws = torch.empty(api.cpattn_unified_workspace_bytes(B, H, S, D), dtype=torch.uint8, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
-    qf, kf, vf = q.reshape(-1), k.reshape(-1), v.reshape(-1)
 
     attn_flops = 4.0 * B * H * S * S * D      # one attention pass
-    step_flops = 2 * attn_flops               # ring + Ulysses
-    launches_per_step = 4                     # ring, Q/K/V permute, head-sharded attention, unpermute
-    n_ev = 5
+    step_flops = 2 * attn_flops               # ring + unified
+    launches_per_step = 4                     # ring; unified: Q/K/V permute, attention, unpermute
+    n_ev = 3
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
 
-    def step(e=None):
+    def step_on(qx, kx, vx, orx, oux, e=None):
         if e: e[0].record(stream)
-        api.cpattn_ring_attention(q, k, v, P, out=out_r, lse=lse_r, stream=stream)
+        api.cpattn_ring_attention(qx, kx, vx, P, out=orx, lse=lse_r, stream=stream)
         if e: e[1].record(stream)
-        api.cpattn_ulysses_permute_qkv(qf, kf, vf, B, S, H, D, U, yq=yq, yk=yk, yv=yv, stream=stream)
+        api.cpattn_unified_attention(qx, kx, vx, P, U, out=oux, lse=lse_u, workspace=ws, stream=stream)
         if e: e[2].record(stream)
-        api.cpattn_head_sharded_attention(yq, yk, yv, B, S, H, D, U, yo=yo, lse=lse_u, stream=stream)
-        if e: e[3].record(stream)
-        api.cpattn_ulysses_unpermute(yo, B, S, H, D, U, x=out_u, stream=stream)
-        if e: e[4].record(stream)
 
     for _ in range(args.warmup):
-        flush.zero_()
-        step()
+        flush_l2(flush)
+        step_on(q, k, v, out_r, out_u)
     torch.cuda.synchronize()
     st, code = api.cpattn_device_status()
     if st != 0:
@@ -340,38 +387,66 @@ def main():
 
     clocks = ClockSampler(dev)
     clocks.start()
-    if world > 1:
-        dist.barrier()
     torch.cuda.synchronize()
     t_wall0 = time.perf_counter()
     for i in range(args.steps):
-        flush.zero_()                 # evict L2 (outside the timed events)
-        step(ev[i])
+        flush_l2(flush)               # evict L2 (outside the timed events)
+        step_on(q, k, v, out_r, out_u, ev[i])
     torch.cuda.synchronize()
     t_wall1 = time.perf_counter()
-    if world > 1:
-        dist.barrier()
     clocks.stop()
 
     per = np.array([[ev[i][j].elapsed_time(ev[i][j + 1]) for j in range(n_ev - 1)] for i in range(args.steps)])
     step_ms = per.sum(axis=1)
-    ms_per_step, flops_per_s = aggregate_over_ranks(float(step_ms.sum()), args.steps, step_flops, world,
-                                                    dist if world > 1 else None, dev)
-    value = flops_per_s / 1e12
+    ms_per_step = float(step_ms.sum()) / args.steps
+    value = step_flops / (ms_per_step * 1e-3) / 1e12
 
     peaks, peaks_kind = load_peaks()
+    peak_tf = float(peaks["bf16_tflops"])
+    peak_tf_sus = float(peaks.get("bf16_tflops_sustained", peak_tf))
+    hbm = float(peaks["hbm_gbs"])
     ring_ms = float(per[:, 0].mean())
     ring_tflops = attn_flops / (ring_ms * 1e-3) / 1e12
-    uattn_ms = float(per[:, 2].mean())
-    perm_ms = float(per[:, 1].mean())        # Q, K and V in one launch
-    unperm_ms = float(per[:, 3].mean())
+    uni_ms = float(per[:, 1].mean())
     tensor_bytes = B * S * H * D * 2
-    peak_tf = float(peaks["bf16_tflops"])
-    roofline = {"bound": "tensor", "kernel": "attn_fwd_kernel<128,bf16> (ring fused, P=4)",
+
+    # HBM-bound kernels of the step's unified flow at the same sizes, each rep
+    # after an L2 flush: the first all-to-all (Q, K and V in one launch; for
+    # B = 1 the unified flow's head-group layout is the Ulysses head-side
+    # layout), the second all-to-all, and the 8-way merge of float32 partials.
+    yq, yk, yv = (torch.empty_like(q) for _ in range(3))
+    ms_pq = median_event_ms(lambda: api.cpattn_ulysses_permute_qkv(q, k, v, B, S, H, D, U, yq=yq, yk=yk, yv=yv,
+                                                                   stream=stream), flush, stream, reps=7)
+    ms_up = median_event_ms(lambda: api.cpattn_ulysses_unpermute(yq, B, S, H, D, U, x=yk, stream=stream),
+                            flush, stream, reps=7)
+    del yq, yk, yv
+    po = torch.randn((P, B, S, H, D), device=dev, dtype=torch.float32)
+    pl = torch.randn((P, B, H, S), device=dev, dtype=torch.float32)
+    ob = torch.empty((B, S, H, D), device=dev, dtype=torch.bfloat16)
+    lo = torch.empty((B, H, S), device=dev, dtype=torch.float32)
+    ms_mg = median_event_ms(lambda: api.cpattn_lse_merge(po, pl, out_bf16=ob, lse_out=lo, want_f32=False,
+                                                         stream=stream), flush, stream, reps=7)
+    del po, pl, ob, lo
+    torch.cuda.empty_cache()
+    merge_bytes = B * H * S * (P * (4 * D + 4) + 2 * D + 4)
+    hbm_kernels = [
+        hbm_entry(f"permute_kernel: Q/K/V to {U} head groups, one launch", 6 * tensor_bytes, ms_pq, hbm, peaks_kind),
+        hbm_entry(f"permute_kernel: output back from {U} head groups", 2 * tensor_bytes, ms_up, hbm, peaks_kind),
+        hbm_entry(f"lse_merge_kernel<128,8>: P={P} fp32 partials -> bf16", merge_bytes, ms_mg, hbm, peaks_kind),
+    ]
+    causal_ms = median_event_ms(lambda: api.cpattn_causal_ring_attention(q, k, v, P, out=out_u, lse=lse_u,
+                                                                         stream=stream), flush, stream, reps=5)
+    tensor_kernels = [
+        tensor_entry(f"unified ring {P} x Ulysses {U} (in the step; 3 launches)", attn_flops, uni_ms, peak_tf),
+        tensor_entry(f"causal ring fused P={P} (visible pairs)", causal_flops(B, H, S, D), causal_ms, peak_tf),
+    ]
+    roofline = {"bound": "tensor", "kernel": f"attn_fwd_kernel<128,bf16> (ring fused, P={P}, in the step)",
                 "achieved": ring_tflops, "peak": peak_tf, "unit": "TFLOP/s", "frac": ring_tflops / peak_tf,
                 "peak_kind": f"bf16_tflops burst, {peaks_kind}",
-                "traffic": stored_traffic("attn_fwd_ring_dit"),
-                "algorithmic_flops_per_launch": attn_flops}
+                "frac_of_sustained": ring_tflops / peak_tf_sus,
+                "traffic": stored_traffic("attn_fwd_ring_video"),
+                "algorithmic_flops_per_launch": attn_flops,
+                "tensor_kernels": tensor_kernels, "hbm_kernels": hbm_kernels}
 
     # ---- end to end through the public API with host buffers
     # Every step uploads its Q, K, V from pinned host memory and downloads
@@ -379,127 +454,248 @@ def main():
     # streams with two device copies of the inputs and outputs, so step i+1's
     # upload and step i-1's download overlap step i's kernels (PCIe is full
     # duplex); the kernels of consecutive steps stay in order on one stream.
-    e2e = None
-    if True:
-        hout_r = torch.empty_like(out_r, device="cpu").pin_memory()
-        hout_u = torch.empty_like(out_u, device="cpu").pin_memory()
-        e2e_steps = max(3, min(args.steps, 50))
-        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
-        bufs = [(q, k, v, out_r, out_u),
-                (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(out_r),
-                 torch.empty_like(out_u))]
-        ev_in = [torch.cuda.Event() for _ in range(2)]
-        ev_comp = [torch.cuda.Event() for _ in range(2)]
-        ev_out = [torch.cuda.Event() for _ in range(2)]
+    hout_r = torch.empty_like(out_r, device="cpu").pin_memory()
+    hout_u = torch.empty_like(out_u, device="cpu").pin_memory()
+    e2e_steps = max(3, min(args.steps, 20))
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    bufs = [(q, k, v, out_r, out_u),
+            (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(out_r),
+             torch.empty_like(out_u))]
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
 
-        def step_on(qx, kx, vx, orx, oux):
-            api.cpattn_ring_attention(qx, kx, vx, P, out=orx, lse=lse_r, stream=stream)
-            api.cpattn_ulysses_permute_qkv(qx.reshape(-1), kx.reshape(-1), vx.reshape(-1), B, S, H, D, U,
-                                           yq=yq, yk=yk, yv=yv, stream=stream)
-            api.cpattn_head_sharded_attention(yq, yk, yv, B, S, H, D, U, yo=yo, lse=lse_u, stream=stream)
-            api.cpattn_ulysses_unpermute(yo, B, S, H, D, U, x=oux, stream=stream)
+    def pipeline(n, e_start=None, e_end=None):
+        if e_start is not None:
+            e_start.record(s_in)
+        for i in range(n):
+            bi = i % 2
+            qx, kx, vx, orx, oux = bufs[bi]
+            if i >= 2:
+                s_in.wait_event(ev_comp[bi])          # step i-2 has finished reading these inputs
+            with torch.cuda.stream(s_in):
+                qx.copy_(hq, non_blocking=True); kx.copy_(hk, non_blocking=True); vx.copy_(hv, non_blocking=True)
+            ev_in[bi].record(s_in)
+            stream.wait_event(ev_in[bi])
+            if i >= 2:
+                stream.wait_event(ev_out[bi])         # step i-2's outputs are on the host
+            step_on(qx, kx, vx, orx, oux)
+            ev_comp[bi].record(stream)
+            s_out.wait_event(ev_comp[bi])
+            with torch.cuda.stream(s_out):
+                hout_r.copy_(orx, non_blocking=True); hout_u.copy_(oux, non_blocking=True)
+            ev_out[bi].record(s_out)
+        if e_end is not None:
+            s_out.wait_event(ev_comp[(n - 1) % 2])
+            e_end.record(s_out)
 
-        def pipeline(n, e_start=None, e_end=None):
-            if e_start is not None:
-                e_start.record(s_in)
-            for i in range(n):
-                bi = i % 2
-                qx, kx, vx, orx, oux = bufs[bi]
-                if i >= 2:
-                    s_in.wait_event(ev_comp[bi])          # step i-2 has finished reading these inputs
-                with torch.cuda.stream(s_in):
-                    qx.copy_(hq, non_blocking=True); kx.copy_(hk, non_blocking=True); vx.copy_(hv, non_blocking=True)
-                ev_in[bi].record(s_in)
-                stream.wait_event(ev_in[bi])
-                if i >= 2:
-                    stream.wait_event(ev_out[bi])         # step i-2's outputs are on the host
-                step_on(qx, kx, vx, orx, oux)
-                ev_comp[bi].record(stream)
-                s_out.wait_event(ev_comp[bi])
-                with torch.cuda.stream(s_out):
-                    hout_r.copy_(orx, non_blocking=True); hout_u.copy_(oux, non_blocking=True)
-                ev_out[bi].record(s_out)
-            if e_end is not None:
-                s_out.wait_event(ev_comp[(n - 1) % 2])
-                e_end.record(s_out)
+    pipeline(2)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    pipeline(e2e_steps, e0, e1)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    # every step computes the same deterministic result: the downloaded
+    # outputs must equal the device outputs
+    if not (torch.equal(hout_r.view(torch.int16), out_r.cpu().view(torch.int16)) and
+            torch.equal(hout_u.view(torch.int16), out_u.cpu().view(torch.int16))):
+        raise RuntimeError("end-to-end pipeline: downloaded outputs differ from the device results")
+    e2e = {"value": step_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+           "h2d_bytes_per_step": 3 * tensor_bytes, "d2h_bytes_per_step": 2 * tensor_bytes,
+           "note": "pinned host Q/K/V in, both outputs out, every step; 3 streams, 2 device buffers"}
+    del bufs
 
-        pipeline(2)
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        pipeline(e2e_steps, e0, e1)
-        torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1) / e2e_steps
-        # every step computes the same deterministic result: the downloaded
-        # outputs must equal the device outputs of the timed steps
-        if not (torch.equal(hout_r.view(torch.int16), out_r.cpu().view(torch.int16)) and
-                torch.equal(hout_u.view(torch.int16), out_u.cpu().view(torch.int16))):
-            raise RuntimeError("end-to-end pipeline: downloaded outputs differ from the device results")
-        e2e = {"value": world * step_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
-               "h2d_bytes_per_step": 3 * tensor_bytes, "d2h_bytes_per_step": 2 * tensor_bytes,
-               "note": "pinned host Q/K/V copied in and both attention outputs copied out every step; "
-                       "uploads, kernels and downloads on three streams, two device buffers"}
-        del bufs
+    # Mean absolute difference of the sharded paths' outputs from unsharded
+    # attention (the fused kernel with one shard), in the MAE style of the
+    # pages' sharded-vs-unsharded check; the paths differ only in rounding order.
+    mono, _ = api.cpattn_ring_attention(q, k, v, 1, want_lse=False, stream=stream)
+    torch.cuda.synchronize()
+    mae = {"ring": float((out_r.float() - mono.float()).abs().mean()),
+           "unified": float((out_u.float() - mono.float()).abs().mean())}
+    del mono
 
-    kernels = {
-        "ring_fused_attention": {"ms": ring_ms, "TFLOP/s": ring_tflops, "frac_bf16_peak": ring_tflops / peak_tf},
-        "head_sharded_attention": {"ms": uattn_ms, "TFLOP/s": attn_flops / (uattn_ms * 1e-3) / 1e12,
-                                   "frac_bf16_peak": attn_flops / (uattn_ms * 1e-3) / 1e12 / peak_tf},
-        "ulysses_permute_qkv_dit": {"ms": perm_ms, "GB/s": 6 * tensor_bytes / (perm_ms * 1e-3) / 1e9},
-        "ulysses_unpermute_dit": {"ms": unperm_ms, "GB/s": 2 * tensor_bytes / (unperm_ms * 1e-3) / 1e9},
+    st, code = api.cpattn_device_status()
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1), RMS-normalised Q/K, bf16)",
+        "config": config_block(cfg), "roofline": roofline, "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks.summary(t_wall0, t_wall1), "e2e": e2e, "device_status": code,
+        "mae_vs_unsharded": mae,
     }
-    if not args.no_breakdown:
-        kernels.update(breakdown(api, torch, dev, flush, peaks, inputs))
-        kernels.update(causal_paths(api, torch, flush, peaks, q, k, v, P, U))
-        kernels.update(backward_paths(api, torch, flush, peaks, q, k, v, P))
-        kernels.update(projection_paths(api, torch, flush, peaks, inputs, B, S, H, D, U))
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, qb, kb, vb)
+    extras = None
+    if args.extras:
+        del q, k, v, out_r, out_u, ws, hq, hk, hv
+        torch.cuda.empty_cache()
+        extras = dit_extras(api, torch, dev, flush, peaks, inputs, args.link_gbs)
+    if extras is not None:
+        print(json.dumps({"extras": extras}))
+    print(json.dumps(line))
 
-    # Accounting: what P GPUs would exchange per rank for this workload (on one
-    # GPU the exchanges are emulated in memory).
+
+def run_multi_gpu(args, world, rank, dev):
+    """N > 1 GPUs (one process each, NCCL): the video workload's sequence is
+    sharded over the ranks and the exchanges are real collectives
+    (context_attention_long_b200.exchange): ring attention over all N ranks
+    with the point-to-point K/V rotation overlapped with each step's kernel,
+    and unified attention on an (N/2 ring) x (Ulysses 2) grid.  The total work
+    is the single-GPU step's (strong scaling); the step time is the max over
+    ranks of each rank's CUDA-event time."""
+    import torch
+    import torch.distributed as dist
+    from context_attention_long_b200 import api, exchange, inputs
+    if world % 2:
+        raise SystemExit("the unified (ring x Ulysses 2) part of the step needs an even number of GPUs")
+    cfg, qb, kb, vb = inputs.config_inputs(WORKLOAD)
+    B, S, H, D = qb.shape
+    U = 2
+    R = world // U
+    lens, ring_lens, subs = multi_gpu_shards(S, world, U)
+    off = np.concatenate([[0], np.cumsum(lens)]).astype(int)
+    a, b = off[rank], off[rank + 1]
+
+    def shard(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits[:, a:b]).view(np.int16)).view(torch.bfloat16)
+
+    hq, hk, hv = (shard(x).pin_memory() for x in (qb, kb, vb))
+    q, k, v = (t.to(dev) for t in (hq, hk, hv))
+    del qb, kb, vb
+    ring_group, uly_group = exchange.unified_groups(R, U)
+    stream = torch.cuda.current_stream()
+    attn_flops = 4.0 * B * H * S * S * D
+    step_flops = 2 * attn_flops
+    launches_per_step = world + (1 + R + 1)     # ring steps; unified: pack, R ring steps, unpack
+
+    def step(e=None):
+        if e: e[0].record(stream)
+        o_r, _ = exchange.ring_attention(q, k, v, None, lens, rotate_method="p2p")
+        if e: e[1].record(stream)
+        o_u, _ = exchange.unified_attention(q, k, v, ring_group, uly_group, ring_lens, subs)
+        if e: e[2].record(stream)
+        return o_r, o_u
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    clocks = ClockSampler(dev)
+    clocks.start()
+    dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(ev[i])
+    torch.cuda.synchronize()
+    t1 = time.perf_counter()
+    dist.barrier()
+    clocks.stop()
+    per = np.array([[ev[i][j].elapsed_time(ev[i][j + 1]) for j in range(2)] for i in range(args.steps)])
+    tot_ms, ring_tot_ms = max_over_ranks([per.sum(), per[:, 0].sum()], world, dist, dev)
+    ms_per_step = tot_ms / args.steps
+    ring_ms = ring_tot_ms / args.steps
+    value = step_flops / (ms_per_step * 1e-3) / 1e12
+
+    # end to end through the public API: this rank's shard uploaded from
+    # pinned host memory and both outputs downloaded, every step
+    ho_r, ho_u = torch.empty_like(hq).pin_memory(), torch.empty_like(hq).pin_memory()
+    e2e_steps = max(3, min(args.steps, 10))
+    dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True); v.copy_(hv, non_blocking=True)
+        o_r, o_u = step()
+        ho_r.copy_(o_r, non_blocking=True); ho_u.copy_(o_u, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks([e0.elapsed_time(e1) / e2e_steps], world, dist, dev)[0]
+
+    peaks, peaks_kind = load_peaks()
+    peak_tf = float(peaks["bf16_tflops"])
+    rank_ring_flops = attn_flops / world
+    st, code = api.cpattn_device_status()
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1), RMS-normalised Q/K, bf16)",
+        "config": config_block(cfg, world),
+        "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128> ring steps incl. overlapped K/V rotation",
+                     "achieved": rank_ring_flops / (ring_ms * 1e-3) / 1e12, "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": rank_ring_flops / (ring_ms * 1e-3) / 1e12 / peak_tf,
+                     "peak_kind": f"bf16_tflops burst, {peaks_kind}", "traffic": None},
+        "gpu_launches": launches_per_step * args.steps, "clocks": clocks.summary(t0, t1),
+        "e2e": {"value": step_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": 3 * B * S * H * D * 2, "d2h_bytes_per_step": 2 * B * S * H * D * 2,
+                "note": "every rank uploads its Q/K/V shard and downloads both outputs; summed over ranks"},
+        "device_status": code,
+    }
+    if rank == 0:
+        print(json.dumps(line))
+    del ring_group, uly_group
+    dist.destroy_process_group()
+
+
+def dit_extras(api, torch, dev, flush, peaks, inputs, link_gbs):
+    """The image-DiT workload's other paths, timed each on its own: the step's
+    kernels at that size, the causal variants, the backward, the fused
+    projections, the exchange accounting and the exchange-selection model."""
+    cfg, qb, kb, vb = inputs.config_inputs("dit")
+    B, S, H, D = qb.shape
+    P, U = cfg["ring_degree"], cfg["ulysses_degree"]
+    q, k, v = (torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev) for x in (qb, kb, vb))
+    stream = torch.cuda.current_stream()
+    attn_flops = 4.0 * B * H * S * S * D
+    peak_tf = float(peaks["bf16_tflops"])
+    hbm = float(peaks["hbm_gbs"])
+    tensor_bytes = B * S * H * D * 2
+    qf, kf, vf = q.reshape(-1), k.reshape(-1), v.reshape(-1)
+    yq, yk, yv, yo = (torch.empty_like(qf) for _ in range(4))
+    out = torch.empty_like(qf)
+    res = {}
+    ms = median_event_ms(lambda: api.cpattn_ring_attention(q, k, v, P, stream=stream), flush, stream)
+    res[f"ring_fused_p{P}"] = {"ms": ms, "TFLOP/s": attn_flops / (ms * 1e-3) / 1e12}
+    ms = median_event_ms(lambda: api.cpattn_ulysses_permute_qkv(qf, kf, vf, B, S, H, D, U, yq=yq, yk=yk, yv=yv,
+                                                                stream=stream), flush, stream)
+    res[f"ulysses_permute_qkv_{U}"] = {"ms": ms, "GB/s": 6 * tensor_bytes / (ms * 1e-3) / 1e9}
+    ms = median_event_ms(lambda: api.cpattn_head_sharded_attention(yq, yk, yv, B, S, H, D, U, yo=yo,
+                                                                   stream=stream), flush, stream)
+    res[f"head_sharded_attention_{U}"] = {"ms": ms, "TFLOP/s": attn_flops / (ms * 1e-3) / 1e12}
+    ms = median_event_ms(lambda: api.cpattn_ulysses_unpermute(yo, B, S, H, D, U, x=out, stream=stream),
+                         flush, stream)
+    res[f"ulysses_unpermute_{U}"] = {"ms": ms, "GB/s": 2 * tensor_bytes / (ms * 1e-3) / 1e9}
+    for key in res:
+        if "GB/s" in res[key]:
+            res[key]["frac_hbm"] = res[key]["GB/s"] / hbm
+        else:
+            res[key]["frac_bf16_peak"] = res[key]["TFLOP/s"] / peak_tf
+    res.update(causal_paths(api, torch, flush, peaks, q, k, v, P, U))
+    res.update(backward_paths(api, torch, flush, peaks, q, k, v, P))
+    res.update(projection_paths(api, torch, flush, peaks, inputs, B, S, H, D, U))
+    ring_tflops = res[f"ring_fused_p{P}"]["TFLOP/s"]
+
+    # Accounting: what P GPUs would exchange per rank for this workload.
     exch = {}
     for mode, deg in (("ring", P), ("ulysses", U), ("kv_gather", P)):
         snd, rcv = api.cpattn_exchange_bytes(mode, B, H, S, D, deg)
         exch[f"{mode}_{deg}"] = {"send": snd[0], "recv": rcv[0]}
     exch["kv_gather_over_ulysses"] = exch[f"kv_gather_{P}"]["recv"] / max(1, exch[f"ulysses_{U}"]["recv"])
-    # The exchange-selection model fed with this run's measured attention
-    # throughput, the measured HBM bandwidth and the measured NVLink peer-copy
-    # bandwidth of this machine's B200s (770 GB/s per direction).
-    exch_plan = {"inputs": {"link_gbs": NVLINK_PEER_GBS, "attn_tflops": round(ring_tflops, 1),
-                            "hbm_gbs": float(peaks["hbm_gbs"])}}
+    # The exchange-selection model fed with this run's measured ring
+    # throughput, the HBM bandwidth and the link bandwidth (--link-gbs;
+    # default NVLink 5 nominal, an assumption, not a measurement).
+    exch_plan = {"inputs": {"link_gbs": link_gbs,
+                            "link_kind": "nominal assumption" if link_gbs == NOMINAL_LINK_GBS else "given",
+                            "attn_tflops": round(ring_tflops, 1), "hbm_gbs": hbm}}
     for deg in (2, 4, 8):
         for causal in (False, True):
-            pl = api.cpattn_plan_exchange(B, H, S, D, deg, NVLINK_PEER_GBS, ring_tflops, float(peaks["hbm_gbs"]),
-                                          causal=causal)
+            pl = api.cpattn_plan_exchange(B, H, S, D, deg, link_gbs, ring_tflops, hbm, causal=causal)
             exch_plan[f"P{deg}" + ("_causal" if causal else "")] = {
                 "best": pl["best"],
                 "us": {m: (None if pl[m]["seconds"] is None else round(pl[m]["seconds"] * 1e6, 1))
                        for m in ("ring", "ulysses", "kv_gather")}}
-
-    # Mean absolute difference of the sharded paths' outputs from unsharded
-    # attention (the fused kernel with one shard), in the MAE style of the
-    # pages' sharded-vs-unsharded check; the paths differ only in rounding order.
-    mono, _ = api.cpattn_ring_attention(q, k, v, 1, stream=stream)
-    torch.cuda.synchronize()
-    mono_f = mono.float()
-    mae = {"ring": float((out_r.float() - mono_f).abs().mean()),
-           "ulysses": float((out_u.view(B, S, H, D).float() - mono_f).abs().mean())}
-    del mono, mono_f
-
-    st, code = api.cpattn_device_status()
-    line = {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1), RMS-normalised Q/K, bf16)",
-        "config": config_block(cfg), "roofline": roofline, "gpu_launches": launches_per_step * args.steps,
-        "clocks": clocks.summary(t_wall0, t_wall1), "e2e": e2e, "kernels": kernels,
-        "device_status": code, "exchange_bytes_per_rank": exch, "exchange_plan": exch_plan,
-        "mae_vs_unsharded": mae,
-    }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(cfg, qb, kb, vb)
-    if rank == 0:
-        print(json.dumps(line))
-    if world > 1:
-        dist.destroy_process_group()
+    return {"workload": f"image-DiT B{B} H{H} S{S} D{D}", "kernels": res, "exchange_bytes_per_rank": exch,
+            "exchange_plan": exch_plan}
 
 
 def causal_flops(B, H, S, D):
@@ -636,43 +832,6 @@ def projection_paths(api, torch, flush, peaks, inputs, B, S, H, D, U):
         "three library GEMMs (Q, K, V) and the Q/K/V permute kernel (context only)")
     rec("context_unfused_output_projection_unpermute_plus_cublas", unfused_out, f_out,
         "unpermute kernel and library GEMM (context only)")
-    return res
-
-
-def breakdown(api, torch, dev, flush, peaks, inputs):
-    """HBM-bound kernels on tensors larger than L2 (video-DiT sizes), each rep
-    after an L2 flush: Ulysses permute / unpermute (degree 2, bf16) and the
-    8-way LSE merge of float32 partials."""
-    vcfg = inputs.CONFIGS["video"]
-    B, S, H, D = vcfg["B"], vcfg["S"], vcfg["H"], vcfg["D"]
-    hbm = float(peaks["hbm_gbs"])
-    n = B * S * H * D
-    x = torch.randn(n, device=dev).to(torch.bfloat16)
-    y = torch.empty_like(x)
-    stream = torch.cuda.current_stream()
-    res = {}
-
-    def timeit(fn):
-        return median_event_ms(fn, flush, stream)
-
-    ms = timeit(lambda: api.cpattn_ulysses_permute(x, B, S, H, D, 2, y=y, stream=stream))
-    gbs = 2 * n * 2 / (ms * 1e-3) / 1e9
-    res["ulysses_permute_video"] = {"ms": ms, "GB/s": gbs, "frac_hbm": gbs / hbm, "bytes": 4 * n}
-    ms = timeit(lambda: api.cpattn_ulysses_unpermute(y, B, S, H, D, 2, x=x, stream=stream))
-    gbs = 2 * n * 2 / (ms * 1e-3) / 1e9
-    res["ulysses_unpermute_video"] = {"ms": ms, "GB/s": gbs, "frac_hbm": gbs / hbm, "bytes": 4 * n}
-    del x, y
-    P = 8
-    po = torch.randn((P, B, S, H, D), device=dev, dtype=torch.float32)
-    pl = torch.randn((P, B, H, S), device=dev, dtype=torch.float32)
-    ob = torch.empty((B, S, H, D), device=dev, dtype=torch.bfloat16)
-    lo = torch.empty((B, H, S), device=dev, dtype=torch.float32)
-    ms = timeit(lambda: api.cpattn_lse_merge(po, pl, out_bf16=ob, lse_out=lo, want_f32=False, stream=stream))
-    mbytes = B * H * S * (P * (4 * D + 4) + 2 * D + 4)
-    gbs = mbytes / (ms * 1e-3) / 1e9
-    res["lse_merge_video_p8"] = {"ms": ms, "GB/s": gbs, "frac_hbm": gbs / hbm, "bytes": mbytes}
-    del po, pl, ob, lo
-    torch.cuda.empty_cache()
     return res
 
 
@@ -824,12 +983,12 @@ def run_sweep(args):
 
 
 def run_single_kernel(args):
-    """Profiling mode: `warmup + steps` launches of one kernel of the step on
-    the image-DiT workload (merge: 4 float32 partials of it), nothing else."""
+    """Profiling mode: `warmup + steps` launches of one kernel (or one flow) on
+    the workload `--workload` (merge: P float32 partials of it), nothing else."""
     import torch
     from context_attention_long_b200 import api, build, inputs
     build.build()
-    cfg, qb, kb, vb = inputs.config_inputs(WORKLOAD)
+    cfg, qb, kb, vb = inputs.config_inputs(args.workload)
     B, S, H, D = qb.shape
     P, U = cfg["ring_degree"], cfg["ulysses_degree"]
     dev = torch.device("cuda", 0)
@@ -853,6 +1012,12 @@ def run_single_kernel(args):
         fn = lambda: api.cpattn_ulysses_permute_qkv(qf, kf, vf, B, S, H, D, U, yq=yq, yk=yk, yv=yv)
     elif args.kernel == "permute":
         fn = lambda: api.cpattn_ulysses_permute(q.reshape(-1), B, S, H, D, U)
+    elif args.kernel == "unpermute":
+        x = torch.empty_like(q.reshape(-1))
+        fn = lambda: api.cpattn_ulysses_unpermute(q.reshape(-1), B, S, H, D, U, x=x)
+    elif args.kernel == "unified":
+        ws = torch.empty(api.cpattn_unified_workspace_bytes(B, H, S, D), dtype=torch.uint8, device=dev)
+        fn = lambda: api.cpattn_unified_attention(q, k, v, P, U, workspace=ws)
     elif args.kernel in ("qkv_projection", "output_projection"):
         Dm = H * D
         xb, wb, wob = inputs.make_projection_inputs(B, S, H, D, Dm, 4321)

@@ -27,6 +27,15 @@ def test_projection_flops_match_counted_multiply_adds():
     assert bench.projection_flops(B, S, H, D, Dm) == (2.0 * count_qkv, 2.0 * count_out)
 
 
-def test_aggregate_over_ranks_single_rank():
-    ms_per_step, per_s = bench.aggregate_over_ranks(10.0, 5, 1e12, 1)
-    assert ms_per_step == 2.0 and per_s == pytest.approx(5e12 / 10e-3)
+def test_max_over_ranks_single_rank_is_the_identity():
+    assert bench.max_over_ranks([10.0, 2.5], 1) == [10.0, 2.5]
+
+
+@pytest.mark.parametrize("S,world", [(32760, 2), (32760, 4), (32760, 8), (10007, 6), (9, 8)])
+def test_multi_gpu_shards_cover_the_sequence_once(S, world):
+    lens, ring_lens, subs = bench.multi_gpu_shards(S, world)
+    assert sum(lens) == S and len(lens) == world and max(lens) - min(lens) <= 1
+    # rank (i, j) = 2 i + j holds sub-shard j of ring chunk i: the same tokens
+    flat = [n for chunk in subs for n in chunk]
+    assert flat == lens
+    assert ring_lens == [sum(c) for c in subs] and sum(ring_lens) == S
