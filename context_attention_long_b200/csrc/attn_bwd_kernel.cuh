@@ -16,14 +16,22 @@
 // tiles (S and dP are computed in both).  A launch covers up to 8 problems
 // (the full tensors, or the head ranks' buffers of the Ulysses flow), each
 // with its own tensor maps, LSE strides and Delta slice.  CTA organisation of
-// each kernel (192 threads, one CTA per SM):
+// each kernel (320 threads, one CTA per SM):
 //   warp 0      TMA producer: the owned tiles once, the walked tiles through
 //               a 2-stage ring
 //   warp 1      TMEM allocator + single-thread MMA issuer (tcgen05.mma)
-//   warps 2-5   one row of the owned tile per thread (TMEM lane): P and dS in
-//               registers, bf16 results back into TMEM, the epilogue
+//   warps 2-9   two threads per row of the owned tile (TMEM lane), one per
+//               half of the walked tile's 128 columns (warps 2-5 the first
+//               half, 6-9 the second): P and dS in registers, bf16 results
+//               back into TMEM, the epilogue.  Two row warps share each
+//               sub-partition, so one's exponentials overlap the other's
+//               loads, stores and waits.
 // TMEM columns: S [0,128) (later P), dP [128,256) (later dS), then the
-// accumulators (dQ; or dV and dK).  The next tile's S is issued as soon as
+// accumulators (dQ; or dV and dK).  Half h of a row packs its bf16 results
+// into columns [64h, 64h + 32) of its region -- the start of the columns it
+// read itself, so the two halves never overwrite each other's inputs -- and
+// the MMAs read K block kk (16 keys or queries) at (kk / 4) * 64 + (kk % 4) * 8.
+// The next tile's S is issued as soon as
 // the row threads have read the current S (dQ kernel) or the current P has
 // been consumed (dK/dV kernel), so the tensor core works while the row
 // threads exponentiate.  Every wait is bounded as in the forward.
@@ -52,7 +60,12 @@ struct BwdSmem {
   static constexpr int kAllocBytes = kBytes + 1024;
 };
 
-constexpr int kBwdThreads = 192;
+constexpr int kBwdRowWarps = 8;
+constexpr int kBwdThreads = 64 + 32 * kBwdRowWarps;
+
+// TMEM column of the bf16 pairs of K-block kk (16 rows of the contraction)
+// inside a packed region (see the layout above).
+__device__ __forceinline__ uint32_t bwd_packed_col(int kk) { return static_cast<uint32_t>((kk >> 2) * 64 + (kk & 3) * 8); }
 constexpr uint32_t kBwdTmemCols = 512;
 
 // Delta[b, h, s] = sum_d dO[b, s, h, d] * O[b, s, h, d], one warp per
@@ -154,9 +167,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __gri
       mbar_init(sb + BAR_VE + 8 * s, 1);
     }
     mbar_init(sb + BAR_S, 1);
-    mbar_init(sb + BAR_SC, 4);
+    mbar_init(sb + BAR_SC, kBwdRowWarps);
     mbar_init(sb + BAR_DP, 1);
-    mbar_init(sb + BAR_DS, 4);
+    mbar_init(sb + BAR_DS, kBwdRowWarps);
     mbar_init(sb + BAR_DQ, 1);
     mbar_init(sb + BAR_TAIL, 1);
     st_shared_volatile(sb + ABORT, 0u);
@@ -232,7 +245,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __gri
         const uint64_t b0 = opaque_u64(dKmn + ((st * L::kTileBytes) >> 4));
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + 256, tmem + 128 + kk * 8, b0 + ((kk * 2048) >> 4), IDESC_DQ, (acc || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + 256, tmem + 128 + bwd_packed_col(kk), b0 + ((kk * 2048) >> 4), IDESC_DQ,
+                 (acc || kk > 0) ? 1u : 0u);
       };
       bool ok = n > 0 && mbar_wait_spin(sb + BAR_QD, 0, abort_flag, tmo, SITE_MMA);
       if (ok) ok = mbar_wait_spin(sb + BAR_KF, 0, abort_flag, tmo, SITE_MMA);
@@ -276,13 +290,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __gri
     }
   } else {
     // ------------------------------------------------------------ row threads
-    const int quad = warp & 3;
+    const int quad = warp & 3;                 // TMEM lane group of this warp
+    const int half = (warp - 2) >> 2;          // which 64 keys of the walked tile
+    const int col0 = half * 64;
     const int row = quad * 32 + lane;
     const int q_pos = q0 + row;
     const bool row_valid = row < q_rows;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t tS = tmem + lane_base;
-    const uint32_t tDP = tmem + lane_base + 128;
+    const uint32_t tS = tmem + lane_base + col0;
+    const uint32_t tDP = tmem + lane_base + 128 + col0;
     const uint32_t tDQ = tmem + lane_base + 256;
     const float c = p.scale_log2;
     const long long li = static_cast<long long>(U.b) * PB.lse_b + static_cast<long long>(U.h + PB.lse_h0) * PB.lse_h + q_pos;
@@ -292,22 +308,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __gri
     bool ok = true;
     for (int j = 0; ok && j < n; ++j) {
       // keys of tile j this row sees: all valid keys, cut at the row's own
-      // position under the causal mask; none for rows past the sequence
+      // position under the causal mask; none for rows past the sequence;
+      // counted from this thread's first key
       int kvalid = min(128, kv_len - j * 128);
       if (p.causal) kvalid = min(kvalid, q_pos - j * 128 + 1);
       if (!row_valid) kvalid = 0;
+      kvalid -= col0;
       bool w = mbar_wait(sb + BAR_S, j & 1, abort_flag, tmo, SITE_SOFTMAX);
       if (__any_sync(0xffffffffu, !w)) { ok = false; break; }
       __syncwarp();
       tc_fence_after();
-      uint32_t s[128];
-      tmem_ld128_wait(tS, s);
+      uint32_t s[64];
+      tmem_ld64_wait(tS, s);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(sb + BAR_SC);
       // P = 2^(S*c - lse2), kept in fp32 over the scores
 #pragma unroll
-      for (int k = 0; k < 128; ++k)
+      for (int k = 0; k < 64; ++k)
         s[k] = __float_as_uint(k < kvalid ? ex2_approx(__uint_as_float(s[k]) * c - lse2) : 0.f);
       w = mbar_wait(sb + BAR_DP, j & 1, abort_flag, tmo, SITE_SOFTMAX);
       if (__any_sync(0xffffffffu, !w)) { ok = false; break; }
@@ -315,7 +333,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __gri
       tc_fence_after();
       // dS = P * (dP - delta), bf16 pairs over the dP columns already read
 #pragma unroll
-      for (int c0 = 0; c0 < 128; c0 += 32) {
+      for (int c0 = 0; c0 < 64; c0 += 32) {
         uint32_t dp[32];
         tmem_ld32_wait(tDP + c0, dp);
         uint32_t pk[16];
@@ -339,14 +357,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __gri
       tc_fence_after();
     }
     if (ok) {
+      // each half of the row writes half of dQ's D columns
       const float scale = p.scale;
+      const int d0 = half * (D / 2);
       __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(PB.dq) +
-                           ((static_cast<long long>(U.b) * p.S + q_pos) * PB.H + U.h) * D;
+                           ((static_cast<long long>(U.b) * p.S + q_pos) * PB.H + U.h) * D + d0;
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
+      for (int c0 = 0; c0 < D / 2; c0 += 32) {
         uint32_t o[32];
         if (n > 0) {
-          tmem_ld32_wait(tDQ + c0, o);
+          tmem_ld32_wait(tDQ + d0 + c0, o);
         } else {
 #pragma unroll
           for (int k = 0; k < 32; ++k) o[k] = 0u;
@@ -416,12 +436,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __gr
       mbar_init(sb + BAR_OE + 8 * s, 1);
     }
     mbar_init(sb + BAR_S, 1);
-    mbar_init(sb + BAR_P, 4);
+    mbar_init(sb + BAR_P, kBwdRowWarps);
     mbar_init(sb + BAR_DP, 1);
-    mbar_init(sb + BAR_DS, 4);
+    mbar_init(sb + BAR_DS, kBwdRowWarps);
     mbar_init(sb + BAR_ACC, 1);
     mbar_init(sb + BAR_TAIL, 1);
-    mbar_init(sb + BAR_VEC, 4);
+    mbar_init(sb + BAR_VEC, kBwdRowWarps);
     st_shared_volatile(sb + ABORT, 0u);
     fence_mbar_init();
   }
@@ -489,7 +509,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __gr
       auto issue_acc = [&](uint32_t d, uint32_t a_tmem, uint64_t b0, bool acc) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(d, a_tmem + kk * 8, b0 + ((kk * 2048) >> 4), IDESC_ACC, (acc || kk > 0) ? 1u : 0u);
+          mma_ts(d, a_tmem + bwd_packed_col(kk), b0 + ((kk * 2048) >> 4), IDESC_ACC, (acc || kk > 0) ? 1u : 0u);
       };
       auto stage_off = [&](int st) { return static_cast<uint64_t>((st * L::kTileBytes) >> 4); };
       bool ok = n > 0 && mbar_wait_spin(sb + BAR_KV, 0, abort_flag, tmo, SITE_MMA);
@@ -537,40 +557,45 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __gr
       mbar_wait(sb + BAR_TAIL, 0, 0u, tmo, SITE_TAIL);
     }
   } else {
-    // ------------------------------------------------------------ row threads (one key each)
-    const int quad = warp & 3;
+    // ------------------------------------------------------------ row threads (two per key)
+    const int quad = warp & 3;                 // TMEM lane group of this warp
+    const int half = (warp - 2) >> 2;          // which 64 queries of the walked tile
+    const int col0 = half * 64;
     const int row = quad * 32 + lane;
-    const int tid = threadIdx.x - 64;            // 0..127 across the four row warps
     const int k_pos = k0 + row;
     const bool row_valid = row < k_rows;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t tS = tmem + lane_base;
-    const uint32_t tDP = tmem + lane_base + 128;
+    const uint32_t tS = tmem + lane_base + col0;
+    const uint32_t tDP = tmem + lane_base + 128 + col0;
     const uint32_t tDV = tmem + lane_base + 256;
     const uint32_t tDK = tmem + lane_base + 256 + D;
     const float c = p.scale_log2;
     const long long lbase = static_cast<long long>(U.b) * PB.lse_b + static_cast<long long>(U.h + PB.lse_h0) * PB.lse_h;
     const long long dbase = (static_cast<long long>(U.b) * PB.H + U.h) * p.S;
     bool ok = true;
-    // Each Q tile's log2-domain LSE and Delta, one value per row thread
-    // (queries past the sequence get LSE = +inf, i.e. P = 0), are loaded one
-    // tile ahead so that their global-memory latency hides behind a tile.
+    // Each Q tile's log2-domain LSE and Delta are published in shared memory
+    // by the first-half threads, one value per thread (queries past the
+    // sequence get LSE = +inf, i.e. P = 0), loaded one tile ahead so that
+    // their global-memory latency hides behind a tile.
     auto load_vec = [&](int i, float &l2, float &dl) {
-      const int q = (qt0 + i) * 128 + tid;
+      const int q = (qt0 + i) * 128 + row;
       l2 = q < p.S ? PB.lse[lbase + q] * 1.4426950408889634f : INFINITY;
       dl = q < p.S ? PB.delta[dbase + q] : 0.f;
     };
     float nl2 = 0.f, ndl = 0.f;
-    if (n > 0) load_vec(0, nl2, ndl);
+    if (n > 0 && half == 0) load_vec(0, nl2, ndl);
     for (int i = 0; ok && i < n; ++i) {
       const int q0 = (qt0 + i) * 128;
       const uint32_t vec = sb + L::kOffVec + (i & 1) * 1024;
-      st_shared_f32(vec + 4 * tid, nl2);
-      st_shared_f32(vec + 512 + 4 * tid, ndl);
-      if (i + 1 < n) load_vec(i + 1, nl2, ndl);
+      if (half == 0) {
+        st_shared_f32(vec + 4 * row, nl2);
+        st_shared_f32(vec + 512 + 4 * row, ndl);
+        if (i + 1 < n) load_vec(i + 1, nl2, ndl);
+      }
       // Every row warp has finished reading the previous use of this buffer
-      // (tile i-2) before it writes tile i's values, and the bounded barrier
-      // below publishes them; no unbounded named barrier.
+      // (tile i-2) before it is written for tile i -- its arrival for tile
+      // i-1 came after those reads -- and the bounded barrier below
+      // publishes the values; no unbounded named barrier.
       __syncwarp();
       if (lane == 0) mbar_arrive(sb + BAR_VEC);
       bool w = mbar_wait(sb + BAR_VEC, i & 1, abort_flag, tmo, SITE_SOFTMAX);
@@ -579,17 +604,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __gr
       if (__any_sync(0xffffffffu, !w)) { ok = false; break; }
       __syncwarp();
       tc_fence_after();
-      uint32_t s[128];
-      tmem_ld128_wait(tS, s);
+      uint32_t s[64];
+      tmem_ld64_wait(tS, s);
       // P^T[k][q] = 2^(S^T*c - lse2[q]) for the queries that see key k.  The
       // per-query values are read as float4 through a plain shared-memory
       // pointer (the barrier waits above are compiler fences), so the loads
       // schedule freely around the exponentials.
-      const float4 *lse4 = reinterpret_cast<const float4 *>(smem_raw + (vec - smem_u32(smem_raw)));
+      const float4 *lse4 = reinterpret_cast<const float4 *>(smem_raw + (vec - smem_u32(smem_raw))) + (col0 >> 2);
       const float4 *del4 = lse4 + 32;
-      const int qlim = p.causal ? k_pos - q0 : 0;   // queries q < qlim do not see this key
+      const int qlim = (p.causal ? k_pos - q0 : 0) - col0;   // queries q < qlim do not see this key
 #pragma unroll
-      for (int q4 = 0; q4 < 32; ++q4) {
+      for (int q4 = 0; q4 < 16; ++q4) {
         const float4 l = lse4[q4];
         const float lv[4] = {l.x, l.y, l.z, l.w};
 #pragma unroll
@@ -600,7 +625,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __gr
         }
       }
 #pragma unroll
-      for (int c0 = 0; c0 < 128; c0 += 32) {
+      for (int c0 = 0; c0 < 64; c0 += 32) {
         uint32_t pk[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) pk[k] = pack_bf16x2(__uint_as_float(s[c0 + 2 * k]), __uint_as_float(s[c0 + 2 * k + 1]));
@@ -616,7 +641,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __gr
       tc_fence_after();
       // dS^T = P^T * (dP^T - delta[q]), bf16 pairs over the dP^T columns read
 #pragma unroll
-      for (int c0 = 0; c0 < 128; c0 += 32) {
+      for (int c0 = 0; c0 < 64; c0 += 32) {
         uint32_t dp[32];
         tmem_ld32_wait(tDP + c0, dp);
         uint32_t pk[16];
@@ -643,13 +668,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __gr
       tc_fence_after();
     }
     if (ok) {
-      const long long roff = ((static_cast<long long>(U.b) * p.S + k_pos) * PB.H + U.h) * D;
+      // each half of the row writes half of the D columns of dV and of dK
+      const int d0 = half * (D / 2);
+      const long long roff = ((static_cast<long long>(U.b) * p.S + k_pos) * PB.H + U.h) * D + d0;
       for (int which = 0; which < 2; ++which) {   // 0: dV, 1: dK (times the softmax scale)
         const float mul = which == 0 ? 1.0f : p.scale;
         __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(which == 0 ? PB.dv : PB.dk) + roff;
-        const uint32_t tsrc = which == 0 ? tDV : tDK;
+        const uint32_t tsrc = (which == 0 ? tDV : tDK) + d0;
 #pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) {
+        for (int c0 = 0; c0 < D / 2; c0 += 32) {
           uint32_t o[32];
           if (n > 0) {
             tmem_ld32_wait(tsrc + c0, o);
