@@ -186,6 +186,26 @@ __device__ __forceinline__ void kv_tile(const AttnParams &p, const AttnSeg &SG, 
   valid = 0;
 }
 
+// Element offset of output row (batch b, sequence position s, Q row grow)
+// of head h, by the problem's output map (see AttnProblem).
+template <int D>
+__device__ __forceinline__ size_t out_row_elems(const AttnProblem &PB, int b, int s, int grow, int h) {
+  if (PB.out_mode == 0) return (static_cast<size_t>(grow) * PB.H + h) * D;
+  long long row;
+  if (PB.out_mode == 1) {
+    int lo = 0, hi = PB.out_nseq - 1;   // the sequence rank holding s (empty ranks skipped)
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (PB.out_seq_off[mid] <= s) lo = mid; else hi = mid - 1;
+    }
+    const int off = PB.out_seq_off[lo], len = PB.out_seq_off[lo + 1] - off;
+    row = static_cast<long long>(PB.out_B) * off + static_cast<long long>(b) * len + (s - off);
+  } else {
+    row = static_cast<long long>(b) * PB.out_S + s;
+  }
+  return (static_cast<size_t>(row) * PB.out_H + PB.out_h0 + h) * D;
+}
+
 template <int D, bool OUT_F32>
 __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnParams p) {
   using L = AttnSmem<D>;
@@ -606,8 +626,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
           const float lt = l * a0 + l1 * a1;
           const bool row_valid = row < rows_left;
           const int grow = q_row0 + row;
-          const size_t row_elems = (static_cast<size_t>(grow) * PB.H + h) * D;
           const int sq = SG.s0 + pair * (kQTilesPerCTA * kQTile) + row;
+          const size_t row_elems = out_row_elems<D>(PB, G.b, sq, grow, h);
           const long long lse_idx = static_cast<long long>(G.b) * PB.lse_b +
                                     static_cast<long long>(h + PB.lse_h0) * PB.lse_h + (sq - PB.lse_pos0);
           // This unit's own state (slots 0 and 1 merged), in log2 units, and
@@ -670,8 +690,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       const int valid_rows = qt == 0 ? min(kQTile, rows_left) : rows_left - kQTile;
       const bool row_valid = row < valid_rows;
       const int grow = q_row0 + qt * kQTile + row;
-      const size_t row_elems = (static_cast<size_t>(grow) * PB.H + h) * D;
       const int sq = SG.s0 + pair * (kQTilesPerCTA * kQTile) + qt * kQTile + row;
+      const size_t row_elems = out_row_elems<D>(PB, G.b, sq, grow, h);
       const long long lse_idx = static_cast<long long>(G.b) * PB.lse_b +
                                 static_cast<long long>(h + PB.lse_h0) * PB.lse_h + (sq - PB.lse_pos0);
       // out = O * w_self + prev * w_prev: w_self = 1/l alone; with a previous

@@ -336,6 +336,9 @@ struct ProblemSpec {
   long long rows_kv = 0;       // rows of K and V when they are a separate buffer
   const float *prev = nullptr; // previous partial state merged into the output (see AttnProblem)
   int lse_pos0 = 0;            // sequence position of LSE column 0
+  int out_mode = 0;            // output map (see AttnProblem)
+  int out_H = 0, out_h0 = 0, out_B = 0, out_S = 0;
+  std::vector<int> out_seq_off;   // out_mode 1: sequence offsets of the ranks (degree + 1 entries)
 };
 struct SegSpec {
   int row0, nrows, s0;
@@ -424,6 +427,14 @@ static int run_attention(const std::vector<ProblemSpec> &probs, const std::vecto
     ap.lse_h0 = ps.lse_h0;
     ap.lse_pos0 = ps.lse_pos0;
     ap.H = ps.H;
+    ap.out_mode = ps.out_mode;
+    ap.out_H = ps.out_H;
+    ap.out_h0 = ps.out_h0;
+    ap.out_B = ps.out_B;
+    ap.out_S = ps.out_S;
+    ap.out_nseq = static_cast<int>(ps.out_seq_off.size()) - 1;
+    if (ap.out_nseq > kMaxRanks) return CPATTN_ERR_DEGREE;
+    for (size_t r = 0; r < ps.out_seq_off.size(); ++r) ap.out_seq_off[r] = ps.out_seq_off[r];
   }
   const float scale_log2 = static_cast<float>((1.0 / std::sqrt(static_cast<double>(D))) * 1.4426950408889634);
 
@@ -855,7 +866,7 @@ static void head_sharded_problems(std::vector<ProblemSpec> &probs, std::vector<i
     ps.q = static_cast<const char *>(yq) + off_bytes;
     ps.k = static_cast<const char *>(yk) + off_bytes;
     ps.v = static_cast<const char *>(yv) + off_bytes;
-    ps.out = static_cast<char *>(yo) + off_bytes;
+    ps.out = yo != nullptr ? static_cast<char *>(yo) + off_bytes : nullptr;
     ps.lse = lse;
     ps.lse_b = static_cast<long long>(H) * S;
     ps.lse_h = S;
@@ -867,12 +878,29 @@ static void head_sharded_problems(std::vector<ProblemSpec> &probs, std::vector<i
   }
 }
 
+// seq_out != nullptr: the output goes to the sequence-side rank buffers
+// (offsets seq_off) instead of the head-side yo (the Ulysses flow's second
+// all-to-all, fused into the epilogue).
 static int head_sharded_attention_impl(const void *yq, const void *yk, const void *yv, void *yo, float *lse, int B,
                                        int H, int S, int D, const std::vector<int> &heads, bool causal,
-                                       cudaStream_t stream) {
+                                       cudaStream_t stream, void *seq_out = nullptr,
+                                       const std::vector<int> &seq_off = {}) {
   std::vector<ProblemSpec> probs;
   std::vector<int> prob_rank;
   head_sharded_problems(probs, prob_rank, yq, yk, yv, yo, lse, B, H, S, D, heads);
+  if (seq_out != nullptr) {
+    const std::vector<int> ho = prefix(heads);
+    for (size_t pi = 0; pi < probs.size(); ++pi) {
+      ProblemSpec &ps = probs[pi];
+      ps.out = seq_out;
+      ps.out_mode = 1;
+      ps.out_H = H;
+      ps.out_h0 = ho[prob_rank[pi]];
+      ps.out_B = B;
+      ps.out_S = S;
+      ps.out_seq_off = seq_off;
+    }
+  }
   std::vector<GroupSpec> groups;
   for (size_t pi = 0; pi < probs.size(); ++pi) {
     for (int b = 0; b < B; ++b) {
@@ -980,7 +1008,7 @@ static int ulysses_common(const void *q, const void *k, const void *v, void *out
   if (st != CPATTN_OK) return st;
   const size_t tensor_bytes = static_cast<size_t>(B) * S * H * D * 2;
   char *ws = static_cast<char *>(workspace);
-  void *yq = ws, *yk = ws + tensor_bytes, *yv = ws + 2 * tensor_bytes, *yo = ws + 3 * tensor_bytes;
+  void *yq = ws, *yk = ws + tensor_bytes, *yv = ws + 2 * tensor_bytes;
   std::vector<int> heads;
   resolve_splits(H, degree, head_splits, heads);
   // first all-to-all: Q, K, V to the head-sharded layout, one launch
@@ -989,16 +1017,12 @@ static int ulysses_common(const void *q, const void *k, const void *v, void *out
     set_qkv(pp, q, k, v, yq, yk, yv);
     if (launch_permute(pp, stream) != cudaSuccess) return CPATTN_ERR_CUDA;
   }
-  // local attention of every head rank over all S tokens of its heads
-  st = head_sharded_attention_impl(yq, yk, yv, yo, lse, B, H, S, D, heads, causal, stream);
-  if (st != CPATTN_OK) return st;
-  // second all-to-all: the output back to the sequence-sharded layout
-  PermuteParams po = pq;
-  po.src[0] = static_cast<const unsigned char *>(yo);
-  po.dst[0] = static_cast<unsigned char *>(out);
-  po.n_tensors = 1;
-  po.direction = 1;
-  return launch_permute(po, stream) == cudaSuccess ? CPATTN_OK : CPATTN_ERR_CUDA;
+  // local attention of every head rank over all S tokens of its heads; the
+  // second all-to-all is fused into its epilogue, which stores each output
+  // row straight into the sequence-sharded rank buffers
+  std::vector<int> seq;
+  resolve_splits(S, degree, seq_splits, seq);
+  return head_sharded_attention_impl(yq, yk, yv, nullptr, lse, B, H, S, D, heads, causal, stream, out, prefix(seq));
 }
 
 int cpattn_ulysses_attention(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H, int S,
@@ -1038,7 +1062,7 @@ static int unified_common(const void *q, const void *k, const void *v, void *out
   const std::vector<int> off = prefix(lens), ho = prefix(heads);
   const size_t tensor_bytes = static_cast<size_t>(B) * S * H * D * 2;
   char *ws = static_cast<char *>(workspace);
-  void *yq = ws, *yk = ws + tensor_bytes, *yv = ws + 2 * tensor_bytes, *yo = ws + 3 * tensor_bytes;
+  void *yq = ws, *yk = ws + tensor_bytes, *yv = ws + 2 * tensor_bytes;
 
   // Permutation within every ring group (ring chunk i): full BSHD rows of the
   // chunk -> head group u buffer laid out [i][B, len_i, H_u, D].
@@ -1063,19 +1087,23 @@ static int unified_common(const void *q, const void *k, const void *v, void *out
   // Ring attention per head group over the chunks (rows B*off_i + b*len_i).
   std::vector<ProblemSpec> probs;
   std::vector<int> prob_rank;
-  head_sharded_problems(probs, prob_rank, yq, yk, yv, yo, lse, B, H, S, D, heads);
+  head_sharded_problems(probs, prob_rank, yq, yk, yv, nullptr, lse, B, H, S, D, heads);
+  // The inverse permutation is fused into the epilogue: each output row goes
+  // straight to the full (B, S, H, D) tensor at its head's global index.
+  for (size_t pi = 0; pi < probs.size(); ++pi) {
+    ProblemSpec &ps = probs[pi];
+    ps.out = out;
+    ps.out_mode = 2;
+    ps.out_H = H;
+    ps.out_h0 = ho[prob_rank[pi]];
+    ps.out_B = B;
+    ps.out_S = S;
+  }
   std::vector<GroupSpec> groups;
   for (size_t pi = 0; pi < probs.size(); ++pi)
     ring_groups(groups, static_cast<int>(pi), B, lens, off, -1, causal,
                 [&](int b, int c) { return B * off[c] + b * lens[c]; });
-  st = run_attention(probs, groups, D, false, causal, stream);
-  if (st != CPATTN_OK) return st;
-  PermuteParams p2 = pp;
-  p2.src[0] = static_cast<const unsigned char *>(yo);
-  p2.dst[0] = static_cast<unsigned char *>(out);
-  p2.n_tensors = 1;
-  p2.direction = 1;
-  return launch_permute(p2, stream) == cudaSuccess ? CPATTN_OK : CPATTN_ERR_CUDA;
+  return run_attention(probs, groups, D, false, causal, stream);
 }
 
 int cpattn_unified_attention(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H, int S,

@@ -28,6 +28,7 @@ namespace cpattn {
 // One CTA processes one unit = (group, head, segment, pair of 128-row Q tiles).
 
 constexpr int kMaxProblems = 8;
+constexpr int kMaxRanks = 64;   // sequence / head ranks of a permutation or an output map
 constexpr int kMaxGroups = 64;
 constexpr int kMaxSegs = 128;
 constexpr int kMaxKV = 512;
@@ -47,6 +48,17 @@ struct alignas(64) AttnProblem {
   int lse_h0;
   int lse_pos0;                   // sequence position of LSE column 0
   int H;
+  // Where a row of out goes (batch b, sequence position s, head h):
+  //   out_mode 0: the row of Q (out has Q's layout);
+  //   out_mode 1: the sequence-side rank buffers (B, len_r, out_H, D) of the
+  //               Ulysses exchange, row out_B*off_r + b*len_r + (s - off_r),
+  //               head out_h0 + h (the second all-to-all, fused);
+  //   out_mode 2: a full (B, out_S, out_H, D) tensor, row b*out_S + s, head
+  //               out_h0 + h.
+  int out_mode;
+  int out_H, out_h0, out_B, out_S;
+  int out_nseq;
+  int out_seq_off[kMaxRanks + 1];
 };
 
 struct AttnGroup {
@@ -140,7 +152,6 @@ cudaError_t launch_lse_merge(const MergeParams &p, cudaStream_t stream);
 //   head side row in buffer u (groups = outer sequence ranges, one group for
 //   plain Ulysses):     B*goff_i + b*glen_i + (s - goff_i)
 //   head buffer u starts at element B*S*hoff_u*D.
-constexpr int kMaxRanks = 64;
 constexpr int kMaxHeads = 1024;
 
 constexpr int kMaxPermuteTensors = 3;   // Q, K and V move in one launch

@@ -269,8 +269,10 @@ size_t cpattn_ulysses_workspace_bytes(int B, int H, int S, int D);
 
 /*
  * Ulysses attention ([CP] "Ulysses Attention"; [USP] section 4): permute Q, K,
- * V to the head-sharded layout, local attention per head rank, unpermute the
- * output.  q, k, v, out are sequence-side rank buffers as `x` in
+ * V to the head-sharded layout (one launch), then local attention per head
+ * rank whose epilogue stores every output row straight into the
+ * sequence-sharded layout -- the second all-to-all, fused into the attention
+ * kernel (one launch).  q, k, v, out are sequence-side rank buffers as `x` in
  * cpattn_ulysses_permute; lse is [B, H, S] (global head and token) or NULL.
  * workspace: device, >= cpattn_ulysses_workspace_bytes, 16-byte aligned,
  * caller-owned scratch (contents undefined after the call).
@@ -294,9 +296,10 @@ size_t cpattn_unified_workspace_bytes(int B, int H, int S, int D);
  * Ring chunks are the outer split of the sequence (ring_lens, or equal);
  * inside ring chunk i the ulysses_degree ranks of that Ulysses group hold
  * sub-shards of it; heads are split by head_splits (or equally).  Steps: per
- * ring group, Ulysses permute of its chunk to head groups; per head group,
- * ring attention over the chunks with the LSE merge; per ring group, the
- * inverse permute of the output.
+ * ring group, Ulysses permute of its chunk to head groups (one launch for all
+ * groups); per head group, ring attention over the chunks with the LSE merge,
+ * whose epilogue stores the output at its token and global head in `out` --
+ * the inverse permute, fused (one launch).
  *
  *   q, k, v, out  full [B, S, H, D] bf16.  lse [B, H, S] or NULL.
  *   ring_lens     host int[ring_degree] or NULL (equal split).
