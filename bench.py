@@ -625,6 +625,43 @@ def run_multi_gpu(args, world, rank, dev):
     peaks, peaks_kind = load_peaks()
     peak_tf = float(peaks["bf16_tflops"])
     rank_ring_flops = attn_flops / world
+
+    # The link as the exchanges use it: one ring hop of this rank's K and V
+    # shard (send to the next rank, receive from the previous), timed on the
+    # device, max over ranks; it feeds the exchange-selection model.
+    hop_bytes = 2 * B * (b - a) * H * D * 2
+    nxt, prv = (rank + 1) % world, (rank - 1) % world
+    kr, vr = torch.empty_like(k), torch.empty_like(v)
+
+    def hop():
+        ops = [dist.P2POp(dist.isend, k.view(torch.uint8).reshape(-1), nxt),
+               dist.P2POp(dist.isend, v.view(torch.uint8).reshape(-1), nxt),
+               dist.P2POp(dist.irecv, kr.view(torch.uint8).reshape(-1), prv),
+               dist.P2POp(dist.irecv, vr.view(torch.uint8).reshape(-1), prv)]
+        for w in dist.batch_isend_irecv(ops):
+            w.wait()
+
+    for _ in range(3):
+        hop()
+    dist.barrier()
+    h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_hops = 10
+    h0.record(stream)
+    for _ in range(n_hops):
+        hop()
+    h1.record(stream)
+    torch.cuda.synchronize()
+    hop_ms = max_over_ranks([h0.elapsed_time(h1) / n_hops], world, dist, dev)[0]
+    link_gbs = hop_bytes / (hop_ms * 1e-3) / 1e9
+    rank_tflops = rank_ring_flops / (ring_ms * 1e-3) / 1e12
+    exch_plan = {"inputs": {"link_gbs": round(link_gbs, 1), "link_kind": "measured: one ring hop of a K/V shard",
+                            "attn_tflops": round(rank_tflops, 1), "hbm_gbs": float(peaks["hbm_gbs"])}}
+    for causal in (False, True):
+        pl = api.cpattn_plan_exchange(B, H, S, D, world, link_gbs, rank_tflops, float(peaks["hbm_gbs"]),
+                                      causal=causal)
+        exch_plan["causal" if causal else "non_causal"] = {
+            "best": pl["best"], "us": {m: (None if pl[m]["seconds"] is None else round(pl[m]["seconds"] * 1e6, 1))
+                                       for m in ("ring", "ulysses", "kv_gather")}}
     st, code = api.cpattn_device_status()
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -639,7 +676,7 @@ def run_multi_gpu(args, world, rank, dev):
         "e2e": {"value": step_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": 3 * B * S * H * D * 2, "d2h_bytes_per_step": 2 * B * S * H * D * 2,
                 "note": "every rank uploads its Q/K/V shard and downloads both outputs; summed over ranks"},
-        "device_status": code,
+        "device_status": code, "exchange_plan": exch_plan,
     }
     if rank == 0:
         print(json.dumps(line))

@@ -1,5 +1,5 @@
 """The multi-GPU exchanges (context_attention_long_b200.exchange) on CPU ranks:
-2 and 4 gloo processes run ring (point-to-point and all-gather rotation),
+2, 3 and 4 gloo processes run ring (point-to-point and all-gather rotation),
 Ulysses, kv_gather and unified attention on their shards of one seeded
 sequence, with the oracle-backed kernel stand-in (tests/exchange_standin.py)
 for the local compute, and every rank checks its rows against the oracle's
@@ -95,7 +95,12 @@ def _cases(world, rank):
         o, l = exchange.kv_gather_attention(q, k, v, None, lens, kernels=K)
         _check(o, l, ref_o[:, a:b], ref_l[:, :, a:b], f"kv_gather {lens}")
 
-    if world == 2:
+    if world == 3:
+        out += [("ring anything", lambda: ring_case(1, 2, 64, [100, 37, 64], False)),
+                ("ring causal", lambda: ring_case(2, 2, 128, [50, 50, 50], True)),
+                ("ulysses anything", lambda: ulysses_case(1, 4, 64, [31, 64, 40], [2, 1, 1], False)),
+                ("kv_gather", lambda: kv_gather_case(1, 3, 64, [10, 70, 0]))]
+    elif world == 2:
         out += [("ring even", lambda: ring_case(2, 3, 64, [96, 96], False)),
                 ("ring uneven causal", lambda: ring_case(1, 2, 128, [130, 61], True)),
                 ("ulysses even", lambda: ulysses_case(2, 4, 64, [80, 80], [2, 2], False)),
@@ -153,7 +158,7 @@ def _worker(rank, world, port, q):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 4])
+@pytest.mark.parametrize("world", [2, 3, 4])
 def test_exchanges_on_gloo_ranks_match_the_oracle(world):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
