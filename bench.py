@@ -987,7 +987,8 @@ def run_sweep(args):
             heads = inputs.front_loaded_splits(H, U) if name == "anything" else None
             ws = torch.empty(api.cpattn_ulysses_workspace_bytes(B, H, S, D), dtype=torch.uint8, device=dev)
             qf, kf, vf = q.reshape(-1), k.reshape(-1), v.reshape(-1)
-            paths.append((f"Ulysses {U}" + (" (Anything)" if seq else "") + " flow: Q/K/V permute + attention + unpermute",
+            paths.append((f"Ulysses {U}" + (" (Anything)" if seq else "") +
+                          " flow: Q/K/V permute + attention (the unpermute fused in its epilogue)",
                           lambda: api.cpattn_ulysses_attention(qf, kf, vf, B, S, H, D, U, seq, heads, workspace=ws)))
             paths.append((f"causal Ulysses {U}" + (" (Anything)" if seq else "") + " flow",
                           lambda: api.cpattn_causal_ulysses_attention(qf, kf, vf, B, S, H, D, U, seq, heads,
