@@ -18,7 +18,7 @@
 // with its own tensor maps, LSE strides and Delta slice.  CTA organisation of
 // each kernel (320 threads, one CTA per SM):
 //   warp 0      TMA producer: the owned tiles once, the walked tiles through
-//               a 2-stage ring
+//               rings of 3 stages (K or Q) and 2 stages (V or dO)
 //   warp 1      TMEM allocator + single-thread MMA issuer (tcgen05.mma)
 //   warps 2-9   two threads per row of the owned tile (TMEM lane), one per
 //               half of the walked tile's 128 columns (warps 2-5 the first
@@ -27,14 +27,16 @@
 //               sub-partition, so one's exponentials overlap the other's
 //               loads, stores and waits.
 // TMEM columns: S [0,128) (later P), dP [128,256) (later dS), then the
-// accumulators (dQ; or dV and dK).  Half h of a row packs its bf16 results
+// accumulators (dQ; or dV and dK); the dQ kernel keeps a second dP buffer in
+// [384,512), so dP(j+1) is computed while dS(j) still waits for the dQ MMA.
+// Half h of a row packs its bf16 results
 // into columns [64h, 64h + 32) of its region -- the start of the columns it
 // read itself, so the two halves never overwrite each other's inputs -- and
 // the MMAs read K block kk (16 keys or queries) at (kk / 4) * 64 + (kk % 4) * 8.
-// The next tile's S is issued as soon as
-// the row threads have read the current S (dQ kernel) or the current P has
-// been consumed (dK/dV kernel), so the tensor core works while the row
-// threads exponentiate.  Every wait is bounded as in the forward.
+// The next tile's S (and, in the dQ kernel, dP) is issued as soon as the row
+// threads have read the current S (dQ kernel) or the current P has been
+// consumed (dK/dV kernel), so the tensor core works while the row threads
+// exponentiate.  Every wait is bounded as in the forward.
 #pragma once
 
 #include "cpattn_internal.h"
@@ -47,18 +49,29 @@ struct BwdSmem {
   static constexpr int kHalves = D / 64;
   static constexpr int kBoxBytes = 128 * 128;          // [128 rows][64 bf16], 128B-swizzled
   static constexpr int kTileBytes = kHalves * kBoxBytes;
-  static constexpr int kStages = 2;
+  // The walked tile a step needs first (K in the dQ kernel, Q in the dK/dV
+  // kernel) is also the one released last (after the step's final MMA), so
+  // it gets three stages: its load starts two steps ahead and its TMA latency
+  // stays off the pipeline.  The other walked tile (V, dO) is released
+  // mid-step, after its last MMA, and two stages are enough.
+  static constexpr int kStagesC = 3;
+  static constexpr int kStagesE = 2;
   static constexpr int kOffA = 0;                       // owned tile 0: Q (dq) or K (dkv)
   static constexpr int kOffB = kOffA + kTileBytes;      // owned tile 1: dO (dq) or V (dkv)
   static constexpr int kOffC = kOffB + kTileBytes;      // walked tile 0 per stage: K (dq) or Q (dkv)
-  static constexpr int kOffE = kOffC + kStages * kTileBytes;   // walked tile 1 per stage: V or dO
-  static constexpr int kOffVec = kOffE + kStages * kTileBytes; // dkv: [stage][lse2 128 | delta 128] floats
-  static constexpr int kOffBar = kOffVec + kStages * 2 * 128 * 4;
-  static constexpr int kNumBars = 16;
+  static constexpr int kOffE = kOffC + kStagesC * kTileBytes;   // walked tile 1 per stage: V or dO
+  static constexpr int kOffVec = kOffE + kStagesE * kTileBytes; // dkv: [2][lse2 128 | delta 128] floats
+  static constexpr int kOffBar = kOffVec + 2 * 2 * 128 * 4;
+  static constexpr int kNumBars = 24;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffMisc + 16;
-  static constexpr int kAllocBytes = kBytes + 1024;
+  // No alignment slack: seven D = 128 tiles leave too little room for one.
+  // The dynamic window starts 1024-aligned (declared so, and checked at
+  // kernel entry: a misaligned window records SITE_LAYOUT and the kernel
+  // returns without touching memory).
+  static constexpr int kAllocBytes = kBytes;
 };
+static_assert(BwdSmem<128>::kAllocBytes <= 232448, "backward shared memory exceeds the per-CTA limit");
 
 constexpr int kBwdRowWarps = 8;
 constexpr int kBwdThreads = 64 + 32 * kBwdRowWarps;
@@ -67,6 +80,9 @@ constexpr int kBwdThreads = 64 + 32 * kBwdRowWarps;
 // inside a packed region (see the layout above).
 __device__ __forceinline__ uint32_t bwd_packed_col(int kk) { return static_cast<uint32_t>((kk >> 2) * 64 + (kk & 3) * 8); }
 constexpr uint32_t kBwdTmemCols = 512;
+// dQ kernel: TMEM column of dP buffer b (dP(j) uses buffer j % 2); dQ sits
+// at [256, 256 + D) between them.
+__device__ __forceinline__ uint32_t bwd_dq_dp_col(int b) { return b ? 384u : 128u; }
 
 // Delta[b, h, s] = sum_d dO[b, s, h, d] * O[b, s, h, d], one warp per
 // (token, head) row: lanes read 8-byte pieces of both rows (coalesced).
@@ -130,18 +146,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __gri
   using L = BwdSmem<D>;
   constexpr uint32_t IDESC_SS = idesc_bf16_f32(128, 128, false);   // S = Q K^T, dP = dO V^T
   constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, D, true);      // dQ += dS K, K MN-major
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t sb = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  extern __shared__ __align__(1024) uint8_t bwd_smem[];
+  const uint32_t sb = smem_u32(bwd_smem);
+  if (sb & 1023u) {
+    if (threadIdx.x == 0) atomicOr(&g_device_status, static_cast<unsigned int>(SITE_LAYOUT));
+    return;
+  }
+  constexpr int KS = L::kStagesC, VS = L::kStagesE;
   constexpr uint32_t BAR_QD = L::kOffBar;          // Q and dO loaded
-  constexpr uint32_t BAR_KF = BAR_QD + 8;          // [2]
-  constexpr uint32_t BAR_KE = BAR_KF + 16;         // [2]
-  constexpr uint32_t BAR_VF = BAR_KE + 16;         // [2]
-  constexpr uint32_t BAR_VE = BAR_VF + 16;         // [2]
-  constexpr uint32_t BAR_S = BAR_VE + 16;          // S(j) in TMEM
+  constexpr uint32_t BAR_KF = BAR_QD + 8;          // [KS]
+  constexpr uint32_t BAR_KE = BAR_KF + 8 * KS;     // [KS]
+  constexpr uint32_t BAR_VF = BAR_KE + 8 * KS;     // [VS]
+  constexpr uint32_t BAR_VE = BAR_VF + 8 * VS;     // [VS]
+  constexpr uint32_t BAR_S = BAR_VE + 8 * VS;      // S(j) in TMEM
   constexpr uint32_t BAR_SC = BAR_S + 8;           // S(j) read by the row threads
-  constexpr uint32_t BAR_DP = BAR_SC + 8;          // dP(j) in TMEM
-  constexpr uint32_t BAR_DS = BAR_DP + 8;          // dS(j) in TMEM
-  constexpr uint32_t BAR_DQ = BAR_DS + 8;          // dQ complete
+  constexpr uint32_t BAR_DP = BAR_SC + 8;          // [2] dP(j) in TMEM buffer j % 2
+  constexpr uint32_t BAR_DS = BAR_DP + 16;         // [2] dS(j) in TMEM buffer j % 2
+  constexpr uint32_t BAR_DQ = BAR_DS + 16;         // dQ complete
   constexpr uint32_t BAR_TAIL = BAR_DQ + 8;
   constexpr uint32_t TMEM_SLOT = L::kOffMisc;
   constexpr uint32_t ABORT = L::kOffMisc + 4;
@@ -160,16 +181,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __gri
 
   if (threadIdx.x == 0) {
     mbar_init(sb + BAR_QD, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < KS; ++s) {
       mbar_init(sb + BAR_KF + 8 * s, 1);
       mbar_init(sb + BAR_KE + 8 * s, 1);
+    }
+    for (int s = 0; s < VS; ++s) {
       mbar_init(sb + BAR_VF + 8 * s, 1);
       mbar_init(sb + BAR_VE + 8 * s, 1);
     }
     mbar_init(sb + BAR_S, 1);
     mbar_init(sb + BAR_SC, kBwdRowWarps);
-    mbar_init(sb + BAR_DP, 1);
-    mbar_init(sb + BAR_DS, kBwdRowWarps);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(sb + BAR_DP + 8 * s, 1);
+      mbar_init(sb + BAR_DS + 8 * s, kBwdRowWarps);
+    }
     mbar_init(sb + BAR_DQ, 1);
     mbar_init(sb + BAR_TAIL, 1);
     st_shared_volatile(sb + ABORT, 0u);
@@ -198,26 +223,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __gri
         tma_load_3d(sb + L::kOffB + hf * L::kBoxBytes, &PB.tm_do, hf * 64, U.h, row_base + q0, sb + BAR_QD);
       }
       for (int j = 0; j < n; ++j) {
-        const int st = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        if (!mbar_wait(sb + BAR_KE + 8 * st, ph ^ 1, abort_flag, tmo, SITE_PRODUCER)) break;
-        mbar_arrive_expect_tx(sb + BAR_KF + 8 * st, L::kTileBytes);
+        const int ks = j % KS, vs = j % VS;
+        const uint32_t kph = (j / KS) & 1, vph = (j / VS) & 1;
+        if (!mbar_wait(sb + BAR_KE + 8 * ks, kph ^ 1, abort_flag, tmo, SITE_PRODUCER)) break;
+        mbar_arrive_expect_tx(sb + BAR_KF + 8 * ks, L::kTileBytes);
         for (int hf = 0; hf < L::kHalves; ++hf)
-          tma_load_3d(sb + L::kOffC + st * L::kTileBytes + hf * L::kBoxBytes, &PB.tm_k, hf * 64, U.h,
-                      row_base + j * 128, sb + BAR_KF + 8 * st);
-        if (!mbar_wait(sb + BAR_VE + 8 * st, ph ^ 1, abort_flag, tmo, SITE_PRODUCER)) break;
-        mbar_arrive_expect_tx(sb + BAR_VF + 8 * st, L::kTileBytes);
+          tma_load_3d(sb + L::kOffC + ks * L::kTileBytes + hf * L::kBoxBytes, &PB.tm_k, hf * 64, U.h,
+                      row_base + j * 128, sb + BAR_KF + 8 * ks);
+        if (!mbar_wait(sb + BAR_VE + 8 * vs, vph ^ 1, abort_flag, tmo, SITE_PRODUCER)) break;
+        mbar_arrive_expect_tx(sb + BAR_VF + 8 * vs, L::kTileBytes);
         for (int hf = 0; hf < L::kHalves; ++hf)
-          tma_load_3d(sb + L::kOffE + st * L::kTileBytes + hf * L::kBoxBytes, &PB.tm_v, hf * 64, U.h,
-                      row_base + j * 128, sb + BAR_VF + 8 * st);
+          tma_load_3d(sb + L::kOffE + vs * L::kTileBytes + hf * L::kBoxBytes, &PB.tm_v, hf * 64, U.h,
+                      row_base + j * 128, sb + BAR_VF + 8 * vs);
       }
       // every stage's last release must arrive before the CTA exits
-      for (int st = 0; st < 2; ++st) {
-        const int uses = n > st ? (n - 1 - st) / 2 + 1 : 0;
-        if (uses == 0) continue;
-        const uint32_t ph = (uses - 1) & 1;
-        mbar_wait(sb + BAR_KE + 8 * st, ph, 0u, tmo, SITE_TAIL);
-        mbar_wait(sb + BAR_VE + 8 * st, ph, 0u, tmo, SITE_TAIL);
+      for (int st = 0; st < KS; ++st) {
+        const int uses = n > st ? (n - 1 - st) / KS + 1 : 0;
+        if (uses > 0) mbar_wait(sb + BAR_KE + 8 * st, (uses - 1) & 1, 0u, tmo, SITE_TAIL);
+      }
+      for (int st = 0; st < VS; ++st) {
+        const int uses = n > st ? (n - 1 - st) / VS + 1 : 0;
+        if (uses > 0) mbar_wait(sb + BAR_VE + 8 * st, (uses - 1) & 1, 0u, tmo, SITE_TAIL);
       }
     }
   } else if (warp == 1) {
@@ -235,19 +261,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __gri
           mma_ss(d, a0 + off, b0 + off, IDESC_SS, kk > 0 ? 1u : 0u);
         }
       };
-      auto issue_s = [&](int st) { issue_ss(tmem, opaque_u64(dQo), opaque_u64(dK + ((st * L::kTileBytes) >> 4))); };
-      auto issue_dp = [&](int st) {
-        issue_ss(tmem + 128, opaque_u64(dDO), opaque_u64(dV + ((st * L::kTileBytes) >> 4)));
+      auto issue_s = [&](int ks) { issue_ss(tmem, opaque_u64(dQo), opaque_u64(dK + ((ks * L::kTileBytes) >> 4))); };
+      auto issue_dp = [&](int buf, int vs) {
+        issue_ss(tmem + bwd_dq_dp_col(buf), opaque_u64(dDO), opaque_u64(dV + ((vs * L::kTileBytes) >> 4)));
       };
       // dQ (+)= dS K: dS (bf16 pairs) from TMEM over dP, K MN-major (keys
       // are rows of 128 bytes): 16 keys = 2048 bytes per MMA.
-      auto issue_dq = [&](int st, bool acc) {
-        const uint64_t b0 = opaque_u64(dKmn + ((st * L::kTileBytes) >> 4));
+      auto issue_dq = [&](int buf, int ks, bool acc) {
+        const uint64_t b0 = opaque_u64(dKmn + ((ks * L::kTileBytes) >> 4));
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + 256, tmem + 128 + bwd_packed_col(kk), b0 + ((kk * 2048) >> 4), IDESC_DQ,
+          mma_ts(tmem + 256, tmem + bwd_dq_dp_col(buf) + bwd_packed_col(kk), b0 + ((kk * 2048) >> 4), IDESC_DQ,
                  (acc || kk > 0) ? 1u : 0u);
       };
+      // S(j+1) and dP(j+1) are issued as soon as the row threads have read
+      // S(j): dP alternates between two TMEM buffers, so dP(j+1) does not wait
+      // for dQ(j) to consume dS(j).  dQ(j) follows dS(j).  The tensor core runs
+      // the three MMAs of a step while the row threads work on the previous one.
       bool ok = n > 0 && mbar_wait_spin(sb + BAR_QD, 0, abort_flag, tmo, SITE_MMA);
       if (ok) ok = mbar_wait_spin(sb + BAR_KF, 0, abort_flag, tmo, SITE_MMA);
       if (ok) {
@@ -258,31 +288,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __gri
       if (ok) ok = mbar_wait_spin(sb + BAR_VF, 0, abort_flag, tmo, SITE_MMA);
       if (ok) {
         tc_fence_after();
-        issue_dp(0);
+        issue_dp(0, 0);
         mma_commit(sb + BAR_DP);
+        mma_commit(sb + BAR_VE);
       }
       for (int j = 0; ok && j < n; ++j) {
-        const int st = j & 1, st1 = (j + 1) & 1;
-        const uint32_t ph1 = ((j + 1) >> 1) & 1;
-        const bool more = j + 1 < n;
+        const int j1 = j + 1;
         if (!mbar_wait_spin(sb + BAR_SC, j & 1, abort_flag, tmo, SITE_MMA)) break;
-        if (more) {   // S(j) has been read: the next S may overwrite it
-          if (!mbar_wait_spin(sb + BAR_KF + 8 * st1, ph1, abort_flag, tmo, SITE_MMA)) break;
+        if (j1 < n) {   // S(j) has been read: the next S may overwrite it
+          const int ks1 = j1 % KS, vs1 = j1 % VS;
+          if (!mbar_wait_spin(sb + BAR_KF + 8 * ks1, (j1 / KS) & 1, abort_flag, tmo, SITE_MMA)) break;
           tc_fence_after();
-          issue_s(st1);
+          issue_s(ks1);
           mma_commit(sb + BAR_S);
-        }
-        if (!mbar_wait_spin(sb + BAR_DS, j & 1, abort_flag, tmo, SITE_MMA)) break;
-        tc_fence_after();
-        issue_dq(st, j > 0);
-        mma_commit(sb + BAR_KE + 8 * st);
-        mma_commit(sb + BAR_VE + 8 * st);
-        if (more) {   // dS(j) is consumed in order before dP(j+1) overwrites it
-          if (!mbar_wait_spin(sb + BAR_VF + 8 * st1, ph1, abort_flag, tmo, SITE_MMA)) break;
+          // dP buffer j1 % 2 last held dS(j-1), consumed by dQ(j-1), issued
+          // earlier on this thread: the tensor core reads it first.
+          if (!mbar_wait_spin(sb + BAR_VF + 8 * vs1, (j1 / VS) & 1, abort_flag, tmo, SITE_MMA)) break;
           tc_fence_after();
-          issue_dp(st1);
-          mma_commit(sb + BAR_DP);
+          issue_dp(j1 & 1, vs1);
+          mma_commit(sb + BAR_DP + 8 * (j1 & 1));
+          mma_commit(sb + BAR_VE + 8 * vs1);
         }
+        if (!mbar_wait_spin(sb + BAR_DS + 8 * (j & 1), (j >> 1) & 1, abort_flag, tmo, SITE_MMA)) break;
+        tc_fence_after();
+        issue_dq(j & 1, j % KS, j > 0);
+        mma_commit(sb + BAR_KE + 8 * (j % KS));
       }
       if (n > 0) mma_commit(sb + BAR_DQ);
       mma_commit(sb + BAR_TAIL);
@@ -298,7 +328,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __gri
     const bool row_valid = row < q_rows;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t tS = tmem + lane_base + col0;
-    const uint32_t tDP = tmem + lane_base + 128 + col0;
     const uint32_t tDQ = tmem + lane_base + 256;
     const float c = p.scale_log2;
     const long long li = static_cast<long long>(U.b) * PB.lse_b + static_cast<long long>(U.h + PB.lse_h0) * PB.lse_h + q_pos;
@@ -327,10 +356,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __gri
 #pragma unroll
       for (int k = 0; k < 64; ++k)
         s[k] = __float_as_uint(k < kvalid ? ex2_approx(__uint_as_float(s[k]) * c - lse2) : 0.f);
-      w = mbar_wait(sb + BAR_DP, j & 1, abort_flag, tmo, SITE_SOFTMAX);
+      w = mbar_wait(sb + BAR_DP + 8 * (j & 1), (j >> 1) & 1, abort_flag, tmo, SITE_SOFTMAX);
       if (__any_sync(0xffffffffu, !w)) { ok = false; break; }
       __syncwarp();
       tc_fence_after();
+      const uint32_t tDP = tmem + lane_base + bwd_dq_dp_col(j & 1) + col0;
       // dS = P * (dP - delta), bf16 pairs over the dP columns already read
 #pragma unroll
       for (int c0 = 0; c0 < 64; c0 += 32) {
@@ -348,7 +378,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __gri
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(sb + BAR_DS);
+      if (lane == 0) mbar_arrive(sb + BAR_DS + 8 * (j & 1));
     }
     if (ok && n > 0) {
       const bool w = mbar_wait(sb + BAR_DQ, 0, abort_flag, tmo, SITE_EPILOGUE);
@@ -397,14 +427,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __gr
   using L = BwdSmem<D>;
   constexpr uint32_t IDESC_SS = idesc_bf16_f32(128, 128, false);   // S^T = K Q^T, dP^T = V dO^T
   constexpr uint32_t IDESC_ACC = idesc_bf16_f32(128, D, true);     // dV += P^T dO, dK += dS^T Q
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t sb = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  extern __shared__ __align__(1024) uint8_t bwd_smem[];
+  const uint32_t sb = smem_u32(bwd_smem);
+  if (sb & 1023u) {
+    if (threadIdx.x == 0) atomicOr(&g_device_status, static_cast<unsigned int>(SITE_LAYOUT));
+    return;
+  }
+  constexpr int QS = L::kStagesC, OS = L::kStagesE;
   constexpr uint32_t BAR_KV = L::kOffBar;          // K and V loaded
-  constexpr uint32_t BAR_QF = BAR_KV + 8;          // [2]
-  constexpr uint32_t BAR_QE = BAR_QF + 16;         // [2]
-  constexpr uint32_t BAR_OF = BAR_QE + 16;         // [2] dO tile full
-  constexpr uint32_t BAR_OE = BAR_OF + 16;         // [2]
-  constexpr uint32_t BAR_S = BAR_OE + 16;          // S^T(i) in TMEM
+  constexpr uint32_t BAR_QF = BAR_KV + 8;          // [QS]
+  constexpr uint32_t BAR_QE = BAR_QF + 8 * QS;     // [QS]
+  constexpr uint32_t BAR_OF = BAR_QE + 8 * QS;     // [OS] dO tile full
+  constexpr uint32_t BAR_OE = BAR_OF + 8 * OS;     // [OS]
+  constexpr uint32_t BAR_S = BAR_OE + 8 * OS;      // S^T(i) in TMEM
   constexpr uint32_t BAR_P = BAR_S + 8;            // P^T(i) written
   constexpr uint32_t BAR_DP = BAR_P + 8;           // dP^T(i) in TMEM
   constexpr uint32_t BAR_DS = BAR_DP + 8;          // dS^T(i) written
@@ -429,9 +464,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __gr
 
   if (threadIdx.x == 0) {
     mbar_init(sb + BAR_KV, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < QS; ++s) {
       mbar_init(sb + BAR_QF + 8 * s, 1);
       mbar_init(sb + BAR_QE + 8 * s, 1);
+    }
+    for (int s = 0; s < OS; ++s) {
       mbar_init(sb + BAR_OF + 8 * s, 1);
       mbar_init(sb + BAR_OE + 8 * s, 1);
     }
@@ -468,26 +505,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __gr
         tma_load_3d(sb + L::kOffB + hf * L::kBoxBytes, &PB.tm_v, hf * 64, U.h, row_base + k0, sb + BAR_KV);
       }
       for (int i = 0; i < n; ++i) {
-        const int st = i & 1;
-        const uint32_t ph = (i >> 1) & 1;
+        const int qs = i % QS, os = i % OS;
+        const uint32_t qph = (i / QS) & 1, oph = (i / OS) & 1;
         const int qrow = row_base + (qt0 + i) * 128;
-        if (!mbar_wait(sb + BAR_QE + 8 * st, ph ^ 1, abort_flag, tmo, SITE_PRODUCER)) break;
-        mbar_arrive_expect_tx(sb + BAR_QF + 8 * st, L::kTileBytes);
+        if (!mbar_wait(sb + BAR_QE + 8 * qs, qph ^ 1, abort_flag, tmo, SITE_PRODUCER)) break;
+        mbar_arrive_expect_tx(sb + BAR_QF + 8 * qs, L::kTileBytes);
         for (int hf = 0; hf < L::kHalves; ++hf)
-          tma_load_3d(sb + L::kOffC + st * L::kTileBytes + hf * L::kBoxBytes, &PB.tm_q, hf * 64, U.h, qrow,
-                      sb + BAR_QF + 8 * st);
-        if (!mbar_wait(sb + BAR_OE + 8 * st, ph ^ 1, abort_flag, tmo, SITE_PRODUCER)) break;
-        mbar_arrive_expect_tx(sb + BAR_OF + 8 * st, L::kTileBytes);
+          tma_load_3d(sb + L::kOffC + qs * L::kTileBytes + hf * L::kBoxBytes, &PB.tm_q, hf * 64, U.h, qrow,
+                      sb + BAR_QF + 8 * qs);
+        if (!mbar_wait(sb + BAR_OE + 8 * os, oph ^ 1, abort_flag, tmo, SITE_PRODUCER)) break;
+        mbar_arrive_expect_tx(sb + BAR_OF + 8 * os, L::kTileBytes);
         for (int hf = 0; hf < L::kHalves; ++hf)
-          tma_load_3d(sb + L::kOffE + st * L::kTileBytes + hf * L::kBoxBytes, &PB.tm_do, hf * 64, U.h, qrow,
-                      sb + BAR_OF + 8 * st);
+          tma_load_3d(sb + L::kOffE + os * L::kTileBytes + hf * L::kBoxBytes, &PB.tm_do, hf * 64, U.h, qrow,
+                      sb + BAR_OF + 8 * os);
       }
-      for (int st = 0; st < 2; ++st) {
-        const int uses = n > st ? (n - 1 - st) / 2 + 1 : 0;
-        if (uses == 0) continue;
-        const uint32_t ph = (uses - 1) & 1;
-        mbar_wait(sb + BAR_QE + 8 * st, ph, 0u, tmo, SITE_TAIL);
-        mbar_wait(sb + BAR_OE + 8 * st, ph, 0u, tmo, SITE_TAIL);
+      for (int st = 0; st < QS; ++st) {
+        const int uses = n > st ? (n - 1 - st) / QS + 1 : 0;
+        if (uses > 0) mbar_wait(sb + BAR_QE + 8 * st, (uses - 1) & 1, 0u, tmo, SITE_TAIL);
+      }
+      for (int st = 0; st < OS; ++st) {
+        const int uses = n > st ? (n - 1 - st) / OS + 1 : 0;
+        if (uses > 0) mbar_wait(sb + BAR_OE + 8 * st, (uses - 1) & 1, 0u, tmo, SITE_TAIL);
       }
     }
   } else if (warp == 1) {
@@ -526,29 +564,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __gr
         mma_commit(sb + BAR_DP);
       }
       for (int i = 0; ok && i < n; ++i) {
-        const int st = i & 1, st1 = (i + 1) & 1;
-        const uint32_t ph1 = ((i + 1) >> 1) & 1;
-        const bool more = i + 1 < n;
-        // dV (+)= P^T dO: P^T (bf16 pairs) from TMEM over S^T, dO MN-major
+        const int i1 = i + 1;
+        const bool more = i1 < n;
+        // dV (+)= P^T dO: P^T (bf16 pairs) from TMEM over S^T, dO MN-major;
+        // dO(i) has no later use, so its stage is released right behind it
         if (!mbar_wait_spin(sb + BAR_P, i & 1, abort_flag, tmo, SITE_MMA)) break;
         tc_fence_after();
-        issue_acc(tmem + 256, tmem, opaque_u64(dOmn + stage_off(st)), i > 0);
+        issue_acc(tmem + 256, tmem, opaque_u64(dOmn + stage_off(i % OS)), i > 0);
+        mma_commit(sb + BAR_OE + 8 * (i % OS));
         if (more) {   // P^T(i) is consumed in order before S^T(i+1) overwrites it
-          if (!mbar_wait_spin(sb + BAR_QF + 8 * st1, ph1, abort_flag, tmo, SITE_MMA)) break;
+          const int qs1 = i1 % QS;
+          if (!mbar_wait_spin(sb + BAR_QF + 8 * qs1, (i1 / QS) & 1, abort_flag, tmo, SITE_MMA)) break;
           tc_fence_after();
-          issue_ss(tmem, opaque_u64(dK), opaque_u64(dQk + stage_off(st1)));
+          issue_ss(tmem, opaque_u64(dK), opaque_u64(dQk + stage_off(qs1)));
           mma_commit(sb + BAR_S);
         }
         // dK (+)= dS^T Q: dS^T (bf16 pairs) from TMEM over dP^T, Q MN-major
         if (!mbar_wait_spin(sb + BAR_DS, i & 1, abort_flag, tmo, SITE_MMA)) break;
         tc_fence_after();
-        issue_acc(tmem + 256 + D, tmem + 128, opaque_u64(dQmn + stage_off(st)), i > 0);
-        mma_commit(sb + BAR_QE + 8 * st);
-        mma_commit(sb + BAR_OE + 8 * st);
+        issue_acc(tmem + 256 + D, tmem + 128, opaque_u64(dQmn + stage_off(i % QS)), i > 0);
+        mma_commit(sb + BAR_QE + 8 * (i % QS));
         if (more) {
-          if (!mbar_wait_spin(sb + BAR_OF + 8 * st1, ph1, abort_flag, tmo, SITE_MMA)) break;
+          const int os1 = i1 % OS;
+          if (!mbar_wait_spin(sb + BAR_OF + 8 * os1, (i1 / OS) & 1, abort_flag, tmo, SITE_MMA)) break;
           tc_fence_after();
-          issue_ss(tmem + 128, opaque_u64(dV), opaque_u64(dOk + stage_off(st1)));
+          issue_ss(tmem + 128, opaque_u64(dV), opaque_u64(dOk + stage_off(os1)));
           mma_commit(sb + BAR_DP);
         }
       }
@@ -610,7 +650,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __gr
       // per-query values are read as float4 through a plain shared-memory
       // pointer (the barrier waits above are compiler fences), so the loads
       // schedule freely around the exponentials.
-      const float4 *lse4 = reinterpret_cast<const float4 *>(smem_raw + (vec - smem_u32(smem_raw))) + (col0 >> 2);
+      const float4 *lse4 = reinterpret_cast<const float4 *>(bwd_smem + (vec - sb)) + (col0 >> 2);
       const float4 *del4 = lse4 + 32;
       const int qlim = (p.causal ? k_pos - q0 : 0) - col0;   // queries q < qlim do not see this key
 #pragma unroll

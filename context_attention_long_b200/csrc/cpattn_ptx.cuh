@@ -23,6 +23,7 @@ enum WaitSite : unsigned int {
   SITE_EPILOGUE = 1u << 3,
   SITE_TAIL = 1u << 4,
   SITE_DEBUG = 1u << 5,
+  SITE_LAYOUT = 1u << 6,   // a kernel found its shared-memory window misaligned and did nothing
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {

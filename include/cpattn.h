@@ -655,7 +655,8 @@ int cpattn_plan_exchange(int B, int H, int S, int D, int elem_bytes, int degree,
 /*
  * Synchronises `stream`, then reads and clears the device status word that the
  * kernels' bounded waits set when a pipeline wait expires.  *code receives the
- * raw word (0 = healthy; otherwise a bit per wait site).  Returns CPATTN_OK,
+ * raw word (0 = healthy; otherwise a bit per wait site; bit 6 means a kernel
+ * found its shared-memory window misaligned and did nothing).  Returns CPATTN_OK,
  * CPATTN_ERR_DEVICE_TIMEOUT if the word was non-zero, or CPATTN_ERR_CUDA.
  */
 int cpattn_device_status(cpattn_stream_t stream, unsigned int *code);
