@@ -352,28 +352,41 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __gri
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(sb + BAR_SC);
-      // P = 2^(S*c - lse2), kept in fp32 over the scores
+      // P = 2^(S*c - lse2), kept in fp32 over the scores: the first 32 keys
+      // before the dP wait (pinned there, so the compiler keeps them ahead of
+      // it), the other 32 interleaved with dS of the first 32, so that the
+      // dS arithmetic issues while the SFU works.
+      auto p_of = [&](int k) {
+        return __float_as_uint(k < kvalid ? ex2_approx(__uint_as_float(s[k]) * c - lse2) : 0.f);
+      };
 #pragma unroll
-      for (int k = 0; k < 64; ++k)
-        s[k] = __float_as_uint(k < kvalid ? ex2_approx(__uint_as_float(s[k]) * c - lse2) : 0.f);
+      for (int k = 0; k < 32; ++k) s[k] = p_of(k);
+#pragma unroll
+      for (int k = 0; k < 32; ++k) reg_pin(s[k]);
       w = mbar_wait(sb + BAR_DP + 8 * (j & 1), (j >> 1) & 1, abort_flag, tmo, SITE_SOFTMAX);
       if (__any_sync(0xffffffffu, !w)) { ok = false; break; }
       __syncwarp();
       tc_fence_after();
       const uint32_t tDP = tmem + lane_base + bwd_dq_dp_col(j & 1) + col0;
       // dS = P * (dP - delta), bf16 pairs over the dP columns already read
-#pragma unroll
-      for (int c0 = 0; c0 < 64; c0 += 32) {
-        uint32_t dp[32];
-        tmem_ld32_wait(tDP + c0, dp);
-        uint32_t pk[16];
+      auto ds_pair = [&](int k, const uint32_t *dp) {
+        return pack_bf16x2(__uint_as_float(s[k]) * (__uint_as_float(dp[0]) - delta),
+                           __uint_as_float(s[k + 1]) * (__uint_as_float(dp[1]) - delta));
+      };
+      {
+        uint32_t dp[32], pk[16];
+        tmem_ld32_wait(tDP, dp);
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
-          const float d0 = __uint_as_float(s[c0 + 2 * k]) * (__uint_as_float(dp[2 * k]) - delta);
-          const float d1 = __uint_as_float(s[c0 + 2 * k + 1]) * (__uint_as_float(dp[2 * k + 1]) - delta);
-          pk[k] = pack_bf16x2(d0, d1);
+          s[32 + 2 * k] = p_of(32 + 2 * k);
+          s[33 + 2 * k] = p_of(33 + 2 * k);
+          pk[k] = ds_pair(2 * k, dp + 2 * k);
         }
-        tmem_st16(tDP + c0 / 2, pk);
+        tmem_st16(tDP, pk);
+        tmem_ld32_wait(tDP + 32, dp);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) pk[k] = ds_pair(32 + 2 * k, dp + 2 * k);
+        tmem_st16(tDP + 16, pk);
       }
       tmem_st_wait();
       tc_fence_before();

@@ -148,6 +148,11 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// Pins a value in a register at this point of the program: an empty volatile
+// asm that reads and "writes" it, so the computation of the value cannot sink
+// past a later volatile asm (a barrier wait).
+__device__ __forceinline__ void reg_pin(uint32_t &v) { asm volatile("" : "+r"(v)); }
+
 // ------------------------------------------------------- packed f32x2 math
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
   uint64_t r;
