@@ -44,6 +44,10 @@
 
 namespace cpattn {
 
+// Device status bit of a backward kernel that found its shared-memory window
+// misaligned (it then returns without touching memory).
+constexpr unsigned int SITE_LAYOUT = 1u << 6;
+
 template <int D>
 struct BwdSmem {
   static constexpr int kHalves = D / 64;
@@ -72,6 +76,11 @@ struct BwdSmem {
   static constexpr int kAllocBytes = kBytes;
 };
 static_assert(BwdSmem<128>::kAllocBytes <= 232448, "backward shared memory exceeds the per-CTA limit");
+
+// Pins a value in a register at this point of the program: an empty volatile
+// asm that reads and "writes" it, so the computation of the value cannot sink
+// past a later volatile asm (a barrier wait).
+__device__ __forceinline__ void reg_pin(uint32_t &v) { asm volatile("" : "+r"(v)); }
 
 constexpr int kBwdRowWarps = 8;
 constexpr int kBwdThreads = 64 + 32 * kBwdRowWarps;
@@ -149,7 +158,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __gri
   extern __shared__ __align__(1024) uint8_t bwd_smem[];
   const uint32_t sb = smem_u32(bwd_smem);
   if (sb & 1023u) {
-    if (threadIdx.x == 0) atomicOr(&g_device_status, static_cast<unsigned int>(SITE_LAYOUT));
+    if (threadIdx.x == 0) atomicOr(&g_device_status, SITE_LAYOUT);
     return;
   }
   constexpr int KS = L::kStagesC, VS = L::kStagesE;
@@ -443,7 +452,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __gr
   extern __shared__ __align__(1024) uint8_t bwd_smem[];
   const uint32_t sb = smem_u32(bwd_smem);
   if (sb & 1023u) {
-    if (threadIdx.x == 0) atomicOr(&g_device_status, static_cast<unsigned int>(SITE_LAYOUT));
+    if (threadIdx.x == 0) atomicOr(&g_device_status, SITE_LAYOUT);
     return;
   }
   constexpr int QS = L::kStagesC, OS = L::kStagesE;

@@ -23,7 +23,6 @@ enum WaitSite : unsigned int {
   SITE_EPILOGUE = 1u << 3,
   SITE_TAIL = 1u << 4,
   SITE_DEBUG = 1u << 5,
-  SITE_LAYOUT = 1u << 6,   // a kernel found its shared-memory window misaligned and did nothing
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -147,11 +146,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-
-// Pins a value in a register at this point of the program: an empty volatile
-// asm that reads and "writes" it, so the computation of the value cannot sink
-// past a later volatile asm (a barrier wait).
-__device__ __forceinline__ void reg_pin(uint32_t &v) { asm volatile("" : "+r"(v)); }
 
 // ------------------------------------------------------- packed f32x2 math
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
