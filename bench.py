@@ -265,7 +265,8 @@ def config_block(cfg, world=1):
     return {"workload": f"video-DiT B{B} H{H} S{S} D{D}: ring {world} (NCCL P2P rotation) + unified ring "
                         f"{world // 2} x Ulysses 2 (NCCL all-to-all), sequence sharded over {world} GPUs",
             "B": B, "H": H, "S": S, "D": D, "ring_degree": world, "ulysses_degree": 2,
-            "parallelism": f"context parallel over {world} GPUs", "l2": "inputs larger than L2"}
+            "parallelism": f"context parallel over {world} GPUs",
+            "l2": "an L2 flush (256 MiB written, then read) on every rank before every timed step"}
 
 
 def cpu_baseline(cfg, q, k, v, budget_s=12.0):
@@ -586,6 +587,7 @@ def run_multi_gpu(args, world, rank, dev):
         if e: e[2].record(stream)
         return o_r, o_u
 
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -596,6 +598,7 @@ def run_multi_gpu(args, world, rank, dev):
     torch.cuda.synchronize()
     t0 = time.perf_counter()
     for i in range(args.steps):
+        flush_l2(flush)       # between steps, outside the events
         step(ev[i])
     torch.cuda.synchronize()
     t1 = time.perf_counter()
