@@ -337,11 +337,11 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)     # before NCCL sees the process group
+    dev = torch.device("cuda", local_rank)
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
     if rank == 0:
         build.build()
     if world > 1:
