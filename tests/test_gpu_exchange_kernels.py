@@ -14,7 +14,7 @@ import oracle
 from context_attention_long_b200 import api, build, exchange, inputs
 
 from exchange_standin import OracleKernels
-from gpu_util import assert_close, f64_of, full_to_rank_buffers, to_dev
+from gpu_util import assert_close, f64_of, full_to_rank_buffers, oracle_rows, sample_positions, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -84,6 +84,38 @@ def test_ring_chunk_steps_match_oracle(B, H, D, lens, causal):
                      f"rank {r} of {lens}")
         # a chunk padded to the longest one (the all-gather layout) gives the same bytes
         assert torch.equal(o.view(torch.int16), op.view(torch.int16)) and torch.equal(l, lp)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_ring_chunk_steps_video_size_sampled(causal):
+    """One rank of the video workload's 8-way ring (B1 H40 S32760 D128) in the
+    launch sequence of the multi-GPU bench: one cpattn_ring_chunk_attention
+    per 4095-row chunk in ring order, the running float32 state merged in the
+    epilogue, the last step in bf16.  Sampled query rows (the shard's edges and
+    random rows) against the oracle over all 32760 keys."""
+    cfg, qb, kb, vb = inputs.config_inputs("video")
+    B, S, H, D = qb.shape
+    P, r = 8, 5
+    lens = [S // P] * P
+    off = np.concatenate([[0], np.cumsum(lens)]).astype(int)
+    q, k, v = (to_dev(x) for x in (qb, kb, vb))
+    o, l = _emulated_ring_rank(q, k, v, lens, r, causal, padded=False)
+    torch.cuda.synchronize()
+    _no_timeouts()
+    local = sample_positions(lens[r], [0, lens[r]], 12, 21 + int(causal))
+    pos = local + off[r]
+    if causal:
+        ref_o = np.zeros((B, len(pos), H, D))
+        ref_l = np.zeros((B, H, len(pos)))
+        for h in range(H):
+            ro, rl = oracle.causal_attention_rows(inputs.bf16_bits_to_f64(qb[0, pos, h]),
+                                                  inputs.bf16_bits_to_f64(kb[0, :, h]),
+                                                  inputs.bf16_bits_to_f64(vb[0, :, h]), pos, np.arange(S))
+            ref_o[0, :, h], ref_l[0, h] = ro, rl
+    else:
+        ref_o, ref_l = oracle_rows(oracle, qb, kb, vb, pos)
+    lc = l.cpu().numpy()[:, :, local]
+    assert_close(f64_of(o)[:, local], lc, ref_o, ref_l, f"video ring rank {r} causal {causal}")
 
 
 @pytest.mark.parametrize("B,H,D,lens,causal", [
