@@ -47,6 +47,19 @@ L2_FLUSH_BYTES = 256 << 20
 NOMINAL_LINK_GBS = 900.0
 
 
+def ring_peak_choice(peaks, peaks_kind, region_s):
+    """Denominator of the step's ring-kernel roofline: the sustained bf16
+    figure when the timed region lasts a second or more (the kernel then runs
+    under the power cap) and the peaks file holds one, else the burst figure.
+    Returns (peak TFLOP/s, label)."""
+    burst = float(peaks["bf16_tflops"])
+    if region_s >= 1.0 and "bf16_tflops_sustained" in peaks:
+        return (float(peaks["bf16_tflops_sustained"]),
+                f"bf16_tflops_sustained, {peaks_kind} (timed region {region_s:.1f} s of back-to-back steps)")
+    note = "" if "bf16_tflops_sustained" in peaks else " (the peaks file holds no sustained figure)"
+    return burst, f"bf16_tflops burst, {peaks_kind}{note}"
+
+
 def load_peaks():
     path = os.path.join(REPO, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -405,8 +418,6 @@ def main():
 
     peaks, peaks_kind = load_peaks()
     peak_tf = float(peaks["bf16_tflops"])
-    has_sustained = "bf16_tflops_sustained" in peaks
-    peak_tf_sus = float(peaks["bf16_tflops_sustained"]) if has_sustained else peak_tf
     hbm = float(peaks["hbm_gbs"])
     ring_ms = float(per[:, 0].mean())
     ring_tflops = attn_flops / (ring_ms * 1e-3) / 1e12
@@ -445,18 +456,14 @@ def main():
     # the power cap, and the denominator is the sustained bf16 figure (a
     # seconds-long cuBLAS loop), else the burst figure.
     region_s = t_wall1 - t_wall0
-    sustained = region_s >= 1.0 and has_sustained
-    ring_peak = peak_tf_sus if sustained else peak_tf
+    ring_peak, ring_peak_kind = ring_peak_choice(peaks, peaks_kind, region_s)
     tensor_kernels = [
         tensor_entry(f"unified ring {P} x Ulysses {U} (in the step; 2 launches)", attn_flops, uni_ms, ring_peak),
         tensor_entry(f"causal ring fused P={P} (visible pairs)", causal_flops(B, H, S, D), causal_ms, peak_tf),
     ]
     roofline = {"bound": "tensor", "kernel": f"attn_fwd_kernel<128,bf16> (ring fused, P={P}, in the step)",
                 "achieved": ring_tflops, "peak": ring_peak, "unit": "TFLOP/s", "frac": ring_tflops / ring_peak,
-                "peak_kind": (f"bf16_tflops_sustained, {peaks_kind} (timed region {region_s:.1f} s of back-to-back "
-                              f"steps)") if sustained else (
-                    f"bf16_tflops burst, {peaks_kind}" + ("" if has_sustained else
-                                                          " (the peaks file holds no sustained figure)")),
+                "peak_kind": ring_peak_kind,
                 "frac_of_burst": ring_tflops / peak_tf,
                 "traffic": stored_traffic("attn_fwd_ring_video"),
                 "algorithmic_flops_per_launch": attn_flops,

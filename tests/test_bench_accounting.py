@@ -39,3 +39,14 @@ def test_multi_gpu_shards_cover_the_sequence_once(S, world):
     flat = [n for chunk in subs for n in chunk]
     assert flat == lens
     assert ring_lens == [sum(c) for c in subs] and sum(ring_lens) == S
+
+
+def test_ring_peak_choice_sustained_only_for_long_regions_with_the_figure():
+    peaks = {"bf16_tflops": 1646.1, "bf16_tflops_sustained": 1450.0, "hbm_gbs": 6547.2}
+    p, kind = bench.ring_peak_choice(peaks, "measured", 1.2)
+    assert p == 1450.0 and kind.startswith("bf16_tflops_sustained, measured")
+    p, kind = bench.ring_peak_choice(peaks, "measured", 0.4)
+    assert p == 1646.1 and kind == "bf16_tflops burst, measured"
+    no_sus = {"bf16_tflops": 1646.1, "hbm_gbs": 6547.2}
+    p, kind = bench.ring_peak_choice(no_sus, "measured", 1.2)
+    assert p == 1646.1 and "no sustained figure" in kind
