@@ -16,8 +16,10 @@
 // move in one launch: every warp takes its tokens of each tensor in turn.
 // One warp moves one token per iteration: lanes take consecutive 16-byte
 // vectors of the token's H*D run (coalesced on the sequence side, and on the
-// head side within each head rank's contiguous block), four vectors in flight
-// per lane.  Bit-exact (plain 16-byte loads and stores).
+// head side within each head rank's contiguous block), kPermuteBatch vectors in
+// flight per lane; per-head offsets and strides sit in shared memory, so a vector's
+// head-side address costs one multiply-add.  Bit-exact (plain 16-byte loads
+// and stores).
 #pragma once
 
 #include "cpattn_internal.h"
@@ -25,6 +27,9 @@
 namespace cpattn {
 
 constexpr int kPermuteThreads = 256;
+// 16-byte vectors a lane loads before it stores them (8 measured slower: the
+// registers they take cost occupancy).
+constexpr int kPermuteBatch = 4;
 
 __device__ __forceinline__ int find_range(const int *off, int n, int x) {
   // largest i in [0, n) with off[i] <= x < off[i+1] (empty ranges skipped)
@@ -37,8 +42,19 @@ __device__ __forceinline__ int find_range(const int *off, int n, int x) {
 }
 
 __global__ void __launch_bounds__(kPermuteThreads) permute_kernel(const __grid_constant__ PermuteParams p) {
-  __shared__ int s_rank[kMaxHeads];   // head -> head rank
-  for (int h = threadIdx.x; h < p.H; h += blockDim.x) s_rank[h] = find_range(p.head_off, p.n_head, h);
+  // Per head h: the byte offset of its first (token, head) row on the head
+  // side, and the stride between consecutive head-side token rows of its
+  // head rank (H_u * row_bytes), so that a vector's address is one
+  // multiply-add from the token's head-side row index.
+  __shared__ long long s_base[kMaxHeads];
+  __shared__ int s_stride[kMaxHeads];   // <= kMaxHeads * 1 MiB < 2^31
+  for (int h = threadIdx.x; h < p.H; h += blockDim.x) {
+    const int u = find_range(p.head_off, p.n_head, h);
+    const int hu0 = p.head_off[u];
+    const int Hu = p.head_off[u + 1] - hu0;
+    s_base[h] = (static_cast<long long>(p.B) * p.S * hu0 + (h - hu0)) * p.row_bytes;
+    s_stride[h] = Hu * p.row_bytes;
+  }
   __syncthreads();
 
   const int lane = threadIdx.x & 31;
@@ -48,6 +64,11 @@ __global__ void __launch_bounds__(kPermuteThreads) permute_kernel(const __grid_c
   const int vpr = p.row_bytes >> 4;                 // 16-byte vectors per (token, head) row
   const int nvec = p.H * vpr;                       // vectors per token
   const long long seq_row_bytes = static_cast<long long>(p.H) * p.row_bytes;
+  // Vector v of a token is (head v / vpr, piece v % vpr).  A lane starts at
+  // v = lane and steps by 32: the (head, piece) pair advances by (32 / vpr,
+  // 32 % vpr) with one carry, so no division runs per vector.
+  const int h_lane = lane / vpr, w_lane = lane - h_lane * vpr;
+  const int dh = 32 / vpr, dw = 32 - dh * vpr;
 
   for (int t = 0; t < p.n_tensors; ++t)
   for (long long tok = warp_id; tok < ntok; tok += nwarps) {
@@ -67,36 +88,36 @@ __global__ void __launch_bounds__(kPermuteThreads) permute_kernel(const __grid_c
     const unsigned char *seq_base = (p.direction == 0 ? p.src[t] : p.dst[t]) + seq_row * seq_row_bytes;
     unsigned char *const head_buf = p.direction == 0 ? p.dst[t] : const_cast<unsigned char *>(p.src[t]);
 
-    for (int v0 = lane; v0 < nvec; v0 += 32 * 4) {
-      uint4 val[4];
-      long long seq_off[4], head_off[4];
+    int h = h_lane, w = w_lane;
+    for (int v0 = lane; v0 < nvec; v0 += 32 * kPermuteBatch) {
+      uint4 val[kPermuteBatch];
+      long long head_off[kPermuteBatch];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
+      for (int k = 0; k < kPermuteBatch; ++k) {
         const int v = v0 + 32 * k;
-        seq_off[k] = -1;
-        if (v < nvec) {
-          const int h = v / vpr;
-          const int w = v - h * vpr;
-          const int u = s_rank[h];
-          const int hu0 = p.head_off[u];
-          const int Hu = p.head_off[u + 1] - hu0;
-          seq_off[k] = static_cast<long long>(v) * 16;
-          head_off[k] = (static_cast<long long>(p.B) * p.S * hu0 + head_row * Hu + (h - hu0)) * p.row_bytes +
-                        static_cast<long long>(w) * 16;
+        if (v < nvec)              // then h < H
+          head_off[k] = s_base[h] + head_row * s_stride[h] + static_cast<long long>(w) * 16;
+        w += dw;
+        h += dh;
+        if (w >= vpr) {
+          w -= vpr;
+          ++h;
         }
       }
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        if (seq_off[k] >= 0) {
-          if (p.direction == 0) val[k] = __ldcs(reinterpret_cast<const uint4 *>(seq_base + seq_off[k]));
+      for (int k = 0; k < kPermuteBatch; ++k) {
+        const int v = v0 + 32 * k;
+        if (v < nvec) {
+          if (p.direction == 0) val[k] = __ldcs(reinterpret_cast<const uint4 *>(seq_base + static_cast<long long>(v) * 16));
           else val[k] = __ldcs(reinterpret_cast<const uint4 *>(head_buf + head_off[k]));
         }
       }
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        if (seq_off[k] >= 0) {
+      for (int k = 0; k < kPermuteBatch; ++k) {
+        const int v = v0 + 32 * k;
+        if (v < nvec) {
           if (p.direction == 0) __stcs(reinterpret_cast<uint4 *>(head_buf + head_off[k]), val[k]);
-          else __stcs(reinterpret_cast<uint4 *>(const_cast<unsigned char *>(seq_base) + seq_off[k]), val[k]);
+          else __stcs(reinterpret_cast<uint4 *>(const_cast<unsigned char *>(seq_base) + static_cast<long long>(v) * 16), val[k]);
         }
       }
     }

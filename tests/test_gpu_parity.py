@@ -141,6 +141,8 @@ PERMUTE_CASES = [
     (1, 9, 5, 8, 2, [4, 5], [2, 3], torch.uint8),       # 8-byte rows: rejected (not a multiple of 16)
     (3, 19, 8, 16, 8, [1, 2, 3, 4, 0, 0, 4, 5], [1] * 8, torch.float32),
     (1, 33, 3, 16, 3, [11, 11, 11], [1, 1, 1], torch.uint8),   # 16-byte rows of bytes
+    (2, 41, 5, 12, 3, [13, 0, 28], [2, 1, 2], torch.float32),  # 48-byte rows: 3 vectors, lanes cross rows
+    (1, 17, 3, 1000, 2, [9, 8], [2, 1], torch.float32),        # 4000-byte rows: 250 vectors per row
     (1, 10007, 30, 128, 4, [2502, 2502, 2502, 2501], [8, 8, 7, 7], torch.bfloat16),
 ]
 
