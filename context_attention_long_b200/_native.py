@@ -16,6 +16,8 @@ P_UINT = ctypes.POINTER(ctypes.c_uint)
 # name -> (restype, argtypes); mirrors include/cpattn.h
 SIGNATURES = {
     "cpattn_status_string": (c_char_p, [c_int]),
+    "cpattn_last_cuda_error": (c_int, []),
+    "cpattn_last_cuda_error_string": (c_char_p, []),
     "cpattn_version": (c_int, []),
     "cpattn_ring_attention": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                       c_int, c_int, c_int, c_int, c_int, P_INT, c_void_p]),

@@ -34,10 +34,16 @@ __all__ = [
 ]
 
 
+CPATTN_ERR_CUDA = 6
+
+
 class CpattnError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {status_string(status)} ({status})")
+        msg = f"{where}: {status_string(status)} ({status})"
+        if status == CPATTN_ERR_CUDA:
+            msg += " -- " + _native.load().cpattn_last_cuda_error_string().decode()
+        super().__init__(msg)
 
 
 def status_string(status: int) -> str:

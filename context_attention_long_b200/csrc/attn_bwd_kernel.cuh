@@ -93,37 +93,68 @@ constexpr uint32_t kBwdTmemCols = 512;
 // at [256, 256 + D) between them.
 __device__ __forceinline__ uint32_t bwd_dq_dp_col(int b) { return b ? 384u : 128u; }
 
-// Delta[b, h, s] = sum_d dO[b, s, h, d] * O[b, s, h, d], one warp per
-// (token, head) row: lanes read 8-byte pieces of both rows (coalesced).
-__global__ void __launch_bounds__(256) attn_bwd_delta_kernel(const __nv_bfloat16 *__restrict__ out,
-                                                             const __nv_bfloat16 *__restrict__ dout,
-                                                             float *__restrict__ delta, int B, int S, int H,
-                                                             int D) {
+// Delta[b, h, s] = sum_d dO[b, s, h, d] * O[b, s, h, d].  A (token, head) row
+// is D / 8 lanes, each on one 16-byte piece of both rows (coalesced); a warp
+// covers 32 / (D / 8) rows per pass and issues the loads of kDeltaPasses passes
+// before it reduces any of them, so that many rows' loads are in flight at
+// once.  The sum order is fixed: the result is deterministic.
+constexpr int kDeltaPasses = 4;
+__global__ void __launch_bounds__(256, 3) attn_bwd_delta_kernel(const __nv_bfloat16 *__restrict__ out,
+                                                                const __nv_bfloat16 *__restrict__ dout,
+                                                                float *__restrict__ delta, int B, int S, int H,
+                                                                int D) {
+  // Rows are (token, head) pairs, B*S*H < 2^31 (checked on the host).
   const int lane = threadIdx.x & 31;
-  const long long warp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const long long nwarps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
-  const long long nrows = static_cast<long long>(B) * S * H;
-  for (long long r = warp; r < nrows; r += nwarps) {
-    const __nv_bfloat16 *o = out + r * D;
-    const __nv_bfloat16 *g = dout + r * D;
-    float acc = 0.f;
-    for (int d = lane * 4; d < D; d += 128) {
-      const uint2 ov = __ldcs(reinterpret_cast<const uint2 *>(o + d));
-      const uint2 gv = __ldcs(reinterpret_cast<const uint2 *>(g + d));
-      const float2 o0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ov.x));
-      const float2 o1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ov.y));
-      const float2 g0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&gv.x));
-      const float2 g1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&gv.y));
-      acc = fmaf(o0.x, g0.x, fmaf(o0.y, g0.y, fmaf(o1.x, g1.x, fmaf(o1.y, g1.y, acc))));
-    }
+  const int lpr = D >> 3;                    // lanes per row (16 for D = 128, 8 for D = 64)
+  const int rpp = 32 / lpr;                  // rows per warp pass
+  const int sub = lane / lpr, piece = lane - sub * lpr;
+  const unsigned warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const unsigned nwarps = (gridDim.x * blockDim.x) >> 5;
+  const unsigned nrows = static_cast<unsigned>(B) * S * H;
+  const unsigned per_iter = static_cast<unsigned>(rpp) * kDeltaPasses;
+  for (unsigned r0 = warp * per_iter; r0 < nrows; r0 += nwarps * per_iter) {
+    uint4 ov[kDeltaPasses], gv[kDeltaPasses];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) {
-      const long long tok = r / H;
-      const int h = static_cast<int>(r - tok * H);
-      const int b = static_cast<int>(tok / S);
-      const int s = static_cast<int>(tok - static_cast<long long>(b) * S);
-      delta[(static_cast<long long>(b) * H + h) * S + s] = acc;
+    for (int u = 0; u < kDeltaPasses; ++u) {
+      const unsigned r = r0 + u * rpp + sub;
+      ov[u] = make_uint4(0u, 0u, 0u, 0u);
+      gv[u] = ov[u];
+      if (r < nrows) {
+        ov[u] = __ldcs(reinterpret_cast<const uint4 *>(out + static_cast<size_t>(r) * D) + piece);
+        gv[u] = __ldcs(reinterpret_cast<const uint4 *>(dout + static_cast<size_t>(r) * D) + piece);
+      }
+    }
+    // (token, head) of row r0 and (batch, position) of that token, once per
+    // iteration; each row below steps from them without dividing.
+    const unsigned tok0 = r0 / H;
+    const int h0 = static_cast<int>(r0 - tok0 * H);
+    const unsigned b0 = tok0 / S;
+    const int s0 = static_cast<int>(tok0 - b0 * S);
+#pragma unroll
+    for (int u = 0; u < kDeltaPasses; ++u) {
+      const uint32_t o4[4] = {ov[u].x, ov[u].y, ov[u].z, ov[u].w};
+      const uint32_t g4[4] = {gv[u].x, gv[u].y, gv[u].z, gv[u].w};
+      float acc = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 o = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&o4[e]));
+        const float2 g = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&g4[e]));
+        acc = fmaf(o.x, g.x, fmaf(o.y, g.y, acc));
+      }
+      for (int off = lpr >> 1; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      const unsigned r = r0 + u * rpp + sub;
+      if (piece == 0 && r < nrows) {
+        int h = h0 + u * rpp + sub, s = s0;
+        unsigned b = b0;
+        while (h >= H) {         // at most kDeltaPasses * rpp / H + 1 steps
+          h -= H;
+          if (++s == S) {
+            s = 0;
+            ++b;
+          }
+        }
+        delta[(static_cast<size_t>(b) * H + h) * S + s] = acc;
+      }
     }
   }
 }

@@ -12,6 +12,7 @@
 #include <climits>
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
 #include <cstdlib>
 #include <cstring>
 #include <memory>
@@ -58,6 +59,14 @@ static int check_attn_shape(int B, int H, int S, int D) {
   return CPATTN_OK;
 }
 
+// The backward also indexes its (token, head) rows in 32 bits: B*S*H < 2^31,
+// which any [B, S, H, D] bf16 tensor that fits in a device's memory meets.
+static int check_bwd_shape(int B, int H, int S, int D) {
+  const int st = check_attn_shape(B, H, S, D);
+  if (st != CPATTN_OK) return st;
+  return static_cast<long long>(B) * S * H >= (1ll << 31) ? CPATTN_ERR_SHAPE : CPATTN_OK;
+}
+
 // Equal split (NULL: total % degree == 0 required, [CP] variants table) or
 // explicit non-negative lengths summing to total ('anything' modes).
 static int resolve_splits(int total, int degree, const int *splits, std::vector<int> &out) {
@@ -84,20 +93,43 @@ static std::vector<int> prefix(const std::vector<int> &lens) {
   return off;
 }
 
+// The CUDA error behind the last CPATTN_ERR_CUDA this thread received, and
+// the step that failed (cpattn_last_cuda_error reports them).
+static thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+static thread_local const char *t_last_cuda_step = "";
+static int cuda_fail(cudaError_t e, const char *step) {
+  t_last_cuda_error = e == cudaSuccess ? cudaErrorUnknown : e;
+  t_last_cuda_step = step;
+  return CPATTN_ERR_CUDA;
+}
+static int cuda_result(cudaError_t e, const char *step) { return e == cudaSuccess ? CPATTN_OK : cuda_fail(e, step); }
+
 // Is the current device an sm_100 part?
 static int check_device(int *dev_out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) {
+  if (cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) {
     cudaGetLastError();
-    return CPATTN_ERR_CUDA;
+    return cuda_fail(e, "device query");
   }
   if (dev < 0 || dev >= kMaxDevices) return CPATTN_ERR_UNSUPPORTED;
+  // The tensor-map encoder is a driver call and needs a context current on
+  // this thread; runtime calls bind the primary context lazily, so a thread
+  // that has made none yet (torch's autograd engine thread, say) has none.
+  // cudaSetDevice binds it; once per thread and device.
+  static thread_local int t_bound_dev = -1;
+  if (t_bound_dev != dev) {
+    if (cudaError_t e = cudaSetDevice(dev); e != cudaSuccess) {
+      cudaGetLastError();
+      return cuda_fail(e, "binding the device's primary context");
+    }
+    t_bound_dev = dev;
+  }
   static std::atomic<int> cc_major[kMaxDevices];   // 0 = not queried yet
   int major = cc_major[dev].load(std::memory_order_relaxed);
   if (major == 0) {
-    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+    if (cudaError_t e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev); e != cudaSuccess) {
       cudaGetLastError();
-      return CPATTN_ERR_CUDA;
+      return cuda_fail(e, "device query");
     }
     cc_major[dev].store(major, std::memory_order_relaxed);
   }
@@ -105,6 +137,10 @@ static int check_device(int *dev_out) {
   if (dev_out) *dev_out = dev;
   return CPATTN_OK;
 }
+
+// What the last failed tensor-map encoding on this thread was given (the step
+// text of the CPATTN_ERR_CUDA it causes).
+static thread_local char t_encode_detail[256] = "tensor map encoding";
 
 static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
@@ -131,6 +167,12 @@ static bool encode_rows_map(CUtensorMap *tm, const void *ptr, int D, int H, long
   CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, es,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    std::snprintf(t_encode_detail, sizeof(t_encode_detail),
+                  "tensor map encoding (driver result %d; address %p, dims %llu x %llu x %llu, strides %llu, %llu)",
+                  static_cast<int>(r), ptr, static_cast<unsigned long long>(dims[0]),
+                  static_cast<unsigned long long>(dims[1]), static_cast<unsigned long long>(dims[2]),
+                  static_cast<unsigned long long>(strides[0]), static_cast<unsigned long long>(strides[1]));
   return r == CUDA_SUCCESS;
 }
 
@@ -146,6 +188,11 @@ static bool encode_matrix_map(CUtensorMap *tm, const void *ptr, long long rows, 
   CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, es,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    std::snprintf(t_encode_detail, sizeof(t_encode_detail),
+                  "tensor map encoding (driver result %d; address %p, dims %llu x %llu, stride %llu)",
+                  static_cast<int>(r), ptr, static_cast<unsigned long long>(dims[0]),
+                  static_cast<unsigned long long>(dims[1]), static_cast<unsigned long long>(strides[0]));
   return r == CUDA_SUCCESS;
 }
 
@@ -230,7 +277,7 @@ cudaError_t launch_attention_backward(const BwdParams &p, int D, const void *con
   int units = 0;
   for (int i = 0; i < p.n_prob; ++i) {
     const long long rows = static_cast<long long>(p.B) * p.S * p.prob[i].H;
-    attn_bwd_delta_kernel<<<grid_for(rows, 256 / 32), 256, 0, stream>>>(
+    attn_bwd_delta_kernel<<<grid_for(rows, (256 / 32) * (32 / (D / 8)) * kDeltaPasses), 256, 0, stream>>>(
         static_cast<const __nv_bfloat16 *>(outs[i]), static_cast<const __nv_bfloat16 *>(douts[i]), p.prob[i].delta,
         p.B, p.S, p.prob[i].H, D);
     cudaError_t e = cudaGetLastError();
@@ -418,7 +465,7 @@ static int run_attention(const std::vector<ProblemSpec> &probs, const std::vecto
     const long long rows_kv = ps.rows_kv > 0 ? ps.rows_kv : ps.rows;
     if (!encode_rows_map(&ap.tm_q, ps.q, D, ps.H, ps.rows) || !encode_rows_map(&ap.tm_k, ps.k, D, ps.H, rows_kv) ||
         !encode_rows_map(&ap.tm_v, ps.v, D, ps.H, rows_kv))
-      return CPATTN_ERR_CUDA;
+      return cuda_fail(cudaErrorInvalidValue, t_encode_detail);
     ap.out = ps.out;
     ap.lse = ps.lse;
     ap.prev = ps.prev;
@@ -462,7 +509,7 @@ static int run_attention(const std::vector<ProblemSpec> &probs, const std::vecto
   auto flush = [&]() -> int {
     close_group();
     if (P->total_units > 0) {
-      if (launch_attention(*P, D, out_f32, stream) != cudaSuccess) return CPATTN_ERR_CUDA;
+      if (cudaError_t e = launch_attention(*P, D, out_f32, stream); e != cudaSuccess) return cuda_fail(e, "attention launch");
     }
     reset();
     return CPATTN_OK;
@@ -662,17 +709,18 @@ static int projection_common(const void *a, const void *w, int B, int S, int H, 
   }
   for (int u = 0; u < degree; ++u)
     for (int h = ho[u]; h < ho[u + 1]; ++h) pp.head_rank[h] = static_cast<unsigned short>(u);
-  if (!encode_matrix_map(&pp.tm_w, w, pp.N, pp.K, kProjBN / 2)) return CPATTN_ERR_CUDA;
+  if (!encode_matrix_map(&pp.tm_w, w, pp.N, pp.K, kProjBN / 2)) return cuda_fail(cudaErrorInvalidValue, t_encode_detail);
   if (out_mode) {
     const char *base = static_cast<const char *>(a);
     for (int u = 0; u < degree; ++u) {
       const int Hu = ho[u + 1] - ho[u];
       if (Hu == 0) continue;
       const size_t off = static_cast<size_t>(B) * S * ho[u] * D * 2;
-      if (!encode_rows_map(&pp.tm_a[u], base + off, D, Hu, static_cast<long long>(B) * S)) return CPATTN_ERR_CUDA;
+      if (!encode_rows_map(&pp.tm_a[u], base + off, D, Hu, static_cast<long long>(B) * S))
+        return cuda_fail(cudaErrorInvalidValue, t_encode_detail);
     }
   } else if (!encode_matrix_map(&pp.tm_a[0], a, pp.M, pp.K, kProjBM)) {
-    return CPATTN_ERR_CUDA;
+    return cuda_fail(cudaErrorInvalidValue, t_encode_detail);
   }
   pp.timeout_ns = wait_timeout_ns();
   return CPATTN_OK;
@@ -784,7 +832,7 @@ int cpattn_lse_merge(const float *part_out, const float *part_lse, int P, int B,
   mp.H = H;
   mp.S = S;
   mp.D = D;
-  return launch_lse_merge(mp, stream) == cudaSuccess ? CPATTN_OK : CPATTN_ERR_CUDA;
+  return cuda_result(launch_lse_merge(mp, stream), "merge launch");
 }
 
 int cpattn_kv_gather_attention(const void *q, const void *k, const void *v, void *out, float *lse, int B, int H,
@@ -827,7 +875,7 @@ int cpattn_ulysses_permute(const void *x, void *y, int B, int S, int H, int D, i
   if (st != CPATTN_OK) return st;
   st = check_device(nullptr);
   if (st != CPATTN_OK) return st;
-  return launch_permute(pp, stream) == cudaSuccess ? CPATTN_OK : CPATTN_ERR_CUDA;
+  return cuda_result(launch_permute(pp, stream), "permute launch");
 }
 
 int cpattn_ulysses_permute_qkv(const void *q, const void *k, const void *v, void *yq, void *yk, void *yv, int B,
@@ -841,7 +889,7 @@ int cpattn_ulysses_permute_qkv(const void *q, const void *k, const void *v, void
   st = check_device(nullptr);
   if (st != CPATTN_OK) return st;
   set_qkv(pp, q, k, v, yq, yk, yv);
-  return launch_permute(pp, stream) == cudaSuccess ? CPATTN_OK : CPATTN_ERR_CUDA;
+  return cuda_result(launch_permute(pp, stream), "permute launch");
 }
 
 int cpattn_ulysses_unpermute(const void *y, void *x, int B, int S, int H, int D, int elem_bytes, int degree,
@@ -851,7 +899,7 @@ int cpattn_ulysses_unpermute(const void *y, void *x, int B, int S, int H, int D,
   if (st != CPATTN_OK) return st;
   st = check_device(nullptr);
   if (st != CPATTN_OK) return st;
-  return launch_permute(pp, stream) == cudaSuccess ? CPATTN_OK : CPATTN_ERR_CUDA;
+  return cuda_result(launch_permute(pp, stream), "permute launch");
 }
 
 // Head-sharded problems: head rank u's buffers start at element B*S*hoff_u*D.
@@ -961,7 +1009,7 @@ int cpattn_ulysses_qkv_projection(const void *x, const void *w_qkv, void *yq, vo
   pp.y[0] = yq;
   pp.y[1] = yk;
   pp.y[2] = yv;
-  return launch_projection(pp, stream) == cudaSuccess ? CPATTN_OK : CPATTN_ERR_CUDA;
+  return cuda_result(launch_projection(pp, stream), "projection launch");
 }
 
 int cpattn_ulysses_output_projection(const void *yo, const void *w_o, void *out, int B, int S, int H, int D, int Dm,
@@ -977,7 +1025,7 @@ int cpattn_ulysses_output_projection(const void *yo, const void *w_o, void *out,
   st = projection_common(yo, w_o, B, S, H, D, Dm, degree, seq_splits, head_splits, true, &pp, pp);
   if (st != CPATTN_OK) return st;
   pp.y[0] = out;
-  return launch_projection(pp, stream) == cudaSuccess ? CPATTN_OK : CPATTN_ERR_CUDA;
+  return cuda_result(launch_projection(pp, stream), "projection launch");
 }
 
 size_t cpattn_ulysses_workspace_bytes(int B, int H, int S, int D) {
@@ -1015,7 +1063,7 @@ static int ulysses_common(const void *q, const void *k, const void *v, void *out
   {
     PermuteParams pp = pq;
     set_qkv(pp, q, k, v, yq, yk, yv);
-    if (launch_permute(pp, stream) != cudaSuccess) return CPATTN_ERR_CUDA;
+    if (cudaError_t e = launch_permute(pp, stream); e != cudaSuccess) return cuda_fail(e, "permute launch");
   }
   // local attention of every head rank over all S tokens of its heads; the
   // second all-to-all is fused into its epilogue, which stores each output
@@ -1082,7 +1130,7 @@ static int unified_common(const void *q, const void *k, const void *v, void *out
     PermuteParams p1 = pp;
     set_qkv(p1, q, k, v, yq, yk, yv);
     p1.direction = 0;
-    if (launch_permute(p1, stream) != cudaSuccess) return CPATTN_ERR_CUDA;
+    if (cudaError_t e = launch_permute(p1, stream); e != cudaSuccess) return cuda_fail(e, "permute launch");
   }
   // Ring attention per head group over the chunks (rows B*off_i + b*len_i).
   std::vector<ProblemSpec> probs;
@@ -1277,7 +1325,7 @@ int cpattn_attention_backward(const void *q, const void *k, const void *v, const
   if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || lse == nullptr || dout == nullptr ||
       dq == nullptr || dk == nullptr || dv == nullptr)
     return CPATTN_ERR_NULL;
-  int st = check_attn_shape(B, H, S, D);
+  int st = check_bwd_shape(B, H, S, D);
   if (st != CPATTN_OK) return st;
   if (workspace == nullptr || workspace_bytes < cpattn_attention_backward_workspace_bytes(B, H, S))
     return CPATTN_ERR_WORKSPACE;
@@ -1291,11 +1339,11 @@ int cpattn_attention_backward(const void *q, const void *k, const void *v, const
   std::memset(P.get(), 0, sizeof(BwdParams));
   if (!backward_problem(P->prob[0], q, k, v, dout, lse, static_cast<long long>(H) * S, S, 0,
                         static_cast<float *>(workspace), dq, dk, dv, B, S, H, D, 0))
-    return CPATTN_ERR_CUDA;
+    return cuda_fail(cudaErrorInvalidValue, t_encode_detail);
   P->n_prob = 1;
   backward_common_params(*P, B, S, D, causal != 0);
   const void *outs[1] = {out}, *douts[1] = {dout};
-  return launch_attention_backward(*P, D, outs, douts, stream) == cudaSuccess ? CPATTN_OK : CPATTN_ERR_CUDA;
+  return cuda_result(launch_attention_backward(*P, D, outs, douts, stream), "backward launch");
 }
 
 size_t cpattn_ulysses_attention_backward_workspace_bytes(int B, int H, int S, int D) {
@@ -1311,7 +1359,7 @@ int cpattn_ulysses_attention_backward(const void *q, const void *k, const void *
   if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || lse == nullptr || dout == nullptr ||
       dq == nullptr || dk == nullptr || dv == nullptr)
     return CPATTN_ERR_NULL;
-  int st = check_attn_shape(B, H, S, D);
+  int st = check_bwd_shape(B, H, S, D);
   if (st != CPATTN_OK) return st;
   if (degree < 1 || degree > kMaxRanks) return CPATTN_ERR_DEGREE;
   std::vector<int> seq_chk, heads;
@@ -1340,13 +1388,13 @@ int cpattn_ulysses_attention_backward(const void *q, const void *k, const void *
   {
     PermuteParams pp = pq;
     set_qkv(pp, q, k, v, y[0], y[1], y[2]);
-    if (launch_permute(pp, stream) != cudaSuccess) return CPATTN_ERR_CUDA;
+    if (cudaError_t e = launch_permute(pp, stream); e != cudaSuccess) return cuda_fail(e, "permute launch");
     pp.src[0] = static_cast<const unsigned char *>(out);
     pp.dst[0] = static_cast<unsigned char *>(y[3]);
     pp.src[1] = static_cast<const unsigned char *>(dout);
     pp.dst[1] = static_cast<unsigned char *>(y[4]);
     pp.n_tensors = 2;
-    if (launch_permute(pp, stream) != cudaSuccess) return CPATTN_ERR_CUDA;
+    if (cudaError_t e = launch_permute(pp, stream); e != cudaSuccess) return cuda_fail(e, "permute launch");
   }
   // the backward of every head rank's local attention, one launch per kernel
   std::unique_ptr<BwdParams> P(new BwdParams);
@@ -1360,7 +1408,8 @@ int cpattn_ulysses_attention_backward(const void *q, const void *k, const void *
     if (n_prob == kMaxProblems) {   // a full parameter table: launch it and start the next
       P->n_prob = n_prob;
       backward_common_params(*P, B, S, D, causal != 0);
-      if (launch_attention_backward(*P, D, outs.data(), douts.data(), stream) != cudaSuccess) return CPATTN_ERR_CUDA;
+      if (cudaError_t e = launch_attention_backward(*P, D, outs.data(), douts.data(), stream); e != cudaSuccess)
+        return cuda_fail(e, "backward launch");
       std::memset(P.get(), 0, sizeof(BwdParams));
       outs.clear();
       douts.clear();
@@ -1372,7 +1421,7 @@ int cpattn_ulysses_attention_backward(const void *q, const void *k, const void *
     if (!backward_problem(P->prob[n_prob], at(0), at(1), at(2), at(4), lse, static_cast<long long>(H) * S, S, ho[u],
                           delta + static_cast<size_t>(B) * ho[u] * S, at(5), at(6), at(7), B, S, heads[u], D,
                           units))
-      return CPATTN_ERR_CUDA;
+      return cuda_fail(cudaErrorInvalidValue, t_encode_detail);
     outs.push_back(at(3));
     douts.push_back(at(4));
     units += B * heads[u] * nt;
@@ -1381,13 +1430,14 @@ int cpattn_ulysses_attention_backward(const void *q, const void *k, const void *
   if (n_prob > 0) {
     P->n_prob = n_prob;
     backward_common_params(*P, B, S, D, causal != 0);
-    if (launch_attention_backward(*P, D, outs.data(), douts.data(), stream) != cudaSuccess) return CPATTN_ERR_CUDA;
+    if (cudaError_t e = launch_attention_backward(*P, D, outs.data(), douts.data(), stream); e != cudaSuccess)
+      return cuda_fail(e, "backward launch");
   }
   // second all-to-all: dQ, dK, dV back to the sequence-sharded layout
   PermuteParams pb = pq;
   set_qkv(pb, y[5], y[6], y[7], dq, dk, dv);
   pb.direction = 1;
-  return launch_permute(pb, stream) == cudaSuccess ? CPATTN_OK : CPATTN_ERR_CUDA;
+  return cuda_result(launch_permute(pb, stream), "permute launch");
 }
 
 int cpattn_exchange_bytes(int mode, int B, int H, int S, int D, int elem_bytes, int degree, const int *seq_splits,
@@ -1508,12 +1558,22 @@ int cpattn_plan_exchange(int B, int H, int S, int D, int elem_bytes, int degree,
   return CPATTN_OK;
 }
 
+int cpattn_last_cuda_error(void) { return static_cast<int>(cpattn::t_last_cuda_error); }
+
+const char *cpattn_last_cuda_error_string(void) {
+  static thread_local char buf[256];
+  const cudaError_t e = cpattn::t_last_cuda_error;
+  if (e == cudaSuccess) return "no CUDA error recorded on this thread";
+  std::snprintf(buf, sizeof(buf), "%s: %s (%s)", cpattn::t_last_cuda_step, cudaGetErrorName(e), cudaGetErrorString(e));
+  return buf;
+}
+
 int cpattn_device_status(cpattn_stream_t stream, unsigned int *code) {
   if (code == nullptr) return CPATTN_ERR_NULL;
   int st = check_device(nullptr);
   if (st != CPATTN_OK) return st;
   unsigned int v = 0;
-  if (read_and_clear_device_status(&v, stream) != cudaSuccess) return CPATTN_ERR_CUDA;
+  if (cudaError_t e = read_and_clear_device_status(&v, stream); e != cudaSuccess) return cuda_fail(e, "status read");
   *code = v;
   return v == 0 ? CPATTN_OK : CPATTN_ERR_DEVICE_TIMEOUT;
 }
@@ -1522,9 +1582,8 @@ int cpattn_debug_wait_timeout(unsigned int timeout_us, cpattn_stream_t stream) {
   if (timeout_us < 1 || timeout_us > 1000000) return CPATTN_ERR_SHAPE;
   int st = check_device(nullptr);
   if (st != CPATTN_OK) return st;
-  return launch_debug_wait(static_cast<unsigned long long>(timeout_us) * 1000ull, stream) == cudaSuccess
-             ? CPATTN_OK
-             : CPATTN_ERR_CUDA;
+  return cuda_result(launch_debug_wait(static_cast<unsigned long long>(timeout_us) * 1000ull, stream),
+                     "debug wait launch");
 }
 
 }  // extern "C"
@@ -1543,9 +1602,9 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[CPATTN_NOALLOC_
 
 static int noalloc_scratch_address(void **out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) {
+  if (cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) {
     cudaGetLastError();
-    return CPATTN_ERR_CUDA;
+    return cuda_fail(e, "device query");
   }
   if (dev < 0 || dev >= kMaxDevices) return CPATTN_ERR_UNSUPPORTED;
   static std::mutex mu;
@@ -1553,9 +1612,9 @@ static int noalloc_scratch_address(void **out) {
   std::lock_guard<std::mutex> lock(mu);
   if (addr[dev] == nullptr) {
     void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+    if (cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch); e != cudaSuccess || p == nullptr) {
       cudaGetLastError();
-      return CPATTN_ERR_CUDA;
+      return cuda_fail(e, "scratch symbol lookup");
     }
     addr[dev] = p;
   }

@@ -34,7 +34,10 @@
  * Contexts.  The library keeps per-device state for the life of the process
  *   (kernel attributes set on first use, cluster sizes, the no-allocation
  *   scratch address): use it under each device's primary context, the one the
- *   CUDA runtime uses, and not across a cudaDeviceReset.
+ *   CUDA runtime uses, and not across a cudaDeviceReset.  An entry point
+ *   called on a thread that has no context current yet (a worker thread that
+ *   made no CUDA call) binds the current device's primary context to that
+ *   thread (cudaSetDevice) before it encodes any tensor map.
  * Memory.  All tensor pointers are DEVICE pointers owned by the caller; the
  *   library allocates no device memory on any call (workspaces come from the
  *   caller; cpattn_ulysses_attention_noalloc uses a static scratch).  Length/split arrays are HOST arrays read only
@@ -81,6 +84,17 @@ typedef enum {
 
 /* Human-readable name of a status code; never NULL. */
 const char *cpattn_status_string(int status);
+
+/*
+ * The CUDA error behind the last CPATTN_ERR_CUDA returned on the calling
+ * thread (a cudaError_t value; 0 if none was recorded), and a description of
+ * it, "<step>: <error name> (<error string>)", where <step> names what failed
+ * (a kernel launch, a device query, a tensor-map encoding, ...).  The string
+ * is thread-local and stays valid until the thread's next call of this
+ * function; never NULL.  Neither call touches the device.
+ */
+int cpattn_last_cuda_error(void);
+const char *cpattn_last_cuda_error_string(void);
 
 /* Library ABI version (major * 10000 + minor * 100 + patch). */
 int cpattn_version(void);
@@ -477,8 +491,9 @@ int cpattn_causal_unified_attention(const void *q, const void *k, const void *v,
  *                       bytes, 4-byte aligned (holds rowsum(dO * O)).
  * Three launches on `stream`: the row sums, a dQ kernel (one CTA per Q tile,
  * walking the K/V tiles) and a dK/dV kernel (one CTA per K/V tile, walking the
- * Q tiles); no atomics.  Errors: NULL, SHAPE, WORKSPACE, ALIGNMENT,
- * UNSUPPORTED, CUDA.
+ * Q tiles); no atomics.  Errors: NULL, SHAPE (also when B*S*H >= 2^31, a
+ * tensor larger than any device memory), WORKSPACE, ALIGNMENT, UNSUPPORTED,
+ * CUDA.
  */
 size_t cpattn_attention_backward_workspace_bytes(int B, int H, int S);
 int cpattn_attention_backward(const void *q, const void *k, const void *v, const void *out,
@@ -501,8 +516,8 @@ int cpattn_attention_backward(const void *q, const void *k, const void *v, const
  *   workspace           device, 16-byte aligned, at least
  *                       cpattn_ulysses_attention_backward_workspace_bytes()
  *                       = 16 * B*S*H*D + 4 * B*H*S bytes.
- * Other arguments, splits and errors as cpattn_ulysses_attention; causal = 1
- * for the causal mask.
+ * Other arguments, splits and errors as cpattn_ulysses_attention (SHAPE also
+ * when B*S*H >= 2^31); causal = 1 for the causal mask.
  */
 size_t cpattn_ulysses_attention_backward_workspace_bytes(int B, int H, int S, int D);
 int cpattn_ulysses_attention_backward(const void *q, const void *k, const void *v,

@@ -207,8 +207,21 @@ def test_debug_hook_validation(lib):
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
 def test_valid_call_without_gpu_reports_cuda_error(lib):
     # Arguments pass validation; with no device the call must return
-    # CPATTN_ERR_CUDA before launching anything.
+    # CPATTN_ERR_CUDA before launching anything, and record on this thread
+    # which CUDA call failed and why.
     assert _ring(lib) == CUDA
+    assert lib.cpattn_last_cuda_error() != 0
+    assert lib.cpattn_last_cuda_error_string().decode().startswith("device query: cudaError")
+
+
+def test_last_cuda_error_is_thread_local(lib):
+    import threading
+    seen = []
+    t = threading.Thread(target=lambda: seen.append((lib.cpattn_last_cuda_error(),
+                                                     lib.cpattn_last_cuda_error_string().decode())))
+    t.start()
+    t.join()
+    assert seen == [(0, "no CUDA error recorded on this thread")]
 
 
 def test_causal_entry_points_validate_like_their_namesakes(lib):
@@ -246,6 +259,8 @@ def test_backward_validation(lib):
     assert f(lse=None) == NULL
     assert f(D=96) == SHAPE
     assert f(S=0) == SHAPE
+    # B*S*H >= 2^31 (here 2 heads x 2^30 tokens): rows are indexed in 32 bits
+    assert f(S=1 << 30, nbytes=1 << 40) == SHAPE
     assert f(ws=None) == WS
     assert f(nbytes=need - 4) == WS
     assert f(dq=FAKE_MIS) == ALIGN
