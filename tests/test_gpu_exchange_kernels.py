@@ -256,6 +256,11 @@ def test_exchange_module_runs_its_cuda_path_on_one_rank():
         rg, ug = exchange.unified_groups(1, 1)
         o, l = exchange.unified_attention(q, k, v, rg, ug)
         assert_close(f64_of(o), f64_of(l), f64_of(ref_o), f64_of(ref_l), "unified")
+        # the configuration object's dispatch (ContextParallelConfig semantics)
+        from context_attention_long_b200.parallel import ContextParallel, ContextParallelConfig
+        for method in ("allgather", "p2p"):
+            o, l = ContextParallel(ContextParallelConfig(rotate_method=method)).attention(q, k, v, return_lse=True)
+            assert_close(f64_of(o), f64_of(l), f64_of(ref_o), f64_of(ref_l), f"config {method}")
         torch.cuda.synchronize()
         _no_timeouts()
     finally:
