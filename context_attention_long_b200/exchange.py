@@ -89,6 +89,9 @@ class CudaKernels:
     def unpermute(self, y, B, S, H, D, degree, seq_splits, head_splits):
         return api.cpattn_ulysses_unpermute(y, B, S, H, D, degree, seq_splits, head_splits)
 
+    def backward(self, q, k, v, out, lse, dout, causal):
+        return api.cpattn_attention_backward(q, k, v, out, lse, dout, causal)
+
 
 def _bytes(t: torch.Tensor) -> torch.Tensor:
     return t.reshape(-1).view(torch.uint8)
@@ -222,10 +225,12 @@ def _ulysses_to_heads(tensors, group, seq, heads, kernels):
     B, Sr, H, D = tensors[0].shape
     S, Hr = sum(seq), heads[r]
     pack_seq = [Sr] + [0] * (P - 1)          # all local tokens as "rank 0"
-    if Sr:
+    if not Sr:
+        packed = [torch.empty(0, dtype=tensors[0].dtype, device=tensors[0].device)] * len(tensors)
+    elif len(tensors) == 3:
         packed = kernels.permute_qkv(*tensors, B, Sr, H, D, P, pack_seq, heads)
     else:
-        packed = [torch.empty(0, dtype=tensors[0].dtype, device=tensors[0].device)] * 3
+        packed = [kernels.permute(x, B, Sr, H, D, P, pack_seq, heads) for x in tensors]
     send_splits = [B * Sr * heads[u] * D for u in range(P)]
     recv_splits = [B * seq[u] * Hr * D for u in range(P)]
     out = []
@@ -271,6 +276,77 @@ def ulysses_attention(q, k, v, group=None, seq_splits=None, head_splits=None, ca
     else:
         yo, lse = yq, torch.empty((B, 0, S), dtype=torch.float32, device=q.device)
     return _ulysses_to_tokens(yo, group, seq, heads, B, H, D, kernels), lse
+
+
+# ---------------------------------------------------- Ulysses, training
+
+def _heads_dense(y, B, S, Hr, D, P, seq, kernels):
+    """Head-side rank buffers (B, S_u, H_r, D), concatenated -> (B, S, H_r, D).
+    For B = 1 the two layouts are the same bytes."""
+    if B == 1 or not Hr or not S:
+        return y.view(B, S, Hr, D)
+    return kernels.permute(y, B, S, Hr, D, P, seq, [Hr] + [0] * (P - 1)).view(B, S, Hr, D)
+
+
+def _heads_rank_buffers(x, B, S, Hr, D, P, seq, kernels):
+    """The inverse of _heads_dense."""
+    if B == 1 or not Hr or not S:
+        return x.reshape(-1)
+    return kernels.unpermute(x.reshape(-1), B, S, Hr, D, P, seq, [Hr] + [0] * (P - 1))
+
+
+class UlyssesAttentionFunction(torch.autograd.Function):
+    """Ulysses attention over the ranks of a group, differentiable ("Ulysses
+    Sequence Parallelism" article, sections 1, 4 and 7: training over long
+    contexts).  The forward is ulysses_attention's and keeps the head-side Q,
+    K, V and output.  The backward sends dO through the same all-to-all, runs
+    the attention backward on this rank's heads over every token, and sends
+    dQ, dK and dV back through the inverse all-to-all."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, group, seq, heads, causal, kernels):
+        P, r = _group_rank(group)
+        B, Sr, H, D = _shape4(q)
+        S, Hr = sum(seq), heads[r]
+        yq, yk, yv = _ulysses_to_heads((q, k, v), group, seq, heads, kernels)
+        if Hr:
+            yo, lse = kernels.rank_buffer(yq, yk, yv, B, S, Hr, D, P, seq, causal)
+        else:
+            yo, lse = yq, torch.empty((B, 0, S), dtype=torch.float32, device=q.device)
+        ctx.save_for_backward(yq, yk, yv, yo, lse)
+        ctx.meta = (group, list(seq), list(heads), bool(causal), kernels, (B, Sr, H, D))
+        return _ulysses_to_tokens(yo, group, seq, heads, B, H, D, kernels)
+
+    @staticmethod
+    def backward(ctx, dout):
+        yq, yk, yv, yo, lse = ctx.saved_tensors
+        group, seq, heads, causal, kernels, (B, Sr, H, D) = ctx.meta
+        P, r = _group_rank(group)
+        S, Hr = sum(seq), heads[r]
+        (ydo,) = _ulysses_to_heads((dout.contiguous(),), group, seq, heads, kernels)
+        grads = []
+        if Hr and S:
+            dense = [_heads_dense(y, B, S, Hr, D, P, seq, kernels) for y in (yq, yk, yv, yo, ydo)]
+            dqh, dkh, dvh = kernels.backward(dense[0], dense[1], dense[2], dense[3], lse, dense[4], causal)
+            grads = [_heads_rank_buffers(g, B, S, Hr, D, P, seq, kernels) for g in (dqh, dkh, dvh)]
+        else:
+            grads = [torch.empty(0, dtype=yq.dtype, device=yq.device)] * 3
+        dq, dk, dv = (_ulysses_to_tokens(g, group, seq, heads, B, H, D, kernels) for g in grads)
+        return dq, dk, dv, None, None, None, None, None
+
+
+def ulysses_attention_trainable(q, k, v, group=None, seq_splits=None, head_splits=None, causal=False, kernels=None):
+    """ulysses_attention as an autograd function: returns out (B, S_r, H, D)
+    bf16 whose gradient flows back to this rank's q, k and v.  Arguments as
+    ulysses_attention's; every rank of the group must run the backward."""
+    kernels = kernels or CudaKernels()
+    P, r = _group_rank(group)
+    B, Sr, H, D = _shape4(q)
+    seq = list(seq_splits) if seq_splits is not None else [Sr] * P
+    heads = list(head_splits) if head_splits is not None else equal_splits(H, P)
+    if len(seq) != P or seq[r] != Sr or len(heads) != P or sum(heads) != H:
+        raise ValueError("splits must have one entry per rank; seq_splits[rank] must be this rank's length")
+    return UlyssesAttentionFunction.apply(q, k, v, group, seq, heads, causal, kernels)
 
 
 # -------------------------------------------------------------- kv_gather

@@ -150,12 +150,28 @@ class ContextParallel:
         float32 LSE that the variant's exchange returns (ring: (B, H, S_r);
         Ulysses: (B, H_r, S) of this rank's heads; unified: (B, H_j, S_i) of
         this rank's head group over its ring chunk).  head_splits: the heads
-        of each Ulysses rank under ulysses_anything (None: front-loaded)."""
+        of each Ulysses rank under ulysses_anything (None: front-loaded).
+        When q, k or v requires a gradient, the Ulysses variant (or a single
+        rank) returns an output that autograd differentiates across the
+        ranks; the ring and unified variants then raise NotImplementedError."""
         cfg = self.config
         B, Sr, H, D = q.shape
+        training = torch.is_grad_enabled() and any(t.requires_grad for t in (q, k, v))
         lens = self._lengths(Sr)
         S = sum(sum(x) for x in lens) if cfg.variant == "unified" else sum(lens)
-        cfg.check(S, H, training=torch.is_grad_enabled() and q.requires_grad)
+        cfg.check(S, H, training=training)
+        if training:
+            # Gradients cross GPUs through the Ulysses exchange (the all-to-alls
+            # run backwards); the ring and unified exchanges are forward only.
+            if cfg.variant not in ("none", "ulysses") or return_lse:
+                raise NotImplementedError("training across GPUs goes through the Ulysses exchange "
+                                          "(ring_degree == 1), without return_lse")
+            heads = None
+            if cfg.ulysses_anything:
+                heads = list(head_splits) if head_splits is not None else exchange.front_loaded_splits(
+                    H, cfg.ulysses_degree)
+            return exchange.ulysses_attention_trainable(q, k, v, self.ulysses_group, lens, heads, causal,
+                                                        kernels=self.kernels)
         if cfg.variant in ("none", "ring"):
             out, lse = exchange.ring_attention(q, k, v, self.ring_group, lens, causal, cfg.rotate_method,
                                                kernels=self.kernels)

@@ -72,3 +72,7 @@ class OracleKernels:
 
     def unpermute(self, y, B, S, H, D, degree, seq_splits, head_splits):
         return self._from_bits(oracle.ulysses_unpermute(self._bits(y), B, S, H, D, degree, seq_splits, head_splits))
+
+    def backward(self, q, k, v, out, lse, dout, causal):
+        grads = oracle.attention_backward(_f64(q), _f64(k), _f64(v), _f64(dout), causal=causal)
+        return tuple(torch.from_numpy(g).to(torch.bfloat16) for g in grads)

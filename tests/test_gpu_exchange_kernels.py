@@ -256,6 +256,20 @@ def test_exchange_module_runs_its_cuda_path_on_one_rank():
         rg, ug = exchange.unified_groups(1, 1)
         o, l = exchange.unified_attention(q, k, v, rg, ug)
         assert_close(f64_of(o), f64_of(l), f64_of(ref_o), f64_of(ref_l), "unified")
+        # the differentiable Ulysses exchange: its gradients against the
+        # single-GPU backward of the same tensors
+        rng = np.random.Generator(np.random.PCG64(78))
+        dout = to_dev(inputs.f32_to_bf16_bits(rng.standard_normal((B, S, H, D)).astype(np.float32)))
+        for causal in (False, True):
+            qq, kk, vv = (x.clone().requires_grad_(True) for x in (q, k, v))
+            o = exchange.ulysses_attention_trainable(qq, kk, vv, causal=causal)
+            o.backward(dout)
+            ro, rl = (api.cpattn_causal_ring_attention if causal else api.cpattn_ring_attention)(q, k, v, 1)
+            refs = api.cpattn_attention_backward(q, k, v, ro, rl, dout, causal)
+            for name, got, ref in zip(("dq", "dk", "dv"), (qq.grad, kk.grad, vv.grad), refs):
+                gref = f64_of(ref)
+                err = np.abs(f64_of(got) - gref)
+                assert err.max() <= 2e-2 * np.abs(gref).max(), f"trainable {name} causal={causal}"
         # the configuration object's dispatch (ContextParallelConfig semantics)
         from context_attention_long_b200.parallel import ContextParallel, ContextParallelConfig
         for method in ("allgather", "p2p"):

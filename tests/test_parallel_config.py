@@ -114,6 +114,34 @@ def _cases(world, rank):
         err = np.abs(out.double().numpy() - ref_o[:, a:b])
         assert err.size == 0 or (err.max() <= 2e-2 and err.mean() <= 2e-3), f"{cfg}: {err.max():.3e}"
 
+    def train(cfg, B, H, D, lens, causal, seed, head_splits=None):
+        """The gradients autograd delivers to this rank's shard against the
+        oracle's backward over the full sequence."""
+        S = sum(lens)
+        qb, kb, vb = inputs.make_qkv(B, S, H, D, seed, D == 128)
+        rng = np.random.Generator(np.random.PCG64(seed + 1))
+        dob = inputs.f32_to_bf16_bits(rng.standard_normal((B, S, H, D)).astype(np.float32))
+        off = np.concatenate([[0], np.cumsum(lens)]).astype(int)
+        a, b = off[rank], off[rank + 1]
+        q, k, v = (bf16(x[:, a:b]).requires_grad_(True) for x in (qb, kb, vb))
+        cp = ContextParallel(cfg, kernels=OracleKernels())
+        out = cp.attention(q, k, v, causal=causal, head_splits=head_splits)
+        out.backward(bf16(dob[:, a:b]))
+        refs = oracle.attention_backward(*(inputs.bf16_bits_to_f64(x) for x in (qb, kb, vb, dob)), causal=causal)
+        for name, t, ref in zip(("dq", "dk", "dv"), (q, k, v), refs):
+            r = ref[:, a:b]
+            g = max(np.max(np.abs(ref)), 1e-30)
+            err = np.abs(t.grad.double().numpy() - r)
+            assert err.size == 0 or (err.max() <= 2e-2 * g and err.mean() <= 2e-3 * g), f"{name} {cfg}"
+
+    def refuse_training(cfg, B, H, D, lens):
+        """No silent gradient-free output: the ring exchange is forward only."""
+        qb, kb, vb = inputs.make_qkv(B, sum(lens), H, D, 19, D == 128)
+        a, b = sum(lens[:rank]), sum(lens[:rank + 1])
+        q, k, v = (bf16(x[:, a:b]).requires_grad_(True) for x in (qb, kb, vb))
+        with pytest.raises(NotImplementedError):
+            ContextParallel(cfg, kernels=OracleKernels()).attention(q, k, v)
+
     C = ContextParallelConfig
     if world == 2:
         return [
@@ -124,12 +152,18 @@ def _cases(world, rank):
             ("ulysses", lambda: run(C(ulysses_degree=2), 2, 4, 64, [64, 64], True, 15)),
             ("ulysses anything", lambda: run(C(ulysses_degree=2, ulysses_anything=True), 1, 3, 64, [77, 50], False,
                                              16, head_splits=[2, 1])),
+            ("ulysses training", lambda: train(C(ulysses_degree=2), 2, 4, 64, [48, 48], True, 17)),
+            ("ulysses anything training", lambda: train(C(ulysses_degree=2, ulysses_anything=True), 1, 3, 64, [40, 29],
+                                                       False, 18, head_splits=[2, 1])),
+            ("ring training refused", lambda: refuse_training(C(ring_degree=2), 1, 2, 64, [32, 32])),
         ]
     return [
         ("unified 2x2", lambda: run(C(ring_degree=2, ulysses_degree=2), 1, 4, 64, [40, 40, 40, 40], False, 21)),
         ("unified 2x2 causal p2p", lambda: run(C(ring_degree=2, ulysses_degree=2, rotate_method="p2p"), 2, 2, 64,
                                                [32, 32, 32, 32], True, 22)),
         ("ring 4", lambda: run(C(ring_degree=4, rotate_method="p2p"), 1, 2, 128, [50, 50, 50, 50], True, 23)),
+        ("ulysses 4 training, an empty head rank", lambda: train(C(ulysses_degree=4, ulysses_anything=True), 2, 3, 64,
+                                                               [20, 0, 30, 25], True, 24, head_splits=[1, 1, 0, 1])),
     ]
 
 
