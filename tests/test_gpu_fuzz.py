@@ -87,3 +87,38 @@ def test_fuzz_ulysses_and_unified(i):
     assert st == 0, f"{what}: device wait expired {code:#x}"
     assert_close(rank_buffers_to_full(f64_of(uo), B, S, H, D, seq), f64_of(ul), ref_o, ref_l, what + " ulysses")
     assert_close(f64_of(fo), f64_of(fl), ref_o, ref_l, what + f" unified R{R} ring_lens={ring_lens}")
+
+
+def _bwd_case(i):
+    rng = np.random.Generator(np.random.PCG64(9500 + i))
+    B = int(rng.integers(1, 3))
+    H = int(rng.integers(1, 5))
+    S = int(rng.integers(1, 700))
+    D = int(rng.choice([64, 128]))
+    causal = bool(rng.random() < 0.5)
+    return B, H, S, D, causal
+
+
+@pytest.mark.parametrize("i", range(32))
+def test_fuzz_backward(i):
+    """The attention backward on seeded random shapes (walks of 1 to 6 tiles,
+    shorter than and past the three-stage load ring, ragged tails) against
+    the fp64 backward oracle, each gradient relative to its largest entry."""
+    B, H, S, D, causal = _bwd_case(i)
+    qb, kb, vb = inputs.make_qkv(B, S, H, D, 9600 + i, D == 128)
+    rng = np.random.Generator(np.random.PCG64(9700 + i))
+    dob = inputs.f32_to_bf16_bits(rng.standard_normal((B, S, H, D)).astype(np.float32))
+    dq_, dk_, dv_, do_ = (to_dev(x) for x in (qb, kb, vb, dob))
+    fwd = api.cpattn_causal_ring_attention if causal else api.cpattn_ring_attention
+    out, lse = fwd(dq_, dk_, dv_, 1)
+    grads = api.cpattn_attention_backward(dq_, dk_, dv_, out, lse, do_, causal=causal)
+    torch.cuda.synchronize()
+    st, code = api.cpattn_device_status()
+    what = f"case {i}: B{B} H{H} S{S} D{D} causal={causal}"
+    assert st == 0, f"{what}: device wait expired {code:#x}"
+    refs = oracle.attention_backward(*(inputs.bf16_bits_to_f64(x) for x in (qb, kb, vb, dob)), causal=causal)
+    for name, got, ref in zip(("dq", "dk", "dv"), grads, refs):
+        g = max(np.max(np.abs(ref)), 1e-30)
+        err = np.abs(f64_of(got) - ref)
+        assert np.all(np.isfinite(f64_of(got))), f"{what} {name}: non-finite"
+        assert err.max() <= 2e-2 * g and err.mean() <= 2e-3 * g, f"{what} {name}: max-abs {err.max():.3e} vs {g:.3e}"
