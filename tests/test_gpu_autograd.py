@@ -23,8 +23,9 @@ def _built():
     build.build()
 
 
-def _grad_close(got, ref, what):
-    g = max(np.max(np.abs(ref)), 1e-30)
+def _grad_close(got, ref, what, dout_max=1.0):
+    # floored at 2^-10 of max|dO|: a single visible key makes dQ = dK = 0 exactly
+    g = max(np.max(np.abs(ref)), 2.0 ** -10 * dout_max, 1e-30)
     err = np.abs(np.asarray(got, dtype=np.float64) - ref)
     assert np.all(np.isfinite(got)), f"{what}: non-finite"
     assert err.max() <= 2e-2 * g, f"{what}: max-abs {err.max():.3e} vs {g:.3e}"
@@ -54,7 +55,8 @@ def test_ring_attention_autograd_matches_oracle(B, S, H, D, P, lens, causal):
     torch.cuda.synchronize()
     refs = oracle.attention_backward(*(inputs.bf16_bits_to_f64(x) for x in (qb, kb, vb, dob)), causal=causal)
     for name, t, ref in zip(("dq", "dk", "dv"), (q, k, v), refs):
-        _grad_close(f64_of(t.grad), ref, f"ring {name} S{S} P{P} causal={causal}")
+        _grad_close(f64_of(t.grad), ref, f"ring {name} S{S} P{P} causal={causal}",
+                    np.abs(inputs.bf16_bits_to_f64(dob)).max())
     st, code = api.cpattn_device_status()
     assert st == 0 and code == 0
 
@@ -73,6 +75,6 @@ def test_ulysses_attention_autograd_matches_oracle(B, S, H, D, P, seq, heads, ca
     refs = oracle.attention_backward(*(inputs.bf16_bits_to_f64(x) for x in (qb, kb, vb, dob)), causal=causal)
     for name, t, ref in zip(("dq", "dk", "dv"), (q, k, v), refs):
         _grad_close(rank_buffers_to_full(f64_of(t.grad), B, S, H, D, seq_l), ref,
-                    f"ulysses {name} S{S} P{P} causal={causal}")
+                    f"ulysses {name} S{S} P{P} causal={causal}", np.abs(inputs.bf16_bits_to_f64(dob)).max())
     st, code = api.cpattn_device_status()
     assert st == 0 and code == 0

@@ -33,10 +33,15 @@ def _no_timeouts():
     assert st == 0 and code == 0, f"device wait expired: code {code:#x}"
 
 
-def assert_grad_close(got, ref, what):
+def assert_grad_close(got, ref, what, dout_max=1.0):
+    """Relative to the largest reference entry g, floored at 2^-10 of the
+    upstream gradient's largest entry: a query with a single visible key has
+    dQ = dK = 0 exactly (the softmax of one score is constant), and the fp32
+    sums dO.V and rowsum(dO*O) then leave rounding residues far below the
+    bf16 resolution of any gradient entry of dO's order."""
     got, ref = np.asarray(got, dtype=np.float64), np.asarray(ref, dtype=np.float64)
     assert np.all(np.isfinite(got)), f"{what}: non-finite"
-    g = max(np.max(np.abs(ref)), 1e-30)
+    g = max(np.max(np.abs(ref)) if ref.size else 0.0, 2.0 ** -10 * dout_max, 1e-30)
     err = np.abs(got - ref)
     assert err.max() <= 2e-2 * g, f"{what}: max-abs {err.max():.3e} vs {g:.3e}"
     assert err.mean() <= 2e-3 * g, f"{what}: mean-abs {err.mean():.3e} vs {g:.3e}"
@@ -63,7 +68,7 @@ def test_backward_matches_oracle(B, S, H, D, causal):
     q, k, v, do = (inputs.bf16_bits_to_f64(x) for x in bits)
     refs = oracle.attention_backward(q, k, v, do, causal=causal)
     for name, got, ref in zip(("dq", "dk", "dv"), grads, refs):
-        assert_grad_close(f64_of(got), ref, f"{name} B{B} S{S} H{H} D{D} causal={causal}")
+        assert_grad_close(f64_of(got), ref, f"{name} B{B} S{S} H{H} D{D} causal={causal}", np.abs(do).max())
 
 
 @pytest.mark.parametrize("causal", [False, True])
@@ -85,7 +90,8 @@ def test_backward_dit_workload_sampled_heads(causal):
         ref = oracle.attention_backward_rows(*(inputs.bf16_bits_to_f64(x[0, :, h]) for x in (qb, kb, vb, dob)),
                                              pos, pos)
         for name, got, r in zip(("dq", "dk", "dv"), (dq, dk, dv), ref):
-            assert_grad_close(f64_of(got)[0, :, h], r, f"dit {name} head {h} causal={causal}")
+            assert_grad_close(f64_of(got)[0, :, h], r, f"dit {name} head {h} causal={causal}",
+                              np.abs(inputs.bf16_bits_to_f64(dob)).max())
 
 
 def test_backward_is_deterministic_and_validates():
@@ -121,4 +127,5 @@ def test_ulysses_backward_matches_oracle(B, S, H, D, P, seq, heads, causal):
     refs = oracle.attention_backward(*(inputs.bf16_bits_to_f64(x) for x in (qb, kb, vb, dob)), causal=causal)
     for name, got, ref in zip(("dq", "dk", "dv"), (dq, dk, dv), refs):
         full = rank_buffers_to_full(f64_of(got), B, S, H, D, seq_l)
-        assert_grad_close(full, ref, f"ulysses {name} B{B} S{S} H{H} P{P} causal={causal}")
+        assert_grad_close(full, ref, f"ulysses {name} B{B} S{S} H{H} P{P} causal={causal}",
+                          np.abs(inputs.bf16_bits_to_f64(dob)).max())

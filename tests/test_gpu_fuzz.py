@@ -117,8 +117,10 @@ def test_fuzz_backward(i):
     what = f"case {i}: B{B} H{H} S{S} D{D} causal={causal}"
     assert st == 0, f"{what}: device wait expired {code:#x}"
     refs = oracle.attention_backward(*(inputs.bf16_bits_to_f64(x) for x in (qb, kb, vb, dob)), causal=causal)
+    dmax = np.abs(inputs.bf16_bits_to_f64(dob)).max()
     for name, got, ref in zip(("dq", "dk", "dv"), grads, refs):
-        g = max(np.max(np.abs(ref)), 1e-30)
+        # floored at 2^-10 of max|dO|: a single visible key makes dQ = dK = 0 exactly
+        g = max(np.max(np.abs(ref)), 2.0 ** -10 * dmax, 1e-30)
         err = np.abs(f64_of(got) - ref)
         assert np.all(np.isfinite(f64_of(got))), f"{what} {name}: non-finite"
         assert err.max() <= 2e-2 * g and err.mean() <= 2e-3 * g, f"{what} {name}: max-abs {err.max():.3e} vs {g:.3e}"
