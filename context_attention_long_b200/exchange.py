@@ -321,18 +321,73 @@ class UlyssesAttentionFunction(torch.autograd.Function):
     def backward(ctx, dout):
         yq, yk, yv, yo, lse = ctx.saved_tensors
         group, seq, heads, causal, kernels, (B, Sr, H, D) = ctx.meta
-        P, r = _group_rank(group)
-        S, Hr = sum(seq), heads[r]
-        (ydo,) = _ulysses_to_heads((dout.contiguous(),), group, seq, heads, kernels)
-        grads = []
-        if Hr and S:
-            dense = [_heads_dense(y, B, S, Hr, D, P, seq, kernels) for y in (yq, yk, yv, yo, ydo)]
-            dqh, dkh, dvh = kernels.backward(dense[0], dense[1], dense[2], dense[3], lse, dense[4], causal)
-            grads = [_heads_rank_buffers(g, B, S, Hr, D, P, seq, kernels) for g in (dqh, dkh, dvh)]
-        else:
-            grads = [torch.empty(0, dtype=yq.dtype, device=yq.device)] * 3
-        dq, dk, dv = (_ulysses_to_tokens(g, group, seq, heads, B, H, D, kernels) for g in grads)
+        dq, dk, dv = _ulysses_backward(yq, yk, yv, yo, lse, dout, group, seq, heads, causal, kernels, B, H, D)
         return dq, dk, dv, None, None, None, None, None
+
+
+def _ulysses_backward(yq, yk, yv, yo, lse, dout, group, seq, heads, causal, kernels, B, H, D):
+    """dQ, dK, dV of this rank's token shard from the head-side Q, K, V,
+    output and LSE of its heads: dO through the first all-to-all, the
+    attention backward on the heads over every token, the gradients through
+    the inverse all-to-all."""
+    P, r = _group_rank(group)
+    S, Hr = sum(seq), heads[r]
+    (ydo,) = _ulysses_to_heads((dout.contiguous(),), group, seq, heads, kernels)
+    if Hr and S:
+        dense = [_heads_dense(y, B, S, Hr, D, P, seq, kernels) for y in (yq, yk, yv, yo, ydo)]
+        dqh, dkh, dvh = kernels.backward(dense[0], dense[1], dense[2], dense[3], lse, dense[4], causal)
+        grads = [_heads_rank_buffers(g, B, S, Hr, D, P, seq, kernels) for g in (dqh, dkh, dvh)]
+    else:
+        grads = [torch.empty(0, dtype=yq.dtype, device=yq.device)] * 3
+    return tuple(_ulysses_to_tokens(g, group, seq, heads, B, H, D, kernels) for g in grads)
+
+
+class HeadSideBackwardFunction(torch.autograd.Function):
+    """An exchange's forward (ring or unified) with its gradient taken on the
+    head side: the gradient of attention depends only on the attention of the
+    full sequence, not on how the forward moved the data.  The backward sends
+    Q, K, V and dO through a Ulysses all-to-all over `group` (whose rank order
+    is the sequence order), recomputes this rank's heads' output and LSE there
+    (one extra forward), runs the attention backward, and sends the gradients
+    back.  Heads are split front-loaded (the Ulysses Anything rule), so any H
+    works, and a rank without heads only moves data."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, forward_fn, group, seq, causal, kernels):
+        ctx.save_for_backward(q, k, v)
+        ctx.meta = (group, list(seq), bool(causal), kernels)
+        with torch.no_grad():
+            return forward_fn(q, k, v)
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v = ctx.saved_tensors
+        group, seq, causal, kernels = ctx.meta
+        P, r = _group_rank(group)
+        B, Sr, H, D = q.shape
+        S, heads = sum(seq), front_loaded_splits(H, P)
+        yq, yk, yv = _ulysses_to_heads((q, k, v), group, seq, heads, kernels)
+        if heads[r] and S:
+            yo, lse = kernels.rank_buffer(yq, yk, yv, B, S, heads[r], D, P, seq, causal)
+        else:
+            yo, lse = yq, torch.empty((B, 0, S), dtype=torch.float32, device=q.device)
+        dq, dk, dv = _ulysses_backward(yq, yk, yv, yo, lse, dout, group, seq, heads, causal, kernels, B, H, D)
+        return dq, dk, dv, None, None, None, None, None
+
+
+def ring_attention_trainable(q, k, v, group=None, chunk_lens=None, causal=False, rotate_method="p2p", kernels=None):
+    """ring_attention's output with a gradient (HeadSideBackwardFunction): the
+    forward is the ring exchange; the backward goes through a Ulysses
+    all-to-all over the same group.  Every rank of the group must run the
+    backward."""
+    kernels = kernels or CudaKernels()
+    P, r = _group_rank(group)
+    B, Sr, H, D = _shape4(q)
+    lens = list(chunk_lens) if chunk_lens is not None else [Sr] * P
+    if len(lens) != P or lens[r] != Sr:
+        raise ValueError("chunk_lens must have one entry per rank; entry `rank` must be this rank's length")
+    fwd = lambda a, b, c: ring_attention(a, b, c, group, lens, causal, rotate_method, kernels)[0]
+    return HeadSideBackwardFunction.apply(q, k, v, fwd, group, lens, causal, kernels)
 
 
 def ulysses_attention_trainable(q, k, v, group=None, seq_splits=None, head_splits=None, causal=False, kernels=None):

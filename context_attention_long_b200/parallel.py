@@ -151,9 +151,10 @@ class ContextParallel:
         Ulysses: (B, H_r, S) of this rank's heads; unified: (B, H_j, S_i) of
         this rank's head group over its ring chunk).  head_splits: the heads
         of each Ulysses rank under ulysses_anything (None: front-loaded).
-        When q, k or v requires a gradient, the Ulysses variant (or a single
-        rank) returns an output that autograd differentiates across the
-        ranks; the ring and unified variants then raise NotImplementedError."""
+        When q, k or v requires a gradient, the output is differentiable
+        across the ranks: the Ulysses exchange runs its all-to-alls
+        backwards, and the ring and unified forwards take their gradient on
+        the head side of a Ulysses all-to-all (one extra forward there)."""
         cfg = self.config
         B, Sr, H, D = q.shape
         training = torch.is_grad_enabled() and any(t.requires_grad for t in (q, k, v))
@@ -161,17 +162,30 @@ class ContextParallel:
         S = sum(sum(x) for x in lens) if cfg.variant == "unified" else sum(lens)
         cfg.check(S, H, training=training)
         if training:
-            # Gradients cross GPUs through the Ulysses exchange (the all-to-alls
-            # run backwards); the ring and unified exchanges are forward only.
-            if cfg.variant not in ("none", "ulysses") or return_lse:
-                raise NotImplementedError("training across GPUs goes through the Ulysses exchange "
-                                          "(ring_degree == 1), without return_lse")
-            heads = None
-            if cfg.ulysses_anything:
-                heads = list(head_splits) if head_splits is not None else exchange.front_loaded_splits(
-                    H, cfg.ulysses_degree)
-            return exchange.ulysses_attention_trainable(q, k, v, self.ulysses_group, lens, heads, causal,
-                                                        kernels=self.kernels)
+            # Gradients cross GPUs through a Ulysses all-to-all: the Ulysses
+            # exchange runs its all-to-alls backwards; the ring and unified
+            # forwards take their gradient on the head side of a Ulysses
+            # all-to-all over a group whose rank order is the sequence order.
+            if return_lse:
+                raise NotImplementedError("return_lse is for inference")
+            if cfg.variant in ("none", "ulysses"):
+                heads = None
+                if cfg.ulysses_anything:
+                    heads = list(head_splits) if head_splits is not None else exchange.front_loaded_splits(
+                        H, cfg.ulysses_degree)
+                return exchange.ulysses_attention_trainable(q, k, v, self.ulysses_group, lens, heads, causal,
+                                                            kernels=self.kernels)
+            if cfg.variant == "ring":
+                return exchange.ring_attention_trainable(q, k, v, self.ring_group, lens, causal, cfg.rotate_method,
+                                                         kernels=self.kernels)
+            if cfg.mesh is not None:
+                raise NotImplementedError("unified training with a custom mesh (its rank order need not be the "
+                                          "sequence order)")
+            kern = self.kernels or exchange.CudaKernels()
+            fwd = lambda a, b, c: exchange.unified_attention(a, b, c, self.ring_group, self.ulysses_group, None,
+                                                             lens, None, causal, cfg.rotate_method, kern)[0]
+            seq = [n for chunk in lens for n in chunk]       # grid rank i * U + j holds sub-shard j of chunk i
+            return exchange.HeadSideBackwardFunction.apply(q, k, v, fwd, None, seq, causal, kern)
         if cfg.variant in ("none", "ring"):
             out, lse = exchange.ring_attention(q, k, v, self.ring_group, lens, causal, cfg.rotate_method,
                                                kernels=self.kernels)

@@ -260,9 +260,11 @@ def test_exchange_module_runs_its_cuda_path_on_one_rank():
         # single-GPU backward of the same tensors
         rng = np.random.Generator(np.random.PCG64(78))
         dout = to_dev(inputs.f32_to_bf16_bits(rng.standard_normal((B, S, H, D)).astype(np.float32)))
-        for causal in (False, True):
+        for causal, trainable in ((False, exchange.ulysses_attention_trainable),
+                                  (True, exchange.ulysses_attention_trainable),
+                                  (True, exchange.ring_attention_trainable)):
             qq, kk, vv = (x.clone().requires_grad_(True) for x in (q, k, v))
-            o = exchange.ulysses_attention_trainable(qq, kk, vv, causal=causal)
+            o = trainable(qq, kk, vv, causal=causal)
             o.backward(dout)
             ro, rl = (api.cpattn_causal_ring_attention if causal else api.cpattn_ring_attention)(q, k, v, 1)
             refs = api.cpattn_attention_backward(q, k, v, ro, rl, dout, causal)

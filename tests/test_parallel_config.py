@@ -134,12 +134,12 @@ def _cases(world, rank):
             err = np.abs(t.grad.double().numpy() - r)
             assert err.size == 0 or (err.max() <= 2e-2 * g and err.mean() <= 2e-3 * g), f"{name} {cfg}"
 
-    def refuse_training(cfg, B, H, D, lens):
-        """No silent gradient-free output: the ring exchange is forward only."""
+    def refuse_training(cfg, B, H, D, lens, error):
+        """Ring Anything is inference only (the pages' variants table)."""
         qb, kb, vb = inputs.make_qkv(B, sum(lens), H, D, 19, D == 128)
         a, b = sum(lens[:rank]), sum(lens[:rank + 1])
         q, k, v = (bf16(x[:, a:b]).requires_grad_(True) for x in (qb, kb, vb))
-        with pytest.raises(NotImplementedError):
+        with pytest.raises(error):
             ContextParallel(cfg, kernels=OracleKernels()).attention(q, k, v)
 
     C = ContextParallelConfig
@@ -155,7 +155,11 @@ def _cases(world, rank):
             ("ulysses training", lambda: train(C(ulysses_degree=2), 2, 4, 64, [48, 48], True, 17)),
             ("ulysses anything training", lambda: train(C(ulysses_degree=2, ulysses_anything=True), 1, 3, 64, [40, 29],
                                                        False, 18, head_splits=[2, 1])),
-            ("ring training refused", lambda: refuse_training(C(ring_degree=2), 1, 2, 64, [32, 32])),
+            ("ring training", lambda: train(C(ring_degree=2), 2, 3, 64, [40, 40], True, 25)),
+            ("ring training, p2p, one head", lambda: train(C(ring_degree=2, rotate_method="p2p"), 1, 1, 128, [33, 33],
+                                                          False, 26)),
+            ("ring anything training refused", lambda: refuse_training(C(ring_degree=2, ring_anything=True), 1, 2, 64,
+                                                                      [40, 23], ValueError)),
         ]
     return [
         ("unified 2x2", lambda: run(C(ring_degree=2, ulysses_degree=2), 1, 4, 64, [40, 40, 40, 40], False, 21)),
@@ -164,6 +168,10 @@ def _cases(world, rank):
         ("ring 4", lambda: run(C(ring_degree=4, rotate_method="p2p"), 1, 2, 128, [50, 50, 50, 50], True, 23)),
         ("ulysses 4 training, an empty head rank", lambda: train(C(ulysses_degree=4, ulysses_anything=True), 2, 3, 64,
                                                                [20, 0, 30, 25], True, 24, head_splits=[1, 1, 0, 1])),
+        ("unified 2x2 training", lambda: train(C(ring_degree=2, ulysses_degree=2), 2, 4, 64, [24, 24, 24, 24], True,
+                                               27)),
+        ("ring 4 training, 3 heads over 4 ranks", lambda: train(C(ring_degree=4, rotate_method="p2p"), 1, 3, 64,
+                                                                [20, 20, 20, 20], False, 28)),
     ]
 
 
