@@ -810,7 +810,8 @@ def backward_paths(api, torch, flush, peaks, q, k, v, P):
     gen = torch.Generator(device=q.device).manual_seed(7)
     do = torch.randn(q.shape, generator=gen, device=q.device).to(torch.bfloat16)
     dq, dk, dv = (torch.empty_like(q) for _ in range(3))
-    ws = torch.empty(api.cpattn_attention_backward_workspace_bytes(B, H, S), dtype=torch.uint8, device=q.device)
+    # with the dS scratch the bindings allocate by default (all heads here)
+    ws = torch.empty(api.backward_workspace_bytes(B, H, S), dtype=torch.uint8, device=q.device)
     peak_tf = float(peaks["bf16_tflops"])
     res = {}
     for causal in (False, True):
@@ -824,12 +825,12 @@ def backward_paths(api, torch, flush, peaks, q, k, v, P):
         tf = backward_flops(B, H, S, D, causal) / (ms * 1e-3) / 1e12
         res["attention_backward" + ("_causal" if causal else "")] = {
             "ms": ms, "TFLOP/s": tf, "frac_bf16_peak": tf / peak_tf,
-            "flops": "2.5x the forward's (10*B*H*S^2*D; causal: visible pairs)", "launches": 3}
+            "flops": "2.5x the forward's (10*B*H*S^2*D; causal: visible pairs)", "launches": 3,
+            "note": "row sums, dK/dV storing dS, dQ GEMM over the stored dS"}
     # the backward of the Ulysses flow (rank buffers; B = 1 here, so they are the full tensors)
     U = 4
     out, lse = api.cpattn_ulysses_attention(q.reshape(-1), k.reshape(-1), v.reshape(-1), B, S, H, D, U, stream=stream)
-    wsu = torch.empty(api.cpattn_ulysses_attention_backward_workspace_bytes(B, H, S, D), dtype=torch.uint8,
-                      device=q.device)
+    wsu = torch.empty(api.backward_workspace_bytes(B, H, S, ulysses_D=D), dtype=torch.uint8, device=q.device)
 
     def run_u():
         api.cpattn_ulysses_attention_backward(q.reshape(-1), k.reshape(-1), v.reshape(-1), out, lse, do.reshape(-1),
@@ -839,7 +840,8 @@ def backward_paths(api, torch, flush, peaks, q, k, v, P):
     ms = median_event_ms(run_u, flush, stream)
     tf = backward_flops(B, H, S, D, False) / (ms * 1e-3) / 1e12
     res[f"ulysses_{U}_backward_flow"] = {"ms": ms, "TFLOP/s": tf, "frac_bf16_peak": tf / peak_tf,
-                                         "launches": 7, "note": "5 permuted in, backward of 4 head ranks, 3 permuted out"}
+                                         "launches": 9, "note": "5 tensors permuted in (2 launches), the row sums of "
+                                         "4 head ranks, dK/dV and the dQ GEMM over all of them, 3 permuted out"}
     return res
 
 
@@ -1010,7 +1012,7 @@ def run_sweep(args):
             gen = torch.Generator(device=dev).manual_seed(7)
             do = torch.randn(q.shape, generator=gen, device=dev).to(torch.bfloat16)
             bq, bk, bv = (torch.empty_like(q) for _ in range(3))
-            bws = torch.empty(api.cpattn_attention_backward_workspace_bytes(B, H, S), dtype=torch.uint8, device=dev)
+            bws = torch.empty(api.backward_workspace_bytes(B, H, S), dtype=torch.uint8, device=dev)
             o_f, l_f = api.cpattn_ring_attention(q, k, v, P, lens)
             o_c, l_c = api.cpattn_causal_ring_attention(q, k, v, P, lens)
             paths.append(("attention backward (dQ, dK, dV)",

@@ -60,6 +60,7 @@ SIGNATURES = {
                                                 c_int, c_int, c_int, c_int, c_int, c_int, P_INT, P_INT,
                                                 c_void_p, c_size_t, c_void_p]),
     "cpattn_attention_backward_workspace_bytes": (c_size_t, [c_int, c_int, c_int]),
+    "cpattn_attention_backward_ds_bytes": (c_size_t, [c_int, c_int, c_int]),
     "cpattn_attention_backward": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                           c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int,
                                           c_void_p, c_size_t, c_void_p]),

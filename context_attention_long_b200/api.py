@@ -25,7 +25,8 @@ __all__ = [
     "cpattn_causal_head_sharded_attention", "cpattn_ulysses_workspace_bytes",
     "cpattn_unified_workspace_bytes", "cpattn_ulysses_attention", "cpattn_causal_ulysses_attention",
     "cpattn_unified_attention", "cpattn_causal_unified_attention",
-    "cpattn_attention_backward_workspace_bytes", "cpattn_attention_backward",
+    "cpattn_attention_backward_workspace_bytes", "cpattn_attention_backward_ds_bytes", "cpattn_attention_backward",
+    "backward_workspace_bytes", "BACKWARD_DS_BUDGET",
     "cpattn_ulysses_attention_backward_workspace_bytes", "cpattn_ulysses_attention_backward",
     "cpattn_ulysses_attention_noalloc", "cpattn_ring_chunk_attention", "cpattn_gathered_kv_attention",
     "cpattn_rank_buffer_attention", "cpattn_front_loaded_splits", "cpattn_exchange_bytes",
@@ -371,15 +372,46 @@ def cpattn_attention_backward_workspace_bytes(B, H, S) -> int:
     return int(_native.load().cpattn_attention_backward_workspace_bytes(B, H, S))
 
 
+def cpattn_attention_backward_ds_bytes(B, S, causal) -> int:
+    return int(_native.load().cpattn_attention_backward_ds_bytes(B, S, 1 if causal else 0))
+
+
+# Default cap on the dS scratch the backward bindings add to a workspace they
+# allocate: the library groups the heads so that their dS tiles fit it, and
+# when one head's tiles exceed it the dQ kernel runs instead.
+BACKWARD_DS_BUDGET = 8 << 30
+
+
+def _ds_scratch_bytes(B, H, S, causal, ds_budget):
+    """Whole heads of dS scratch within the budget, plus the 256 bytes the
+    library may skip to align it (0: no scratch)."""
+    per = cpattn_attention_backward_ds_bytes(B, S, causal)
+    budget = BACKWARD_DS_BUDGET if ds_budget is None else int(ds_budget)
+    heads = min(H, budget // per) if per > 0 else 0
+    return 256 + heads * per if heads > 0 else 0
+
+
+def backward_workspace_bytes(B, H, S, causal=False, ds_budget=None, ulysses_D=None) -> int:
+    """Bytes of the workspace the backward bindings allocate: the minimum of
+    cpattn_attention_backward (or, given ulysses_D, of the Ulysses backward
+    flow) plus whole heads of dS scratch within ds_budget.  A workspace sized
+    for causal=False also serves the causal backward."""
+    base = (cpattn_attention_backward_workspace_bytes(B, H, S) if ulysses_D is None else
+            cpattn_ulysses_attention_backward_workspace_bytes(B, H, S, ulysses_D))
+    return base + _ds_scratch_bytes(B, H, S, causal, ds_budget)
+
+
 def cpattn_attention_backward(q, k, v, out, lse, dout, causal=False, dq=None, dk=None, dv=None, workspace=None,
-                              stream=None):
+                              stream=None, ds_budget=None):
     """Gradient of attention over full (B,S,H,D) bf16 tensors given the
-    forward's output and LSE; returns (dq, dk, dv) in bf16."""
+    forward's output and LSE; returns (dq, dk, dv) in bf16.  An allocated
+    workspace holds up to ds_budget bytes (default BACKWARD_DS_BUDGET) of dS
+    scratch; 0 selects the dQ kernel that recomputes S and dP."""
     B, S, H, D = _bshd(q)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    workspace = _workspace(cpattn_attention_backward_workspace_bytes(B, H, S), q.device, workspace)
+    workspace = _workspace(backward_workspace_bytes(B, H, S, causal, ds_budget), q.device, workspace)
     for t, name in ((k, "k"), (v, "v"), (out, "out"), (dout, "dout"), (dq, "dq"), (dk, "dk"), (dv, "dv")):
         _need(t, q.numel(), torch.bfloat16, name)
     _need(lse, B * H * S, torch.float32, "lse")
@@ -398,13 +430,14 @@ def cpattn_ulysses_attention_backward_workspace_bytes(B, H, S, D) -> int:
 
 def cpattn_ulysses_attention_backward(q, k, v, out, lse, dout, B, S, H, D, degree, seq_splits=None,
                                       head_splits=None, causal=False, dq=None, dk=None, dv=None, workspace=None,
-                                      stream=None):
+                                      stream=None, ds_budget=None):
     """Backward of the Ulysses flow on sequence-sharded rank buffers (flat
-    bf16); returns (dq, dk, dv) in the same layout."""
+    bf16); returns (dq, dk, dv) in the same layout.  ds_budget as
+    cpattn_attention_backward."""
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    workspace = _workspace(cpattn_ulysses_attention_backward_workspace_bytes(B, H, S, D), q.device, workspace)
+    workspace = _workspace(backward_workspace_bytes(B, H, S, causal, ds_budget, ulysses_D=D), q.device, workspace)
     for t, name in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout"), (dq, "dq"), (dk, "dk"), (dv, "dv")):
         _need(t, _flat_numel(B, S, H, D), torch.bfloat16, name)
     _need(lse, B * H * S, torch.float32, "lse")

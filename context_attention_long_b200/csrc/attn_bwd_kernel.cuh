@@ -11,12 +11,18 @@
 // Parallelism article, sections 1 and 7, causal masking by position ids); the
 // causal mask here is the forward's: key j is visible to query i iff j <= i.
 //
-// Two kernels, so that no gradient needs atomics: the dQ kernel owns a Q tile
-// and walks the K/V tiles; the dK/dV kernel owns a K/V tile and walks the Q
-// tiles (S and dP are computed in both).  A launch covers up to 8 problems
-// (the full tensors, or the head ranks' buffers of the Ulysses flow), each
-// with its own tensor maps, LSE strides and Delta slice.  CTA organisation of
-// each kernel (320 threads, one CTA per SM):
+// No gradient needs atomics.  The dK/dV kernel owns a K/V tile and walks the
+// Q tiles.  dQ comes one of two ways:
+//   - with dS scratch (the default of the bindings): the dK/dV kernel also
+//     stores dS in bf16 (a shared-memory staging tile and asynchronous bulk
+//     stores), and the dQ GEMM (attn_bwd_dq_gemm_kernel) computes dS K from
+//     it, bound by the HBM reads of dS -- S and dP are formed once;
+//   - without: the dQ kernel owns a Q tile, walks the K/V tiles and forms S,
+//     P, dP and dS again (the same values, bit for bit).
+// A launch covers up to 8 problems (the full tensors, the head ranks' buffers
+// of the Ulysses flow, or groups of their heads whose dS fits the scratch),
+// each with its own tensor maps, LSE strides and Delta slice.  CTA
+// organisation of the dQ and dK/dV kernels (320 threads, one CTA per SM):
 //   warp 0      TMA producer: the owned tiles once, the walked tiles through
 //               rings of 3 stages (K or Q) and 2 stages (V or dO)
 //   warp 1      TMEM allocator + single-thread MMA issuer (tcgen05.mma)
@@ -48,7 +54,7 @@ namespace cpattn {
 // misaligned (it then returns without touching memory).
 constexpr unsigned int SITE_LAYOUT = 1u << 6;
 
-template <int D>
+template <int D, int kQStages = 3, bool kStaging = false>
 struct BwdSmem {
   static constexpr int kHalves = D / 64;
   static constexpr int kBoxBytes = 128 * 128;          // [128 rows][64 bf16], 128B-swizzled
@@ -57,14 +63,16 @@ struct BwdSmem {
   // kernel) is also the one released last (after the step's final MMA), so
   // it gets three stages: its load starts two steps ahead and its TMA latency
   // stays off the pipeline.  The other walked tile (V, dO) is released
-  // mid-step, after its last MMA, and two stages are enough.
-  static constexpr int kStagesC = 3;
+  // mid-step, after its last MMA, and two stages are enough.  The dK/dV
+  // kernel that stores dS gives the third stage up for the dS staging tile.
+  static constexpr int kStagesC = kQStages;
   static constexpr int kStagesE = 2;
   static constexpr int kOffA = 0;                       // owned tile 0: Q (dq) or K (dkv)
   static constexpr int kOffB = kOffA + kTileBytes;      // owned tile 1: dO (dq) or V (dkv)
   static constexpr int kOffC = kOffB + kTileBytes;      // walked tile 0 per stage: K (dq) or Q (dkv)
   static constexpr int kOffE = kOffC + kStagesC * kTileBytes;   // walked tile 1 per stage: V or dO
-  static constexpr int kOffVec = kOffE + kStagesE * kTileBytes; // dkv: [2][lse2 128 | delta 128] floats
+  static constexpr int kOffStaging = kOffE + kStagesE * kTileBytes;   // dkv with dS stores: one dS tile
+  static constexpr int kOffVec = kOffStaging + (kStaging ? kBwdDsTileBytes : 0);  // dkv: [2][lse2 128 | delta 128] floats
   static constexpr int kOffBar = kOffVec + 2 * 2 * 128 * 4;
   static constexpr int kNumBars = 24;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
@@ -75,7 +83,8 @@ struct BwdSmem {
   // returns without touching memory).
   static constexpr int kAllocBytes = kBytes;
 };
-static_assert(BwdSmem<128>::kAllocBytes <= 232448, "backward shared memory exceeds the per-CTA limit");
+static_assert(BwdSmem<128>::kAllocBytes <= 232448 && BwdSmem<128, 2, true>::kAllocBytes <= 232448,
+              "backward shared memory exceeds the per-CTA limit");
 
 // Pins a value in a register at this point of the program: an empty volatile
 // asm that reads and "writes" it, so the computation of the value cannot sink
@@ -159,25 +168,30 @@ __global__ void __launch_bounds__(256, 3) attn_bwd_delta_kernel(const __nv_bfloa
   }
 }
 
-// Units of both kernels: (problem, b, h, 128-row tile) with the tile index
-// fastest; problems occupy consecutive unit ranges.
+// Units: (problem, b, h, 128-row tile) over the problem's heads [h0, h0 + nh),
+// the tile index fastest (with last_first, the last tile of a head first);
+// problems occupy consecutive unit ranges.  hl = h - h0.
 struct BwdUnit {
-  int pi, b, h, t;
+  int pi, b, h, hl, t;
 };
-__device__ __forceinline__ BwdUnit bwd_unit(const BwdParams &p, bool last_first) {
+__device__ __forceinline__ BwdUnit bwd_unit_at(const BwdParams &p, int idx, bool last_first) {
   const int nt = (p.S + 127) / 128;
   BwdUnit u;
   int pi = 0;
-  while (pi + 1 < p.n_prob && p.prob[pi + 1].unit_base <= static_cast<int>(blockIdx.x)) ++pi;
-  const int local = static_cast<int>(blockIdx.x) - p.prob[pi].unit_base;
-  const int H = p.prob[pi].H;
+  while (pi + 1 < p.n_prob && p.prob[pi + 1].unit_base <= idx) ++pi;
+  const int local = idx - p.prob[pi].unit_base;
+  const int NH = p.prob[pi].nh;
   const int t_in = local % nt;
   const int bh = local / nt;
   u.pi = pi;
-  u.h = bh % H;
-  u.b = bh / H;
+  u.hl = bh % NH;
+  u.h = p.prob[pi].h0 + u.hl;
+  u.b = bh / NH;
   u.t = last_first ? nt - 1 - t_in : t_in;
   return u;
+}
+__device__ __forceinline__ BwdUnit bwd_unit(const BwdParams &p, bool last_first) {
+  return bwd_unit_at(p, static_cast<int>(blockIdx.x), last_first);
 }
 
 // ===================================================================== dQ
@@ -475,9 +489,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __gri
 }
 
 // =================================================================== dK, dV
-template <int D>
+// kDs: also store dS for the dQ GEMM (every problem's ds set), through a
+// shared-memory staging tile and asynchronous bulk stores.
+template <int D, bool kDs>
 __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __grid_constant__ BwdParams p) {
-  using L = BwdSmem<D>;
+  using L = BwdSmem<D, kDs ? 2 : 3, kDs>;
   constexpr uint32_t IDESC_SS = idesc_bf16_f32(128, 128, false);   // S^T = K Q^T, dP^T = V dO^T
   constexpr uint32_t IDESC_ACC = idesc_bf16_f32(128, D, true);     // dV += P^T dO, dK += dS^T Q
   extern __shared__ __align__(1024) uint8_t bwd_smem[];
@@ -680,6 +696,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __gr
     for (int i = 0; ok && i < n; ++i) {
       const int q0 = (qt0 + i) * 128;
       const uint32_t vec = sb + L::kOffVec + (i & 1) * 1024;
+      // this warp's 4 KB of the dS tile: keys [32 quad, 32 quad + 32), query
+      // groups [8 half, 8 half + 8), in the tile layout (and in the staging
+      // tile at the same offset)
+      const uint32_t ds_part = static_cast<uint32_t>(quad * 8192 + half * 4096);
+      unsigned char *const ds_dst =
+          kDs ? PB.ds + bwd_ds_tile_index(U.b, U.hl, PB.nh, nt, qt0 + i, U.t, p.causal != 0) * kBwdDsTileBytes + ds_part
+              : nullptr;
+      const uint32_t ds_stage = sb + L::kOffStaging + ds_part;
       if (half == 0) {
         st_shared_f32(vec + 4 * row, nl2);
         st_shared_f32(vec + 512 + 4 * row, ndl);
@@ -705,7 +729,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __gr
       // schedule freely around the exponentials.
       const float4 *lse4 = reinterpret_cast<const float4 *>(bwd_smem + (vec - sb)) + (col0 >> 2);
       const float4 *del4 = lse4 + 32;
-      const int qlim = (p.causal ? k_pos - q0 : 0) - col0;   // queries q < qlim do not see this key
+      // queries q < qlim do not see this key; a key past the sequence (its K
+      // and V rows are the next batch element's, or TMA fill) is seen by none,
+      // so its P and dS are exactly 0 -- the stored dS meets real K rows of
+      // that position in the dQ GEMM
+      const int qlim = row_valid ? (p.causal ? k_pos - q0 : 0) - col0 : 64;
 #pragma unroll
       for (int q4 = 0; q4 < 16; ++q4) {
         const float4 l = lse4[q4];
@@ -733,6 +761,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __gr
       __syncwarp();
       tc_fence_after();
       // dS^T = P^T * (dP^T - delta[q]), bf16 pairs over the dP^T columns read
+      if (kDs) {
+        // the staging tile is free once the previous tile's bulk store has
+        // read it (issued a whole tile ago)
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
+      }
 #pragma unroll
       for (int c0 = 0; c0 < 64; c0 += 32) {
         uint32_t dp[32];
@@ -748,12 +782,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __gr
                                        __uint_as_float(s[q + 3]) * (__uint_as_float(dp[4 * k4 + 3]) - dl.w));
         }
         tmem_st16(tDP + c0 / 2, pk);
+        if (kDs) {
+          // the same bf16 values for the dQ GEMM: 8 queries (16 bytes) per
+          // store, lanes on consecutive keys (512 contiguous bytes a warp)
+#pragma unroll
+          for (int g = 0; g < 4; ++g)
+            st_shared_v4(ds_stage + ((c0 >> 3) + g) * 512 + lane * 16, pk[4 * g], pk[4 * g + 1], pk[4 * g + 2],
+                         pk[4 * g + 3]);
+        }
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(sb + BAR_DS);
+      if (kDs) {
+        // After dS is published (the proxy fence waits for this thread's
+        // shared-memory writes): the bulk store drains in the background
+        // while the row threads go on, evicted first from L2, where the Q
+        // and dO tiles that every CTA of the head walks should stay.
+        fence_proxy_async_shared();
+        __syncwarp();
+        if (lane == 0) {
+          bulk_store_hint(ds_dst, ds_stage, 4096, l2_evict_first_policy());
+          bulk_commit();
+        }
+      }
     }
+    if (kDs && lane == 0) bulk_wait_all();
     if (ok && n > 0) {
       const bool w = mbar_wait(sb + BAR_ACC, 0, abort_flag, tmo, SITE_EPILOGUE);
       if (__any_sync(0xffffffffu, !w)) ok = false;
@@ -795,6 +850,214 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __gr
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kBwdTmemCols);
+  }
+}
+
+// ============================================================== dQ GEMM
+// dQ = dS K * scale over the dS tiles that the dK/dV kernel stored, so that S
+// and dP are not computed a second time: per unit (b, h, Q tile) the products
+// of the walked K tiles accumulate in TMEM.  A is the dS tile, MN-major
+// (queries contiguous in groups of 8, the un-swizzled core-matrix layout) and
+// loaded with one 32 KB bulk copy; B is the K tile, MN-major with the 128-byte
+// swizzle (as in the dQ kernel).  The kernel is bound by the HBM reads of the
+// dS tiles (32 KB per tile pair).  Persistent: one CTA per SM walks the units
+// blockIdx.x, blockIdx.x + gridDim.x, ...; two TMEM accumulators, so that the
+// epilogue of one unit overlaps the loads and MMAs of the next.  Units run
+// head by head (the CTAs at work share a few heads' K tiles in L2), the last
+// Q tile of a head first under the causal mask; the stride of the walk mixes
+// long and short causal units in every CTA.
+//   warp 0      producer: the dS tile (bulk copy) and the K tile (TMA) per stage
+//   warp 1      TMEM allocator + single-thread MMA issuer
+//   warps 2-5   epilogue: one dQ row per thread (TMEM lane), scaled, bf16
+template <int D>
+struct BwdGemmSmem {
+  static constexpr int kATile = kBwdDsTileBytes;            // dS tile, 32 KB
+  static constexpr int kBTile = BwdSmem<D>::kTileBytes;     // K tile
+  static constexpr int kStage = kATile + kBTile;            // a multiple of 1024: the K tile stays swizzle-aligned
+  static constexpr int kStages = D == 128 ? 3 : 4;
+  static constexpr int kOffBar = kStages * kStage;
+  static constexpr int kNumBars = 2 * kStages + 5;          // full[S], empty[S], acc_full[2], acc_empty[2], tail
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kBytes = kOffMisc + 16;
+  static constexpr int kAllocBytes = kBytes;
+};
+static_assert(BwdGemmSmem<128>::kAllocBytes <= 232448 && BwdGemmSmem<64>::kAllocBytes <= 232448,
+              "dQ GEMM shared memory exceeds the per-CTA limit");
+constexpr int kBwdGemmThreads = 192;
+
+template <int D>
+__global__ void __launch_bounds__(kBwdGemmThreads, 1)
+    attn_bwd_dq_gemm_kernel(const __grid_constant__ BwdParams p, int n_units) {
+  using L = BwdGemmSmem<D>;
+  using T = BwdSmem<D>;
+  constexpr uint32_t IDESC = idesc_bf16_f32(128, D, true, true);   // dS and K both MN-major
+  constexpr uint32_t kAccCols = 2 * D;
+  extern __shared__ __align__(1024) uint8_t bwd_smem[];
+  const uint32_t sb = smem_u32(bwd_smem);
+  if (sb & 1023u) {
+    if (threadIdx.x == 0) atomicOr(&g_device_status, SITE_LAYOUT);
+    return;
+  }
+  constexpr int ST = L::kStages;
+  constexpr uint32_t BAR_FULL = L::kOffBar;                 // [ST] stage loaded
+  constexpr uint32_t BAR_EMPTY = BAR_FULL + 8 * ST;         // [ST] stage consumed by the MMAs
+  constexpr uint32_t BAR_AF = BAR_EMPTY + 8 * ST;           // [2] accumulator complete
+  constexpr uint32_t BAR_AE = BAR_AF + 16;                  // [2] accumulator read out
+  constexpr uint32_t BAR_TAIL = BAR_AE + 16;
+  constexpr uint32_t TMEM_SLOT = L::kOffMisc;
+  constexpr uint32_t ABORT = L::kOffMisc + 4;
+  static_assert(BAR_TAIL + 8 <= L::kOffMisc, "barrier area");
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint64_t tmo = p.timeout_ns;
+  const int nt = (p.S + 127) / 128;
+  const bool causal = p.causal != 0;
+  // K tiles a Q tile walks: the keys at or before its last query (causal).
+  auto walked = [&](int t) {
+    const int q0 = t * 128;
+    const int kv_len = causal ? min(p.S, q0 + 128) : p.S;
+    return (kv_len + 127) / 128;
+  };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(sb + BAR_FULL + 8 * s, 1);
+      mbar_init(sb + BAR_EMPTY + 8 * s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(sb + BAR_AF + 8 * a, 1);
+      mbar_init(sb + BAR_AE + 8 * a, 4);   // one arrival per epilogue warp
+    }
+    mbar_init(sb + BAR_TAIL, 1);
+    st_shared_volatile(sb + ABORT, 0u);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(sb + TMEM_SLOT, kAccCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ld_shared_volatile(sb + TMEM_SLOT);
+  const uint32_t abort_flag = sb + ABORT;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      for (int pi = 0; pi < p.n_prob; ++pi) tma_prefetch_desc(&p.prob[pi].tm_k);
+      // the dS tiles are read once: evicted first, so that the K tiles, read
+      // by every Q tile of their head, stay in L2
+      const uint64_t once = l2_evict_first_policy();
+      int it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+        const BwdUnit U = bwd_unit_at(p, u, causal);
+        const BwdProblem &PB = p.prob[U.pi];
+        const int n = walked(U.t);
+        const unsigned char *a0 = PB.ds + bwd_ds_tile_index(U.b, U.hl, PB.nh, nt, U.t, 0, causal) * kBwdDsTileBytes;
+        for (int j = 0; j < n; ++j, ++it) {
+          const int st = it % ST;
+          if (!mbar_wait(sb + BAR_EMPTY + 8 * st, ((it / ST) & 1) ^ 1, abort_flag, tmo, SITE_PRODUCER)) {
+            ok = false;
+            break;
+          }
+          const uint32_t full = sb + BAR_FULL + 8 * st;
+          const uint32_t dst = sb + st * L::kStage;
+          mbar_arrive_expect_tx(full, L::kStage);
+          bulk_load_hint(dst, a0 + static_cast<long long>(j) * kBwdDsTileBytes, L::kATile, full, once);
+          for (int hf = 0; hf < T::kHalves; ++hf)
+            tma_load_3d(dst + L::kATile + hf * T::kBoxBytes, &PB.tm_k, hf * 64, U.h, U.b * p.S + j * 128, full);
+        }
+      }
+      // Before the CTA exits, every stage's last use has been consumed by the
+      // MMAs (so its loads landed) and its release arrived here (bounded).
+      for (int j = 0; j < ST && j < it; ++j) {
+        const int i = it - 1 - j;
+        mbar_wait(sb + BAR_EMPTY + 8 * (i % ST), (i / ST) & 1, 0u, tmo, SITE_TAIL);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int it = 0, local = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x, ++local) {
+        const BwdUnit U = bwd_unit_at(p, u, causal);
+        const int n = walked(U.t);
+        const int a = local & 1;
+        if (!mbar_wait_spin(sb + BAR_AE + 8 * a, ((local >> 1) & 1) ^ 1, abort_flag, tmo, SITE_MMA)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + a * D;
+        for (int j = 0; j < n; ++j, ++it) {
+          const int st = it % ST;
+          if (!mbar_wait_spin(sb + BAR_FULL + 8 * st, (it / ST) & 1, abort_flag, tmo, SITE_MMA)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          // dS: core matrices of 8 keys x 8 queries, 128 bytes apart along the
+          // keys (LBO) and 512 bytes apart along the queries (SBO); the 16
+          // keys of MMA kk start at quarter kk / 2 (8 KB each), half kk % 2.
+          // K: rows of 128 bytes, 16 keys = 2048 bytes.
+          const uint64_t da = opaque_u64(smem_desc_plain(sb + st * L::kStage, 128, 512));
+          const uint64_t db = opaque_u64(smem_desc_sw128(sb + st * L::kStage + L::kATile, T::kBoxBytes, 1024));
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(d, da + ((((kk >> 1) * 8192) + (kk & 1) * 256) >> 4), db + ((kk * 2048) >> 4), IDESC,
+                   (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(sb + BAR_EMPTY + 8 * st);
+        }
+        if (ok) mma_commit(sb + BAR_AF + 8 * a);
+      }
+      // Drain: every issued MMA has completed before TMEM is released.
+      mma_commit(sb + BAR_TAIL);
+      mbar_wait(sb + BAR_TAIL, 0, 0u, tmo, SITE_TAIL);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;   // accumulator row = TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    int local = 0;
+    for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++local) {
+      const int a = local & 1;
+      const bool w = mbar_wait(sb + BAR_AF + 8 * a, (local >> 1) & 1, abort_flag, tmo, SITE_EPILOGUE);
+      if (__any_sync(0xffffffffu, !w)) break;
+      __syncwarp();
+      tc_fence_after();
+      const BwdUnit U = bwd_unit_at(p, u, causal);
+      const BwdProblem &PB = p.prob[U.pi];
+      const int q = U.t * 128 + r;
+      const bool row_ok = q < p.S;
+      __nv_bfloat16 *dst =
+          static_cast<__nv_bfloat16 *>(PB.dq) + ((static_cast<long long>(U.b) * p.S + q) * PB.H + U.h) * D;
+#pragma unroll 1
+      for (int c = 0; c < D; c += 32) {
+        uint32_t v[32];
+        __syncwarp();
+        tmem_ld32_wait(tmem + lane_base + a * D + c, v);   // the whole warp, converged
+        if (!row_ok) continue;
+        uint4 *d4 = reinterpret_cast<uint4 *>(dst + c);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          d4[k] = make_uint4(
+              pack_bf16x2(__uint_as_float(v[8 * k]) * p.scale, __uint_as_float(v[8 * k + 1]) * p.scale),
+              pack_bf16x2(__uint_as_float(v[8 * k + 2]) * p.scale, __uint_as_float(v[8 * k + 3]) * p.scale),
+              pack_bf16x2(__uint_as_float(v[8 * k + 4]) * p.scale, __uint_as_float(v[8 * k + 5]) * p.scale),
+              pack_bf16x2(__uint_as_float(v[8 * k + 6]) * p.scale, __uint_as_float(v[8 * k + 7]) * p.scale));
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sb + BAR_AE + 8 * a);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kAccCols);
   }
 }
 

@@ -250,6 +250,7 @@ template <int D>
 static cudaError_t launch_bwd_d(const BwdParams &p, int units, cudaStream_t stream) {
   static std::mutex mu;
   static bool configured[kMaxDevices] = {false};
+  static int sms[kMaxDevices] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
   {
@@ -258,32 +259,53 @@ static cudaError_t launch_bwd_d(const BwdParams &p, int units, cudaStream_t stre
       cudaError_t e = cudaFuncSetAttribute(attn_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            BwdSmem<D>::kAllocBytes);
       if (e != cudaSuccess) return e;
-      e = cudaFuncSetAttribute(attn_bwd_dkv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      e = cudaFuncSetAttribute(attn_bwd_dkv_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                BwdSmem<D>::kAllocBytes);
+      if (e != cudaSuccess) return e;
+      e = cudaFuncSetAttribute(attn_bwd_dkv_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               BwdSmem<D, 2, true>::kAllocBytes);
+      if (e != cudaSuccess) return e;
+      e = cudaFuncSetAttribute(attn_bwd_dq_gemm_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               BwdGemmSmem<D>::kAllocBytes);
+      if (e != cudaSuccess) return e;
+      e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
       if (e != cudaSuccess) return e;
       configured[dev] = true;
     }
   }
-  attn_bwd_dq_kernel<D><<<static_cast<unsigned>(units), kBwdThreads, BwdSmem<D>::kAllocBytes, stream>>>(p);
+  const bool with_ds = p.prob[0].ds != nullptr;
+  if (!with_ds) {
+    attn_bwd_dq_kernel<D><<<static_cast<unsigned>(units), kBwdThreads, BwdSmem<D>::kAllocBytes, stream>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (with_ds)
+    attn_bwd_dkv_kernel<D, true><<<static_cast<unsigned>(units), kBwdThreads, BwdSmem<D, 2, true>::kAllocBytes,
+                                   stream>>>(p);
+  else
+    attn_bwd_dkv_kernel<D, false><<<static_cast<unsigned>(units), kBwdThreads, BwdSmem<D>::kAllocBytes, stream>>>(p);
   cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  attn_bwd_dkv_kernel<D><<<static_cast<unsigned>(units), kBwdThreads, BwdSmem<D>::kAllocBytes, stream>>>(p);
+  if (e != cudaSuccess || !with_ds) return e;
+  // one CTA per SM (its shared memory admits no second), each walking units
+  const int grid = std::min(units, std::max(sms[dev], 1));
+  attn_bwd_dq_gemm_kernel<D><<<static_cast<unsigned>(grid), kBwdGemmThreads, BwdGemmSmem<D>::kAllocBytes, stream>>>(
+      p, units);
   return cudaGetLastError();
 }
 
-cudaError_t launch_attention_backward(const BwdParams &p, int D, const void *const *outs, const void *const *douts,
-                                      cudaStream_t stream) {
+cudaError_t launch_bwd_delta(const void *out, const void *dout, float *delta, int B, int S, int H, int D,
+                             cudaStream_t stream) {
+  const long long rows = static_cast<long long>(B) * S * H;
+  if (rows == 0) return cudaSuccess;
+  attn_bwd_delta_kernel<<<grid_for(rows, (256 / 32) * (32 / (D / 8)) * kDeltaPasses), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16 *>(out), static_cast<const __nv_bfloat16 *>(dout), delta, B, S, H, D);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_kernels(const BwdParams &p, int D, cudaStream_t stream) {
   const int nt = (p.S + 127) / 128;
   int units = 0;
-  for (int i = 0; i < p.n_prob; ++i) {
-    const long long rows = static_cast<long long>(p.B) * p.S * p.prob[i].H;
-    attn_bwd_delta_kernel<<<grid_for(rows, (256 / 32) * (32 / (D / 8)) * kDeltaPasses), 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16 *>(outs[i]), static_cast<const __nv_bfloat16 *>(douts[i]), p.prob[i].delta,
-        p.B, p.S, p.prob[i].H, D);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    units += p.B * p.prob[i].H * nt;
-  }
+  for (int i = 0; i < p.n_prob; ++i) units += p.B * p.prob[i].nh * nt;
   if (units == 0) return cudaSuccess;
   return D == 128 ? launch_bwd_d<128>(p, units, stream) : launch_bwd_d<64>(p, units, stream);
 }
@@ -1288,10 +1310,16 @@ size_t cpattn_attention_backward_workspace_bytes(int B, int H, int S) {
   return static_cast<size_t>(B) * H * S * sizeof(float);
 }
 
+size_t cpattn_attention_backward_ds_bytes(int B, int S, int causal) {
+  if (B < 1 || S < 1) return 0;
+  const int nt = (S + 127) / 128;
+  return static_cast<size_t>(B) * static_cast<size_t>(bwd_ds_tiles_per_head(nt, causal != 0)) * kBwdDsTileBytes;
+}
+
 // One backward problem over [B, S, H, D] tensors; LSE index b*lse_b + (h + lse_h0)*lse_h + s.
 static bool backward_problem(BwdProblem &pb, const void *q, const void *k, const void *v, const void *dout,
                              const float *lse, long long lse_b, long long lse_h, int lse_h0, float *delta, void *dq,
-                             void *dk, void *dv, int B, int S, int H, int D, int unit_base) {
+                             void *dk, void *dv, int B, int S, int H, int D) {
   std::memset(&pb, 0, sizeof(pb));
   const long long rows = static_cast<long long>(B) * S;
   if (!encode_rows_map(&pb.tm_q, q, D, H, rows) || !encode_rows_map(&pb.tm_k, k, D, H, rows) ||
@@ -1302,11 +1330,12 @@ static bool backward_problem(BwdProblem &pb, const void *q, const void *k, const
   pb.lse_h = lse_h;
   pb.lse_h0 = lse_h0;
   pb.H = H;
+  pb.h0 = 0;
+  pb.nh = H;
   pb.delta = delta;
   pb.dq = dq;
   pb.dk = dk;
   pb.dv = dv;
-  pb.unit_base = unit_base;
   return true;
 }
 
@@ -1319,6 +1348,66 @@ static void backward_common_params(BwdParams &P, int B, int S, int D, bool causa
   P.timeout_ns = wait_timeout_ns();
 }
 
+// The part of a workspace past its first `used` bytes, from a 256-byte
+// boundary, as dS scratch.
+static void ds_scratch(void *workspace, size_t workspace_bytes, size_t used, unsigned char *&scratch,
+                       size_t &scratch_bytes) {
+  const size_t start = (used + 255) & ~static_cast<size_t>(255);
+  const uintptr_t base = (reinterpret_cast<uintptr_t>(workspace) + start + 255) & ~static_cast<uintptr_t>(255);
+  const size_t skip = base - reinterpret_cast<uintptr_t>(workspace);
+  scratch = nullptr;
+  scratch_bytes = 0;
+  if (workspace_bytes > skip) {
+    scratch = reinterpret_cast<unsigned char *>(base);
+    scratch_bytes = workspace_bytes - skip;
+  }
+}
+
+// The gradient kernels over `sets` (problems covering all their heads, Delta
+// computed).  When the scratch holds the dS tiles of at least one head, the
+// heads are cut into groups whose tiles fit the scratch together (up to
+// kMaxProblems groups per launch): the dK/dV kernel stores dS and the dQ GEMM
+// reads it.  The scratch is reused by the next launch, which the stream orders
+// after the GEMM that read it.  Otherwise the dQ kernel recomputes S and dP.
+static cudaError_t run_bwd_sets(const std::vector<BwdProblem> &sets, unsigned char *scratch, size_t scratch_bytes,
+                                int B, int S, int D, bool causal, cudaStream_t stream) {
+  const size_t per_head = cpattn_attention_backward_ds_bytes(B, S, causal ? 1 : 0);
+  const long long cap = (scratch != nullptr && per_head > 0) ? static_cast<long long>(scratch_bytes / per_head) : 0;
+  const int nt = (S + 127) / 128;
+  std::unique_ptr<BwdParams> P(new BwdParams);
+  std::memset(P.get(), 0, sizeof(BwdParams));
+  int n_prob = 0, units = 0;
+  long long used = 0;
+  auto flush = [&]() -> cudaError_t {
+    if (n_prob == 0) return cudaSuccess;
+    P->n_prob = n_prob;
+    backward_common_params(*P, B, S, D, causal);
+    const cudaError_t e = launch_bwd_kernels(*P, D, stream);
+    std::memset(P.get(), 0, sizeof(BwdParams));
+    n_prob = 0;
+    units = 0;
+    used = 0;
+    return e;
+  };
+  for (const BwdProblem &set : sets) {
+    for (int h = 0; h < set.H;) {
+      if (n_prob == kMaxProblems || (cap > 0 && used == cap))
+        if (cudaError_t e = flush(); e != cudaSuccess) return e;
+      BwdProblem &pb = P->prob[n_prob];
+      pb = set;
+      pb.h0 = h;
+      pb.nh = cap > 0 ? static_cast<int>(std::min<long long>(set.H - h, cap - used)) : set.H;
+      pb.ds = cap > 0 ? scratch + static_cast<size_t>(used) * per_head : nullptr;
+      pb.unit_base = units;
+      units += B * pb.nh * nt;
+      used += cap > 0 ? pb.nh : 0;
+      h += pb.nh;
+      ++n_prob;
+    }
+  }
+  return flush();
+}
+
 int cpattn_attention_backward(const void *q, const void *k, const void *v, const void *out, const float *lse,
                               const void *dout, void *dq, void *dk, void *dv, int B, int H, int S, int D,
                               int causal, void *workspace, size_t workspace_bytes, cpattn_stream_t stream) {
@@ -1327,23 +1416,25 @@ int cpattn_attention_backward(const void *q, const void *k, const void *v, const
     return CPATTN_ERR_NULL;
   int st = check_bwd_shape(B, H, S, D);
   if (st != CPATTN_OK) return st;
-  if (workspace == nullptr || workspace_bytes < cpattn_attention_backward_workspace_bytes(B, H, S))
-    return CPATTN_ERR_WORKSPACE;
+  const size_t delta_bytes = cpattn_attention_backward_workspace_bytes(B, H, S);
+  if (workspace == nullptr || workspace_bytes < delta_bytes) return CPATTN_ERR_WORKSPACE;
   const void *ptrs[8] = {q, k, v, out, dout, dq, dk, dv};
   for (const void *ptr : ptrs)
     if (!aligned16(ptr)) return CPATTN_ERR_ALIGNMENT;
   if (!aligned4(lse) || !aligned4(workspace)) return CPATTN_ERR_ALIGNMENT;
   st = check_device(nullptr);
   if (st != CPATTN_OK) return st;
-  std::unique_ptr<BwdParams> P(new BwdParams);
-  std::memset(P.get(), 0, sizeof(BwdParams));
-  if (!backward_problem(P->prob[0], q, k, v, dout, lse, static_cast<long long>(H) * S, S, 0,
-                        static_cast<float *>(workspace), dq, dk, dv, B, S, H, D, 0))
+  std::vector<BwdProblem> sets(1);
+  float *delta = static_cast<float *>(workspace);
+  if (!backward_problem(sets[0], q, k, v, dout, lse, static_cast<long long>(H) * S, S, 0, delta, dq, dk, dv, B, S,
+                        H, D))
     return cuda_fail(cudaErrorInvalidValue, t_encode_detail);
-  P->n_prob = 1;
-  backward_common_params(*P, B, S, D, causal != 0);
-  const void *outs[1] = {out}, *douts[1] = {dout};
-  return cuda_result(launch_attention_backward(*P, D, outs, douts, stream), "backward launch");
+  unsigned char *scratch;
+  size_t scratch_bytes;
+  ds_scratch(workspace, workspace_bytes, delta_bytes, scratch, scratch_bytes);
+  if (cudaError_t e = launch_bwd_delta(out, dout, delta, B, S, H, D, stream); e != cudaSuccess)
+    return cuda_fail(e, "backward launch");
+  return cuda_result(run_bwd_sets(sets, scratch, scratch_bytes, B, S, D, causal != 0, stream), "backward launch");
 }
 
 size_t cpattn_ulysses_attention_backward_workspace_bytes(int B, int H, int S, int D) {
@@ -1367,8 +1458,8 @@ int cpattn_ulysses_attention_backward(const void *q, const void *k, const void *
   if (st != CPATTN_OK) return st;
   st = resolve_splits(H, degree, head_splits, heads);
   if (st != CPATTN_OK) return st;
-  if (workspace == nullptr || workspace_bytes < cpattn_ulysses_attention_backward_workspace_bytes(B, H, S, D))
-    return CPATTN_ERR_WORKSPACE;
+  const size_t base_bytes = cpattn_ulysses_attention_backward_workspace_bytes(B, H, S, D);
+  if (workspace == nullptr || workspace_bytes < base_bytes) return CPATTN_ERR_WORKSPACE;
   PermuteParams pq;
   st = permute_common(q, workspace, B, S, H, D, 2, degree, seq_splits, head_splits, 0, pq);
   if (st != CPATTN_OK) return st;
@@ -1378,12 +1469,16 @@ int cpattn_ulysses_attention_backward(const void *q, const void *k, const void *
   if (!aligned4(lse)) return CPATTN_ERR_ALIGNMENT;
   st = check_device(nullptr);
   if (st != CPATTN_OK) return st;
-  // workspace: head-side yq, yk, yv, yo, ydo, ydq, ydk, ydv, then Delta per head rank
+  // workspace: head-side yq, yk, yv, yo, ydo, ydq, ydk, ydv, then Delta per
+  // head rank, then (optionally) dS scratch
   const size_t tb = static_cast<size_t>(B) * S * H * D * 2;
   char *ws = static_cast<char *>(workspace);
   void *y[8];
   for (int i = 0; i < 8; ++i) y[i] = ws + i * tb;
   float *delta = reinterpret_cast<float *>(ws + 8 * tb);
+  unsigned char *scratch;
+  size_t scratch_bytes;
+  ds_scratch(workspace, workspace_bytes, base_bytes, scratch, scratch_bytes);
   // first all-to-all: Q, K, V, then O and dO, to the head-sharded layout
   {
     PermuteParams pp = pq;
@@ -1396,43 +1491,25 @@ int cpattn_ulysses_attention_backward(const void *q, const void *k, const void *
     pp.n_tensors = 2;
     if (cudaError_t e = launch_permute(pp, stream); e != cudaSuccess) return cuda_fail(e, "permute launch");
   }
-  // the backward of every head rank's local attention, one launch per kernel
-  std::unique_ptr<BwdParams> P(new BwdParams);
-  std::memset(P.get(), 0, sizeof(BwdParams));
+  // the backward of every head rank's local attention: one problem per head
+  // rank, its Delta first
   const std::vector<int> ho = prefix(heads);
-  const int nt = (S + 127) / 128;
-  std::vector<const void *> outs, douts;
-  int n_prob = 0, units = 0;
+  std::vector<BwdProblem> sets;
+  sets.reserve(degree);
   for (int u = 0; u < degree; ++u) {
     if (heads[u] == 0) continue;
-    if (n_prob == kMaxProblems) {   // a full parameter table: launch it and start the next
-      P->n_prob = n_prob;
-      backward_common_params(*P, B, S, D, causal != 0);
-      if (cudaError_t e = launch_attention_backward(*P, D, outs.data(), douts.data(), stream); e != cudaSuccess)
-        return cuda_fail(e, "backward launch");
-      std::memset(P.get(), 0, sizeof(BwdParams));
-      outs.clear();
-      douts.clear();
-      n_prob = 0;
-      units = 0;
-    }
     const size_t off = static_cast<size_t>(B) * S * ho[u] * D * 2;
     auto at = [&](int i) { return static_cast<void *>(static_cast<char *>(y[i]) + off); };
-    if (!backward_problem(P->prob[n_prob], at(0), at(1), at(2), at(4), lse, static_cast<long long>(H) * S, S, ho[u],
-                          delta + static_cast<size_t>(B) * ho[u] * S, at(5), at(6), at(7), B, S, heads[u], D,
-                          units))
+    float *dl = delta + static_cast<size_t>(B) * ho[u] * S;
+    sets.emplace_back();
+    if (!backward_problem(sets.back(), at(0), at(1), at(2), at(4), lse, static_cast<long long>(H) * S, S, ho[u], dl,
+                          at(5), at(6), at(7), B, S, heads[u], D))
       return cuda_fail(cudaErrorInvalidValue, t_encode_detail);
-    outs.push_back(at(3));
-    douts.push_back(at(4));
-    units += B * heads[u] * nt;
-    ++n_prob;
-  }
-  if (n_prob > 0) {
-    P->n_prob = n_prob;
-    backward_common_params(*P, B, S, D, causal != 0);
-    if (cudaError_t e = launch_attention_backward(*P, D, outs.data(), douts.data(), stream); e != cudaSuccess)
+    if (cudaError_t e = launch_bwd_delta(at(3), at(4), dl, B, S, heads[u], D, stream); e != cudaSuccess)
       return cuda_fail(e, "backward launch");
   }
+  if (cudaError_t e = run_bwd_sets(sets, scratch, scratch_bytes, B, S, D, causal != 0, stream); e != cudaSuccess)
+    return cuda_fail(e, "backward launch");
   // second all-to-all: dQ, dK, dV back to the sequence-sharded layout
   PermuteParams pb = pq;
   set_qkv(pb, y[5], y[6], y[7], dq, dk, dv);

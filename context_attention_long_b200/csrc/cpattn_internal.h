@@ -113,11 +113,29 @@ struct alignas(64) BwdProblem {
   long long lse_b;
   long long lse_h;
   int lse_h0;
-  int H;
+  int H;                                 // heads of the tensors
+  int h0, nh;                            // the heads [h0, h0 + nh) that this problem's units cover
   float *delta;                          // [B, H, S] rowsum(dO * O) of this problem
   void *dq, *dk, *dv;                    // [B, S, H, D] bf16
+  // dS tiles of heads [h0, h0 + nh): written by the dK/dV kernel, read by the
+  // dQ GEMM (null: the dQ kernel recomputes S and dP instead).  Tile (b, h,
+  // q tile, k tile) at bwd_ds_tile_index * kBwdDsTileBytes, each tile
+  // [4 quarters of 32 keys][16 groups of 8 queries][32 keys][8 queries] bf16;
+  // 256-byte aligned.
+  unsigned char *ds;
   int unit_base;                         // first unit (blockIdx) of this problem
 };
+constexpr int kBwdDsTileBytes = 128 * 128 * 2;
+// dS tiles per (b, h): every (q tile, k tile) pair, or under the causal mask
+// only the pairs with kt <= qt (the dK/dV kernel walks no others).  A Q tile's
+// k tiles are consecutive either way.
+__host__ __device__ inline long long bwd_ds_tiles_per_head(int nt, bool causal) {
+  return causal ? static_cast<long long>(nt) * (nt + 1) / 2 : static_cast<long long>(nt) * nt;
+}
+__host__ __device__ inline long long bwd_ds_tile_index(int b, int hl, int nh, int nt, int qt, int kt, bool causal) {
+  const long long within = causal ? static_cast<long long>(qt) * (qt + 1) / 2 + kt : static_cast<long long>(qt) * nt + kt;
+  return (static_cast<long long>(b) * nh + hl) * bwd_ds_tiles_per_head(nt, causal) + within;
+}
 struct BwdParams {
   BwdProblem prob[kMaxProblems];
   int n_prob;
@@ -127,9 +145,13 @@ struct BwdParams {
   float scale;                           // D**-0.5
   unsigned long long timeout_ns;
 };
-// outs/douts: per problem the forward output and its gradient (for the row sums).
-cudaError_t launch_attention_backward(const BwdParams &p, int D, const void *const *outs, const void *const *douts,
-                                      cudaStream_t stream);
+// Delta = rowsum(dO * O) over [B, S, H, D] tensors into delta[B, H, S].
+cudaError_t launch_bwd_delta(const void *out, const void *dout, float *delta, int B, int S, int H, int D,
+                             cudaStream_t stream);
+// The gradient kernels over every problem of p (Delta already computed): with
+// dS tiles (every problem's ds set) the dK/dV kernel stores dS and the dQ
+// GEMM follows; without, the dQ and dK/dV kernels.
+cudaError_t launch_bwd_kernels(const BwdParams &p, int D, cudaStream_t stream);
 
 // ---------------------------------------------------------------- LSE merge
 struct MergeParams {

@@ -488,14 +488,26 @@ int cpattn_causal_unified_attention(const void *q, const void *k, const void *v,
  *   dq, dk, dv          [B, S, H, D] bf16 device, written.
  *   workspace           device, at least
  *                       cpattn_attention_backward_workspace_bytes(B, H, S)
- *                       bytes, 4-byte aligned (holds rowsum(dO * O)).
- * Three launches on `stream`: the row sums, a dQ kernel (one CTA per Q tile,
- * walking the K/V tiles) and a dK/dV kernel (one CTA per K/V tile, walking the
- * Q tiles); no atomics.  Errors: NULL, SHAPE (also when B*S*H >= 2^31, a
- * tensor larger than any device memory), WORKSPACE, ALIGNMENT, UNSUPPORTED,
- * CUDA.
+ *                       bytes, 4-byte aligned (holds rowsum(dO * O)).  Bytes
+ *                       beyond that, from the next 256-byte boundary, are
+ *                       scratch for dS: each head takes
+ *                       cpattn_attention_backward_ds_bytes(B, S, causal).
+ * With scratch for at least one head: the row sums, then per group of heads
+ * whose dS fits the scratch together (all heads in one group when it holds
+ * H heads' worth) a dK/dV kernel (one CTA per K/V tile, walking the Q tiles)
+ * that also stores dS in bf16, and a dQ GEMM (dQ = dS K * D**-0.5, persistent,
+ * reading the stored dS).  Without: the row sums, a dQ kernel (one CTA per Q
+ * tile, walking the K/V tiles and computing S and dP again) and the dK/dV
+ * kernel.  No atomics either way, and dK and dV are the same bytes in both;
+ * dQ differs by the rounding of the dS the two kernels form.  Errors: NULL,
+ * SHAPE (also when B*S*H >= 2^31, a tensor larger than any device memory),
+ * WORKSPACE, ALIGNMENT, UNSUPPORTED, CUDA.
  */
 size_t cpattn_attention_backward_workspace_bytes(int B, int H, int S);
+/* Bytes of dS scratch one head takes: B * 32 KB per (Q tile, K tile) pair of
+ * 128-row tiles, all pairs, or under the causal mask (causal != 0) those with
+ * the K tile at or before the Q tile.  0 when B or S < 1. */
+size_t cpattn_attention_backward_ds_bytes(int B, int S, int causal);
 int cpattn_attention_backward(const void *q, const void *k, const void *v, const void *out,
                               const float *lse, const void *dout, void *dq, void *dk, void *dv,
                               int B, int H, int S, int D, int causal, void *workspace,
@@ -505,9 +517,9 @@ int cpattn_attention_backward(const void *q, const void *k, const void *v, const
  * Backward of the Ulysses flow ([USP] section 4 run in reverse for training,
  * sections 1 and 7): the first all-to-all takes Q, K, V, the forward output O
  * and its gradient dO to the head-sharded layout (two launches), the attention
- * backward runs on every head rank's buffers (one dQ and one dK/dV launch for
- * up to 8 head ranks), and the second all-to-all brings dQ, dK and dV back to
- * the sequence-sharded layout.
+ * backward of cpattn_attention_backward runs on every head rank's buffers (its
+ * kernels cover up to 8 head ranks, or groups of heads, per launch), and the
+ * second all-to-all brings dQ, dK and dV back to the sequence-sharded layout.
  *
  *   q, k, v, out, dout  sequence-sharded rank buffers, as the inputs and the
  *                       output of cpattn_ulysses_attention; read only.
@@ -515,7 +527,9 @@ int cpattn_attention_backward(const void *q, const void *k, const void *v, const
  *   dq, dk, dv          sequence-sharded rank buffers, written.
  *   workspace           device, 16-byte aligned, at least
  *                       cpattn_ulysses_attention_backward_workspace_bytes()
- *                       = 16 * B*S*H*D + 4 * B*H*S bytes.
+ *                       = 16 * B*S*H*D + 4 * B*H*S bytes; bytes beyond that,
+ *                       from the next 256-byte boundary, are dS scratch as in
+ *                       cpattn_attention_backward.
  * Other arguments, splits and errors as cpattn_ulysses_attention (SHAPE also
  * when B*S*H >= 2^31); causal = 1 for the causal mask.
  */

@@ -268,6 +268,42 @@ def test_backward_validation(lib):
         assert f() == CUDA
 
 
+def test_backward_ds_bytes(lib):
+    """dS scratch per head: B x 32 KB (a 128 x 128 bf16 tile) per (Q tile, K
+    tile) pair the dK/dV kernel walks -- every pair, or under the causal mask
+    the pairs whose K tile starts at or before the Q tile's last query
+    (counted here by brute force)."""
+    for B, S in ((1, 1), (2, 300), (1, 4608), (3, 257), (1, 9216)):
+        nt = (S + 127) // 128
+        causal_pairs = sum(1 for qt in range(nt) for kt in range(nt) if kt * 128 <= min(S, qt * 128 + 128) - 1)
+        assert lib.cpattn_attention_backward_ds_bytes(B, S, 0) == B * nt * nt * 128 * 128 * 2
+        assert lib.cpattn_attention_backward_ds_bytes(B, S, 1) == B * causal_pairs * 128 * 128 * 2
+    assert lib.cpattn_attention_backward_ds_bytes(1, 4608, 0) == 42467328     # image-DiT: 42.5 MB per head
+    assert lib.cpattn_attention_backward_ds_bytes(0, 256, 0) == 0
+    assert lib.cpattn_attention_backward_ds_bytes(1, 0, 1) == 0
+
+
+def test_backward_workspace_budget():
+    """The bindings add whole heads of dS scratch within the budget (plus
+    256 bytes of alignment slack), or none when one head does not fit."""
+    from context_attention_long_b200 import api
+    base = api.cpattn_attention_backward_workspace_bytes(2, 5, 300)
+    per = api.cpattn_attention_backward_ds_bytes(2, 300, False)
+    assert api.backward_workspace_bytes(2, 5, 300) == base + 256 + 5 * per
+    assert api.backward_workspace_bytes(2, 5, 300, ds_budget=0) == base
+    assert api.backward_workspace_bytes(2, 5, 300, ds_budget=per - 1) == base
+    assert api.backward_workspace_bytes(2, 5, 300, ds_budget=2 * per + 7) == base + 256 + 2 * per
+    per_c = api.cpattn_attention_backward_ds_bytes(2, 300, True)
+    assert api.backward_workspace_bytes(2, 5, 300, causal=True, ds_budget=2 * per) == base + 256 + 3 * per_c
+    ubase = api.cpattn_ulysses_attention_backward_workspace_bytes(2, 5, 300, 64)
+    assert api.backward_workspace_bytes(2, 5, 300, ulysses_D=64, ds_budget=per) == ubase + 256 + per
+    # the video workload: 2.1 GB of dS per head, so the default budget takes 3 of its 40 heads
+    per_v = api.cpattn_attention_backward_ds_bytes(1, 32760, False)
+    assert per_v == 256 * 256 * 32768
+    assert api.backward_workspace_bytes(1, 40, 32760) == (api.cpattn_attention_backward_workspace_bytes(1, 40, 32760)
+                                                          + 256 + (api.BACKWARD_DS_BUDGET // per_v) * per_v)
+
+
 def test_ulysses_backward_validation(lib):
     need = lib.cpattn_ulysses_attention_backward_workspace_bytes(1, 4, 8, 64)
     assert need == 16 * 1 * 8 * 4 * 64 + 4 * 1 * 4 * 8

@@ -2,7 +2,11 @@
 backward oracle: dQ, dK and dV for seeded inputs and a seeded upstream
 gradient, causal and not, over tile-spanning and ragged shapes, D = 64 and
 128, S = 1, and the image-DiT workload on sampled rows.  The forward output
-and LSE come from the library's own forward.
+and LSE come from the library's own forward.  Each small case runs on the
+backward's three paths: dS stored by the dK/dV kernel and read by the dQ GEMM
+with every head in one group, the same in groups of one head (a workspace
+with one head's dS scratch), and the dQ kernel that recomputes S and dP (no
+scratch).
 
 Tolerance: every gradient is compared relative to its largest reference
 entry g = max|ref|: max-abs error <= 2e-2 * g and mean-abs error <= 2e-3 * g.
@@ -47,24 +51,36 @@ def assert_grad_close(got, ref, what, dout_max=1.0):
     assert err.mean() <= 2e-3 * g, f"{what}: mean-abs {err.mean():.3e} vs {g:.3e}"
 
 
-def _run(B, S, H, D, causal, seed):
+# ds_budget of each path (None: the binding's default, every head at once here;
+# "one": one head's dS scratch, so the heads run in groups of one)
+PATHS = {"gemm": None, "gemm_groups": "one", "dq_kernel": 0}
+
+
+def _budget(path, B, S, causal):
+    b = PATHS[path]
+    return api.cpattn_attention_backward_ds_bytes(B, S, causal) if b == "one" else b
+
+
+def _run(B, S, H, D, causal, seed, path="gemm"):
     qb, kb, vb = inputs.make_qkv(B, S, H, D, seed, D == 128)
     rng = np.random.Generator(np.random.PCG64(seed + 1))
     dob = inputs.f32_to_bf16_bits(rng.standard_normal((B, S, H, D)).astype(np.float32))
     q, k, v, do = (to_dev(x) for x in (qb, kb, vb, dob))
     fwd = api.cpattn_causal_ring_attention if causal else api.cpattn_ring_attention
     out, lse = fwd(q, k, v, 1)
-    dq, dk, dv = api.cpattn_attention_backward(q, k, v, out, lse, do, causal=causal)
+    dq, dk, dv = api.cpattn_attention_backward(q, k, v, out, lse, do, causal=causal,
+                                               ds_budget=_budget(path, B, S, causal))
     torch.cuda.synchronize()
     _no_timeouts()
     return (qb, kb, vb, dob), (dq, dk, dv)
 
 
+@pytest.mark.parametrize("path", list(PATHS))
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("B,S,H,D", [(1, 256, 2, 64), (2, 300, 3, 128), (1, 129, 2, 128), (1, 1, 1, 64),
                                      (1, 640, 2, 128)])
-def test_backward_matches_oracle(B, S, H, D, causal):
-    bits, grads = _run(B, S, H, D, causal, 31 + S)
+def test_backward_matches_oracle(B, S, H, D, causal, path):
+    bits, grads = _run(B, S, H, D, causal, 31 + S, path)
     q, k, v, do = (inputs.bf16_bits_to_f64(x) for x in bits)
     refs = oracle.attention_backward(q, k, v, do, causal=causal)
     for name, got, ref in zip(("dq", "dk", "dv"), grads, refs):
@@ -94,6 +110,37 @@ def test_backward_dit_workload_sampled_heads(causal):
                               np.abs(inputs.bf16_bits_to_f64(dob)).max())
 
 
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("B,S,H,D", [(2, 300, 5, 128), (1, 520, 3, 64)])
+def test_backward_paths_agree(B, S, H, D, causal):
+    """dK and dV come from the same dK/dV kernel on every path: the same
+    bytes.  dQ from the GEMM reads the same stored dS tiles whatever the
+    grouping of the heads: the same bytes too.  The dQ kernel forms its own dS
+    (checked against the oracle above)."""
+    runs = {path: _run(B, S, H, D, causal, 300 + S, path)[1] for path in PATHS}
+    two = api.cpattn_attention_backward_ds_bytes(B, S, causal) * 2
+
+    def bits(t):
+        return t.view(torch.int16)
+
+    for path, (dq, dk, dv) in runs.items():
+        assert torch.equal(bits(dk), bits(runs["gemm"][1])), f"dk {path}"
+        assert torch.equal(bits(dv), bits(runs["gemm"][2])), f"dv {path}"
+    assert torch.equal(bits(runs["gemm_groups"][0]), bits(runs["gemm"][0]))
+    # groups of two heads (the last group holds one when H is odd)
+    qb, kb, vb = inputs.make_qkv(B, S, H, D, 300 + S, D == 128)
+    rng = np.random.Generator(np.random.PCG64(301 + S))
+    dob = inputs.f32_to_bf16_bits(rng.standard_normal((B, S, H, D)).astype(np.float32))
+    q, k, v, do = (to_dev(x) for x in (qb, kb, vb, dob))
+    fwd = api.cpattn_causal_ring_attention if causal else api.cpattn_ring_attention
+    out, lse = fwd(q, k, v, 1)
+    g2 = api.cpattn_attention_backward(q, k, v, out, lse, do, causal=causal, ds_budget=two)
+    torch.cuda.synchronize()
+    _no_timeouts()
+    for a, b in zip(g2, runs["gemm"]):
+        assert torch.equal(bits(a), bits(b))
+
+
 def test_backward_is_deterministic_and_validates():
     bits, g1 = _run(1, 384, 2, 128, True, 5)
     _, g2 = _run(1, 384, 2, 128, True, 5)
@@ -105,15 +152,16 @@ def test_backward_is_deterministic_and_validates():
     assert lib.cpattn_attention_backward(F, F, F, F, F, F, F, F, F, 1, 2, 384, 128, 0, F, 16, None) == 8
 
 
+@pytest.mark.parametrize("path", list(PATHS))
 @pytest.mark.parametrize("B,S,H,D,P,seq,heads,causal", [
     (1, 256, 4, 64, 2, None, None, False),
     (2, 300, 7, 128, 3, [100, 50, 150], [3, 2, 2], True),
     (1, 1000, 6, 128, 4, [250, 250, 250, 250], [2, 2, 1, 1], False),
     (1, 320, 10, 64, 10, None, None, True),     # 10 head ranks: more problems than one launch holds
 ])
-def test_ulysses_backward_matches_oracle(B, S, H, D, P, seq, heads, causal):
+def test_ulysses_backward_matches_oracle(B, S, H, D, P, seq, heads, causal, path):
     """The backward of the Ulysses flow on sequence-sharded rank buffers, with
-    the forward's output and LSE from the Ulysses forward."""
+    the forward's output and LSE from the Ulysses forward, on each path."""
     seq_l = seq or [S // P] * P
     qb, kb, vb = inputs.make_qkv(B, S, H, D, 90 + S, D == 128)
     rng = np.random.Generator(np.random.PCG64(91 + S))
@@ -121,7 +169,8 @@ def test_ulysses_backward_matches_oracle(B, S, H, D, P, seq, heads, causal):
     q, k, v, do = (to_dev(full_to_rank_buffers(x, seq_l)) for x in (qb, kb, vb, dob))
     fwd = api.cpattn_causal_ulysses_attention if causal else api.cpattn_ulysses_attention
     out, lse = fwd(q, k, v, B, S, H, D, P, seq, heads)
-    dq, dk, dv = api.cpattn_ulysses_attention_backward(q, k, v, out, lse, do, B, S, H, D, P, seq, heads, causal)
+    dq, dk, dv = api.cpattn_ulysses_attention_backward(q, k, v, out, lse, do, B, S, H, D, P, seq, heads, causal,
+                                                       ds_budget=_budget(path, B, S, causal))
     torch.cuda.synchronize()
     _no_timeouts()
     refs = oracle.attention_backward(*(inputs.bf16_bits_to_f64(x) for x in (qb, kb, vb, dob)), causal=causal)
