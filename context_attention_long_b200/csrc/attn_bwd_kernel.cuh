@@ -863,9 +863,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __gr
 // dS tiles (32 KB per tile pair).  Persistent: one CTA per SM walks the units
 // blockIdx.x, blockIdx.x + gridDim.x, ...; two TMEM accumulators, so that the
 // epilogue of one unit overlaps the loads and MMAs of the next.  Units run
-// head by head (the CTAs at work share a few heads' K tiles in L2), the last
-// Q tile of a head first under the causal mask; the stride of the walk mixes
-// long and short causal units in every CTA.
+// head by head (the CTAs at work share a few heads' K tiles in L2); under the
+// causal mask in pairs of equal total length (bwd_gemm_unit).
 //   warp 0      producer: the dS tile (bulk copy) and the K tile (TMA) per stage
 //   warp 1      TMEM allocator + single-thread MMA issuer
 //   warps 2-5   epilogue: one dQ row per thread (TMEM lane), scaled, bf16
@@ -885,9 +884,42 @@ static_assert(BwdGemmSmem<128>::kAllocBytes <= 232448 && BwdGemmSmem<64>::kAlloc
               "dQ GEMM shared memory exceeds the per-CTA limit");
 constexpr int kBwdGemmThreads = 192;
 
+// The k-th unit of this CTA's walk.  The CTA takes work items blockIdx.x,
+// blockIdx.x + gridDim.x, ... in head order.  Without the causal mask an item
+// is one Q tile.  Under it an item pairs Q tile nt - 1 - j with Q tile j of
+// the same (b, h): together they walk nt + 1 K tiles, so that every item has
+// the same length and the round-robin stays balanced.  Returns 0 when the walk
+// is done, 1 for a unit, -1 for the second of a pair that is its first (the
+// middle tile of an odd nt), which every role skips alike.
+__device__ __forceinline__ int bwd_gemm_unit(const BwdParams &p, int k, bool causal, BwdUnit &u) {
+  const int nt = (p.S + 127) / 128;
+  const int per = causal ? (nt + 1) / 2 : nt;   // items per (b, h)
+  const int sub = causal ? (k & 1) : 0;
+  int item = static_cast<int>(blockIdx.x) + (causal ? (k >> 1) : k) * static_cast<int>(gridDim.x);
+  int pi = 0;
+  for (; pi < p.n_prob; ++pi) {
+    const int items = p.B * p.prob[pi].nh * per;
+    if (item < items) break;
+    item -= items;
+  }
+  if (pi == p.n_prob) return 0;
+  const int bh = item / per, j = item - bh * per;
+  const int NH = p.prob[pi].nh;
+  u.pi = pi;
+  u.hl = bh % NH;
+  u.h = p.prob[pi].h0 + u.hl;
+  u.b = bh / NH;
+  if (!causal) {
+    u.t = j;
+    return 1;
+  }
+  u.t = sub == 0 ? nt - 1 - j : j;
+  return (sub == 1 && j == nt - 1 - j) ? -1 : 1;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kBwdGemmThreads, 1)
-    attn_bwd_dq_gemm_kernel(const __grid_constant__ BwdParams p, int n_units) {
+    attn_bwd_dq_gemm_kernel(const __grid_constant__ BwdParams p) {
   using L = BwdGemmSmem<D>;
   using T = BwdSmem<D>;
   constexpr uint32_t IDESC = idesc_bf16_f32(128, D, true, true);   // dS and K both MN-major
@@ -952,8 +984,11 @@ __global__ void __launch_bounds__(kBwdGemmThreads, 1)
       const uint64_t once = l2_evict_first_policy();
       int it = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
-        const BwdUnit U = bwd_unit_at(p, u, causal);
+      for (int k = 0; ok; ++k) {
+        BwdUnit U;
+        const int got = bwd_gemm_unit(p, k, causal, U);
+        if (got == 0) break;
+        if (got < 0) continue;
         const BwdProblem &PB = p.prob[U.pi];
         const int n = walked(U.t);
         const unsigned char *a0 = PB.ds + bwd_ds_tile_index(U.b, U.hl, PB.nh, nt, U.t, 0, causal) * kBwdDsTileBytes;
@@ -983,11 +1018,16 @@ __global__ void __launch_bounds__(kBwdGemmThreads, 1)
     if (lane == 0) {
       int it = 0, local = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x, ++local) {
-        const BwdUnit U = bwd_unit_at(p, u, causal);
+      for (int k = 0; ok; ++k) {
+        BwdUnit U;
+        const int got = bwd_gemm_unit(p, k, causal, U);
+        if (got == 0) break;
+        if (got < 0) continue;
         const int n = walked(U.t);
         const int a = local & 1;
-        if (!mbar_wait_spin(sb + BAR_AE + 8 * a, ((local >> 1) & 1) ^ 1, abort_flag, tmo, SITE_MMA)) break;
+        const uint32_t use = static_cast<uint32_t>(local >> 1);   // uses of accumulator a before this one
+        ++local;
+        if (!mbar_wait_spin(sb + BAR_AE + 8 * a, (use & 1) ^ 1, abort_flag, tmo, SITE_MMA)) break;
         tc_fence_after();
         const uint32_t d = tmem + a * D;
         for (int j = 0; j < n; ++j, ++it) {
@@ -1021,13 +1061,18 @@ __global__ void __launch_bounds__(kBwdGemmThreads, 1)
     const int r = quarter * 32 + lane;   // accumulator row = TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     int local = 0;
-    for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++local) {
+    for (int k = 0;; ++k) {
+      BwdUnit U;
+      const int got = bwd_gemm_unit(p, k, causal, U);
+      if (got == 0) break;
+      if (got < 0) continue;
       const int a = local & 1;
-      const bool w = mbar_wait(sb + BAR_AF + 8 * a, (local >> 1) & 1, abort_flag, tmo, SITE_EPILOGUE);
+      const uint32_t use = static_cast<uint32_t>(local >> 1);
+      ++local;
+      const bool w = mbar_wait(sb + BAR_AF + 8 * a, use & 1, abort_flag, tmo, SITE_EPILOGUE);
       if (__any_sync(0xffffffffu, !w)) break;
       __syncwarp();
       tc_fence_after();
-      const BwdUnit U = bwd_unit_at(p, u, causal);
       const BwdProblem &PB = p.prob[U.pi];
       const int q = U.t * 128 + r;
       const bool row_ok = q < p.S;

@@ -289,7 +289,7 @@ static cudaError_t launch_bwd_d(const BwdParams &p, int units, cudaStream_t stre
   // one CTA per SM (its shared memory admits no second), each walking units
   const int grid = std::min(units, std::max(sms[dev], 1));
   attn_bwd_dq_gemm_kernel<D><<<static_cast<unsigned>(grid), kBwdGemmThreads, BwdGemmSmem<D>::kAllocBytes, stream>>>(
-      p, units);
+      p);
   return cudaGetLastError();
 }
 
