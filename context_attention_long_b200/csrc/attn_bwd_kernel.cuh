@@ -194,6 +194,21 @@ __device__ __forceinline__ BwdUnit bwd_unit(const BwdParams &p, bool last_first)
   return bwd_unit_at(p, static_cast<int>(blockIdx.x), last_first);
 }
 
+// Element offset of the gradient row of (batch b, sequence position s, head
+// h) by the problem's output map (see BwdProblem).
+template <int D>
+__device__ __forceinline__ long long bwd_out_elems(const BwdProblem &PB, int B, int S, int b, int s, int h) {
+  if (PB.out_mode == 0) return ((static_cast<long long>(b) * S + s) * PB.H + h) * D;
+  int lo = 0, hi = PB.out_nseq - 1;   // the sequence rank holding s (empty ranks are never found)
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (PB.out_seq_off[mid] <= s) lo = mid; else hi = mid - 1;
+  }
+  const int off = PB.out_seq_off[lo], len = PB.out_seq_off[lo + 1] - off;
+  const long long row = static_cast<long long>(B) * off + static_cast<long long>(b) * len + (s - off);
+  return (row * PB.out_H + PB.out_h0 + h) * D;
+}
+
 // ===================================================================== dQ
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
@@ -458,7 +473,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dq_kernel(const __gri
       const float scale = p.scale;
       const int d0 = half * (D / 2);
       __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(PB.dq) +
-                           ((static_cast<long long>(U.b) * p.S + q_pos) * PB.H + U.h) * D + d0;
+                           (row_valid ? bwd_out_elems<D>(PB, p.B, p.S, U.b, q_pos, U.h) : 0) + d0;
 #pragma unroll
       for (int c0 = 0; c0 < D / 2; c0 += 32) {
         uint32_t o[32];
@@ -818,7 +833,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_dkv_kernel(const __gr
     if (ok) {
       // each half of the row writes half of the D columns of dV and of dK
       const int d0 = half * (D / 2);
-      const long long roff = ((static_cast<long long>(U.b) * p.S + k_pos) * PB.H + U.h) * D + d0;
+      const long long roff = (row_valid ? bwd_out_elems<D>(PB, p.B, p.S, U.b, k_pos, U.h) : 0) + d0;
       for (int which = 0; which < 2; ++which) {   // 0: dV, 1: dK (times the softmax scale)
         const float mul = which == 0 ? 1.0f : p.scale;
         __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(which == 0 ? PB.dv : PB.dk) + roff;
@@ -1076,8 +1091,7 @@ __global__ void __launch_bounds__(kBwdGemmThreads, 1)
       const BwdProblem &PB = p.prob[U.pi];
       const int q = U.t * 128 + r;
       const bool row_ok = q < p.S;
-      __nv_bfloat16 *dst =
-          static_cast<__nv_bfloat16 *>(PB.dq) + ((static_cast<long long>(U.b) * p.S + q) * PB.H + U.h) * D;
+      __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(PB.dq) + (row_ok ? bwd_out_elems<D>(PB, p.B, p.S, U.b, q, U.h) : 0);
 #pragma unroll 1
       for (int c = 0; c < D; c += 32) {
         uint32_t v[32];

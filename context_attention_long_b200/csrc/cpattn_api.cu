@@ -1439,7 +1439,7 @@ int cpattn_attention_backward(const void *q, const void *k, const void *v, const
 
 size_t cpattn_ulysses_attention_backward_workspace_bytes(int B, int H, int S, int D) {
   if (B < 1 || H < 1 || S < 1 || D < 1) return 0;
-  return static_cast<size_t>(8) * B * S * H * D * 2 + static_cast<size_t>(B) * H * S * sizeof(float);
+  return static_cast<size_t>(5) * B * S * H * D * 2 + static_cast<size_t>(B) * H * S * sizeof(float);
 }
 
 int cpattn_ulysses_attention_backward(const void *q, const void *k, const void *v, const void *out,
@@ -1469,13 +1469,13 @@ int cpattn_ulysses_attention_backward(const void *q, const void *k, const void *
   if (!aligned4(lse)) return CPATTN_ERR_ALIGNMENT;
   st = check_device(nullptr);
   if (st != CPATTN_OK) return st;
-  // workspace: head-side yq, yk, yv, yo, ydo, ydq, ydk, ydv, then Delta per
-  // head rank, then (optionally) dS scratch
+  // workspace: head-side yq, yk, yv, yo, ydo, then Delta per head rank, then
+  // (optionally) dS scratch
   const size_t tb = static_cast<size_t>(B) * S * H * D * 2;
   char *ws = static_cast<char *>(workspace);
-  void *y[8];
-  for (int i = 0; i < 8; ++i) y[i] = ws + i * tb;
-  float *delta = reinterpret_cast<float *>(ws + 8 * tb);
+  void *y[5];
+  for (int i = 0; i < 5; ++i) y[i] = ws + i * tb;
+  float *delta = reinterpret_cast<float *>(ws + 5 * tb);
   unsigned char *scratch;
   size_t scratch_bytes;
   ds_scratch(workspace, workspace_bytes, base_bytes, scratch, scratch_bytes);
@@ -1492,8 +1492,10 @@ int cpattn_ulysses_attention_backward(const void *q, const void *k, const void *
     if (cudaError_t e = launch_permute(pp, stream); e != cudaSuccess) return cuda_fail(e, "permute launch");
   }
   // the backward of every head rank's local attention: one problem per head
-  // rank, its Delta first
+  // rank, its Delta first.  The kernels store dQ, dK and dV straight into the
+  // sequence-sharded rank buffers (the second all-to-all, fused).
   const std::vector<int> ho = prefix(heads);
+  const std::vector<int> so = prefix(seq_chk);
   std::vector<BwdProblem> sets;
   sets.reserve(degree);
   for (int u = 0; u < degree; ++u) {
@@ -1502,19 +1504,19 @@ int cpattn_ulysses_attention_backward(const void *q, const void *k, const void *
     auto at = [&](int i) { return static_cast<void *>(static_cast<char *>(y[i]) + off); };
     float *dl = delta + static_cast<size_t>(B) * ho[u] * S;
     sets.emplace_back();
-    if (!backward_problem(sets.back(), at(0), at(1), at(2), at(4), lse, static_cast<long long>(H) * S, S, ho[u], dl,
-                          at(5), at(6), at(7), B, S, heads[u], D))
+    BwdProblem &pb = sets.back();
+    if (!backward_problem(pb, at(0), at(1), at(2), at(4), lse, static_cast<long long>(H) * S, S, ho[u], dl, dq, dk,
+                          dv, B, S, heads[u], D))
       return cuda_fail(cudaErrorInvalidValue, t_encode_detail);
+    pb.out_mode = 1;
+    pb.out_H = H;
+    pb.out_h0 = ho[u];
+    pb.out_nseq = degree;
+    for (int r = 0; r <= degree; ++r) pb.out_seq_off[r] = so[r];
     if (cudaError_t e = launch_bwd_delta(at(3), at(4), dl, B, S, heads[u], D, stream); e != cudaSuccess)
       return cuda_fail(e, "backward launch");
   }
-  if (cudaError_t e = run_bwd_sets(sets, scratch, scratch_bytes, B, S, D, causal != 0, stream); e != cudaSuccess)
-    return cuda_fail(e, "backward launch");
-  // second all-to-all: dQ, dK, dV back to the sequence-sharded layout
-  PermuteParams pb = pq;
-  set_qkv(pb, y[5], y[6], y[7], dq, dk, dv);
-  pb.direction = 1;
-  return cuda_result(launch_permute(pb, stream), "permute launch");
+  return cuda_result(run_bwd_sets(sets, scratch, scratch_bytes, B, S, D, causal != 0, stream), "backward launch");
 }
 
 int cpattn_exchange_bytes(int mode, int B, int H, int S, int D, int elem_bytes, int degree, const int *seq_splits,

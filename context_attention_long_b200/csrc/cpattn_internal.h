@@ -116,7 +116,16 @@ struct alignas(64) BwdProblem {
   int H;                                 // heads of the tensors
   int h0, nh;                            // the heads [h0, h0 + nh) that this problem's units cover
   float *delta;                          // [B, H, S] rowsum(dO * O) of this problem
-  void *dq, *dk, *dv;                    // [B, S, H, D] bf16
+  void *dq, *dk, *dv;                    // bf16 gradients, rows placed by the output map below
+  // Where a gradient row goes (batch b, sequence position s, head h):
+  //   out_mode 0: [B, S, H, D], the inputs' layout;
+  //   out_mode 1: the sequence-side rank buffers (B, len_r, out_H, D) of the
+  //               Ulysses exchange, row B*off_r + b*len_r + (s - off_r), head
+  //               out_h0 + h (the backward flow's second all-to-all, fused).
+  int out_mode;
+  int out_H, out_h0;
+  int out_nseq;
+  int out_seq_off[kMaxRanks + 1];
   // dS tiles of heads [h0, h0 + nh): written by the dK/dV kernel, read by the
   // dQ GEMM (null: the dQ kernel recomputes S and dP instead).  Tile (b, h,
   // q tile, k tile) at bwd_ds_tile_index * kBwdDsTileBytes, each tile

@@ -516,10 +516,11 @@ int cpattn_attention_backward(const void *q, const void *k, const void *v, const
 /*
  * Backward of the Ulysses flow ([USP] section 4 run in reverse for training,
  * sections 1 and 7): the first all-to-all takes Q, K, V, the forward output O
- * and its gradient dO to the head-sharded layout (two launches), the attention
- * backward of cpattn_attention_backward runs on every head rank's buffers (its
- * kernels cover up to 8 head ranks, or groups of heads, per launch), and the
- * second all-to-all brings dQ, dK and dV back to the sequence-sharded layout.
+ * and its gradient dO to the head-sharded layout (two launches), and the
+ * attention backward of cpattn_attention_backward runs on every head rank's
+ * buffers (its kernels cover up to 8 head ranks, or groups of heads, per
+ * launch).  The second all-to-all is fused: the kernels store dQ, dK and dV
+ * straight into the sequence-sharded rank buffers.
  *
  *   q, k, v, out, dout  sequence-sharded rank buffers, as the inputs and the
  *                       output of cpattn_ulysses_attention; read only.
@@ -527,7 +528,8 @@ int cpattn_attention_backward(const void *q, const void *k, const void *v, const
  *   dq, dk, dv          sequence-sharded rank buffers, written.
  *   workspace           device, 16-byte aligned, at least
  *                       cpattn_ulysses_attention_backward_workspace_bytes()
- *                       = 16 * B*S*H*D + 4 * B*H*S bytes; bytes beyond that,
+ *                       = 10 * B*S*H*D + 4 * B*H*S bytes (head-side Q, K, V,
+ *                       O and dO, and the row sums); bytes beyond that,
  *                       from the next 256-byte boundary, are dS scratch as in
  *                       cpattn_attention_backward.
  * Other arguments, splits and errors as cpattn_ulysses_attention (SHAPE also
