@@ -124,3 +124,37 @@ def test_fuzz_backward(i):
         err = np.abs(f64_of(got) - ref)
         assert np.all(np.isfinite(f64_of(got))), f"{what} {name}: non-finite"
         assert err.max() <= 2e-2 * g and err.mean() <= 2e-3 * g, f"{what} {name}: max-abs {err.max():.3e} vs {g:.3e}"
+
+
+@pytest.mark.parametrize("i", range(16))
+def test_fuzz_ulysses_backward(i):
+    """The backward of the Ulysses flow on seeded random shapes, sequence
+    splits and head splits (ranks without tokens or heads included), causal
+    and not: the gradients stored straight into the sequence-sharded rank
+    buffers against the fp64 backward oracle; the path (dQ GEMM with every
+    head at once, in groups of one head, or the dQ kernel) rotates with i."""
+    B, H, S, D, causal = _bwd_case(200 + i)
+    rng = np.random.Generator(np.random.PCG64(9900 + i))
+    U = int(rng.integers(2, min(H, 4) + 1)) if H >= 2 else 1
+    seq = inputs.random_splits(S, U, 9910 + i)
+    heads = inputs.random_splits(H, U, 9920 + i)
+    qb, kb, vb = inputs.make_qkv(B, S, H, D, 9930 + i, D == 128)
+    dob = inputs.f32_to_bf16_bits(rng.standard_normal((B, S, H, D)).astype(np.float32))
+    q, k, v, do = (to_dev(full_to_rank_buffers(x, seq)) for x in (qb, kb, vb, dob))
+    fwd = api.cpattn_causal_ulysses_attention if causal else api.cpattn_ulysses_attention
+    out, lse = fwd(q, k, v, B, S, H, D, U, seq, heads)
+    budget = [None, api.cpattn_attention_backward_ds_bytes(B, S, causal), 0][i % 3]
+    grads = api.cpattn_ulysses_attention_backward(q, k, v, out, lse, do, B, S, H, D, U, seq, heads, causal,
+                                                  ds_budget=budget)
+    torch.cuda.synchronize()
+    st, code = api.cpattn_device_status()
+    what = f"case {i}: B{B} H{H} S{S} D{D} U{U} seq={seq} heads={heads} causal={causal} budget={budget}"
+    assert st == 0, f"{what}: device wait expired {code:#x}"
+    refs = oracle.attention_backward(*(inputs.bf16_bits_to_f64(x) for x in (qb, kb, vb, dob)), causal=causal)
+    dmax = np.abs(inputs.bf16_bits_to_f64(dob)).max()
+    for name, got, ref in zip(("dq", "dk", "dv"), grads, refs):
+        full = rank_buffers_to_full(f64_of(got), B, S, H, D, seq)
+        g = max(np.max(np.abs(ref)), 2.0 ** -10 * dmax, 1e-30)   # a single visible key makes dQ = dK = 0 exactly
+        err = np.abs(full - ref)
+        assert np.all(np.isfinite(full)), f"{what} {name}: non-finite"
+        assert err.max() <= 2e-2 * g and err.mean() <= 2e-3 * g, f"{what} {name}: max-abs {err.max():.3e} vs {g:.3e}"
