@@ -38,6 +38,13 @@ constexpr int kMaxRingDegree = kMaxKV;
 constexpr int kMaxGatherDegree = 1024;
 constexpr int kMaxDevices = 64;
 
+// Kernel parameters (the __grid_constant__ parameter blocks) are limited to
+// 32764 bytes.
+static_assert(sizeof(AttnParams) <= 32764, "AttnParams exceeds the kernel parameter limit");
+static_assert(sizeof(BwdParams) <= 32764, "BwdParams exceeds the kernel parameter limit");
+static_assert(sizeof(ProjParams) <= 32764, "ProjParams exceeds the kernel parameter limit");
+static_assert(sizeof(PermuteParams) <= 32764 && sizeof(MergeParams) <= 32764, "kernel parameter limit");
+
 static unsigned long long wait_timeout_ns() {
   static unsigned long long v = [] {
     const char *e = std::getenv("CPATTN_WAIT_TIMEOUT_MS");
