@@ -612,9 +612,17 @@ static ProblemSpec full_problem(const void *q, const void *k, const void *v, voi
 
 // Ring plan over a [rows, H, D] tensor whose batch-b chunk c occupies rows
 // row_of(b, c) .. + lens[c] at sequence positions off[c] ..; `step` < 0: all
-// chunks in ring order (fused); otherwise only chunk (r - step) mod P.  Under
-// the causal mask a chunk after shard r is invisible to all of its queries
-// and is left out (its ring-step partial is the empty one: out 0, lse -inf).
+// chunks (fused); otherwise only chunk (r - step) mod P.  Without the mask a
+// fused shard walks the chunks in ring order from its own.  Under the causal
+// mask a chunk after shard r is invisible to all of its queries and is left
+// out (its ring-step partial is the empty one: out 0, lse -inf), and a fused
+// shard walks the chunks it sees in sequence order, 0 .. r, its own chunk
+// (the one the mask cuts) last -- so the keys that the first Q tile of a pair
+// cannot see come last in the walk.  Every shard's causal walk is then a
+// prefix of the next shard's: where a batch element's shards are contiguous
+// rows, the fused causal plan is one segment over all of them with the chunks
+// in sequence order, its Q tiles paired across shard boundaries (no lone tile
+// per shard), and each row still walks chunks 0 .. r.
 template <class RowOf>
 static void ring_groups(std::vector<GroupSpec> &groups, int prob, int B, const std::vector<int> &lens,
                         const std::vector<int> &off, int step, bool causal, RowOf row_of) {
@@ -623,21 +631,35 @@ static void ring_groups(std::vector<GroupSpec> &groups, int prob, int B, const s
     GroupSpec g;
     g.prob = prob;
     g.b = b;
+    bool contiguous = causal && step < 0;
+    for (int c = 0; contiguous && c + 1 < P; ++c) contiguous = row_of(b, c + 1) == row_of(b, c) + lens[c];
+    if (contiguous) {
+      SegSpec s;
+      s.row0 = row_of(b, 0);
+      s.nrows = off[P];
+      s.s0 = off[0];
+      for (int c = 0; c < P; ++c)
+        if (lens[c] > 0) s.kv.push_back(AttnKV{row_of(b, c), lens[c], off[c]});
+      g.segs.push_back(std::move(s));
+      groups.push_back(std::move(g));
+      continue;
+    }
     for (int i = 0; i < P; ++i) {
       const int r = causal ? P - 1 - i : i;   // causal: the shard that sees most chunks first
       SegSpec s;
       s.row0 = row_of(b, r);
       s.nrows = lens[r];
       s.s0 = off[r];
-      for (int i_t = 0; i_t < P; ++i_t) {
-        // Causal fused plans visit the shard's own chunk (the one the mask
-        // cuts) after the earlier chunks, so that the keys the first Q tile
-        // of a pair cannot see come last in the walk.
-        const int t = (causal && step < 0) ? (i_t + 1) % P : i_t;
-        if (step >= 0 && t != step) continue;
-        const int c = ((r - t) % P + P) % P;  // chunk held by rank r after t hand-offs
-        if (causal && c > r) continue;
-        if (lens[c] > 0) s.kv.push_back(AttnKV{row_of(b, c), lens[c], off[c]});
+      if (causal && step < 0) {
+        for (int c = 0; c <= r; ++c)
+          if (lens[c] > 0) s.kv.push_back(AttnKV{row_of(b, c), lens[c], off[c]});
+      } else {
+        for (int t = 0; t < P; ++t) {
+          if (step >= 0 && t != step) continue;
+          const int c = ((r - t) % P + P) % P;  // chunk held by rank r after t hand-offs
+          if (causal && c > r) continue;
+          if (lens[c] > 0) s.kv.push_back(AttnKV{row_of(b, c), lens[c], off[c]});
+        }
       }
       g.segs.push_back(std::move(s));
     }
@@ -1275,9 +1297,10 @@ int cpattn_gathered_kv_attention(const void *q, const void *k, const void *v, vo
     sg.nrows = Sq;
     sg.s0 = off[rank];
     for (int i_t = 0; i_t < degree; ++i_t) {
-      // Ring order from this rank's own chunk; under the causal mask the
-      // chunks after the shard are invisible and the own chunk, the one the
-      // mask cuts, is visited last (as in the fused causal ring).
+      // Ring order from this rank's own chunk (the order the chunks arrive
+      // in); under the causal mask the chunks after the shard are invisible
+      // and the own chunk, the one the mask cuts, is visited last, so that
+      // the keys the first Q tile of a pair cannot see come last in the walk.
       const int t = causal ? (i_t + 1) % degree : i_t;
       const int c = ((rank - t) % degree + degree) % degree;
       if (causal && c > rank) continue;
