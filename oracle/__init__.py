@@ -49,7 +49,7 @@ from .attention import (
     ring_step_partials,
     kv_gather_attention,
 )
-from .backward import attention_backward, attention_backward_rows
+from .backward import attention_backward, attention_backward_rows, attention_backward_sampled
 from .projection import (
     project_rows,
     ulysses_qkv_projection,
@@ -69,5 +69,6 @@ __all__ = [
     "offsets", "ring_order", "ring_attention", "ring_step_partials",
     "kv_gather_attention", "ulysses_permute", "ulysses_unpermute",
     "ulysses_attention", "unified_attention", "attention_backward", "attention_backward_rows",
+    "attention_backward_sampled",
     "project_rows", "ulysses_qkv_projection", "ulysses_output_projection", "token_order_rows",
 ]

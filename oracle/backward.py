@@ -65,3 +65,52 @@ def attention_backward(q, k, v, dout, causal=False):
             g = attention_backward_rows(q[b, :, h], k[b, :, h], v[b, :, h], dout[b, :, h], pos, pos)
             dq[b, :, h], dk[b, :, h], dv[b, :, h] = g
     return dq, dk, dv
+
+
+def attention_backward_sampled(q, k, v, dout, q_rows, k_rows, causal=False, block=1024):
+    """The same gradient for one (batch, head) of a long sequence, at sampled
+    rows only: q, k, v, dout (S, D); returns dq[q_rows], dk[k_rows] and
+    dv[k_rows] without forming the S x S matrices.  A forward over blocks of
+    query rows gives every row's log-sum-exp L_i, output O_i and
+    Delta_i = dO_i . O_i.  Then, by the definition above, a query row i has
+    P_i = exp(S_i - L_i), dS_i = P_i * (dO_i V^T - Delta_i) and
+    dQ_i = dS_i K * scale; a key row j has the column P_:j = exp(S_:j - L),
+    dV_j = P_:j^T dO, dS_:j = P_:j * (dO v_j - Delta) and dK_j = dS_:j^T Q * scale.
+    Causal: key j is visible to query i iff j <= i."""
+    q, k, v, dout = (np.asarray(x, dtype=np.float64) for x in (q, k, v, dout))
+    S, D = q.shape
+    scale = softmax_scale(D)
+    lse = np.empty(S)
+    delta = np.empty(S)
+    keys = np.arange(S)
+    for i0 in range(0, S, block):
+        i1 = min(S, i0 + block)
+        s = (q[i0:i1] @ k.T) * scale
+        if causal:
+            s = np.where(keys[None, :] <= np.arange(i0, i1)[:, None], s, -np.inf)
+        m = s.max(axis=1, keepdims=True)
+        e = np.exp(s - m)
+        ell = e.sum(axis=1, keepdims=True)
+        lse[i0:i1] = (m + np.log(ell))[:, 0]
+        o = (e / ell) @ v
+        delta[i0:i1] = (dout[i0:i1] * o).sum(axis=1)
+    q_rows, k_rows = np.asarray(q_rows), np.asarray(k_rows)
+    dq = np.empty((len(q_rows), D))
+    for n, i in enumerate(q_rows):
+        s = (k @ q[i]) * scale
+        p = np.exp(s - lse[i])
+        if causal:
+            p = np.where(keys <= i, p, 0.0)
+        ds = p * (v @ dout[i] - delta[i])
+        dq[n] = (ds @ k) * scale
+    dk = np.empty((len(k_rows), D))
+    dv = np.empty((len(k_rows), D))
+    for n, j in enumerate(k_rows):
+        s = (q @ k[j]) * scale
+        p = np.exp(s - lse)
+        if causal:
+            p = np.where(keys >= j, p, 0.0)
+        dv[n] = p @ dout
+        ds = p * (dout @ v[j] - delta)
+        dk[n] = (ds @ q) * scale
+    return dq, dk, dv

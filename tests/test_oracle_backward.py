@@ -85,3 +85,27 @@ def test_planted_missing_scale_is_caught(monkeypatch):
     monkeypatch.setattr(ob, "attention_backward_rows", no_scale)
     with pytest.raises(AssertionError):
         test_backward_matches_torch_autograd_float64(1, 7, 2, 8, False)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("S,D,block", [(37, 8, 8), (300, 16, 128)])
+def test_sampled_backward_matches_torch_autograd_float64(S, D, block, causal):
+    """The sampled-row form of the gradient (a blockwise forward for the row
+    statistics, then single rows and key columns) against torch autograd in
+    float64, over blocks smaller than S with a ragged last block; first,
+    last and interior rows, keys and queries sampled separately."""
+    q, k, v, do = (_rand((S, D), s) for s in (11, 12, 13, 14))
+    q_rows = [0, 1, S // 2, S - 1]
+    k_rows = [0, S // 3, S - 2, S - 1]
+    dq, dk, dv = oracle.attention_backward_sampled(q, k, v, do, q_rows, k_rows, causal=causal, block=block)
+    tq, tk, tv = (torch.from_numpy(x)[None, None].clone().requires_grad_(True) for x in (q, k, v))
+    o = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=causal)
+    o.backward(torch.from_numpy(do)[None, None])
+    assert np.max(np.abs(dq - tq.grad[0, 0].numpy()[q_rows])) < 1e-11
+    assert np.max(np.abs(dk - tk.grad[0, 0].numpy()[k_rows])) < 1e-11
+    assert np.max(np.abs(dv - tv.grad[0, 0].numpy()[k_rows])) < 1e-11
+    # and the full-matrix form, row for row
+    pos = np.arange(S) if causal else None
+    fq, fk, fv = oracle.attention_backward_rows(q, k, v, do, pos, pos)
+    assert np.max(np.abs(dq - fq[q_rows])) < 1e-12 and np.max(np.abs(dk - fk[k_rows])) < 1e-12
+    assert np.max(np.abs(dv - fv[k_rows])) < 1e-12
