@@ -297,7 +297,7 @@ def test_backward_workspace_budget():
     assert api.backward_workspace_bytes(2, 5, 300, causal=True, ds_budget=2 * per) == base + 256 + 3 * per_c
     ubase = api.cpattn_ulysses_attention_backward_workspace_bytes(2, 5, 300, 64)
     assert api.backward_workspace_bytes(2, 5, 300, ulysses_D=64, ds_budget=per) == ubase + 256 + per
-    # the video workload: 2.1 GB of dS per head, so the default budget takes 3 of its 40 heads
+    # the video workload: 2 GiB of dS per head, so the default budget takes 4 of its 40 heads
     per_v = api.cpattn_attention_backward_ds_bytes(1, 32760, False)
     assert per_v == 256 * 256 * 32768
     assert api.backward_workspace_bytes(1, 40, 32760) == (api.cpattn_attention_backward_workspace_bytes(1, 40, 32760)

@@ -141,6 +141,35 @@ def test_backward_paths_agree(B, S, H, D, causal):
         assert torch.equal(bits(a), bits(b))
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_video_workload_sampled(causal):
+    """Video shapes (B1 H40 S32760 D128), the largest configuration, on the
+    default path: the bindings' dS budget holds 4 of the 40 heads (7 under
+    the causal mask), so the backward runs in 10 (6) head groups.  The oracle
+    checks sampled rows (tile edges, the ends, seeded interior rows) of heads
+    0 and 39, in the first and the last group."""
+    cfg, qb, kb, vb = inputs.config_inputs("video")
+    B, S, H, D = qb.shape
+    per = api.cpattn_attention_backward_ds_bytes(B, S, causal)
+    assert api.BACKWARD_DS_BUDGET // per < H        # several head groups
+    rng = np.random.Generator(np.random.PCG64(78))
+    dob = inputs.f32_to_bf16_bits(rng.standard_normal((B, S, H, D)).astype(np.float32))
+    q, k, v, do = (to_dev(x) for x in (qb, kb, vb, dob))
+    fwd = api.cpattn_causal_ring_attention if causal else api.cpattn_ring_attention
+    out, lse = fwd(q, k, v, cfg["ring_degree"])
+    dq, dk, dv = api.cpattn_attention_backward(q, k, v, out, lse, do, causal=causal)
+    torch.cuda.synchronize()
+    _no_timeouts()
+    rows = sorted({0, 1, 127, 128, 4095, 4096, S // 2, S - 129, S - 128, S - 2, S - 1} |
+                  {int(x) for x in rng.integers(0, S, size=8)})
+    dmax = np.abs(inputs.bf16_bits_to_f64(dob)).max()
+    for h in (0, H - 1):
+        ref = oracle.attention_backward_sampled(*(inputs.bf16_bits_to_f64(x[0, :, h]) for x in (qb, kb, vb, dob)),
+                                                rows, rows, causal=causal)
+        for name, got, r in zip(("dq", "dk", "dv"), (dq, dk, dv), ref):
+            assert_grad_close(f64_of(got[0, rows, h]), r, f"video {name} head {h} causal={causal}", dmax)
+
+
 def test_backward_is_deterministic_and_validates():
     bits, g1 = _run(1, 384, 2, 128, True, 5)
     _, g2 = _run(1, 384, 2, 128, True, 5)
