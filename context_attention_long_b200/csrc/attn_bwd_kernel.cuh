@@ -24,12 +24,14 @@
 // each with its own tensor maps, LSE strides and Delta slice.  CTA
 // organisation of the dQ and dK/dV kernels (320 threads, one CTA per SM):
 //   warp 0      TMA producer: the owned tiles once, the walked tiles through
-//               rings of 3 stages (K or Q) and 2 stages (V or dO)
+//               rings of 3 stages (K or Q) and 2 stages (V or dO); the dK/dV
+//               kernel that stores dS has 2 Q stages and a dS staging tile
 //   warp 1      TMEM allocator + single-thread MMA issuer (tcgen05.mma)
 //   warps 2-9   two threads per row of the owned tile (TMEM lane), one per
 //               half of the walked tile's 128 columns (warps 2-5 the first
 //               half, 6-9 the second): P and dS in registers, bf16 results
-//               back into TMEM, the epilogue.  Two row warps share each
+//               back into TMEM (and dS to the staging tile, whose 4 KB part
+//               each warp then bulk-stores), the epilogue.  Two row warps share each
 //               sub-partition, so one's exponentials overlap the other's
 //               loads, stores and waits.
 // TMEM columns: S [0,128) (later P), dP [128,256) (later dS), then the
