@@ -401,17 +401,30 @@ def backward_workspace_bytes(B, H, S, causal=False, ds_budget=None, ulysses_D=No
     return base + _ds_scratch_bytes(B, H, S, causal, ds_budget)
 
 
+def _allocation_budget(device, ds_budget):
+    """The dS budget for a workspace the binding allocates itself: the given
+    one, or by default BACKWARD_DS_BUDGET capped at half the device's free
+    memory (a smaller scratch only means more head groups)."""
+    if ds_budget is not None:
+        return int(ds_budget)
+    free, _ = torch.cuda.mem_get_info(device)
+    return min(BACKWARD_DS_BUDGET, free // 2)
+
+
 def cpattn_attention_backward(q, k, v, out, lse, dout, causal=False, dq=None, dk=None, dv=None, workspace=None,
                               stream=None, ds_budget=None):
     """Gradient of attention over full (B,S,H,D) bf16 tensors given the
     forward's output and LSE; returns (dq, dk, dv) in bf16.  An allocated
-    workspace holds up to ds_budget bytes (default BACKWARD_DS_BUDGET) of dS
-    scratch; 0 selects the dQ kernel that recomputes S and dP."""
+    workspace holds up to ds_budget bytes of dS scratch (default
+    BACKWARD_DS_BUDGET, capped at half the device's free memory); 0 selects
+    the dQ kernel that recomputes S and dP."""
     B, S, H, D = _bshd(q)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    workspace = _workspace(backward_workspace_bytes(B, H, S, causal, ds_budget), q.device, workspace)
+    if workspace is None:
+        workspace = _workspace(backward_workspace_bytes(B, H, S, causal, _allocation_budget(q.device, ds_budget)),
+                               q.device, None)
     for t, name in ((k, "k"), (v, "v"), (out, "out"), (dout, "dout"), (dq, "dq"), (dk, "dk"), (dv, "dv")):
         _need(t, q.numel(), torch.bfloat16, name)
     _need(lse, B * H * S, torch.float32, "lse")
@@ -437,7 +450,9 @@ def cpattn_ulysses_attention_backward(q, k, v, out, lse, dout, B, S, H, D, degre
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    workspace = _workspace(backward_workspace_bytes(B, H, S, causal, ds_budget, ulysses_D=D), q.device, workspace)
+    if workspace is None:
+        workspace = _workspace(backward_workspace_bytes(B, H, S, causal, _allocation_budget(q.device, ds_budget),
+                                                        ulysses_D=D), q.device, None)
     for t, name in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout"), (dq, "dq"), (dk, "dk"), (dv, "dv")):
         _need(t, _flat_numel(B, S, H, D), torch.bfloat16, name)
     _need(lse, B * H * S, torch.float32, "lse")
