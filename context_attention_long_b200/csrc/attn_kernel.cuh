@@ -132,7 +132,7 @@ __device__ __forceinline__ Unit decode_unit(const AttnParams &p) {
   if (p.causal) u.pair = (SG.nrows + kQTilesPerCTA * kQTile - 1) / (kQTilesPerCTA * kQTile) - 1 - u.pair;
   u.q_row0 = SG.row0 + u.pair * (kQTilesPerCTA * kQTile);
   u.rows_left = SG.nrows - u.pair * (kQTilesPerCTA * kQTile);
-  u.has_q1 = u.rows_left > kQTile;
+  u.has_q1 = u.rows_left > kQTile || SG.q1_rows > 0;
   u.q_last = SG.s0 + u.pair * (kQTilesPerCTA * kQTile) + min(u.rows_left, kQTilesPerCTA * kQTile) - 1;
   int n = 0;
   for (int i = 0; i < SG.kv_count; ++i) n += (kv_rows_seen(p, p.kv[SG.kv_first + i], u.q_last) + kKVTile - 1) / kKVTile;
@@ -283,9 +283,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       mbar_arrive_expect_tx(sb + BAR_Q, (has_q1 ? 2 : 1) * L::kTileBytes);
       for (int hf = 0; hf < L::kHalves; ++hf)
         tma_load_3d(sQ + hf * L::kBoxBytes, &PB.tm_q, hf * 64, h, q_row0, sb + BAR_Q);
-      if (has_q1)
+      if (has_q1) {
+        const int q1_row = SG.q1_rows > 0 ? SG.q1_row0 : q_row0 + kQTile;   // a paired lone tile, or the next one
         for (int hf = 0; hf < L::kHalves; ++hf)
-          tma_load_3d(sQ + L::kTileBytes + hf * L::kBoxBytes, &PB.tm_q, hf * 64, h, q_row0 + kQTile, sb + BAR_Q);
+          tma_load_3d(sQ + L::kTileBytes + hf * L::kBoxBytes, &PB.tm_q, hf * 64, h, q1_row, sb + BAR_Q);
+      }
       bool ok = true;
       auto load_kv = [&](int st, uint32_t ph, int row) -> bool {
         if (!mbar_wait(sb + BAR_KE + 8 * st, ph ^ 1, abort_flag, tmo, SITE_PRODUCER)) return false;
@@ -485,7 +487,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
     const float c = p.scale_log2;
     // Sequence position of this thread's query row (both slots of a split
     // unit hold the same rows).
-    const int q_pos = SG.s0 + pair * (kQTilesPerCTA * kQTile) + (split ? 0 : qt * kQTile) + row;
+    const bool paired_lone = qt == 1 && SG.q1_rows > 0;   // slot 1 holds another shard's lone tile
+    const int q_pos = paired_lone ? SG.q1_s0 + row
+                                  : SG.s0 + pair * (kQTilesPerCTA * kQTile) + (split ? 0 : qt * kQTile) + row;
     const bool causal = p.causal != 0;
     // K/V tiles [g_lo, g_hi) of the segment belong to this slot.
     const int g_lo = (split && qt == 1) ? U.n0 : 0;
@@ -687,10 +691,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
         }
       }
     } else if (active && ok) {
-      const int valid_rows = qt == 0 ? min(kQTile, rows_left) : rows_left - kQTile;
+      const int valid_rows = qt == 0 ? min(kQTile, rows_left) : (paired_lone ? SG.q1_rows : rows_left - kQTile);
       const bool row_valid = row < valid_rows;
-      const int grow = q_row0 + qt * kQTile + row;
-      const int sq = SG.s0 + pair * (kQTilesPerCTA * kQTile) + qt * kQTile + row;
+      const int grow = paired_lone ? SG.q1_row0 + row : q_row0 + qt * kQTile + row;
+      const int sq = paired_lone ? SG.q1_s0 + row : SG.s0 + pair * (kQTilesPerCTA * kQTile) + qt * kQTile + row;
       const size_t row_elems = out_row_elems<D>(PB, G.b, sq, grow, h);
       const long long lse_idx = static_cast<long long>(G.b) * PB.lse_b +
                                 static_cast<long long>(h + PB.lse_h0) * PB.lse_h + (sq - PB.lse_pos0);

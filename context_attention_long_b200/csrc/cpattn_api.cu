@@ -420,6 +420,7 @@ struct SegSpec {
   int row0, nrows, s0;
   std::vector<AttnKV> kv;
   int split = 0;   // a lone Q tile: split its K/V tiles between the two slots
+  int q1_row0 = 0, q1_s0 = 0, q1_rows = 0;   // a lone tile paired with another shard's lone tile in slot 1
 };
 struct GroupSpec {
   int prob, b;
@@ -432,9 +433,79 @@ struct GroupSpec {
 // hold its rows and divide its K/V tiles, merged with the LSE rule at the
 // end), about half the work of a pair; those units are placed after every
 // full pair, so they fill the gaps of the last wave instead of adding one.
-static std::vector<GroupSpec> longest_first(const std::vector<GroupSpec> &groups) {
+// Without the causal mask, two lone tiles of one group whose K/V lists hold
+// the same chunks (the shards of a fused ring: each walks every chunk, from
+// its own) share one CTA as a pair: slot 1 takes the second tile's rows and
+// both walk the first tile's list.  The second tile's keys are the same; only
+// the order of its online-softmax steps (so its rounding) follows the other
+// shard.  This replaces two split units, whose slots each stream their own
+// K/V tiles and merge at the end, by one pair unit on one K/V stream.
+static bool same_kv_set(std::vector<AttnKV> a, std::vector<AttnKV> b) {
+  auto key = [](const AttnKV &x, const AttnKV &y) { return x.row0 < y.row0; };
+  std::sort(a.begin(), a.end(), key);
+  std::sort(b.begin(), b.end(), key);
+  if (a.size() != b.size()) return false;
+  for (size_t i = 0; i < a.size(); ++i)
+    if (a[i].row0 != b[i].row0 || a[i].nrows != b[i].nrows || a[i].s0 != b[i].s0) return false;
+  return true;
+}
+static void pair_lone_tiles(GroupSpec &g) {
+  std::vector<SegSpec> out;
+  std::vector<bool> used(g.segs.size(), false);
+  for (size_t i = 0; i < g.segs.size(); ++i) {
+    if (used[i]) continue;
+    used[i] = true;
+    SegSpec a = g.segs[i];
+    for (size_t j = i + 1; j < g.segs.size(); ++j) {
+      if (used[j] || g.segs[j].nrows <= 0 || a.nrows <= 0 || !same_kv_set(a.kv, g.segs[j].kv)) continue;
+      used[j] = true;
+      a.split = 0;
+      a.q1_row0 = g.segs[j].row0;
+      a.q1_s0 = g.segs[j].s0;
+      a.q1_rows = g.segs[j].nrows;
+      break;
+    }
+    out.push_back(std::move(a));
+  }
+  g.segs = std::move(out);
+}
+
+// SMs of the current device (cached per device).
+static int device_sm_count() {
+  static std::mutex mu;
+  static int sms[kMaxDevices] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev >= 0 && dev < kMaxDevices && sms[dev] == 0 &&
+      cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    sms[dev] = 0;
+  return (dev >= 0 && dev < kMaxDevices && sms[dev] > 0) ? sms[dev] : 148;
+}
+
+// Makespan, in half units, of the longest-first schedule over `sms` SMs of
+// n2 units of length 2 followed by n1 of length 1.
+static long long lpt_half_units(long long n2, long long n1, int sms) {
+  std::vector<long long> load(static_cast<size_t>(std::max(1, sms)), 0);
+  auto put = [&](long long w, long long n) {
+    for (long long i = 0; i < n; ++i) {
+      std::pop_heap(load.begin(), load.end(), std::greater<long long>());
+      load.back() += w;
+      std::push_heap(load.begin(), load.end(), std::greater<long long>());
+    }
+  };
+  std::make_heap(load.begin(), load.end(), std::greater<long long>());
+  put(2, n2);
+  put(1, n1);
+  return *std::max_element(load.begin(), load.end());
+}
+
+// heads[prob]: the head count of each problem (units run once per head).
+static std::vector<GroupSpec> longest_first(const std::vector<GroupSpec> &groups, bool causal,
+                                            const std::vector<int> &heads) {
   constexpr int kPairRows = kQTilesPerCTA * kQTile;
-  std::vector<GroupSpec> head, tail;
+  std::vector<GroupSpec> head, tail, tail_paired;
+  long long n_pairs = 0, n_lone = 0, n_cross = 0, n_single = 0;   // units, over all heads
   for (const GroupSpec &g : groups) {
     GroupSpec main_g{g.prob, g.b, {}}, tail_g{g.prob, g.b, {}};
     for (const SegSpec &s : g.segs) {
@@ -458,8 +529,24 @@ static std::vector<GroupSpec> longest_first(const std::vector<GroupSpec> &groups
       main_g.segs.push_back(std::move(m));
       tail_g.segs.push_back(std::move(t));
     }
+    const long long H = heads[g.prob];
+    for (const SegSpec &s : main_g.segs) n_pairs += H * ((s.nrows + kPairRows - 1) / kPairRows);
     if (!main_g.segs.empty()) head.push_back(std::move(main_g));
-    if (!tail_g.segs.empty()) tail.push_back(std::move(tail_g));
+    if (tail_g.segs.empty()) continue;
+    GroupSpec paired = tail_g;
+    if (!causal) pair_lone_tiles(paired);
+    n_lone += H * static_cast<long long>(tail_g.segs.size());
+    for (const SegSpec &s : paired.segs) (s.q1_rows > 0 ? n_cross : n_single) += H;
+    tail.push_back(std::move(tail_g));
+    tail_paired.push_back(std::move(paired));
+  }
+  // Paired lone tiles walk as long as a full pair; split units take about half
+  // as long and fill the last wave.  Pair them unless that lengthens the
+  // longest-first schedule (in half units: a pair 2, a split unit 1).
+  if (n_cross > 0) {
+    const int sms = device_sm_count();
+    if (lpt_half_units(n_pairs + n_cross, n_single, sms) <= lpt_half_units(n_pairs, n_lone, sms))
+      tail = std::move(tail_paired);
   }
   for (GroupSpec &g : tail) head.push_back(std::move(g));
   return head;
@@ -485,7 +572,9 @@ static int causal_head_block(const GroupSpec &gs, int D, int H) {
 // launches them in order on `stream`.
 static int run_attention(const std::vector<ProblemSpec> &probs, const std::vector<GroupSpec> &groups_in, int D,
                          bool out_f32, bool causal, cudaStream_t stream) {
-  const std::vector<GroupSpec> groups = longest_first(groups_in);
+  std::vector<int> heads(probs.size());
+  for (size_t i = 0; i < probs.size(); ++i) heads[i] = probs[i].H;
+  const std::vector<GroupSpec> groups = longest_first(groups_in, causal, heads);
   std::vector<AttnProblem> encoded(probs.size());
   for (size_t i = 0; i < probs.size(); ++i) {
     const ProblemSpec &ps = probs[i];
@@ -585,6 +674,9 @@ static int run_attention(const std::vector<ProblemSpec> &probs, const std::vecto
       sg.kv_count = need_kv;
       sg.tile_base = g.tiles_per_head;
       sg.split = ss.split;
+      sg.q1_row0 = ss.q1_row0;
+      sg.q1_s0 = ss.q1_s0;
+      sg.q1_rows = ss.q1_rows;
       for (const AttnKV &kv : ss.kv) P->kv[n_kv++] = kv;
       g.seg_count += 1;
       g.tiles_per_head += (ss.nrows + kQTilesPerCTA * kQTile - 1) / (kQTilesPerCTA * kQTile);

@@ -79,6 +79,10 @@ struct AttnSeg {
   int kv_count;   // number of K/V ranges (0: empty -> out 0, lse -inf)
   int tile_base;  // first tile pair of this segment within the group's head
   int split;      // 1: a lone Q tile whose K/V tiles are split between the two slots
+  // q1_rows > 0: a lone tile of rows [row0, row0 + nrows) paired with another
+  // shard's lone tile (q1_rows rows from q1_row0, position q1_s0) in slot 1;
+  // both walk this segment's K/V list (no causal mask, so both see every key).
+  int q1_row0, q1_s0, q1_rows;
 };
 
 struct AttnKV {
