@@ -840,9 +840,9 @@ def backward_paths(api, torch, flush, peaks, q, k, v, P):
     ms = median_event_ms(run_u, flush, stream)
     tf = backward_flops(B, H, S, D, False) / (ms * 1e-3) / 1e12
     res[f"ulysses_{U}_backward_flow"] = {"ms": ms, "TFLOP/s": tf, "frac_bf16_peak": tf / peak_tf,
-                                         "launches": 8, "note": "5 tensors permuted in (2 launches), the row sums of "
-                                         "4 head ranks, dK/dV and the dQ GEMM over all of them, storing the gradients "
-                                         "in the sequence-sharded layout"}
+                                         "launches": 5, "note": "5 tensors permuted in (2 launches), the row sums of "
+                                         "the 4 head ranks in one launch, dK/dV and the dQ GEMM over all of them, "
+                                         "storing the gradients in the sequence-sharded layout"}
     return res
 
 

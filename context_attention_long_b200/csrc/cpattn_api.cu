@@ -1618,6 +1618,14 @@ int cpattn_ulysses_attention_backward(const void *q, const void *k, const void *
   // sequence-sharded rank buffers (the second all-to-all, fused).
   const std::vector<int> ho = prefix(heads);
   const std::vector<int> so = prefix(seq_chk);
+  // With equal head splits the head-side O and dO buffers of all ranks, and
+  // their Delta slices, are one [degree * B, S, H / degree, D] tensor set:
+  // one row-sum launch covers every rank.
+  const bool even_heads = std::all_of(heads.begin(), heads.end(), [&](int x) { return x == heads[0]; });
+  if (even_heads && heads[0] > 0) {
+    if (cudaError_t e = launch_bwd_delta(y[3], y[4], delta, degree * B, S, heads[0], D, stream); e != cudaSuccess)
+      return cuda_fail(e, "backward launch");
+  }
   std::vector<BwdProblem> sets;
   sets.reserve(degree);
   for (int u = 0; u < degree; ++u) {
@@ -1635,8 +1643,10 @@ int cpattn_ulysses_attention_backward(const void *q, const void *k, const void *
     pb.out_h0 = ho[u];
     pb.out_nseq = degree;
     for (int r = 0; r <= degree; ++r) pb.out_seq_off[r] = so[r];
-    if (cudaError_t e = launch_bwd_delta(at(3), at(4), dl, B, S, heads[u], D, stream); e != cudaSuccess)
-      return cuda_fail(e, "backward launch");
+    if (!even_heads) {
+      if (cudaError_t e = launch_bwd_delta(at(3), at(4), dl, B, S, heads[u], D, stream); e != cudaSuccess)
+        return cuda_fail(e, "backward launch");
+    }
   }
   return cuda_result(run_bwd_sets(sets, scratch, scratch_bytes, B, S, D, causal != 0, stream), "backward launch");
 }
