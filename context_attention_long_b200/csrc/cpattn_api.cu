@@ -230,6 +230,19 @@ cudaError_t launch_attention(const AttnParams &p, int D, bool out_f32, cudaStrea
   return out_f32 ? launch_attn_t<64, true>(p, stream) : launch_attn_t<64, false>(p, stream);
 }
 
+// SMs of the current device (cached per device).
+static int device_sm_count() {
+  static std::mutex mu;
+  static int sms[kMaxDevices] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev >= 0 && dev < kMaxDevices && sms[dev] == 0 &&
+      cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    sms[dev] = 0;
+  return (dev >= 0 && dev < kMaxDevices && sms[dev] > 0) ? sms[dev] : 148;
+}
+
 static int grid_for(long long work_items, int items_per_block) {
   long long blocks = (work_items + items_per_block - 1) / items_per_block;
   blocks = std::max<long long>(1, std::min<long long>(blocks, 148ll * 16));
@@ -304,7 +317,10 @@ cudaError_t launch_bwd_delta(const void *out, const void *dout, float *delta, in
                              cudaStream_t stream) {
   const long long rows = static_cast<long long>(B) * S * H;
   if (rows == 0) return cudaSuccess;
-  attn_bwd_delta_kernel<<<grid_for(rows, (256 / 32) * (32 / (D / 8)) * kDeltaPasses), 256, 0, stream>>>(
+  // as many CTAs as are resident at once (three per SM): every warp walks
+  // several row groups instead of a new CTA starting for each
+  const int grid = std::min(grid_for(rows, (256 / 32) * (32 / (D / 8)) * kDeltaPasses), 3 * device_sm_count());
+  attn_bwd_delta_kernel<<<grid, 256, 0, stream>>>(
       static_cast<const __nv_bfloat16 *>(out), static_cast<const __nv_bfloat16 *>(dout), delta, B, S, H, D);
   return cudaGetLastError();
 }
@@ -470,18 +486,6 @@ static void pair_lone_tiles(GroupSpec &g) {
   g.segs = std::move(out);
 }
 
-// SMs of the current device (cached per device).
-static int device_sm_count() {
-  static std::mutex mu;
-  static int sms[kMaxDevices] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  std::lock_guard<std::mutex> lock(mu);
-  if (dev >= 0 && dev < kMaxDevices && sms[dev] == 0 &&
-      cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    sms[dev] = 0;
-  return (dev >= 0 && dev < kMaxDevices && sms[dev] > 0) ? sms[dev] : 148;
-}
 
 // Makespan, in half units, of the longest-first schedule over `sms` SMs of
 // n2 units of length 2 followed by n1 of length 1.
