@@ -191,14 +191,7 @@ __device__ __forceinline__ void tma_load_3d(uint32_t smem_dst, const CUtensorMap
 }
 // Untiled bulk copy global -> shared of `bytes` bytes (a multiple of 16, both
 // addresses 16-byte aligned), completing on an mbarrier with transaction
-// bytes.  No multicast.
-__device__ __forceinline__ void bulk_load(uint32_t smem_dst, const void *src, uint32_t bytes, uint32_t bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                   smem_dst),
-               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
-               : "memory");
-}
-// The same with an L2 cache policy (from l2_evict_first_policy).
+// bytes, with an L2 cache policy (from l2_evict_first_policy).  No multicast.
 __device__ __forceinline__ void bulk_load_hint(uint32_t smem_dst, const void *src, uint32_t bytes, uint32_t bar,
                                                uint64_t policy) {
   asm volatile(
@@ -214,15 +207,10 @@ __device__ __forceinline__ uint64_t l2_evict_first_policy() {
   return p;
 }
 // Untiled bulk copy shared -> global of `bytes` bytes (a multiple of 16, both
-// addresses 16-byte aligned), tracked by this thread's bulk groups.  The
-// generic-proxy writes it copies must be fenced to the async proxy first
-// (fence_proxy_async_shared by every writing thread, then a barrier).
-__device__ __forceinline__ void bulk_store(void *dst, uint32_t smem_src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(reinterpret_cast<uint64_t>(dst)),
-               "r"(smem_src), "r"(bytes)
-               : "memory");
-}
-// The same with an L2 cache policy.
+// addresses 16-byte aligned) with an L2 cache policy, tracked by this
+// thread's bulk groups.  The generic-proxy writes it copies must be fenced to
+// the async proxy first (fence_proxy_async_shared by every writing thread,
+// then a barrier).
 __device__ __forceinline__ void bulk_store_hint(void *dst, uint32_t smem_src, uint32_t bytes, uint64_t policy) {
   asm volatile("cp.async.bulk.global.shared::cta.bulk_group.L2::cache_hint [%0], [%1], %2, %3;" ::"l"(
                    reinterpret_cast<uint64_t>(dst)),
